@@ -1,0 +1,251 @@
+/*
+ * rlscan.h - C ABI of librlscan: RL credit assignment as one first-order
+ * linear-recurrence scan, on CUDA kernels for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  The rl-triton paper (arXiv:2608.17641, abstract) recasts
+ * seven credit-assignment estimators as instances of one first-order linear
+ * recurrence x_t = a_t * x_{t+-1} + b_t, solved by an associative scan over
+ * (a, b) pairs with the operator (a1, b1) o (a2, b2) = (a1 a2, a1 b2 + b1).
+ * Each entry point below is one estimator of the rl-triton README's
+ * "Kernels" table (compute_gae ... compute_episodic_prefix_sum); its call
+ * follows the README's "Usage" example (rewards, values, terminateds, gamma,
+ * lambda_) and the with-truncations paragraph under "Performance"
+ * (terminations + time-limit truncations + bootstrap values).
+ *
+ * Common conventions (every entry point):
+ *   - Layout: every [E, T] array is row-major and contiguous, T (seq_len)
+ *     fastest: element (e, t) is at index e*T + t.  Retrace's per-action
+ *     arrays are [E, T, A], A fastest.  E = num_envs, T = seq_len.
+ *   - Memory: every pointer is DEVICE memory on the current device, owned by
+ *     the caller, which keeps it alive until the stream reaches the call.
+ *     Inputs are read, never written.  Outputs are written in full, must be
+ *     preallocated, and must not overlap any input or each other
+ *     (RLSCAN_ERR_INVALID_ARG).  16-byte-aligned pointers take the vectorised
+ *     path; any other alignment is accepted and runs a scalar-load path.
+ *   - Flags (terminateds, truncateds, dones) are float32; a flag is set iff it
+ *     is nonzero.  terminated at t: the episode ends at t, nothing is
+ *     bootstrapped and the trace is cut.  truncated at t: the episode ends at
+ *     t, its value is bootstrapped from bootstrap_values[e, t] and the trace is
+ *     cut.  If both are set, terminated wins.  bootstrap_values is read only
+ *     where a step is truncated.
+ *   - last_values (nullable, [E]): the value after the last step of each row
+ *     when that step carries no flag; NULL means 0.
+ *   - Forward estimators (eligibility traces, prefix sum) reset after a done:
+ *     dones[e, t-1] != 0 starts a new episode at t.
+ *   - Results equal the sequential definition up to fp32 rounding (the scan
+ *     re-associates); the int32 prefix sum is exact (two's-complement wrap).
+ *   - Asynchrony: every compute call only enqueues work on `stream` (NULL =
+ *     the legacy default stream); it never allocates, never synchronises and
+ *     returns as soon as the kernel is launched.  E == 0 or T == 0 is a no-op
+ *     returning RLSCAN_OK.  Calls are thread-safe.
+ *   - Workspace: long rows (a row that spans several tiles) and rows that do
+ *     not align with tiles need a device workspace of
+ *     rlscan_workspace_bytes(E, T) bytes, 16-byte aligned, zero-filled before
+ *     its first use (rlscan_workspace_init or cudaMemset) and left zero-filled
+ *     by every call.  Shapes that need none accept ws = NULL.  A workspace
+ *     holds one call's progress flags: calls that share one must be ordered
+ *     on one stream (or otherwise serialised).
+ *   - Errors: a nonzero return is an rlscan_status; nothing was enqueued
+ *     unless it is RLSCAN_ERR_CUDA from the launch itself.
+ *     rlscan_last_error() gives a message for the calling thread.
+ */
+#ifndef RLSCAN_H
+#define RLSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RLSCAN_VERSION 100 /* 1.0.0 */
+
+/* Every entry point is exported from librlscan.so (built with hidden
+ * visibility for everything else). */
+#if defined(__GNUC__)
+#define RLSCAN_API __attribute__((visibility("default")))
+#else
+#define RLSCAN_API
+#endif
+
+typedef enum rlscan_status {
+    RLSCAN_OK = 0,
+    RLSCAN_ERR_INVALID_ARG = 1, /* NULL required pointer, E/T/A < 0 or too large, non-finite
+                                   gamma/lambda/rho_bar/c_bar, truncateds without
+                                   bootstrap_values, overlapping buffers */
+    RLSCAN_ERR_UNSUPPORTED = 2, /* unknown dtype, A above RLSCAN_MAX_ACTIONS */
+    RLSCAN_ERR_WORKSPACE = 3,   /* the shape needs a workspace and ws is NULL, too small or
+                                   not 16-byte aligned */
+    RLSCAN_ERR_CUDA = 4,        /* a CUDA runtime call failed (message in rlscan_last_error) */
+    RLSCAN_ERR_TIMEOUT = 5      /* reported by rlscan_check: a kernel gave up a bounded wait
+                                   for a neighbouring tile, or found its workspace not
+                                   zero-filled; that call's output is invalid and the
+                                   workspace should be re-initialised */
+} rlscan_status;
+
+typedef enum rlscan_dtype {
+    RLSCAN_F32 = 0,
+    RLSCAN_I32 = 1
+} rlscan_dtype;
+
+/* Largest action count accepted by rlscan_retrace. */
+#define RLSCAN_MAX_ACTIONS 96
+
+/*
+ * GAE (README "Kernels": compute_gae, "backward scan over delta + gamma
+ * lambda A"; Usage example for the positional arguments).
+ *   delta_t = r_t + gamma * boot_t - V_t
+ *   A_t = delta_t + gamma lambda A_{t+1} while the episode goes on, A_t = delta_t
+ *   at a flagged step, A_T = 0; boot_t = V_{t+1} (V_T = last value), the
+ *   bootstrap value at a truncation, 0 at a termination.
+ * rewards, values [E,T] required; terminateds [E,T] nullable (no
+ * terminations); truncateds [E,T] nullable; bootstrap_values [E,T] required
+ * iff truncateds is given; last_values [E] nullable; advantages [E,T] output.
+ */
+RLSCAN_API int rlscan_gae(const float *rewards, const float *values, const float *terminateds,
+               const float *truncateds, const float *bootstrap_values, const float *last_values,
+               float *advantages, int64_t E, int64_t T, float gamma, float lambda_, void *ws,
+               size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * V-Trace (README "Kernels": compute_vtrace, "IS-weighted targets and
+ * advantages"; IMPALA, Espeholt et al. 2018, section 4.1).
+ *   rho_t = min(rho_bar, exp(log_rho_t)),  c_t = lambda min(c_bar, exp(log_rho_t))
+ *   D_t = rho_t (r_t + gamma boot_t - V_t) + gamma c_t D_{t+1} (cut at flags), D_T = 0
+ *   vs_t = V_t + D_t
+ *   pg_advantages_t = rho_t (r_t + gamma boot'_t - V_t), boot'_t = vs_{t+1}
+ *   while the episode goes on (vs_T = last value), the bootstrap value at a
+ *   truncation, 0 at a termination.
+ * lambda_ = 1 is IMPALA's v-trace.  log_rhos, rewards, values required;
+ * others as rlscan_gae; vs and pg_advantages [E,T] outputs.
+ */
+RLSCAN_API int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values,
+                  const float *terminateds, const float *truncateds,
+                  const float *bootstrap_values, const float *last_values, float *vs,
+                  float *pg_advantages, int64_t E, int64_t T, float gamma, float lambda_,
+                  float rho_bar, float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Retrace(lambda) (README "Kernels": compute_retrace, "off-policy return
+ * estimate with truncated IS ratios"; with-truncations paragraph:
+ * terminated and truncated are both mandatory and there is no bootstrap
+ * argument, the continuation value being folded into next_q_values_all at
+ * every step; Munos et al. 2016).
+ *   V'_t = sum_a next_target_probs[e,t,a] next_q_values_all[e,t,a]
+ *          (A == 1: V'_t = next_q_values_all[e,t], next_target_probs NULL)
+ *   delta_t = r_t + gamma (terminated_t ? 0 : V'_t) - q_t
+ *   Dq_t = delta_t + gamma lambda min(c_bar, exp(log_rho_{t+1})) Dq_{t+1} while
+ *   the episode goes on and t < T-1; Dq_t = delta_t otherwise
+ *   q_ret_t = q_t + Dq_t
+ * next_q_values_all[e,t,:] = Q(x_{t+1}, .) (the final observation's values at
+ * a truncation; ignored at a termination); next_target_probs[e,t,:] =
+ * pi(. | x_{t+1}); log_rhos[e,t] = log pi(a_t|x_t) - log mu(a_t|x_t);
+ * q_values[e,t] = Q(x_t, a_t).  1 <= A <= RLSCAN_MAX_ACTIONS.
+ */
+RLSCAN_API int rlscan_retrace(const float *rewards, const float *q_values, const float *next_q_values_all,
+                   const float *next_target_probs, const float *log_rhos,
+                   const float *terminateds, const float *truncateds, float *q_ret, int64_t E,
+                   int64_t T, int64_t A, float gamma, float lambda_, float c_bar, void *ws,
+                   size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * TD(lambda) returns (README "Kernels": compute_lambda_returns, "lambda-return
+ * targets mixing one-step TD and Monte Carlo").
+ *   G_t = r_t + gamma ((1 - lambda) V_{t+1} + lambda G_{t+1}) while the episode goes on,
+ *   G_t = r_t + gamma bootstrap_value_t at a truncation, G_t = r_t at a termination,
+ *   V_T = G_T = last value.  Arguments as rlscan_gae; returns [E,T] output.
+ */
+RLSCAN_API int rlscan_lambda_returns(const float *rewards, const float *values, const float *terminateds,
+                          const float *truncateds, const float *bootstrap_values,
+                          const float *last_values, float *returns, int64_t E, int64_t T,
+                          float gamma, float lambda_, void *ws, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/*
+ * Discounted returns (README "Kernels": compute_discounted_returns,
+ * "discounted reward-to-go").
+ *   R_t = r_t + gamma R_{t+1} while the episode goes on, r_t + gamma bootstrap_value_t
+ *   at a truncation, r_t at a termination; R_T = last value.
+ * rewards required; terminateds, truncateds, last_values nullable;
+ * bootstrap_values required iff truncateds; returns [E,T] output.
+ */
+RLSCAN_API int rlscan_discounted_returns(const float *rewards, const float *terminateds,
+                              const float *truncateds, const float *bootstrap_values,
+                              const float *last_values, float *returns, int64_t E, int64_t T,
+                              float gamma, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Eligibility traces (README "Kernels": compute_eligibility_traces,
+ * "accumulating forward traces e[t] = x[t] + gamma lambda (1 - d) e[t-1]").
+ *   e_t = x_t + gamma lambda e_{t-1} if t > 0 and dones[t-1] == 0, else x_t.
+ * x required, dones nullable (no resets); traces [E,T] output.
+ */
+RLSCAN_API int rlscan_eligibility_traces(const float *x, const float *dones, float *traces, int64_t E,
+                              int64_t T, float gamma, float lambda_, void *ws, size_t ws_bytes,
+                              cudaStream_t stream);
+
+/*
+ * Episodic prefix sum (README "Kernels": compute_episodic_prefix_sum,
+ * "episodic cumulative sum with done-mask resets").
+ *   y_t = x_t + y_{t-1} if t > 0 and dones[t-1] == 0, else x_t.
+ * x and out are [E,T] of `dtype`: RLSCAN_F32 (float) or RLSCAN_I32 (int32,
+ * exact, wrapping modulo 2^32).  dones float32 [E,T], nullable.
+ */
+RLSCAN_API int rlscan_episodic_prefix_sum(const void *x, int dtype, const float *dones, void *out,
+                               int64_t E, int64_t T, void *ws, size_t ws_bytes,
+                               cudaStream_t stream);
+
+/*
+ * Workspace size in bytes that any entry point above needs for an [E, T]
+ * problem (any A); 0 if no call of that shape needs one.  Negative or
+ * overflowing shapes return 0 and the compute call then rejects them.
+ */
+RLSCAN_API size_t rlscan_workspace_bytes(int64_t E, int64_t T);
+
+/* Zero-fill a workspace on `stream` (cudaMemsetAsync). */
+RLSCAN_API int rlscan_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear this device's error word, which
+ * kernels set when a bounded wait gave up.  Returns RLSCAN_OK,
+ * RLSCAN_ERR_TIMEOUT, or RLSCAN_ERR_CUDA if the stream reports an error.
+ * For debugging and tests; compute calls never synchronise.
+ */
+RLSCAN_API int rlscan_check(cudaStream_t stream);
+
+/* Message for the last failing call on this thread ("" if none). */
+RLSCAN_API const char *rlscan_last_error(void);
+
+/* RLSCAN_VERSION of the built library. */
+RLSCAN_API int rlscan_version(void);
+
+/*
+ * Test hook for the bounded waits between tiles.  spin_limit: maximum
+ * polls (each with a short sleep) before a tile gives up waiting for its
+ * predecessor (0 restores the default, about a second).  withhold_tile: the
+ * index, in scan order, of one tile that never publishes its result (-1,
+ * the default, for none), so that a test can make the wait run out and
+ * check that rlscan_check reports RLSCAN_ERR_TIMEOUT without hanging.  Not
+ * for production use; applies to calls made after it on any thread.
+ */
+RLSCAN_API int rlscan_debug_set_lookback(uint32_t spin_limit, int64_t withhold_tile);
+
+/*
+ * Launch plan that a call of this shape takes (for tests and tools):
+ * writes tile size in elements, threads per block, whether tiles exchange
+ * carries through the workspace (1) or not (0), and the tile count.
+ * actions: 1 for every estimator except rlscan_retrace with A > 1, whose
+ * action count it is (that call stages per-action rows in shared memory and
+ * uses smaller tiles).
+ */
+RLSCAN_API int rlscan_plan(int64_t E, int64_t T, int64_t actions, int64_t *tile_elems, int *threads,
+                int *lookback, int64_t *num_tiles);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RLSCAN_H */

@@ -1,0 +1,555 @@
+// estimators.cuh - coefficient builders and epilogues of the seven rlscan
+// estimators, one struct each, plugged into tile_scan_kernel.
+//
+// Each builder turns the estimator's inputs at step t into the pair (a_t, b_t)
+// of x_t = a_t x_{t-+1} + b_t (rl-triton abstract: "algorithm-specific fused
+// kernels constructing their recurrence coefficients on-chip") and each
+// epilogue turns the scanned x_t into the estimator's outputs.  The
+// definitions follow the rl-triton README "Kernels" table (one row per
+// estimator) and its with-truncations paragraph:
+//   - terminated_t: episode ends at t, no bootstrap, trace cut (a_t = 0);
+//   - truncated_t (and not terminated): episode ends at t, bootstrap with
+//     bootstrap_values[t], trace cut;
+//   - last step of a row with no flag: bootstrap with last_values[row] (0 if
+//     absent) folded into b_t, and a_t = 0 so rows never mix;
+//   - forward estimators reset after a done: a_t = 0 when t == 0 or
+//     dones[t-1] != 0.
+#pragma once
+
+#include "scan_core.cuh"
+
+namespace rlscan {
+
+struct StepFlags {
+    bool term, trn, cont;
+};
+__device__ __forceinline__ StepFlags step_flags(float te, float tr) {
+    StepFlags f;
+    f.term = te != 0.0f;
+    f.trn = (tr != 0.0f) && !f.term;
+    f.cont = !f.term && !f.trn;
+    return f;
+}
+
+// Next element's value of a plane, seen by each thread's last element: the
+// next lane's first element, or (last lane of the warp) a direct load.
+template <int V>
+__device__ __forceinline__ float next_halo(const float *__restrict__ p, const float (&own)[V], long long i0,
+                                           long long n, int lane) {
+    float h = __shfl_down_sync(kFullMask, own[0], 1);
+    if (lane == 31) h = load_one(p, i0 + V, n);
+    return h;
+}
+// Previous element's value, seen by each thread's first element.
+template <int V>
+__device__ __forceinline__ float prev_halo(const float *__restrict__ p, const float (&own)[V], long long i0,
+                                           long long n, int lane) {
+    float h = __shfl_up_sync(kFullMask, own[V - 1], 1);
+    if (lane == 0) h = load_one(p, i0 - 1, n);
+    return h;
+}
+
+__device__ __forceinline__ float row_last_value(const float *__restrict__ lv, long long row, long long rows) {
+    return load_one(lv, row, rows);
+}
+
+// ---------------------------------------------------------------------------
+// GAE: x = A,  a_t = gamma lambda (episode goes on, not row end), b_t = delta_t
+// ---------------------------------------------------------------------------
+struct GaeEst {
+    static constexpr bool kBackward = true;
+    using AT = float;
+    using BT = float;
+    struct Params {
+        const float *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        float *advantages;
+        float gamma, lambda_;
+    };
+    template <int V>
+    struct State {
+        float r[V], v[V], te[V], tr[V], out[V];
+        float v_next;
+    };
+    template <int NT, int V>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+                                                State<V> &S, unsigned char *) {
+        load_plane<V>(P.rewards, i0, g.n, S.r);
+        load_plane<V>(P.values, i0, g.n, S.v);
+        load_plane<V>(P.terminateds, i0, g.n, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        S.v_next = next_halo<V>(P.values, S.v, i0, g.n, lane);
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+                                                  float (&a)[V], float (&b)[V]) {
+        RowPos rp = row_pos(i0, g.seq_len);
+        const float gl = P.gamma * P.lambda_;
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (i0 + k < g.n) {
+                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const bool rowend = rp.t == g.seq_len - 1;
+                float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
+                if (rowend) nv = row_last_value(P.last_values, rp.row, g.rows);
+                const float boot = f.cont ? nv : (f.trn ? __ldg(P.bootstrap_values + i0 + k) : 0.0f);
+                a[k] = (f.cont && !rowend) ? gl : 0.0f;
+                b[k] = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
+            } else {
+                a[k] = 1.0f;
+                b[k] = 0.0f;
+            }
+            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+        S.out[k] = x;
+    }
+    template <int V>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
+        store_plane<V>(P.advantages, i0, g.n, S.out);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// TD(lambda): x = G,  a_t = gamma lambda, b_t = r_t + gamma (1 - lambda) V_{t+1}
+// ---------------------------------------------------------------------------
+struct LambdaReturnsEst {
+    static constexpr bool kBackward = true;
+    using AT = float;
+    using BT = float;
+    struct Params {
+        const float *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        float *returns;
+        float gamma, lambda_;
+    };
+    template <int V>
+    struct State {
+        float r[V], v[V], te[V], tr[V], out[V];
+        float v_next;
+    };
+    template <int NT, int V>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+                                                State<V> &S, unsigned char *) {
+        load_plane<V>(P.rewards, i0, g.n, S.r);
+        load_plane<V>(P.values, i0, g.n, S.v);
+        load_plane<V>(P.terminateds, i0, g.n, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        S.v_next = next_halo<V>(P.values, S.v, i0, g.n, lane);
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+                                                  float (&a)[V], float (&b)[V]) {
+        RowPos rp = row_pos(i0, g.seq_len);
+        const float gl = P.gamma * P.lambda_;
+        const float one_minus_l = 1.0f - P.lambda_;
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (i0 + k < g.n) {
+                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const bool rowend = rp.t == g.seq_len - 1;
+                if (f.cont) {
+                    if (rowend) { // G_{t+1} = V_{t+1} = last value
+                        const float lv = row_last_value(P.last_values, rp.row, g.rows);
+                        a[k] = 0.0f;
+                        b[k] = fmaf(P.gamma, fmaf(one_minus_l, lv, P.lambda_ * lv), S.r[k]);
+                    } else {
+                        const float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
+                        a[k] = gl;
+                        b[k] = fmaf(P.gamma * one_minus_l, nv, S.r[k]);
+                    }
+                } else {
+                    a[k] = 0.0f;
+                    b[k] = f.trn ? fmaf(P.gamma, __ldg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
+                }
+            } else {
+                a[k] = 1.0f;
+                b[k] = 0.0f;
+            }
+            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+        S.out[k] = x;
+    }
+    template <int V>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
+        store_plane<V>(P.returns, i0, g.n, S.out);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Discounted returns: x = R,  a_t = gamma, b_t = r_t
+// ---------------------------------------------------------------------------
+struct ReturnsEst {
+    static constexpr bool kBackward = true;
+    using AT = float;
+    using BT = float;
+    struct Params {
+        const float *rewards, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        float *returns;
+        float gamma;
+    };
+    template <int V>
+    struct State {
+        float r[V], te[V], tr[V], out[V];
+    };
+    template <int NT, int V>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int,
+                                                State<V> &S, unsigned char *) {
+        load_plane<V>(P.rewards, i0, g.n, S.r);
+        load_plane<V>(P.terminateds, i0, g.n, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+                                                  float (&a)[V], float (&b)[V]) {
+        RowPos rp = row_pos(i0, g.seq_len);
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (i0 + k < g.n) {
+                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const bool rowend = rp.t == g.seq_len - 1;
+                if (f.cont) {
+                    a[k] = rowend ? 0.0f : P.gamma;
+                    b[k] = rowend ? fmaf(P.gamma, row_last_value(P.last_values, rp.row, g.rows), S.r[k]) : S.r[k];
+                } else {
+                    a[k] = 0.0f;
+                    b[k] = f.trn ? fmaf(P.gamma, __ldg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
+                }
+            } else {
+                a[k] = 1.0f;
+                b[k] = 0.0f;
+            }
+            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+        S.out[k] = x;
+    }
+    template <int V>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
+        store_plane<V>(P.returns, i0, g.n, S.out);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// V-Trace: x = D = vs - V,  a_t = gamma c_t, b_t = rho_t delta_t;
+// epilogue vs_t = V_t + D_t and pg_t = rho_t (r_t + gamma vs_{t+1} - V_t).
+// ---------------------------------------------------------------------------
+struct VtraceEst {
+    static constexpr bool kBackward = true;
+    using AT = float;
+    using BT = float;
+    struct Params {
+        const float *log_rhos, *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        float *vs, *pg_advantages;
+        float gamma, lambda_, rho_bar, c_bar;
+    };
+    template <int V>
+    struct State {
+        float lr[V], r[V], v[V], te[V], tr[V];
+        float rho[V], boot_pg[V]; // pg bootstrap base; vs_{t+1} adds D_{t+1} where chained
+        float vs[V], pg[V];
+        float v_next;
+        unsigned chained; // bit k: pg bootstraps on vs_{t+1}
+    };
+    template <int NT, int V>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+                                                State<V> &S, unsigned char *) {
+        load_plane<V>(P.log_rhos, i0, g.n, S.lr);
+        load_plane<V>(P.rewards, i0, g.n, S.r);
+        load_plane<V>(P.values, i0, g.n, S.v);
+        load_plane<V>(P.terminateds, i0, g.n, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        S.v_next = next_halo<V>(P.values, S.v, i0, g.n, lane);
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+                                                  float (&a)[V], float (&b)[V]) {
+        RowPos rp = row_pos(i0, g.seq_len);
+        S.chained = 0u;
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (i0 + k < g.n) {
+                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const bool rowend = rp.t == g.seq_len - 1;
+                const float ratio = expf(S.lr[k]);
+                const float rho = fminf(P.rho_bar, ratio);
+                const float c = P.lambda_ * fminf(P.c_bar, ratio);
+                float boot;
+                if (f.cont) {
+                    boot = rowend ? row_last_value(P.last_values, rp.row, g.rows)
+                                  : ((k + 1 < V) ? S.v[k + 1] : S.v_next);
+                } else {
+                    boot = f.trn ? __ldg(P.bootstrap_values + i0 + k) : 0.0f;
+                }
+                a[k] = (f.cont && !rowend) ? P.gamma * c : 0.0f;
+                b[k] = rho * (fmaf(P.gamma, boot, S.r[k]) - S.v[k]);
+                S.rho[k] = rho;
+                S.boot_pg[k] = boot;
+                if (f.cont && !rowend) S.chained |= (1u << k);
+            } else {
+                a[k] = 1.0f;
+                b[k] = 0.0f;
+                S.rho[k] = 0.0f;
+                S.boot_pg[k] = 0.0f;
+            }
+            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &P, State<V> &S, int k, float x, float x_next) {
+        S.vs[k] = S.v[k] + x;
+        // vs_{t+1} = V_{t+1} + D_{t+1}; boot_pg holds V_{t+1} where chained
+        const float boot = (S.chained >> k) & 1u ? S.boot_pg[k] + x_next : S.boot_pg[k];
+        S.pg[k] = S.rho[k] * (fmaf(P.gamma, boot, S.r[k]) - S.v[k]);
+    }
+    template <int V>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
+        store_plane<V>(P.vs, i0, g.n, S.vs);
+        store_plane<V>(P.pg_advantages, i0, g.n, S.pg);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Retrace(lambda): x = Q_ret - q,  a_t = gamma c_{t+1}, b_t = delta_t.
+// kMulti: V'_t = sum_a pi'[t,a] Q'[t,a] from the per-action rows, staged in
+// shared memory by 1-D bulk copies; otherwise V'_t = next_q_values_all[t].
+// ---------------------------------------------------------------------------
+template <bool kMulti>
+struct RetraceEst {
+    static constexpr bool kBackward = true;
+    using AT = float;
+    using BT = float;
+    struct Params {
+        const float *rewards, *q_values, *next_q_values_all, *next_target_probs, *log_rhos, *terminateds,
+            *truncateds;
+        float *q_ret;
+        long long actions;
+        float gamma, lambda_, c_bar;
+        unsigned copy_spin_limit;
+    };
+    template <int V>
+    struct State {
+        float r[V], q[V], vnext[V], lr[V], te[V], tr[V], out[V];
+        float lr_next;
+    };
+
+    // Expected next-state value of each of this thread's elements.
+    template <int NT, int V>
+    static __device__ __forceinline__ void stage_expected_values(const Params &P, const Geometry &g, long long i0,
+                                                                 State<V> &S, unsigned char *smem) {
+        constexpr int TILE = NT * V;
+        const int tid = threadIdx.x;
+        const long long tile0 = i0 - (long long)tid * V;
+        const long long left = g.n - tile0;
+        const int nvalid = left < TILE ? (int)left : TILE;
+        const int A = (int)P.actions;
+        uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
+        float *sq = reinterpret_cast<float *>(smem + 128);
+        float *sp = sq + (size_t)TILE * A;
+        float *vp = sp + (size_t)TILE * A;
+        const float *gq = P.next_q_values_all + tile0 * A;
+        const float *gp = P.next_target_probs + tile0 * A;
+        const uint32_t bytes = (uint32_t)nvalid * (uint32_t)A * 4u;
+        const bool bulk = (bytes % 16u == 0u) && ((reinterpret_cast<uintptr_t>(gq) & 15u) == 0) &&
+                          ((reinterpret_cast<uintptr_t>(gp) & 15u) == 0);
+        if (bulk) {
+            if (tid == 0) {
+                mbar_init(bar, 1);
+                mbar_arrive_expect_tx(bar, 2u * bytes);
+                bulk_copy_g2s(sq, gq, bytes, bar);
+                bulk_copy_g2s(sp, gp, bytes, bar);
+            }
+            __syncthreads(); // barrier initialised before anyone polls it
+            bool ok = mbar_try_wait(bar, 0);
+            for (unsigned polls = 0; !ok && polls < P.copy_spin_limit; ++polls) ok = mbar_try_wait(bar, 0);
+            if (!ok) atomicOr(&g_device_error, kErrCopyTimeout);
+        } else {
+            const int total = nvalid * A;
+            for (int idx = tid; idx < total; idx += NT) {
+                sq[idx] = __ldg(gq + idx);
+                sp[idx] = __ldg(gp + idx);
+            }
+            __syncthreads();
+        }
+        // one element per thread per pass, neighbouring lanes on neighbouring
+        // elements (row stride A words: at most 2-way bank conflicts for even A)
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const int e = tid + NT * k;
+            if (e < nvalid) {
+                const float *qe = sq + (size_t)e * A;
+                const float *pe = sp + (size_t)e * A;
+                float s = 0.0f;
+                for (int act = 0; act < A; ++act) s = fmaf(pe[act], qe[act], s);
+                vp[e] = s;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const int e = tid * V + k;
+            S.vnext[k] = e < nvalid ? vp[e] : 0.0f;
+        }
+    }
+
+    template <int NT, int V>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+                                                State<V> &S, unsigned char *smem) {
+        load_plane<V>(P.rewards, i0, g.n, S.r);
+        load_plane<V>(P.q_values, i0, g.n, S.q);
+        load_plane<V>(P.log_rhos, i0, g.n, S.lr);
+        load_plane<V>(P.terminateds, i0, g.n, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        S.lr_next = next_halo<V>(P.log_rhos, S.lr, i0, g.n, lane);
+        if constexpr (kMulti) {
+            stage_expected_values<NT, V>(P, g, i0, S, smem);
+        } else {
+            load_plane<V>(P.next_q_values_all, i0, g.n, S.vnext);
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+                                                  float (&a)[V], float (&b)[V]) {
+        RowPos rp = row_pos(i0, g.seq_len);
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (i0 + k < g.n) {
+                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const bool rowend = rp.t == g.seq_len - 1;
+                const float boot = f.term ? 0.0f : S.vnext[k];
+                b[k] = fmaf(P.gamma, boot, S.r[k]) - S.q[k];
+                if (f.cont && !rowend) {
+                    const float lr1 = (k + 1 < V) ? S.lr[k + 1] : S.lr_next;
+                    a[k] = P.gamma * (P.lambda_ * fminf(P.c_bar, expf(lr1)));
+                } else {
+                    a[k] = 0.0f;
+                }
+            } else {
+                a[k] = 1.0f;
+                b[k] = 0.0f;
+            }
+            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+        S.out[k] = S.q[k] + x;
+    }
+    template <int V>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
+        store_plane<V>(P.q_ret, i0, g.n, S.out);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Forward estimators.  Eligibility traces: x = e, a_t = gamma lambda,
+// b_t = x_t.  fp32 prefix sum: the same with a_t = 1 (kind tag only names
+// the kernel).
+// ---------------------------------------------------------------------------
+template <int kKind> // 0 = eligibility traces, 1 = fp32 episodic prefix sum
+struct ForwardF32Est {
+    static constexpr bool kBackward = false;
+    using AT = float;
+    using BT = float;
+    struct Params {
+        const float *x, *dones;
+        float *out;
+        float decay; // gamma lambda, or 1
+    };
+    template <int V>
+    struct State {
+        float x[V], d[V], out[V];
+        float d_prev;
+    };
+    template <int NT, int V>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+                                                State<V> &S, unsigned char *) {
+        load_plane<V>(P.x, i0, g.n, S.x);
+        load_plane<V>(P.dones, i0, g.n, S.d);
+        S.d_prev = prev_halo<V>(P.dones, S.d, i0, g.n, lane);
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+                                                  float (&a)[V], float (&b)[V]) {
+        RowPos rp = row_pos(i0, g.seq_len);
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (i0 + k < g.n) {
+                const float dp = (k > 0) ? S.d[k - 1] : S.d_prev;
+                a[k] = (rp.t == 0 || dp != 0.0f) ? 0.0f : P.decay;
+                b[k] = S.x[k];
+            } else {
+                a[k] = 1.0f;
+                b[k] = 0.0f;
+            }
+            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+        S.out[k] = x;
+    }
+    template <int V>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
+        store_plane<V>(P.out, i0, g.n, S.out);
+    }
+};
+using TracesEst = ForwardF32Est<0>;
+using PrefixF32Est = ForwardF32Est<1>;
+
+// int32 episodic prefix sum: a in {0, 1}, exact wrapping sums.
+struct PrefixI32Est {
+    static constexpr bool kBackward = false;
+    using AT = uint32_t;
+    using BT = int32_t;
+    struct Params {
+        const int32_t *x;
+        const float *dones;
+        int32_t *out;
+    };
+    template <int V>
+    struct State {
+        int32_t x[V], out[V];
+        float d[V];
+        float d_prev;
+    };
+    template <int NT, int V>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+                                                State<V> &S, unsigned char *) {
+        load_plane<V>(P.x, i0, g.n, S.x);
+        load_plane<V>(P.dones, i0, g.n, S.d);
+        S.d_prev = prev_halo<V>(P.dones, S.d, i0, g.n, lane);
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &, const Geometry &g, long long i0, State<V> &S,
+                                                  uint32_t (&a)[V], int32_t (&b)[V]) {
+        RowPos rp = row_pos(i0, g.seq_len);
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (i0 + k < g.n) {
+                const float dp = (k > 0) ? S.d[k - 1] : S.d_prev;
+                a[k] = (rp.t == 0 || dp != 0.0f) ? 0u : 1u;
+                b[k] = S.x[k];
+            } else {
+                a[k] = 1u;
+                b[k] = 0;
+            }
+            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, int32_t x, int32_t) {
+        S.out[k] = x;
+    }
+    template <int V>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
+        store_plane<V>(P.out, i0, g.n, S.out);
+    }
+};
+
+} // namespace rlscan

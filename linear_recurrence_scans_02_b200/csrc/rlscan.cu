@@ -1,0 +1,522 @@
+// rlscan.cu - host side of librlscan: argument checks, launch planning and
+// the extern "C" entry points declared in include/rlscan.h.
+//
+// Each entry point validates its arguments on the host (nothing touches the
+// GPU before the launch), picks a tile plan for the [E, T] shape, and
+// launches one tile_scan_kernel instantiation on the caller's stream with
+// programmatic dependent launch allowed, so the kernel's prologue can
+// overlap the tail of whatever ran before it on that stream.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "../../include/rlscan.h"
+#include "estimators.cuh"
+
+namespace rlscan {
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int ok() {
+    g_last_error.clear();
+    return RLSCAN_OK;
+}
+
+// About a second of polling (each poll sleeps up to ~1 us).
+constexpr unsigned kDefaultSpinLimit = 1u << 20;
+std::atomic<unsigned> g_spin_limit{kDefaultSpinLimit};
+std::atomic<long long> g_withhold{-1};
+
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *v = std::getenv("RLSCAN_DISABLE_PDL");
+        return !(v && v[0] && v[0] != '0');
+    }();
+    return on;
+}
+
+// ---------------------------------------------------------------------------
+// Tile plans.  A tile is S = NT * V consecutive elements of the flattened
+// [E*T] array.  Tiles need the look-back only when a tile boundary can fall
+// inside a row (S not a multiple of T, more than one tile).
+// ---------------------------------------------------------------------------
+enum Cfg { C512 = 0, C1024, C2048, C4096, R512, R256, R128, kNumCfg };
+constexpr int kCfgTile[kNumCfg] = {512, 1024, 2048, 4096, 512, 256, 128};
+constexpr int kCfgThreads[kNumCfg] = {128, 256, 256, 512, 128, 64, 32};
+
+struct Plan {
+    Cfg cfg;
+    bool lookback;
+    long long ntiles;
+};
+
+// Fill the GPU: with fewer tiles than this the plan prefers smaller tiles.
+constexpr long long kNumSMs = 148;
+constexpr long long kMinTiles = 2 * kNumSMs;
+
+long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+Plan make_plan(long long E, long long T, long long actions) {
+    const long long n = E * T;
+    Plan p{};
+    if (actions > 1) {
+        p.cfg = actions <= 24 ? R512 : (actions <= 48 ? R256 : R128);
+        const long long S = kCfgTile[p.cfg];
+        p.ntiles = ceil_div(n, S);
+        p.lookback = p.ntiles > 1 && (S % T) != 0;
+        return p;
+    }
+    const Cfg gen[4] = {C512, C1024, C2048, C4096};
+    // 1) tiles that hold whole rows: no look-back.  Largest such tile that
+    //    still fills the GPU, else the smallest one.
+    int aligned = -1;
+    for (int c = 3; c >= 0; --c) {
+        const long long S = kCfgTile[gen[c]];
+        if (S % T == 0 && ceil_div(n, S) >= kMinTiles) { aligned = c; break; }
+    }
+    if (aligned < 0) {
+        for (int c = 0; c < 4; ++c)
+            if (kCfgTile[gen[c]] % T == 0) { aligned = c; break; }
+    }
+    if (aligned >= 0) {
+        const long long nt = ceil_div(n, kCfgTile[gen[aligned]]);
+        const long long nt_small = ceil_div(n, kCfgTile[C512]);
+        // whole rows unless that leaves SMs idle and splitting rows would not
+        if (nt >= kNumSMs || nt_small <= nt) {
+            p.cfg = gen[aligned];
+            p.ntiles = nt;
+            p.lookback = false;
+            return p;
+        }
+        // too few whole-row tiles: split rows over 512-element tiles instead
+        p.cfg = C512;
+        p.ntiles = nt_small;
+        p.lookback = true;
+        return p;
+    }
+    // 2) rows that do not align with any tile: look-back, largest tile that
+    //    still fills the GPU.
+    p.cfg = C512;
+    for (int c = 2; c >= 0; --c) {
+        if (ceil_div(n, kCfgTile[gen[c]]) >= kMinTiles) { p.cfg = gen[c]; break; }
+    }
+    p.ntiles = ceil_div(n, kCfgTile[p.cfg]);
+    p.lookback = p.ntiles > 1;
+    return p;
+}
+
+size_t workspace_for(const Plan &p) {
+    return p.lookback ? sizeof(WsHeader) + sizeof(TileSlot) * (size_t)p.ntiles : 0;
+}
+
+size_t multi_smem_bytes(Cfg cfg, long long actions) {
+    const size_t S = (size_t)kCfgTile[cfg];
+    return 128 + (2 * S * (size_t)actions + S) * sizeof(float);
+}
+
+// ---------------------------------------------------------------------------
+// Argument checks
+// ---------------------------------------------------------------------------
+constexpr long long kMaxElems = 1ll << 40;
+
+int check_shape(long long E, long long T, long long A = 1) {
+    if (E < 0 || T < 0) return fail(RLSCAN_ERR_INVALID_ARG, "E and T must be >= 0 (got E=%lld, T=%lld)", E, T);
+    if (E > 0 && T > 0 && (E > kMaxElems / T || E * T > kMaxElems / (A > 0 ? A : 1)))
+        return fail(RLSCAN_ERR_INVALID_ARG, "E*T*A too large (E=%lld, T=%lld, A=%lld)", E, T, A);
+    if (E > 0 && T > 0 && ceil_div(E * T, 128) >= (1ll << 31) - 1)
+        return fail(RLSCAN_ERR_INVALID_ARG, "E*T too large for one launch");
+    return RLSCAN_OK;
+}
+
+int check_scalar(float v, const char *name) {
+    if (!std::isfinite(v)) return fail(RLSCAN_ERR_INVALID_ARG, "%s must be finite", name);
+    return RLSCAN_OK;
+}
+
+struct Span {
+    const void *p;
+    size_t bytes;
+    const char *name;
+};
+
+bool overlap(const Span &a, const Span &b) {
+    if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+    const uintptr_t a0 = (uintptr_t)a.p, a1 = a0 + a.bytes;
+    const uintptr_t b0 = (uintptr_t)b.p, b1 = b0 + b.bytes;
+    return a0 < b1 && b0 < a1;
+}
+
+// Every output against every input and every other output.
+int check_aliasing(const Span *ins, int nin, const Span *outs, int nout) {
+    for (int o = 0; o < nout; ++o) {
+        for (int i = 0; i < nin; ++i)
+            if (overlap(outs[o], ins[i]))
+                return fail(RLSCAN_ERR_INVALID_ARG, "output %s overlaps input %s", outs[o].name, ins[i].name);
+        for (int q = o + 1; q < nout; ++q)
+            if (overlap(outs[o], outs[q]))
+                return fail(RLSCAN_ERR_INVALID_ARG, "outputs %s and %s overlap", outs[o].name, outs[q].name);
+    }
+    return RLSCAN_OK;
+}
+
+int require(const void *p, const char *name) {
+    if (p == nullptr) return fail(RLSCAN_ERR_INVALID_ARG, "%s must not be NULL", name);
+    return RLSCAN_OK;
+}
+
+#define RLSCAN_TRY(expr)                                                                                   \
+    do {                                                                                                   \
+        int rc_ = (expr);                                                                                  \
+        if (rc_ != RLSCAN_OK) return rc_;                                                                  \
+    } while (0)
+
+// ---------------------------------------------------------------------------
+// Launch
+// ---------------------------------------------------------------------------
+template <class Est, int NT, int V, bool LB>
+cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const Lookback &lb, size_t smem,
+                       cudaStream_t stream) {
+    auto kern = tile_scan_kernel<Est, NT, V, LB>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g.ntiles);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, P, g, lb);
+}
+
+template <class Est, Cfg C>
+cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, const Lookback &lb, bool lookback,
+                       size_t smem, cudaStream_t s) {
+    constexpr int NT = kCfgThreads[C];
+    constexpr int V = kCfgTile[C] / NT;
+    return lookback ? launch_one<Est, NT, V, true>(P, g, lb, smem, s)
+                    : launch_one<Est, NT, V, false>(P, g, lb, smem, s);
+}
+
+template <class Est>
+int run(const char *name, const typename Est::Params &P, long long E, long long T, long long actions, void *ws,
+        size_t ws_bytes, cudaStream_t stream) {
+    const Plan plan = make_plan(E, T, actions);
+    Geometry g;
+    g.n = E * T;
+    g.seq_len = T;
+    g.ntiles = plan.ntiles;
+    g.rows = E;
+    Lookback lb{};
+    lb.withhold = -1;
+    lb.spin_limit = g_spin_limit.load();
+    if (plan.lookback) {
+        const size_t need = workspace_for(plan);
+        if (ws == nullptr || ws_bytes < need)
+            return fail(RLSCAN_ERR_WORKSPACE, "%s: shape E=%lld T=%lld needs a %zu-byte workspace (got %s, %zu bytes)",
+                        name, E, T, need, ws ? "a buffer" : "NULL", ws_bytes);
+        if (((uintptr_t)ws & 15u) != 0) return fail(RLSCAN_ERR_WORKSPACE, "%s: workspace must be 16-byte aligned", name);
+        lb.hdr = static_cast<WsHeader *>(ws);
+        lb.slots = reinterpret_cast<TileSlot *>(static_cast<char *>(ws) + sizeof(WsHeader));
+        lb.withhold = g_withhold.load();
+    }
+    const size_t smem = actions > 1 ? multi_smem_bytes(plan.cfg, actions) : 0;
+    cudaError_t e;
+    switch (plan.cfg) {
+    case C512: e = launch_cfg<Est, C512>(P, g, lb, plan.lookback, smem, stream); break;
+    case C1024: e = launch_cfg<Est, C1024>(P, g, lb, plan.lookback, smem, stream); break;
+    case C2048: e = launch_cfg<Est, C2048>(P, g, lb, plan.lookback, smem, stream); break;
+    case C4096: e = launch_cfg<Est, C4096>(P, g, lb, plan.lookback, smem, stream); break;
+    default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+    }
+    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
+    return ok();
+}
+
+// Multi-action Retrace uses its own (smaller) tiles; the register-only
+// configurations are never instantiated for it and vice versa.
+template <class Est>
+int run_multi(const char *name, const typename Est::Params &P, long long E, long long T, long long actions,
+              void *ws, size_t ws_bytes, cudaStream_t stream) {
+    const Plan plan = make_plan(E, T, actions);
+    Geometry g;
+    g.n = E * T;
+    g.seq_len = T;
+    g.ntiles = plan.ntiles;
+    g.rows = E;
+    Lookback lb{};
+    lb.withhold = -1;
+    lb.spin_limit = g_spin_limit.load();
+    if (plan.lookback) {
+        const size_t need = workspace_for(plan);
+        if (ws == nullptr || ws_bytes < need)
+            return fail(RLSCAN_ERR_WORKSPACE, "%s: shape E=%lld T=%lld A=%lld needs a %zu-byte workspace", name, E, T,
+                        actions, need);
+        if (((uintptr_t)ws & 15u) != 0) return fail(RLSCAN_ERR_WORKSPACE, "%s: workspace must be 16-byte aligned", name);
+        lb.hdr = static_cast<WsHeader *>(ws);
+        lb.slots = reinterpret_cast<TileSlot *>(static_cast<char *>(ws) + sizeof(WsHeader));
+        lb.withhold = g_withhold.load();
+    }
+    const size_t smem = multi_smem_bytes(plan.cfg, actions);
+    cudaError_t e;
+    switch (plan.cfg) {
+    case R512: e = launch_cfg<Est, R512>(P, g, lb, plan.lookback, smem, stream); break;
+    case R256: e = launch_cfg<Est, R256>(P, g, lb, plan.lookback, smem, stream); break;
+    case R128: e = launch_cfg<Est, R128>(P, g, lb, plan.lookback, smem, stream); break;
+    default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+    }
+    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
+    return ok();
+}
+
+size_t plane_bytes(long long E, long long T) { return (size_t)(E * T) * sizeof(float); }
+
+} // namespace
+} // namespace rlscan
+
+using namespace rlscan;
+
+extern "C" {
+
+int rlscan_gae(const float *rewards, const float *values, const float *terminateds, const float *truncateds,
+               const float *bootstrap_values, const float *last_values, float *advantages, int64_t E, int64_t T,
+               float gamma, float lambda_, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(values, "values"));
+    RLSCAN_TRY(require(advantages, "advantages"));
+    if (truncateds && !bootstrap_values) return fail(RLSCAN_ERR_INVALID_ARG, "truncateds given without bootstrap_values");
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{rewards, pb, "rewards"}, {values, pb, "values"}, {terminateds, pb, "terminateds"},
+                        {truncateds, pb, "truncateds"}, {bootstrap_values, pb, "bootstrap_values"},
+                        {last_values, (size_t)E * 4, "last_values"}};
+    const Span outs[] = {{advantages, pb, "advantages"}};
+    RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
+    GaeEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
+                     last_values, advantages, gamma, lambda_};
+    return run<GaeEst>("rlscan_gae", P, E, T, 1, ws, ws_bytes, stream);
+}
+
+int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
+                  const float *truncateds, const float *bootstrap_values, const float *last_values, float *vs,
+                  float *pg_advantages, int64_t E, int64_t T, float gamma, float lambda_, float rho_bar,
+                  float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    RLSCAN_TRY(check_scalar(rho_bar, "rho_bar"));
+    RLSCAN_TRY(check_scalar(c_bar, "c_bar"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(log_rhos, "log_rhos"));
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(values, "values"));
+    RLSCAN_TRY(require(vs, "vs"));
+    RLSCAN_TRY(require(pg_advantages, "pg_advantages"));
+    if (truncateds && !bootstrap_values) return fail(RLSCAN_ERR_INVALID_ARG, "truncateds given without bootstrap_values");
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{log_rhos, pb, "log_rhos"}, {rewards, pb, "rewards"}, {values, pb, "values"},
+                        {terminateds, pb, "terminateds"}, {truncateds, pb, "truncateds"},
+                        {bootstrap_values, pb, "bootstrap_values"}, {last_values, (size_t)E * 4, "last_values"}};
+    const Span outs[] = {{vs, pb, "vs"}, {pg_advantages, pb, "pg_advantages"}};
+    RLSCAN_TRY(check_aliasing(ins, 7, outs, 2));
+    VtraceEst::Params P{log_rhos, rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
+                        last_values, vs, pg_advantages, gamma, lambda_, rho_bar, c_bar};
+    return run<VtraceEst>("rlscan_vtrace", P, E, T, 1, ws, ws_bytes, stream);
+}
+
+int rlscan_retrace(const float *rewards, const float *q_values, const float *next_q_values_all,
+                   const float *next_target_probs, const float *log_rhos, const float *terminateds,
+                   const float *truncateds, float *q_ret, int64_t E, int64_t T, int64_t A, float gamma,
+                   float lambda_, float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    if (A < 1) return fail(RLSCAN_ERR_INVALID_ARG, "A must be >= 1 (got %lld)", (long long)A);
+    if (A > RLSCAN_MAX_ACTIONS)
+        return fail(RLSCAN_ERR_UNSUPPORTED, "A=%lld exceeds RLSCAN_MAX_ACTIONS=%d", (long long)A, RLSCAN_MAX_ACTIONS);
+    RLSCAN_TRY(check_shape(E, T, A));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    RLSCAN_TRY(check_scalar(c_bar, "c_bar"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(q_values, "q_values"));
+    RLSCAN_TRY(require(next_q_values_all, "next_q_values_all"));
+    RLSCAN_TRY(require(log_rhos, "log_rhos"));
+    RLSCAN_TRY(require(terminateds, "terminateds"));
+    RLSCAN_TRY(require(truncateds, "truncateds"));
+    RLSCAN_TRY(require(q_ret, "q_ret"));
+    if (A > 1 && next_target_probs == nullptr)
+        return fail(RLSCAN_ERR_INVALID_ARG, "next_target_probs is required when A > 1");
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{rewards, pb, "rewards"}, {q_values, pb, "q_values"},
+                        {next_q_values_all, pb * (size_t)A, "next_q_values_all"},
+                        {A > 1 ? next_target_probs : nullptr, pb * (size_t)A, "next_target_probs"},
+                        {log_rhos, pb, "log_rhos"}, {terminateds, pb, "terminateds"}, {truncateds, pb, "truncateds"}};
+    const Span outs[] = {{q_ret, pb, "q_ret"}};
+    RLSCAN_TRY(check_aliasing(ins, 7, outs, 1));
+    if (A == 1) {
+        RetraceEst<false>::Params P{rewards, q_values, next_q_values_all, nullptr, log_rhos, terminateds,
+                                    truncateds, q_ret, 1, gamma, lambda_, c_bar, 0u};
+        return run<RetraceEst<false>>("rlscan_retrace", P, E, T, 1, ws, ws_bytes, stream);
+    }
+    RetraceEst<true>::Params P{rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds,
+                               truncateds, q_ret, A, gamma, lambda_, c_bar, 1u << 24};
+    return run_multi<RetraceEst<true>>("rlscan_retrace", P, E, T, A, ws, ws_bytes, stream);
+}
+
+int rlscan_lambda_returns(const float *rewards, const float *values, const float *terminateds,
+                          const float *truncateds, const float *bootstrap_values, const float *last_values,
+                          float *returns, int64_t E, int64_t T, float gamma, float lambda_, void *ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(values, "values"));
+    RLSCAN_TRY(require(returns, "returns"));
+    if (truncateds && !bootstrap_values) return fail(RLSCAN_ERR_INVALID_ARG, "truncateds given without bootstrap_values");
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{rewards, pb, "rewards"}, {values, pb, "values"}, {terminateds, pb, "terminateds"},
+                        {truncateds, pb, "truncateds"}, {bootstrap_values, pb, "bootstrap_values"},
+                        {last_values, (size_t)E * 4, "last_values"}};
+    const Span outs[] = {{returns, pb, "returns"}};
+    RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
+    LambdaReturnsEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
+                               last_values, returns, gamma, lambda_};
+    return run<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, 1, ws, ws_bytes, stream);
+}
+
+int rlscan_discounted_returns(const float *rewards, const float *terminateds, const float *truncateds,
+                              const float *bootstrap_values, const float *last_values, float *returns, int64_t E,
+                              int64_t T, float gamma, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(returns, "returns"));
+    if (truncateds && !bootstrap_values) return fail(RLSCAN_ERR_INVALID_ARG, "truncateds given without bootstrap_values");
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{rewards, pb, "rewards"}, {terminateds, pb, "terminateds"}, {truncateds, pb, "truncateds"},
+                        {bootstrap_values, pb, "bootstrap_values"}, {last_values, (size_t)E * 4, "last_values"}};
+    const Span outs[] = {{returns, pb, "returns"}};
+    RLSCAN_TRY(check_aliasing(ins, 5, outs, 1));
+    ReturnsEst::Params P{rewards, terminateds, truncateds, truncateds ? bootstrap_values : nullptr, last_values,
+                         returns, gamma};
+    return run<ReturnsEst>("rlscan_discounted_returns", P, E, T, 1, ws, ws_bytes, stream);
+}
+
+int rlscan_eligibility_traces(const float *x, const float *dones, float *traces, int64_t E, int64_t T, float gamma,
+                              float lambda_, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(x, "x"));
+    RLSCAN_TRY(require(traces, "traces"));
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{x, pb, "x"}, {dones, pb, "dones"}};
+    const Span outs[] = {{traces, pb, "traces"}};
+    RLSCAN_TRY(check_aliasing(ins, 2, outs, 1));
+    TracesEst::Params P{x, dones, traces, gamma * lambda_};
+    return run<TracesEst>("rlscan_eligibility_traces", P, E, T, 1, ws, ws_bytes, stream);
+}
+
+int rlscan_episodic_prefix_sum(const void *x, int dtype, const float *dones, void *out, int64_t E, int64_t T,
+                               void *ws, size_t ws_bytes, cudaStream_t stream) {
+    if (dtype != RLSCAN_F32 && dtype != RLSCAN_I32) return fail(RLSCAN_ERR_UNSUPPORTED, "unknown dtype %d", dtype);
+    RLSCAN_TRY(check_shape(E, T));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(x, "x"));
+    RLSCAN_TRY(require(out, "out"));
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{x, pb, "x"}, {dones, pb, "dones"}};
+    const Span outs[] = {{out, pb, "out"}};
+    RLSCAN_TRY(check_aliasing(ins, 2, outs, 1));
+    if (dtype == RLSCAN_F32) {
+        PrefixF32Est::Params P{static_cast<const float *>(x), dones, static_cast<float *>(out), 1.0f};
+        return run<PrefixF32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream);
+    }
+    PrefixI32Est::Params P{static_cast<const int32_t *>(x), dones, static_cast<int32_t *>(out)};
+    return run<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream);
+}
+
+size_t rlscan_workspace_bytes(int64_t E, int64_t T) {
+    if (E <= 0 || T <= 0 || E > kMaxElems / T) return 0;
+    size_t need = 0;
+    const long long probe_actions[] = {1, 2, 25, 49};
+    for (long long a : probe_actions) {
+        const size_t w = workspace_for(make_plan(E, T, a));
+        if (w > need) need = w;
+    }
+    return need;
+}
+
+int rlscan_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream) {
+    if (ws_bytes == 0) return ok();
+    if (ws == nullptr) return fail(RLSCAN_ERR_INVALID_ARG, "ws must not be NULL");
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, stream);
+    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int rlscan_check(cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "stream error: %s", cudaGetErrorString(e));
+    unsigned word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof word);
+    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+    if (word != 0) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+        if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "clearing the error word: %s", cudaGetErrorString(e));
+        return fail(RLSCAN_ERR_TIMEOUT, "a kernel gave up a bounded wait (error word 0x%x)", word);
+    }
+    return ok();
+}
+
+const char *rlscan_last_error(void) { return g_last_error.c_str(); }
+
+int rlscan_version(void) { return RLSCAN_VERSION; }
+
+int rlscan_debug_set_lookback(uint32_t spin_limit, int64_t withhold_tile) {
+    g_spin_limit.store(spin_limit == 0 ? kDefaultSpinLimit : spin_limit);
+    g_withhold.store(withhold_tile < 0 ? -1 : (long long)withhold_tile);
+    return ok();
+}
+
+int rlscan_plan(int64_t E, int64_t T, int64_t actions, int64_t *tile_elems, int *threads, int *lookback,
+                int64_t *num_tiles) {
+    if (E <= 0 || T <= 0) return fail(RLSCAN_ERR_INVALID_ARG, "E and T must be > 0");
+    if (actions < 1 || actions > RLSCAN_MAX_ACTIONS) return fail(RLSCAN_ERR_INVALID_ARG, "bad action count");
+    RLSCAN_TRY(check_shape(E, T, actions));
+    const Plan p = make_plan(E, T, actions);
+    if (tile_elems) *tile_elems = kCfgTile[p.cfg];
+    if (threads) *threads = kCfgThreads[p.cfg];
+    if (lookback) *lookback = p.lookback ? 1 : 0;
+    if (num_tiles) *num_tiles = p.ntiles;
+    return ok();
+}
+
+} // extern "C"

@@ -1,0 +1,523 @@
+// scan_core.cuh - the tile scan shared by every rlscan estimator.
+//
+// The rl-triton paper (arXiv:2608.17641, abstract) solves every estimator as
+// one first-order linear recurrence x_t = a_t x_{t-+1} + b_t with the
+// associative operator (a1, b1) o (a2, b2) = (a1 a2, a1 b2 + b1), where
+// (a2, b2) is the map applied first.  This file holds that operator and one
+// single-pass scan over the flattened [E*T] array:
+//
+//   * the array is cut into tiles of S = NT*V consecutive elements, one CTA
+//     per tile; each thread owns V consecutive elements (128-bit loads);
+//   * rows never leak into each other because each estimator's coefficient
+//     builder sets a = 0 on the first element of a row in scan order (the
+//     row's last value is folded into b there), the same cut a done makes;
+//   * in-thread sequential compose -> warp shuffle scan -> shared-memory scan
+//     of warp aggregates -> (optional) decoupled look-back over the
+//     aggregates of earlier tiles -> per-thread carry -> sequential epilogue;
+//   * look-back is only compiled in when a tile boundary can fall inside a
+//     row; tiles take their scan-order index from an atomic counter so a
+//     tile only ever waits for tiles that are already running, and every
+//     wait is bounded.
+//
+// Scan order is memory order for forward recurrences and reversed memory
+// order for backward ones.  "Earlier" below always means earlier in scan
+// order.
+#pragma once
+
+#include <cstdint>
+#include <type_traits>
+#include <cuda_runtime.h>
+
+namespace rlscan {
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+// Device-wide error word: bit 0 = a look-back wait gave up, bit 1 = a bulk
+// copy wait gave up, bit 2 = a workspace was not zero-filled at launch.
+// Read and cleared by rlscan_check().
+__device__ unsigned int g_device_error = 0;
+constexpr unsigned kErrLookbackTimeout = 1u;
+constexpr unsigned kErrCopyTimeout = 2u;
+constexpr unsigned kErrWorkspaceState = 4u; // workspace was not zero-filled at launch
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+
+// Programmatic dependent launch: wait until the preceding grid on the stream
+// has completed and its memory is visible (a no-op without the launch
+// attribute), and let the next grid start its prologue early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_gpu(unsigned *p, unsigned v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// mbarrier + 1-D bulk copy (TMA engine, no tensor map, no multicast).
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+// Copy `bytes` (multiple of 16; both addresses 16-byte aligned) from global
+// to this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Scan algebra.  A pair (a, b) is the map x -> a x + b.  combine(p1, p2)
+// replaces p1 with p1 o p2 (p2 applied first).  a == 0 cuts the chain: the
+// earlier value is not read, so a non-finite value never crosses an episode
+// or row boundary.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float apply_pair(float a, float b, float x) { return a == 0.0f ? b : fmaf(a, x, b); }
+__device__ __forceinline__ void combine(float &a1, float &b1, float a2, float b2) {
+    b1 = apply_pair(a1, b1, b2);
+    a1 = a1 * a2;
+}
+__device__ __forceinline__ float identity_a(float) { return 1.0f; }
+__device__ __forceinline__ float identity_b(float) { return 0.0f; }
+__device__ __forceinline__ unsigned to_bits(float v) { return __float_as_uint(v); }
+__device__ __forceinline__ float from_bits(unsigned u, float) { return __uint_as_float(u); }
+
+// Integer pairs with a 0/1 multiplier: exact two's-complement sums.
+__device__ __forceinline__ int32_t apply_pair(uint32_t a, int32_t b, int32_t x) {
+    return a ? static_cast<int32_t>(static_cast<uint32_t>(b) + static_cast<uint32_t>(x)) : b;
+}
+__device__ __forceinline__ void combine(uint32_t &a1, int32_t &b1, uint32_t a2, int32_t b2) {
+    b1 = apply_pair(a1, b1, b2);
+    a1 = a1 & a2;
+}
+__device__ __forceinline__ uint32_t identity_a(uint32_t) { return 1u; }
+__device__ __forceinline__ int32_t identity_b(int32_t) { return 0; }
+__device__ __forceinline__ unsigned to_bits(uint32_t v) { return v; }
+__device__ __forceinline__ unsigned to_bits(int32_t v) { return static_cast<unsigned>(v); }
+__device__ __forceinline__ uint32_t from_bits(unsigned u, uint32_t) { return u; }
+__device__ __forceinline__ int32_t from_bits(unsigned u, int32_t) { return static_cast<int32_t>(u); }
+
+// Inclusive warp scan in scan order: forward = increasing lane, backward =
+// decreasing lane.
+template <bool kBackward, class AT, class BT>
+__device__ __forceinline__ void warp_inclusive_scan(AT &a, BT &b, int lane) {
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        if (kBackward) {
+            AT ao = __shfl_down_sync(kFullMask, a, d);
+            BT bo = __shfl_down_sync(kFullMask, b, d);
+            if (lane + d < 32) combine(a, b, ao, bo);
+        } else {
+            AT ao = __shfl_up_sync(kFullMask, a, d);
+            BT bo = __shfl_up_sync(kFullMask, b, d);
+            if (lane >= d) combine(a, b, ao, bo);
+        }
+    }
+}
+
+// Exclusive value of an inclusive warp scan (identity on the first lane in
+// scan order).
+template <bool kBackward, class AT, class BT>
+__device__ __forceinline__ void warp_exclusive_from_inclusive(AT ia, BT ib, int lane, AT &ea, BT &eb) {
+    if (kBackward) {
+        ea = __shfl_down_sync(kFullMask, ia, 1);
+        eb = __shfl_down_sync(kFullMask, ib, 1);
+        if (lane == 31) { ea = identity_a(ia); eb = identity_b(ib); }
+    } else {
+        ea = __shfl_up_sync(kFullMask, ia, 1);
+        eb = __shfl_up_sync(kFullMask, ib, 1);
+        if (lane == 0) { ea = identity_a(ia); eb = identity_b(ib); }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Workspace for the look-back: a header with the tile counter, and one
+// 16-byte slot per tile.  status: 0 = nothing yet, 1 = the tile's aggregate
+// (a, b) is published, 2 = its inclusive value x (the carry into the next
+// tile) is published.  The last CTA to finish zeroes every status and both
+// counters, so the workspace is left as it was found.
+// ---------------------------------------------------------------------------
+
+struct WsHeader {
+    unsigned tile_counter;
+    unsigned done_counter;
+    unsigned pad[30];
+};
+static_assert(sizeof(WsHeader) == 128, "header is one 128-byte line");
+
+struct TileSlot {
+    unsigned status;
+    unsigned a;
+    unsigned b;
+    unsigned x;
+};
+static_assert(sizeof(TileSlot) == 16, "slot is 16 bytes");
+
+struct Lookback {
+    WsHeader *hdr;       // nullptr when the launch needs no look-back
+    TileSlot *slots;
+    unsigned spin_limit; // polls before a wait gives up
+    long long withhold;  // scan-order tile that never publishes (test hook), -1 = none
+};
+
+// Geometry of one launch over the flattened [E*T] array.
+struct Geometry {
+    long long n;       // E * T
+    long long seq_len; // T
+    long long ntiles;
+    long long rows;    // E
+};
+
+// Element (scan) position helpers: t index and row of the element at flat
+// index i, computed once per thread and then advanced element by element.
+struct RowPos {
+    long long t;
+    long long row;
+};
+__device__ __forceinline__ RowPos row_pos(long long i, long long T) {
+    RowPos p;
+    if (i < 0) i = 0;
+    if ((unsigned long long)i <= 0xffffffffull && (unsigned long long)T <= 0xffffffffull) {
+        unsigned ui = (unsigned)i, ut = (unsigned)T;
+        p.row = ui / ut;
+        p.t = ui - (unsigned)p.row * ut;
+    } else {
+        p.row = i / T;
+        p.t = i - p.row * T;
+    }
+    return p;
+}
+
+// Single-lane decoupled look-back.  Publishes this tile's aggregate (or its
+// inclusive value when it needs no carry), walks back over earlier tiles
+// composing their aggregates until it meets an inclusive value or an
+// aggregate that cuts the chain (a == 0), publishes its own inclusive value
+// and returns the carry into this tile.
+template <class AT, class BT>
+__device__ BT lookback_carry(const Lookback &lb, long long j, bool needs_carry, AT ta, BT tb) {
+    TileSlot *me = lb.slots + j;
+    const bool publish = (j != lb.withhold);
+    if (!needs_carry) {
+        if (publish) {
+            st_relaxed_gpu(&me->x, to_bits(tb));
+            st_release_gpu(&me->status, 2u);
+        }
+        return identity_b(tb);
+    }
+    const bool cut = (ta == AT(0)); // the tile's own chain is cut: its output needs no carry
+    if (publish) {
+        if (cut) {
+            st_relaxed_gpu(&me->x, to_bits(tb));
+            st_release_gpu(&me->status, 2u);
+        } else {
+            st_relaxed_gpu(&me->a, to_bits(ta));
+            st_relaxed_gpu(&me->b, to_bits(tb));
+            st_release_gpu(&me->status, 1u);
+        }
+    }
+    AT acc_a = identity_a(ta);
+    BT acc_b = identity_b(tb);
+    BT carry = identity_b(tb);
+    for (long long k = j - 1;; --k) {
+        if (k < 0) { // unreachable: scan-order tile 0 never needs a carry
+            atomicOr(&g_device_error, kErrLookbackTimeout);
+            carry = acc_b;
+            break;
+        }
+        const TileSlot *s = lb.slots + k;
+        unsigned st = ld_acquire_gpu(&s->status);
+        unsigned ns = 32, polls = 0;
+        while (st == 0u) {
+            if (++polls > lb.spin_limit) break;
+            __nanosleep(ns);
+            if (ns < 1024u) ns <<= 1;
+            st = ld_acquire_gpu(&s->status);
+        }
+        if (st == 0u) { // gave up: report, and continue as if the carry were zero
+            atomicOr(&g_device_error, kErrLookbackTimeout);
+            carry = acc_b;
+            break;
+        }
+        if (st == 2u) {
+            BT xk = from_bits(ld_relaxed_gpu(&s->x), tb);
+            carry = apply_pair(acc_a, acc_b, xk);
+            break;
+        }
+        AT ak = from_bits(ld_relaxed_gpu(&s->a), ta);
+        BT bk = from_bits(ld_relaxed_gpu(&s->b), tb);
+        combine(acc_a, acc_b, ak, bk);
+        if (ak == AT(0)) { // the earlier chain is cut here
+            carry = acc_b;
+            break;
+        }
+    }
+    if (publish && !cut) {
+        st_relaxed_gpu(&me->x, to_bits(apply_pair(ta, tb, carry)));
+        st_release_gpu(&me->status, 2u);
+    }
+    return carry;
+}
+
+// Last CTA out resets the workspace.
+template <int NT>
+__device__ __forceinline__ void lookback_release(const Lookback &lb, long long ntiles) {
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        unsigned prev = atomicAdd(&lb.hdr->done_counter, 1u);
+        s_last = (prev == (unsigned)(ntiles - 1));
+        __threadfence();
+    }
+    __syncthreads();
+    if (s_last) {
+        for (long long i = threadIdx.x; i < ntiles; i += NT) lb.slots[i].status = 0u;
+        if (threadIdx.x == 0) {
+            lb.hdr->tile_counter = 0u;
+            lb.hdr->done_counter = 0u;
+        }
+        __threadfence();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Vector loads / stores of V consecutive elements (V a multiple of 4).  The
+// 128-bit path needs a 16-byte-aligned base and a full vector; otherwise each
+// element is loaded on its own.  Elements at or past n read as zero / are not
+// written.  A null plane reads as zeros.
+// ---------------------------------------------------------------------------
+
+template <int V, class T>
+__device__ __forceinline__ void load_plane(const T *__restrict__ p, long long i0, long long n, T (&o)[V]) {
+    static_assert(V % 4 == 0, "V must be a multiple of 4");
+    static_assert(sizeof(T) == 4, "32-bit planes only");
+    if (p == nullptr) {
+#pragma unroll
+        for (int k = 0; k < V; ++k) o[k] = T(0);
+        return;
+    }
+    const bool vec = ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) && (i0 + V <= n);
+    if (vec) {
+#pragma unroll
+        for (int k = 0; k < V; k += 4) {
+            if constexpr (std::is_same<T, float>::value) {
+                float4 q = __ldg(reinterpret_cast<const float4 *>(p + i0 + k));
+                o[k] = q.x; o[k + 1] = q.y; o[k + 2] = q.z; o[k + 3] = q.w;
+            } else {
+                int4 q = __ldg(reinterpret_cast<const int4 *>(p + i0 + k));
+                o[k] = q.x; o[k + 1] = q.y; o[k + 2] = q.z; o[k + 3] = q.w;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < V; ++k) o[k] = (i0 + k < n && i0 + k >= 0) ? __ldg(p + i0 + k) : T(0);
+    }
+}
+
+template <int V, class T>
+__device__ __forceinline__ void store_plane(T *__restrict__ p, long long i0, long long n, const T (&o)[V]) {
+    const bool vec = ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) && (i0 + V <= n);
+    if (vec) {
+#pragma unroll
+        for (int k = 0; k < V; k += 4) {
+            if constexpr (std::is_same<T, float>::value) {
+                __stcs(reinterpret_cast<float4 *>(p + i0 + k), make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]));
+            } else {
+                __stcs(reinterpret_cast<int4 *>(p + i0 + k), make_int4(o[k], o[k + 1], o[k + 2], o[k + 3]));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < V; ++k)
+            if (i0 + k < n) p[i0 + k] = o[k];
+    }
+}
+
+// Scalar element of a plane (null -> 0), for halos and rare reads.
+template <class T>
+__device__ __forceinline__ T load_one(const T *__restrict__ p, long long i, long long n) {
+    return (p != nullptr && i >= 0 && i < n) ? __ldg(p + i) : T(0);
+}
+
+// ---------------------------------------------------------------------------
+// The tile kernel.  Est supplies (see estimators.cuh):
+//   kBackward, AT, BT, Params, State<V>,
+//   load<NT, V>(P, g, i0, lane, S, dyn_smem)    -- every thread, incl. past n
+//   coeffs<V>(P, g, i0, S, a, b)                -- (a, b) per element, identity past n
+//   out<V>(P, S, k, x, x_prev)                  -- record output k (x_prev = value
+//                                                  of the element before it in scan order)
+//   store<V>(P, g, i0, S)
+// ---------------------------------------------------------------------------
+
+template <class Est, int NT, int V, bool kLookback>
+__global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Params P, const Geometry g,
+                                                       const Lookback lb) {
+    using AT = typename Est::AT;
+    using BT = typename Est::BT;
+    constexpr bool kBwd = Est::kBackward;
+    constexpr int NW = NT / 32;
+    static_assert(NT % 32 == 0 && NW <= 32, "block must be whole warps, at most 32");
+
+    __shared__ AT s_wa[NW];
+    __shared__ BT s_wb[NW];
+    __shared__ BT s_wx[NW];
+    __shared__ long long s_tile;
+    extern __shared__ __align__(128) unsigned char dyn_smem[];
+
+    griddep_wait();
+    griddep_launch_dependents();
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+
+    long long j; // tile index in scan order
+    if constexpr (kLookback) {
+        if (tid == 0) s_tile = (long long)atomicAdd(&lb.hdr->tile_counter, 1u);
+        __syncthreads();
+        j = s_tile;
+        if (j >= g.ntiles) { // counter was not zero at launch: touch nothing, report
+            if (tid == 0) atomicOr(&g_device_error, kErrWorkspaceState);
+            return;
+        }
+    } else {
+        j = blockIdx.x;
+    }
+    const long long m = kBwd ? (g.ntiles - 1 - j) : j; // tile index in memory
+    const long long tile0 = m * (long long)(NT * V);
+    const long long i0 = tile0 + (long long)tid * V;
+
+    typename Est::template State<V> S;
+    Est::template load<NT, V>(P, g, i0, lane, S, dyn_smem);
+
+    AT a[V];
+    BT b[V];
+    Est::template coeffs<V>(P, g, i0, S, a, b);
+
+    // thread aggregate, composed in scan order
+    AT ta;
+    BT tb;
+    if (kBwd) {
+        ta = a[V - 1];
+        tb = b[V - 1];
+#pragma unroll
+        for (int k = V - 2; k >= 0; --k) {
+            AT na = a[k];
+            BT nb = b[k];
+            combine(na, nb, ta, tb);
+            ta = na;
+            tb = nb;
+        }
+    } else {
+        ta = a[0];
+        tb = b[0];
+#pragma unroll
+        for (int k = 1; k < V; ++k) {
+            AT na = a[k];
+            BT nb = b[k];
+            combine(na, nb, ta, tb);
+            ta = na;
+            tb = nb;
+        }
+    }
+
+    AT ia = ta;
+    BT ib = tb;
+    warp_inclusive_scan<kBwd>(ia, ib, lane);
+    AT ea;
+    BT eb;
+    warp_exclusive_from_inclusive<kBwd>(ia, ib, lane, ea, eb);
+    if (lane == (kBwd ? 0 : 31)) {
+        s_wa[warp] = ia;
+        s_wb[warp] = ib;
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        AT wa = lane < NW ? s_wa[lane] : identity_a(ta);
+        BT wb = lane < NW ? s_wb[lane] : identity_b(tb);
+        warp_inclusive_scan<kBwd>(wa, wb, lane);
+        AT wea;
+        BT web;
+        warp_exclusive_from_inclusive<kBwd>(wa, wb, lane, wea, web);
+        BT carry = identity_b(tb);
+        if constexpr (kLookback) {
+            const AT tile_a = __shfl_sync(kFullMask, wa, kBwd ? 0 : NW - 1);
+            const BT tile_b = __shfl_sync(kFullMask, wb, kBwd ? 0 : NW - 1);
+            if (lane == 0) {
+                bool needs_carry;
+                if (kBwd) {
+                    const long long end = tile0 + (long long)(NT * V);
+                    needs_carry = end < g.n && (end % g.seq_len) != 0;
+                } else {
+                    needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
+                }
+                carry = lookback_carry<AT, BT>(lb, j, needs_carry, tile_a, tile_b);
+            }
+            carry = __shfl_sync(kFullMask, carry, 0);
+        }
+        if (lane < NW) s_wx[lane] = apply_pair(wea, web, carry);
+    }
+    __syncthreads();
+
+    // sequential epilogue over this thread's elements in scan order
+    BT x = apply_pair(ea, eb, s_wx[warp]);
+    if (kBwd) {
+#pragma unroll
+        for (int k = V - 1; k >= 0; --k) {
+            const BT prev = x;
+            x = apply_pair(a[k], b[k], x);
+            Est::template out<V>(P, S, k, x, prev);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const BT prev = x;
+            x = apply_pair(a[k], b[k], x);
+            Est::template out<V>(P, S, k, x, prev);
+        }
+    }
+    Est::template store<V>(P, g, i0, S);
+
+    if constexpr (kLookback) lookback_release<NT>(lb, g.ntiles);
+}
+
+} // namespace rlscan

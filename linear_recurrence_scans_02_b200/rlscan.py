@@ -1,0 +1,355 @@
+"""Thin ctypes binding of ``librlscan.so`` (C ABI declared in include/rlscan.h).
+
+Argument marshalling only: every step of every estimator runs in the CUDA
+kernels behind the C entry points.  PyTorch supplies device memory and the
+current CUDA stream.  There is no fallback: if the library is missing this
+module fails to import, and the C calls fail on a machine without a GPU.
+
+Two layers, named after the C ABI and the rl-triton README ("Kernels" table
+and "Usage" example):
+
+* ``rlscan_<estimator>(...)`` - the C call with tensors: inputs and
+  preallocated outputs, E and T taken from the tensor shapes, the workspace
+  supplied from a per-stream cache when the shape needs one, the stream being
+  ``torch.cuda.current_stream()``.
+* ``compute_<estimator>(...)`` - allocate the outputs and call the above;
+  ``compute_gae(rewards, values, terminateds, gamma=..., lambda_=...)`` is the
+  README's usage line.
+
+All tensors are CUDA, contiguous, float32 ``[E, T]`` (int32 allowed for the
+prefix sum input/output, ``[E, T, A]`` for Retrace's per-action arrays).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import _build
+
+__all__ = [
+    "RlscanError", "library_path",
+    "rlscan_gae", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
+    "rlscan_discounted_returns", "rlscan_eligibility_traces", "rlscan_episodic_prefix_sum",
+    "rlscan_workspace_bytes", "rlscan_check", "rlscan_plan", "rlscan_debug_set_lookback",
+    "compute_gae", "compute_vtrace", "compute_retrace", "compute_lambda_returns",
+    "compute_discounted_returns", "compute_eligibility_traces", "compute_episodic_prefix_sum",
+]
+
+RLSCAN_OK = 0
+RLSCAN_ERR_INVALID_ARG = 1
+RLSCAN_ERR_UNSUPPORTED = 2
+RLSCAN_ERR_WORKSPACE = 3
+RLSCAN_ERR_CUDA = 4
+RLSCAN_ERR_TIMEOUT = 5
+RLSCAN_F32 = 0
+RLSCAN_I32 = 1
+
+_STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
+
+
+class RlscanError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"rlscan error {_STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def _load_library():
+    path = _build.LIB
+    if not os.path.exists(path):
+        raise ImportError(
+            f"librlscan.so is not built ({path}); build it with "
+            "`python -c 'import __graft_entry__ as g; g.build()'` or "
+            "`python linear_recurrence_scans_02_b200/_build.py`")
+    lib = ctypes.CDLL(path)
+    P, I64, F, SZ, S, INT = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
+                             ctypes.c_void_p, ctypes.c_int)
+    sigs = {
+        "rlscan_gae": [P] * 7 + [I64, I64, F, F, P, SZ, S],
+        "rlscan_vtrace": [P] * 9 + [I64, I64, F, F, F, F, P, SZ, S],
+        "rlscan_retrace": [P] * 8 + [I64, I64, I64, F, F, F, P, SZ, S],
+        "rlscan_lambda_returns": [P] * 7 + [I64, I64, F, F, P, SZ, S],
+        "rlscan_discounted_returns": [P] * 6 + [I64, I64, F, P, SZ, S],
+        "rlscan_eligibility_traces": [P] * 3 + [I64, I64, F, F, P, SZ, S],
+        "rlscan_episodic_prefix_sum": [P, INT, P, P, I64, I64, P, SZ, S],
+        "rlscan_workspace_init": [P, SZ, S],
+        "rlscan_check": [S],
+        "rlscan_version": [],
+        "rlscan_debug_set_lookback": [ctypes.c_uint32, I64],
+        "rlscan_plan": [I64, I64, I64, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int),
+                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int64)],
+    }
+    for name, argtypes in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = argtypes
+        fn.restype = ctypes.c_int
+    lib.rlscan_workspace_bytes.argtypes = [I64, I64]
+    lib.rlscan_workspace_bytes.restype = ctypes.c_size_t
+    lib.rlscan_last_error.argtypes = []
+    lib.rlscan_last_error.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load_library()
+
+
+def _raise_on(status: int):
+    if status != RLSCAN_OK:
+        raise RlscanError(status, _lib.rlscan_last_error().decode(errors="replace"))
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------
+
+def _ptr(t, name, shape=None, dtypes=(torch.float32,), device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must have dtype in {dtypes}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr() or None
+
+
+def _shape(t, name):
+    if not isinstance(t, torch.Tensor) or t.dim() != 2:
+        raise ValueError(f"{name} must be a [num_envs, seq_len] tensor")
+    return int(t.shape[0]), int(t.shape[1])
+
+
+def _stream_handle(device):
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+class _WorkspaceCache:
+    """One zero-filled workspace per (device, stream), grown on demand.
+
+    The library leaves a workspace zero-filled after every call, so a cached
+    buffer is reused as is by later calls on the same stream (which the
+    stream orders)."""
+
+    def __init__(self):
+        self._bufs = {}
+        self._lock = threading.Lock()
+
+    def get(self, device, stream, nbytes):
+        if nbytes == 0:
+            return None, 0
+        key = (device.index, stream)
+        with self._lock:
+            buf = self._bufs.get(key)
+            if buf is None or buf.numel() < nbytes:
+                size = max(nbytes, 0 if buf is None else 2 * buf.numel())
+                buf = torch.zeros(size, dtype=torch.uint8, device=device)
+                self._bufs[key] = buf
+        return buf.data_ptr(), buf.numel()
+
+
+_ws_cache = _WorkspaceCache()
+
+
+def _workspace(device, E, T, ws):
+    stream = _stream_handle(device)
+    if ws is not None:
+        return _ptr(ws, "ws", dtypes=(torch.uint8,), device=device), ws.numel(), stream
+    need = int(_lib.rlscan_workspace_bytes(E, T))
+    p, n = _ws_cache.get(device, stream, need)
+    return p, n, stream
+
+
+def rlscan_workspace_bytes(num_envs: int, seq_len: int) -> int:
+    return int(_lib.rlscan_workspace_bytes(int(num_envs), int(seq_len)))
+
+
+def rlscan_check(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel reported a timed-out wait."""
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    _raise_on(_lib.rlscan_check(s))
+
+
+def rlscan_plan(num_envs: int, seq_len: int, actions: int = 1) -> dict:
+    te, th, lb, nt = ctypes.c_int64(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int64()
+    _raise_on(_lib.rlscan_plan(num_envs, seq_len, actions, ctypes.byref(te), ctypes.byref(th),
+                               ctypes.byref(lb), ctypes.byref(nt)))
+    return {"tile_elems": te.value, "threads": th.value, "lookback": bool(lb.value), "num_tiles": nt.value}
+
+
+def rlscan_debug_set_lookback(spin_limit: int = 0, withhold_tile: int = -1) -> None:
+    _raise_on(_lib.rlscan_debug_set_lookback(int(spin_limit), int(withhold_tile)))
+
+
+# ---------------------------------------------------------------------------
+# rlscan_* : the C calls with tensors (outputs preallocated)
+# ---------------------------------------------------------------------------
+
+def rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages,
+               gamma, lambda_, ws=None):
+    E, T = _shape(rewards, "rewards")
+    dev = rewards.device
+    sh = (E, T)
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_gae(
+        _ptr(rewards, "rewards", sh, device=dev), _ptr(values, "values", sh, device=dev),
+        _ptr(terminateds, "terminateds", sh, device=dev), _ptr(truncateds, "truncateds", sh, device=dev),
+        _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
+        _ptr(last_values, "last_values", (E,), device=dev), _ptr(advantages, "advantages", sh, device=dev),
+        E, T, float(gamma), float(lambda_), wp, wn, s))
+
+
+def rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values,
+                  vs, pg_advantages, gamma, lambda_=1.0, rho_bar=1.0, c_bar=1.0, ws=None):
+    E, T = _shape(rewards, "rewards")
+    dev = rewards.device
+    sh = (E, T)
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_vtrace(
+        _ptr(log_rhos, "log_rhos", sh, device=dev), _ptr(rewards, "rewards", sh, device=dev),
+        _ptr(values, "values", sh, device=dev), _ptr(terminateds, "terminateds", sh, device=dev),
+        _ptr(truncateds, "truncateds", sh, device=dev),
+        _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
+        _ptr(last_values, "last_values", (E,), device=dev), _ptr(vs, "vs", sh, device=dev),
+        _ptr(pg_advantages, "pg_advantages", sh, device=dev),
+        E, T, float(gamma), float(lambda_), float(rho_bar), float(c_bar), wp, wn, s))
+
+
+def rlscan_retrace(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds,
+                   truncateds, q_ret, gamma, lambda_, c_bar=1.0, ws=None):
+    E, T = _shape(rewards, "rewards")
+    dev = rewards.device
+    sh = (E, T)
+    if next_q_values_all.dim() == 2:
+        A, sh3 = 1, sh
+    else:
+        A = int(next_q_values_all.shape[2])
+        sh3 = (E, T, A)
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_retrace(
+        _ptr(rewards, "rewards", sh, device=dev), _ptr(q_values, "q_values", sh, device=dev),
+        _ptr(next_q_values_all, "next_q_values_all", sh3, device=dev),
+        _ptr(next_target_probs, "next_target_probs", sh3, device=dev),
+        _ptr(log_rhos, "log_rhos", sh, device=dev), _ptr(terminateds, "terminateds", sh, device=dev),
+        _ptr(truncateds, "truncateds", sh, device=dev), _ptr(q_ret, "q_ret", sh, device=dev),
+        E, T, A, float(gamma), float(lambda_), float(c_bar), wp, wn, s))
+
+
+def rlscan_lambda_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, returns,
+                          gamma, lambda_, ws=None):
+    E, T = _shape(rewards, "rewards")
+    dev = rewards.device
+    sh = (E, T)
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_lambda_returns(
+        _ptr(rewards, "rewards", sh, device=dev), _ptr(values, "values", sh, device=dev),
+        _ptr(terminateds, "terminateds", sh, device=dev), _ptr(truncateds, "truncateds", sh, device=dev),
+        _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
+        _ptr(last_values, "last_values", (E,), device=dev), _ptr(returns, "returns", sh, device=dev),
+        E, T, float(gamma), float(lambda_), wp, wn, s))
+
+
+def rlscan_discounted_returns(rewards, terminateds, truncateds, bootstrap_values, last_values, returns,
+                              gamma, ws=None):
+    E, T = _shape(rewards, "rewards")
+    dev = rewards.device
+    sh = (E, T)
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_discounted_returns(
+        _ptr(rewards, "rewards", sh, device=dev), _ptr(terminateds, "terminateds", sh, device=dev),
+        _ptr(truncateds, "truncateds", sh, device=dev),
+        _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
+        _ptr(last_values, "last_values", (E,), device=dev), _ptr(returns, "returns", sh, device=dev),
+        E, T, float(gamma), wp, wn, s))
+
+
+def rlscan_eligibility_traces(x, dones, traces, gamma, lambda_, ws=None):
+    E, T = _shape(x, "x")
+    dev = x.device
+    sh = (E, T)
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_eligibility_traces(
+        _ptr(x, "x", sh, device=dev), _ptr(dones, "dones", sh, device=dev), _ptr(traces, "traces", sh, device=dev),
+        E, T, float(gamma), float(lambda_), wp, wn, s))
+
+
+def rlscan_episodic_prefix_sum(x, dones, out, ws=None):
+    E, T = _shape(x, "x")
+    dev = x.device
+    sh = (E, T)
+    if x.dtype not in (torch.float32, torch.int32):
+        raise TypeError("x must be float32 or int32")
+    if out.dtype != x.dtype:
+        raise TypeError("out must have the dtype of x")
+    dtype = RLSCAN_F32 if x.dtype == torch.float32 else RLSCAN_I32
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_episodic_prefix_sum(
+        _ptr(x, "x", sh, (torch.float32, torch.int32), device=dev), dtype, _ptr(dones, "dones", sh, device=dev),
+        _ptr(out, "out", sh, (torch.float32, torch.int32), device=dev), E, T, wp, wn, s))
+
+
+# ---------------------------------------------------------------------------
+# compute_* : allocate outputs, call the above (README "Kernels" names)
+# ---------------------------------------------------------------------------
+
+def compute_gae(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
+                bootstrap_values=None, last_values=None):
+    adv = torch.empty_like(rewards)
+    rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, gamma, lambda_)
+    return adv
+
+
+def compute_vtrace(log_rhos, rewards, values, terminateds, gamma=0.99, lambda_=1.0, rho_bar=1.0, c_bar=1.0, *,
+                   truncateds=None, bootstrap_values=None, last_values=None):
+    vs = torch.empty_like(rewards)
+    pg = torch.empty_like(rewards)
+    rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values, vs, pg,
+                  gamma, lambda_, rho_bar, c_bar)
+    return vs, pg
+
+
+def compute_retrace(rewards, q_values, next_q_values_all, log_rhos, terminateds, truncateds, gamma=0.99,
+                    lambda_=0.95, c_bar=1.0, *, next_target_probs=None):
+    q_ret = torch.empty_like(rewards)
+    rlscan_retrace(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds, truncateds,
+                   q_ret, gamma, lambda_, c_bar)
+    return q_ret
+
+
+def compute_lambda_returns(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
+                           bootstrap_values=None, last_values=None):
+    ret = torch.empty_like(rewards)
+    rlscan_lambda_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, ret, gamma,
+                          lambda_)
+    return ret
+
+
+def compute_discounted_returns(rewards, terminateds=None, gamma=0.99, *, truncateds=None, bootstrap_values=None,
+                               last_values=None):
+    ret = torch.empty_like(rewards)
+    rlscan_discounted_returns(rewards, terminateds, truncateds, bootstrap_values, last_values, ret, gamma)
+    return ret
+
+
+def compute_eligibility_traces(x, dones=None, gamma=0.99, lambda_=0.95):
+    out = torch.empty_like(x)
+    rlscan_eligibility_traces(x, dones, out, gamma, lambda_)
+    return out
+
+
+def compute_episodic_prefix_sum(x, dones=None):
+    out = torch.empty_like(x)
+    rlscan_episodic_prefix_sum(x, dones, out)
+    return out

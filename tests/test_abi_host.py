@@ -1,0 +1,171 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every
+entry point declared in include/rlscan.h, and rejects bad arguments on the
+host before any CUDA call (fake device addresses are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rlscan.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RLSCAN_API\s+[\w\s\*]+?\b(rlscan_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib(rlscan_lib_path):
+    # These tests hand the library fake device addresses that must be rejected
+    # on the host; they are meant for a machine without a GPU, so that a
+    # validation bug can never turn into a launch on real memory.
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("host-validation tests with fake pointers run only without a GPU")
+    except ImportError:
+        pass
+    L = ctypes.CDLL(rlscan_lib_path)
+    P, I64, F, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    L.rlscan_gae.argtypes = [P] * 7 + [I64, I64, F, F, P, SZ, P]
+    L.rlscan_vtrace.argtypes = [P] * 9 + [I64, I64, F, F, F, F, P, SZ, P]
+    L.rlscan_retrace.argtypes = [P] * 8 + [I64, I64, I64, F, F, F, P, SZ, P]
+    L.rlscan_lambda_returns.argtypes = [P] * 7 + [I64, I64, F, F, P, SZ, P]
+    L.rlscan_discounted_returns.argtypes = [P] * 6 + [I64, I64, F, P, SZ, P]
+    L.rlscan_eligibility_traces.argtypes = [P] * 3 + [I64, I64, F, F, P, SZ, P]
+    L.rlscan_episodic_prefix_sum.argtypes = [P, ctypes.c_int, P, P, I64, I64, P, SZ, P]
+    L.rlscan_workspace_bytes.argtypes = [I64, I64]
+    L.rlscan_workspace_bytes.restype = SZ
+    L.rlscan_last_error.restype = ctypes.c_char_p
+    L.rlscan_plan.argtypes = [I64, I64, I64, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_int),
+                              ctypes.POINTER(ctypes.c_int), ctypes.POINTER(I64)]
+    return L
+
+
+def test_header_declares_the_seven_estimators():
+    syms = declared_symbols()
+    for est in ("gae", "vtrace", "retrace", "lambda_returns", "discounted_returns", "eligibility_traces",
+                "episodic_prefix_sum"):
+        assert f"rlscan_{est}" in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 14
+    for s in syms:
+        assert hasattr(lib, s), f"{s} declared in rlscan.h but not exported"
+
+
+def test_version(lib):
+    assert lib.rlscan_version() == 100
+
+
+# fake, never-dereferenced device addresses, far apart
+A, B, C, D, O1, O2 = (0x10000000 * k for k in range(1, 7))
+E, T = 4, 128
+
+
+def msg(lib):
+    return lib.rlscan_last_error().decode()
+
+
+def test_zero_sized_is_noop(lib):
+    assert lib.rlscan_gae(None, None, None, None, None, None, None, 0, 128, 0.99, 0.95, None, 0, None) == OK
+    assert lib.rlscan_gae(None, None, None, None, None, None, None, 8, 0, 0.99, 0.95, None, 0, None) == OK
+
+
+@pytest.mark.parametrize("E_,T_", [(-1, 4), (4, -1)])
+def test_negative_shape_rejected(lib, E_, T_):
+    assert lib.rlscan_gae(A, B, C, None, None, None, O1, E_, T_, 0.99, 0.95, None, 0, None) == INVALID
+
+
+def test_null_required_pointer_rejected(lib):
+    assert lib.rlscan_gae(None, B, C, None, None, None, O1, E, T, 0.99, 0.95, None, 0, None) == INVALID
+    assert "rewards" in msg(lib)
+    assert lib.rlscan_gae(A, B, C, None, None, None, None, E, T, 0.99, 0.95, None, 0, None) == INVALID
+
+
+def test_non_finite_parameters_rejected(lib):
+    assert lib.rlscan_gae(A, B, C, None, None, None, O1, E, T, float("nan"), 0.95, None, 0, None) == INVALID
+    assert lib.rlscan_vtrace(A, B, C, D, None, None, None, O1, O2, E, T, 0.99, 1.0, float("inf"), 1.0,
+                             None, 0, None) == INVALID
+
+
+def test_truncateds_need_bootstrap_values(lib):
+    assert lib.rlscan_gae(A, B, C, D, None, None, O1, E, T, 0.99, 0.95, None, 0, None) == INVALID
+    assert "bootstrap" in msg(lib)
+    assert lib.rlscan_discounted_returns(A, C, D, None, None, O1, E, T, 0.99, None, 0, None) == INVALID
+
+
+def test_output_overlapping_input_rejected(lib):
+    # advantages starts inside values
+    assert lib.rlscan_gae(A, B, C, None, None, None, B + 64, E, T, 0.99, 0.95, None, 0, None) == INVALID
+    assert "overlaps" in msg(lib)
+    # the two V-Trace outputs overlap each other
+    assert lib.rlscan_vtrace(A, B, C, D, None, None, None, O1, O1 + 4, E, T, 0.99, 1.0, 1.0, 1.0,
+                             None, 0, None) == INVALID
+
+
+def test_retrace_argument_rules(lib):
+    # truncateds is mandatory
+    assert lib.rlscan_retrace(A, B, C, None, D, O2, None, O1, E, T, 1, 0.99, 0.95, 1.0, None, 0, None) == INVALID
+    # probabilities required for A > 1
+    assert lib.rlscan_retrace(A, B, C, None, D, O2, O2 + 0x1000000, O1, E, T, 18, 0.99, 0.95, 1.0,
+                              None, 0, None) == INVALID
+    assert lib.rlscan_retrace(A, B, C, None, D, O2, O2 + 0x1000000, O1, E, T, 0, 0.99, 0.95, 1.0,
+                              None, 0, None) == INVALID
+    assert lib.rlscan_retrace(A, B, C, C, D, O2, O2 + 0x1000000, O1, E, T, 97, 0.99, 0.95, 1.0,
+                              None, 0, None) == UNSUPPORTED
+
+
+def test_prefix_sum_dtype_rejected(lib):
+    assert lib.rlscan_episodic_prefix_sum(A, 7, None, O1, E, T, None, 0, None) == UNSUPPORTED
+
+
+def plan(lib, E_, T_, A_=1):
+    te, th, lb, nt = ctypes.c_int64(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int64()
+    assert lib.rlscan_plan(E_, T_, A_, ctypes.byref(te), ctypes.byref(th), ctypes.byref(lb), ctypes.byref(nt)) == OK
+    return te.value, th.value, bool(lb.value), nt.value
+
+
+@pytest.mark.parametrize("E_,T_", [(4096, 128), (64, 512), (4096, 32), (1024, 2048), (65536, 4096), (256, 1024)])
+def test_plan_whole_rows_need_no_workspace(lib, E_, T_):
+    tile, threads, lookback, ntiles = plan(lib, E_, T_)
+    assert not lookback and tile % T_ == 0 and ntiles * tile >= E_ * T_
+    assert tile == threads * (4 if tile <= 1024 else 8)
+
+
+@pytest.mark.parametrize("E_,T_", [(16, 262144), (4096, 129), (3, 4097), (16, 4096)])
+def test_plan_split_rows_need_workspace(lib, E_, T_):
+    tile, threads, lookback, ntiles = plan(lib, E_, T_)
+    assert lookback
+    need = lib.rlscan_workspace_bytes(E_, T_)
+    assert need >= 128 + 16 * ntiles
+
+
+def test_missing_workspace_rejected(lib):
+    # 16 x 262144 splits rows over tiles: a workspace is required
+    assert lib.rlscan_gae(A, B, C, None, None, None, O1, 16, 262144, 0.99, 0.95, None, 0, None) == WORKSPACE
+    _, _, lookback, ntiles = plan(lib, 16, 262144)
+    need = 128 + 16 * ntiles  # what this call's plan needs
+    assert lookback and lib.rlscan_workspace_bytes(16, 262144) >= need
+    assert lib.rlscan_gae(A, B, C, None, None, None, O1, 16, 262144, 0.99, 0.95, D, need - 16, None) == WORKSPACE
+    assert lib.rlscan_gae(A, B, C, None, None, None, O1, 16, 262144, 0.99, 0.95, D + 4, need, None) == WORKSPACE
+
+
+def test_workspace_bytes_bounds(lib):
+    assert lib.rlscan_workspace_bytes(0, 10) == 0
+    assert lib.rlscan_workspace_bytes(-1, 10) == 0
+    # multi-action Retrace with 512-element tiles splits 4096-step rows
+    assert lib.rlscan_workspace_bytes(4096, 128) == 0
+    assert lib.rlscan_workspace_bytes(16, 262144) > 0
+
+
+def test_binding_imports_without_gpu():
+    import linear_recurrence_scans_02_b200 as pkg
+    assert callable(pkg.compute_gae) and callable(pkg.rlscan_gae)
+    assert os.path.exists(pkg.library_path())

@@ -1,0 +1,195 @@
+"""GPU parity: every estimator through the C ABI against the CPU oracle, on
+seeded inputs, element by element (tests/gpu_common.py gives the tolerance).
+
+Shapes span every tile plan the library picks: whole rows per tile (512 to
+4096-element tiles), rows split over tiles with the decoupled look-back,
+ragged tails (E*T not a multiple of the tile or of 4), single-step rows and
+rows shorter than a vector.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import (BACKWARD_KEYS, BACKWARD_RUN, check, dev, inputs_backward, run_gae, run_prefix,
+                        run_retrace, run_traces, run_vtrace, strip)
+from linear_recurrence_scans_02_b200 import rlscan as R
+from linear_recurrence_scans_02_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 1), (1, 2), (3, 3), (2, 5), (4, 31), (3, 33), (5, 127), (8, 128), (5, 129), (64, 512),
+          (300, 32), (2, 1000), (7, 2048), (16, 4096), (3, 4097), (1, 9000), (1100, 7)]
+
+
+@pytest.mark.parametrize("E,T", SHAPES, ids=lambda v: str(v))
+@pytest.mark.parametrize("est", sorted(BACKWARD_RUN))
+@pytest.mark.parametrize("variant", ["plain", "trunc", "trunc_lv"])
+def test_backward_estimators(est, E, T, variant):
+    d = inputs_backward(E, T, seed=E * 7919 + T, p_term=0.02,
+                        p_trunc=0.02 if variant != "plain" else 0.0, last_values=variant == "trunc_lv")
+    d = strip(d, BACKWARD_KEYS[est])
+    lam = 0.95 if est != "vtrace" else 1.0
+    check(BACKWARD_RUN[est](d, gamma=0.99, lam=lam), T, f"{est} {E}x{T} {variant}")
+
+
+@pytest.mark.parametrize("E,T", SHAPES, ids=lambda v: str(v))
+@pytest.mark.parametrize("variant", ["plain", "trunc"])
+def test_retrace_single_action(E, T, variant):
+    d = W.retrace_inputs(E, T, seed=E + 31 * T, p_term=0.02, p_trunc=0.02 if variant == "trunc" else 0.0)
+    check(run_retrace(d), T, f"retrace {E}x{T} {variant}")
+
+
+@pytest.mark.parametrize("E,T", SHAPES, ids=lambda v: str(v))
+def test_forward_estimators(E, T):
+    d = W.trace_inputs(E, T, seed=E * 13 + T, p_done=0.03)
+    check(run_traces(d), T, f"traces {E}x{T}")
+    check(run_prefix(d), T, f"prefix f32 {E}x{T}")
+    di = W.prefix_inputs_i32(E, T, seed=E * 17 + T, p_done=0.03)
+    check(run_prefix(di), T, f"prefix i32 {E}x{T}")
+
+
+@pytest.mark.parametrize("A", [2, 3, 18, 25, 49, 96])
+@pytest.mark.parametrize("E,T", [(3, 5), (4, 128), (5, 129), (2, 700), (8, 2048)], ids=lambda v: str(v))
+def test_retrace_multi_action(A, E, T):
+    d = W.off_policy_inputs(E, T, A=A, seed=A * 101 + T, p_term=0.01, p_trunc=0.01)
+    check(run_retrace(d), T, f"retrace A={A} {E}x{T}")
+
+
+@pytest.mark.parametrize("est", sorted(BACKWARD_RUN) + ["retrace", "traces", "prefix"])
+@pytest.mark.parametrize("flags", ["none", "all", "first", "last", "trunc_last"])
+def test_flag_edge_cases(est, flags):
+    E, T = 6, 257
+    d = inputs_backward(E, T, seed=3, p_term=0.0, p_trunc=0.0, last_values=True)
+    term = np.zeros((E, T), np.float32)
+    trunc = np.zeros((E, T), np.float32)
+    if flags == "all":
+        term[:] = 1
+    elif flags == "first":
+        term[:, 0] = 1
+    elif flags == "last":
+        term[:, -1] = 1
+    elif flags == "trunc_last":
+        trunc[:, -1] = 1
+        trunc[:, 100] = 1
+    d["terminateds"], d["truncateds"] = term, trunc
+    d["bootstrap_values"] = W.normal((E, T), 3, W.S_BOOT)
+    if est in BACKWARD_RUN:
+        lam = 1.0 if est == "vtrace" else 0.95
+        check(BACKWARD_RUN[est](strip(d, BACKWARD_KEYS[est]), gamma=0.99, lam=lam), T, f"{est} {flags}")
+    elif est == "retrace":
+        r = W.retrace_inputs(E, T, seed=3)
+        r["terminateds"], r["truncateds"] = term, trunc
+        check(run_retrace(r), T, f"retrace {flags}")
+    else:
+        x = {"x": d["rewards"], "dones": np.maximum(term, trunc)}
+        check(run_traces(x) if est == "traces" else run_prefix(x), T, f"{est} {flags}")
+
+
+@pytest.mark.parametrize("gamma,lam", [(0.0, 0.95), (1.0, 1.0), (0.99, 0.0), (0.99, 1.0), (0.5, 0.5)])
+def test_parameter_extremes(gamma, lam):
+    E, T = 9, 300
+    d = inputs_backward(E, T, seed=11, p_term=0.01, p_trunc=0.01, last_values=True)
+    for est in ("gae", "lambda_returns", "discounted_returns"):
+        check(BACKWARD_RUN[est](strip(d, BACKWARD_KEYS[est]), gamma=gamma, lam=lam), T, f"{est} g={gamma} l={lam}")
+    check(run_vtrace(strip(d, BACKWARD_KEYS["vtrace"]), gamma=gamma, lam=lam, rho_bar=1.0, c_bar=1.0), T,
+          f"vtrace g={gamma} l={lam}")
+    check(run_vtrace(strip(d, BACKWARD_KEYS["vtrace"]), gamma=gamma, lam=lam, rho_bar=0.7, c_bar=1.3), T,
+          f"vtrace clip g={gamma} l={lam}")
+    r = W.retrace_inputs(E, T, seed=12, p_term=0.01, p_trunc=0.01)
+    check(run_retrace(r, gamma=gamma, lam=lam, c_bar=0.8), T, f"retrace g={gamma} l={lam}")
+    x = W.trace_inputs(E, T, seed=13)
+    check(run_traces(x, gamma=gamma, lam=lam), T, f"traces g={gamma} l={lam}")
+
+
+@pytest.mark.parametrize("offset", [1, 2, 3])
+@pytest.mark.parametrize("E,T", [(64, 128), (5, 129), (4, 3000)], ids=lambda v: str(v))
+def test_unaligned_pointers(offset, E, T):
+    d = inputs_backward(E, T, seed=offset, p_term=0.02, p_trunc=0.02, last_values=True)
+    for est in sorted(BACKWARD_RUN):
+        lam = 1.0 if est == "vtrace" else 0.95
+        check(BACKWARD_RUN[est](strip(d, BACKWARD_KEYS[est]), gamma=0.99, lam=lam, offset=offset), T,
+              f"{est} offset={offset}")
+    check(run_retrace(W.retrace_inputs(E, T, seed=offset), offset=offset), T, f"retrace offset={offset}")
+    check(run_retrace(W.off_policy_inputs(E, T, A=5, seed=offset), offset=offset), T, f"retrace A5 offset={offset}")
+    x = W.trace_inputs(E, T, seed=offset)
+    check(run_traces(x, offset=offset), T, f"traces offset={offset}")
+    check(run_prefix(W.prefix_inputs_i32(E, T, seed=offset), offset=offset), T, f"prefix i32 offset={offset}")
+
+
+def test_prefix_sum_int32_wraps_exactly():
+    E, T = 5, 3000
+    x = np.full((E, T), 2 ** 31 - 5, dtype=np.int64)
+    x[1] = -(2 ** 31)
+    x[2, ::3] = 2 ** 30
+    x = x.astype(np.int32)
+    d = np.zeros((E, T), np.float32)
+    d[0, 1000] = 1.0
+    d[3, ::7] = 1.0
+    check(run_prefix({"x": x, "dones": d}), T, "prefix i32 wrap")
+    check(run_prefix({"x": x}), T, "prefix i32 wrap no dones")
+
+
+def test_nonfinite_input_stays_in_its_episode():
+    E, T = 4, 200
+    d = inputs_backward(E, T, seed=5, p_term=0.0)
+    d["terminateds"][:, 99] = 1.0
+    d["rewards"][:, 150] = np.inf  # second episode only
+    gpu, ref = run_gae(strip(d, BACKWARD_KEYS["gae"]))
+    torch.cuda.synchronize()
+    g = gpu["advantages"].cpu().numpy()
+    assert np.isfinite(g[:, :100]).all(), "an inf leaked across the episode boundary"
+    np.testing.assert_allclose(g[:, :100], ref["advantages"][:, :100], rtol=1e-4, atol=1e-4)
+
+
+def test_workspace_left_zero_and_reused():
+    E, T = 3, 70000  # rows split over tiles
+    plan = R.rlscan_plan(E, T)
+    assert plan["lookback"]
+    need = R.rlscan_workspace_bytes(E, T)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    d = strip(inputs_backward(E, T, seed=1, p_term=0.0005), BACKWARD_KEYS["gae"])
+    t = {k: dev(v) for k, v in d.items()}
+    outs = []
+    for _ in range(3):
+        out = torch.empty(E, T, device="cuda")
+        R.rlscan_gae(t["rewards"], t["values"], t["terminateds"], None, None, None, out, 0.99, 0.95, ws=ws)
+        torch.cuda.synchronize()
+        assert int(ws.count_nonzero()) == 0, "workspace not left zero-filled"
+        outs.append(out)
+    R.rlscan_check()
+    _, ref = run_gae(d)
+    for out in outs:
+        check(({"advantages": out}, ref), T, "gae with explicit workspace")
+
+
+def test_non_default_stream():
+    E, T = 16, 5000
+    d = strip(inputs_backward(E, T, seed=2), BACKWARD_KEYS["gae"])
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        pair = run_gae(d)
+    s.synchronize()
+    check(pair, T, "gae on a side stream")
+
+
+def test_lookback_wait_times_out_cleanly():
+    """A tile that never publishes makes its successors' bounded waits run
+    out: the call must finish, report RLSCAN_ERR_TIMEOUT, leave the workspace
+    zero-filled, and the next normal call must be correct."""
+    E, T = 2, 4096 * 4
+    assert R.rlscan_plan(E, T)["lookback"]
+    d = strip(inputs_backward(E, T, seed=9, p_term=0.0), BACKWARD_KEYS["discounted_returns"])
+    t = {k: dev(v) for k, v in d.items()}
+    out = torch.empty(E, T, device="cuda")
+    try:
+        R.rlscan_debug_set_lookback(spin_limit=2000, withhold_tile=0)
+        # tile 0 in scan order never publishes; rows split over tiles wait on it
+        R.rlscan_discounted_returns(t["rewards"], t["terminateds"], None, None, None, out, 0.99)
+        with pytest.raises(R.RlscanError) as ei:
+            R.rlscan_check()
+        assert ei.value.status == R.RLSCAN_ERR_TIMEOUT
+    finally:
+        R.rlscan_debug_set_lookback(0, -1)
+    R.rlscan_check()  # error word was cleared
+    check(run_gae(strip(inputs_backward(E, T, seed=10), BACKWARD_KEYS["gae"])), T, "gae after a timeout")
+    R.rlscan_check()
