@@ -1,0 +1,619 @@
+#!/usr/bin/env python
+"""Benchmark: the seven rlscan estimators at num_envs=4096, seq_len=128, fp32.
+
+One step = one pass of the whole hot path over one batch: GAE, V-Trace,
+Retrace (single action), TD(lambda) returns, discounted returns, eligibility
+traces, and the episodic prefix sum on fp32 and on int32 input, each on its
+own seeded synthetic [4096, 128] inputs (the rl-triton README's production
+regime, "Performance" section).  Reported:
+
+  value       env-steps/s of the whole job: N * E * T * K / (device time of K
+              steps, max over ranks), inputs resident in HBM;
+  per_estimator  env-steps/s and HBM GB/s per estimator, from back-to-back
+              launches of that estimator alone;
+  roofline    achieved / measured HBM copy bandwidth for the dominant kernel;
+  e2e         the same metric with host->device copies of every step's inputs
+              (pinned memory) and device->host copies of its outputs inside
+              the timed region;
+  cpu_baseline  the CPU oracle timed on this host on a bounded sample.
+
+Timing: CUDA events on the launching stream around CUDA-graph replays; every
+step reads a different buffer set, and the sets together are larger than 4x
+the L2 cache, so every launch streams from HBM.  `--impl reference` times the
+CPU oracle (the reference arm: there is no runnable reference code) on the
+same workload and metric.
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
+torch.distributed.run, one process per GPU, each on its own batch (weak
+scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+E_ENVS, T_STEPS = 4096, 128
+GAMMA, LAMBDA = 0.99, 0.95
+P_DONE = 0.005
+L2_BYTES = 126 * 1024 * 1024
+ROTATE_BYTES = 4 * L2_BYTES
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD = "all seven estimators fp32, num_envs=4096, seq_len=128"
+
+# estimator -> (input planes, output planes, bytes per env-step moved)
+ESTIMATORS = {
+    "gae": (["rewards", "values", "terminateds"], ["advantages"]),
+    "vtrace": (["log_rhos", "rewards", "values", "terminateds"], ["vs", "pg_advantages"]),
+    "retrace": (["rewards", "q_values", "next_q_values_all", "log_rhos", "terminateds", "truncateds"], ["q_ret"]),
+    "lambda_returns": (["rewards", "values", "terminateds"], ["returns"]),
+    "discounted_returns": (["rewards", "terminateds"], ["returns"]),
+    "eligibility_traces": (["x", "dones"], ["traces"]),
+    "prefix_sum_f32": (["x", "dones"], ["out"]),
+    "prefix_sum_i32": (["x", "dones"], ["out"]),
+}
+INT_PLANES = {("prefix_sum_i32", "x"), ("prefix_sum_i32", "out")}
+
+
+def bytes_per_env_step(est: str) -> int:
+    ins, outs = ESTIMATORS[est]
+    return 4 * (len(ins) + len(outs))
+
+
+STEP_BYTES_PER_ENV_STEP = sum(bytes_per_env_step(e) for e in ESTIMATORS)
+
+
+def host_inputs(seed: int = 0) -> dict:
+    """Seeded [4096, 128] inputs of every estimator (numpy, host)."""
+    from linear_recurrence_scans_02_b200 import workloads as W
+    E, T = E_ENVS, T_STEPS
+    g = W.gae_inputs(E, T, seed, p_term=P_DONE)
+    v = W.vtrace_inputs(E, T, seed + 1, p_term=P_DONE)
+    r = W.retrace_inputs(E, T, seed + 2, p_term=P_DONE)
+    lr = W.gae_inputs(E, T, seed + 3, p_term=P_DONE)
+    dr = W.gae_inputs(E, T, seed + 4, p_term=P_DONE)
+    et = W.trace_inputs(E, T, seed + 5, p_done=P_DONE)
+    pf = W.trace_inputs(E, T, seed + 6, p_done=P_DONE)
+    pi = W.prefix_inputs_i32(E, T, seed + 7, p_done=P_DONE)
+    return {"gae": g, "vtrace": v, "retrace": r, "lambda_returns": lr, "discounted_returns": dr,
+            "eligibility_traces": et, "prefix_sum_f32": pf, "prefix_sum_i32": pi}
+
+
+# ---------------------------------------------------------------------------
+# device buffer sets
+# ---------------------------------------------------------------------------
+
+class BufferSet:
+    """All planes of all estimators for one batch, carved out of one
+    contiguous device buffer: inputs first, then outputs, so one copy moves
+    a step's inputs and one copy its outputs."""
+
+    def __init__(self, torch, device, estimators, in_buf=None, out_buf=None):
+        plane = E_ENVS * T_STEPS
+        self.estimators = list(estimators)
+        self.in_names = [(e, p) for e in self.estimators for p in ESTIMATORS[e][0]]
+        self.out_names = [(e, p) for e in self.estimators for p in ESTIMATORS[e][1]]
+        self.in_buf = in_buf if in_buf is not None else torch.empty(len(self.in_names) * plane, dtype=torch.float32,
+                                                                    device=device)
+        self.out_buf = out_buf if out_buf is not None else torch.empty(len(self.out_names) * plane,
+                                                                       dtype=torch.float32, device=device)
+        self.t = {}
+        for i, key in enumerate(self.in_names):
+            self.t[key] = self._view(self.in_buf, i, key)
+        for i, key in enumerate(self.out_names):
+            self.t[key] = self._view(self.out_buf, i, key)
+
+    @staticmethod
+    def _view(buf, i, key):
+        import torch
+        plane = E_ENVS * T_STEPS
+        v = buf[i * plane:(i + 1) * plane].view(E_ENVS, T_STEPS)
+        return v.view(torch.int32) if key in INT_PLANES else v
+
+    def fill_from_host(self, host):
+        import torch
+        for (e, p) in self.in_names:
+            src = host[e][p]
+            self.t[(e, p)].copy_(torch.from_numpy(np.ascontiguousarray(src)))
+
+    def calls(self, R):
+        """One closure per estimator: the C-ABI call on this set."""
+        t = self.t
+        c = {}
+        if "gae" in self.estimators:
+            c["gae"] = lambda: R.rlscan_gae(t["gae", "rewards"], t["gae", "values"], t["gae", "terminateds"],
+                                            None, None, None, t["gae", "advantages"], GAMMA, LAMBDA)
+        if "vtrace" in self.estimators:
+            c["vtrace"] = lambda: R.rlscan_vtrace(
+                t["vtrace", "log_rhos"], t["vtrace", "rewards"], t["vtrace", "values"], t["vtrace", "terminateds"],
+                None, None, None, t["vtrace", "vs"], t["vtrace", "pg_advantages"], GAMMA, 1.0, 1.0, 1.0)
+        if "retrace" in self.estimators:
+            c["retrace"] = lambda: R.rlscan_retrace(
+                t["retrace", "rewards"], t["retrace", "q_values"], t["retrace", "next_q_values_all"], None,
+                t["retrace", "log_rhos"], t["retrace", "terminateds"], t["retrace", "truncateds"],
+                t["retrace", "q_ret"], GAMMA, LAMBDA, 1.0)
+        if "lambda_returns" in self.estimators:
+            c["lambda_returns"] = lambda: R.rlscan_lambda_returns(
+                t["lambda_returns", "rewards"], t["lambda_returns", "values"], t["lambda_returns", "terminateds"],
+                None, None, None, t["lambda_returns", "returns"], GAMMA, LAMBDA)
+        if "discounted_returns" in self.estimators:
+            c["discounted_returns"] = lambda: R.rlscan_discounted_returns(
+                t["discounted_returns", "rewards"], t["discounted_returns", "terminateds"], None, None, None,
+                t["discounted_returns", "returns"], GAMMA)
+        if "eligibility_traces" in self.estimators:
+            c["eligibility_traces"] = lambda: R.rlscan_eligibility_traces(
+                t["eligibility_traces", "x"], t["eligibility_traces", "dones"], t["eligibility_traces", "traces"],
+                GAMMA, LAMBDA)
+        if "prefix_sum_f32" in self.estimators:
+            c["prefix_sum_f32"] = lambda: R.rlscan_episodic_prefix_sum(
+                t["prefix_sum_f32", "x"], t["prefix_sum_f32", "dones"], t["prefix_sum_f32", "out"])
+        if "prefix_sum_i32" in self.estimators:
+            c["prefix_sum_i32"] = lambda: R.rlscan_episodic_prefix_sum(
+                t["prefix_sum_i32", "x"], t["prefix_sum_i32", "dones"], t["prefix_sum_i32", "out"])
+        return c
+
+
+# ---------------------------------------------------------------------------
+# clocks sampling
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, path: str | None = None):
+        self.gpu_index = gpu_index
+        self.gpu_id = str(gpu_index)
+        try:  # name the device by UUID: CUDA and nvidia-smi may number GPUs differently
+            import torch
+            uuid = str(torch.cuda.get_device_properties(gpu_index).uuid)
+            self.gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
+        self.proc = None
+        self.path = path or os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self) -> dict:
+        return summarize_clocks(self.path if self.proc is not None else None)
+
+
+def summarize_clocks(path) -> dict:
+    """Median SM clock under load, max clock, and the throttle reasons seen."""
+    if not path or not os.path.exists(path):
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+    rows = []
+    for line in open(path):
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                         "hw_slowdown": parts[5], "hw_thermal_slowdown": parts[6],
+                         "sw_thermal_slowdown": parts[7], "sw_power_cap": parts[8]})
+        except ValueError:
+            continue
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+    smax = max(r["max"] for r in rows)
+    loaded = [r for r in rows if r["power"] > 200.0] or rows
+    reasons = sorted({k for r in loaded for k in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                                   "sw_power_cap") if r[k].lower() == "active"})
+    return {"sm_mhz": float(np.median([r["sm"] for r in loaded])), "sm_max_mhz": smax, "reasons": reasons,
+            "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# ncu DRAM traffic (profiles/dram_traffic.md): valid only for the exact
+# kernel source it was captured from
+# ---------------------------------------------------------------------------
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_recurrence_scans_02_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(est: str):
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha()
+    for line in open(path):
+        m = re.match(r"\|\s*(\w+)\s*\|\s*([0-9]+)\s*\|\s*([0-9a-f]+)\s*\|", line)
+        if m and m.group(1) == est and m.group(3) == sha:
+            return int(m.group(2))
+    return None
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        v = float(json.load(open(path))["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_pass(host, rows: slice):
+    """All eight oracle calls on a block of rows (the oracle as it stands)."""
+    import oracle as O
+    g, v, r, lr, dr, et, pf, pi = (host[k] for k in ESTIMATORS)
+    s = lambda a: a[rows]
+    O.gae(s(g["rewards"]), s(g["values"]), s(g["terminateds"]), GAMMA, LAMBDA)
+    O.vtrace(s(v["log_rhos"]), s(v["rewards"]), s(v["values"]), s(v["terminateds"]), GAMMA, 1.0, 1.0, 1.0)
+    O.retrace(s(r["rewards"]), s(r["q_values"]), s(r["next_q_values_all"]), s(r["log_rhos"]), s(r["terminateds"]),
+              s(r["truncateds"]), GAMMA, LAMBDA, 1.0)
+    O.lambda_returns(s(lr["rewards"]), s(lr["values"]), s(lr["terminateds"]), GAMMA, LAMBDA)
+    O.discounted_returns(s(dr["rewards"]), s(dr["terminateds"]), GAMMA)
+    O.eligibility_traces(s(et["x"]), s(et["dones"]), GAMMA, LAMBDA)
+    O.episodic_prefix_sum(s(pf["x"]), s(pf["dones"]))
+    O.episodic_prefix_sum(s(pi["x"]), s(pi["dones"]))
+
+
+def time_oracle(host, rows_per_call: int, threads: int, min_seconds: float, max_calls: int | None = None):
+    """Run the oracle over `rows_per_call` rows split across `threads` host
+    threads (ctypes releases the GIL), repeatedly, until `min_seconds` have
+    passed.  Returns (env-steps/s, calls, seconds)."""
+    chunk = max(1, rows_per_call // threads)
+    blocks = [slice(i, min(i + chunk, rows_per_call)) for i in range(0, rows_per_call, chunk)]
+    calls, t0 = 0, time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as pool:
+        while True:
+            list(pool.map(lambda b: oracle_pass(host, b), blocks))
+            calls += 1
+            el = time.perf_counter() - t0
+            if el >= min_seconds or (max_calls is not None and calls >= max_calls):
+                break
+    return calls * rows_per_call * T_STEPS / el, calls, el
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier_sync(world):
+    import torch
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def capture(torch, fns, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for f in fns:
+            f()
+    return g
+
+
+def run_gpu(args):
+    import torch
+    from linear_recurrence_scans_02_b200 import rlscan as R
+
+    world, rank, local = dist_setup(args.gpus)
+    device = torch.device("cuda", local)
+    host = host_inputs(seed=1000 * rank)
+    per_set_bytes = STEP_BYTES_PER_ENV_STEP * E_ENVS * T_STEPS
+    n_sets = max(2, -(-ROTATE_BYTES // per_set_bytes))
+    sets = [BufferSet(torch, device, ESTIMATORS) for _ in range(n_sets)]
+    for s in sets:
+        s.fill_from_host(host)
+    torch.cuda.synchronize()
+    names = list(ESTIMATORS)
+    side = torch.cuda.Stream(device)
+
+    # eager warm-up of every call (also checks for errors outside capture)
+    for s in sets:
+        for f in s.calls(R).values():
+            f()
+    R.rlscan_check()
+
+    # one graph per step (one buffer set each), and one graph for a whole
+    # round over all sets, so K steps cost K // n_sets + K % n_sets replays
+    step_graphs = [capture(torch, list(s.calls(R).values()), side) for s in sets]
+    round_graph = capture(torch, [f for s in sets for f in s.calls(R).values()], side)
+    torch.cuda.synchronize()
+
+    def run_steps(k0, count):
+        k = k0
+        while count > 0:
+            if k % n_sets == 0 and count >= n_sets:
+                round_graph.replay()
+                k += n_sets
+                count -= n_sets
+            else:
+                step_graphs[k % n_sets].replay()
+                k += 1
+                count -= 1
+
+    clocks = ClockSampler(local)
+    with clocks:
+        stream = torch.cuda.current_stream(device)
+        run_steps(0, args.warmup)
+        barrier_sync(world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        run_steps(0, args.steps)
+        ev1.record(stream)
+        barrier_sync(world)
+        step_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+
+        # per-estimator: back-to-back launches of one estimator over buffer
+        # sets whose total exceeds 4x L2
+        per_est = {}
+        for est in names:
+            nbytes = bytes_per_env_step(est) * E_ENVS * T_STEPS
+            n_rot = max(2, -(-ROTATE_BYTES // nbytes))
+            est_sets = [sets[i % n_sets] for i in range(n_rot)] if n_rot <= n_sets else None
+            if est_sets is None:  # need more distinct buffers than the step sets hold
+                est_sets = sets + [BufferSet(torch, device, [est]) for _ in range(n_rot - n_sets)]
+                for s in est_sets[n_sets:]:
+                    s.fill_from_host(host)
+            fns = [s.calls(R)[est] for s in est_sets]
+            for f in fns:
+                f()
+            g = capture(torch, fns, side)
+            reps = max(3, -(-max(args.steps, 200) // len(fns)))
+            for _ in range(2):
+                g.replay()
+            barrier_sync(world)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            b.record(stream)
+            barrier_sync(world)
+            ms = max_over_ranks(a.elapsed_time(b), world)
+            launches = reps * len(fns)
+            us = 1000.0 * ms / launches
+            per_est[est] = {"us_per_launch": us, "bytes_per_launch": nbytes, "launches": launches,
+                            "env_steps_per_s": E_ENVS * T_STEPS / (us * 1e-6),
+                            "gb_per_s": nbytes / (us * 1e-6) / 1e9}
+            del g
+            extra = est_sets[n_sets:]
+            del est_sets, fns, extra
+        R.rlscan_check()
+
+        # e2e: every step copies its inputs host -> device from pinned memory,
+        # runs the eight calls and copies its outputs device -> host, on three
+        # streams (copy-in, compute, copy-out) ordered by events, so the copies
+        # of one step overlap the compute of its neighbours
+        pinned_in = [torch.empty(sets[0].in_buf.numel(), dtype=torch.float32, pin_memory=True) for _ in range(2)]
+        pinned_out = [torch.empty(sets[0].out_buf.numel(), dtype=torch.float32, pin_memory=True) for _ in range(2)]
+        for p in pinned_in:
+            p.copy_(sets[0].in_buf.cpu())
+        e2e_steps = max(3, min(args.steps, args.e2e_steps))
+        s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
+        ev_in = [torch.cuda.Event() for _ in range(n_sets)]
+        ev_comp = [torch.cuda.Event() for _ in range(n_sets)]
+        ev_out = [torch.cuda.Event() for _ in range(n_sets)]
+
+        def e2e_step(k):
+            i = k % n_sets
+            s_in.wait_event(ev_comp[i])           # set i's inputs no longer being read
+            with torch.cuda.stream(s_in):
+                sets[i].in_buf.copy_(pinned_in[k % 2], non_blocking=True)
+            ev_in[i].record(s_in)
+            s_comp.wait_event(ev_in[i])
+            s_comp.wait_event(ev_out[i])          # set i's outputs already copied out
+            with torch.cuda.stream(s_comp):
+                step_graphs[i].replay()
+            ev_comp[i].record(s_comp)
+            s_out.wait_event(ev_comp[i])
+            with torch.cuda.stream(s_out):
+                pinned_out[k % 2].copy_(sets[i].out_buf, non_blocking=True)
+            ev_out[i].record(s_out)
+
+        for k in range(args.warmup):
+            e2e_step(k)
+        barrier_sync(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s_in)
+        for k in range(e2e_steps):
+            e2e_step(args.warmup + k)
+        b.record(s_out)
+        barrier_sync(world)
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world)
+        R.rlscan_check()
+    clk = clocks.summary()
+
+    # CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        rows = min(E_ENVS, 512 * threads)
+        v, calls, el = time_oracle(host, rows, threads, min_seconds=args.cpu_seconds)
+        cpu = {"value": v, "unit": "env-steps/s", "cores": threads, "kind": "oracle",
+               "sample": f"{calls} passes of the fp64 oracle over {rows} of 4096 rows x 128 steps, all 8 "
+                         f"estimator calls, rows split over {threads} host threads, {el:.1f} s"}
+
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_hbm_peak()
+    dominant = max(per_est, key=lambda e: per_est[e]["us_per_launch"])
+    d = per_est[dominant]
+    for est, rec in per_est.items():
+        rec["frac_of_hbm_peak"] = rec["gb_per_s"] / peak
+    value = world * E_ENVS * T_STEPS * args.steps / (step_ms * 1e-3)
+    h2d = sets[0].in_buf.numel() * 4
+    d2h = sets[0].out_buf.numel() * 4
+    line = {
+        "metric": "env-steps/s and HBM GB/s (% of peak) per estimator at 4096x128 fp32",
+        "value": value, "unit": "env-steps/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (int32 for the integer prefix sum)", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "num_envs": E_ENVS, "seq_len": T_STEPS,
+                   "estimators": names, "gamma": GAMMA, "lambda": LAMBDA, "p_done": P_DONE,
+                   "bytes_per_env_step": STEP_BYTES_PER_ENV_STEP,
+                   "l2": f"inputs larger than L2: {n_sets} rotating buffer sets, "
+                         f"{n_sets * per_set_bytes / 2**20:.0f} MiB > 4x126 MB",
+                   "timing": "CUDA events around CUDA-graph replays (a graph holds a round of steps)",
+                   "parallelism": f"replicas x{world}, each rank its own batch"},
+        "hbm_gb_per_s_step": STEP_BYTES_PER_ENV_STEP * E_ENVS * T_STEPS * args.steps / (step_ms * 1e-3) / 1e9,
+        "per_estimator": per_est,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": d["gb_per_s"], "peak": peak,
+                     "unit": "GB/s", "frac": d["gb_per_s"] / peak,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6.65 TB/s",
+                     "traffic": recorded_traffic(dominant),
+                     "algorithmic_bytes": d["bytes_per_launch"]},
+        "e2e": {"value": world * E_ENVS * T_STEPS * e2e_steps / (e2e_ms * 1e-3), "unit": "env-steps/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "path": "per step: pinned host -> device copy of its inputs, the eight C-ABI calls, "
+                        "device -> pinned host copy of its outputs; copy-in / compute / copy-out "
+                        "on three streams"},
+        "gpu_launches": args.steps * len(names),
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle on a bounded sample of the workload."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    host = host_inputs(seed=0)
+    threads = os.cpu_count() or 1
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        time_oracle(host, rows, threads, min_seconds=0.0, max_calls=1)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time_oracle(host, rows, threads, min_seconds=0.0, max_calls=1)
+    el = time.perf_counter() - t0
+    value = args.steps * rows * T_STEPS / el
+    sample = f"each step: the fp64 oracle on {rows} of 4096 rows x 128 steps, all 8 estimator calls, " \
+             f"{threads} host threads"
+    line = {"metric": "env-steps/s and HBM GB/s (% of peak) per estimator at 4096x128 fp32", "value": value,
+            "unit": "env-steps/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "num_envs": E_ENVS, "seq_len": T_STEPS, "sample_rows": rows},
+            "cpu_baseline": {"value": value, "unit": "env-steps/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "env-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_profile_case(args):
+    """Small case for ncu: `n` eager launches of every estimator, one
+    [4096, 128] buffer set (about 70 MB on the device), synchronised after
+    each estimator.  Prints nothing to time."""
+    import torch
+    from linear_recurrence_scans_02_b200 import rlscan as R
+    torch.cuda.set_device(0)
+    bs = BufferSet(torch, torch.device("cuda", 0), ESTIMATORS)
+    bs.fill_from_host(host_inputs(seed=0))
+    calls = bs.calls(R)
+    for est in (args.profile_only.split(",") if args.profile_only else list(ESTIMATORS)):
+        for _ in range(args.profile_launches):
+            calls[est]()
+        torch.cuda.synchronize()
+    R.rlscan_check()
+    print(f"profile case done: {args.profile_launches} launches per estimator")
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["rlscan", "reference"], default="rlscan")
+    ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--profile-launches", type=int, default=0,
+                    help="run N eager launches of each estimator and exit (small case for ncu)")
+    ap.add_argument("--profile-only", default="", help="comma-separated estimators for --profile-launches")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.profile_launches > 0:
+        return run_profile_case(args)
+    try:
+        return run_gpu(args)
+    finally:
+        if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -31,22 +31,47 @@ __device__ __forceinline__ StepFlags step_flags(float te, float tr) {
     return f;
 }
 
-// Next element's value of a plane, seen by each thread's last element: the
-// next lane's first element, or (last lane of the warp) a direct load.
+// Halo elements.  Each thread's last element needs the next element of a
+// plane (backward estimators) or its first element the previous one (forward
+// estimators); inside a warp that value comes from the neighbouring lane by a
+// shuffle, and the warp's edge lane loads it directly.  The edge load is
+// issued before the plane's own loads (fetch_*), so it is in flight with them
+// instead of waiting behind the shuffle that needs the loaded data.
 template <int V>
-__device__ __forceinline__ float next_halo(const float *__restrict__ p, const float (&own)[V], long long i0,
-                                           long long n, int lane) {
-    float h = __shfl_down_sync(kFullMask, own[0], 1);
-    if (lane == 31) h = load_one(p, i0 + V, n);
-    return h;
+__device__ __forceinline__ float fetch_next(const float *__restrict__ p, long long i0, long long n, int lane) {
+    return lane == 31 ? load_one(p, i0 + V, n) : 0.0f;
 }
-// Previous element's value, seen by each thread's first element.
 template <int V>
-__device__ __forceinline__ float prev_halo(const float *__restrict__ p, const float (&own)[V], long long i0,
-                                           long long n, int lane) {
-    float h = __shfl_up_sync(kFullMask, own[V - 1], 1);
-    if (lane == 0) h = load_one(p, i0 - 1, n);
-    return h;
+__device__ __forceinline__ float next_halo(const float (&own)[V], float fetched, int lane) {
+    const float h = __shfl_down_sync(kFullMask, own[0], 1);
+    return lane == 31 ? fetched : h;
+}
+__device__ __forceinline__ float fetch_prev(const float *__restrict__ p, long long i0, long long n, int lane) {
+    return lane == 0 ? load_one(p, i0 - 1, n) : 0.0f;
+}
+template <int V>
+__device__ __forceinline__ float prev_halo(const float (&own)[V], float fetched, int lane) {
+    const float h = __shfl_up_sync(kFullMask, own[V - 1], 1);
+    return lane == 0 ? fetched : h;
+}
+
+// L2 prefetch of one tile of up to six input planes, one plane per thread
+// (threads 0..5), before the kernel waits for the previous grid.
+__device__ __forceinline__ void prefetch_planes(const Geometry &g, long long tile0, int S, const void *p0,
+                                                const void *p1 = nullptr, const void *p2 = nullptr,
+                                                const void *p3 = nullptr, const void *p4 = nullptr,
+                                                const void *p5 = nullptr) {
+    const long long left = g.n - tile0;
+    const long long cnt = left < S ? left : S;
+    switch (threadIdx.x) {
+    case 0: prefetch_l2(p0, tile0, cnt, 4); break;
+    case 1: prefetch_l2(p1, tile0, cnt, 4); break;
+    case 2: prefetch_l2(p2, tile0, cnt, 4); break;
+    case 3: prefetch_l2(p3, tile0, cnt, 4); break;
+    case 4: prefetch_l2(p4, tile0, cnt, 4); break;
+    case 5: prefetch_l2(p5, tile0, cnt, 4); break;
+    default: break;
+    }
 }
 
 __device__ __forceinline__ float row_last_value(const float *__restrict__ lv, long long row, long long rows) {
@@ -70,14 +95,18 @@ struct GaeEst {
         float r[V], v[V], te[V], tr[V], out[V];
         float v_next;
     };
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds);
+    }
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
         load_plane<V>(P.rewards, i0, g.n, S.r);
         load_plane<V>(P.values, i0, g.n, S.v);
         load_plane<V>(P.terminateds, i0, g.n, S.te);
         load_plane<V>(P.truncateds, i0, g.n, S.tr);
-        S.v_next = next_halo<V>(P.values, S.v, i0, g.n, lane);
+        S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
@@ -91,7 +120,7 @@ struct GaeEst {
                 const bool rowend = rp.t == g.seq_len - 1;
                 float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
                 if (rowend) nv = row_last_value(P.last_values, rp.row, g.rows);
-                const float boot = f.cont ? nv : (f.trn ? __ldg(P.bootstrap_values + i0 + k) : 0.0f);
+                const float boot = f.cont ? nv : (f.trn ? __ldcg(P.bootstrap_values + i0 + k) : 0.0f);
                 a[k] = (f.cont && !rowend) ? gl : 0.0f;
                 b[k] = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
             } else {
@@ -128,14 +157,18 @@ struct LambdaReturnsEst {
         float r[V], v[V], te[V], tr[V], out[V];
         float v_next;
     };
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds);
+    }
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
         load_plane<V>(P.rewards, i0, g.n, S.r);
         load_plane<V>(P.values, i0, g.n, S.v);
         load_plane<V>(P.terminateds, i0, g.n, S.te);
         load_plane<V>(P.truncateds, i0, g.n, S.tr);
-        S.v_next = next_halo<V>(P.values, S.v, i0, g.n, lane);
+        S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
@@ -160,7 +193,7 @@ struct LambdaReturnsEst {
                     }
                 } else {
                     a[k] = 0.0f;
-                    b[k] = f.trn ? fmaf(P.gamma, __ldg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
+                    b[k] = f.trn ? fmaf(P.gamma, __ldcg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
                 }
             } else {
                 a[k] = 1.0f;
@@ -195,6 +228,9 @@ struct ReturnsEst {
     struct State {
         float r[V], te[V], tr[V], out[V];
     };
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.rewards, P.terminateds, P.truncateds);
+    }
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int,
                                                 State<V> &S, unsigned char *) {
@@ -216,7 +252,7 @@ struct ReturnsEst {
                     b[k] = rowend ? fmaf(P.gamma, row_last_value(P.last_values, rp.row, g.rows), S.r[k]) : S.r[k];
                 } else {
                     a[k] = 0.0f;
-                    b[k] = f.trn ? fmaf(P.gamma, __ldg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
+                    b[k] = f.trn ? fmaf(P.gamma, __ldcg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
                 }
             } else {
                 a[k] = 1.0f;
@@ -256,15 +292,19 @@ struct VtraceEst {
         float v_next;
         unsigned chained; // bit k: pg bootstraps on vs_{t+1}
     };
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds);
+    }
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
         load_plane<V>(P.log_rhos, i0, g.n, S.lr);
         load_plane<V>(P.rewards, i0, g.n, S.r);
         load_plane<V>(P.values, i0, g.n, S.v);
         load_plane<V>(P.terminateds, i0, g.n, S.te);
         load_plane<V>(P.truncateds, i0, g.n, S.tr);
-        S.v_next = next_halo<V>(P.values, S.v, i0, g.n, lane);
+        S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
@@ -284,7 +324,7 @@ struct VtraceEst {
                     boot = rowend ? row_last_value(P.last_values, rp.row, g.rows)
                                   : ((k + 1 < V) ? S.v[k + 1] : S.v_next);
                 } else {
-                    boot = f.trn ? __ldg(P.bootstrap_values + i0 + k) : 0.0f;
+                    boot = f.trn ? __ldcg(P.bootstrap_values + i0 + k) : 0.0f;
                 }
                 a[k] = (f.cont && !rowend) ? P.gamma * c : 0.0f;
                 b[k] = rho * (fmaf(P.gamma, boot, S.r[k]) - S.v[k]);
@@ -338,6 +378,17 @@ struct RetraceEst {
         float lr_next;
     };
 
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.rewards, P.q_values, P.log_rhos, P.terminateds, P.truncateds,
+                        kMulti ? nullptr : P.next_q_values_all);
+        if constexpr (kMulti) {
+            const long long left = g.n - tile0;
+            const long long cnt = left < S ? left : S;
+            if (threadIdx.x == 6) prefetch_l2(P.next_q_values_all, tile0 * P.actions, cnt * P.actions, 4);
+            if (threadIdx.x == 7) prefetch_l2(P.next_target_probs, tile0 * P.actions, cnt * P.actions, 4);
+        }
+    }
+
     // Expected next-state value of each of this thread's elements.
     template <int NT, int V>
     static __device__ __forceinline__ void stage_expected_values(const Params &P, const Geometry &g, long long i0,
@@ -359,6 +410,9 @@ struct RetraceEst {
                           ((reinterpret_cast<uintptr_t>(gp) & 15u) == 0);
         if (bulk) {
             if (tid == 0) {
+                // the previous grid wrote these rows with ordinary stores; order
+                // them before the bulk copies, which read through the async proxy
+                asm volatile("fence.proxy.async;" ::: "memory");
                 mbar_init(bar, 1);
                 mbar_arrive_expect_tx(bar, 2u * bytes);
                 bulk_copy_g2s(sq, gq, bytes, bar);
@@ -371,8 +425,8 @@ struct RetraceEst {
         } else {
             const int total = nvalid * A;
             for (int idx = tid; idx < total; idx += NT) {
-                sq[idx] = __ldg(gq + idx);
-                sp[idx] = __ldg(gp + idx);
+                sq[idx] = __ldcg(gq + idx);
+                sp[idx] = __ldcg(gp + idx);
             }
             __syncthreads();
         }
@@ -400,12 +454,13 @@ struct RetraceEst {
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *smem) {
+        const float h_lr_next = fetch_next<V>(P.log_rhos, i0, g.n, lane);
         load_plane<V>(P.rewards, i0, g.n, S.r);
         load_plane<V>(P.q_values, i0, g.n, S.q);
         load_plane<V>(P.log_rhos, i0, g.n, S.lr);
         load_plane<V>(P.terminateds, i0, g.n, S.te);
         load_plane<V>(P.truncateds, i0, g.n, S.tr);
-        S.lr_next = next_halo<V>(P.log_rhos, S.lr, i0, g.n, lane);
+        S.lr_next = next_halo<V>(S.lr, h_lr_next, lane);
         if constexpr (kMulti) {
             stage_expected_values<NT, V>(P, g, i0, S, smem);
         } else {
@@ -466,12 +521,16 @@ struct ForwardF32Est {
         float x[V], d[V], out[V];
         float d_prev;
     };
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.x, P.dones);
+    }
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const float h_d_prev = fetch_prev(P.dones, i0, g.n, lane);
         load_plane<V>(P.x, i0, g.n, S.x);
         load_plane<V>(P.dones, i0, g.n, S.d);
-        S.d_prev = prev_halo<V>(P.dones, S.d, i0, g.n, lane);
+        S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
     }
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
@@ -518,12 +577,16 @@ struct PrefixI32Est {
         float d[V];
         float d_prev;
     };
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.x, P.dones);
+    }
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const float h_d_prev = fetch_prev(P.dones, i0, g.n, lane);
         load_plane<V>(P.x, i0, g.n, S.x);
         load_plane<V>(P.dones, i0, g.n, S.d);
-        S.d_prev = prev_halo<V>(P.dones, S.d, i0, g.n, lane);
+        S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
     }
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &, const Geometry &g, long long i0, State<V> &S,

@@ -63,7 +63,16 @@ struct Plan {
     Cfg cfg;
     bool lookback;
     long long ntiles;
+    int mode; // kModeBlock / kModeLookback / kModeWarp
 };
+
+// Scan mode of a plan: look-back when rows span tiles; warp-local when
+// every warp's 32*V elements hold whole rows; otherwise a block scan.
+Plan with_mode(Plan p, long long T) {
+    const long long warp_elems = 32ll * (kCfgTile[p.cfg] / kCfgThreads[p.cfg]);
+    p.mode = p.lookback ? kModeLookback : ((warp_elems % T == 0) ? kModeWarp : kModeBlock);
+    return p;
+}
 
 // Fill the GPU: with fewer tiles than this the plan prefers smaller tiles.
 constexpr long long kNumSMs = 148;
@@ -71,7 +80,7 @@ constexpr long long kMinTiles = 2 * kNumSMs;
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 
-Plan make_plan(long long E, long long T, long long actions) {
+Plan make_plan_tiles(long long E, long long T, long long actions) {
     const long long n = E * T;
     Plan p{};
     if (actions > 1) {
@@ -119,6 +128,8 @@ Plan make_plan(long long E, long long T, long long actions) {
     p.lookback = p.ntiles > 1;
     return p;
 }
+
+Plan make_plan(long long E, long long T, long long actions) { return with_mode(make_plan_tiles(E, T, actions), T); }
 
 size_t workspace_for(const Plan &p) {
     return p.lookback ? sizeof(WsHeader) + sizeof(TileSlot) * (size_t)p.ntiles : 0;
@@ -188,10 +199,10 @@ int require(const void *p, const char *name) {
 // ---------------------------------------------------------------------------
 // Launch
 // ---------------------------------------------------------------------------
-template <class Est, int NT, int V, bool LB>
+template <class Est, int NT, int V, int kMode>
 cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const Lookback &lb, size_t smem,
                        cudaStream_t stream) {
-    auto kern = tile_scan_kernel<Est, NT, V, LB>;
+    auto kern = tile_scan_kernel<Est, NT, V, kMode>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -210,12 +221,15 @@ cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const L
 }
 
 template <class Est, Cfg C>
-cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, const Lookback &lb, bool lookback,
+cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, const Lookback &lb, int mode,
                        size_t smem, cudaStream_t s) {
     constexpr int NT = kCfgThreads[C];
     constexpr int V = kCfgTile[C] / NT;
-    return lookback ? launch_one<Est, NT, V, true>(P, g, lb, smem, s)
-                    : launch_one<Est, NT, V, false>(P, g, lb, smem, s);
+    switch (mode) {
+    case kModeLookback: return launch_one<Est, NT, V, kModeLookback>(P, g, lb, smem, s);
+    case kModeWarp: return launch_one<Est, NT, V, kModeWarp>(P, g, lb, smem, s);
+    default: return launch_one<Est, NT, V, kModeBlock>(P, g, lb, smem, s);
+    }
 }
 
 template <class Est>
@@ -243,10 +257,10 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
     const size_t smem = actions > 1 ? multi_smem_bytes(plan.cfg, actions) : 0;
     cudaError_t e;
     switch (plan.cfg) {
-    case C512: e = launch_cfg<Est, C512>(P, g, lb, plan.lookback, smem, stream); break;
-    case C1024: e = launch_cfg<Est, C1024>(P, g, lb, plan.lookback, smem, stream); break;
-    case C2048: e = launch_cfg<Est, C2048>(P, g, lb, plan.lookback, smem, stream); break;
-    case C4096: e = launch_cfg<Est, C4096>(P, g, lb, plan.lookback, smem, stream); break;
+    case C512: e = launch_cfg<Est, C512>(P, g, lb, plan.mode, smem, stream); break;
+    case C1024: e = launch_cfg<Est, C1024>(P, g, lb, plan.mode, smem, stream); break;
+    case C2048: e = launch_cfg<Est, C2048>(P, g, lb, plan.mode, smem, stream); break;
+    case C4096: e = launch_cfg<Est, C4096>(P, g, lb, plan.mode, smem, stream); break;
     default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
     }
     if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
@@ -280,9 +294,9 @@ int run_multi(const char *name, const typename Est::Params &P, long long E, long
     const size_t smem = multi_smem_bytes(plan.cfg, actions);
     cudaError_t e;
     switch (plan.cfg) {
-    case R512: e = launch_cfg<Est, R512>(P, g, lb, plan.lookback, smem, stream); break;
-    case R256: e = launch_cfg<Est, R256>(P, g, lb, plan.lookback, smem, stream); break;
-    case R128: e = launch_cfg<Est, R128>(P, g, lb, plan.lookback, smem, stream); break;
+    case R512: e = launch_cfg<Est, R512>(P, g, lb, plan.mode, smem, stream); break;
+    case R256: e = launch_cfg<Est, R256>(P, g, lb, plan.mode, smem, stream); break;
+    case R128: e = launch_cfg<Est, R128>(P, g, lb, plan.mode, smem, stream); break;
     default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
     }
     if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));

@@ -103,6 +103,22 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
         : "memory");
 }
 
+// Hint: bring [p + first, p + first + count) elements of a plane into L2.  The
+// range is shrunk to 16-byte boundaries inside it, so nothing outside the
+// caller's buffer is touched.  A prefetch has no effect on memory ordering,
+// so it may be issued before griddep_wait(), while the previous grid on the
+// stream is still running.
+__device__ __forceinline__ void prefetch_l2(const void *p, long long first, long long count, int elem_bytes) {
+    if (p == nullptr || count <= 0) return;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p) + (uintptr_t)first * (uintptr_t)elem_bytes;
+    const uintptr_t lo = (a + 15u) & ~(uintptr_t)15u;
+    const uintptr_t hi = (a + (uintptr_t)count * (uintptr_t)elem_bytes) & ~(uintptr_t)15u;
+    if (hi <= lo) return;
+    const uintptr_t len = hi - lo;
+    if (len > 0xffff0u) return; // only tile-sized ranges are prefetched
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo), "r"((uint32_t)len) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Scan algebra.  A pair (a, b) is the map x -> a x + b.  combine(p1, p2)
 // replaces p1 with p1 o p2 (p2 applied first).  a == 0 cuts the chain: the
@@ -172,8 +188,8 @@ __device__ __forceinline__ void warp_exclusive_from_inclusive(AT ia, BT ib, int 
 // Workspace for the look-back: a header with the tile counter, and one
 // 16-byte slot per tile.  status: 0 = nothing yet, 1 = the tile's aggregate
 // (a, b) is published, 2 = its inclusive value x (the carry into the next
-// tile) is published.  The last CTA to finish zeroes every status and both
-// counters, so the workspace is left as it was found.
+// tile) is published.  The last CTA to finish zeroes every slot and both
+// counters, so the workspace is left zero-filled, as it was found.
 // ---------------------------------------------------------------------------
 
 struct WsHeader {
@@ -309,7 +325,8 @@ __device__ __forceinline__ void lookback_release(const Lookback &lb, long long n
     }
     __syncthreads();
     if (s_last) {
-        for (long long i = threadIdx.x; i < ntiles; i += NT) lb.slots[i].status = 0u;
+        for (long long i = threadIdx.x; i < ntiles; i += NT)
+            *reinterpret_cast<uint4 *>(lb.slots + i) = make_uint4(0u, 0u, 0u, 0u);
         if (threadIdx.x == 0) {
             lb.hdr->tile_counter = 0u;
             lb.hdr->done_counter = 0u;
@@ -323,6 +340,12 @@ __device__ __forceinline__ void lookback_release(const Lookback &lb, long long n
 // 128-bit path needs a 16-byte-aligned base and a full vector; otherwise each
 // element is loaded on its own.  Elements at or past n read as zero / are not
 // written.  A null plane reads as zeros.
+//
+// Loads are coherent and cached in L2 only (ld.global.cg), never through the
+// read-only path: with programmatic dependent launch this kernel starts while
+// the previous grid may still be writing these inputs, so they are not
+// read-only for the whole life of this kernel.  Every element is read once,
+// so L1 would not help anyway.
 // ---------------------------------------------------------------------------
 
 template <int V, class T>
@@ -339,16 +362,16 @@ __device__ __forceinline__ void load_plane(const T *__restrict__ p, long long i0
 #pragma unroll
         for (int k = 0; k < V; k += 4) {
             if constexpr (std::is_same<T, float>::value) {
-                float4 q = __ldg(reinterpret_cast<const float4 *>(p + i0 + k));
+                float4 q = __ldcg(reinterpret_cast<const float4 *>(p + i0 + k));
                 o[k] = q.x; o[k + 1] = q.y; o[k + 2] = q.z; o[k + 3] = q.w;
             } else {
-                int4 q = __ldg(reinterpret_cast<const int4 *>(p + i0 + k));
+                int4 q = __ldcg(reinterpret_cast<const int4 *>(p + i0 + k));
                 o[k] = q.x; o[k + 1] = q.y; o[k + 2] = q.z; o[k + 3] = q.w;
             }
         }
     } else {
 #pragma unroll
-        for (int k = 0; k < V; ++k) o[k] = (i0 + k < n && i0 + k >= 0) ? __ldg(p + i0 + k) : T(0);
+        for (int k = 0; k < V; ++k) o[k] = (i0 + k < n && i0 + k >= 0) ? __ldcg(p + i0 + k) : T(0);
     }
 }
 
@@ -374,7 +397,7 @@ __device__ __forceinline__ void store_plane(T *__restrict__ p, long long i0, lon
 // Scalar element of a plane (null -> 0), for halos and rare reads.
 template <class T>
 __device__ __forceinline__ T load_one(const T *__restrict__ p, long long i, long long n) {
-    return (p != nullptr && i >= 0 && i < n) ? __ldg(p + i) : T(0);
+    return (p != nullptr && i >= 0 && i < n) ? __ldcg(p + i) : T(0);
 }
 
 // ---------------------------------------------------------------------------
@@ -387,12 +410,22 @@ __device__ __forceinline__ T load_one(const T *__restrict__ p, long long i, long
 //   store<V>(P, g, i0, S)
 // ---------------------------------------------------------------------------
 
-template <class Est, int NT, int V, bool kLookback>
+// Scan modes of one launch:
+//   kModeBlock     tiles hold whole rows; warps exchange carries in shared memory
+//   kModeLookback  rows span tiles; tiles exchange carries through the workspace
+//   kModeWarp      every warp's 32*V elements hold whole rows: no block scan at all
+constexpr int kModeBlock = 0;
+constexpr int kModeLookback = 1;
+constexpr int kModeWarp = 2;
+
+template <class Est, int NT, int V, int kMode>
 __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Params P, const Geometry g,
                                                        const Lookback lb) {
     using AT = typename Est::AT;
     using BT = typename Est::BT;
     constexpr bool kBwd = Est::kBackward;
+    constexpr bool kLookback = kMode == kModeLookback;
+    constexpr bool kWarpLocal = kMode == kModeWarp;
     constexpr int NW = NT / 32;
     static_assert(NT % 32 == 0 && NW <= 32, "block must be whole warps, at most 32");
 
@@ -402,12 +435,23 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
     __shared__ long long s_tile;
     extern __shared__ __align__(128) unsigned char dyn_smem[];
 
-    griddep_wait();
-    griddep_launch_dependents();
-
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
+
+    // Start this tile's DRAM reads before waiting for the previous grid on
+    // the stream: the L2 prefetch overlaps them with that grid's tail.  With
+    // the look-back the tile index is only known after the wait; blockIdx.x
+    // is the likely one (a wrong guess only costs a wasted prefetch).  Once
+    // the wait returns, let the next grid launch (it waits for this one to
+    // complete before touching memory).
+    {
+        const long long jg = blockIdx.x;
+        const long long mg = kBwd ? (g.ntiles - 1 - jg) : jg;
+        Est::prefetch(P, g, mg * (long long)(NT * V), NT * V);
+    }
+    griddep_wait();
+    griddep_launch_dependents();
 
     long long j; // tile index in scan order
     if constexpr (kLookback) {
@@ -465,41 +509,48 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
     AT ea;
     BT eb;
     warp_exclusive_from_inclusive<kBwd>(ia, ib, lane, ea, eb);
-    if (lane == (kBwd ? 0 : 31)) {
-        s_wa[warp] = ia;
-        s_wb[warp] = ib;
-    }
-    __syncthreads();
-
-    if (warp == 0) {
-        AT wa = lane < NW ? s_wa[lane] : identity_a(ta);
-        BT wb = lane < NW ? s_wb[lane] : identity_b(tb);
-        warp_inclusive_scan<kBwd>(wa, wb, lane);
-        AT wea;
-        BT web;
-        warp_exclusive_from_inclusive<kBwd>(wa, wb, lane, wea, web);
-        BT carry = identity_b(tb);
-        if constexpr (kLookback) {
-            const AT tile_a = __shfl_sync(kFullMask, wa, kBwd ? 0 : NW - 1);
-            const BT tile_b = __shfl_sync(kFullMask, wb, kBwd ? 0 : NW - 1);
-            if (lane == 0) {
-                bool needs_carry;
-                if (kBwd) {
-                    const long long end = tile0 + (long long)(NT * V);
-                    needs_carry = end < g.n && (end % g.seq_len) != 0;
-                } else {
-                    needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
-                }
-                carry = lookback_carry<AT, BT>(lb, j, needs_carry, tile_a, tile_b);
-            }
-            carry = __shfl_sync(kFullMask, carry, 0);
+    BT x;
+    if constexpr (kWarpLocal) {
+        // the warp's first element in scan order starts a row: nothing flows in
+        x = apply_pair(ea, eb, identity_b(tb));
+    } else {
+        // value flowing into this warp: block scan of warp aggregates, plus
+        // the carry from earlier tiles when rows span tiles
+        if (lane == (kBwd ? 0 : 31)) {
+            s_wa[warp] = ia;
+            s_wb[warp] = ib;
         }
-        if (lane < NW) s_wx[lane] = apply_pair(wea, web, carry);
+        __syncthreads();
+        if (warp == 0) {
+            AT wa = lane < NW ? s_wa[lane] : identity_a(ta);
+            BT wb = lane < NW ? s_wb[lane] : identity_b(tb);
+            warp_inclusive_scan<kBwd>(wa, wb, lane);
+            AT wea;
+            BT web;
+            warp_exclusive_from_inclusive<kBwd>(wa, wb, lane, wea, web);
+            BT carry = identity_b(tb);
+            if constexpr (kLookback) {
+                const AT tile_a = __shfl_sync(kFullMask, wa, kBwd ? 0 : NW - 1);
+                const BT tile_b = __shfl_sync(kFullMask, wb, kBwd ? 0 : NW - 1);
+                if (lane == 0) {
+                    bool needs_carry;
+                    if (kBwd) {
+                        const long long end = tile0 + (long long)(NT * V);
+                        needs_carry = end < g.n && (end % g.seq_len) != 0;
+                    } else {
+                        needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
+                    }
+                    carry = lookback_carry<AT, BT>(lb, j, needs_carry, tile_a, tile_b);
+                }
+                carry = __shfl_sync(kFullMask, carry, 0);
+            }
+            if (lane < NW) s_wx[lane] = apply_pair(wea, web, carry);
+        }
+        __syncthreads();
+        x = apply_pair(ea, eb, s_wx[warp]);
     }
-    __syncthreads();
 
     // sequential epilogue over this thread's elements in scan order
-    BT x = apply_pair(ea, eb, s_wx[warp]);
     if (kBwd) {
 #pragma unroll
         for (int k = V - 1; k >= 0; --k) {

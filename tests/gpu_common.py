@@ -44,12 +44,19 @@ def empty_like_dev(a, offset=0, dtype=None):
     return flat[offset:].view(shape)
 
 
-def assert_close(gpu, ref, tol, what=""):
+def assert_close(gpu, ref, tol, what="", row_scale=False):
+    """|gpu - ref| <= tol * (1 + |ref|) per element.  row_scale=True measures
+    against the largest |ref| of the element's row instead: an fp32 scan's
+    rounding error follows the size of its running values, so where those
+    grow large and then cancel, only a row-relative bound is attainable."""
     g = gpu.detach().double().cpu().numpy() if isinstance(gpu, torch.Tensor) else np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     assert g.shape == ref.shape, (g.shape, ref.shape)
     err = np.abs(g - ref)
-    bound = tol * (1.0 + np.abs(ref))
+    if row_scale:
+        bound = tol * (1.0 + np.max(np.abs(ref), axis=-1, keepdims=True))
+    else:
+        bound = tol * (1.0 + np.abs(ref))
     bad = ~(err <= bound)
     if bad.any():
         idx = np.unravel_index(np.argmax(np.where(bad, err / bound, 0)), ref.shape)
