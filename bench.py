@@ -241,10 +241,11 @@ def summarize_clocks(path) -> dict:
 # ---------------------------------------------------------------------------
 
 def kernel_source_sha() -> str:
+    """Hash of the device code (the kernel headers), not of the host file."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_recurrence_scans_02_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith(".cuh"):
             h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
 
