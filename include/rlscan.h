@@ -199,6 +199,36 @@ RLSCAN_API int rlscan_episodic_prefix_sum(const void *x, int dtype, const float 
                                cudaStream_t stream);
 
 /*
+ * GAE with a fixed scratch area instead of a caller-supplied workspace.
+ * No counterpart in the paper: the paper's kernels allocate their own
+ * temporaries.  For callers that cannot allocate device memory: code whose
+ * host application owns the whole device-memory budget and forbids
+ * allocations from plugins, and latency-bound loops that must not call
+ * cudaMalloc (which synchronises the device).  It computes exactly what
+ * rlscan_gae computes, with the same arguments minus ws / ws_bytes.
+ *
+ * Scratch: one static device array of RLSCAN_NOALLOC_SCRATCH_BYTES bytes,
+ * held on every GPU that loads the library until the process exits.  The
+ * first call on a device looks up that array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  Every call clears the part of the array it uses with
+ * cudaMemsetAsync on `stream` and allocates nothing.
+ * Limit: shapes whose tile plan needs more scratch than the array holds
+ * (rows split over more than about 65,000 tiles) return RLSCAN_ERR_WORKSPACE
+ * with the sizes in rlscan_last_error().
+ * All calls on one device share that device's array, which keeps the last
+ * call's contents: two calls whose kernels may run at the same time on one
+ * device (for example on two streams with no ordering between them) race on
+ * it, so the caller must serialise them.  Calls on different devices use
+ * different copies.
+ */
+#define RLSCAN_NOALLOC_SCRATCH_BYTES (1u << 20)
+RLSCAN_API int rlscan_gae_noalloc(const float *rewards, const float *values, const float *terminateds,
+                                  const float *truncateds, const float *bootstrap_values,
+                                  const float *last_values, float *advantages, int64_t E, int64_t T,
+                                  float gamma, float lambda_, cudaStream_t stream);
+
+/*
  * Workspace size in bytes that any entry point above needs for an [E, T]
  * problem (any A); 0 if no call of that shape needs one.  Negative or
  * overflowing shapes return 0 and the compute call then rejects them.

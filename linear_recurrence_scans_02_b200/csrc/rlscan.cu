@@ -8,6 +8,7 @@
 // overlap the tail of whatever ran before it on that stream.
 #include <atomic>
 #include <cmath>
+#include <mutex>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -308,6 +309,40 @@ size_t plane_bytes(long long E, long long T) { return (size_t)(E * T) * sizeof(f
 } // namespace
 } // namespace rlscan
 
+// Fixed scratch of rlscan_gae_noalloc: the look-back workspace for callers
+// that cannot allocate one.  In host code this name is only a handle for
+// cudaGetSymbolAddress, never an address to pass to a kernel.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RLSCAN_NOALLOC_SCRATCH_BYTES];
+
+namespace rlscan {
+namespace {
+
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of this device's copy of the scratch array, looked up once
+// per device with that device current.
+int noalloc_scratch(void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(RLSCAN_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return fail(RLSCAN_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return RLSCAN_OK;
+}
+
+} // namespace
+} // namespace rlscan
+
 using namespace rlscan;
 
 extern "C" {
@@ -474,6 +509,41 @@ int rlscan_episodic_prefix_sum(const void *x, int dtype, const float *dones, voi
     }
     PrefixI32Est::Params P{static_cast<const int32_t *>(x), dones, static_cast<int32_t *>(out)};
     return run<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream);
+}
+
+int rlscan_gae_noalloc(const float *rewards, const float *values, const float *terminateds, const float *truncateds,
+                       const float *bootstrap_values, const float *last_values, float *advantages, int64_t E,
+                       int64_t T, float gamma, float lambda_, cudaStream_t stream) {
+    // the same host checks as rlscan_gae, so a rejected call enqueues nothing
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(values, "values"));
+    RLSCAN_TRY(require(advantages, "advantages"));
+    if (truncateds && !bootstrap_values) return fail(RLSCAN_ERR_INVALID_ARG, "truncateds given without bootstrap_values");
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{rewards, pb, "rewards"}, {values, pb, "values"}, {terminateds, pb, "terminateds"},
+                        {truncateds, pb, "truncateds"}, {bootstrap_values, pb, "bootstrap_values"},
+                        {last_values, (size_t)E * 4, "last_values"}};
+    const Span outs[] = {{advantages, pb, "advantages"}};
+    RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
+    const size_t need = workspace_for(make_plan(E, T, 1));
+    if (need > RLSCAN_NOALLOC_SCRATCH_BYTES)
+        return fail(RLSCAN_ERR_WORKSPACE,
+                    "rlscan_gae_noalloc: shape E=%lld T=%lld needs %zu bytes of scratch; the fixed scratch holds %u",
+                    (long long)E, (long long)T, need, (unsigned)RLSCAN_NOALLOC_SCRATCH_BYTES);
+    void *ws = nullptr;
+    if (need > 0) {
+        RLSCAN_TRY(noalloc_scratch(&ws));
+        // the array keeps the previous call's contents: the tile counters and
+        // flags this call uses must start at zero
+        cudaError_t e = cudaMemsetAsync(ws, 0, need, stream);
+        if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
+    }
+    return rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages, E, T, gamma,
+                      lambda_, ws, need, stream);
 }
 
 size_t rlscan_workspace_bytes(int64_t E, int64_t T) {

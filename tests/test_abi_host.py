@@ -38,6 +38,7 @@ def lib(rlscan_lib_path):
     L.rlscan_discounted_returns.argtypes = [P] * 6 + [I64, I64, F, P, SZ, P]
     L.rlscan_eligibility_traces.argtypes = [P] * 3 + [I64, I64, F, F, P, SZ, P]
     L.rlscan_episodic_prefix_sum.argtypes = [P, ctypes.c_int, P, P, I64, I64, P, SZ, P]
+    L.rlscan_gae_noalloc.argtypes = [P] * 7 + [I64, I64, F, F, P]
     L.rlscan_workspace_bytes.argtypes = [I64, I64]
     L.rlscan_workspace_bytes.restype = SZ
     L.rlscan_last_error.restype = ctypes.c_char_p
@@ -169,3 +170,13 @@ def test_binding_imports_without_gpu():
     import linear_recurrence_scans_02_b200 as pkg
     assert callable(pkg.compute_gae) and callable(pkg.rlscan_gae)
     assert os.path.exists(pkg.library_path())
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
+    # 1 x (2^27 + 1) steps split over ~65,600 tiles needs more than 1 MiB of scratch
+    T_big = (1 << 27) + 1
+    far = [(k + 1) << 32 for k in range(4)]  # 512 MiB planes, 4 GiB apart: no overlap
+    assert lib.rlscan_gae_noalloc(far[0], far[1], far[2], None, None, None, far[3], 1, T_big, 0.99, 0.95,
+                                  None) == WORKSPACE
+    assert "fixed scratch holds" in msg(lib)
+    assert lib.rlscan_gae_noalloc(None, B, C, None, None, None, O1, 4, 128, 0.99, 0.95, None) == INVALID
