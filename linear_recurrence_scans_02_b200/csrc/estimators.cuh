@@ -109,17 +109,17 @@ struct GaeEst {
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
     template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
-        RowPos rp = row_pos(i0, g.seq_len);
         const float gl = P.gamma * P.lambda_;
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if (i0 + k < g.n) {
+            if ((rm.valid >> k) & 1u) {
                 const StepFlags f = step_flags(S.te[k], S.tr[k]);
-                const bool rowend = rp.t == g.seq_len - 1;
+                const bool rowend = (rm.end >> k) & 1u;
                 float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
-                if (rowend) nv = row_last_value(P.last_values, rp.row, g.rows);
+                if (rowend) nv = row_last_value(P.last_values, row_of(rm, k), g.rows);
                 const float boot = f.cont ? nv : (f.trn ? __ldcg(P.bootstrap_values + i0 + k) : 0.0f);
                 a[k] = (f.cont && !rowend) ? gl : 0.0f;
                 b[k] = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
@@ -127,11 +127,10 @@ struct GaeEst {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
             }
-            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
         }
     }
     template <int V>
-    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
     template <int V>
@@ -171,19 +170,19 @@ struct LambdaReturnsEst {
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
     template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
-        RowPos rp = row_pos(i0, g.seq_len);
         const float gl = P.gamma * P.lambda_;
         const float one_minus_l = 1.0f - P.lambda_;
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if (i0 + k < g.n) {
+            if ((rm.valid >> k) & 1u) {
                 const StepFlags f = step_flags(S.te[k], S.tr[k]);
-                const bool rowend = rp.t == g.seq_len - 1;
+                const bool rowend = (rm.end >> k) & 1u;
                 if (f.cont) {
                     if (rowend) { // G_{t+1} = V_{t+1} = last value
-                        const float lv = row_last_value(P.last_values, rp.row, g.rows);
+                        const float lv = row_last_value(P.last_values, row_of(rm, k), g.rows);
                         a[k] = 0.0f;
                         b[k] = fmaf(P.gamma, fmaf(one_minus_l, lv, P.lambda_ * lv), S.r[k]);
                     } else {
@@ -199,11 +198,10 @@ struct LambdaReturnsEst {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
             }
-            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
         }
     }
     template <int V>
-    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
     template <int V>
@@ -239,17 +237,17 @@ struct ReturnsEst {
         load_plane<V>(P.truncateds, i0, g.n, S.tr);
     }
     template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
-        RowPos rp = row_pos(i0, g.seq_len);
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if (i0 + k < g.n) {
+            if ((rm.valid >> k) & 1u) {
                 const StepFlags f = step_flags(S.te[k], S.tr[k]);
-                const bool rowend = rp.t == g.seq_len - 1;
+                const bool rowend = (rm.end >> k) & 1u;
                 if (f.cont) {
                     a[k] = rowend ? 0.0f : P.gamma;
-                    b[k] = rowend ? fmaf(P.gamma, row_last_value(P.last_values, rp.row, g.rows), S.r[k]) : S.r[k];
+                    b[k] = rowend ? fmaf(P.gamma, row_last_value(P.last_values, row_of(rm, k), g.rows), S.r[k]) : S.r[k];
                 } else {
                     a[k] = 0.0f;
                     b[k] = f.trn ? fmaf(P.gamma, __ldcg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
@@ -258,11 +256,10 @@ struct ReturnsEst {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
             }
-            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
         }
     }
     template <int V>
-    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
     template <int V>
@@ -287,10 +284,10 @@ struct VtraceEst {
     template <int V>
     struct State {
         float lr[V], r[V], v[V], te[V], tr[V];
-        float rho[V], boot_pg[V]; // pg bootstrap base; vs_{t+1} adds D_{t+1} where chained
+        float rho[V];
         float vs[V], pg[V];
         float v_next;
-        unsigned chained; // bit k: pg bootstraps on vs_{t+1}
+        unsigned chained; // bit k: the trace goes on to t+1 inside the row
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds);
@@ -307,21 +304,21 @@ struct VtraceEst {
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
     template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
-        RowPos rp = row_pos(i0, g.seq_len);
         S.chained = 0u;
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if (i0 + k < g.n) {
+            if ((rm.valid >> k) & 1u) {
                 const StepFlags f = step_flags(S.te[k], S.tr[k]);
-                const bool rowend = rp.t == g.seq_len - 1;
+                const bool rowend = (rm.end >> k) & 1u;
                 const float ratio = expf(S.lr[k]);
                 const float rho = fminf(P.rho_bar, ratio);
                 const float c = P.lambda_ * fminf(P.c_bar, ratio);
                 float boot;
                 if (f.cont) {
-                    boot = rowend ? row_last_value(P.last_values, rp.row, g.rows)
+                    boot = rowend ? row_last_value(P.last_values, row_of(rm, k), g.rows)
                                   : ((k + 1 < V) ? S.v[k + 1] : S.v_next);
                 } else {
                     boot = f.trn ? __ldcg(P.bootstrap_values + i0 + k) : 0.0f;
@@ -329,23 +326,23 @@ struct VtraceEst {
                 a[k] = (f.cont && !rowend) ? P.gamma * c : 0.0f;
                 b[k] = rho * (fmaf(P.gamma, boot, S.r[k]) - S.v[k]);
                 S.rho[k] = rho;
-                S.boot_pg[k] = boot;
                 if (f.cont && !rowend) S.chained |= (1u << k);
             } else {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
                 S.rho[k] = 0.0f;
-                S.boot_pg[k] = 0.0f;
             }
-            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
         }
     }
+    // vs_t = V_t + D_t.  pg_t = rho_t (r_t + gamma boot'_t - V_t) differs from
+    // b_t = rho_t (r_t + gamma boot_t - V_t) only where the trace goes on,
+    // where boot'_t = vs_{t+1} = V_{t+1} + D_{t+1} and boot_t = V_{t+1}:
+    // there pg_t = b_t + rho_t gamma D_{t+1}; elsewhere pg_t = b_t.
     template <int V>
-    static __device__ __forceinline__ void out(const Params &P, State<V> &S, int k, float x, float x_next) {
+    static __device__ __forceinline__ void out(const Params &P, State<V> &S, int k, float x, float x_next,
+                                               float b_k) {
         S.vs[k] = S.v[k] + x;
-        // vs_{t+1} = V_{t+1} + D_{t+1}; boot_pg holds V_{t+1} where chained
-        const float boot = (S.chained >> k) & 1u ? S.boot_pg[k] + x_next : S.boot_pg[k];
-        S.pg[k] = S.rho[k] * (fmaf(P.gamma, boot, S.r[k]) - S.v[k]);
+        S.pg[k] = ((S.chained >> k) & 1u) ? fmaf(S.rho[k] * P.gamma, x_next, b_k) : b_k;
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
@@ -468,14 +465,14 @@ struct RetraceEst {
         }
     }
     template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
-        RowPos rp = row_pos(i0, g.seq_len);
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if (i0 + k < g.n) {
+            if ((rm.valid >> k) & 1u) {
                 const StepFlags f = step_flags(S.te[k], S.tr[k]);
-                const bool rowend = rp.t == g.seq_len - 1;
+                const bool rowend = (rm.end >> k) & 1u;
                 const float boot = f.term ? 0.0f : S.vnext[k];
                 b[k] = fmaf(P.gamma, boot, S.r[k]) - S.q[k];
                 if (f.cont && !rowend) {
@@ -488,11 +485,10 @@ struct RetraceEst {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
             }
-            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
         }
     }
     template <int V>
-    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = S.q[k] + x;
     }
     template <int V>
@@ -533,24 +529,23 @@ struct ForwardF32Est {
         S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
     }
     template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0, State<V> &S,
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
-        RowPos rp = row_pos(i0, g.seq_len);
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if (i0 + k < g.n) {
+            if ((rm.valid >> k) & 1u) {
                 const float dp = (k > 0) ? S.d[k - 1] : S.d_prev;
-                a[k] = (rp.t == 0 || dp != 0.0f) ? 0.0f : P.decay;
+                a[k] = (((rm.start >> k) & 1u) || dp != 0.0f) ? 0.0f : P.decay;
                 b[k] = S.x[k];
             } else {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
             }
-            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
         }
     }
     template <int V>
-    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float) {
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
     template <int V>
@@ -589,24 +584,23 @@ struct PrefixI32Est {
         S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
     }
     template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &, const Geometry &g, long long i0, State<V> &S,
+    static __device__ __forceinline__ void coeffs(const Params &, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S,
                                                   uint32_t (&a)[V], int32_t (&b)[V]) {
-        RowPos rp = row_pos(i0, g.seq_len);
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if (i0 + k < g.n) {
+            if ((rm.valid >> k) & 1u) {
                 const float dp = (k > 0) ? S.d[k - 1] : S.d_prev;
-                a[k] = (rp.t == 0 || dp != 0.0f) ? 0u : 1u;
+                a[k] = (((rm.start >> k) & 1u) || dp != 0.0f) ? 0u : 1u;
                 b[k] = S.x[k];
             } else {
                 a[k] = 1u;
                 b[k] = 0;
             }
-            if (++rp.t == g.seq_len) { rp.t = 0; ++rp.row; }
         }
     }
     template <int V>
-    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, int32_t x, int32_t) {
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, int32_t x, int32_t, int32_t) {
         S.out[k] = x;
     }
     template <int V>

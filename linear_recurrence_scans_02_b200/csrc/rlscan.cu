@@ -56,9 +56,12 @@ bool pdl_enabled() {
 // [E*T] array.  Tiles need the look-back only when a tile boundary can fall
 // inside a row (S not a multiple of T, more than one tile).
 // ---------------------------------------------------------------------------
+// Eight elements per thread keeps a grid's share of each SM small, so the
+// next launch on the stream can be resident (and prefetching) while this one
+// runs; the 512-element tile (four per thread) is for small problems.
 enum Cfg { C512 = 0, C1024, C2048, C4096, R512, R256, R128, kNumCfg };
 constexpr int kCfgTile[kNumCfg] = {512, 1024, 2048, 4096, 512, 256, 128};
-constexpr int kCfgThreads[kNumCfg] = {128, 256, 256, 512, 128, 64, 32};
+constexpr int kCfgThreads[kNumCfg] = {128, 128, 256, 512, 128, 64, 32};
 
 struct Plan {
     Cfg cfg;
@@ -80,6 +83,13 @@ constexpr long long kNumSMs = 148;
 constexpr long long kMinTiles = 2 * kNumSMs;
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+int pow2_shift(long long T) {
+    if (T <= 0 || (T & (T - 1)) != 0) return -1;
+    int s = 0;
+    while ((1ll << s) < T) ++s;
+    return s;
+}
 
 Plan make_plan_tiles(long long E, long long T, long long actions) {
     const long long n = E * T;
@@ -242,6 +252,7 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
     g.seq_len = T;
     g.ntiles = plan.ntiles;
     g.rows = E;
+    g.t_shift = pow2_shift(T);
     Lookback lb{};
     lb.withhold = -1;
     lb.spin_limit = g_spin_limit.load();
@@ -279,6 +290,7 @@ int run_multi(const char *name, const typename Est::Params &P, long long E, long
     g.seq_len = T;
     g.ntiles = plan.ntiles;
     g.rows = E;
+    g.t_shift = pow2_shift(T);
     Lookback lb{};
     lb.withhold = -1;
     lb.spin_limit = g_spin_limit.load();

@@ -220,26 +220,57 @@ struct Geometry {
     long long seq_len; // T
     long long ntiles;
     long long rows;    // E
+    int t_shift;       // log2(T) when T is a power of two, else -1
 };
 
-// Element (scan) position helpers: t index and row of the element at flat
-// index i, computed once per thread and then advanced element by element.
-struct RowPos {
-    long long t;
-    long long row;
+// Where a thread's V elements sit in their rows, as bit masks over k:
+// end bit k = element k is the last step of its row (t == T-1), start bit
+// k = element k is the first (t == 0), valid bit k = element k exists
+// (i0 + k < n); row0 = row of element 0.  When V divides T (the common
+// case) a thread's elements share one row, so only element V-1 can end a
+// row and only element 0 can start one: one division (a shift for powers of
+// two) per thread instead of per-element bookkeeping.
+struct RowMasks {
+    unsigned end, start, valid;
+    long long row0;
 };
-__device__ __forceinline__ RowPos row_pos(long long i, long long T) {
-    RowPos p;
-    if (i < 0) i = 0;
-    if ((unsigned long long)i <= 0xffffffffull && (unsigned long long)T <= 0xffffffffull) {
-        unsigned ui = (unsigned)i, ut = (unsigned)T;
-        p.row = ui / ut;
-        p.t = ui - (unsigned)p.row * ut;
+template <int V>
+__device__ __forceinline__ RowMasks row_masks(long long i0, const Geometry &g) {
+    RowMasks m;
+    const long long T = g.seq_len;
+    long long t0;
+    if (g.t_shift >= 0) {
+        m.row0 = i0 >> g.t_shift;
+        t0 = i0 & (T - 1);
+    } else if ((unsigned long long)i0 <= 0xffffffffull && (unsigned long long)T <= 0xffffffffull) {
+        const unsigned q = (unsigned)i0 / (unsigned)T;
+        m.row0 = q;
+        t0 = (unsigned)i0 - q * (unsigned)T;
     } else {
-        p.row = i / T;
-        p.t = i - p.row * T;
+        m.row0 = i0 / T;
+        t0 = i0 - m.row0 * T;
     }
-    return p;
+    const long long left = g.n - i0;
+    m.valid = left >= V ? ((1u << V) - 1u) : (left > 0 ? ((1u << left) - 1u) : 0u);
+    if (T % V == 0) {
+        m.end = (t0 + V == T) ? (1u << (V - 1)) : 0u;
+        m.start = (t0 == 0) ? 1u : 0u;
+    } else {
+        m.end = 0u;
+        m.start = 0u;
+        long long t = t0;
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (t == T - 1) m.end |= 1u << k;
+            if (t == 0) m.start |= 1u << k;
+            if (++t == T) t = 0;
+        }
+    }
+    return m;
+}
+// Row of element k (only needed where element k ends a row).
+__device__ __forceinline__ long long row_of(const RowMasks &m, int k) {
+    return m.row0 + __popc(m.end & ((1u << k) - 1u));
 }
 
 // Single-lane decoupled look-back.  Publishes this tile's aggregate (or its
@@ -404,9 +435,10 @@ __device__ __forceinline__ T load_one(const T *__restrict__ p, long long i, long
 // The tile kernel.  Est supplies (see estimators.cuh):
 //   kBackward, AT, BT, Params, State<V>,
 //   load<NT, V>(P, g, i0, lane, S, dyn_smem)    -- every thread, incl. past n
-//   coeffs<V>(P, g, i0, S, a, b)                -- (a, b) per element, identity past n
-//   out<V>(P, S, k, x, x_prev)                  -- record output k (x_prev = value
-//                                                  of the element before it in scan order)
+//   coeffs<V>(P, g, i0, rm, S, a, b)            -- (a, b) per element, identity past n
+//   out<V>(P, S, k, x, x_prev, b_k)             -- record output k (x_prev = value
+//                                                  of the element before it in scan order,
+//                                                  b_k = its scan coefficient b)
 //   store<V>(P, g, i0, S)
 // ---------------------------------------------------------------------------
 
@@ -474,7 +506,8 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
 
     AT a[V];
     BT b[V];
-    Est::template coeffs<V>(P, g, i0, S, a, b);
+    const RowMasks rm = row_masks<V>(i0, g);
+    Est::template coeffs<V>(P, g, i0, rm, S, a, b);
 
     // thread aggregate, composed in scan order
     AT ta;
@@ -556,14 +589,14 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
         for (int k = V - 1; k >= 0; --k) {
             const BT prev = x;
             x = apply_pair(a[k], b[k], x);
-            Est::template out<V>(P, S, k, x, prev);
+            Est::template out<V>(P, S, k, x, prev, b[k]);
         }
     } else {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
             const BT prev = x;
             x = apply_pair(a[k], b[k], x);
-            Est::template out<V>(P, S, k, x, prev);
+            Est::template out<V>(P, S, k, x, prev, b[k]);
         }
     }
     Est::template store<V>(P, g, i0, S);

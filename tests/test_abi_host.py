@@ -137,7 +137,7 @@ def plan(lib, E_, T_, A_=1):
 def test_plan_whole_rows_need_no_workspace(lib, E_, T_):
     tile, threads, lookback, ntiles = plan(lib, E_, T_)
     assert not lookback and tile % T_ == 0 and ntiles * tile >= E_ * T_
-    assert tile == threads * (4 if tile <= 1024 else 8)
+    assert tile == threads * (4 if tile == 512 else 8)
 
 
 @pytest.mark.parametrize("E_,T_", [(16, 262144), (4096, 129), (3, 4097), (16, 4096)])
