@@ -337,14 +337,25 @@ def barrier_sync(world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank passes its own device-timed value."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(world: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job env-steps/s: every rank processes its own E x T batch per step."""
+    return world * E_ENVS * T_STEPS * steps / (elapsed_ms * 1e-3)
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch (weak scaling over independent env rows)."""
+    return 1000 * rank
 
 
 def capture(torch, fns, stream):
@@ -361,7 +372,7 @@ def run_gpu(args):
 
     world, rank, local = dist_setup(args.gpus)
     device = torch.device("cuda", local)
-    host = host_inputs(seed=1000 * rank)
+    host = host_inputs(seed=rank_seed(rank))
     per_set_bytes = STEP_BYTES_PER_ENV_STEP * E_ENVS * T_STEPS
     n_sets = max(2, -(-ROTATE_BYTES // per_set_bytes))
     sets = [BufferSet(torch, device, ESTIMATORS) for _ in range(n_sets)]
@@ -503,7 +514,7 @@ def run_gpu(args):
     d = per_est[dominant]
     for est, rec in per_est.items():
         rec["frac_of_hbm_peak"] = rec["gb_per_s"] / peak
-    value = world * E_ENVS * T_STEPS * args.steps / (step_ms * 1e-3)
+    value = job_value(world, args.steps, step_ms)
     h2d = sets[0].in_buf.numel() * 4
     d2h = sets[0].out_buf.numel() * 4
     line = {
@@ -526,7 +537,7 @@ def run_gpu(args):
                      else "fallback 6.65 TB/s",
                      "traffic": recorded_traffic(dominant),
                      "algorithmic_bytes": d["bytes_per_launch"]},
-        "e2e": {"value": world * E_ENVS * T_STEPS * e2e_steps / (e2e_ms * 1e-3), "unit": "env-steps/s",
+        "e2e": {"value": job_value(world, e2e_steps, e2e_ms), "unit": "env-steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "path": "per step: pinned host -> device copy of its inputs, the eight C-ABI calls, "
                         "device -> pinned host copy of its outputs; copy-in / compute / copy-out "

@@ -141,3 +141,20 @@ def prefix_inputs_i32(E: int, T: int, seed: int = 0, p_done: float = 0.005,
                       lo: int = -100, hi: int = 100) -> dict:
     return {"x": int_uniform((E, T), lo, hi, seed, S_XI),
             "dones": bernoulli((E, T), p_done, seed, S_DONE)}
+
+
+def device_inputs(kind: str, E: int, T: int, seed: int, device, p_done: float):
+    """Large inputs drawn on the GPU with a seeded torch generator (for sizes
+    whose host generation would dominate a test): kind "gae" gives rewards,
+    values, terminateds; kind "trace" gives x, dones.  Rows are independent,
+    so a test can copy any subset of rows back for the oracle."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    normal = lambda: torch.randn((E, T), generator=g, device=device, dtype=torch.float32)
+    flags = lambda: (torch.rand((E, T), generator=g, device=device) < p_done).to(torch.float32)
+    if kind == "gae":
+        return {"rewards": normal(), "values": normal(), "terminateds": flags()}
+    if kind == "trace":
+        return {"x": normal(), "dones": flags()}
+    raise ValueError(kind)
