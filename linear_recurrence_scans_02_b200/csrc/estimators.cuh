@@ -23,10 +23,11 @@ namespace rlscan {
 struct StepFlags {
     bool term, trn, cont;
 };
+template <bool kTrunc = true>
 __device__ __forceinline__ StepFlags step_flags(float te, float tr) {
     StepFlags f;
     f.term = te != 0.0f;
-    f.trn = (tr != 0.0f) && !f.term;
+    f.trn = kTrunc && (tr != 0.0f) && !f.term;
     f.cont = !f.term && !f.trn;
     return f;
 }
@@ -101,22 +102,23 @@ struct GaeEst {
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const bool vec = g.vec_ok && i0 + V <= g.n;
         const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
-        load_plane<V>(P.rewards, i0, g.n, S.r);
-        load_plane<V>(P.values, i0, g.n, S.v);
-        load_plane<V>(P.terminateds, i0, g.n, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
+        load_plane<V>(P.values, i0, g.n, vec, S.v);
+        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kTrunc>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
         const float gl = P.gamma * P.lambda_;
 #pragma unroll
         for (int k = 0; k < V; ++k) {
             if ((rm.valid >> k) & 1u) {
-                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
                 const bool rowend = (rm.end >> k) & 1u;
                 float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
                 if (rowend) nv = row_last_value(P.last_values, row_of(rm, k), g.rows);
@@ -129,13 +131,23 @@ struct GaeEst {
             }
         }
     }
+    // one uniform branch per thread: without truncations the truncation
+    // logic is compiled out of the per-element loop
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
+        if (P.truncateds != nullptr)
+            coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
+        else
+            coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+    }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.advantages, i0, g.n, S.out);
+        store_plane<V>(P.advantages, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
     }
 };
 
@@ -162,15 +174,16 @@ struct LambdaReturnsEst {
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const bool vec = g.vec_ok && i0 + V <= g.n;
         const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
-        load_plane<V>(P.rewards, i0, g.n, S.r);
-        load_plane<V>(P.values, i0, g.n, S.v);
-        load_plane<V>(P.terminateds, i0, g.n, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
+        load_plane<V>(P.values, i0, g.n, vec, S.v);
+        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kTrunc>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
         const float gl = P.gamma * P.lambda_;
@@ -178,7 +191,7 @@ struct LambdaReturnsEst {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
             if ((rm.valid >> k) & 1u) {
-                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
                 const bool rowend = (rm.end >> k) & 1u;
                 if (f.cont) {
                     if (rowend) { // G_{t+1} = V_{t+1} = last value
@@ -200,13 +213,23 @@ struct LambdaReturnsEst {
             }
         }
     }
+    // one uniform branch per thread: without truncations the truncation
+    // logic is compiled out of the per-element loop
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
+        if (P.truncateds != nullptr)
+            coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
+        else
+            coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+    }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.returns, i0, g.n, S.out);
+        store_plane<V>(P.returns, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
     }
 };
 
@@ -232,18 +255,19 @@ struct ReturnsEst {
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int,
                                                 State<V> &S, unsigned char *) {
-        load_plane<V>(P.rewards, i0, g.n, S.r);
-        load_plane<V>(P.terminateds, i0, g.n, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        const bool vec = g.vec_ok && i0 + V <= g.n;
+        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
+        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kTrunc>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
             if ((rm.valid >> k) & 1u) {
-                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
                 const bool rowend = (rm.end >> k) & 1u;
                 if (f.cont) {
                     a[k] = rowend ? 0.0f : P.gamma;
@@ -258,13 +282,23 @@ struct ReturnsEst {
             }
         }
     }
+    // one uniform branch per thread: without truncations the truncation
+    // logic is compiled out of the per-element loop
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
+        if (P.truncateds != nullptr)
+            coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
+        else
+            coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+    }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.returns, i0, g.n, S.out);
+        store_plane<V>(P.returns, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
     }
 };
 
@@ -295,23 +329,24 @@ struct VtraceEst {
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const bool vec = g.vec_ok && i0 + V <= g.n;
         const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
-        load_plane<V>(P.log_rhos, i0, g.n, S.lr);
-        load_plane<V>(P.rewards, i0, g.n, S.r);
-        load_plane<V>(P.values, i0, g.n, S.v);
-        load_plane<V>(P.terminateds, i0, g.n, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        load_plane<V>(P.log_rhos, i0, g.n, vec, S.lr);
+        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
+        load_plane<V>(P.values, i0, g.n, vec, S.v);
+        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kTrunc>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
         S.chained = 0u;
 #pragma unroll
         for (int k = 0; k < V; ++k) {
             if ((rm.valid >> k) & 1u) {
-                const StepFlags f = step_flags(S.te[k], S.tr[k]);
+                const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
                 const bool rowend = (rm.end >> k) & 1u;
                 const float ratio = expf(S.lr[k]);
                 const float rho = fminf(P.rho_bar, ratio);
@@ -338,6 +373,16 @@ struct VtraceEst {
     // b_t = rho_t (r_t + gamma boot_t - V_t) only where the trace goes on,
     // where boot'_t = vs_{t+1} = V_{t+1} + D_{t+1} and boot_t = V_{t+1}:
     // there pg_t = b_t + rho_t gamma D_{t+1}; elsewhere pg_t = b_t.
+    // one uniform branch per thread: without truncations the truncation
+    // logic is compiled out of the per-element loop
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
+        if (P.truncateds != nullptr)
+            coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
+        else
+            coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+    }
     template <int V>
     static __device__ __forceinline__ void out(const Params &P, State<V> &S, int k, float x, float x_next,
                                                float b_k) {
@@ -346,8 +391,8 @@ struct VtraceEst {
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.vs, i0, g.n, S.vs);
-        store_plane<V>(P.pg_advantages, i0, g.n, S.pg);
+        store_plane<V>(P.vs, i0, g.n, g.vec_ok && i0 + V <= g.n, S.vs);
+        store_plane<V>(P.pg_advantages, i0, g.n, g.vec_ok && i0 + V <= g.n, S.pg);
     }
 };
 
@@ -451,17 +496,18 @@ struct RetraceEst {
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *smem) {
+        const bool vec = g.vec_ok && i0 + V <= g.n;
         const float h_lr_next = fetch_next<V>(P.log_rhos, i0, g.n, lane);
-        load_plane<V>(P.rewards, i0, g.n, S.r);
-        load_plane<V>(P.q_values, i0, g.n, S.q);
-        load_plane<V>(P.log_rhos, i0, g.n, S.lr);
-        load_plane<V>(P.terminateds, i0, g.n, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, S.tr);
+        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
+        load_plane<V>(P.q_values, i0, g.n, vec, S.q);
+        load_plane<V>(P.log_rhos, i0, g.n, vec, S.lr);
+        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
+        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
         S.lr_next = next_halo<V>(S.lr, h_lr_next, lane);
         if constexpr (kMulti) {
             stage_expected_values<NT, V>(P, g, i0, S, smem);
         } else {
-            load_plane<V>(P.next_q_values_all, i0, g.n, S.vnext);
+            load_plane<V>(P.next_q_values_all, i0, g.n, vec, S.vnext);
         }
     }
     template <int V>
@@ -493,7 +539,7 @@ struct RetraceEst {
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.q_ret, i0, g.n, S.out);
+        store_plane<V>(P.q_ret, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
     }
 };
 
@@ -523,9 +569,10 @@ struct ForwardF32Est {
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const bool vec = g.vec_ok && i0 + V <= g.n;
         const float h_d_prev = fetch_prev(P.dones, i0, g.n, lane);
-        load_plane<V>(P.x, i0, g.n, S.x);
-        load_plane<V>(P.dones, i0, g.n, S.d);
+        load_plane<V>(P.x, i0, g.n, vec, S.x);
+        load_plane<V>(P.dones, i0, g.n, vec, S.d);
         S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
     }
     template <int V>
@@ -550,7 +597,7 @@ struct ForwardF32Est {
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.out, i0, g.n, S.out);
+        store_plane<V>(P.out, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
     }
 };
 using TracesEst = ForwardF32Est<0>;
@@ -578,9 +625,10 @@ struct PrefixI32Est {
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
+        const bool vec = g.vec_ok && i0 + V <= g.n;
         const float h_d_prev = fetch_prev(P.dones, i0, g.n, lane);
-        load_plane<V>(P.x, i0, g.n, S.x);
-        load_plane<V>(P.dones, i0, g.n, S.d);
+        load_plane<V>(P.x, i0, g.n, vec, S.x);
+        load_plane<V>(P.dones, i0, g.n, vec, S.d);
         S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
     }
     template <int V>
@@ -605,7 +653,7 @@ struct PrefixI32Est {
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.out, i0, g.n, S.out);
+        store_plane<V>(P.out, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
     }
 };
 

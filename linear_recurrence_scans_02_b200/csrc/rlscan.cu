@@ -13,6 +13,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <initializer_list>
 #include <string>
 
 #include "../../include/rlscan.h"
@@ -58,7 +59,7 @@ bool pdl_enabled() {
 // ---------------------------------------------------------------------------
 // Eight elements per thread keeps a grid's share of each SM small, so the
 // next launch on the stream can be resident (and prefetching) while this one
-// runs; the 512-element tile (four per thread) is for small problems.
+// runs; the 512-element tile (four per thread) is for small look-back plans.
 enum Cfg { C512 = 0, C1024, C2048, C4096, R512, R256, R128, kNumCfg };
 constexpr int kCfgTile[kNumCfg] = {512, 1024, 2048, 4096, 512, 256, 128};
 constexpr int kCfgThreads[kNumCfg] = {128, 128, 256, 512, 128, 64, 32};
@@ -101,46 +102,49 @@ Plan make_plan_tiles(long long E, long long T, long long actions) {
         p.lookback = p.ntiles > 1 && (S % T) != 0;
         return p;
     }
-    const Cfg gen[4] = {C512, C1024, C2048, C4096};
-    // 1) tiles that hold whole rows: no look-back.  Largest such tile that
-    //    still fills the GPU, else the smallest one.
-    int aligned = -1;
-    for (int c = 3; c >= 0; --c) {
-        const long long S = kCfgTile[gen[c]];
-        if (S % T == 0 && ceil_div(n, S) >= kMinTiles) { aligned = c; break; }
-    }
-    if (aligned < 0) {
-        for (int c = 0; c < 4; ++c)
-            if (kCfgTile[gen[c]] % T == 0) { aligned = c; break; }
-    }
-    if (aligned >= 0) {
-        const long long nt = ceil_div(n, kCfgTile[gen[aligned]]);
-        const long long nt_small = ceil_div(n, kCfgTile[C512]);
-        // whole rows unless that leaves SMs idle and splitting rows would not
-        if (nt >= kNumSMs || nt_small <= nt) {
-            p.cfg = gen[aligned];
+    // Small CTAs (128 threads x 8 elements) overlap best, both with each
+    // other inside a launch and with the neighbouring launches; larger tiles
+    // only where a row needs them to stay inside one tile.
+    const Cfg whole_rows[3] = {C1024, C2048, C4096};
+    for (Cfg c : whole_rows) {
+        const long long S = kCfgTile[c];
+        if (S % T != 0) continue;
+        const long long nt = ceil_div(n, S);
+        const long long nt_split = ceil_div(n, kCfgTile[C1024]);
+        // whole rows, unless that leaves SMs idle while split rows would not
+        if (nt >= kNumSMs || nt_split <= nt) {
+            p.cfg = c;
             p.ntiles = nt;
             p.lookback = false;
             return p;
         }
-        // too few whole-row tiles: split rows over 512-element tiles instead
-        p.cfg = C512;
-        p.ntiles = nt_small;
-        p.lookback = true;
-        return p;
+        break;
     }
-    // 2) rows that do not align with any tile: look-back, largest tile that
-    //    still fills the GPU.
-    p.cfg = C512;
-    for (int c = 2; c >= 0; --c) {
-        if (ceil_div(n, kCfgTile[gen[c]]) >= kMinTiles) { p.cfg = gen[c]; break; }
-    }
+    // rows span tiles (long or odd-length rows, or too few rows to fill the
+    // GPU): 1024-element tiles with the look-back, 512 when that gives too few
+    p.cfg = ceil_div(n, kCfgTile[C1024]) >= kMinTiles ? C1024 : C512;
     p.ntiles = ceil_div(n, kCfgTile[p.cfg]);
-    p.lookback = p.ntiles > 1;
+    p.lookback = p.ntiles > 1 && (kCfgTile[p.cfg] % T != 0);
     return p;
 }
 
 Plan make_plan(long long E, long long T, long long actions) { return with_mode(make_plan_tiles(E, T, actions), T); }
+
+// Warp-local mode: a row spans T / V lanes (T a power of two dividing 32 V);
+// the shuffle scan needs to reach that far only.
+int scan_lanes_for(const Plan &p, long long T) {
+    if (p.mode != kModeWarp) return 32;
+    const long long V = kCfgTile[p.cfg] / kCfgThreads[p.cfg];
+    const long long lanes = T >= V ? T / V : 1;
+    return (int)(lanes < 32 ? lanes : 32);
+}
+
+// True when every given pointer is NULL or 16-byte aligned.
+bool aligned16(std::initializer_list<const void *> ptrs) {
+    for (const void *p : ptrs)
+        if (p != nullptr && ((uintptr_t)p & 15u) != 0) return false;
+    return true;
+}
 
 size_t workspace_for(const Plan &p) {
     return p.lookback ? sizeof(WsHeader) + sizeof(TileSlot) * (size_t)p.ntiles : 0;
@@ -245,7 +249,7 @@ cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, const L
 
 template <class Est>
 int run(const char *name, const typename Est::Params &P, long long E, long long T, long long actions, void *ws,
-        size_t ws_bytes, cudaStream_t stream) {
+        size_t ws_bytes, cudaStream_t stream, bool vec_ok) {
     const Plan plan = make_plan(E, T, actions);
     Geometry g;
     g.n = E * T;
@@ -253,6 +257,8 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
     g.ntiles = plan.ntiles;
     g.rows = E;
     g.t_shift = pow2_shift(T);
+    g.vec_ok = vec_ok ? 1 : 0;
+    g.scan_lanes = scan_lanes_for(plan, T);
     Lookback lb{};
     lb.withhold = -1;
     lb.spin_limit = g_spin_limit.load();
@@ -283,7 +289,7 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
 // configurations are never instantiated for it and vice versa.
 template <class Est>
 int run_multi(const char *name, const typename Est::Params &P, long long E, long long T, long long actions,
-              void *ws, size_t ws_bytes, cudaStream_t stream) {
+              void *ws, size_t ws_bytes, cudaStream_t stream, bool vec_ok) {
     const Plan plan = make_plan(E, T, actions);
     Geometry g;
     g.n = E * T;
@@ -291,6 +297,8 @@ int run_multi(const char *name, const typename Est::Params &P, long long E, long
     g.ntiles = plan.ntiles;
     g.rows = E;
     g.t_shift = pow2_shift(T);
+    g.vec_ok = vec_ok ? 1 : 0;
+    g.scan_lanes = scan_lanes_for(plan, T);
     Lookback lb{};
     lb.withhold = -1;
     lb.spin_limit = g_spin_limit.load();
@@ -378,7 +386,8 @@ int rlscan_gae(const float *rewards, const float *values, const float *terminate
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
     GaeEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                      last_values, advantages, gamma, lambda_};
-    return run<GaeEst>("rlscan_gae", P, E, T, 1, ws, ws_bytes, stream);
+    return run<GaeEst>("rlscan_gae", P, E, T, 1, ws, ws_bytes, stream,
+                       aligned16({rewards, values, terminateds, truncateds, advantages}));
 }
 
 int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
@@ -405,7 +414,8 @@ int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *valu
     RLSCAN_TRY(check_aliasing(ins, 7, outs, 2));
     VtraceEst::Params P{log_rhos, rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                         last_values, vs, pg_advantages, gamma, lambda_, rho_bar, c_bar};
-    return run<VtraceEst>("rlscan_vtrace", P, E, T, 1, ws, ws_bytes, stream);
+    return run<VtraceEst>("rlscan_vtrace", P, E, T, 1, ws, ws_bytes, stream,
+                          aligned16({log_rhos, rewards, values, terminateds, truncateds, vs, pg_advantages}));
 }
 
 int rlscan_retrace(const float *rewards, const float *q_values, const float *next_q_values_all,
@@ -439,11 +449,14 @@ int rlscan_retrace(const float *rewards, const float *q_values, const float *nex
     if (A == 1) {
         RetraceEst<false>::Params P{rewards, q_values, next_q_values_all, nullptr, log_rhos, terminateds,
                                     truncateds, q_ret, 1, gamma, lambda_, c_bar, 0u};
-        return run<RetraceEst<false>>("rlscan_retrace", P, E, T, 1, ws, ws_bytes, stream);
+        return run<RetraceEst<false>>("rlscan_retrace", P, E, T, 1, ws, ws_bytes, stream,
+                                      aligned16({rewards, q_values, next_q_values_all, log_rhos, terminateds,
+                                                 truncateds, q_ret}));
     }
     RetraceEst<true>::Params P{rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds,
                                truncateds, q_ret, A, gamma, lambda_, c_bar, 1u << 24};
-    return run_multi<RetraceEst<true>>("rlscan_retrace", P, E, T, A, ws, ws_bytes, stream);
+    return run_multi<RetraceEst<true>>("rlscan_retrace", P, E, T, A, ws, ws_bytes, stream,
+                                       aligned16({rewards, q_values, log_rhos, terminateds, truncateds, q_ret}));
 }
 
 int rlscan_lambda_returns(const float *rewards, const float *values, const float *terminateds,
@@ -466,7 +479,8 @@ int rlscan_lambda_returns(const float *rewards, const float *values, const float
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
     LambdaReturnsEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                                last_values, returns, gamma, lambda_};
-    return run<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, 1, ws, ws_bytes, stream);
+    return run<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, 1, ws, ws_bytes, stream,
+                                 aligned16({rewards, values, terminateds, truncateds, returns}));
 }
 
 int rlscan_discounted_returns(const float *rewards, const float *terminateds, const float *truncateds,
@@ -485,7 +499,8 @@ int rlscan_discounted_returns(const float *rewards, const float *terminateds, co
     RLSCAN_TRY(check_aliasing(ins, 5, outs, 1));
     ReturnsEst::Params P{rewards, terminateds, truncateds, truncateds ? bootstrap_values : nullptr, last_values,
                          returns, gamma};
-    return run<ReturnsEst>("rlscan_discounted_returns", P, E, T, 1, ws, ws_bytes, stream);
+    return run<ReturnsEst>("rlscan_discounted_returns", P, E, T, 1, ws, ws_bytes, stream,
+                           aligned16({rewards, terminateds, truncateds, returns}));
 }
 
 int rlscan_eligibility_traces(const float *x, const float *dones, float *traces, int64_t E, int64_t T, float gamma,
@@ -501,7 +516,8 @@ int rlscan_eligibility_traces(const float *x, const float *dones, float *traces,
     const Span outs[] = {{traces, pb, "traces"}};
     RLSCAN_TRY(check_aliasing(ins, 2, outs, 1));
     TracesEst::Params P{x, dones, traces, gamma * lambda_};
-    return run<TracesEst>("rlscan_eligibility_traces", P, E, T, 1, ws, ws_bytes, stream);
+    return run<TracesEst>("rlscan_eligibility_traces", P, E, T, 1, ws, ws_bytes, stream,
+                          aligned16({x, dones, traces}));
 }
 
 int rlscan_episodic_prefix_sum(const void *x, int dtype, const float *dones, void *out, int64_t E, int64_t T,
@@ -517,10 +533,12 @@ int rlscan_episodic_prefix_sum(const void *x, int dtype, const float *dones, voi
     RLSCAN_TRY(check_aliasing(ins, 2, outs, 1));
     if (dtype == RLSCAN_F32) {
         PrefixF32Est::Params P{static_cast<const float *>(x), dones, static_cast<float *>(out), 1.0f};
-        return run<PrefixF32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream);
+        return run<PrefixF32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream,
+                                 aligned16({x, dones, out}));
     }
     PrefixI32Est::Params P{static_cast<const int32_t *>(x), dones, static_cast<int32_t *>(out)};
-    return run<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream);
+    return run<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream,
+                             aligned16({x, dones, out}));
 }
 
 int rlscan_gae_noalloc(const float *rewards, const float *values, const float *terminateds, const float *truncateds,

@@ -152,11 +152,14 @@ __device__ __forceinline__ uint32_t from_bits(unsigned u, uint32_t) { return u; 
 __device__ __forceinline__ int32_t from_bits(unsigned u, int32_t) { return static_cast<int32_t>(u); }
 
 // Inclusive warp scan in scan order: forward = increasing lane, backward =
-// decreasing lane.
+// decreasing lane.  `width` (a power of two) bounds the distance a value
+// must travel: when rows start every `width` lanes, later steps would only
+// combine across a row boundary, where a = 0 already cuts the chain.
 template <bool kBackward, class AT, class BT>
-__device__ __forceinline__ void warp_inclusive_scan(AT &a, BT &b, int lane) {
+__device__ __forceinline__ void warp_inclusive_scan(AT &a, BT &b, int lane, int width = 32) {
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
+        if (d >= width) break;
         if (kBackward) {
             AT ao = __shfl_down_sync(kFullMask, a, d);
             BT bo = __shfl_down_sync(kFullMask, b, d);
@@ -221,6 +224,8 @@ struct Geometry {
     long long ntiles;
     long long rows;    // E
     int t_shift;       // log2(T) when T is a power of two, else -1
+    int vec_ok;        // every plane pointer of the call is 16-byte aligned
+    int scan_lanes;    // warp-local mode: lanes one row spans (a power of two <= 32)
 };
 
 // Where a thread's V elements sit in their rows, as bit masks over k:
@@ -379,8 +384,11 @@ __device__ __forceinline__ void lookback_release(const Lookback &lb, long long n
 // so L1 would not help anyway.
 // ---------------------------------------------------------------------------
 
+// `vec`: the caller's per-thread flag "all planes 16-byte aligned and this
+// thread's V elements all exist" (one test per thread, not per plane).
 template <int V, class T>
-__device__ __forceinline__ void load_plane(const T *__restrict__ p, long long i0, long long n, T (&o)[V]) {
+__device__ __forceinline__ void load_plane(const T *__restrict__ p, long long i0, long long n, bool vec,
+                                           T (&o)[V]) {
     static_assert(V % 4 == 0, "V must be a multiple of 4");
     static_assert(sizeof(T) == 4, "32-bit planes only");
     if (p == nullptr) {
@@ -388,7 +396,6 @@ __device__ __forceinline__ void load_plane(const T *__restrict__ p, long long i0
         for (int k = 0; k < V; ++k) o[k] = T(0);
         return;
     }
-    const bool vec = ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) && (i0 + V <= n);
     if (vec) {
 #pragma unroll
         for (int k = 0; k < V; k += 4) {
@@ -407,8 +414,8 @@ __device__ __forceinline__ void load_plane(const T *__restrict__ p, long long i0
 }
 
 template <int V, class T>
-__device__ __forceinline__ void store_plane(T *__restrict__ p, long long i0, long long n, const T (&o)[V]) {
-    const bool vec = ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) && (i0 + V <= n);
+__device__ __forceinline__ void store_plane(T *__restrict__ p, long long i0, long long n, bool vec,
+                                            const T (&o)[V]) {
     if (vec) {
 #pragma unroll
         for (int k = 0; k < V; k += 4) {
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
 
     AT ia = ta;
     BT ib = tb;
-    warp_inclusive_scan<kBwd>(ia, ib, lane);
+    warp_inclusive_scan<kBwd>(ia, ib, lane, kWarpLocal ? g.scan_lanes : 32);
     AT ea;
     BT eb;
     warp_exclusive_from_inclusive<kBwd>(ia, ib, lane, ea, eb);
