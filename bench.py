@@ -389,9 +389,37 @@ def run_gpu(args):
     R.rlscan_check()
 
     # one graph per step (one buffer set each), and one graph for a whole
-    # round over all sets, so K steps cost K // n_sets + K % n_sets replays
-    step_graphs = [capture(torch, list(s.calls(R).values()), side) for s in sets]
-    round_graph = capture(torch, [f for s in sets for f in s.calls(R).values()], side)
+    # round over all sets, so K steps cost K // n_sets + K % n_sets replays.
+    # The eight calls of a step are independent, so a step is captured as
+    # eight parallel branches (fork/join on events); --serial-steps chains
+    # them on one stream instead.
+    branches = [torch.cuda.Stream(device) for _ in names]
+
+    def step_fns(s, parallel):
+        fns = list(s.calls(R).values())
+        if not parallel:
+            return fns
+
+        def step():
+            cur = torch.cuda.current_stream(device)
+            fork = torch.cuda.Event()
+            fork.record(cur)
+            joins = []
+            for f, b in zip(fns, branches):
+                b.wait_stream(cur)
+                with torch.cuda.stream(b):
+                    f()
+                j = torch.cuda.Event()
+                j.record(b)
+                joins.append(j)
+            for j in joins:
+                cur.wait_event(j)
+        return [step]
+
+    parallel = not args.serial_steps
+    step_graphs = [capture(torch, step_fns(s, parallel), side) for s in sets]
+    round_graph = capture(torch, [f for s in sets for f in step_fns(s, parallel)], side)
+    serial_round = capture(torch, [f for s in sets for f in step_fns(s, False)], side)
     torch.cuda.synchronize()
 
     def run_steps(k0, count):
@@ -417,6 +445,19 @@ def run_gpu(args):
         ev1.record(stream)
         barrier_sync(world)
         step_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+
+        # the same steps as one chain on one stream, for reference
+        serial_reps = max(1, args.steps // n_sets)
+        for _ in range(2):
+            serial_round.replay()
+        barrier_sync(world)
+        sa, sb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sa.record(stream)
+        for _ in range(serial_reps):
+            serial_round.replay()
+        sb.record(stream)
+        barrier_sync(world)
+        serial_step_ms = max_over_ranks(sa.elapsed_time(sb), world) / (serial_reps * n_sets)
 
         # per-estimator: back-to-back launches of one estimator over buffer
         # sets whose total exceeds 4x L2
@@ -520,7 +561,8 @@ def run_gpu(args):
     line = {
         "metric": "env-steps/s and HBM GB/s (% of peak) per estimator at 4096x128 fp32",
         "value": value, "unit": "env-steps/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": step_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": step_ms / args.steps, "ms_per_step_serial_chain": serial_step_ms,
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 (int32 for the integer prefix sum)", "data": "synthetic",
         "config": {"workload": WORKLOAD, "num_envs": E_ENVS, "seq_len": T_STEPS,
                    "estimators": names, "gamma": GAMMA, "lambda": LAMBDA, "p_done": P_DONE,
@@ -528,6 +570,8 @@ def run_gpu(args):
                    "l2": f"inputs larger than L2: {n_sets} rotating buffer sets, "
                          f"{n_sets * per_set_bytes / 2**20:.0f} MiB > 4x126 MB",
                    "timing": "CUDA events around CUDA-graph replays (a graph holds a round of steps)",
+                   "step": ("the eight independent calls of a step as parallel graph branches"
+                            if parallel else "the eight calls of a step chained on one stream"),
                    "parallelism": f"replicas x{world}, each rank its own batch"},
         "hbm_gb_per_s_step": STEP_BYTES_PER_ENV_STEP * E_ENVS * T_STEPS * args.steps / (step_ms * 1e-3) / 1e9,
         "per_estimator": per_est,
@@ -607,6 +651,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["rlscan", "reference"], default="rlscan")
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--serial-steps", action="store_true",
+                    help="chain a step's eight calls on one stream instead of parallel graph branches")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--profile-launches", type=int, default=0,
