@@ -110,18 +110,18 @@ struct GaeEst {
         load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
-    template <int V, bool kTrunc>
+    template <int V, bool kTrunc, bool kFast>
     static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
         const float gl = P.gamma * P.lambda_;
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if ((rm.valid >> k) & 1u) {
+            if (elem_valid<kFast, V>(rm, k)) {
                 const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
-                const bool rowend = (rm.end >> k) & 1u;
+                const bool rowend = elem_row_end<kFast, V>(rm, k);
                 float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
-                if (rowend) nv = row_last_value(P.last_values, row_of(rm, k), g.rows);
+                if (rowend) nv = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
                 const float boot = f.cont ? nv : (f.trn ? __ldcg(P.bootstrap_values + i0 + k) : 0.0f);
                 a[k] = (f.cont && !rowend) ? gl : 0.0f;
                 b[k] = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
@@ -131,15 +131,19 @@ struct GaeEst {
             }
         }
     }
-    // one uniform branch per thread: without truncations the truncation
-    // logic is compiled out of the per-element loop
+    // uniform branches per thread: without truncations the truncation logic
+    // is compiled out of the per-element loop, and on the fast path (all V
+    // elements present, V divides T) so are the per-element row tests
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr)
-            coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
-        else
-            coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+        if (P.truncateds != nullptr) {
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, i0, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, i0, rm, S, a, b);
+        } else {
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, i0, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, i0, rm, S, a, b);
+        }
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
@@ -182,7 +186,7 @@ struct LambdaReturnsEst {
         load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
-    template <int V, bool kTrunc>
+    template <int V, bool kTrunc, bool kFast>
     static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
@@ -190,38 +194,44 @@ struct LambdaReturnsEst {
         const float one_minus_l = 1.0f - P.lambda_;
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if ((rm.valid >> k) & 1u) {
+            if (elem_valid<kFast, V>(rm, k)) {
                 const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
-                const bool rowend = (rm.end >> k) & 1u;
+                const bool rowend = elem_row_end<kFast, V>(rm, k);
+                // G_t = r_t + gamma * boot_t + (scan) gamma lambda G_{t+1}, with
+                // boot_t = (1 - lambda) V_{t+1} inside the row, the last value at a
+                // row end (G_{t+1} = V_{t+1} = last value), the bootstrap value at a
+                // truncation and 0 at a termination
+                float boot = 0.0f;
+                if (f.trn) boot = __ldcg(P.bootstrap_values + i0 + k);
                 if (f.cont) {
-                    if (rowend) { // G_{t+1} = V_{t+1} = last value
-                        const float lv = row_last_value(P.last_values, row_of(rm, k), g.rows);
-                        a[k] = 0.0f;
-                        b[k] = fmaf(P.gamma, fmaf(one_minus_l, lv, P.lambda_ * lv), S.r[k]);
+                    if (rowend) {
+                        const float lv = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
+                        boot = fmaf(one_minus_l, lv, P.lambda_ * lv);
                     } else {
-                        const float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
-                        a[k] = gl;
-                        b[k] = fmaf(P.gamma * one_minus_l, nv, S.r[k]);
+                        boot = one_minus_l * ((k + 1 < V) ? S.v[k + 1] : S.v_next);
                     }
-                } else {
-                    a[k] = 0.0f;
-                    b[k] = f.trn ? fmaf(P.gamma, __ldcg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
                 }
+                a[k] = (f.cont && !rowend) ? gl : 0.0f;
+                b[k] = fmaf(P.gamma, boot, S.r[k]);
             } else {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
             }
         }
     }
-    // one uniform branch per thread: without truncations the truncation
-    // logic is compiled out of the per-element loop
+    // uniform branches per thread: without truncations the truncation logic
+    // is compiled out of the per-element loop, and on the fast path (all V
+    // elements present, V divides T) so are the per-element row tests
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr)
-            coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
-        else
-            coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+        if (P.truncateds != nullptr) {
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, i0, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, i0, rm, S, a, b);
+        } else {
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, i0, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, i0, rm, S, a, b);
+        }
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
@@ -260,37 +270,42 @@ struct ReturnsEst {
         load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
         load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
     }
-    template <int V, bool kTrunc>
+    template <int V, bool kTrunc, bool kFast>
     static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if ((rm.valid >> k) & 1u) {
+            if (elem_valid<kFast, V>(rm, k)) {
                 const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
-                const bool rowend = (rm.end >> k) & 1u;
-                if (f.cont) {
-                    a[k] = rowend ? 0.0f : P.gamma;
-                    b[k] = rowend ? fmaf(P.gamma, row_last_value(P.last_values, row_of(rm, k), g.rows), S.r[k]) : S.r[k];
-                } else {
-                    a[k] = 0.0f;
-                    b[k] = f.trn ? fmaf(P.gamma, __ldcg(P.bootstrap_values + i0 + k), S.r[k]) : S.r[k];
-                }
+                const bool rowend = elem_row_end<kFast, V>(rm, k);
+                // what this step bootstraps from outside the scan: the row's
+                // last value at a row end, the bootstrap value at a
+                // truncation, nothing otherwise (the scan carries R_{t+1})
+                float boot = 0.0f;
+                if (f.trn) boot = __ldcg(P.bootstrap_values + i0 + k);
+                if (f.cont && rowend) boot = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
+                a[k] = (f.cont && !rowend) ? P.gamma : 0.0f;
+                b[k] = fmaf(P.gamma, boot, S.r[k]);
             } else {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
             }
         }
     }
-    // one uniform branch per thread: without truncations the truncation
-    // logic is compiled out of the per-element loop
+    // uniform branches per thread: without truncations the truncation logic
+    // is compiled out of the per-element loop, and on the fast path (all V
+    // elements present, V divides T) so are the per-element row tests
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr)
-            coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
-        else
-            coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+        if (P.truncateds != nullptr) {
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, i0, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, i0, rm, S, a, b);
+        } else {
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, i0, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, i0, rm, S, a, b);
+        }
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
@@ -338,22 +353,22 @@ struct VtraceEst {
         load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
-    template <int V, bool kTrunc>
+    template <int V, bool kTrunc, bool kFast>
     static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
         S.chained = 0u;
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if ((rm.valid >> k) & 1u) {
+            if (elem_valid<kFast, V>(rm, k)) {
                 const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
-                const bool rowend = (rm.end >> k) & 1u;
-                const float ratio = expf(S.lr[k]);
+                const bool rowend = elem_row_end<kFast, V>(rm, k);
+                const float ratio = __expf(S.lr[k]);
                 const float rho = fminf(P.rho_bar, ratio);
                 const float c = P.lambda_ * fminf(P.c_bar, ratio);
                 float boot;
                 if (f.cont) {
-                    boot = rowend ? row_last_value(P.last_values, row_of(rm, k), g.rows)
+                    boot = rowend ? row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows)
                                   : ((k + 1 < V) ? S.v[k + 1] : S.v_next);
                 } else {
                     boot = f.trn ? __ldcg(P.bootstrap_values + i0 + k) : 0.0f;
@@ -373,15 +388,19 @@ struct VtraceEst {
     // b_t = rho_t (r_t + gamma boot_t - V_t) only where the trace goes on,
     // where boot'_t = vs_{t+1} = V_{t+1} + D_{t+1} and boot_t = V_{t+1}:
     // there pg_t = b_t + rho_t gamma D_{t+1}; elsewhere pg_t = b_t.
-    // one uniform branch per thread: without truncations the truncation
-    // logic is compiled out of the per-element loop
+    // uniform branches per thread: without truncations the truncation logic
+    // is compiled out of the per-element loop, and on the fast path (all V
+    // elements present, V divides T) so are the per-element row tests
     template <int V>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr)
-            coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
-        else
-            coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+        if (P.truncateds != nullptr) {
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, i0, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, i0, rm, S, a, b);
+        } else {
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, i0, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, i0, rm, S, a, b);
+        }
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &P, State<V> &S, int k, float x, float x_next,
@@ -510,20 +529,20 @@ struct RetraceEst {
             load_plane<V>(P.next_q_values_all, i0, g.n, vec, S.vnext);
         }
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kFast>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if ((rm.valid >> k) & 1u) {
+            if (elem_valid<kFast, V>(rm, k)) {
                 const StepFlags f = step_flags(S.te[k], S.tr[k]);
-                const bool rowend = (rm.end >> k) & 1u;
+                const bool rowend = elem_row_end<kFast, V>(rm, k);
                 const float boot = f.term ? 0.0f : S.vnext[k];
                 b[k] = fmaf(P.gamma, boot, S.r[k]) - S.q[k];
                 if (f.cont && !rowend) {
                     const float lr1 = (k + 1 < V) ? S.lr[k + 1] : S.lr_next;
-                    a[k] = P.gamma * (P.lambda_ * fminf(P.c_bar, expf(lr1)));
+                    a[k] = P.gamma * (P.lambda_ * fminf(P.c_bar, __expf(lr1)));
                 } else {
                     a[k] = 0.0f;
                 }
@@ -532,6 +551,13 @@ struct RetraceEst {
                 b[k] = 0.0f;
             }
         }
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S, float (&a)[V],
+                                                  float (&b)[V]) {
+        if (rm.fast) coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
+        else coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
@@ -575,21 +601,28 @@ struct ForwardF32Est {
         load_plane<V>(P.dones, i0, g.n, vec, S.d);
         S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kFast>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if ((rm.valid >> k) & 1u) {
+            if (elem_valid<kFast, V>(rm, k)) {
                 const float dp = (k > 0) ? S.d[k - 1] : S.d_prev;
-                a[k] = (((rm.start >> k) & 1u) || dp != 0.0f) ? 0.0f : P.decay;
+                a[k] = (elem_row_start<kFast, V>(rm, k) || dp != 0.0f) ? 0.0f : P.decay;
                 b[k] = S.x[k];
             } else {
                 a[k] = 1.0f;
                 b[k] = 0.0f;
             }
         }
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S, float (&a)[V],
+                                                  float (&b)[V]) {
+        if (rm.fast) coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
+        else coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
@@ -631,21 +664,28 @@ struct PrefixI32Est {
         load_plane<V>(P.dones, i0, g.n, vec, S.d);
         S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &, const Geometry &g, long long i0,
+    template <int V, bool kFast>
+    static __device__ __forceinline__ void coeffs_impl(const Params &, const Geometry &g, long long i0,
                                                   const RowMasks &rm, State<V> &S,
                                                   uint32_t (&a)[V], int32_t (&b)[V]) {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            if ((rm.valid >> k) & 1u) {
+            if (elem_valid<kFast, V>(rm, k)) {
                 const float dp = (k > 0) ? S.d[k - 1] : S.d_prev;
-                a[k] = (((rm.start >> k) & 1u) || dp != 0.0f) ? 0u : 1u;
+                a[k] = (elem_row_start<kFast, V>(rm, k) || dp != 0.0f) ? 0u : 1u;
                 b[k] = S.x[k];
             } else {
                 a[k] = 1u;
                 b[k] = 0;
             }
         }
+    }
+    template <int V>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+                                                  const RowMasks &rm, State<V> &S, uint32_t (&a)[V],
+                                                  int32_t (&b)[V]) {
+        if (rm.fast) coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
+        else coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, int32_t x, int32_t, int32_t) {

@@ -238,6 +238,7 @@ struct Geometry {
 struct RowMasks {
     unsigned end, start, valid;
     long long row0;
+    bool fast; // all V elements exist and V divides T: only element V-1 can end a row, only 0 start one
 };
 template <int V>
 __device__ __forceinline__ RowMasks row_masks(long long i0, const Geometry &g) {
@@ -257,6 +258,7 @@ __device__ __forceinline__ RowMasks row_masks(long long i0, const Geometry &g) {
     }
     const long long left = g.n - i0;
     m.valid = left >= V ? ((1u << V) - 1u) : (left > 0 ? ((1u << left) - 1u) : 0u);
+    m.fast = (T % V == 0) && (left >= V);
     if (T % V == 0) {
         m.end = (t0 + V == T) ? (1u << (V - 1)) : 0u;
         m.start = (t0 == 0) ? 1u : 0u;
@@ -276,6 +278,25 @@ __device__ __forceinline__ RowMasks row_masks(long long i0, const Geometry &g) {
 // Row of element k (only needed where element k ends a row).
 __device__ __forceinline__ long long row_of(const RowMasks &m, int k) {
     return m.row0 + __popc(m.end & ((1u << k) - 1u));
+}
+
+// Per-element tests, folded at compile time on the fast path (k is a
+// constant once the element loop is unrolled).
+template <bool kFast, int V>
+__device__ __forceinline__ bool elem_valid(const RowMasks &m, int k) {
+    return kFast || ((m.valid >> k) & 1u);
+}
+template <bool kFast, int V>
+__device__ __forceinline__ bool elem_row_end(const RowMasks &m, int k) {
+    return kFast ? (k == V - 1 && ((m.end >> (V - 1)) & 1u)) : ((m.end >> k) & 1u);
+}
+template <bool kFast, int V>
+__device__ __forceinline__ bool elem_row_start(const RowMasks &m, int k) {
+    return kFast ? (k == 0 && (m.start & 1u)) : ((m.start >> k) & 1u);
+}
+template <bool kFast>
+__device__ __forceinline__ long long elem_row(const RowMasks &m, int k) {
+    return kFast ? m.row0 : row_of(m, k);
 }
 
 // Single-lane decoupled look-back.  Publishes this tile's aggregate (or its

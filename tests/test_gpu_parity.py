@@ -193,3 +193,28 @@ def test_lookback_wait_times_out_cleanly():
     R.rlscan_check()  # error word was cleared
     check(run_gae(strip(inputs_backward(E, T, seed=10), BACKWARD_KEYS["gae"])), T, "gae after a timeout")
     R.rlscan_check()
+
+
+@pytest.mark.parametrize("est", sorted(BACKWARD_RUN) + ["retrace"])
+def test_truncation_at_every_position_in_a_thread(est):
+    """A truncation (or termination) on each of the 16 first steps of a row,
+    one per row, with distinctive bootstrap values: catches a builder that
+    mishandles a flag at one position of a thread's 8 elements.  Rewards and
+    values are zero, so every output is made of bootstrap values alone."""
+    E, T = 32, 128
+    z = np.zeros((E, T), np.float32)
+    term, trunc = z.copy(), z.copy()
+    for e in range(16):
+        trunc[e, e] = 1.0
+        term[16 + e, e] = 1.0
+    bv = (100.0 + np.arange(E * T, dtype=np.float32)).reshape(E, T)
+    lv = (7.0 + np.arange(E, dtype=np.float32))
+    d = {"rewards": z.copy(), "values": z.copy(), "terminateds": term, "truncateds": trunc,
+         "bootstrap_values": bv, "last_values": lv, "log_rhos": z.copy()}
+    if est == "retrace":
+        r = {"rewards": z.copy(), "q_values": z.copy(), "next_q_values_all": bv.copy(), "log_rhos": z.copy(),
+             "terminateds": term, "truncateds": trunc}
+        check(run_retrace(r, gamma=0.5, lam=0.5), T, "retrace flag positions")
+        return
+    lam = 1.0 if est == "vtrace" else 0.5
+    check(BACKWARD_RUN[est](strip(d, BACKWARD_KEYS[est]), gamma=0.5, lam=lam), T, f"{est} flag positions")
