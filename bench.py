@@ -65,10 +65,16 @@ ESTIMATORS = {
     "prefix_sum_i32": (["x", "dones"], ["out"]),
 }
 INT_PLANES = {("prefix_sum_i32", "x"), ("prefix_sum_i32", "out")}
+# calls timed beside the step (not part of it): the fused GAE + TD(lambda)
+# pass that replaces the two separate calls
+EXTRA_CALLS = {
+    "gae_with_returns": (["rewards", "values", "terminateds"], ["advantages", "returns"]),
+}
+PLANES = {**ESTIMATORS, **EXTRA_CALLS}
 
 
 def bytes_per_env_step(est: str) -> int:
-    ins, outs = ESTIMATORS[est]
+    ins, outs = PLANES[est]
     return 4 * (len(ins) + len(outs))
 
 
@@ -87,8 +93,9 @@ def host_inputs(seed: int = 0) -> dict:
     et = W.trace_inputs(E, T, seed + 5, p_done=P_DONE)
     pf = W.trace_inputs(E, T, seed + 6, p_done=P_DONE)
     pi = W.prefix_inputs_i32(E, T, seed + 7, p_done=P_DONE)
+    gr = W.gae_inputs(E, T, seed + 8, p_term=P_DONE)
     return {"gae": g, "vtrace": v, "retrace": r, "lambda_returns": lr, "discounted_returns": dr,
-            "eligibility_traces": et, "prefix_sum_f32": pf, "prefix_sum_i32": pi}
+            "eligibility_traces": et, "prefix_sum_f32": pf, "prefix_sum_i32": pi, "gae_with_returns": gr}
 
 
 # ---------------------------------------------------------------------------
@@ -103,8 +110,8 @@ class BufferSet:
     def __init__(self, torch, device, estimators, in_buf=None, out_buf=None):
         plane = E_ENVS * T_STEPS
         self.estimators = list(estimators)
-        self.in_names = [(e, p) for e in self.estimators for p in ESTIMATORS[e][0]]
-        self.out_names = [(e, p) for e in self.estimators for p in ESTIMATORS[e][1]]
+        self.in_names = [(e, p) for e in self.estimators for p in PLANES[e][0]]
+        self.out_names = [(e, p) for e in self.estimators for p in PLANES[e][1]]
         self.in_buf = in_buf if in_buf is not None else torch.empty(len(self.in_names) * plane, dtype=torch.float32,
                                                                     device=device)
         self.out_buf = out_buf if out_buf is not None else torch.empty(len(self.out_names) * plane,
@@ -159,6 +166,11 @@ class BufferSet:
         if "prefix_sum_f32" in self.estimators:
             c["prefix_sum_f32"] = lambda: R.rlscan_episodic_prefix_sum(
                 t["prefix_sum_f32", "x"], t["prefix_sum_f32", "dones"], t["prefix_sum_f32", "out"])
+        if "gae_with_returns" in self.estimators:
+            c["gae_with_returns"] = lambda: R.rlscan_gae_with_returns(
+                t["gae_with_returns", "rewards"], t["gae_with_returns", "values"],
+                t["gae_with_returns", "terminateds"], None, None, None, t["gae_with_returns", "advantages"],
+                t["gae_with_returns", "returns"], GAMMA, LAMBDA)
         if "prefix_sum_i32" in self.estimators:
             c["prefix_sum_i32"] = lambda: R.rlscan_episodic_prefix_sum(
                 t["prefix_sum_i32", "x"], t["prefix_sum_i32", "dones"], t["prefix_sum_i32", "out"])
@@ -462,13 +474,15 @@ def run_gpu(args):
         # per-estimator: back-to-back launches of one estimator over buffer
         # sets whose total exceeds 4x L2
         per_est = {}
-        for est in names:
+        for est in names + list(EXTRA_CALLS):
             nbytes = bytes_per_env_step(est) * E_ENVS * T_STEPS
             n_rot = max(2, -(-ROTATE_BYTES // nbytes))
-            est_sets = [sets[i % n_sets] for i in range(n_rot)] if n_rot <= n_sets else None
-            if est_sets is None:  # need more distinct buffers than the step sets hold
-                est_sets = sets + [BufferSet(torch, device, [est]) for _ in range(n_rot - n_sets)]
-                for s in est_sets[n_sets:]:
+            if est in ESTIMATORS:
+                est_sets = sets + [BufferSet(torch, device, [est]) for _ in range(max(0, n_rot - n_sets))]
+            else:  # a call outside the step: buffers of its own only
+                est_sets = [BufferSet(torch, device, [est]) for _ in range(n_rot)]
+            for s in est_sets:
+                if est not in s.estimators or s not in sets:
                     s.fill_from_host(host)
             fns = [s.calls(R)[est] for s in est_sets]
             for f in fns:
@@ -491,8 +505,7 @@ def run_gpu(args):
                             "env_steps_per_s": E_ENVS * T_STEPS / (us * 1e-6),
                             "gb_per_s": nbytes / (us * 1e-6) / 1e9}
             del g
-            extra = est_sets[n_sets:]
-            del est_sets, fns, extra
+            del est_sets, fns
         R.rlscan_check()
 
         # e2e: every step copies its inputs host -> device from pinned memory,
@@ -551,6 +564,12 @@ def run_gpu(args):
     if rank != 0:
         return 0
     peak, peak_kind = measured_hbm_peak()
+    extra = {e: per_est.pop(e) for e in list(EXTRA_CALLS)}
+    for e, rec in extra.items():
+        rec["frac_of_hbm_peak"] = rec["gb_per_s"] / peak
+    if "gae_with_returns" in extra:
+        extra["gae_with_returns"]["separate_gae_plus_lambda_returns_us"] = (
+            per_est["gae"]["us_per_launch"] + per_est["lambda_returns"]["us_per_launch"])
     dominant = max(per_est, key=lambda e: per_est[e]["us_per_launch"])
     d = per_est[dominant]
     for est, rec in per_est.items():
@@ -575,6 +594,7 @@ def run_gpu(args):
                    "parallelism": f"replicas x{world}, each rank its own batch"},
         "hbm_gb_per_s_step": STEP_BYTES_PER_ENV_STEP * E_ENVS * T_STEPS * args.steps / (step_ms * 1e-3) / 1e9,
         "per_estimator": per_est,
+        "fused_calls": extra,
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": d["gb_per_s"], "peak": peak,
                      "unit": "GB/s", "frac": d["gb_per_s"] / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"

@@ -111,6 +111,23 @@ RLSCAN_API int rlscan_gae(const float *rewards, const float *values, const float
                size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * GAE and TD(lambda) returns in one pass (README "Kernels": compute_gae and
+ * compute_lambda_returns over the same rewards, values and flags).  The
+ * lambda-return equals the GAE advantage plus the value at every step
+ * (Schulman et al. 2016, GAE section on value targets), so one scan gives
+ * both: advantages_t = A_t as rlscan_gae, returns_t = A_t + V_t, which equals
+ * rlscan_lambda_returns on the same inputs up to fp32 rounding.  Reads the
+ * inputs once for both outputs (20 bytes per env-step instead of 32 for the
+ * two calls).  Arguments as rlscan_gae plus the `returns` output [E,T]; the
+ * two outputs must not overlap each other or any input.
+ */
+RLSCAN_API int rlscan_gae_with_returns(const float *rewards, const float *values, const float *terminateds,
+                                       const float *truncateds, const float *bootstrap_values,
+                                       const float *last_values, float *advantages, float *returns, int64_t E,
+                                       int64_t T, float gamma, float lambda_, void *ws, size_t ws_bytes,
+                                       cudaStream_t stream);
+
+/*
  * V-Trace (README "Kernels": compute_vtrace, "IS-weighted targets and
  * advantages"; IMPALA, Espeholt et al. 2018, section 4.1).
  *   rho_t = min(rho_bar, exp(log_rho_t)),  c_t = lambda min(c_bar, exp(log_rho_t))

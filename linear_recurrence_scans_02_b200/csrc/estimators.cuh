@@ -80,20 +80,25 @@ __device__ __forceinline__ float row_last_value(const float *__restrict__ lv, lo
 }
 
 // ---------------------------------------------------------------------------
-// GAE: x = A,  a_t = gamma lambda (episode goes on, not row end), b_t = delta_t
+// GAE: x = A,  a_t = gamma lambda (episode goes on, not row end), b_t = delta_t.
+// kWithReturns: also write the TD(lambda) returns G_t = A_t + V_t from the
+// same pass (the lambda-return equals the GAE advantage plus the value,
+// step for step, within episodes and across truncations).
 // ---------------------------------------------------------------------------
-struct GaeEst {
+template <bool kWithReturns>
+struct GaeEstT {
     static constexpr bool kBackward = true;
     using AT = float;
     using BT = float;
     struct Params {
         const float *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
         float *advantages;
+        float *returns; // kWithReturns only
         float gamma, lambda_;
     };
     template <int V>
     struct State {
-        float r[V], v[V], te[V], tr[V], out[V];
+        float r[V], v[V], te[V], tr[V], out[V], ret[V];
         float v_next;
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
@@ -148,12 +153,17 @@ struct GaeEst {
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
+        if constexpr (kWithReturns) S.ret[k] = x + S.v[k];
     }
     template <int V>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.advantages, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
+        const bool vec = g.vec_ok && i0 + V <= g.n;
+        store_plane<V>(P.advantages, i0, g.n, vec, S.out);
+        if constexpr (kWithReturns) store_plane<V>(P.returns, i0, g.n, vec, S.ret);
     }
 };
+using GaeEst = GaeEstT<false>;
+using GaeReturnsEst = GaeEstT<true>;
 
 // ---------------------------------------------------------------------------
 // TD(lambda): x = G,  a_t = gamma lambda, b_t = r_t + gamma (1 - lambda) V_{t+1}

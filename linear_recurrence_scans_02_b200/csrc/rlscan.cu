@@ -385,9 +385,34 @@ int rlscan_gae(const float *rewards, const float *values, const float *terminate
     const Span outs[] = {{advantages, pb, "advantages"}};
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
     GaeEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
-                     last_values, advantages, gamma, lambda_};
+                     last_values, advantages, nullptr, gamma, lambda_};
     return run<GaeEst>("rlscan_gae", P, E, T, 1, ws, ws_bytes, stream,
                        aligned16({rewards, values, terminateds, truncateds, advantages}));
+}
+
+int rlscan_gae_with_returns(const float *rewards, const float *values, const float *terminateds,
+                            const float *truncateds, const float *bootstrap_values, const float *last_values,
+                            float *advantages, float *returns, int64_t E, int64_t T, float gamma, float lambda_,
+                            void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(values, "values"));
+    RLSCAN_TRY(require(advantages, "advantages"));
+    RLSCAN_TRY(require(returns, "returns"));
+    if (truncateds && !bootstrap_values) return fail(RLSCAN_ERR_INVALID_ARG, "truncateds given without bootstrap_values");
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{rewards, pb, "rewards"}, {values, pb, "values"}, {terminateds, pb, "terminateds"},
+                        {truncateds, pb, "truncateds"}, {bootstrap_values, pb, "bootstrap_values"},
+                        {last_values, (size_t)E * 4, "last_values"}};
+    const Span outs[] = {{advantages, pb, "advantages"}, {returns, pb, "returns"}};
+    RLSCAN_TRY(check_aliasing(ins, 6, outs, 2));
+    GaeReturnsEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
+                            last_values, advantages, returns, gamma, lambda_};
+    return run<GaeReturnsEst>("rlscan_gae_with_returns", P, E, T, 1, ws, ws_bytes, stream,
+                              aligned16({rewards, values, terminateds, truncateds, advantages, returns}));
 }
 
 int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,

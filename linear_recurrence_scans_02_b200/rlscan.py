@@ -31,10 +31,10 @@ from . import _build
 
 __all__ = [
     "RlscanError", "library_path",
-    "rlscan_gae", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
+    "rlscan_gae", "rlscan_gae_with_returns", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
     "rlscan_discounted_returns", "rlscan_eligibility_traces", "rlscan_episodic_prefix_sum",
     "rlscan_workspace_bytes", "rlscan_check", "rlscan_plan", "rlscan_debug_set_lookback",
-    "compute_gae", "compute_vtrace", "compute_retrace", "compute_lambda_returns",
+    "compute_gae", "compute_gae_with_returns", "compute_vtrace", "compute_retrace", "compute_lambda_returns",
     "compute_discounted_returns", "compute_eligibility_traces", "compute_episodic_prefix_sum",
 ]
 
@@ -72,6 +72,7 @@ def _load_library():
                              ctypes.c_void_p, ctypes.c_int)
     sigs = {
         "rlscan_gae": [P] * 7 + [I64, I64, F, F, P, SZ, S],
+        "rlscan_gae_with_returns": [P] * 8 + [I64, I64, F, F, P, SZ, S],
         "rlscan_vtrace": [P] * 9 + [I64, I64, F, F, F, F, P, SZ, S],
         "rlscan_retrace": [P] * 8 + [I64, I64, I64, F, F, F, P, SZ, S],
         "rlscan_lambda_returns": [P] * 7 + [I64, I64, F, F, P, SZ, S],
@@ -211,6 +212,20 @@ def rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_
         E, T, float(gamma), float(lambda_), wp, wn, s))
 
 
+def rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages,
+                            returns, gamma, lambda_, ws=None):
+    E, T = _shape(rewards, "rewards")
+    dev = rewards.device
+    sh = (E, T)
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_gae_with_returns(
+        _ptr(rewards, "rewards", sh, device=dev), _ptr(values, "values", sh, device=dev),
+        _ptr(terminateds, "terminateds", sh, device=dev), _ptr(truncateds, "truncateds", sh, device=dev),
+        _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
+        _ptr(last_values, "last_values", (E,), device=dev), _ptr(advantages, "advantages", sh, device=dev),
+        _ptr(returns, "returns", sh, device=dev), E, T, float(gamma), float(lambda_), wp, wn, s))
+
+
 def rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values,
                   vs, pg_advantages, gamma, lambda_=1.0, rho_bar=1.0, c_bar=1.0, ws=None):
     E, T = _shape(rewards, "rewards")
@@ -309,6 +324,16 @@ def compute_gae(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, trunc
     adv = torch.empty_like(rewards)
     rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, gamma, lambda_)
     return adv
+
+
+def compute_gae_with_returns(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
+                             bootstrap_values=None, last_values=None):
+    """(advantages, returns) from one pass: returns = advantages + values."""
+    adv = torch.empty_like(rewards)
+    ret = torch.empty_like(rewards)
+    rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret,
+                            gamma, lambda_)
+    return adv, ret
 
 
 def compute_vtrace(log_rhos, rewards, values, terminateds, gamma=0.99, lambda_=1.0, rho_bar=1.0, c_bar=1.0, *,

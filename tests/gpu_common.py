@@ -174,3 +174,18 @@ BACKWARD_KEYS = {
 }
 BACKWARD_RUN = {"gae": run_gae, "lambda_returns": run_lambda_returns, "discounted_returns": run_discounted_returns,
                 "vtrace": run_vtrace}
+
+
+def run_gae_with_returns(d, gamma=W.GAMMA, lam=W.LAMBDA, offset=0):
+    """The fused call against two independent oracle functions: GAE for the
+    advantages and TD(lambda) for the returns."""
+    t = {k: dev(v, offset) for k, v in d.items()}
+    adv = empty_like_dev(d["rewards"], offset)
+    ret = empty_like_dev(d["rewards"], offset)
+    R.rlscan_gae_with_returns(t["rewards"], t["values"], t.get("terminateds"), t.get("truncateds"),
+                              t.get("bootstrap_values"), t.get("last_values"), adv, ret, gamma, lam)
+    args = (d.get("truncateds"), d.get("bootstrap_values"), d.get("last_values"))
+    radv = oracle.gae(d["rewards"], d["values"], d.get("terminateds"), np.float32(gamma), np.float32(lam), *args)
+    rret = oracle.lambda_returns(d["rewards"], d["values"], d.get("terminateds"), np.float32(gamma),
+                                 np.float32(lam), *args)
+    return {"advantages": adv, "returns": ret}, {"advantages": radv, "returns": rret}

@@ -33,6 +33,7 @@ def lib(rlscan_lib_path):
     P, I64, F, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
     L.rlscan_gae.argtypes = [P] * 7 + [I64, I64, F, F, P, SZ, P]
     L.rlscan_vtrace.argtypes = [P] * 9 + [I64, I64, F, F, F, F, P, SZ, P]
+    L.rlscan_gae_with_returns.argtypes = [P] * 8 + [I64, I64, F, F, P, SZ, P]
     L.rlscan_retrace.argtypes = [P] * 8 + [I64, I64, I64, F, F, F, P, SZ, P]
     L.rlscan_lambda_returns.argtypes = [P] * 7 + [I64, I64, F, F, P, SZ, P]
     L.rlscan_discounted_returns.argtypes = [P] * 6 + [I64, I64, F, P, SZ, P]
@@ -180,3 +181,9 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
                                   None) == WORKSPACE
     assert "fixed scratch holds" in msg(lib)
     assert lib.rlscan_gae_noalloc(None, B, C, None, None, None, O1, 4, 128, 0.99, 0.95, None) == INVALID
+
+
+def test_gae_with_returns_rejects_overlapping_outputs(lib):
+    assert lib.rlscan_gae_with_returns(A, B, C, None, None, None, O1, O1 + 8, E, T, 0.99, 0.95, None, 0, None) == INVALID
+    assert lib.rlscan_gae_with_returns(A, B, C, None, None, None, O1, None, E, T, 0.99, 0.95, None, 0, None) == INVALID
+    assert lib.rlscan_gae_with_returns(A, B, C, None, None, None, O1, B, E, T, 0.99, 0.95, None, 0, None) == INVALID

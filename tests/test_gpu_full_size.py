@@ -16,8 +16,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_common import assert_close, assert_equal_int, check, dev, run_gae, run_lambda_returns, \
-    run_discounted_returns, run_prefix, run_retrace, run_traces, run_vtrace, tol_for
+from gpu_common import assert_close, assert_equal_int, check, dev, run_gae, run_gae_with_returns, \
+    run_lambda_returns, run_discounted_returns, run_prefix, run_retrace, run_traces, run_vtrace, tol_for
 from linear_recurrence_scans_02_b200 import rlscan as R
 from linear_recurrence_scans_02_b200 import workloads as W
 
@@ -35,6 +35,7 @@ def test_all_estimators_4096x128():
     d = W.gae_inputs(E, T, seed=1, p_term=0.005)
     check(run_gae(d, G, L), T, "gae")
     check(run_lambda_returns(d, G, L), T, "lambda_returns")
+    check(run_gae_with_returns(d, G, L), T, "gae+returns")
     check(run_discounted_returns({k: d[k] for k in ("rewards", "terminateds")}, G), T, "returns")
     v = W.vtrace_inputs(E, T, seed=2, p_term=0.005)
     check(run_vtrace(v, G, 1.0, 1.0, 1.0), T, "vtrace lambda=1")
@@ -51,6 +52,7 @@ def test_truncation_path_4096x128():
     d = W.vtrace_inputs(E, T, seed=6, p_term=0.005, p_trunc=0.005)
     keys = ("rewards", "values", "terminateds", "truncateds", "bootstrap_values")
     check(run_gae({k: d[k] for k in keys}, G, L), T, "gae trunc")
+    check(run_gae_with_returns({k: d[k] for k in keys}, G, L), T, "gae+returns trunc")
     check(run_lambda_returns({k: d[k] for k in keys}, G, L), T, "lambda trunc")
     check(run_discounted_returns({k: d[k] for k in keys if k != "values"}, G), T, "returns trunc")
     check(run_vtrace(d, G, 1.0, 1.0, 1.0), T, "vtrace trunc")

@@ -10,8 +10,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_common import (BACKWARD_KEYS, BACKWARD_RUN, check, dev, inputs_backward, run_gae, run_prefix,
-                        run_retrace, run_traces, run_vtrace, strip)
+from gpu_common import (BACKWARD_KEYS, BACKWARD_RUN, check, dev, inputs_backward, run_gae, run_gae_with_returns,
+                        run_prefix, run_retrace, run_traces, run_vtrace, strip)
 from linear_recurrence_scans_02_b200 import rlscan as R
 from linear_recurrence_scans_02_b200 import workloads as W
 
@@ -218,3 +218,18 @@ def test_truncation_at_every_position_in_a_thread(est):
         return
     lam = 1.0 if est == "vtrace" else 0.5
     check(BACKWARD_RUN[est](strip(d, BACKWARD_KEYS[est]), gamma=0.5, lam=lam), T, f"{est} flag positions")
+
+
+@pytest.mark.parametrize("E,T", SHAPES, ids=lambda v: str(v))
+@pytest.mark.parametrize("variant", ["plain", "trunc", "trunc_lv"])
+def test_gae_with_returns(E, T, variant):
+    d = inputs_backward(E, T, seed=E * 31 + T, p_term=0.02, p_trunc=0.02 if variant != "plain" else 0.0,
+                        last_values=variant == "trunc_lv")
+    check(run_gae_with_returns(strip(d, BACKWARD_KEYS["gae"]), gamma=0.99, lam=0.95), T,
+          f"gae+returns {E}x{T} {variant}")
+
+
+@pytest.mark.parametrize("offset", [1, 3])
+def test_gae_with_returns_unaligned(offset):
+    d = inputs_backward(5, 129, seed=offset, p_term=0.02, p_trunc=0.02, last_values=True)
+    check(run_gae_with_returns(strip(d, BACKWARD_KEYS["gae"]), offset=offset), 129, f"gae+returns offset={offset}")
