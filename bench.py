@@ -69,13 +69,18 @@ INT_PLANES = {("prefix_sum_i32", "x"), ("prefix_sum_i32", "out")}
 # pass that replaces the two separate calls
 EXTRA_CALLS = {
     "gae_with_returns": (["rewards", "values", "terminateds"], ["advantages", "returns"]),
+    # the same pass on reduced-byte inputs: bf16 rewards and values, uint8 dones
+    "gae_with_returns_bf16_u8": (["rewards", "values", "terminateds"], ["advantages", "returns"]),
 }
 PLANES = {**ESTIMATORS, **EXTRA_CALLS}
+# planes stored narrower than fp32 (element bytes); outputs stay fp32
+NARROW = {("gae_with_returns_bf16_u8", "rewards"): 2, ("gae_with_returns_bf16_u8", "values"): 2,
+          ("gae_with_returns_bf16_u8", "terminateds"): 1}
 
 
 def bytes_per_env_step(est: str) -> int:
     ins, outs = PLANES[est]
-    return 4 * (len(ins) + len(outs))
+    return sum(NARROW.get((est, p), 4) for p in ins + outs)
 
 
 STEP_BYTES_PER_ENV_STEP = sum(bytes_per_env_step(e) for e in ESTIMATORS)
@@ -95,7 +100,8 @@ def host_inputs(seed: int = 0) -> dict:
     pi = W.prefix_inputs_i32(E, T, seed + 7, p_done=P_DONE)
     gr = W.gae_inputs(E, T, seed + 8, p_term=P_DONE)
     return {"gae": g, "vtrace": v, "retrace": r, "lambda_returns": lr, "discounted_returns": dr,
-            "eligibility_traces": et, "prefix_sum_f32": pf, "prefix_sum_i32": pi, "gae_with_returns": gr}
+            "eligibility_traces": et, "prefix_sum_f32": pf, "prefix_sum_i32": pi, "gae_with_returns": gr,
+            "gae_with_returns_bf16_u8": gr}
 
 
 # ---------------------------------------------------------------------------
@@ -126,14 +132,18 @@ class BufferSet:
     def _view(buf, i, key):
         import torch
         plane = E_ENVS * T_STEPS
-        v = buf[i * plane:(i + 1) * plane].view(E_ENVS, T_STEPS)
+        v = buf[i * plane:(i + 1) * plane]
+        if key in NARROW:  # the first plane-size elements of the narrow dtype
+            dt = {2: torch.bfloat16, 1: torch.uint8}[NARROW[key]]
+            return v.view(dt)[:plane].view(E_ENVS, T_STEPS)
+        v = v.view(E_ENVS, T_STEPS)
         return v.view(torch.int32) if key in INT_PLANES else v
 
     def fill_from_host(self, host):
         import torch
         for (e, p) in self.in_names:
-            src = host[e][p]
-            self.t[(e, p)].copy_(torch.from_numpy(np.ascontiguousarray(src)))
+            src = torch.from_numpy(np.ascontiguousarray(host[e][p]))
+            self.t[(e, p)].copy_(src.to(self.t[(e, p)].dtype))
 
     def calls(self, R):
         """One closure per estimator: the C-ABI call on this set."""
@@ -171,6 +181,10 @@ class BufferSet:
                 t["gae_with_returns", "rewards"], t["gae_with_returns", "values"],
                 t["gae_with_returns", "terminateds"], None, None, None, t["gae_with_returns", "advantages"],
                 t["gae_with_returns", "returns"], GAMMA, LAMBDA)
+        if "gae_with_returns_bf16_u8" in self.estimators:
+            k = "gae_with_returns_bf16_u8"
+            c[k] = lambda: R.rlscan_gae_typed(t[k, "rewards"], t[k, "values"], t[k, "terminateds"], None, None, None,
+                                              t[k, "advantages"], t[k, "returns"], GAMMA, LAMBDA)
         if "prefix_sum_i32" in self.estimators:
             c["prefix_sum_i32"] = lambda: R.rlscan_episodic_prefix_sum(
                 t["prefix_sum_i32", "x"], t["prefix_sum_i32", "dones"], t["prefix_sum_i32", "out"])

@@ -88,7 +88,10 @@ typedef enum rlscan_status {
 
 typedef enum rlscan_dtype {
     RLSCAN_F32 = 0,
-    RLSCAN_I32 = 1
+    RLSCAN_I32 = 1,
+    RLSCAN_BF16 = 2,
+    RLSCAN_F16 = 3,
+    RLSCAN_U8 = 4
 } rlscan_dtype;
 
 /* Largest action count accepted by rlscan_retrace. */
@@ -126,6 +129,25 @@ RLSCAN_API int rlscan_gae_with_returns(const float *rewards, const float *values
                                        const float *last_values, float *advantages, float *returns, int64_t E,
                                        int64_t T, float gamma, float lambda_, void *ws, size_t ws_bytes,
                                        cudaStream_t stream);
+
+/*
+ * GAE (and, when `returns` is not NULL, the TD(lambda) returns of the same
+ * pass, as rlscan_gae_with_returns) from reduced-byte inputs: rewards,
+ * values and bootstrap_values of `value_dtype` (RLSCAN_F32, RLSCAN_BF16 or
+ * RLSCAN_F16), terminateds and truncateds of `flag_dtype` (RLSCAN_F32 or
+ * RLSCAN_U8, one byte per flag, set iff nonzero; a bool tensor is RLSCAN_U8).
+ * The path is memory-bound, so narrower inputs are fewer bytes: bf16 values
+ * with u8 flags move 9 bytes per env-step for GAE instead of 16.  Inputs are
+ * widened to fp32 in registers and all arithmetic and both outputs are fp32,
+ * so results equal the fp32 entry points run on the widened inputs up to
+ * fp32 rounding.  last_values stays fp32 [E].  Other arguments and errors as
+ * rlscan_gae; an unsupported dtype returns RLSCAN_ERR_UNSUPPORTED.
+ */
+RLSCAN_API int rlscan_gae_typed(const void *rewards, const void *values, const void *terminateds,
+                                const void *truncateds, const void *bootstrap_values, const float *last_values,
+                                float *advantages, float *returns, int64_t E, int64_t T, float gamma,
+                                float lambda_, int value_dtype, int flag_dtype, void *ws, size_t ws_bytes,
+                                cudaStream_t stream);
 
 /*
  * V-Trace (README "Kernels": compute_vtrace, "IS-weighted targets and

@@ -23,11 +23,11 @@ namespace rlscan {
 struct StepFlags {
     bool term, trn, cont;
 };
-template <bool kTrunc = true>
-__device__ __forceinline__ StepFlags step_flags(float te, float tr) {
+template <bool kTrunc = true, class F = float>
+__device__ __forceinline__ StepFlags step_flags(F te, F tr) {
     StepFlags f;
-    f.term = te != 0.0f;
-    f.trn = kTrunc && (tr != 0.0f) && !f.term;
+    f.term = te != F(0);
+    f.trn = kTrunc && (tr != F(0)) && !f.term;
     f.cont = !f.term && !f.trn;
     return f;
 }
@@ -85,34 +85,46 @@ __device__ __forceinline__ float row_last_value(const float *__restrict__ lv, lo
 // same pass (the lambda-return equals the GAE advantage plus the value,
 // step for step, within episodes and across truncations).
 // ---------------------------------------------------------------------------
-template <bool kWithReturns>
+template <bool kWithReturns, class ValT = float, class FlagT = float>
 struct GaeEstT {
     static constexpr bool kBackward = true;
     using AT = float;
     using BT = float;
     struct Params {
-        const float *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        const ValT *rewards, *values;
+        const FlagT *terminateds, *truncateds;
+        const ValT *bootstrap_values;
+        const float *last_values;
         float *advantages;
-        float *returns; // kWithReturns only
+        float *returns; // kWithReturns only; may be null there
         float gamma, lambda_;
     };
     template <int V>
     struct State {
-        float r[V], v[V], te[V], tr[V], out[V], ret[V];
+        float r[V], v[V], out[V], ret[V];
+        FlagReg<FlagT> te[V], tr[V];
         float v_next;
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
-        prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds);
+        const long long left = g.n - tile0;
+        const long long cnt = left < S ? left : S;
+        switch (threadIdx.x) {
+        case 0: prefetch_l2(P.rewards, tile0, cnt, sizeof(ValT)); break;
+        case 1: prefetch_l2(P.values, tile0, cnt, sizeof(ValT)); break;
+        case 2: prefetch_l2(P.terminateds, tile0, cnt, sizeof(FlagT)); break;
+        case 3: prefetch_l2(P.truncateds, tile0, cnt, sizeof(FlagT)); break;
+        default: break;
+        }
     }
     template <int NT, int V>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
                                                 State<V> &S, unsigned char *) {
         const bool vec = g.vec_ok && i0 + V <= g.n;
-        const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
-        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
-        load_plane<V>(P.values, i0, g.n, vec, S.v);
-        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
+        const float h_v_next = lane == 31 ? load_one_widen(P.values, i0 + V, g.n) : 0.0f;
+        load_plane_widen<V>(P.rewards, i0, g.n, vec, S.r);
+        load_plane_widen<V>(P.values, i0, g.n, vec, S.v);
+        load_flags<V>(P.terminateds, i0, g.n, vec, S.te);
+        load_flags<V>(P.truncateds, i0, g.n, vec, S.tr);
         S.v_next = next_halo<V>(S.v, h_v_next, lane);
     }
     template <int V, bool kTrunc, bool kFast>
@@ -127,7 +139,7 @@ struct GaeEstT {
                 const bool rowend = elem_row_end<kFast, V>(rm, k);
                 float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
                 if (rowend) nv = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
-                const float boot = f.cont ? nv : (f.trn ? __ldcg(P.bootstrap_values + i0 + k) : 0.0f);
+                const float boot = f.cont ? nv : (f.trn ? load_one_widen(P.bootstrap_values, i0 + k, g.n) : 0.0f);
                 a[k] = (f.cont && !rowend) ? gl : 0.0f;
                 b[k] = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
             } else {
@@ -159,11 +171,16 @@ struct GaeEstT {
     static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
         const bool vec = g.vec_ok && i0 + V <= g.n;
         store_plane<V>(P.advantages, i0, g.n, vec, S.out);
-        if constexpr (kWithReturns) store_plane<V>(P.returns, i0, g.n, vec, S.ret);
+        if constexpr (kWithReturns) {
+            if (P.returns != nullptr) store_plane<V>(P.returns, i0, g.n, vec, S.ret);
+        }
     }
 };
 using GaeEst = GaeEstT<false>;
 using GaeReturnsEst = GaeEstT<true>;
+// reduced-byte inputs (returns written when P.returns is set)
+template <class ValT, class FlagT>
+using GaeTypedEst = GaeEstT<true, ValT, FlagT>;
 
 // ---------------------------------------------------------------------------
 // TD(lambda): x = G,  a_t = gamma lambda, b_t = r_t + gamma (1 - lambda) V_{t+1}

@@ -415,6 +415,57 @@ int rlscan_gae_with_returns(const float *rewards, const float *values, const flo
                               aligned16({rewards, values, terminateds, truncateds, advantages, returns}));
 }
 
+int rlscan_gae_typed(const void *rewards, const void *values, const void *terminateds, const void *truncateds,
+                     const void *bootstrap_values, const float *last_values, float *advantages, float *returns,
+                     int64_t E, int64_t T, float gamma, float lambda_, int value_dtype, int flag_dtype, void *ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+    size_t vsz, fsz;
+    switch (value_dtype) {
+    case RLSCAN_F32: vsz = 4; break;
+    case RLSCAN_BF16:
+    case RLSCAN_F16: vsz = 2; break;
+    default: return fail(RLSCAN_ERR_UNSUPPORTED, "value_dtype %d not supported (F32, BF16, F16)", value_dtype);
+    }
+    switch (flag_dtype) {
+    case RLSCAN_F32: fsz = 4; break;
+    case RLSCAN_U8: fsz = 1; break;
+    default: return fail(RLSCAN_ERR_UNSUPPORTED, "flag_dtype %d not supported (F32, U8)", flag_dtype);
+    }
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(values, "values"));
+    RLSCAN_TRY(require(advantages, "advantages"));
+    if (truncateds && !bootstrap_values) return fail(RLSCAN_ERR_INVALID_ARG, "truncateds given without bootstrap_values");
+    const size_t n = (size_t)(E * T);
+    const Span ins[] = {{rewards, n * vsz, "rewards"}, {values, n * vsz, "values"},
+                        {terminateds, n * fsz, "terminateds"}, {truncateds, n * fsz, "truncateds"},
+                        {bootstrap_values, n * vsz, "bootstrap_values"}, {last_values, (size_t)E * 4, "last_values"}};
+    const Span outs[] = {{advantages, n * 4, "advantages"}, {returns, n * 4, "returns"}};
+    RLSCAN_TRY(check_aliasing(ins, 6, outs, 2));
+    const bool vec = aligned16({rewards, values, terminateds, truncateds, advantages, returns});
+    const void *bv = truncateds ? bootstrap_values : nullptr;
+#define RLSCAN_GAE_TYPED(VT, FT)                                                                                  \
+    do {                                                                                                          \
+        typename GaeTypedEst<VT, FT>::Params P{static_cast<const VT *>(rewards), static_cast<const VT *>(values), \
+                                               static_cast<const FT *>(terminateds),                               \
+                                               static_cast<const FT *>(truncateds), static_cast<const VT *>(bv),  \
+                                               last_values, advantages, returns, gamma, lambda_};                  \
+        return run<GaeTypedEst<VT, FT>>("rlscan_gae_typed", P, E, T, 1, ws, ws_bytes, stream, vec);              \
+    } while (0)
+    if (flag_dtype == RLSCAN_U8) {
+        if (value_dtype == RLSCAN_BF16) RLSCAN_GAE_TYPED(__nv_bfloat16, uint8_t);
+        if (value_dtype == RLSCAN_F16) RLSCAN_GAE_TYPED(__half, uint8_t);
+        RLSCAN_GAE_TYPED(float, uint8_t);
+    }
+    if (value_dtype == RLSCAN_BF16) RLSCAN_GAE_TYPED(__nv_bfloat16, float);
+    if (value_dtype == RLSCAN_F16) RLSCAN_GAE_TYPED(__half, float);
+    RLSCAN_GAE_TYPED(float, float);
+#undef RLSCAN_GAE_TYPED
+}
+
 int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
                   const float *truncateds, const float *bootstrap_values, const float *last_values, float *vs,
                   float *pg_advantages, int64_t E, int64_t T, float gamma, float lambda_, float rho_bar,

@@ -27,6 +27,8 @@
 #include <cstdint>
 #include <type_traits>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace rlscan {
 
@@ -458,6 +460,111 @@ template <class T>
 __device__ __forceinline__ T load_one(const T *__restrict__ p, long long i, long long n) {
     return (p != nullptr && i >= 0 && i < n) ? __ldcg(p + i) : T(0);
 }
+
+// Reduced-byte planes, widened to fp32 in registers: bf16 or fp16 values,
+// uint8 flags (nonzero = set).  The vector path reads V * sizeof(T) bytes per
+// thread in one load (16 bytes for eight bf16, 8 bytes for eight flags).
+__device__ __forceinline__ float widen(uint16_t bits, __nv_bfloat16) { return __uint_as_float((uint32_t)bits << 16); }
+__device__ __forceinline__ float widen(uint16_t bits, __half) { return __half2float(__ushort_as_half(bits)); }
+__device__ __forceinline__ float widen(uint8_t byte, uint8_t) { return byte != 0 ? 1.0f : 0.0f; }
+
+template <int V, class T>
+__device__ __forceinline__ void load_plane_widen(const T *__restrict__ p, long long i0, long long n, bool vec,
+                                                 float (&o)[V]) {
+    if constexpr (std::is_same<T, float>::value) {
+        load_plane<V>(p, i0, n, vec, o);
+    } else {
+        static_assert(sizeof(T) == 1 || sizeof(T) == 2, "8- or 16-bit planes");
+        using Bits = typename std::conditional<sizeof(T) == 2, uint16_t, uint8_t>::type;
+        const Bits *q = reinterpret_cast<const Bits *>(p);
+        if (q == nullptr) {
+#pragma unroll
+            for (int k = 0; k < V; ++k) o[k] = 0.0f;
+            return;
+        }
+        constexpr int kBytes = V * (int)sizeof(T);
+        if (vec) {
+            uint32_t w[kBytes / 4 > 0 ? kBytes / 4 : 1];
+            if constexpr (kBytes == 16) {
+                const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(q + i0));
+                w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+            } else if constexpr (kBytes == 8) {
+                const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(q + i0));
+                w[0] = v.x; w[1] = v.y;
+            } else {
+                static_assert(kBytes == 4, "V * sizeof(T) must be 4, 8 or 16 bytes");
+                w[0] = __ldcg(reinterpret_cast<const unsigned int *>(q + i0));
+            }
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                const uint32_t word = w[(k * (int)sizeof(T)) / 4];
+                const int shift = 8 * ((k * (int)sizeof(T)) % 4);
+                if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+                    // a bf16 is the high half of an fp32: one shift or mask
+                    o[k] = __uint_as_float(shift == 0 ? (word << 16) : (word & 0xffff0000u));
+                } else {
+                    o[k] = widen((Bits)(word >> shift), T());
+                }
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                const long long i = i0 + k;
+                o[k] = (i >= 0 && i < n) ? widen((Bits)__ldcg(q + i), T()) : 0.0f;
+            }
+        }
+    }
+}
+
+// Flags as registers: fp32 flags stay floats, uint8 flags stay integers
+// (the byte itself); either way a flag is set iff nonzero.
+template <class FlagT>
+using FlagReg = typename std::conditional<std::is_same<FlagT, float>::value, float, uint32_t>::type;
+
+template <int V, class T>
+__device__ __forceinline__ void load_flags(const T *__restrict__ p, long long i0, long long n, bool vec,
+                                           FlagReg<T> (&o)[V]) {
+    if constexpr (std::is_same<T, float>::value) {
+        load_plane<V>(p, i0, n, vec, o);
+    } else {
+        static_assert(std::is_same<T, uint8_t>::value, "float or uint8 flags");
+        if (p == nullptr) {
+#pragma unroll
+            for (int k = 0; k < V; ++k) o[k] = 0u;
+            return;
+        }
+        if (vec) {
+            uint32_t w[V / 4];
+            if constexpr (V == 8) {
+                const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(p + i0));
+                w[0] = v.x; w[1] = v.y;
+            } else {
+                static_assert(V == 4, "V must be 4 or 8");
+                w[0] = __ldcg(reinterpret_cast<const unsigned int *>(p + i0));
+            }
+#pragma unroll
+            for (int k = 0; k < V; ++k) o[k] = (w[k / 4] >> (8 * (k % 4))) & 0xffu;
+        } else {
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                const long long i = i0 + k;
+                o[k] = (i >= 0 && i < n) ? (uint32_t)__ldcg(p + i) : 0u;
+            }
+        }
+    }
+}
+
+template <class T>
+__device__ __forceinline__ float load_one_widen(const T *__restrict__ p, long long i, long long n) {
+    if constexpr (std::is_same<T, float>::value) {
+        return load_one(p, i, n);
+    } else {
+        using Bits = typename std::conditional<sizeof(T) == 2, uint16_t, uint8_t>::type;
+        const Bits *q = reinterpret_cast<const Bits *>(p);
+        return (q != nullptr && i >= 0 && i < n) ? widen((Bits)__ldcg(q + i), T()) : 0.0f;
+    }
+}
+
 
 // ---------------------------------------------------------------------------
 // The tile kernel.  Est supplies (see estimators.cuh):

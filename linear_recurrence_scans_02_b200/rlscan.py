@@ -31,7 +31,7 @@ from . import _build
 
 __all__ = [
     "RlscanError", "library_path",
-    "rlscan_gae", "rlscan_gae_with_returns", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
+    "rlscan_gae", "rlscan_gae_with_returns", "rlscan_gae_typed", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
     "rlscan_discounted_returns", "rlscan_eligibility_traces", "rlscan_episodic_prefix_sum",
     "rlscan_workspace_bytes", "rlscan_check", "rlscan_plan", "rlscan_debug_set_lookback",
     "compute_gae", "compute_gae_with_returns", "compute_vtrace", "compute_retrace", "compute_lambda_returns",
@@ -46,6 +46,11 @@ RLSCAN_ERR_CUDA = 4
 RLSCAN_ERR_TIMEOUT = 5
 RLSCAN_F32 = 0
 RLSCAN_I32 = 1
+RLSCAN_BF16 = 2
+RLSCAN_F16 = 3
+RLSCAN_U8 = 4
+_VALUE_DTYPES = {torch.float32: RLSCAN_F32, torch.bfloat16: RLSCAN_BF16, torch.float16: RLSCAN_F16}
+_FLAG_DTYPES = {torch.float32: RLSCAN_F32, torch.uint8: RLSCAN_U8, torch.bool: RLSCAN_U8}
 
 _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
 
@@ -73,6 +78,7 @@ def _load_library():
     sigs = {
         "rlscan_gae": [P] * 7 + [I64, I64, F, F, P, SZ, S],
         "rlscan_gae_with_returns": [P] * 8 + [I64, I64, F, F, P, SZ, S],
+        "rlscan_gae_typed": [P] * 8 + [I64, I64, F, F, INT, INT, P, SZ, S],
         "rlscan_vtrace": [P] * 9 + [I64, I64, F, F, F, F, P, SZ, S],
         "rlscan_retrace": [P] * 8 + [I64, I64, I64, F, F, F, P, SZ, S],
         "rlscan_lambda_returns": [P] * 7 + [I64, I64, F, F, P, SZ, S],
@@ -226,6 +232,36 @@ def rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_
         _ptr(returns, "returns", sh, device=dev), E, T, float(gamma), float(lambda_), wp, wn, s))
 
 
+def rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages,
+                     returns, gamma, lambda_, ws=None):
+    """GAE (+ TD(lambda) returns when `returns` is given) from reduced-byte
+    inputs: rewards / values / bootstrap_values float32, bfloat16 or float16
+    (one dtype for the three), flags float32, uint8 or bool; fp32 outputs."""
+    E, T = _shape(rewards, "rewards")
+    dev = rewards.device
+    sh = (E, T)
+    vdt = _VALUE_DTYPES.get(rewards.dtype)
+    if vdt is None:
+        raise TypeError(f"rewards dtype {rewards.dtype} not supported")
+    flags = [f for f in (terminateds, truncateds) if f is not None]
+    fdt = _FLAG_DTYPES.get(flags[0].dtype) if flags else RLSCAN_F32
+    if fdt is None:
+        raise TypeError(f"flag dtype {flags[0].dtype} not supported")
+    vt = (rewards.dtype,)
+    ft = (flags[0].dtype,) if flags else (torch.float32,)
+    wp, wn, s = _workspace(dev, E, T, ws)
+    _raise_on(_lib.rlscan_gae_typed(
+        _ptr(rewards, "rewards", sh, vt, dev), _ptr(values, "values", sh, vt, dev),
+        _ptr(terminateds, "terminateds", sh, ft, dev), _ptr(truncateds, "truncateds", sh, ft, dev),
+        _ptr(bootstrap_values, "bootstrap_values", sh, vt, dev),
+        _ptr(last_values, "last_values", (E,), device=dev), _ptr(advantages, "advantages", sh, device=dev),
+        _ptr(returns, "returns", sh, device=dev), E, T, float(gamma), float(lambda_), vdt, fdt, wp, wn, s))
+
+
+def _reduced_bytes(*tensors):
+    return any(t is not None and t.dtype != torch.float32 for t in tensors)
+
+
 def rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values,
                   vs, pg_advantages, gamma, lambda_=1.0, rho_bar=1.0, c_bar=1.0, ws=None):
     E, T = _shape(rewards, "rewards")
@@ -321,18 +357,29 @@ def rlscan_episodic_prefix_sum(x, dones, out, ws=None):
 
 def compute_gae(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
                 bootstrap_values=None, last_values=None):
-    adv = torch.empty_like(rewards)
-    rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, gamma, lambda_)
+    """Advantages (fp32).  bf16/fp16 values or uint8/bool flags take the
+    reduced-byte entry point."""
+    adv = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
+    if _reduced_bytes(rewards, values, terminateds, truncateds, bootstrap_values):
+        rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, None, gamma,
+                         lambda_)
+    else:
+        rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, gamma, lambda_)
     return adv
 
 
 def compute_gae_with_returns(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
                              bootstrap_values=None, last_values=None):
-    """(advantages, returns) from one pass: returns = advantages + values."""
-    adv = torch.empty_like(rewards)
-    ret = torch.empty_like(rewards)
-    rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret,
-                            gamma, lambda_)
+    """(advantages, returns) from one pass: returns = advantages + values.
+    bf16/fp16 values or uint8/bool flags take the reduced-byte entry point."""
+    adv = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
+    ret = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
+    if _reduced_bytes(rewards, values, terminateds, truncateds, bootstrap_values):
+        rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret, gamma,
+                         lambda_)
+    else:
+        rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret,
+                                gamma, lambda_)
     return adv, ret
 
 

@@ -34,6 +34,7 @@ def lib(rlscan_lib_path):
     L.rlscan_gae.argtypes = [P] * 7 + [I64, I64, F, F, P, SZ, P]
     L.rlscan_vtrace.argtypes = [P] * 9 + [I64, I64, F, F, F, F, P, SZ, P]
     L.rlscan_gae_with_returns.argtypes = [P] * 8 + [I64, I64, F, F, P, SZ, P]
+    L.rlscan_gae_typed.argtypes = [P] * 8 + [I64, I64, F, F, ctypes.c_int, ctypes.c_int, P, SZ, P]
     L.rlscan_retrace.argtypes = [P] * 8 + [I64, I64, I64, F, F, F, P, SZ, P]
     L.rlscan_lambda_returns.argtypes = [P] * 7 + [I64, I64, F, F, P, SZ, P]
     L.rlscan_discounted_returns.argtypes = [P] * 6 + [I64, I64, F, P, SZ, P]
@@ -187,3 +188,12 @@ def test_gae_with_returns_rejects_overlapping_outputs(lib):
     assert lib.rlscan_gae_with_returns(A, B, C, None, None, None, O1, O1 + 8, E, T, 0.99, 0.95, None, 0, None) == INVALID
     assert lib.rlscan_gae_with_returns(A, B, C, None, None, None, O1, None, E, T, 0.99, 0.95, None, 0, None) == INVALID
     assert lib.rlscan_gae_with_returns(A, B, C, None, None, None, O1, B, E, T, 0.99, 0.95, None, 0, None) == INVALID
+
+
+def test_gae_typed_dtype_rules(lib):
+    BF16, F16, U8, I32 = 2, 3, 4, 1
+    assert lib.rlscan_gae_typed(A, B, C, None, None, None, O1, None, E, T, 0.99, 0.95, I32, U8, None, 0, None) == UNSUPPORTED
+    assert lib.rlscan_gae_typed(A, B, C, None, None, None, O1, None, E, T, 0.99, 0.95, BF16, BF16, None, 0, None) == UNSUPPORTED
+    # 2-byte values: planes of E*T*2 bytes; the output starting inside one is an overlap
+    assert lib.rlscan_gae_typed(A, B, C, None, None, None, A + 2, None, E, T, 0.99, 0.95, BF16, U8, None, 0, None) == INVALID
+    assert lib.rlscan_gae_typed(A, B, C, D, None, None, O1, None, E, T, 0.99, 0.95, F16, U8, None, 0, None) == INVALID
