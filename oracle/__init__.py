@@ -50,9 +50,9 @@ def _load():
                 "oracle_retrace": [_f32p] * 7 + [_f64p, _i64, _i64, _i64, _dbl, _dbl, _dbl],
                 "oracle_lambda_returns": [_f32p] * 6 + [_f64p, _i64, _i64, _dbl, _dbl],
                 "oracle_discounted_returns": [_f32p] * 5 + [_f64p, _i64, _i64, _dbl],
-                "oracle_eligibility_traces": [_f32p, _f32p, _f64p, _i64, _i64, _dbl, _dbl],
-                "oracle_episodic_prefix_sum_f32": [_f32p, _f32p, _f64p, _i64, _i64],
-                "oracle_episodic_prefix_sum_i32": [_i32p, _f32p, _i32p, _i64, _i64],
+                "oracle_eligibility_traces": [_f32p, _f32p, _f64p, _i64, _i64, _dbl, _dbl, ctypes.c_int],
+                "oracle_episodic_prefix_sum_f32": [_f32p, _f32p, _f64p, _i64, _i64, ctypes.c_int],
+                "oracle_episodic_prefix_sum_i32": [_i32p, _f32p, _i32p, _i64, _i64, ctypes.c_int],
             }
             for name, args in sigs.items():
                 fn = getattr(lib, name)
@@ -150,18 +150,22 @@ def discounted_returns(rewards, terminateds, gamma, truncateds=None, bootstrap_v
     return out
 
 
-def eligibility_traces(x, dones, gamma, lambda_):
+def eligibility_traces(x, dones, gamma, lambda_, done_starts_episode=False):
+    """done_starts_episode: read dones[t] as "t starts an episode" instead of
+    the default "t-1 ended one"."""
     E, T = _shape2(x)
     keep = [_f32(x, (E, T)), _f32(dones, (E, T))]
     out = np.empty((E, T), dtype=np.float64)
     rc = _load().oracle_eligibility_traces(*[k[1] for k in keep], out.ctypes.data_as(_f64p),
-                                           E, T, float(gamma), float(lambda_))
+                                           E, T, float(gamma), float(lambda_),
+                                           int(bool(done_starts_episode)))
     _check(rc, "eligibility_traces")
     return out
 
 
-def episodic_prefix_sum(x, dones):
-    """fp32 input -> fp64 output; int32 input -> int32 output (wrapping)."""
+def episodic_prefix_sum(x, dones, done_starts_episode=False):
+    """fp32 input -> fp64 output; int32 input -> int32 output (wrapping).
+    done_starts_episode as for eligibility_traces."""
     xa = np.asarray(x)
     E, T = _shape2(xa)
     d, dp = _f32(dones, (E, T))
@@ -169,11 +173,13 @@ def episodic_prefix_sum(x, dones):
         xi = np.ascontiguousarray(xa)
         out = np.empty((E, T), dtype=np.int32)
         rc = _load().oracle_episodic_prefix_sum_i32(xi.ctypes.data_as(_i32p), dp,
-                                                     out.ctypes.data_as(_i32p), E, T)
+                                                     out.ctypes.data_as(_i32p), E, T,
+                                                     int(bool(done_starts_episode)))
     else:
         xf, xp = _f32(xa, (E, T))
         out = np.empty((E, T), dtype=np.float64)
-        rc = _load().oracle_episodic_prefix_sum_f32(xp, dp, out.ctypes.data_as(_f64p), E, T)
+        rc = _load().oracle_episodic_prefix_sum_f32(xp, dp, out.ctypes.data_as(_f64p), E, T,
+                                                     int(bool(done_starts_episode)))
     _check(rc, "episodic_prefix_sum")
     return out
 

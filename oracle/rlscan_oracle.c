@@ -28,7 +28,9 @@
  *   - the value after the last step of a row (t = T-1, no flag) is
  *     last_values[e], or 0 when last_values is NULL;
  *   - forward estimators reset after a done: d[t-1] != 0 starts a new
- *     episode at t;
+ *     episode at t.  The README's trace formula writes (1-d) without a
+ *     subscript, so its other reading, d[t] != 0 marks t itself as the first
+ *     step of an episode, is the `done_starts_episode` argument;
  *   - a cut trace is a branch, not a multiplication by zero, so a non-finite
  *     value never leaks across an episode boundary.
  * All arithmetic is fp64 on the fp32 inputs widened exactly.
@@ -298,13 +300,16 @@ int oracle_discounted_returns(const float *rewards, const float *terminateds,
 
 /*
  * Eligibility traces (README "Kernels": accumulating forward traces
- * e[t] = x[t] + gamma*lambda*(1-d)*e[t-1]; the done that ends an episode at
- * t-1 resets the trace at t):
+ * e[t] = x[t] + gamma*lambda*(1-d)*e[t-1]).  Default reading: the done that
+ * ends an episode at t-1 resets the trace at t,
  *   e_t = x_t + gamma*lambda e_{t-1}   if t > 0 and d_{t-1} == 0,
- *   e_t = x_t                          otherwise.
+ *   e_t = x_t                          otherwise;
+ * with done_starts_episode != 0 the flag is read at t itself (d_t in place of
+ * d_{t-1} above: t is the first step of a new episode).
  */
 int oracle_eligibility_traces(const float *x, const float *dones, double *traces,
-                              int64_t E, int64_t T, double gamma, double lambda_)
+                              int64_t E, int64_t T, double gamma, double lambda_,
+                              int done_starts_episode)
 {
     if (check_common(x, traces, E, T))
         return ORACLE_EINVAL;
@@ -314,7 +319,8 @@ int oracle_eligibility_traces(const float *x, const float *dones, double *traces
         for (int64_t t = 0; t < T; ++t) {
             const int64_t i = row + t;
             double cur = (double)x[i];
-            if (t > 0 && !is_set(dones, i - 1))
+            const int reset = done_starts_episode ? is_set(dones, i) : (t > 0 && is_set(dones, i - 1));
+            if (t > 0 && !reset)
                 cur += gamma * lambda_ * prev;
             traces[i] = cur;
             prev = cur;
@@ -326,10 +332,11 @@ int oracle_eligibility_traces(const float *x, const float *dones, double *traces
 /*
  * Episodic prefix sum, fp32 input (README "Kernels": "episodic cumulative sum
  * with done-mask resets"):
- *   y_t = x_t + y_{t-1}   if t > 0 and d_{t-1} == 0,   y_t = x_t otherwise.
+ *   y_t = x_t + y_{t-1}   if t > 0 and d_{t-1} == 0,   y_t = x_t otherwise;
+ * with done_starts_episode != 0, d_t replaces d_{t-1}.
  */
 int oracle_episodic_prefix_sum_f32(const float *x, const float *dones, double *out,
-                                   int64_t E, int64_t T)
+                                   int64_t E, int64_t T, int done_starts_episode)
 {
     if (check_common(x, out, E, T))
         return ORACLE_EINVAL;
@@ -339,7 +346,8 @@ int oracle_episodic_prefix_sum_f32(const float *x, const float *dones, double *o
         for (int64_t t = 0; t < T; ++t) {
             const int64_t i = row + t;
             double cur = (double)x[i];
-            if (t > 0 && !is_set(dones, i - 1))
+            const int reset = done_starts_episode ? is_set(dones, i) : (t > 0 && is_set(dones, i - 1));
+            if (t > 0 && !reset)
                 cur += prev;
             out[i] = cur;
             prev = cur;
@@ -354,7 +362,7 @@ int oracle_episodic_prefix_sum_f32(const float *x, const float *dones, double *o
  * that overflows wraps the way 32-bit integer addition does.
  */
 int oracle_episodic_prefix_sum_i32(const int32_t *x, const float *dones, int32_t *out,
-                                   int64_t E, int64_t T)
+                                   int64_t E, int64_t T, int done_starts_episode)
 {
     if (check_common(x, out, E, T))
         return ORACLE_EINVAL;
@@ -364,7 +372,8 @@ int oracle_episodic_prefix_sum_i32(const int32_t *x, const float *dones, int32_t
         for (int64_t t = 0; t < T; ++t) {
             const int64_t i = row + t;
             int64_t cur = (int64_t)x[i];
-            if (t > 0 && !is_set(dones, i - 1))
+            const int reset = done_starts_episode ? is_set(dones, i) : (t > 0 && is_set(dones, i - 1));
+            if (t > 0 && !reset)
                 cur += prev;
             /* reduce modulo 2^32 into [-2^31, 2^31) */
             uint32_t low = (uint32_t)((uint64_t)cur & 0xffffffffu);

@@ -51,11 +51,17 @@ MUTANTS = {
     # discounted returns ignore the last value
     "returns_no_last_value": ("double r_next = last_value(last_values, e);", "double r_next = 0.0;"),
     # eligibility traces reset on d_t instead of d_{t-1}
-    "traces_reset_on_same_step": ("if (t > 0 && !is_set(dones, i - 1))\n                cur += gamma * lambda_ * prev;",
-                                  "if (t > 0 && !is_set(dones, i))\n                cur += gamma * lambda_ * prev;"),
+    "traces_reset_on_same_step": (": (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += gamma * lambda_ * prev;",
+                                  ": is_set(dones, i);\n            if (t > 0 && !reset)\n                cur += gamma * lambda_ * prev;"),
+    # the done-starts-episode reading of the trace still resets one step late
+    "traces_starts_reads_previous": ("const int reset = done_starts_episode ? is_set(dones, i) : (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += gamma * lambda_ * prev;",
+                                     "const int reset = (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += gamma * lambda_ * prev;"),
     # prefix sum never resets
-    "prefix_no_reset": ("if (t > 0 && !is_set(dones, i - 1))\n                cur += prev;\n            out[i] = cur;",
+    "prefix_no_reset": ("if (t > 0 && !reset)\n                cur += prev;\n            out[i] = cur;",
                         "if (t > 0)\n                cur += prev;\n            out[i] = cur;"),
+    # int32 prefix sum under the done-starts-episode reading resets one step early (reads the next flag)
+    "prefix_i32_starts_reads_next": ("done_starts_episode ? is_set(dones, i) : (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += prev;\n            /* reduce",
+                                     "done_starts_episode ? (t + 1 < T && is_set(dones, i + 1)) : (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += prev;\n            /* reduce"),
     # int32 prefix sum saturates instead of wrapping
     "prefix_i32_saturates": ("int64_t wrapped = (low >= 0x80000000u) ? (int64_t)low - 4294967296LL : (int64_t)low;",
                              "int64_t wrapped = cur > 2147483647LL ? 2147483647LL : (cur < -2147483648LL ? -2147483648LL : cur); (void)low;"),

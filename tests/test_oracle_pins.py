@@ -55,6 +55,8 @@ def _parse_golden(path):
             cur[key] = vals[0]
         elif key in ("gamma", "lambda", "rho_bar", "c_bar"):
             cur[key] = float(vals[0])
+        elif key == "done_starts_episode":
+            cur[key] = bool(int(vals[0]))
         else:
             cur["in"][key] = np.array([[float(v) for v in vals]], dtype=np.float32)
     return cases
@@ -84,9 +86,10 @@ def _run_golden(case):
                                         i["terminateds"], i["truncateds"], case["gamma"], case["lambda"],
                                         case["c_bar"])}
     if est == "eligibility_traces":
-        return {"traces": oracle.eligibility_traces(i["x"], i["dones"], case["gamma"], case["lambda"])}
+        return {"traces": oracle.eligibility_traces(i["x"], i["dones"], case["gamma"], case["lambda"],
+                                                    case.get("done_starts_episode", False))}
     if est == "episodic_prefix_sum":
-        return {"out": oracle.episodic_prefix_sum(i["x"], i["dones"])}
+        return {"out": oracle.episodic_prefix_sum(i["x"], i["dones"], case.get("done_starts_episode", False))}
     raise KeyError(est)
 
 
@@ -217,13 +220,24 @@ def _episode_start(d, t):
     return s
 
 
-def bf_traces(x, d, gl):
-    return [sum((gl ** (t - k) * F(float(x[k])) for k in range(_episode_start(d, t), t + 1)), F(0))
+def _episode_start_at_flag(d, t):
+    # done-starts-episode reading: the episode holding t starts at the last
+    # flagged step <= t (or at 0)
+    s = t
+    while s > 0 and d[s] == 0:
+        s -= 1
+    return s
+
+
+def bf_traces(x, d, gl, starts=False):
+    first = _episode_start_at_flag if starts else _episode_start
+    return [sum((gl ** (t - k) * F(float(x[k])) for k in range(first(d, t), t + 1)), F(0))
             for t in range(len(x))]
 
 
-def bf_prefix(x, d):
-    return [sum((F(float(x[k])) for k in range(_episode_start(d, t), t + 1)), F(0))
+def bf_prefix(x, d, starts=False):
+    first = _episode_start_at_flag if starts else _episode_start
+    return [sum((F(float(x[k])) for k in range(first(d, t), t + 1)), F(0))
             for t in range(len(x))]
 
 
@@ -350,6 +364,44 @@ def test_brute_force_traces_prefix_exact(seed):
     got = oracle.episodic_prefix_sum(xi[None], d[None])[0]
     want = bf_prefix(xi.astype(np.float32), d)
     assert [int(a) for a in got] == [int(b) for b in want]
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_brute_force_traces_prefix_done_starts_episode(seed):
+    # sum over the episode that holds t, its first step being the last flagged
+    # step <= t: written out from the definition, not from the oracle's loop
+    rng = np.random.default_rng(900 + seed)
+    T = int(rng.integers(1, 12))
+    x = _dyadic_row(rng, T)
+    d = _flags(rng, T, 0.3)
+    _exact(oracle.eligibility_traces(x[None], d[None], float(G), float(L), True)[0],
+           bf_traces(x, d, G * L, starts=True))
+    _exact(oracle.episodic_prefix_sum(x[None], d[None], True)[0], bf_prefix(x, d, starts=True))
+    xi = rng.integers(-100, 101, size=T).astype(np.int32)
+    got = oracle.episodic_prefix_sum(xi[None], d[None], True)[0]
+    want = bf_prefix(xi.astype(np.float32), d, starts=True)
+    assert [int(a) for a in got] == [int(b) for b in want]
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_done_conventions_are_one_step_shifts(seed):
+    # a flag that starts an episode at t is a flag that ended one at t - 1:
+    # the two readings agree once the flags move one step; the flag at t = 0
+    # (nothing before it to end) changes nothing under either
+    x = W.trace_inputs(3, 97, seed=40 + seed, p_done=0.08)
+    xi = W.prefix_inputs_i32(3, 97, seed=40 + seed, p_done=0.08)
+    d = x["dones"]
+    d_ends = np.zeros_like(d)
+    d_ends[:, :-1] = d[:, 1:]
+    for fn, src in ((lambda a, z, s: oracle.eligibility_traces(a, z, 0.99, 0.95, s), x["x"]),
+                    (oracle.episodic_prefix_sum, x["x"]), (oracle.episodic_prefix_sum, xi["x"])):
+        starts = fn(src, d, True)
+        np.testing.assert_array_equal(starts, fn(src, d_ends, False))
+        d0 = d.copy()
+        d0[:, 0] = 1 - d0[:, 0]
+        np.testing.assert_array_equal(starts, fn(src, d0, True))
+    # and the two readings differ wherever a flag sits inside a row
+    assert not np.array_equal(oracle.episodic_prefix_sum(x["x"], d, True), oracle.episodic_prefix_sum(x["x"], d))
 
 
 # --------------------------------------------------------------------------
