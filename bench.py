@@ -71,7 +71,10 @@ EXTRA_CALLS = {
     "gae_with_returns": (["rewards", "values", "terminateds"], ["advantages", "returns"]),
     # the same pass on reduced-byte inputs: bf16 rewards and values, uint8 dones
     "gae_with_returns_bf16_u8": (["rewards", "values", "terminateds"], ["advantages", "returns"]),
+    # GAE on the time-major layout: every plane [seq_len, num_envs]
+    "gae_time_major": (["rewards", "values", "terminateds"], ["advantages"]),
 }
+TIME_MAJOR = {"gae_time_major"}
 PLANES = {**ESTIMATORS, **EXTRA_CALLS}
 # planes stored narrower than fp32 (element bytes); outputs stay fp32
 NARROW = {("gae_with_returns_bf16_u8", "rewards"): 2, ("gae_with_returns_bf16_u8", "values"): 2,
@@ -99,9 +102,10 @@ def host_inputs(seed: int = 0) -> dict:
     pf = W.trace_inputs(E, T, seed + 6, p_done=P_DONE)
     pi = W.prefix_inputs_i32(E, T, seed + 7, p_done=P_DONE)
     gr = W.gae_inputs(E, T, seed + 8, p_term=P_DONE)
+    gt = {k: np.ascontiguousarray(v.T) for k, v in W.gae_inputs(E, T, seed + 9, p_term=P_DONE).items()}
     return {"gae": g, "vtrace": v, "retrace": r, "lambda_returns": lr, "discounted_returns": dr,
             "eligibility_traces": et, "prefix_sum_f32": pf, "prefix_sum_i32": pi, "gae_with_returns": gr,
-            "gae_with_returns_bf16_u8": gr}
+            "gae_with_returns_bf16_u8": gr, "gae_time_major": gt}
 
 
 # ---------------------------------------------------------------------------
@@ -136,7 +140,7 @@ class BufferSet:
         if key in NARROW:  # the first plane-size elements of the narrow dtype
             dt = {2: torch.bfloat16, 1: torch.uint8}[NARROW[key]]
             return v.view(dt)[:plane].view(E_ENVS, T_STEPS)
-        v = v.view(E_ENVS, T_STEPS)
+        v = v.view(T_STEPS, E_ENVS) if key[0] in TIME_MAJOR else v.view(E_ENVS, T_STEPS)
         return v.view(torch.int32) if key in INT_PLANES else v
 
     def fill_from_host(self, host):
@@ -185,6 +189,10 @@ class BufferSet:
             k = "gae_with_returns_bf16_u8"
             c[k] = lambda: R.rlscan_gae_typed(t[k, "rewards"], t[k, "values"], t[k, "terminateds"], None, None, None,
                                               t[k, "advantages"], t[k, "returns"], GAMMA, LAMBDA)
+        if "gae_time_major" in self.estimators:
+            k = "gae_time_major"
+            c[k] = lambda: R.rlscan_gae(t[k, "rewards"], t[k, "values"], t[k, "terminateds"], None, None, None,
+                                        t[k, "advantages"], GAMMA, LAMBDA, time_major=True)
         if "prefix_sum_i32" in self.estimators:
             c["prefix_sum_i32"] = lambda: R.rlscan_episodic_prefix_sum(
                 t["prefix_sum_i32", "x"], t["prefix_sum_i32", "dones"], t["prefix_sum_i32", "out"])

@@ -268,6 +268,70 @@ RLSCAN_API int rlscan_gae_noalloc(const float *rewards, const float *values, con
                                   float gamma, float lambda_, cudaStream_t stream);
 
 /*
+ * Layout and episode-boundary options (the _ex entry points).
+ *
+ * Each estimator above has an _ex twin that takes one more argument,
+ * `options`, an OR of the bits below, placed just before `ws`; all other
+ * arguments mean what they mean above, and options == 0 is exactly the plain
+ * call (the plain names are wrappers that pass 0).
+ *
+ *   RLSCAN_OPT_TIME_MAJOR: every [E, T] array (inputs and outputs) is
+ *     instead [T, E], E (num_envs) fastest: element (e, t) is at index
+ *     t*E + e, the rollout-buffer layout of vectorised environments that write
+ *     one row of E per step.  last_values stays [E].  Rows are still scanned
+ *     independently; a time-major call needs no workspace (ws may be NULL)
+ *     and reads and writes each element once with coalesced accesses along E.
+ *     rlscan_retrace_ex takes it with A == 1 only (RLSCAN_ERR_UNSUPPORTED
+ *     otherwise).
+ *   RLSCAN_OPT_DONE_STARTS_EPISODE (forward estimators only: eligibility
+ *     traces and the episodic prefix sum): dones[e, t] != 0 marks step t as
+ *     the FIRST step of a new episode (the reset-flag convention: a "first" or
+ *     "is_init" mask), instead of the default, where it marks t as the last
+ *     step so that t+1 starts afresh.  With it, y_t = x_t where dones[t] != 0
+ *     and the recurrence continues elsewhere.  Passing it to a backward
+ *     estimator is RLSCAN_ERR_INVALID_ARG.
+ * Unknown bits are RLSCAN_ERR_INVALID_ARG.
+ */
+#define RLSCAN_OPT_TIME_MAJOR 1u
+#define RLSCAN_OPT_DONE_STARTS_EPISODE 2u
+
+RLSCAN_API int rlscan_gae_ex(const float *rewards, const float *values, const float *terminateds,
+                             const float *truncateds, const float *bootstrap_values, const float *last_values,
+                             float *advantages, int64_t E, int64_t T, float gamma, float lambda_,
+                             unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream);
+RLSCAN_API int rlscan_gae_with_returns_ex(const float *rewards, const float *values, const float *terminateds,
+                                          const float *truncateds, const float *bootstrap_values,
+                                          const float *last_values, float *advantages, float *returns, int64_t E,
+                                          int64_t T, float gamma, float lambda_, unsigned options, void *ws,
+                                          size_t ws_bytes, cudaStream_t stream);
+RLSCAN_API int rlscan_vtrace_ex(const float *log_rhos, const float *rewards, const float *values,
+                                const float *terminateds, const float *truncateds, const float *bootstrap_values,
+                                const float *last_values, float *vs, float *pg_advantages, int64_t E, int64_t T,
+                                float gamma, float lambda_, float rho_bar, float c_bar, unsigned options,
+                                void *ws, size_t ws_bytes, cudaStream_t stream);
+RLSCAN_API int rlscan_retrace_ex(const float *rewards, const float *q_values, const float *next_q_values_all,
+                                 const float *next_target_probs, const float *log_rhos, const float *terminateds,
+                                 const float *truncateds, float *q_ret, int64_t E, int64_t T, int64_t A,
+                                 float gamma, float lambda_, float c_bar, unsigned options, void *ws,
+                                 size_t ws_bytes, cudaStream_t stream);
+RLSCAN_API int rlscan_lambda_returns_ex(const float *rewards, const float *values, const float *terminateds,
+                                        const float *truncateds, const float *bootstrap_values,
+                                        const float *last_values, float *returns, int64_t E, int64_t T,
+                                        float gamma, float lambda_, unsigned options, void *ws, size_t ws_bytes,
+                                        cudaStream_t stream);
+RLSCAN_API int rlscan_discounted_returns_ex(const float *rewards, const float *terminateds,
+                                            const float *truncateds, const float *bootstrap_values,
+                                            const float *last_values, float *returns, int64_t E, int64_t T,
+                                            float gamma, unsigned options, void *ws, size_t ws_bytes,
+                                            cudaStream_t stream);
+RLSCAN_API int rlscan_eligibility_traces_ex(const float *x, const float *dones, float *traces, int64_t E,
+                                            int64_t T, float gamma, float lambda_, unsigned options, void *ws,
+                                            size_t ws_bytes, cudaStream_t stream);
+RLSCAN_API int rlscan_episodic_prefix_sum_ex(const void *x, int dtype, const float *dones, void *out, int64_t E,
+                                             int64_t T, unsigned options, void *ws, size_t ws_bytes,
+                                             cudaStream_t stream);
+
+/*
  * Workspace size in bytes that any entry point above needs for an [E, T]
  * problem (any A); 0 if no call of that shape needs one.  Negative or
  * overflowing shapes return 0 and the compute call then rejects them.

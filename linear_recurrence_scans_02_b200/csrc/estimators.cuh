@@ -13,7 +13,8 @@
 //   - last step of a row with no flag: bootstrap with last_values[row] (0 if
 //     absent) folded into b_t, and a_t = 0 so rows never mix;
 //   - forward estimators reset after a done: a_t = 0 when t == 0 or
-//     dones[t-1] != 0.
+//     dones[t-1] != 0 (or, with reset_on_flag, dones[t] != 0: the flag marks
+//     the first step of an episode).
 #pragma once
 
 #include "scan_core.cuh"
@@ -30,30 +31,6 @@ __device__ __forceinline__ StepFlags step_flags(F te, F tr) {
     f.trn = kTrunc && (tr != F(0)) && !f.term;
     f.cont = !f.term && !f.trn;
     return f;
-}
-
-// Halo elements.  Each thread's last element needs the next element of a
-// plane (backward estimators) or its first element the previous one (forward
-// estimators); inside a warp that value comes from the neighbouring lane by a
-// shuffle, and the warp's edge lane loads it directly.  The edge load is
-// issued before the plane's own loads (fetch_*), so it is in flight with them
-// instead of waiting behind the shuffle that needs the loaded data.
-template <int V>
-__device__ __forceinline__ float fetch_next(const float *__restrict__ p, long long i0, long long n, int lane) {
-    return lane == 31 ? load_one(p, i0 + V, n) : 0.0f;
-}
-template <int V>
-__device__ __forceinline__ float next_halo(const float (&own)[V], float fetched, int lane) {
-    const float h = __shfl_down_sync(kFullMask, own[0], 1);
-    return lane == 31 ? fetched : h;
-}
-__device__ __forceinline__ float fetch_prev(const float *__restrict__ p, long long i0, long long n, int lane) {
-    return lane == 0 ? load_one(p, i0 - 1, n) : 0.0f;
-}
-template <int V>
-__device__ __forceinline__ float prev_halo(const float (&own)[V], float fetched, int lane) {
-    const float h = __shfl_up_sync(kFullMask, own[V - 1], 1);
-    return lane == 0 ? fetched : h;
 }
 
 // L2 prefetch of one tile of up to six input planes, one plane per thread
@@ -116,19 +93,18 @@ struct GaeEstT {
         default: break;
         }
     }
-    template <int NT, int V>
-    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
-        const bool vec = g.vec_ok && i0 + V <= g.n;
-        const float h_v_next = lane == 31 ? load_one_widen(P.values, i0 + V, g.n) : 0.0f;
-        load_plane_widen<V>(P.rewards, i0, g.n, vec, S.r);
-        load_plane_widen<V>(P.values, i0, g.n, vec, S.v);
-        load_flags<V>(P.terminateds, i0, g.n, vec, S.te);
-        load_flags<V>(P.truncateds, i0, g.n, vec, S.tr);
-        S.v_next = next_halo<V>(S.v, h_v_next, lane);
+        const float h_v_next = pos.fetch_next(P.values);
+        pos.load_widen(P.rewards, S.r);
+        pos.load_widen(P.values, S.v);
+        pos.load_flag(P.terminateds, S.te);
+        pos.load_flag(P.truncateds, S.tr);
+        S.v_next = pos.next(S.v, h_v_next);
     }
-    template <int V, bool kTrunc, bool kFast>
-    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kTrunc, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
         const float gl = P.gamma * P.lambda_;
@@ -139,7 +115,7 @@ struct GaeEstT {
                 const bool rowend = elem_row_end<kFast, V>(rm, k);
                 float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
                 if (rowend) nv = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
-                const float boot = f.cont ? nv : (f.trn ? load_one_widen(P.bootstrap_values, i0 + k, g.n) : 0.0f);
+                const float boot = f.cont ? nv : (f.trn ? pos.one(P.bootstrap_values, k) : 0.0f);
                 a[k] = (f.cont && !rowend) ? gl : 0.0f;
                 b[k] = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
             } else {
@@ -151,15 +127,15 @@ struct GaeEstT {
     // uniform branches per thread: without truncations the truncation logic
     // is compiled out of the per-element loop, and on the fast path (all V
     // elements present, V divides T) so are the per-element row tests
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if (P.truncateds != nullptr) {
-            if (rm.fast) coeffs_impl<V, true, true>(P, g, i0, rm, S, a, b);
-            else coeffs_impl<V, true, false>(P, g, i0, rm, S, a, b);
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
-            if (rm.fast) coeffs_impl<V, false, true>(P, g, i0, rm, S, a, b);
-            else coeffs_impl<V, false, false>(P, g, i0, rm, S, a, b);
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, pos, rm, S, a, b);
         }
     }
     template <int V>
@@ -167,12 +143,11 @@ struct GaeEstT {
         S.out[k] = x;
         if constexpr (kWithReturns) S.ret[k] = x + S.v[k];
     }
-    template <int V>
-    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        const bool vec = g.vec_ok && i0 + V <= g.n;
-        store_plane<V>(P.advantages, i0, g.n, vec, S.out);
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.advantages, S.out);
         if constexpr (kWithReturns) {
-            if (P.returns != nullptr) store_plane<V>(P.returns, i0, g.n, vec, S.ret);
+            if (P.returns != nullptr) pos.store(P.returns, S.ret);
         }
     }
 };
@@ -202,19 +177,18 @@ struct LambdaReturnsEst {
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds);
     }
-    template <int NT, int V>
-    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
-        const bool vec = g.vec_ok && i0 + V <= g.n;
-        const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
-        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
-        load_plane<V>(P.values, i0, g.n, vec, S.v);
-        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
-        S.v_next = next_halo<V>(S.v, h_v_next, lane);
+        const float h_v_next = pos.fetch_next(P.values);
+        pos.load(P.rewards, S.r);
+        pos.load(P.values, S.v);
+        pos.load(P.terminateds, S.te);
+        pos.load(P.truncateds, S.tr);
+        S.v_next = pos.next(S.v, h_v_next);
     }
-    template <int V, bool kTrunc, bool kFast>
-    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kTrunc, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
         const float gl = P.gamma * P.lambda_;
@@ -229,7 +203,7 @@ struct LambdaReturnsEst {
                 // row end (G_{t+1} = V_{t+1} = last value), the bootstrap value at a
                 // truncation and 0 at a termination
                 float boot = 0.0f;
-                if (f.trn) boot = __ldcg(P.bootstrap_values + i0 + k);
+                if (f.trn) boot = pos.one(P.bootstrap_values, k);
                 if (f.cont) {
                     if (rowend) {
                         const float lv = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
@@ -249,24 +223,24 @@ struct LambdaReturnsEst {
     // uniform branches per thread: without truncations the truncation logic
     // is compiled out of the per-element loop, and on the fast path (all V
     // elements present, V divides T) so are the per-element row tests
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if (P.truncateds != nullptr) {
-            if (rm.fast) coeffs_impl<V, true, true>(P, g, i0, rm, S, a, b);
-            else coeffs_impl<V, true, false>(P, g, i0, rm, S, a, b);
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
-            if (rm.fast) coeffs_impl<V, false, true>(P, g, i0, rm, S, a, b);
-            else coeffs_impl<V, false, false>(P, g, i0, rm, S, a, b);
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, pos, rm, S, a, b);
         }
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
-    template <int V>
-    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.returns, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.returns, S.out);
     }
 };
 
@@ -289,16 +263,15 @@ struct ReturnsEst {
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.rewards, P.terminateds, P.truncateds);
     }
-    template <int NT, int V>
-    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int,
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
-        const bool vec = g.vec_ok && i0 + V <= g.n;
-        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
-        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
+        pos.load(P.rewards, S.r);
+        pos.load(P.terminateds, S.te);
+        pos.load(P.truncateds, S.tr);
     }
-    template <int V, bool kTrunc, bool kFast>
-    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kTrunc, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
 #pragma unroll
@@ -310,7 +283,7 @@ struct ReturnsEst {
                 // last value at a row end, the bootstrap value at a
                 // truncation, nothing otherwise (the scan carries R_{t+1})
                 float boot = 0.0f;
-                if (f.trn) boot = __ldcg(P.bootstrap_values + i0 + k);
+                if (f.trn) boot = pos.one(P.bootstrap_values, k);
                 if (f.cont && rowend) boot = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
                 a[k] = (f.cont && !rowend) ? P.gamma : 0.0f;
                 b[k] = fmaf(P.gamma, boot, S.r[k]);
@@ -323,24 +296,24 @@ struct ReturnsEst {
     // uniform branches per thread: without truncations the truncation logic
     // is compiled out of the per-element loop, and on the fast path (all V
     // elements present, V divides T) so are the per-element row tests
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if (P.truncateds != nullptr) {
-            if (rm.fast) coeffs_impl<V, true, true>(P, g, i0, rm, S, a, b);
-            else coeffs_impl<V, true, false>(P, g, i0, rm, S, a, b);
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
-            if (rm.fast) coeffs_impl<V, false, true>(P, g, i0, rm, S, a, b);
-            else coeffs_impl<V, false, false>(P, g, i0, rm, S, a, b);
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, pos, rm, S, a, b);
         }
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
-    template <int V>
-    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.returns, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.returns, S.out);
     }
 };
 
@@ -368,20 +341,19 @@ struct VtraceEst {
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds);
     }
-    template <int NT, int V>
-    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
-        const bool vec = g.vec_ok && i0 + V <= g.n;
-        const float h_v_next = fetch_next<V>(P.values, i0, g.n, lane);
-        load_plane<V>(P.log_rhos, i0, g.n, vec, S.lr);
-        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
-        load_plane<V>(P.values, i0, g.n, vec, S.v);
-        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
-        S.v_next = next_halo<V>(S.v, h_v_next, lane);
+        const float h_v_next = pos.fetch_next(P.values);
+        pos.load(P.log_rhos, S.lr);
+        pos.load(P.rewards, S.r);
+        pos.load(P.values, S.v);
+        pos.load(P.terminateds, S.te);
+        pos.load(P.truncateds, S.tr);
+        S.v_next = pos.next(S.v, h_v_next);
     }
-    template <int V, bool kTrunc, bool kFast>
-    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kTrunc, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
         S.chained = 0u;
@@ -398,7 +370,7 @@ struct VtraceEst {
                     boot = rowend ? row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows)
                                   : ((k + 1 < V) ? S.v[k + 1] : S.v_next);
                 } else {
-                    boot = f.trn ? __ldcg(P.bootstrap_values + i0 + k) : 0.0f;
+                    boot = f.trn ? pos.one(P.bootstrap_values, k) : 0.0f;
                 }
                 a[k] = (f.cont && !rowend) ? P.gamma * c : 0.0f;
                 b[k] = rho * (fmaf(P.gamma, boot, S.r[k]) - S.v[k]);
@@ -418,15 +390,15 @@ struct VtraceEst {
     // uniform branches per thread: without truncations the truncation logic
     // is compiled out of the per-element loop, and on the fast path (all V
     // elements present, V divides T) so are the per-element row tests
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if (P.truncateds != nullptr) {
-            if (rm.fast) coeffs_impl<V, true, true>(P, g, i0, rm, S, a, b);
-            else coeffs_impl<V, true, false>(P, g, i0, rm, S, a, b);
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
-            if (rm.fast) coeffs_impl<V, false, true>(P, g, i0, rm, S, a, b);
-            else coeffs_impl<V, false, false>(P, g, i0, rm, S, a, b);
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, pos, rm, S, a, b);
         }
     }
     template <int V>
@@ -435,10 +407,10 @@ struct VtraceEst {
         S.vs[k] = S.v[k] + x;
         S.pg[k] = ((S.chained >> k) & 1u) ? fmaf(S.rho[k] * P.gamma, x_next, b_k) : b_k;
     }
-    template <int V>
-    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.vs, i0, g.n, g.vec_ok && i0 + V <= g.n, S.vs);
-        store_plane<V>(P.pg_advantages, i0, g.n, g.vec_ok && i0 + V <= g.n, S.pg);
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.vs, S.vs);
+        pos.store(P.pg_advantages, S.pg);
     }
 };
 
@@ -539,25 +511,26 @@ struct RetraceEst {
         }
     }
 
-    template <int NT, int V>
-    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *smem) {
-        const bool vec = g.vec_ok && i0 + V <= g.n;
-        const float h_lr_next = fetch_next<V>(P.log_rhos, i0, g.n, lane);
-        load_plane<V>(P.rewards, i0, g.n, vec, S.r);
-        load_plane<V>(P.q_values, i0, g.n, vec, S.q);
-        load_plane<V>(P.log_rhos, i0, g.n, vec, S.lr);
-        load_plane<V>(P.terminateds, i0, g.n, vec, S.te);
-        load_plane<V>(P.truncateds, i0, g.n, vec, S.tr);
-        S.lr_next = next_halo<V>(S.lr, h_lr_next, lane);
+        const float h_lr_next = pos.fetch_next(P.log_rhos);
+        pos.load(P.rewards, S.r);
+        pos.load(P.q_values, S.q);
+        pos.load(P.log_rhos, S.lr);
+        pos.load(P.terminateds, S.te);
+        pos.load(P.truncateds, S.tr);
+        S.lr_next = pos.next(S.lr, h_lr_next);
         if constexpr (kMulti) {
-            stage_expected_values<NT, V>(P, g, i0, S, smem);
+            // per-action rows are staged for row-major tiles only (time-major
+            // calls with more than one action are rejected on the host)
+            stage_expected_values<NT, V>(P, g, pos.index(0), S, smem);
         } else {
-            load_plane<V>(P.next_q_values_all, i0, g.n, vec, S.vnext);
+            pos.load(P.next_q_values_all, S.vnext);
         }
     }
-    template <int V, bool kFast>
-    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
 #pragma unroll
@@ -579,20 +552,20 @@ struct RetraceEst {
             }
         }
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V],
                                                   float (&b)[V]) {
-        if (rm.fast) coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
-        else coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+        if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = S.q[k] + x;
     }
-    template <int V>
-    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.q_ret, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.q_ret, S.out);
     }
 };
 
@@ -609,7 +582,8 @@ struct ForwardF32Est {
     struct Params {
         const float *x, *dones;
         float *out;
-        float decay; // gamma lambda, or 1
+        float decay;       // gamma lambda, or 1
+        int reset_on_flag; // 0: dones[t-1] != 0 resets at t; 1: dones[t] != 0 resets at t
     };
     template <int V>
     struct State {
@@ -619,23 +593,22 @@ struct ForwardF32Est {
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.x, P.dones);
     }
-    template <int NT, int V>
-    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
-        const bool vec = g.vec_ok && i0 + V <= g.n;
-        const float h_d_prev = fetch_prev(P.dones, i0, g.n, lane);
-        load_plane<V>(P.x, i0, g.n, vec, S.x);
-        load_plane<V>(P.dones, i0, g.n, vec, S.d);
-        S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
+        const float h_d_prev = pos.fetch_prev(P.dones);
+        pos.load(P.x, S.x);
+        pos.load(P.dones, S.d);
+        S.d_prev = pos.prev(S.d, h_d_prev);
     }
-    template <int V, bool kFast>
-    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, long long i0,
+    template <int V, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S,
                                                   float (&a)[V], float (&b)[V]) {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
             if (elem_valid<kFast, V>(rm, k)) {
-                const float dp = (k > 0) ? S.d[k - 1] : S.d_prev;
+                const float dp = P.reset_on_flag ? S.d[k] : ((k > 0) ? S.d[k - 1] : S.d_prev);
                 a[k] = (elem_row_start<kFast, V>(rm, k) || dp != 0.0f) ? 0.0f : P.decay;
                 b[k] = S.x[k];
             } else {
@@ -644,20 +617,20 @@ struct ForwardF32Est {
             }
         }
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V],
                                                   float (&b)[V]) {
-        if (rm.fast) coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
-        else coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+        if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
         S.out[k] = x;
     }
-    template <int V>
-    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.out, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.out, S.out);
     }
 };
 using TracesEst = ForwardF32Est<0>;
@@ -672,6 +645,7 @@ struct PrefixI32Est {
         const int32_t *x;
         const float *dones;
         int32_t *out;
+        int reset_on_flag; // as ForwardF32Est
     };
     template <int V>
     struct State {
@@ -682,23 +656,22 @@ struct PrefixI32Est {
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.x, P.dones);
     }
-    template <int NT, int V>
-    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, long long i0, int lane,
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
-        const bool vec = g.vec_ok && i0 + V <= g.n;
-        const float h_d_prev = fetch_prev(P.dones, i0, g.n, lane);
-        load_plane<V>(P.x, i0, g.n, vec, S.x);
-        load_plane<V>(P.dones, i0, g.n, vec, S.d);
-        S.d_prev = prev_halo<V>(S.d, h_d_prev, lane);
+        const float h_d_prev = pos.fetch_prev(P.dones);
+        pos.load(P.x, S.x);
+        pos.load(P.dones, S.d);
+        S.d_prev = pos.prev(S.d, h_d_prev);
     }
-    template <int V, bool kFast>
-    static __device__ __forceinline__ void coeffs_impl(const Params &, const Geometry &g, long long i0,
+    template <int V, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S,
                                                   uint32_t (&a)[V], int32_t (&b)[V]) {
 #pragma unroll
         for (int k = 0; k < V; ++k) {
             if (elem_valid<kFast, V>(rm, k)) {
-                const float dp = (k > 0) ? S.d[k - 1] : S.d_prev;
+                const float dp = P.reset_on_flag ? S.d[k] : ((k > 0) ? S.d[k - 1] : S.d_prev);
                 a[k] = (elem_row_start<kFast, V>(rm, k) || dp != 0.0f) ? 0u : 1u;
                 b[k] = S.x[k];
             } else {
@@ -707,20 +680,20 @@ struct PrefixI32Est {
             }
         }
     }
-    template <int V>
-    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, long long i0,
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, uint32_t (&a)[V],
                                                   int32_t (&b)[V]) {
-        if (rm.fast) coeffs_impl<V, true>(P, g, i0, rm, S, a, b);
-        else coeffs_impl<V, false>(P, g, i0, rm, S, a, b);
+        if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }
     template <int V>
     static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, int32_t x, int32_t, int32_t) {
         S.out[k] = x;
     }
-    template <int V>
-    static __device__ __forceinline__ void store(const Params &P, const Geometry &g, long long i0, State<V> &S) {
-        store_plane<V>(P.out, i0, g.n, g.vec_ok && i0 + V <= g.n, S.out);
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.out, S.out);
     }
 };
 

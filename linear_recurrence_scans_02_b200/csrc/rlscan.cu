@@ -10,6 +10,7 @@
 #include <cmath>
 #include <mutex>
 #include <cstdarg>
+#include <climits>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -326,6 +327,46 @@ int run_multi(const char *name, const typename Est::Params &P, long long E, long
 
 size_t plane_bytes(long long E, long long T) { return (size_t)(E * T) * sizeof(float); }
 
+// Option bits of the _ex entry points; `forward` estimators also take
+// RLSCAN_OPT_DONE_STARTS_EPISODE.
+int check_options(unsigned options, bool forward) {
+    const unsigned known = RLSCAN_OPT_TIME_MAJOR | (forward ? RLSCAN_OPT_DONE_STARTS_EPISODE : 0u);
+    if (options & ~known)
+        return fail(RLSCAN_ERR_INVALID_ARG, "unknown or inapplicable option bits 0x%x", options & ~known);
+    return RLSCAN_OK;
+}
+
+// Time-major [T, E] launch: one block per 32 envs, 16 warps x 8 timesteps per
+// segment; no workspace.
+constexpr int kTmWarps = 16;
+constexpr int kTmV = 8;
+
+template <class Est>
+int run_time_major(const char *name, const typename Est::Params &P, long long E, long long T, cudaStream_t stream) {
+    if (E > (long long)INT_MAX / (kTmV + 1))
+        return fail(RLSCAN_ERR_UNSUPPORTED, "%s: the time-major layout takes E <= %d", name, INT_MAX / (kTmV + 1));
+    Geometry g;
+    g.n = E * T;
+    g.seq_len = T;
+    g.rows = E;
+    g.ntiles = ceil_div(E, 32);
+    g.t_shift = pow2_shift(T);
+    g.vec_ok = 0;
+    g.scan_lanes = 32;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g.ntiles);
+    cfg.blockDim = dim3(kTmWarps * 32);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, kTmWarps, kTmV>, P, g);
+    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
+    return ok();
+}
+
 } // namespace
 } // namespace rlscan
 
@@ -367,9 +408,10 @@ using namespace rlscan;
 
 extern "C" {
 
-int rlscan_gae(const float *rewards, const float *values, const float *terminateds, const float *truncateds,
+int rlscan_gae_ex(const float *rewards, const float *values, const float *terminateds, const float *truncateds,
                const float *bootstrap_values, const float *last_values, float *advantages, int64_t E, int64_t T,
-               float gamma, float lambda_, void *ws, size_t ws_bytes, cudaStream_t stream) {
+               float gamma, float lambda_, unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, false));
     RLSCAN_TRY(check_shape(E, T));
     RLSCAN_TRY(check_scalar(gamma, "gamma"));
     RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
@@ -386,14 +428,22 @@ int rlscan_gae(const float *rewards, const float *values, const float *terminate
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
     GaeEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                      last_values, advantages, nullptr, gamma, lambda_};
+    if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<GaeEst>("rlscan_gae", P, E, T, stream);
     return run<GaeEst>("rlscan_gae", P, E, T, 1, ws, ws_bytes, stream,
                        aligned16({rewards, values, terminateds, truncateds, advantages}));
 }
 
-int rlscan_gae_with_returns(const float *rewards, const float *values, const float *terminateds,
+int rlscan_gae(const float *rewards, const float *values, const float *terminateds, const float *truncateds,
+               const float *bootstrap_values, const float *last_values, float *advantages, int64_t E, int64_t T,
+               float gamma, float lambda_, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_gae_ex(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages, E, T, gamma, lambda_, 0u, ws, ws_bytes, stream);
+}
+
+int rlscan_gae_with_returns_ex(const float *rewards, const float *values, const float *terminateds,
                             const float *truncateds, const float *bootstrap_values, const float *last_values,
                             float *advantages, float *returns, int64_t E, int64_t T, float gamma, float lambda_,
-                            void *ws, size_t ws_bytes, cudaStream_t stream) {
+                            unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, false));
     RLSCAN_TRY(check_shape(E, T));
     RLSCAN_TRY(check_scalar(gamma, "gamma"));
     RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
@@ -411,8 +461,17 @@ int rlscan_gae_with_returns(const float *rewards, const float *values, const flo
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 2));
     GaeReturnsEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                             last_values, advantages, returns, gamma, lambda_};
+    if (options & RLSCAN_OPT_TIME_MAJOR)
+        return run_time_major<GaeReturnsEst>("rlscan_gae_with_returns", P, E, T, stream);
     return run<GaeReturnsEst>("rlscan_gae_with_returns", P, E, T, 1, ws, ws_bytes, stream,
                               aligned16({rewards, values, terminateds, truncateds, advantages, returns}));
+}
+
+int rlscan_gae_with_returns(const float *rewards, const float *values, const float *terminateds,
+                            const float *truncateds, const float *bootstrap_values, const float *last_values,
+                            float *advantages, float *returns, int64_t E, int64_t T, float gamma, float lambda_,
+                            void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_gae_with_returns_ex(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages, returns, E, T, gamma, lambda_, 0u, ws, ws_bytes, stream);
 }
 
 int rlscan_gae_typed(const void *rewards, const void *values, const void *terminateds, const void *truncateds,
@@ -466,10 +525,11 @@ int rlscan_gae_typed(const void *rewards, const void *values, const void *termin
 #undef RLSCAN_GAE_TYPED
 }
 
-int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
+int rlscan_vtrace_ex(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
                   const float *truncateds, const float *bootstrap_values, const float *last_values, float *vs,
                   float *pg_advantages, int64_t E, int64_t T, float gamma, float lambda_, float rho_bar,
-                  float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                  float c_bar, unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, false));
     RLSCAN_TRY(check_shape(E, T));
     RLSCAN_TRY(check_scalar(gamma, "gamma"));
     RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
@@ -490,14 +550,23 @@ int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *valu
     RLSCAN_TRY(check_aliasing(ins, 7, outs, 2));
     VtraceEst::Params P{log_rhos, rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                         last_values, vs, pg_advantages, gamma, lambda_, rho_bar, c_bar};
+    if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<VtraceEst>("rlscan_vtrace", P, E, T, stream);
     return run<VtraceEst>("rlscan_vtrace", P, E, T, 1, ws, ws_bytes, stream,
                           aligned16({log_rhos, rewards, values, terminateds, truncateds, vs, pg_advantages}));
 }
 
-int rlscan_retrace(const float *rewards, const float *q_values, const float *next_q_values_all,
+int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
+                  const float *truncateds, const float *bootstrap_values, const float *last_values, float *vs,
+                  float *pg_advantages, int64_t E, int64_t T, float gamma, float lambda_, float rho_bar,
+                  float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_vtrace_ex(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values, vs, pg_advantages, E, T, gamma, lambda_, rho_bar, c_bar, 0u, ws, ws_bytes, stream);
+}
+
+int rlscan_retrace_ex(const float *rewards, const float *q_values, const float *next_q_values_all,
                    const float *next_target_probs, const float *log_rhos, const float *terminateds,
                    const float *truncateds, float *q_ret, int64_t E, int64_t T, int64_t A, float gamma,
-                   float lambda_, float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                   float lambda_, float c_bar, unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, false));
     if (A < 1) return fail(RLSCAN_ERR_INVALID_ARG, "A must be >= 1 (got %lld)", (long long)A);
     if (A > RLSCAN_MAX_ACTIONS)
         return fail(RLSCAN_ERR_UNSUPPORTED, "A=%lld exceeds RLSCAN_MAX_ACTIONS=%d", (long long)A, RLSCAN_MAX_ACTIONS);
@@ -525,20 +594,31 @@ int rlscan_retrace(const float *rewards, const float *q_values, const float *nex
     if (A == 1) {
         RetraceEst<false>::Params P{rewards, q_values, next_q_values_all, nullptr, log_rhos, terminateds,
                                     truncateds, q_ret, 1, gamma, lambda_, c_bar, 0u};
+        if (options & RLSCAN_OPT_TIME_MAJOR)
+            return run_time_major<RetraceEst<false>>("rlscan_retrace", P, E, T, stream);
         return run<RetraceEst<false>>("rlscan_retrace", P, E, T, 1, ws, ws_bytes, stream,
                                       aligned16({rewards, q_values, next_q_values_all, log_rhos, terminateds,
                                                  truncateds, q_ret}));
     }
+    if (options & RLSCAN_OPT_TIME_MAJOR)
+        return fail(RLSCAN_ERR_UNSUPPORTED, "rlscan_retrace: the time-major layout takes A == 1 only");
     RetraceEst<true>::Params P{rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds,
                                truncateds, q_ret, A, gamma, lambda_, c_bar, 1u << 24};
     return run_multi<RetraceEst<true>>("rlscan_retrace", P, E, T, A, ws, ws_bytes, stream,
                                        aligned16({rewards, q_values, log_rhos, terminateds, truncateds, q_ret}));
 }
 
-int rlscan_lambda_returns(const float *rewards, const float *values, const float *terminateds,
+int rlscan_retrace(const float *rewards, const float *q_values, const float *next_q_values_all,
+                   const float *next_target_probs, const float *log_rhos, const float *terminateds,
+                   const float *truncateds, float *q_ret, int64_t E, int64_t T, int64_t A, float gamma,
+                   float lambda_, float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_retrace_ex(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds, truncateds, q_ret, E, T, A, gamma, lambda_, c_bar, 0u, ws, ws_bytes, stream);
+}
+
+int rlscan_lambda_returns_ex(const float *rewards, const float *values, const float *terminateds,
                           const float *truncateds, const float *bootstrap_values, const float *last_values,
-                          float *returns, int64_t E, int64_t T, float gamma, float lambda_, void *ws,
-                          size_t ws_bytes, cudaStream_t stream) {
+                          float *returns, int64_t E, int64_t T, float gamma, float lambda_, unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, false));
     RLSCAN_TRY(check_shape(E, T));
     RLSCAN_TRY(check_scalar(gamma, "gamma"));
     RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
@@ -555,13 +635,23 @@ int rlscan_lambda_returns(const float *rewards, const float *values, const float
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
     LambdaReturnsEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                                last_values, returns, gamma, lambda_};
+    if (options & RLSCAN_OPT_TIME_MAJOR)
+        return run_time_major<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, stream);
     return run<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, 1, ws, ws_bytes, stream,
                                  aligned16({rewards, values, terminateds, truncateds, returns}));
 }
 
-int rlscan_discounted_returns(const float *rewards, const float *terminateds, const float *truncateds,
+int rlscan_lambda_returns(const float *rewards, const float *values, const float *terminateds,
+                          const float *truncateds, const float *bootstrap_values, const float *last_values,
+                          float *returns, int64_t E, int64_t T, float gamma, float lambda_, void *ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_lambda_returns_ex(rewards, values, terminateds, truncateds, bootstrap_values, last_values, returns, E, T, gamma, lambda_, 0u, ws, ws_bytes, stream);
+}
+
+int rlscan_discounted_returns_ex(const float *rewards, const float *terminateds, const float *truncateds,
                               const float *bootstrap_values, const float *last_values, float *returns, int64_t E,
-                              int64_t T, float gamma, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                              int64_t T, float gamma, unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, false));
     RLSCAN_TRY(check_shape(E, T));
     RLSCAN_TRY(check_scalar(gamma, "gamma"));
     if (E == 0 || T == 0) return ok();
@@ -575,12 +665,21 @@ int rlscan_discounted_returns(const float *rewards, const float *terminateds, co
     RLSCAN_TRY(check_aliasing(ins, 5, outs, 1));
     ReturnsEst::Params P{rewards, terminateds, truncateds, truncateds ? bootstrap_values : nullptr, last_values,
                          returns, gamma};
+    if (options & RLSCAN_OPT_TIME_MAJOR)
+        return run_time_major<ReturnsEst>("rlscan_discounted_returns", P, E, T, stream);
     return run<ReturnsEst>("rlscan_discounted_returns", P, E, T, 1, ws, ws_bytes, stream,
                            aligned16({rewards, terminateds, truncateds, returns}));
 }
 
-int rlscan_eligibility_traces(const float *x, const float *dones, float *traces, int64_t E, int64_t T, float gamma,
-                              float lambda_, void *ws, size_t ws_bytes, cudaStream_t stream) {
+int rlscan_discounted_returns(const float *rewards, const float *terminateds, const float *truncateds,
+                              const float *bootstrap_values, const float *last_values, float *returns, int64_t E,
+                              int64_t T, float gamma, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_discounted_returns_ex(rewards, terminateds, truncateds, bootstrap_values, last_values, returns, E, T, gamma, 0u, ws, ws_bytes, stream);
+}
+
+int rlscan_eligibility_traces_ex(const float *x, const float *dones, float *traces, int64_t E, int64_t T, float gamma,
+                              float lambda_, unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, true));
     RLSCAN_TRY(check_shape(E, T));
     RLSCAN_TRY(check_scalar(gamma, "gamma"));
     RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
@@ -591,13 +690,21 @@ int rlscan_eligibility_traces(const float *x, const float *dones, float *traces,
     const Span ins[] = {{x, pb, "x"}, {dones, pb, "dones"}};
     const Span outs[] = {{traces, pb, "traces"}};
     RLSCAN_TRY(check_aliasing(ins, 2, outs, 1));
-    TracesEst::Params P{x, dones, traces, gamma * lambda_};
+    TracesEst::Params P{x, dones, traces, gamma * lambda_, (options & RLSCAN_OPT_DONE_STARTS_EPISODE) ? 1 : 0};
+    if (options & RLSCAN_OPT_TIME_MAJOR)
+        return run_time_major<TracesEst>("rlscan_eligibility_traces", P, E, T, stream);
     return run<TracesEst>("rlscan_eligibility_traces", P, E, T, 1, ws, ws_bytes, stream,
                           aligned16({x, dones, traces}));
 }
 
-int rlscan_episodic_prefix_sum(const void *x, int dtype, const float *dones, void *out, int64_t E, int64_t T,
-                               void *ws, size_t ws_bytes, cudaStream_t stream) {
+int rlscan_eligibility_traces(const float *x, const float *dones, float *traces, int64_t E, int64_t T, float gamma,
+                              float lambda_, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_eligibility_traces_ex(x, dones, traces, E, T, gamma, lambda_, 0u, ws, ws_bytes, stream);
+}
+
+int rlscan_episodic_prefix_sum_ex(const void *x, int dtype, const float *dones, void *out, int64_t E, int64_t T,
+                               unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, true));
     if (dtype != RLSCAN_F32 && dtype != RLSCAN_I32) return fail(RLSCAN_ERR_UNSUPPORTED, "unknown dtype %d", dtype);
     RLSCAN_TRY(check_shape(E, T));
     if (E == 0 || T == 0) return ok();
@@ -608,13 +715,22 @@ int rlscan_episodic_prefix_sum(const void *x, int dtype, const float *dones, voi
     const Span outs[] = {{out, pb, "out"}};
     RLSCAN_TRY(check_aliasing(ins, 2, outs, 1));
     if (dtype == RLSCAN_F32) {
-        PrefixF32Est::Params P{static_cast<const float *>(x), dones, static_cast<float *>(out), 1.0f};
+        PrefixF32Est::Params P{static_cast<const float *>(x), dones, static_cast<float *>(out), 1.0f, (options & RLSCAN_OPT_DONE_STARTS_EPISODE) ? 1 : 0};
+        if (options & RLSCAN_OPT_TIME_MAJOR)
+            return run_time_major<PrefixF32Est>("rlscan_episodic_prefix_sum", P, E, T, stream);
         return run<PrefixF32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream,
                                  aligned16({x, dones, out}));
     }
-    PrefixI32Est::Params P{static_cast<const int32_t *>(x), dones, static_cast<int32_t *>(out)};
+    PrefixI32Est::Params P{static_cast<const int32_t *>(x), dones, static_cast<int32_t *>(out), (options & RLSCAN_OPT_DONE_STARTS_EPISODE) ? 1 : 0};
+    if (options & RLSCAN_OPT_TIME_MAJOR)
+        return run_time_major<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, stream);
     return run<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, 1, ws, ws_bytes, stream,
                              aligned16({x, dones, out}));
+}
+
+int rlscan_episodic_prefix_sum(const void *x, int dtype, const float *dones, void *out, int64_t E, int64_t T,
+                               void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_episodic_prefix_sum_ex(x, dtype, dones, out, E, T, 0u, ws, ws_bytes, stream);
 }
 
 int rlscan_gae_noalloc(const float *rewards, const float *values, const float *terminateds, const float *truncateds,

@@ -567,14 +567,157 @@ __device__ __forceinline__ float load_one_widen(const T *__restrict__ p, long lo
 
 
 // ---------------------------------------------------------------------------
+// Element positions.  A builder never indexes memory itself: it asks a
+// position policy for "my V elements" of a plane, for the halo element after
+// (or before) them, for element k of a sparse plane, and to store its V
+// outputs.  Two layouts:
+//   RowMajorPos   [E, T] with T contiguous: a thread owns V consecutive
+//                 elements of the flattened array (128-bit vector loads; the
+//                 halo comes from the neighbouring lane by a shuffle);
+//   TimeMajorPos  [T, E] with E contiguous: a thread owns V consecutive
+//                 timesteps of one env; lanes are consecutive envs, so each
+//                 load instruction reads one contiguous 128-byte line per warp.
+// ---------------------------------------------------------------------------
+template <int V>
+struct RowMajorPos {
+    static constexpr bool kRowMajor = true;
+    long long i0, n;
+    bool vec;
+    int lane;
+    __device__ __forceinline__ long long index(int k) const { return i0 + k; }
+    template <class T>
+    __device__ __forceinline__ void load(const T *p, T (&o)[V]) const { load_plane<V>(p, i0, n, vec, o); }
+    template <class T>
+    __device__ __forceinline__ void load_widen(const T *p, float (&o)[V]) const {
+        load_plane_widen<V>(p, i0, n, vec, o);
+    }
+    template <class T>
+    __device__ __forceinline__ void load_flag(const T *p, FlagReg<T> (&o)[V]) const {
+        load_flags<V>(p, i0, n, vec, o);
+    }
+    template <class T>
+    __device__ __forceinline__ float fetch_next(const T *p) const {
+        return lane == 31 ? load_one_widen(p, i0 + V, n) : 0.0f;
+    }
+    __device__ __forceinline__ float next(const float (&own)[V], float fetched) const {
+        const float h = __shfl_down_sync(kFullMask, own[0], 1);
+        return lane == 31 ? fetched : h;
+    }
+    template <class T>
+    __device__ __forceinline__ float fetch_prev(const T *p) const {
+        return lane == 0 ? load_one_widen(p, i0 - 1, n) : 0.0f;
+    }
+    __device__ __forceinline__ float prev(const float (&own)[V], float fetched) const {
+        const float h = __shfl_up_sync(kFullMask, own[V - 1], 1);
+        return lane == 0 ? fetched : h;
+    }
+    template <class T>
+    __device__ __forceinline__ float one(const T *p, int k) const { return load_one_widen(p, i0 + k, n); }
+    template <class T>
+    __device__ __forceinline__ void store(T *p, const T (&o)[V]) const { store_plane<V>(p, i0, n, vec, o); }
+};
+
+template <int V>
+struct TimeMajorPos {
+    static constexpr bool kRowMajor = false;
+    long long base; // index of element k = 0: t0 * E + e
+    int stride;     // E: elements between consecutive timesteps (the host keeps (V + 1) * E < 2^31)
+    long long e;    // the env (row)
+    int kbeg, kend; // element k exists iff kbeg <= k < kend (clamped to [-1, V + 1])
+    bool fast;      // all V elements exist and V divides T (t0 is a multiple of V)
+    __device__ __forceinline__ static TimeMajorPos make(long long e, long long t0, long long E, long long T,
+                                                        bool env_ok) {
+        TimeMajorPos p;
+        p.base = t0 * E + e;
+        p.stride = (int)E;
+        p.e = e;
+        const long long lo = -t0, hi = T - t0;
+        p.kbeg = env_ok ? (int)max(min(lo, (long long)V + 1), -1ll) : V + 1;
+        p.kend = env_ok ? (int)max(min(hi, (long long)V + 1), -1ll) : V + 1;
+        p.fast = env_ok && T % V == 0 && p.kbeg <= 0 && p.kend >= V;
+        return p;
+    }
+    // Element k of plane p: one 64-bit base per plane, 32-bit offsets shared
+    // by all planes.
+    template <class T_>
+    __device__ __forceinline__ const T_ *at(const T_ *p, int k) const { return (p + base) + k * stride; }
+    template <class T_>
+    __device__ __forceinline__ T_ *at(T_ *p, int k) const { return (p + base) + k * stride; }
+    __device__ __forceinline__ bool ok(int k) const { return k >= kbeg && k < kend; }
+    template <class T_>
+    __device__ __forceinline__ float widen_at(const T_ *p, int k) const {
+        if constexpr (std::is_same<T_, float>::value) {
+            return __ldcg(at(p, k));
+        } else {
+            using Bits = typename std::conditional<sizeof(T_) == 2, uint16_t, uint8_t>::type;
+            return widen((Bits)__ldcg(reinterpret_cast<const Bits *>(at(p, k))), T_());
+        }
+    }
+    template <class T_>
+    __device__ __forceinline__ void load(const T_ *p, T_ (&o)[V]) const {
+#pragma unroll
+        for (int k = 0; k < V; ++k) o[k] = (p != nullptr && ok(k)) ? __ldcg(at(p, k)) : T_(0);
+    }
+    template <class T_>
+    __device__ __forceinline__ void load_widen(const T_ *p, float (&o)[V]) const {
+#pragma unroll
+        for (int k = 0; k < V; ++k) o[k] = (p != nullptr && ok(k)) ? widen_at(p, k) : 0.0f;
+    }
+    template <class T_>
+    __device__ __forceinline__ void load_flag(const T_ *p, FlagReg<T_> (&o)[V]) const {
+        if constexpr (std::is_same<T_, float>::value) {
+            load(p, o);
+        } else {
+#pragma unroll
+            for (int k = 0; k < V; ++k) o[k] = (p != nullptr && ok(k)) ? (uint32_t)__ldcg(at(p, k)) : 0u;
+        }
+    }
+    template <class T_>
+    __device__ __forceinline__ float one(const T_ *p, int k) const {
+        return (p != nullptr && ok(k)) ? widen_at(p, k) : 0.0f;
+    }
+    template <class T_>
+    __device__ __forceinline__ float fetch_next(const T_ *p) const { return one(p, V); }
+    __device__ __forceinline__ float next(const float (&)[V], float fetched) const { return fetched; }
+    template <class T_>
+    __device__ __forceinline__ float fetch_prev(const T_ *p) const { return one(p, -1); }
+    __device__ __forceinline__ float prev(const float (&)[V], float fetched) const { return fetched; }
+    template <class T_>
+    __device__ __forceinline__ void store(T_ *p, const T_ (&o)[V]) const {
+#pragma unroll
+        for (int k = 0; k < V; ++k)
+            if (ok(k)) __stcs(at(p, k), o[k]);
+    }
+};
+
+// Row masks of a time-major thread: its V timesteps t0.. of env e (row e).
+// Element k is the row's first step iff t0 + k == 0 (k == kbeg >= 0) and its
+// last iff t0 + k == T - 1 (k == kend - 1 < V).
+template <int V>
+__device__ __forceinline__ RowMasks time_major_masks(const TimeMajorPos<V> &pos) {
+    RowMasks m;
+    m.row0 = pos.e;
+    m.valid = 0u;
+#pragma unroll
+    for (int k = 0; k < V; ++k)
+        if (pos.ok(k)) m.valid |= 1u << k;
+    m.start = (pos.kbeg >= 0 && pos.kbeg < V && pos.kbeg < pos.kend) ? (1u << pos.kbeg) : 0u;
+    m.end = (pos.kend >= 1 && pos.kend <= V && pos.kbeg < pos.kend) ? (1u << (pos.kend - 1)) : 0u;
+    m.fast = pos.fast;
+    return m;
+}
+
+// ---------------------------------------------------------------------------
 // The tile kernel.  Est supplies (see estimators.cuh):
 //   kBackward, AT, BT, Params, State<V>,
-//   load<NT, V>(P, g, i0, lane, S, dyn_smem)    -- every thread, incl. past n
-//   coeffs<V>(P, g, i0, rm, S, a, b)            -- (a, b) per element, identity past n
+//   load<NT, V>(P, g, pos, S, dyn_smem)         -- every thread, incl. past n
+//   coeffs<V>(P, g, pos, rm, S, a, b)           -- (a, b) per element, identity past n
 //   out<V>(P, S, k, x, x_prev, b_k)             -- record output k (x_prev = value
 //                                                  of the element before it in scan order,
 //                                                  b_k = its scan coefficient b)
-//   store<V>(P, g, i0, S)
+//   store<V>(P, g, pos, S)
+// where `pos` is the thread's element-position policy (RowMajorPos or
+// TimeMajorPos).
 // ---------------------------------------------------------------------------
 
 // Scan modes of one launch:
@@ -636,13 +779,14 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
     const long long tile0 = m * (long long)(NT * V);
     const long long i0 = tile0 + (long long)tid * V;
 
+    const RowMajorPos<V> pos{i0, g.n, g.vec_ok != 0 && i0 + V <= g.n, lane};
     typename Est::template State<V> S;
-    Est::template load<NT, V>(P, g, i0, lane, S, dyn_smem);
+    Est::template load<NT, V>(P, g, pos, S, dyn_smem);
 
     AT a[V];
     BT b[V];
     const RowMasks rm = row_masks<V>(i0, g);
-    Est::template coeffs<V>(P, g, i0, rm, S, a, b);
+    Est::template coeffs<V>(P, g, pos, rm, S, a, b);
 
     // thread aggregate, composed in scan order
     AT ta;
@@ -734,9 +878,111 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
             Est::template out<V>(P, S, k, x, prev, b[k]);
         }
     }
-    Est::template store<V>(P, g, i0, S);
+    Est::template store<V>(P, g, pos, S);
 
     if constexpr (kLookback) lookback_release<NT>(lb, g.ntiles);
+}
+
+// ---------------------------------------------------------------------------
+// The time-major kernel, for [T, E] arrays (E contiguous).  A block owns 32
+// envs (one per lane) and walks their rows in segments of NW * V timesteps,
+// in scan order: warp w holds timesteps [segment + w V, + V) of its lane's
+// env, composes them in registers, and the block chains the NW chunk
+// aggregates of each env through shared memory, starting from the value the
+// previous segment left.  Every load and store instruction of a warp covers
+// 32 consecutive envs at one timestep, i.e. contiguous memory.  Rows never
+// span blocks, so no workspace and no look-back are needed.
+// ---------------------------------------------------------------------------
+template <class Est, int NW, int V>
+__global__ void __launch_bounds__(NW * 32) time_major_scan_kernel(const typename Est::Params P, const Geometry g) {
+    using AT = typename Est::AT;
+    using BT = typename Est::BT;
+    constexpr bool kBwd = Est::kBackward;
+    constexpr long long kSeg = (long long)NW * V;
+    __shared__ AT s_a[NW][32];
+    __shared__ BT s_b[NW][32];
+    __shared__ BT s_x[NW][32];
+    __shared__ BT s_carry[32];
+
+    griddep_wait();
+    griddep_launch_dependents();
+
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;
+    const long long E = g.rows, T = g.seq_len;
+    const long long e = (long long)blockIdx.x * 32 + lane;
+    const bool env_ok = e < E;
+    const long long nseg = (T + kSeg - 1) / kSeg;
+    if (w == 0) s_carry[lane] = BT(0);
+
+    for (long long si = 0; si < nseg; ++si) {
+        const long long seg = kBwd ? nseg - 1 - si : si;
+        const TimeMajorPos<V> pos = TimeMajorPos<V>::make(e, seg * kSeg + (long long)w * V, E, T, env_ok);
+        typename Est::template State<V> S;
+        Est::template load<NW * 32, V>(P, g, pos, S, nullptr);
+        AT a[V];
+        BT b[V];
+        const RowMasks rm = time_major_masks<V>(pos);
+        Est::template coeffs<V>(P, g, pos, rm, S, a, b);
+
+        AT ta;
+        BT tb;
+        if (kBwd) {
+            ta = a[V - 1];
+            tb = b[V - 1];
+#pragma unroll
+            for (int k = V - 2; k >= 0; --k) {
+                AT na = a[k];
+                BT nb = b[k];
+                combine(na, nb, ta, tb);
+                ta = na;
+                tb = nb;
+            }
+        } else {
+            ta = a[0];
+            tb = b[0];
+#pragma unroll
+            for (int k = 1; k < V; ++k) {
+                AT na = a[k];
+                BT nb = b[k];
+                combine(na, nb, ta, tb);
+                ta = na;
+                tb = nb;
+            }
+        }
+        s_a[w][lane] = ta;
+        s_b[w][lane] = tb;
+        __syncthreads();
+        if (w == 0) { // chain this env's chunks in scan order
+            BT x = s_carry[lane];
+#pragma unroll
+            for (int j = 0; j < NW; ++j) {
+                const int ww = kBwd ? NW - 1 - j : j;
+                s_x[ww][lane] = x;
+                x = apply_pair(s_a[ww][lane], s_b[ww][lane], x);
+            }
+            s_carry[lane] = x;
+        }
+        __syncthreads();
+        BT x = s_x[w][lane];
+        if (kBwd) {
+#pragma unroll
+            for (int k = V - 1; k >= 0; --k) {
+                const BT prev = x;
+                x = apply_pair(a[k], b[k], x);
+                Est::template out<V>(P, S, k, x, prev, b[k]);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                const BT prev = x;
+                x = apply_pair(a[k], b[k], x);
+                Est::template out<V>(P, S, k, x, prev, b[k]);
+            }
+        }
+        Est::template store<V>(P, g, pos, S);
+        __syncthreads(); // shared arrays are reused by the next segment
+    }
 }
 
 } // namespace rlscan

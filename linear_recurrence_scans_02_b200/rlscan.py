@@ -18,6 +18,11 @@ and "Usage" example):
 
 All tensors are CUDA, contiguous, float32 ``[E, T]`` (int32 allowed for the
 prefix sum input/output, ``[E, T, A]`` for Retrace's per-action arrays).
+Keyword options of the float32 entry points: ``time_major=True`` takes every
+``[E, T]`` array as ``[T, E]`` instead (envs contiguous, the rollout-buffer
+layout; no workspace), and, for eligibility traces and the prefix sum,
+``done_starts_episode=True`` reads ``dones[t]`` as "step t starts an episode"
+rather than "step t ends one".
 """
 from __future__ import annotations
 
@@ -49,6 +54,8 @@ RLSCAN_I32 = 1
 RLSCAN_BF16 = 2
 RLSCAN_F16 = 3
 RLSCAN_U8 = 4
+RLSCAN_OPT_TIME_MAJOR = 1
+RLSCAN_OPT_DONE_STARTS_EPISODE = 2
 _VALUE_DTYPES = {torch.float32: RLSCAN_F32, torch.bfloat16: RLSCAN_BF16, torch.float16: RLSCAN_F16}
 _FLAG_DTYPES = {torch.float32: RLSCAN_F32, torch.uint8: RLSCAN_U8, torch.bool: RLSCAN_U8}
 
@@ -73,8 +80,8 @@ def _load_library():
             "`python -c 'import __graft_entry__ as g; g.build()'` or "
             "`python linear_recurrence_scans_02_b200/_build.py`")
     lib = ctypes.CDLL(path)
-    P, I64, F, SZ, S, INT = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
-                             ctypes.c_void_p, ctypes.c_int)
+    P, I64, F, SZ, S, INT, U = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
+                                ctypes.c_void_p, ctypes.c_int, ctypes.c_uint)
     sigs = {
         "rlscan_gae": [P] * 7 + [I64, I64, F, F, P, SZ, S],
         "rlscan_gae_with_returns": [P] * 8 + [I64, I64, F, F, P, SZ, S],
@@ -85,6 +92,14 @@ def _load_library():
         "rlscan_discounted_returns": [P] * 6 + [I64, I64, F, P, SZ, S],
         "rlscan_eligibility_traces": [P] * 3 + [I64, I64, F, F, P, SZ, S],
         "rlscan_episodic_prefix_sum": [P, INT, P, P, I64, I64, P, SZ, S],
+        "rlscan_gae_ex": [P] * 7 + [I64, I64, F, F, U, P, SZ, S],
+        "rlscan_gae_with_returns_ex": [P] * 8 + [I64, I64, F, F, U, P, SZ, S],
+        "rlscan_vtrace_ex": [P] * 9 + [I64, I64, F, F, F, F, U, P, SZ, S],
+        "rlscan_retrace_ex": [P] * 8 + [I64, I64, I64, F, F, F, U, P, SZ, S],
+        "rlscan_lambda_returns_ex": [P] * 7 + [I64, I64, F, F, U, P, SZ, S],
+        "rlscan_discounted_returns_ex": [P] * 6 + [I64, I64, F, U, P, SZ, S],
+        "rlscan_eligibility_traces_ex": [P] * 3 + [I64, I64, F, F, U, P, SZ, S],
+        "rlscan_episodic_prefix_sum_ex": [P, INT, P, P, I64, I64, U, P, SZ, S],
         "rlscan_workspace_init": [P, SZ, S],
         "rlscan_check": [S],
         "rlscan_version": [],
@@ -204,32 +219,48 @@ def rlscan_debug_set_lookback(spin_limit: int = 0, withhold_tile: int = -1) -> N
 # rlscan_* : the C calls with tensors (outputs preallocated)
 # ---------------------------------------------------------------------------
 
+def _layout(t, name, time_major):
+    """(E, T, plane shape, options) of an [E, T] (or time-major [T, E]) call."""
+    if not isinstance(t, torch.Tensor) or t.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D tensor ([num_envs, seq_len], or [seq_len, num_envs] "
+                         "with time_major=True)")
+    if time_major:
+        T, E = int(t.shape[0]), int(t.shape[1])
+        return E, T, (T, E), RLSCAN_OPT_TIME_MAJOR
+    E, T = int(t.shape[0]), int(t.shape[1])
+    return E, T, (E, T), 0
+
+
+def _ws_for(dev, E, T, ws, opts):
+    if opts & RLSCAN_OPT_TIME_MAJOR:  # rows never span blocks: no workspace
+        return None, 0, _stream_handle(dev)
+    return _workspace(dev, E, T, ws)
+
+
 def rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages,
-               gamma, lambda_, ws=None):
-    E, T = _shape(rewards, "rewards")
+               gamma, lambda_, ws=None, *, time_major=False):
+    E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
-    sh = (E, T)
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_gae(
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_gae_ex(
         _ptr(rewards, "rewards", sh, device=dev), _ptr(values, "values", sh, device=dev),
         _ptr(terminateds, "terminateds", sh, device=dev), _ptr(truncateds, "truncateds", sh, device=dev),
         _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
         _ptr(last_values, "last_values", (E,), device=dev), _ptr(advantages, "advantages", sh, device=dev),
-        E, T, float(gamma), float(lambda_), wp, wn, s))
+        E, T, float(gamma), float(lambda_), opts, wp, wn, s))
 
 
 def rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages,
-                            returns, gamma, lambda_, ws=None):
-    E, T = _shape(rewards, "rewards")
+                            returns, gamma, lambda_, ws=None, *, time_major=False):
+    E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
-    sh = (E, T)
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_gae_with_returns(
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_gae_with_returns_ex(
         _ptr(rewards, "rewards", sh, device=dev), _ptr(values, "values", sh, device=dev),
         _ptr(terminateds, "terminateds", sh, device=dev), _ptr(truncateds, "truncateds", sh, device=dev),
         _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
         _ptr(last_values, "last_values", (E,), device=dev), _ptr(advantages, "advantages", sh, device=dev),
-        _ptr(returns, "returns", sh, device=dev), E, T, float(gamma), float(lambda_), wp, wn, s))
+        _ptr(returns, "returns", sh, device=dev), E, T, float(gamma), float(lambda_), opts, wp, wn, s))
 
 
 def rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages,
@@ -263,92 +294,91 @@ def _reduced_bytes(*tensors):
 
 
 def rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values,
-                  vs, pg_advantages, gamma, lambda_=1.0, rho_bar=1.0, c_bar=1.0, ws=None):
-    E, T = _shape(rewards, "rewards")
+                  vs, pg_advantages, gamma, lambda_=1.0, rho_bar=1.0, c_bar=1.0, ws=None, *, time_major=False):
+    E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
-    sh = (E, T)
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_vtrace(
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_vtrace_ex(
         _ptr(log_rhos, "log_rhos", sh, device=dev), _ptr(rewards, "rewards", sh, device=dev),
         _ptr(values, "values", sh, device=dev), _ptr(terminateds, "terminateds", sh, device=dev),
         _ptr(truncateds, "truncateds", sh, device=dev),
         _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
         _ptr(last_values, "last_values", (E,), device=dev), _ptr(vs, "vs", sh, device=dev),
         _ptr(pg_advantages, "pg_advantages", sh, device=dev),
-        E, T, float(gamma), float(lambda_), float(rho_bar), float(c_bar), wp, wn, s))
+        E, T, float(gamma), float(lambda_), float(rho_bar), float(c_bar), opts, wp, wn, s))
 
 
 def rlscan_retrace(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds,
-                   truncateds, q_ret, gamma, lambda_, c_bar=1.0, ws=None):
-    E, T = _shape(rewards, "rewards")
+                   truncateds, q_ret, gamma, lambda_, c_bar=1.0, ws=None, *, time_major=False):
+    E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
-    sh = (E, T)
     if next_q_values_all.dim() == 2:
         A, sh3 = 1, sh
     else:
         A = int(next_q_values_all.shape[2])
-        sh3 = (E, T, A)
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_retrace(
+        sh3 = sh + (A,)
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_retrace_ex(
         _ptr(rewards, "rewards", sh, device=dev), _ptr(q_values, "q_values", sh, device=dev),
         _ptr(next_q_values_all, "next_q_values_all", sh3, device=dev),
         _ptr(next_target_probs, "next_target_probs", sh3, device=dev),
         _ptr(log_rhos, "log_rhos", sh, device=dev), _ptr(terminateds, "terminateds", sh, device=dev),
         _ptr(truncateds, "truncateds", sh, device=dev), _ptr(q_ret, "q_ret", sh, device=dev),
-        E, T, A, float(gamma), float(lambda_), float(c_bar), wp, wn, s))
+        E, T, A, float(gamma), float(lambda_), float(c_bar), opts, wp, wn, s))
 
 
 def rlscan_lambda_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, returns,
-                          gamma, lambda_, ws=None):
-    E, T = _shape(rewards, "rewards")
+                          gamma, lambda_, ws=None, *, time_major=False):
+    E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
-    sh = (E, T)
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_lambda_returns(
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_lambda_returns_ex(
         _ptr(rewards, "rewards", sh, device=dev), _ptr(values, "values", sh, device=dev),
         _ptr(terminateds, "terminateds", sh, device=dev), _ptr(truncateds, "truncateds", sh, device=dev),
         _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
         _ptr(last_values, "last_values", (E,), device=dev), _ptr(returns, "returns", sh, device=dev),
-        E, T, float(gamma), float(lambda_), wp, wn, s))
+        E, T, float(gamma), float(lambda_), opts, wp, wn, s))
 
 
 def rlscan_discounted_returns(rewards, terminateds, truncateds, bootstrap_values, last_values, returns,
-                              gamma, ws=None):
-    E, T = _shape(rewards, "rewards")
+                              gamma, ws=None, *, time_major=False):
+    E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
-    sh = (E, T)
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_discounted_returns(
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_discounted_returns_ex(
         _ptr(rewards, "rewards", sh, device=dev), _ptr(terminateds, "terminateds", sh, device=dev),
         _ptr(truncateds, "truncateds", sh, device=dev),
         _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
         _ptr(last_values, "last_values", (E,), device=dev), _ptr(returns, "returns", sh, device=dev),
-        E, T, float(gamma), wp, wn, s))
+        E, T, float(gamma), opts, wp, wn, s))
 
 
-def rlscan_eligibility_traces(x, dones, traces, gamma, lambda_, ws=None):
-    E, T = _shape(x, "x")
+def rlscan_eligibility_traces(x, dones, traces, gamma, lambda_, ws=None, *, time_major=False,
+                              done_starts_episode=False):
+    E, T, sh, opts = _layout(x, "x", time_major)
+    if done_starts_episode:
+        opts |= RLSCAN_OPT_DONE_STARTS_EPISODE
     dev = x.device
-    sh = (E, T)
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_eligibility_traces(
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_eligibility_traces_ex(
         _ptr(x, "x", sh, device=dev), _ptr(dones, "dones", sh, device=dev), _ptr(traces, "traces", sh, device=dev),
-        E, T, float(gamma), float(lambda_), wp, wn, s))
+        E, T, float(gamma), float(lambda_), opts, wp, wn, s))
 
 
-def rlscan_episodic_prefix_sum(x, dones, out, ws=None):
-    E, T = _shape(x, "x")
+def rlscan_episodic_prefix_sum(x, dones, out, ws=None, *, time_major=False, done_starts_episode=False):
+    E, T, sh, opts = _layout(x, "x", time_major)
+    if done_starts_episode:
+        opts |= RLSCAN_OPT_DONE_STARTS_EPISODE
     dev = x.device
-    sh = (E, T)
     if x.dtype not in (torch.float32, torch.int32):
         raise TypeError("x must be float32 or int32")
     if out.dtype != x.dtype:
         raise TypeError("out must have the dtype of x")
     dtype = RLSCAN_F32 if x.dtype == torch.float32 else RLSCAN_I32
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_episodic_prefix_sum(
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_episodic_prefix_sum_ex(
         _ptr(x, "x", sh, (torch.float32, torch.int32), device=dev), dtype, _ptr(dones, "dones", sh, device=dev),
-        _ptr(out, "out", sh, (torch.float32, torch.int32), device=dev), E, T, wp, wn, s))
+        _ptr(out, "out", sh, (torch.float32, torch.int32), device=dev), E, T, opts, wp, wn, s))
 
 
 # ---------------------------------------------------------------------------
@@ -356,72 +386,81 @@ def rlscan_episodic_prefix_sum(x, dones, out, ws=None):
 # ---------------------------------------------------------------------------
 
 def compute_gae(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
-                bootstrap_values=None, last_values=None):
+                bootstrap_values=None, last_values=None, time_major=False):
     """Advantages (fp32).  bf16/fp16 values or uint8/bool flags take the
-    reduced-byte entry point."""
+    reduced-byte entry point (row-major only)."""
     adv = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
     if _reduced_bytes(rewards, values, terminateds, truncateds, bootstrap_values):
+        if time_major:
+            raise ValueError("reduced-byte inputs take the row-major [num_envs, seq_len] layout only")
         rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, None, gamma,
                          lambda_)
     else:
-        rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, gamma, lambda_)
+        rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, gamma, lambda_,
+                   time_major=time_major)
     return adv
 
 
 def compute_gae_with_returns(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
-                             bootstrap_values=None, last_values=None):
+                             bootstrap_values=None, last_values=None, time_major=False):
     """(advantages, returns) from one pass: returns = advantages + values.
-    bf16/fp16 values or uint8/bool flags take the reduced-byte entry point."""
+    bf16/fp16 values or uint8/bool flags take the reduced-byte entry point
+    (row-major only)."""
     adv = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
     ret = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
     if _reduced_bytes(rewards, values, terminateds, truncateds, bootstrap_values):
+        if time_major:
+            raise ValueError("reduced-byte inputs take the row-major [num_envs, seq_len] layout only")
         rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret, gamma,
                          lambda_)
     else:
         rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret,
-                                gamma, lambda_)
+                                gamma, lambda_, time_major=time_major)
     return adv, ret
 
 
 def compute_vtrace(log_rhos, rewards, values, terminateds, gamma=0.99, lambda_=1.0, rho_bar=1.0, c_bar=1.0, *,
-                   truncateds=None, bootstrap_values=None, last_values=None):
+                   truncateds=None, bootstrap_values=None, last_values=None, time_major=False):
     vs = torch.empty_like(rewards)
     pg = torch.empty_like(rewards)
     rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values, vs, pg,
-                  gamma, lambda_, rho_bar, c_bar)
+                  gamma, lambda_, rho_bar, c_bar, time_major=time_major)
     return vs, pg
 
 
 def compute_retrace(rewards, q_values, next_q_values_all, log_rhos, terminateds, truncateds, gamma=0.99,
-                    lambda_=0.95, c_bar=1.0, *, next_target_probs=None):
+                    lambda_=0.95, c_bar=1.0, *, next_target_probs=None, time_major=False):
     q_ret = torch.empty_like(rewards)
     rlscan_retrace(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds, truncateds,
-                   q_ret, gamma, lambda_, c_bar)
+                   q_ret, gamma, lambda_, c_bar, time_major=time_major)
     return q_ret
 
 
 def compute_lambda_returns(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
-                           bootstrap_values=None, last_values=None):
+                           bootstrap_values=None, last_values=None, time_major=False):
     ret = torch.empty_like(rewards)
     rlscan_lambda_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, ret, gamma,
-                          lambda_)
+                          lambda_, time_major=time_major)
     return ret
 
 
 def compute_discounted_returns(rewards, terminateds=None, gamma=0.99, *, truncateds=None, bootstrap_values=None,
-                               last_values=None):
+                               last_values=None, time_major=False):
     ret = torch.empty_like(rewards)
-    rlscan_discounted_returns(rewards, terminateds, truncateds, bootstrap_values, last_values, ret, gamma)
+    rlscan_discounted_returns(rewards, terminateds, truncateds, bootstrap_values, last_values, ret, gamma,
+                              time_major=time_major)
     return ret
 
 
-def compute_eligibility_traces(x, dones=None, gamma=0.99, lambda_=0.95):
+def compute_eligibility_traces(x, dones=None, gamma=0.99, lambda_=0.95, *, time_major=False,
+                               done_starts_episode=False):
     out = torch.empty_like(x)
-    rlscan_eligibility_traces(x, dones, out, gamma, lambda_)
+    rlscan_eligibility_traces(x, dones, out, gamma, lambda_, time_major=time_major,
+                              done_starts_episode=done_starts_episode)
     return out
 
 
-def compute_episodic_prefix_sum(x, dones=None):
+def compute_episodic_prefix_sum(x, dones=None, *, time_major=False, done_starts_episode=False):
     out = torch.empty_like(x)
-    rlscan_episodic_prefix_sum(x, dones, out)
+    rlscan_episodic_prefix_sum(x, dones, out, time_major=time_major, done_starts_episode=done_starts_episode)
     return out

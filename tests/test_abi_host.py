@@ -41,6 +41,11 @@ def lib(rlscan_lib_path):
     L.rlscan_eligibility_traces.argtypes = [P] * 3 + [I64, I64, F, F, P, SZ, P]
     L.rlscan_episodic_prefix_sum.argtypes = [P, ctypes.c_int, P, P, I64, I64, P, SZ, P]
     L.rlscan_gae_noalloc.argtypes = [P] * 7 + [I64, I64, F, F, P]
+    U = ctypes.c_uint
+    L.rlscan_gae_ex.argtypes = [P] * 7 + [I64, I64, F, F, U, P, SZ, P]
+    L.rlscan_retrace_ex.argtypes = [P] * 8 + [I64, I64, I64, F, F, F, U, P, SZ, P]
+    L.rlscan_eligibility_traces_ex.argtypes = [P] * 3 + [I64, I64, F, F, U, P, SZ, P]
+    L.rlscan_episodic_prefix_sum_ex.argtypes = [P, ctypes.c_int, P, P, I64, I64, U, P, SZ, P]
     L.rlscan_workspace_bytes.argtypes = [I64, I64]
     L.rlscan_workspace_bytes.restype = SZ
     L.rlscan_last_error.restype = ctypes.c_char_p
@@ -197,3 +202,30 @@ def test_gae_typed_dtype_rules(lib):
     # 2-byte values: planes of E*T*2 bytes; the output starting inside one is an overlap
     assert lib.rlscan_gae_typed(A, B, C, None, None, None, A + 2, None, E, T, 0.99, 0.95, BF16, U8, None, 0, None) == INVALID
     assert lib.rlscan_gae_typed(A, B, C, D, None, None, O1, None, E, T, 0.99, 0.95, F16, U8, None, 0, None) == INVALID
+
+
+TIME_MAJOR, DONE_STARTS = 1, 2
+
+
+def test_ex_option_bits(lib):
+    # unknown bits, and the forward-only reset convention on a backward estimator
+    for bad in (4, 0x80000000, DONE_STARTS, TIME_MAJOR | DONE_STARTS):
+        assert lib.rlscan_gae_ex(A, B, C, None, None, None, O1, E, T, 0.99, 0.95, bad, None, 0, None) == INVALID
+        assert "option" in msg(lib)
+    assert lib.rlscan_eligibility_traces_ex(A, C, O1, E, T, 0.99, 0.95, 8, None, 0, None) == INVALID
+    assert lib.rlscan_episodic_prefix_sum_ex(A, 0, C, O1, E, T, 16, None, 0, None) == INVALID
+    # argument checks still run under the options
+    assert lib.rlscan_gae_ex(None, B, C, None, None, None, O1, E, T, 0.99, 0.95, TIME_MAJOR, None, 0, None) == INVALID
+    assert lib.rlscan_eligibility_traces_ex(A, C, A + 8, E, T, 0.99, 0.95, DONE_STARTS, None, 0, None) == INVALID
+
+
+def test_ex_time_major_limits(lib):
+    # multi-action Retrace has no time-major form
+    assert lib.rlscan_retrace_ex(A, B, C, C, D, O2, O2 + 0x1000000, O1, E, T, 4, 0.99, 0.95, 1.0, TIME_MAJOR,
+                                 None, 0, None) == UNSUPPORTED
+    # E above the time-major limit ((8 + 1) E must stay below 2^31)
+    E_big = (2 ** 31 - 1) // 9 + 1
+    far = [(k + 1) << 33 for k in range(4)]  # ~1 GB planes, 8 GiB apart: no overlap
+    assert lib.rlscan_gae_ex(far[0], far[1], far[2], None, None, None, far[3], E_big, 1, 0.99, 0.95, TIME_MAJOR,
+                             None, 0, None) == UNSUPPORTED
+    assert "time-major" in msg(lib)
