@@ -667,13 +667,13 @@ def run_reference(args):
 
 
 def run_profile_case(args):
-    """Small case for ncu: `n` eager launches of every estimator, one
-    [4096, 128] buffer set (about 70 MB on the device), synchronised after
-    each estimator.  Prints nothing to time."""
+    """Small case for ncu: `n` eager launches of every estimator (and of the
+    calls timed beside the step), one [4096, 128] buffer set (about 110 MB on
+    the device), synchronised after each estimator.  Prints nothing to time."""
     import torch
     from linear_recurrence_scans_02_b200 import rlscan as R
     torch.cuda.set_device(0)
-    bs = BufferSet(torch, torch.device("cuda", 0), ESTIMATORS)
+    bs = BufferSet(torch, torch.device("cuda", 0), PLANES)
     bs.fill_from_host(host_inputs(seed=0))
     calls = bs.calls(R)
     for est in (args.profile_only.split(",") if args.profile_only else list(ESTIMATORS)):

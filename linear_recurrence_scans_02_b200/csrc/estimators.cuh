@@ -93,6 +93,17 @@ struct GaeEstT {
         default: break;
         }
     }
+    // Input planes read element by element (the time-major kernel's prefetch).
+    static constexpr int kInputPlanes = 4;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        switch (i) {
+        case 0: return {P.rewards, (int)sizeof(ValT)};
+        case 1: return {P.values, (int)sizeof(ValT)};
+        case 2: return {P.terminateds, (int)sizeof(FlagT)};
+        case 3: return {P.truncateds, (int)sizeof(FlagT)};
+        default: return {nullptr, 0};
+        }
+    }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
@@ -176,6 +187,11 @@ struct LambdaReturnsEst {
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds);
+    }
+    static constexpr int kInputPlanes = 4;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        const float *p[4] = {P.rewards, P.values, P.terminateds, P.truncateds};
+        return {i < 4 ? p[i] : nullptr, 4};
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
@@ -263,6 +279,11 @@ struct ReturnsEst {
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.rewards, P.terminateds, P.truncateds);
     }
+    static constexpr int kInputPlanes = 3;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        const float *p[3] = {P.rewards, P.terminateds, P.truncateds};
+        return {i < 3 ? p[i] : nullptr, 4};
+    }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
@@ -340,6 +361,11 @@ struct VtraceEst {
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds);
+    }
+    static constexpr int kInputPlanes = 5;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        const float *p[5] = {P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds};
+        return {i < 5 ? p[i] : nullptr, 4};
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
@@ -447,6 +473,13 @@ struct RetraceEst {
             if (threadIdx.x == 6) prefetch_l2(P.next_q_values_all, tile0 * P.actions, cnt * P.actions, 4);
             if (threadIdx.x == 7) prefetch_l2(P.next_target_probs, tile0 * P.actions, cnt * P.actions, 4);
         }
+    }
+    // single-action form only (the time-major kernel takes A == 1)
+    static constexpr int kInputPlanes = 6;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        const float *p[6] = {P.rewards, P.q_values, P.log_rhos, P.terminateds, P.truncateds,
+                             kMulti ? nullptr : P.next_q_values_all};
+        return {i < 6 ? p[i] : nullptr, 4};
     }
 
     // Expected next-state value of each of this thread's elements.
@@ -593,6 +626,11 @@ struct ForwardF32Est {
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.x, P.dones);
     }
+    static constexpr int kInputPlanes = 2;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        const void *p[2] = {P.x, P.dones};
+        return {i < 2 ? p[i] : nullptr, 4};
+    }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
@@ -655,6 +693,11 @@ struct PrefixI32Est {
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.x, P.dones);
+    }
+    static constexpr int kInputPlanes = 2;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        const void *p[2] = {P.x, P.dones};
+        return {i < 2 ? p[i] : nullptr, 4};
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,

@@ -336,33 +336,57 @@ int check_options(unsigned options, bool forward) {
     return RLSCAN_OK;
 }
 
-// Time-major [T, E] launch: one block per 32 envs, 16 warps x 8 timesteps per
-// segment; no workspace.
-constexpr int kTmWarps = 16;
+// Time-major [T, E] launch: a block owns G envs; a warp covers 32 / G
+// chunks of kTmV timesteps of each; nw warps make a segment, the block walks
+// the rows segment by segment.  No workspace.
 constexpr int kTmV = 8;
+
+struct TmPlan {
+    int G, nw;
+};
+
+// Wider env groups (longer contiguous runs per load) while the grid keeps
+// about one block per SM; rows of several segments (T > 256) favour more,
+// smaller blocks.  Measured at E x T = 1024..65536 x 128, 4096 x 1024 and
+// 512 x 4096.  The segment covers the row, up to 16 warps.
+TmPlan tm_plan(long long E, long long T) {
+    TmPlan p;
+    const long long kMinBlocks = 120;
+    p.G = (E / 32 >= kMinBlocks && T <= 256) ? 32 : (E / 16 >= kMinBlocks ? 16 : 8);
+    const long long chunks = ceil_div(T, kTmV);
+    const long long nw = ceil_div(chunks, 32 / p.G);
+    p.nw = (int)(nw < 1 ? 1 : (nw > kTmMaxWarps ? kTmMaxWarps : nw));
+    return p;
+}
 
 template <class Est>
 int run_time_major(const char *name, const typename Est::Params &P, long long E, long long T, cudaStream_t stream) {
     if (E > (long long)INT_MAX / (kTmV + 1))
         return fail(RLSCAN_ERR_UNSUPPORTED, "%s: the time-major layout takes E <= %d", name, INT_MAX / (kTmV + 1));
+    const TmPlan tp = tm_plan(E, T);
     Geometry g;
     g.n = E * T;
     g.seq_len = T;
     g.rows = E;
-    g.ntiles = ceil_div(E, 32);
+    g.ntiles = ceil_div(T, (long long)tp.nw * (32 / tp.G) * kTmV); // segments per row
     g.t_shift = pow2_shift(T);
     g.vec_ok = 0;
     g.scan_lanes = 32;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)g.ntiles);
-    cfg.blockDim = dim3(kTmWarps * 32);
+    cfg.gridDim = dim3((unsigned)ceil_div(E, tp.G));
+    cfg.blockDim = dim3(tp.nw * 32);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, kTmWarps, kTmV>, P, g);
+    cudaError_t e;
+    switch (tp.G) {
+    case 32: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 32, kTmV>, P, g); break;
+    case 16: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 16, kTmV>, P, g); break;
+    default: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 8, kTmV>, P, g); break;
+    }
     if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
     return ok();
 }

@@ -223,7 +223,7 @@ struct Lookback {
 struct Geometry {
     long long n;       // E * T
     long long seq_len; // T
-    long long ntiles;
+    long long ntiles;  // tiles (tile kernel) or segments per row (time-major kernel)
     long long rows;    // E
     int t_shift;       // log2(T) when T is a power of two, else -1
     int vec_ok;        // every plane pointer of the call is 16-byte aligned
@@ -884,104 +884,191 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
 }
 
 // ---------------------------------------------------------------------------
-// The time-major kernel, for [T, E] arrays (E contiguous).  A block owns 32
-// envs (one per lane) and walks their rows in segments of NW * V timesteps,
-// in scan order: warp w holds timesteps [segment + w V, + V) of its lane's
-// env, composes them in registers, and the block chains the NW chunk
-// aggregates of each env through shared memory, starting from the value the
-// previous segment left.  Every load and store instruction of a warp covers
-// 32 consecutive envs at one timestep, i.e. contiguous memory.  Rows never
-// span blocks, so no workspace and no look-back are needed.
+// The time-major kernel, for [T, E] arrays (E contiguous).  A block owns G
+// consecutive envs and walks their rows in segments, in scan order.  Within
+// a warp, lane l serves env l % G and chunk l / G: the warp covers 32 / G
+// chunks of V timesteps of its G envs, so each load instruction of a warp
+// reads 32 / G runs of G consecutive envs (whole 32-byte sectors for G >= 8).
+// A segment is nw warps x 32 / G chunks x V timesteps.  Chunk aggregates
+// are scanned across a warp's chunks with shuffles (stride G lanes), the
+// warps of a segment are chained per env through shared memory, and the
+// value a segment leaves is the carry into the next one.  Rows never span
+// blocks, so no workspace and no look-back are needed.
 // ---------------------------------------------------------------------------
-template <class Est, int NW, int V>
-__global__ void __launch_bounds__(NW * 32) time_major_scan_kernel(const typename Est::Params P, const Geometry g) {
+struct PlaneRef {
+    const void *p;
+    int bytes; // element size
+};
+
+constexpr int kTmMaxWarps = 16;
+
+__device__ __forceinline__ void prefetch_line_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+template <class Est, int G, int V>
+__global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const typename Est::Params P,
+                                                                           const Geometry g) {
     using AT = typename Est::AT;
     using BT = typename Est::BT;
     constexpr bool kBwd = Est::kBackward;
-    constexpr long long kSeg = (long long)NW * V;
-    __shared__ AT s_a[NW][32];
-    __shared__ BT s_b[NW][32];
-    __shared__ BT s_x[NW][32];
-    __shared__ BT s_carry[32];
-
-    griddep_wait();
-    griddep_launch_dependents();
+    constexpr int CPW = 32 / G; // chunks per warp
+    static_assert(G >= 1 && G <= 32 && 32 % G == 0, "G divides the warp");
+    __shared__ AT s_a[kTmMaxWarps][G];
+    __shared__ BT s_b[kTmMaxWarps][G];
+    __shared__ BT s_x[kTmMaxWarps][G];
+    __shared__ BT s_carry[G];
 
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5;
+    const int es = lane % G; // env within the block
+    const int cs = lane / G; // chunk within the warp
     const long long E = g.rows, T = g.seq_len;
-    const long long e = (long long)blockIdx.x * 32 + lane;
+    const long long e0 = (long long)blockIdx.x * G;
+    const long long e = e0 + es;
     const bool env_ok = e < E;
-    const long long nseg = (T + kSeg - 1) / kSeg;
-    if (w == 0) s_carry[lane] = BT(0);
+    const int S = nw * CPW * V;       // timesteps per segment (<= 16 * 32 * V)
+    const long long nseg = g.ntiles;  // ceil(T / S), from the host
+
+    // L2 prefetch of the first segment's input rows, before waiting for the
+    // previous grid (L2 is coherent, so a prefetched line is never stale)
+    {
+        const long long t_first = kBwd ? (nseg - 1) * S : 0;
+        const int rows = (int)((T - t_first) < S ? (T - t_first) : S);
+        const int envs = (int)((E - e0) < G ? (E - e0) : G);
+#pragma unroll
+        for (int plane = 0; plane < Est::kInputPlanes; ++plane) {
+            const PlaneRef pr = Est::input_plane(P, plane);
+            if (pr.p == nullptr) continue;
+            for (int r = threadIdx.x; r < rows; r += blockDim.x) {
+                const char *row = static_cast<const char *>(pr.p) + ((t_first + r) * E + e0) * pr.bytes;
+                prefetch_line_l2(row);
+                const char *last = row + (envs - 1) * pr.bytes;
+                if (((uintptr_t)row >> 7) != ((uintptr_t)last >> 7)) prefetch_line_l2(last);
+            }
+        }
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+
+    if (threadIdx.x < G) s_carry[threadIdx.x] = identity_b(BT());
 
     for (long long si = 0; si < nseg; ++si) {
         const long long seg = kBwd ? nseg - 1 - si : si;
-        const TimeMajorPos<V> pos = TimeMajorPos<V>::make(e, seg * kSeg + (long long)w * V, E, T, env_ok);
-        typename Est::template State<V> S;
-        Est::template load<NW * 32, V>(P, g, pos, S, nullptr);
+        const long long t0 = seg * S + (w * CPW + cs) * V;
+        const TimeMajorPos<V> pos = TimeMajorPos<V>::make(e, t0, E, T, env_ok);
+        typename Est::template State<V> St;
+        Est::template load<kTmMaxWarps * 32, V>(P, g, pos, St, nullptr);
         AT a[V];
         BT b[V];
         const RowMasks rm = time_major_masks<V>(pos);
-        Est::template coeffs<V>(P, g, pos, rm, S, a, b);
+        Est::template coeffs<V>(P, g, pos, rm, St, a, b);
 
-        AT ta;
-        BT tb;
+        // chunk aggregate, composed in scan order
+        AT ia;
+        BT ib;
         if (kBwd) {
-            ta = a[V - 1];
-            tb = b[V - 1];
+            ia = a[V - 1];
+            ib = b[V - 1];
 #pragma unroll
             for (int k = V - 2; k >= 0; --k) {
                 AT na = a[k];
                 BT nb = b[k];
-                combine(na, nb, ta, tb);
-                ta = na;
-                tb = nb;
+                combine(na, nb, ia, ib);
+                ia = na;
+                ib = nb;
             }
         } else {
-            ta = a[0];
-            tb = b[0];
+            ia = a[0];
+            ib = b[0];
 #pragma unroll
             for (int k = 1; k < V; ++k) {
                 AT na = a[k];
                 BT nb = b[k];
-                combine(na, nb, ta, tb);
-                ta = na;
-                tb = nb;
+                combine(na, nb, ia, ib);
+                ia = na;
+                ib = nb;
             }
         }
-        s_a[w][lane] = ta;
-        s_b[w][lane] = tb;
-        __syncthreads();
-        if (w == 0) { // chain this env's chunks in scan order
-            BT x = s_carry[lane];
+        const AT own_a = ia;
+
+        // inclusive scan over the warp's chunks of each env (lanes G apart)
 #pragma unroll
-            for (int j = 0; j < NW; ++j) {
-                const int ww = kBwd ? NW - 1 - j : j;
-                s_x[ww][lane] = x;
-                x = apply_pair(s_a[ww][lane], s_b[ww][lane], x);
+        for (int d = 1; d < CPW; d <<= 1) {
+            if (kBwd) {
+                const AT oa = __shfl_down_sync(kFullMask, ia, d * G);
+                const BT ob = __shfl_down_sync(kFullMask, ib, d * G);
+                if (cs + d < CPW) combine(ia, ib, oa, ob);
+            } else {
+                const AT oa = __shfl_up_sync(kFullMask, ia, d * G);
+                const BT ob = __shfl_up_sync(kFullMask, ib, d * G);
+                if (cs >= d) combine(ia, ib, oa, ob);
             }
-            s_carry[lane] = x;
+        }
+        AT ea = identity_a(own_a);
+        BT eb = identity_b(ib);
+        if constexpr (CPW > 1) {
+            const AT xa = kBwd ? __shfl_down_sync(kFullMask, ia, G) : __shfl_up_sync(kFullMask, ia, G);
+            const BT xb = kBwd ? __shfl_down_sync(kFullMask, ib, G) : __shfl_up_sync(kFullMask, ib, G);
+            if (kBwd ? (cs + 1 < CPW) : (cs > 0)) {
+                ea = xa;
+                eb = xb;
+            }
+        }
+        if (cs == (kBwd ? 0 : CPW - 1)) { // the warp's aggregate per env
+            s_a[w][es] = ia;
+            s_b[w][es] = ib;
         }
         __syncthreads();
-        BT x = s_x[w][lane];
+        if (threadIdx.x < G) { // chain this env's warps in scan order
+            const int ee = threadIdx.x;
+            BT x = s_carry[ee];
+            // four warps at a time: their shared loads issue together, ahead
+            // of the dependent applies
+            for (int j0 = 0; j0 < nw; j0 += 4) {
+                AT qa[4];
+                BT qb[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int ww = kBwd ? nw - 1 - (j0 + q) : j0 + q;
+                    const bool in = j0 + q < nw;
+                    qa[q] = in ? s_a[ww][ee] : identity_a(AT());
+                    qb[q] = in ? s_b[ww][ee] : identity_b(BT());
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (j0 + q < nw) {
+                        const int ww = kBwd ? nw - 1 - (j0 + q) : j0 + q;
+                        s_x[ww][ee] = x;
+                        x = apply_pair(qa[q], qb[q], x);
+                    }
+                }
+            }
+            s_carry[ee] = x;
+        }
+        __syncthreads();
+        // shared arrays: the next segment writes s_a / s_b before its first
+        // barrier, after every read of them here (before this barrier), and
+        // s_x / s_carry only after that barrier, when every thread has read
+        // s_x below; so no third barrier is needed
+        BT x = apply_pair(ea, eb, s_x[w][es]);
         if (kBwd) {
 #pragma unroll
             for (int k = V - 1; k >= 0; --k) {
                 const BT prev = x;
                 x = apply_pair(a[k], b[k], x);
-                Est::template out<V>(P, S, k, x, prev, b[k]);
+                Est::template out<V>(P, St, k, x, prev, b[k]);
             }
         } else {
 #pragma unroll
             for (int k = 0; k < V; ++k) {
                 const BT prev = x;
                 x = apply_pair(a[k], b[k], x);
-                Est::template out<V>(P, S, k, x, prev, b[k]);
+                Est::template out<V>(P, St, k, x, prev, b[k]);
             }
         }
-        Est::template store<V>(P, g, pos, S);
-        __syncthreads(); // shared arrays are reused by the next segment
+        Est::template store<V>(P, g, pos, St);
     }
 }
 
