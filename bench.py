@@ -51,6 +51,8 @@ P_DONE = 0.005
 L2_BYTES = 126 * 1024 * 1024
 ROTATE_BYTES = 4 * L2_BYTES
 FALLBACK_HBM_GBS = 6650.0
+REPEATS = 5            # timed repeats per estimator (median reported)
+ISOLATED_SAMPLES = 21  # single calls on an idle stream per estimator
 WORKLOAD = "all seven estimators fp32, num_envs=4096, seq_len=128"
 
 # estimator -> (input planes, output planes, bytes per env-step moved)
@@ -197,6 +199,45 @@ class BufferSet:
             c["prefix_sum_i32"] = lambda: R.rlscan_episodic_prefix_sum(
                 t["prefix_sum_i32", "x"], t["prefix_sum_i32", "dones"], t["prefix_sum_i32", "out"])
         return c
+
+    def batch_call(self, R):
+        """The step's calls as ONE C-ABI request (rlscan_batch): one fused
+        launch runs every estimator's tiles."""
+        t = self.t
+        e = self.estimators
+        calls = []
+        if "gae" in e:
+            calls.append(dict(kind="gae", rewards=t["gae", "rewards"], values=t["gae", "values"],
+                              terminateds=t["gae", "terminateds"], advantages=t["gae", "advantages"],
+                              gamma=GAMMA, lambda_=LAMBDA))
+        if "vtrace" in e:
+            k = "vtrace"
+            calls.append(dict(kind="vtrace", log_rhos=t[k, "log_rhos"], rewards=t[k, "rewards"], values=t[k, "values"],
+                              terminateds=t[k, "terminateds"], vs=t[k, "vs"], pg_advantages=t[k, "pg_advantages"],
+                              gamma=GAMMA, lambda_=1.0, rho_bar=1.0, c_bar=1.0))
+        if "retrace" in e:
+            k = "retrace"
+            calls.append(dict(kind="retrace", rewards=t[k, "rewards"], q_values=t[k, "q_values"],
+                              next_q_values_all=t[k, "next_q_values_all"], next_target_probs=None,
+                              log_rhos=t[k, "log_rhos"], terminateds=t[k, "terminateds"],
+                              truncateds=t[k, "truncateds"], q_ret=t[k, "q_ret"], gamma=GAMMA, lambda_=LAMBDA,
+                              c_bar=1.0))
+        if "lambda_returns" in e:
+            k = "lambda_returns"
+            calls.append(dict(kind=k, rewards=t[k, "rewards"], values=t[k, "values"], terminateds=t[k, "terminateds"],
+                              returns=t[k, "returns"], gamma=GAMMA, lambda_=LAMBDA))
+        if "discounted_returns" in e:
+            k = "discounted_returns"
+            calls.append(dict(kind=k, rewards=t[k, "rewards"], terminateds=t[k, "terminateds"],
+                              returns=t[k, "returns"], gamma=GAMMA))
+        if "eligibility_traces" in e:
+            k = "eligibility_traces"
+            calls.append(dict(kind=k, x=t[k, "x"], dones=t[k, "dones"], traces=t[k, "traces"], gamma=GAMMA,
+                              lambda_=LAMBDA))
+        for k in ("prefix_sum_f32", "prefix_sum_i32"):
+            if k in e:
+                calls.append(dict(kind="episodic_prefix_sum", x=t[k, "x"], dones=t[k, "dones"], out=t[k, "out"]))
+        return lambda: R.rlscan_batch(calls)
 
 
 # ---------------------------------------------------------------------------
@@ -424,14 +465,18 @@ def run_gpu(args):
 
     # one graph per step (one buffer set each), and one graph for a whole
     # round over all sets, so K steps cost K // n_sets + K % n_sets replays.
-    # The eight calls of a step are independent, so a step is captured as
-    # eight parallel branches (fork/join on events); --serial-steps chains
-    # them on one stream instead.
+    # A step is one rlscan_batch request holding the eight calls (one fused
+    # launch).  For reference the same steps are also timed as eight
+    # separate launches, as parallel graph branches (fork/join on events) and
+    # chained on one stream; --parallel-steps / --serial-steps time those as
+    # the step instead.
     branches = [torch.cuda.Stream(device) for _ in names]
 
-    def step_fns(s, parallel):
+    def step_fns(s, how):
+        if how == "batch":
+            return [s.batch_call(R)]
         fns = list(s.calls(R).values())
-        if not parallel:
+        if how == "serial":
             return fns
 
         def step():
@@ -450,10 +495,15 @@ def run_gpu(args):
                 cur.wait_event(j)
         return [step]
 
-    parallel = not args.serial_steps
-    step_graphs = [capture(torch, step_fns(s, parallel), side) for s in sets]
-    round_graph = capture(torch, [f for s in sets for f in step_fns(s, parallel)], side)
-    serial_round = capture(torch, [f for s in sets for f in step_fns(s, False)], side)
+    how = "serial" if args.serial_steps else ("parallel" if args.parallel_steps else "batch")
+    for s in sets:  # eager warm-up of the step as timed (checks the request outside capture)
+        for f in step_fns(s, how):
+            f()
+    R.rlscan_check()
+    step_graphs = [capture(torch, step_fns(s, how), side) for s in sets]
+    round_graph = capture(torch, [f for s in sets for f in step_fns(s, how)], side)
+    ref_rounds = {h: capture(torch, [f for s in sets for f in step_fns(s, h)], side)
+                  for h in ("batch", "parallel", "serial") if h != how}
     torch.cuda.synchronize()
 
     def run_steps(k0, count):
@@ -480,18 +530,20 @@ def run_gpu(args):
         barrier_sync(world)
         step_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
 
-        # the same steps as one chain on one stream, for reference
-        serial_reps = max(1, args.steps // n_sets)
-        for _ in range(2):
-            serial_round.replay()
-        barrier_sync(world)
-        sa, sb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        sa.record(stream)
-        for _ in range(serial_reps):
-            serial_round.replay()
-        sb.record(stream)
-        barrier_sync(world)
-        serial_step_ms = max_over_ranks(sa.elapsed_time(sb), world) / (serial_reps * n_sets)
+        # the same steps launched the other ways, for reference
+        ref_step_ms = {}
+        ref_reps = max(1, args.steps // n_sets)
+        for h, rg in ref_rounds.items():
+            for _ in range(2):
+                rg.replay()
+            barrier_sync(world)
+            sa, sb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            sa.record(stream)
+            for _ in range(ref_reps):
+                rg.replay()
+            sb.record(stream)
+            barrier_sync(world)
+            ref_step_ms[h] = max_over_ranks(sa.elapsed_time(sb), world) / (ref_reps * n_sets)
 
         # per-estimator: back-to-back launches of one estimator over buffer
         # sets whose total exceeds 4x L2
@@ -513,17 +565,33 @@ def run_gpu(args):
             reps = max(3, -(-max(args.steps, 200) // len(fns)))
             for _ in range(2):
                 g.replay()
-            barrier_sync(world)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(reps):
-                g.replay()
-            b.record(stream)
-            barrier_sync(world)
-            ms = max_over_ranks(a.elapsed_time(b), world)
+            samples = []
+            for _ in range(REPEATS):  # median over repeats of >= 200 back-to-back launches
+                barrier_sync(world)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                b.record(stream)
+                barrier_sync(world)
+                samples.append(1000.0 * max_over_ranks(a.elapsed_time(b), world) / (reps * len(fns)))
+            us = float(np.median(samples))
             launches = reps * len(fns)
-            us = 1000.0 * ms / launches
+            # one call on an idle stream, host launch included (binding + C ABI
+            # + kernel), median over ISOLATED_SAMPLES calls
+            iso = []
+            for i in range(ISOLATED_SAMPLES):
+                f = fns[i % len(fns)]
+                torch.cuda.synchronize()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                f()
+                b.record(stream)
+                torch.cuda.synchronize()
+                iso.append(1000.0 * a.elapsed_time(b))
             per_est[est] = {"us_per_launch": us, "bytes_per_launch": nbytes, "launches": launches,
+                            "repeats": REPEATS, "us_per_launch_range": [min(samples), max(samples)],
+                            "isolated_call_us": float(np.median(iso)),
                             "env_steps_per_s": E_ENVS * T_STEPS / (us * 1e-6),
                             "gb_per_s": nbytes / (us * 1e-6) / 1e9}
             del g
@@ -579,9 +647,13 @@ def run_gpu(args):
         threads = os.cpu_count() or 1
         rows = min(E_ENVS, 512 * threads)
         v, calls, el = time_oracle(host, rows, threads, min_seconds=args.cpu_seconds)
+        v1, calls1, el1 = time_oracle(host, 64, 1, min_seconds=max(1.0, args.cpu_seconds / 4))
         cpu = {"value": v, "unit": "env-steps/s", "cores": threads, "kind": "oracle",
                "sample": f"{calls} passes of the fp64 oracle over {rows} of 4096 rows x 128 steps, all 8 "
-                         f"estimator calls, rows split over {threads} host threads, {el:.1f} s"}
+                         f"estimator calls, rows split over {threads} host threads, {el:.1f} s",
+               "single_thread": {"value": v1, "cores": 1,
+                                 "sample": f"{calls1} passes over 64 rows x 128 steps, all 8 estimator "
+                                           f"calls, one thread, {el1:.1f} s"}}
 
     if rank != 0:
         return 0
@@ -602,7 +674,10 @@ def run_gpu(args):
     line = {
         "metric": "env-steps/s and HBM GB/s (% of peak) per estimator at 4096x128 fp32",
         "value": value, "unit": "env-steps/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": step_ms / args.steps, "ms_per_step_serial_chain": serial_step_ms,
+        "ms_per_step": step_ms / args.steps,
+        "ms_per_step_other_launch_schemes": {
+            {"batch": "one_fused_launch", "parallel": "eight_launches_parallel_branches",
+             "serial": "eight_launches_one_stream"}[h]: v for h, v in ref_step_ms.items()},
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 (int32 for the integer prefix sum)", "data": "synthetic",
         "config": {"workload": WORKLOAD, "num_envs": E_ENVS, "seq_len": T_STEPS,
@@ -611,8 +686,9 @@ def run_gpu(args):
                    "l2": f"inputs larger than L2: {n_sets} rotating buffer sets, "
                          f"{n_sets * per_set_bytes / 2**20:.0f} MiB > 4x126 MB",
                    "timing": "CUDA events around CUDA-graph replays (a graph holds a round of steps)",
-                   "step": ("the eight independent calls of a step as parallel graph branches"
-                            if parallel else "the eight calls of a step chained on one stream"),
+                   "step": {"batch": "the eight calls of a step as one rlscan_batch request (one fused launch)",
+                            "parallel": "the eight calls of a step as parallel graph branches",
+                            "serial": "the eight calls of a step chained on one stream"}[how],
                    "parallelism": f"replicas x{world}, each rank its own batch"},
         "hbm_gb_per_s_step": STEP_BYTES_PER_ENV_STEP * E_ENVS * T_STEPS * args.steps / (step_ms * 1e-3) / 1e9,
         "per_estimator": per_est,
@@ -625,10 +701,10 @@ def run_gpu(args):
                      "algorithmic_bytes": d["bytes_per_launch"]},
         "e2e": {"value": job_value(world, e2e_steps, e2e_ms), "unit": "env-steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "path": "per step: pinned host -> device copy of its inputs, the eight C-ABI calls, "
-                        "device -> pinned host copy of its outputs; copy-in / compute / copy-out "
+                "path": "per step: pinned host -> device copy of its inputs, the step as timed above "
+                        "(C ABI), device -> pinned host copy of its outputs; copy-in / compute / copy-out "
                         "on three streams"},
-        "gpu_launches": args.steps * len(names),
+        "gpu_launches": args.steps * (1 if how == "batch" else len(names)),
         "clocks": clk,
         "cpu_baseline": cpu,
     }
@@ -666,6 +742,78 @@ def run_reference(args):
     return 0
 
 
+# size grid of the four single-input-family estimators, plus the long-row case
+SWEEP_E = (256, 4096, 65536)
+SWEEP_T = (32, 128, 1024, 4096)
+SWEEP_LONG = (16, 262144)
+SWEEP_EST = ("gae", "discounted_returns", "eligibility_traces", "prefix_sum_f32")
+
+
+def run_sweep(args):
+    """Per-launch time of GAE, discounted returns, eligibility traces and the
+    f32 prefix sum over E x T in {256, 4096, 65536} x {32, 128, 1024, 4096}
+    and at 16 x 262144 (gamma 0.999, dones 1e-4).  Inputs drawn on the
+    device; each point launches back to back in a CUDA graph over rotating
+    buffer sets (>= 4x L2), median of five repeats.  One JSON line per point."""
+    import torch
+    from linear_recurrence_scans_02_b200 import rlscan as R
+    from linear_recurrence_scans_02_b200 import workloads as W
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peak, peak_kind = measured_hbm_peak()
+    side = torch.cuda.Stream(device)
+    stream = torch.cuda.current_stream(device)
+    points = [(E, T) for E in SWEEP_E for T in SWEEP_T] + [SWEEP_LONG]
+    for (E, T) in points:
+        long_row = (E, T) == SWEEP_LONG
+        gamma, p_done = (0.999, 1e-4) if long_row else (GAMMA, P_DONE)
+        for est in SWEEP_EST:
+            nbytes = bytes_per_env_step(est) * E * T
+            nset = min(64, max(2, -(-ROTATE_BYTES // nbytes)))
+            fns = []
+            for k in range(nset):
+                fam = "gae" if est in ("gae", "discounted_returns") else "trace"
+                d = W.device_inputs(fam, E, T, seed=1000 + k, device=device, p_done=p_done)
+                out = torch.empty(E, T, device=device)
+                if est == "gae":
+                    fns.append(lambda d=d, o=out: R.rlscan_gae(d["rewards"], d["values"], d["terminateds"], None,
+                                                               None, None, o, gamma, LAMBDA))
+                elif est == "discounted_returns":
+                    fns.append(lambda d=d, o=out: R.rlscan_discounted_returns(d["rewards"], d["terminateds"], None,
+                                                                              None, None, o, gamma))
+                elif est == "eligibility_traces":
+                    fns.append(lambda d=d, o=out: R.rlscan_eligibility_traces(d["x"], d["dones"], o, gamma, LAMBDA))
+                else:
+                    fns.append(lambda d=d, o=out: R.rlscan_episodic_prefix_sum(d["x"], d["dones"], o))
+            for f in fns:
+                f()
+            R.rlscan_check()
+            g = capture(torch, fns, side)
+            reps = max(3, -(-200 // len(fns)))
+            g.replay()
+            samples = []
+            for _ in range(REPEATS):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                b.record(stream)
+                torch.cuda.synchronize()
+                samples.append(1000.0 * a.elapsed_time(b) / (reps * len(fns)))
+            R.rlscan_check()
+            us = float(np.median(samples))
+            plan = R.rlscan_plan(E, T)
+            print(json.dumps({"sweep": est, "num_envs": E, "seq_len": T, "us_per_launch": us,
+                              "bytes_per_launch": nbytes, "gb_per_s": nbytes / (us * 1e-6) / 1e9,
+                              "frac_of_hbm_peak": nbytes / (us * 1e-6) / 1e9 / peak, "peak": peak,
+                              "peak_source": peak_kind, "env_steps_per_s": E * T / (us * 1e-6),
+                              "buffer_sets": len(fns), "launches_per_repeat": reps * len(fns),
+                              "plan": plan}), flush=True)
+            del g, fns
+            torch.cuda.empty_cache()
+    return 0
+
+
 def run_profile_case(args):
     """Small case for ncu: `n` eager launches of every estimator (and of the
     calls timed beside the step), one [4096, 128] buffer set (about 110 MB on
@@ -676,7 +824,8 @@ def run_profile_case(args):
     bs = BufferSet(torch, torch.device("cuda", 0), PLANES)
     bs.fill_from_host(host_inputs(seed=0))
     calls = bs.calls(R)
-    for est in (args.profile_only.split(",") if args.profile_only else list(ESTIMATORS)):
+    calls["batch"] = bs.batch_call(R)  # the step's eight calls as one request
+    for est in (args.profile_only.split(",") if args.profile_only else list(ESTIMATORS) + ["batch"]):
         for _ in range(args.profile_launches):
             calls[est]()
         torch.cuda.synchronize()
@@ -694,18 +843,24 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--serial-steps", action="store_true",
-                    help="chain a step's eight calls on one stream instead of parallel graph branches")
+                    help="time a step as its eight calls chained on one stream (not one batch request)")
+    ap.add_argument("--parallel-steps", action="store_true",
+                    help="time a step as its eight calls in parallel graph branches (not one batch request)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--profile-launches", type=int, default=0,
                     help="run N eager launches of each estimator and exit (small case for ncu)")
     ap.add_argument("--profile-only", default="", help="comma-separated estimators for --profile-launches")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time four estimators over the E x T size grid and 16 x 262144, one JSON line per point")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
     if args.profile_launches > 0:
         return run_profile_case(args)
+    if args.sweep:
+        return run_sweep(args)
     try:
         return run_gpu(args)
     finally:

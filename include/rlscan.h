@@ -332,6 +332,71 @@ RLSCAN_API int rlscan_episodic_prefix_sum_ex(const void *x, int dtype, const flo
                                              cudaStream_t stream);
 
 /*
+ * Several independent estimator calls in one request (no counterpart on the
+ * pages, whose kernels each take one call): an RL update often needs several
+ * estimators, or one estimator over several reward streams, on one batch.
+ * Each rlscan_call describes one call of an entry point above; rlscan_batch
+ * validates every call as that entry point would, then launches every call
+ * whose rows fit whole in 1024-element tiles (row-major, 1024 a multiple of
+ * T, every kind below, A == 1 for Retrace) as ONE fused kernel, each block
+ * running one tile of one call, and each remaining call by its own launch.
+ * Results are those of the individual calls, bit for bit.
+ *
+ * kind and argument slots (the pointer arguments of the entry point, in its
+ * order; unused slots NULL):
+ *   RLSCAN_KIND_GAE                 in: rewards values terminateds truncateds bootstrap_values last_values
+ *                                   out: advantages
+ *   RLSCAN_KIND_GAE_WITH_RETURNS    in: as GAE; out: advantages returns
+ *   RLSCAN_KIND_VTRACE              in: log_rhos rewards values terminateds truncateds bootstrap_values
+ *                                       last_values; out: vs pg_advantages
+ *   RLSCAN_KIND_RETRACE             in: rewards q_values next_q_values_all next_target_probs log_rhos
+ *                                       terminateds truncateds; out: q_ret
+ *   RLSCAN_KIND_LAMBDA_RETURNS      in: as GAE; out: returns
+ *   RLSCAN_KIND_DISCOUNTED_RETURNS  in: rewards terminateds truncateds bootstrap_values last_values;
+ *                                   out: returns
+ *   RLSCAN_KIND_ELIGIBILITY_TRACES  in: x dones; out: traces
+ *   RLSCAN_KIND_EPISODIC_PREFIX_SUM in: x dones; out: out  (dtype RLSCAN_F32 or RLSCAN_I32)
+ * Scalars a kind does not take are ignored (lambda_ for discounted returns,
+ * rho_bar and c_bar outside V-Trace and Retrace, A outside Retrace, dtype
+ * outside the prefix sum).  options: as for the _ex entry points.
+ *
+ * The calls run concurrently: no call's output may overlap any other
+ * call's inputs or outputs (RLSCAN_ERR_INVALID_ARG).  ws / ws_bytes: one
+ * workspace, at least the largest rlscan_workspace_bytes of the calls that
+ * need one (they run one after another on `stream`).  ncalls == 0 is a no-op.
+ * Errors: a nonzero return names the first failing call in
+ * rlscan_last_error(); nothing was enqueued unless it is RLSCAN_ERR_CUDA
+ * from a launch.
+ */
+typedef enum rlscan_kind {
+    RLSCAN_KIND_GAE = 1,
+    RLSCAN_KIND_GAE_WITH_RETURNS = 2,
+    RLSCAN_KIND_VTRACE = 3,
+    RLSCAN_KIND_RETRACE = 4,
+    RLSCAN_KIND_LAMBDA_RETURNS = 5,
+    RLSCAN_KIND_DISCOUNTED_RETURNS = 6,
+    RLSCAN_KIND_ELIGIBILITY_TRACES = 7,
+    RLSCAN_KIND_EPISODIC_PREFIX_SUM = 8
+} rlscan_kind;
+
+#define RLSCAN_CALL_MAX_IN 8
+#define RLSCAN_CALL_MAX_OUT 2
+/* Largest number of calls in one rlscan_batch request. */
+#define RLSCAN_BATCH_MAX 16
+
+typedef struct rlscan_call {
+    int kind;       /* rlscan_kind */
+    int dtype;      /* RLSCAN_KIND_EPISODIC_PREFIX_SUM: RLSCAN_F32 or RLSCAN_I32 */
+    unsigned options;
+    int64_t E, T, A;
+    float gamma, lambda_, rho_bar, c_bar;
+    const void *in[RLSCAN_CALL_MAX_IN];
+    void *out[RLSCAN_CALL_MAX_OUT];
+} rlscan_call;
+
+RLSCAN_API int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Workspace size in bytes that any entry point above needs for an [E, T]
  * problem (any A); 0 if no call of that shape needs one.  Negative or
  * overflowing shapes return 0 and the compute call then rejects them.

@@ -1,0 +1,122 @@
+// batch.cuh - one launch for several independent estimator calls.
+//
+// A fused grid is the concatenation of the calls' tile grids: block b runs
+// tile b - tile_begin of the call whose range holds b, through the same tile
+// body (and so the same arithmetic, bit for bit) as that call's own launch.
+// Only calls whose plan is the 128-thread x 8-element tile without the
+// look-back are fused, so every block of the grid has the same shape.
+#pragma once
+
+#include "estimators.cuh"
+
+namespace rlscan {
+
+enum FusedKind {
+    kFkGae = 0,
+    kFkGaeReturns,
+    kFkVtrace,
+    kFkRetrace1,
+    kFkLambda,
+    kFkReturns,
+    kFkTraces,
+    kFkPrefixF32,
+    kFkPrefixI32,
+    kNumFusedKinds
+};
+
+template <class Est>
+struct FusedKindOf {
+    static constexpr int value = -1;
+};
+template <>
+struct FusedKindOf<GaeEst> {
+    static constexpr int value = kFkGae;
+};
+template <>
+struct FusedKindOf<GaeReturnsEst> {
+    static constexpr int value = kFkGaeReturns;
+};
+template <>
+struct FusedKindOf<VtraceEst> {
+    static constexpr int value = kFkVtrace;
+};
+template <>
+struct FusedKindOf<RetraceEst<false>> {
+    static constexpr int value = kFkRetrace1;
+};
+template <>
+struct FusedKindOf<LambdaReturnsEst> {
+    static constexpr int value = kFkLambda;
+};
+template <>
+struct FusedKindOf<ReturnsEst> {
+    static constexpr int value = kFkReturns;
+};
+template <>
+struct FusedKindOf<TracesEst> {
+    static constexpr int value = kFkTraces;
+};
+template <>
+struct FusedKindOf<PrefixF32Est> {
+    static constexpr int value = kFkPrefixF32;
+};
+template <>
+struct FusedKindOf<PrefixI32Est> {
+    static constexpr int value = kFkPrefixI32;
+};
+
+constexpr int kFusedNT = 128; // the 1024-element tile: 128 threads x 8 elements
+constexpr int kFusedV = 8;
+constexpr int kFusedParamBytes = 128;
+constexpr int kFusedMax = 16;
+
+struct FusedItem {
+    alignas(16) unsigned char params[kFusedParamBytes]; // the call's Est::Params
+    Geometry g;
+    long long tile_begin; // first block of this call in the fused grid
+    int kind;             // FusedKind
+    int mode;             // kModeWarp or kModeBlock
+};
+
+struct FusedBatch {
+    FusedItem item[kFusedMax];
+    int n;
+};
+
+template <class Est, int kMode>
+__device__ __forceinline__ void fused_tile(const FusedItem &it, long long block, unsigned char *smem) {
+    const auto &P = *reinterpret_cast<const typename Est::Params *>(it.params);
+    const Lookback lb{nullptr, nullptr, 0u, -1}; // no look-back in a fused launch
+    tile_scan_body<Est, kFusedNT, kFusedV, kMode>(P, it.g, lb, block, smem);
+}
+
+template <class Est>
+__device__ __forceinline__ void fused_tile_any_mode(const FusedItem &it, long long block, unsigned char *smem) {
+    if (it.mode == kModeWarp)
+        fused_tile<Est, kModeWarp>(it, block, smem);
+    else
+        fused_tile<Est, kModeBlock>(it, block, smem);
+}
+
+__global__ void __launch_bounds__(kFusedNT) fused_tile_kernel(const __grid_constant__ FusedBatch b) {
+    extern __shared__ __align__(128) unsigned char dyn_smem[];
+    int idx = 0;
+    for (int i = 1; i < b.n; ++i)
+        if ((long long)blockIdx.x >= b.item[i].tile_begin) idx = i;
+    const FusedItem &it = b.item[idx];
+    const long long block = (long long)blockIdx.x - it.tile_begin;
+    switch (it.kind) {
+    case kFkGae: fused_tile_any_mode<GaeEst>(it, block, dyn_smem); break;
+    case kFkGaeReturns: fused_tile_any_mode<GaeReturnsEst>(it, block, dyn_smem); break;
+    case kFkVtrace: fused_tile_any_mode<VtraceEst>(it, block, dyn_smem); break;
+    case kFkRetrace1: fused_tile_any_mode<RetraceEst<false>>(it, block, dyn_smem); break;
+    case kFkLambda: fused_tile_any_mode<LambdaReturnsEst>(it, block, dyn_smem); break;
+    case kFkReturns: fused_tile_any_mode<ReturnsEst>(it, block, dyn_smem); break;
+    case kFkTraces: fused_tile_any_mode<TracesEst>(it, block, dyn_smem); break;
+    case kFkPrefixF32: fused_tile_any_mode<PrefixF32Est>(it, block, dyn_smem); break;
+    case kFkPrefixI32: fused_tile_any_mode<PrefixI32Est>(it, block, dyn_smem); break;
+    default: break;
+    }
+}
+
+} // namespace rlscan

@@ -18,7 +18,7 @@
 #include <string>
 
 #include "../../include/rlscan.h"
-#include "estimators.cuh"
+#include "batch.cuh"
 
 namespace rlscan {
 namespace {
@@ -122,8 +122,11 @@ Plan make_plan_tiles(long long E, long long T, long long actions) {
         break;
     }
     // rows span tiles (long or odd-length rows, or too few rows to fill the
-    // GPU): 1024-element tiles with the look-back, 512 when that gives too few
-    p.cfg = ceil_div(n, kCfgTile[C1024]) >= kMinTiles ? C1024 : C512;
+    // GPU): look-back over 2048-element tiles (fewer tiles per row, so a
+    // shorter chain of carries), 1024 or 512 when that gives too few tiles
+    p.cfg = ceil_div(n, kCfgTile[C2048]) >= kMinTiles
+                ? C2048
+                : (ceil_div(n, kCfgTile[C1024]) >= kMinTiles ? C1024 : C512);
     p.ntiles = ceil_div(n, kCfgTile[p.cfg]);
     p.lookback = p.ntiles > 1 && (kCfgTile[p.cfg] % T != 0);
     return p;
@@ -213,6 +216,22 @@ int require(const void *p, const char *name) {
     } while (0)
 
 // ---------------------------------------------------------------------------
+// Batch requests (rlscan_batch).  While a request is being served on this
+// thread, the launch helpers either only validate (dry pass: every call is
+// checked before anything is enqueued) or record fusable calls into one
+// fused launch and launch the others as usual.
+// ---------------------------------------------------------------------------
+enum BatchPass { kBatchDry = 1, kBatchRecord = 2 };
+struct BatchState {
+    int pass;
+    FusedBatch fb;
+    long long tiles;
+};
+thread_local BatchState *g_batch = nullptr;
+
+bool batch_dry() { return g_batch != nullptr && g_batch->pass == kBatchDry; }
+
+// ---------------------------------------------------------------------------
 // Launch
 // ---------------------------------------------------------------------------
 template <class Est, int NT, int V, int kMode>
@@ -273,6 +292,23 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
         lb.slots = reinterpret_cast<TileSlot *>(static_cast<char *>(ws) + sizeof(WsHeader));
         lb.withhold = g_withhold.load();
     }
+    if (batch_dry()) return ok();
+    if constexpr (FusedKindOf<Est>::value >= 0) {
+        if (g_batch != nullptr && plan.cfg == C1024 && plan.mode != kModeLookback && actions == 1 &&
+            g_batch->fb.n < kFusedMax) {
+            static_assert(sizeof(typename Est::Params) <= kFusedParamBytes, "params fit a fused item");
+            static_assert(kCfgThreads[C1024] == kFusedNT && kCfgTile[C1024] == kFusedNT * kFusedV, "fused tile");
+            FusedItem &it = g_batch->fb.item[g_batch->fb.n++];
+            std::memset(it.params, 0, sizeof it.params);
+            std::memcpy(it.params, &P, sizeof P);
+            it.g = g;
+            it.tile_begin = g_batch->tiles;
+            it.kind = FusedKindOf<Est>::value;
+            it.mode = plan.mode;
+            g_batch->tiles += plan.ntiles;
+            return ok();
+        }
+    }
     const size_t smem = actions > 1 ? multi_smem_bytes(plan.cfg, actions) : 0;
     cudaError_t e;
     switch (plan.cfg) {
@@ -313,6 +349,7 @@ int run_multi(const char *name, const typename Est::Params &P, long long E, long
         lb.slots = reinterpret_cast<TileSlot *>(static_cast<char *>(ws) + sizeof(WsHeader));
         lb.withhold = g_withhold.load();
     }
+    if (batch_dry()) return ok();
     const size_t smem = multi_smem_bytes(plan.cfg, actions);
     cudaError_t e;
     switch (plan.cfg) {
@@ -363,6 +400,7 @@ template <class Est>
 int run_time_major(const char *name, const typename Est::Params &P, long long E, long long T, cudaStream_t stream) {
     if (E > (long long)INT_MAX / (kTmV + 1))
         return fail(RLSCAN_ERR_UNSUPPORTED, "%s: the time-major layout takes E <= %d", name, INT_MAX / (kTmV + 1));
+    if (batch_dry()) return ok();
     const TmPlan tp = tm_plan(E, T);
     Geometry g;
     g.n = E * T;
@@ -846,6 +884,128 @@ int rlscan_plan(int64_t E, int64_t T, int64_t actions, int64_t *tile_elems, int 
     if (threads) *threads = kCfgThreads[p.cfg];
     if (lookback) *lookback = p.lookback ? 1 : 0;
     if (num_tiles) *num_tiles = p.ntiles;
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// rlscan_batch
+// ---------------------------------------------------------------------------
+
+// Byte extent of argument slot `slot` of a call (its input when in_slot,
+// else its output); 0 for slots the kind does not have.
+static size_t call_slot_bytes(const rlscan_call &c, bool in_slot, int slot) {
+    const size_t plane = (size_t)(c.E * c.T) * 4u, row = (size_t)c.E * 4u;
+    if (!in_slot) {
+        const int nout = (c.kind == RLSCAN_KIND_GAE_WITH_RETURNS || c.kind == RLSCAN_KIND_VTRACE) ? 2 : 1;
+        return slot < nout ? plane : 0;
+    }
+    switch (c.kind) {
+    case RLSCAN_KIND_GAE:
+    case RLSCAN_KIND_GAE_WITH_RETURNS:
+    case RLSCAN_KIND_LAMBDA_RETURNS: return slot < 5 ? plane : (slot == 5 ? row : 0);
+    case RLSCAN_KIND_VTRACE: return slot < 6 ? plane : (slot == 6 ? row : 0);
+    case RLSCAN_KIND_RETRACE: return (slot == 2 || slot == 3) ? plane * (size_t)(c.A > 0 ? c.A : 1) : (slot < 7 ? plane : 0);
+    case RLSCAN_KIND_DISCOUNTED_RETURNS: return slot < 4 ? plane : (slot == 4 ? row : 0);
+    case RLSCAN_KIND_ELIGIBILITY_TRACES:
+    case RLSCAN_KIND_EPISODIC_PREFIX_SUM: return slot < 2 ? plane : 0;
+    default: return 0;
+    }
+}
+
+static int call_dispatch(const rlscan_call &c, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    const float *const *in = reinterpret_cast<const float *const *>(c.in);
+    float *const *out = reinterpret_cast<float *const *>(c.out);
+    switch (c.kind) {
+    case RLSCAN_KIND_GAE:
+        return rlscan_gae_ex(in[0], in[1], in[2], in[3], in[4], in[5], out[0], c.E, c.T, c.gamma, c.lambda_,
+                             c.options, ws, ws_bytes, stream);
+    case RLSCAN_KIND_GAE_WITH_RETURNS:
+        return rlscan_gae_with_returns_ex(in[0], in[1], in[2], in[3], in[4], in[5], out[0], out[1], c.E, c.T,
+                                          c.gamma, c.lambda_, c.options, ws, ws_bytes, stream);
+    case RLSCAN_KIND_VTRACE:
+        return rlscan_vtrace_ex(in[0], in[1], in[2], in[3], in[4], in[5], in[6], out[0], out[1], c.E, c.T, c.gamma,
+                                c.lambda_, c.rho_bar, c.c_bar, c.options, ws, ws_bytes, stream);
+    case RLSCAN_KIND_RETRACE:
+        return rlscan_retrace_ex(in[0], in[1], in[2], in[3], in[4], in[5], in[6], out[0], c.E, c.T, c.A, c.gamma,
+                                 c.lambda_, c.c_bar, c.options, ws, ws_bytes, stream);
+    case RLSCAN_KIND_LAMBDA_RETURNS:
+        return rlscan_lambda_returns_ex(in[0], in[1], in[2], in[3], in[4], in[5], out[0], c.E, c.T, c.gamma,
+                                        c.lambda_, c.options, ws, ws_bytes, stream);
+    case RLSCAN_KIND_DISCOUNTED_RETURNS:
+        return rlscan_discounted_returns_ex(in[0], in[1], in[2], in[3], in[4], out[0], c.E, c.T, c.gamma,
+                                            c.options, ws, ws_bytes, stream);
+    case RLSCAN_KIND_ELIGIBILITY_TRACES:
+        return rlscan_eligibility_traces_ex(in[0], in[1], out[0], c.E, c.T, c.gamma, c.lambda_, c.options, ws,
+                                            ws_bytes, stream);
+    case RLSCAN_KIND_EPISODIC_PREFIX_SUM:
+        return rlscan_episodic_prefix_sum_ex(c.in[0], c.dtype, in[1], c.out[0], c.E, c.T, c.options, ws, ws_bytes,
+                                             stream);
+    default: return fail(RLSCAN_ERR_INVALID_ARG, "unknown kind %d", c.kind);
+    }
+}
+
+// Runs every call of the request in the given pass; the first failure is
+// reported with its call index.
+static int batch_pass(BatchState &st, const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+    g_batch = &st;
+    for (int i = 0; i < ncalls; ++i) {
+        const int rc = call_dispatch(calls[i], ws, ws_bytes, stream);
+        if (rc != RLSCAN_OK) {
+            g_batch = nullptr;
+            const std::string msg = g_last_error;
+            return fail(rc, "call %d: %s", i, msg.c_str());
+        }
+    }
+    g_batch = nullptr;
+    return RLSCAN_OK;
+}
+
+int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    if (ncalls < 0 || ncalls > RLSCAN_BATCH_MAX)
+        return fail(RLSCAN_ERR_INVALID_ARG, "ncalls must be in [0, %d] (got %d)", RLSCAN_BATCH_MAX, ncalls);
+    if (ncalls == 0) return ok();
+    if (calls == nullptr) return fail(RLSCAN_ERR_INVALID_ARG, "calls must not be NULL");
+    if (g_batch != nullptr) return fail(RLSCAN_ERR_INVALID_ARG, "rlscan_batch is not reentrant");
+    // 1. every call checked as its entry point would, nothing enqueued
+    BatchState st{};
+    st.pass = kBatchDry;
+    RLSCAN_TRY(batch_pass(st, calls, ncalls, ws, ws_bytes, stream));
+    // 2. calls run concurrently: no output of one may overlap anything of another
+    for (int i = 0; i < ncalls; ++i) {
+        for (int j = i + 1; j < ncalls; ++j) {
+            Span ins[2 * RLSCAN_CALL_MAX_IN], outs[2 * RLSCAN_CALL_MAX_OUT];
+            int ni = 0, no = 0;
+            const rlscan_call *pair[2] = {&calls[i], &calls[j]};
+            for (const rlscan_call *c : pair) {
+                const bool empty = c->E == 0 || c->T == 0;
+                for (int k = 0; k < RLSCAN_CALL_MAX_IN; ++k)
+                    ins[ni++] = {empty ? nullptr : c->in[k], call_slot_bytes(*c, true, k), "an input"};
+                for (int k = 0; k < RLSCAN_CALL_MAX_OUT; ++k)
+                    outs[no++] = {empty ? nullptr : c->out[k], call_slot_bytes(*c, false, k), "an output"};
+            }
+            if (check_aliasing(ins, ni, outs, no) != RLSCAN_OK) {
+                const std::string msg = g_last_error;
+                return fail(RLSCAN_ERR_INVALID_ARG, "calls %d and %d: %s", i, j, msg.c_str());
+            }
+        }
+    }
+    // 3. launch: unfusable calls one by one, the rest recorded for one launch
+    st = BatchState{};
+    st.pass = kBatchRecord;
+    RLSCAN_TRY(batch_pass(st, calls, ncalls, ws, ws_bytes, stream));
+    if (st.fb.n == 0) return ok();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)st.tiles);
+    cfg.blockDim = dim3(kFusedNT);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_tile_kernel, st.fb);
+    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "rlscan_batch: fused launch failed: %s", cudaGetErrorString(e));
     return ok();
 }
 

@@ -64,6 +64,17 @@ __device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned *p) {
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// Four relaxed 32-bit loads in one instruction (no ordering among them).
+__device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+// With a preceding relaxed load, the acquire pattern of the PTX memory model.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -301,15 +312,24 @@ __device__ __forceinline__ long long elem_row(const RowMasks &m, int k) {
     return kFast ? m.row0 : row_of(m, k);
 }
 
-// Single-lane decoupled look-back.  Publishes this tile's aggregate (or its
-// inclusive value when it needs no carry), walks back over earlier tiles
-// composing their aggregates until it meets an inclusive value or an
-// aggregate that cuts the chain (a == 0), publishes its own inclusive value
-// and returns the carry into this tile.
+// Warp-wide decoupled look-back, called by all 32 lanes of one warp.
+// Lane 0 publishes this tile's aggregate (or its inclusive value when it
+// needs no carry, or when its own chain is cut).  The warp then inspects
+// 32 x kLbPerLane earlier tiles at once, lane i reading tiles
+// base - i kLbPerLane - m, m = 0 .. kLbPerLane - 1 (nearest first): when one
+// of them holds an inclusive value, the carry is that value passed through
+// the aggregates of the nearer tiles; otherwise all hold aggregates, whose
+// composition is folded in before the next window.  A tile whose own chain
+// is cut always publishes an inclusive value, so the walk ends at the row's
+// first tile at the latest.  Lane 0 then publishes this tile's inclusive
+// value.  Every wait is bounded; a wait that gives up sets the device error
+// word and the walk ends as if the carry were zero.
+constexpr int kLbPerLane = 1;
+
 template <class AT, class BT>
-__device__ BT lookback_carry(const Lookback &lb, long long j, bool needs_carry, AT ta, BT tb) {
+__device__ BT lookback_carry(const Lookback &lb, long long j, bool needs_carry, AT ta, BT tb, int lane) {
     TileSlot *me = lb.slots + j;
-    const bool publish = (j != lb.withhold);
+    const bool publish = (j != lb.withhold) && lane == 0;
     if (!needs_carry) {
         if (publish) {
             st_relaxed_gpu(&me->x, to_bits(tb));
@@ -328,38 +348,82 @@ __device__ BT lookback_carry(const Lookback &lb, long long j, bool needs_carry, 
             st_release_gpu(&me->status, 1u);
         }
     }
-    AT acc_a = identity_a(ta);
+    constexpr int M = kLbPerLane;
+    AT acc_a = identity_a(ta); // composition of the aggregates walked so far
     BT acc_b = identity_b(tb);
     BT carry = identity_b(tb);
-    for (long long k = j - 1;; --k) {
-        if (k < 0) { // unreachable: scan-order tile 0 never needs a carry
-            atomicOr(&g_device_error, kErrLookbackTimeout);
+    for (long long base = j - 1;; base -= 32 * M) {
+        const long long k0 = base - (long long)lane * M;
+        // statuses by relaxed loads, all in flight together; then one fence
+        // (relaxed load + fence = acquire) before the published values are read
+        unsigned st[M];
+#pragma unroll
+        for (int m = 0; m < M; ++m) st[m] = (k0 - m >= 0) ? ld_relaxed_gpu(&lb.slots[k0 - m].status) : 2u;
+        bool gave_up = false;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            unsigned ns = 32, polls = 0;
+            while (st[m] == 0u) {
+                if (++polls > lb.spin_limit) {
+                    gave_up = true;
+                    break;
+                }
+                __nanosleep(ns);
+                if (ns < 256u) ns <<= 1;
+                st[m] = ld_relaxed_gpu(&lb.slots[k0 - m].status);
+            }
+        }
+        if (__any_sync(kFullMask, gave_up)) {
+            if (lane == 0) atomicOr(&g_device_error, kErrLookbackTimeout);
             carry = acc_b;
             break;
         }
-        const TileSlot *s = lb.slots + k;
-        unsigned st = ld_acquire_gpu(&s->status);
-        unsigned ns = 32, polls = 0;
-        while (st == 0u) {
-            if (++polls > lb.spin_limit) break;
-            __nanosleep(ns);
-            if (ns < 1024u) ns <<= 1;
-            st = ld_acquire_gpu(&s->status);
+        fence_acq_rel_gpu();
+        uint4 slot[M];
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            slot[m] = (k0 - m >= 0) ? ld_relaxed_gpu_v4(&lb.slots[k0 - m]) : make_uint4(0u, 0u, 0u, 0u);
+        // this lane's M tiles composed nearest-outermost, stopping at the
+        // first inclusive value or cut (a == 0: the map ignores what came before)
+        AT la = identity_a(ta);
+        BT lb_ = identity_b(tb);
+        bool stop = false;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            if (stop) break;
+            const long long k = k0 - m;
+            AT ka;
+            BT kb;
+            if (k < 0) { // nothing flows in from before the array (unreachable in a well-formed walk)
+                ka = AT(0);
+                kb = identity_b(tb);
+            } else if (st[m] == 2u) { // an inclusive value: the map x -> x_k
+                ka = AT(0);
+                kb = from_bits(slot[m].w, tb);
+            } else { // an aggregate (a, b), published before status 1
+                ka = from_bits(slot[m].y, ta);
+                kb = from_bits(slot[m].z, tb);
+            }
+            combine(la, lb_, ka, kb);
+            stop = (ka == AT(0));
         }
-        if (st == 0u) { // gave up: report, and continue as if the carry were zero
-            atomicOr(&g_device_error, kErrLookbackTimeout);
-            carry = acc_b;
-            break;
+        const unsigned stops = __ballot_sync(kFullMask, stop);
+        const int last = stops ? __ffs(stops) - 1 : 31;
+        if (lane > last) { // farther than the nearest stop: contributes nothing
+            la = identity_a(ta);
+            lb_ = identity_b(tb);
         }
-        if (st == 2u) {
-            BT xk = from_bits(ld_relaxed_gpu(&s->x), tb);
-            carry = apply_pair(acc_a, acc_b, xk);
-            break;
+        // ordered composition over lanes 0..last: lane 0 (nearest) applied last
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const AT oa = __shfl_down_sync(kFullMask, la, d);
+            const BT ob = __shfl_down_sync(kFullMask, lb_, d);
+            if (lane + d < 32) combine(la, lb_, oa, ob);
         }
-        AT ak = from_bits(ld_relaxed_gpu(&s->a), ta);
-        BT bk = from_bits(ld_relaxed_gpu(&s->b), tb);
-        combine(acc_a, acc_b, ak, bk);
-        if (ak == AT(0)) { // the earlier chain is cut here
+        la = __shfl_sync(kFullMask, la, 0);
+        lb_ = __shfl_sync(kFullMask, lb_, 0);
+        combine(acc_a, acc_b, la, lb_);
+        if (stops) { // the composed map starts from a cut: its b is the carry
             carry = acc_b;
             break;
         }
@@ -728,9 +792,11 @@ constexpr int kModeBlock = 0;
 constexpr int kModeLookback = 1;
 constexpr int kModeWarp = 2;
 
+// The body of one tile, for a launch whose block `block` owns that tile
+// (the tile kernel below, or one part of a fused launch).
 template <class Est, int NT, int V, int kMode>
-__global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Params P, const Geometry g,
-                                                       const Lookback lb) {
+__device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, const Geometry &g, const Lookback &lb,
+                                               const long long block, unsigned char *dyn_smem) {
     using AT = typename Est::AT;
     using BT = typename Est::BT;
     constexpr bool kBwd = Est::kBackward;
@@ -743,7 +809,6 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
     __shared__ BT s_wb[NW];
     __shared__ BT s_wx[NW];
     __shared__ long long s_tile;
-    extern __shared__ __align__(128) unsigned char dyn_smem[];
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -751,12 +816,12 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
 
     // Start this tile's DRAM reads before waiting for the previous grid on
     // the stream: the L2 prefetch overlaps them with that grid's tail.  With
-    // the look-back the tile index is only known after the wait; blockIdx.x
-    // is the likely one (a wrong guess only costs a wasted prefetch).  Once
-    // the wait returns, let the next grid launch (it waits for this one to
-    // complete before touching memory).
+    // the look-back the tile index is only known after the wait; the block
+    // index is the likely one (a wrong guess only costs a wasted prefetch).
+    // Once the wait returns, let the next grid launch (it waits for this one
+    // to complete before touching memory).
     {
-        const long long jg = blockIdx.x;
+        const long long jg = block;
         const long long mg = kBwd ? (g.ntiles - 1 - jg) : jg;
         Est::prefetch(P, g, mg * (long long)(NT * V), NT * V);
     }
@@ -773,7 +838,7 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
             return;
         }
     } else {
-        j = blockIdx.x;
+        j = block;
     }
     const long long m = kBwd ? (g.ntiles - 1 - j) : j; // tile index in memory
     const long long tile0 = m * (long long)(NT * V);
@@ -844,17 +909,14 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
             if constexpr (kLookback) {
                 const AT tile_a = __shfl_sync(kFullMask, wa, kBwd ? 0 : NW - 1);
                 const BT tile_b = __shfl_sync(kFullMask, wb, kBwd ? 0 : NW - 1);
-                if (lane == 0) {
-                    bool needs_carry;
-                    if (kBwd) {
-                        const long long end = tile0 + (long long)(NT * V);
-                        needs_carry = end < g.n && (end % g.seq_len) != 0;
-                    } else {
-                        needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
-                    }
-                    carry = lookback_carry<AT, BT>(lb, j, needs_carry, tile_a, tile_b);
+                bool needs_carry;
+                if (kBwd) {
+                    const long long end = tile0 + (long long)(NT * V);
+                    needs_carry = end < g.n && (end % g.seq_len) != 0;
+                } else {
+                    needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
                 }
-                carry = __shfl_sync(kFullMask, carry, 0);
+                carry = lookback_carry<AT, BT>(lb, j, needs_carry, tile_a, tile_b, lane);
             }
             if (lane < NW) s_wx[lane] = apply_pair(wea, web, carry);
         }
@@ -881,6 +943,13 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
     Est::template store<V>(P, g, pos, S);
 
     if constexpr (kLookback) lookback_release<NT>(lb, g.ntiles);
+}
+
+template <class Est, int NT, int V, int kMode>
+__global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Params P, const Geometry g,
+                                                       const Lookback lb) {
+    extern __shared__ __align__(128) unsigned char dyn_smem[];
+    tile_scan_body<Est, NT, V, kMode>(P, g, lb, (long long)blockIdx.x, dyn_smem);
 }
 
 // ---------------------------------------------------------------------------

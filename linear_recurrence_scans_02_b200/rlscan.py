@@ -38,7 +38,7 @@ __all__ = [
     "RlscanError", "library_path",
     "rlscan_gae", "rlscan_gae_with_returns", "rlscan_gae_typed", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
     "rlscan_discounted_returns", "rlscan_eligibility_traces", "rlscan_episodic_prefix_sum",
-    "rlscan_workspace_bytes", "rlscan_check", "rlscan_plan", "rlscan_debug_set_lookback",
+    "rlscan_batch", "rlscan_workspace_bytes", "rlscan_check", "rlscan_plan", "rlscan_debug_set_lookback",
     "compute_gae", "compute_gae_with_returns", "compute_vtrace", "compute_retrace", "compute_lambda_returns",
     "compute_discounted_returns", "compute_eligibility_traces", "compute_episodic_prefix_sum",
 ]
@@ -66,6 +66,14 @@ class RlscanError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"rlscan error {_STATUS_NAMES.get(status, status)}: {message}")
         self.status = status
+
+
+class _Call(ctypes.Structure):
+    """struct rlscan_call of include/rlscan.h."""
+    _fields_ = [("kind", ctypes.c_int), ("dtype", ctypes.c_int), ("options", ctypes.c_uint),
+                ("E", ctypes.c_int64), ("T", ctypes.c_int64), ("A", ctypes.c_int64),
+                ("gamma", ctypes.c_float), ("lambda_", ctypes.c_float), ("rho_bar", ctypes.c_float),
+                ("c_bar", ctypes.c_float), ("inp", ctypes.c_void_p * 8), ("out", ctypes.c_void_p * 2)]
 
 
 def library_path() -> str:
@@ -100,6 +108,7 @@ def _load_library():
         "rlscan_discounted_returns_ex": [P] * 6 + [I64, I64, F, U, P, SZ, S],
         "rlscan_eligibility_traces_ex": [P] * 3 + [I64, I64, F, F, U, P, SZ, S],
         "rlscan_episodic_prefix_sum_ex": [P, INT, P, P, I64, I64, U, P, SZ, S],
+        "rlscan_batch": [ctypes.POINTER(_Call), INT, P, SZ, S],
         "rlscan_workspace_init": [P, SZ, S],
         "rlscan_check": [S],
         "rlscan_version": [],
@@ -379,6 +388,85 @@ def rlscan_episodic_prefix_sum(x, dones, out, ws=None, *, time_major=False, done
     _raise_on(_lib.rlscan_episodic_prefix_sum_ex(
         _ptr(x, "x", sh, (torch.float32, torch.int32), device=dev), dtype, _ptr(dones, "dones", sh, device=dev),
         _ptr(out, "out", sh, (torch.float32, torch.int32), device=dev), E, T, opts, wp, wn, s))
+
+
+# ---------------------------------------------------------------------------
+# rlscan_batch: several independent calls in one request
+# ---------------------------------------------------------------------------
+
+_BACKWARD_IN = ("rewards", "values", "terminateds", "truncateds", "bootstrap_values", "last_values")
+_BATCH_KINDS = {
+    # kind: (C enum, input slots, output slots)
+    "gae": (1, _BACKWARD_IN, ("advantages",)),
+    "gae_with_returns": (2, _BACKWARD_IN, ("advantages", "returns")),
+    "vtrace": (3, ("log_rhos",) + _BACKWARD_IN, ("vs", "pg_advantages")),
+    "retrace": (4, ("rewards", "q_values", "next_q_values_all", "next_target_probs", "log_rhos", "terminateds",
+                    "truncateds"), ("q_ret",)),
+    "lambda_returns": (5, _BACKWARD_IN, ("returns",)),
+    "discounted_returns": (6, ("rewards", "terminateds", "truncateds", "bootstrap_values", "last_values"),
+                           ("returns",)),
+    "eligibility_traces": (7, ("x", "dones"), ("traces",)),
+    "episodic_prefix_sum": (8, ("x", "dones"), ("out",)),
+}
+_BATCH_SCALARS = {"gamma": 0.99, "lambda_": 0.95, "rho_bar": 1.0, "c_bar": 1.0}
+
+
+def rlscan_batch(calls, ws=None):
+    """Several independent estimator calls in one request (C: rlscan_batch).
+
+    `calls` is a list of dicts, each with "kind" (a key of the rlscan_*
+    functions: "gae", "gae_with_returns", "vtrace", "retrace",
+    "lambda_returns", "discounted_returns", "eligibility_traces",
+    "episodic_prefix_sum"), its tensors under the argument names of that
+    function (outputs preallocated), its scalars (gamma, lambda_, rho_bar,
+    c_bar; V-Trace's lambda_ defaults to 1.0) and optionally time_major /
+    done_starts_episode.  Calls whose rows fit 1024-element tiles run as one
+    fused launch; the results equal the individual calls bit for bit."""
+    if len(calls) > 16:
+        raise ValueError("at most 16 calls per request")
+    arr = (_Call * max(1, len(calls)))()
+    dev = None
+    ws_need = 0
+    for n, call in enumerate(calls):
+        kind = call["kind"]
+        if kind not in _BATCH_KINDS:
+            raise ValueError(f"unknown kind {kind!r}")
+        code, in_names, out_names = _BATCH_KINDS[kind]
+        first = call[in_names[0]]
+        dev = first.device if dev is None else dev
+        tm = bool(call.get("time_major", False))
+        E, T, sh, opts = _layout(first, in_names[0], tm)
+        if call.get("done_starts_episode", False):
+            opts |= RLSCAN_OPT_DONE_STARTS_EPISODE
+        c = arr[n]
+        c.kind, c.options, c.E, c.T, c.A = code, opts, E, T, 1
+        for k, v in _BATCH_SCALARS.items():
+            setattr(c, k, float(call.get(k, 1.0 if (kind == "vtrace" and k == "lambda_") else v)))
+        dtypes = (torch.float32,)
+        if kind == "episodic_prefix_sum":
+            dtypes = (torch.float32, torch.int32)
+            c.dtype = RLSCAN_F32 if first.dtype == torch.float32 else RLSCAN_I32
+        if kind == "retrace" and call["next_q_values_all"].dim() == 3:
+            c.A = int(call["next_q_values_all"].shape[2])
+        for i, name in enumerate(in_names):
+            shape = (E,) if name == "last_values" else (sh + (c.A,) if name in ("next_q_values_all",
+                                                                               "next_target_probs") and c.A > 1
+                                                         else sh)
+            dt = dtypes if name == "x" else (torch.float32,)
+            c.inp[i] = _ptr(call.get(name), name, shape, dt, dev)
+        for i, name in enumerate(out_names):
+            dt = dtypes if name == "out" else (torch.float32,)
+            c.out[i] = _ptr(call.get(name), name, sh, dt, dev)
+        if not tm:
+            ws_need = max(ws_need, int(_lib.rlscan_workspace_bytes(E, T)))
+    if not calls:
+        return
+    stream = _stream_handle(dev)
+    if ws is not None:
+        wp, wn = _ptr(ws, "ws", dtypes=(torch.uint8,), device=dev), ws.numel()
+    else:
+        wp, wn = _ws_cache.get(dev, stream, ws_need)
+    _raise_on(_lib.rlscan_batch(arr, len(calls), wp, wn, stream))
 
 
 # ---------------------------------------------------------------------------

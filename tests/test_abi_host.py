@@ -229,3 +229,64 @@ def test_ex_time_major_limits(lib):
     assert lib.rlscan_gae_ex(far[0], far[1], far[2], None, None, None, far[3], E_big, 1, 0.99, 0.95, TIME_MAJOR,
                              None, 0, None) == UNSUPPORTED
     assert "time-major" in msg(lib)
+
+
+class _Call(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("dtype", ctypes.c_int), ("options", ctypes.c_uint),
+                ("E", ctypes.c_int64), ("T", ctypes.c_int64), ("A", ctypes.c_int64),
+                ("gamma", ctypes.c_float), ("lambda_", ctypes.c_float), ("rho_bar", ctypes.c_float),
+                ("c_bar", ctypes.c_float), ("inp", ctypes.c_void_p * 8), ("out", ctypes.c_void_p * 2)]
+
+
+def _gae_call(r, v, d, out):
+    c = _Call()
+    c.kind, c.E, c.T, c.A, c.gamma, c.lambda_ = 1, E, T, 1, 0.99, 0.95
+    c.inp[0], c.inp[1], c.inp[2], c.out[0] = r, v, d, out
+    return c
+
+
+def test_batch_host_rules(lib):
+    lib.rlscan_batch.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    assert lib.rlscan_batch(None, 0, None, 0, None) == OK
+    arr = (_Call * 2)()
+    assert lib.rlscan_batch(arr, 17, None, 0, None) == INVALID
+    assert lib.rlscan_batch(None, 1, None, 0, None) == INVALID
+    arr[0] = _gae_call(A, B, C, O1)
+    arr[0].kind = 99
+    assert lib.rlscan_batch(arr, 1, None, 0, None) == INVALID
+    assert "call 0" in msg(lib) and "kind" in msg(lib)
+    # two calls writing one buffer: rejected before anything is launched
+    arr[0] = _gae_call(A, B, C, O1)
+    arr[1] = _gae_call(A, B, C, O1 + 64)
+    assert lib.rlscan_batch(arr, 2, None, 0, None) == INVALID
+    assert "calls 0 and 1" in msg(lib)
+    # one call's output over the other call's input
+    arr[1] = _gae_call(O1 + 8, B, C, O2)
+    assert lib.rlscan_batch(arr, 2, None, 0, None) == INVALID
+    # a call failing its own checks is named
+    arr[1] = _gae_call(None, B, C, O2)
+    assert lib.rlscan_batch(arr, 2, None, 0, None) == INVALID
+    assert "call 1" in msg(lib) and "rewards" in msg(lib)
+
+
+def test_batch_call_layout_matches_the_header(tmp_path):
+    # compile a C probe of struct rlscan_call against include/rlscan.h and
+    # compare its layout with the binding's ctypes mirror
+    import subprocess
+    import sys
+    src = tmp_path / "lay.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "rlscan.h"\n'
+                   'int main(void) { printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(rlscan_call), '
+                   'offsetof(rlscan_call, E), offsetof(rlscan_call, gamma), offsetof(rlscan_call, c_bar), '
+                   'offsetof(rlscan_call, in), offsetof(rlscan_call, out)); return 0; }\n')
+    exe = tmp_path / "lay"
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, "-o", str(exe), str(src)],
+                   check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    sys.path.insert(0, ROOT)
+    from linear_recurrence_scans_02_b200.rlscan import _Call as Mirror
+    want = [ctypes.sizeof(Mirror), Mirror.E.offset, Mirror.gamma.offset, Mirror.c_bar.offset, Mirror.inp.offset,
+            Mirror.out.offset]
+    assert got == want
+    assert [ctypes.sizeof(_Call), _Call.inp.offset] == [want[0], want[4]]

@@ -1,0 +1,219 @@
+"""GPU tests of rlscan_batch: several independent calls in one request.
+
+A fused launch runs each call's tiles through the same tile body as the
+call's own launch, so every output must equal the individual call's output
+bit for bit; the individual calls are themselves checked against the oracle
+by the parity tests, and the fused outputs are also compared with the oracle
+here, at the parity tolerance (|gpu - oracle| <= 1e-4 (1 + |oracle|); the
+int32 prefix sum exactly).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_common import assert_close, assert_equal_int, dev
+from linear_recurrence_scans_02_b200 import rlscan as R
+from linear_recurrence_scans_02_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+G, L = W.GAMMA, W.LAMBDA
+
+
+def _nan(shape, dtype=torch.float32):
+    return torch.full(shape, float("nan") if dtype == torch.float32 else -123456, dtype=dtype, device="cuda")
+
+
+def _calls_for(E, T, seed, trunc=False, time_major=False):
+    """One call of every fusable kind on seeded [E, T] inputs; returns the
+    calls (outputs NaN-filled) and the oracle's outputs for each."""
+    tmx = (lambda a: np.ascontiguousarray(a.T)) if time_major else (lambda a: a)
+    sh = (T, E) if time_major else (E, T)
+    b = W.vtrace_inputs(E, T, seed, p_term=0.01, p_trunc=0.01 if trunc else 0.0, last_values=True)
+    r = W.retrace_inputs(E, T, seed + 1, p_term=0.01, p_trunc=0.01)
+    f = W.trace_inputs(E, T, seed + 2, p_done=0.02)
+    fi = W.prefix_inputs_i32(E, T, seed + 3, p_done=0.02)
+    t = {k: dev(tmx(v) if v.ndim == 2 else v) for k, v in b.items()}
+    tr = {k: dev(tmx(v)) for k, v in r.items()}
+    tf = {k: dev(tmx(v)) for k, v in f.items()}
+    tfi = {k: dev(tmx(v)) for k, v in fi.items()}
+    back = {k: t.get(k) for k in ("rewards", "values", "terminateds", "truncateds", "bootstrap_values",
+                                  "last_values")}
+    extra = {"time_major": time_major}
+    calls = [
+        dict(kind="gae", advantages=_nan(sh), gamma=G, lambda_=L, **back, **extra),
+        dict(kind="gae_with_returns", advantages=_nan(sh), returns=_nan(sh), gamma=G, lambda_=L, **back, **extra),
+        dict(kind="vtrace", log_rhos=t["log_rhos"], vs=_nan(sh), pg_advantages=_nan(sh), gamma=G, lambda_=0.95,
+             rho_bar=1.0, c_bar=0.9, **back, **extra),
+        dict(kind="retrace", q_ret=_nan(sh), gamma=G, lambda_=L, c_bar=1.0, next_target_probs=None, **tr, **extra),
+        dict(kind="lambda_returns", returns=_nan(sh), gamma=G, lambda_=L, **back, **extra),
+        dict(kind="discounted_returns", returns=_nan(sh), gamma=G,
+             **{k: back[k] for k in ("rewards", "terminateds", "truncateds", "bootstrap_values", "last_values")},
+             **extra),
+        dict(kind="eligibility_traces", x=tf["x"], dones=tf["dones"], traces=_nan(sh), gamma=G, lambda_=L, **extra),
+        dict(kind="episodic_prefix_sum", x=tf["x"], dones=tf["dones"], out=_nan(sh), **extra),
+        dict(kind="episodic_prefix_sum", x=tfi["x"], dones=tfi["dones"], out=_nan(sh, torch.int32), **extra),
+    ]
+    args = (b.get("truncateds"), b.get("bootstrap_values"), b["last_values"])
+    g32, l32 = np.float32(G), np.float32(L)
+    refs = [
+        {"advantages": oracle.gae(b["rewards"], b["values"], b["terminateds"], g32, l32, *args)},
+        {"advantages": oracle.gae(b["rewards"], b["values"], b["terminateds"], g32, l32, *args),
+         "returns": oracle.lambda_returns(b["rewards"], b["values"], b["terminateds"], g32, l32, *args)},
+        dict(zip(("vs", "pg_advantages"),
+                 oracle.vtrace(b["log_rhos"], b["rewards"], b["values"], b["terminateds"], g32, np.float32(0.95),
+                               np.float32(1.0), np.float32(0.9), *args))),
+        {"q_ret": oracle.retrace(r["rewards"], r["q_values"], r["next_q_values_all"], r["log_rhos"],
+                                 r["terminateds"], r["truncateds"], g32, l32, np.float32(1.0))},
+        {"returns": oracle.lambda_returns(b["rewards"], b["values"], b["terminateds"], g32, l32, *args)},
+        {"returns": oracle.discounted_returns(b["rewards"], b["terminateds"], g32, *args)},
+        {"traces": oracle.eligibility_traces(f["x"], f["dones"], g32, l32)},
+        {"out": oracle.episodic_prefix_sum(f["x"], f["dones"])},
+        {"out": oracle.episodic_prefix_sum(fi["x"], fi["dones"])},
+    ]
+    return calls, refs
+
+
+def _single(call):
+    """The same call through its own entry point, into fresh outputs."""
+    c = dict(call)
+    kind = c.pop("kind")
+    tm = c.pop("time_major", False)
+    outs = {k: torch.empty_like(v) for k, v in c.items()
+            if k in ("advantages", "returns", "vs", "pg_advantages", "q_ret", "traces", "out")}
+    c.update(outs)
+    if kind == "gae":
+        R.rlscan_gae(c["rewards"], c["values"], c["terminateds"], c["truncateds"], c["bootstrap_values"],
+                     c["last_values"], c["advantages"], c["gamma"], c["lambda_"], time_major=tm)
+    elif kind == "gae_with_returns":
+        R.rlscan_gae_with_returns(c["rewards"], c["values"], c["terminateds"], c["truncateds"],
+                                  c["bootstrap_values"], c["last_values"], c["advantages"], c["returns"],
+                                  c["gamma"], c["lambda_"], time_major=tm)
+    elif kind == "vtrace":
+        R.rlscan_vtrace(c["log_rhos"], c["rewards"], c["values"], c["terminateds"], c["truncateds"],
+                        c["bootstrap_values"], c["last_values"], c["vs"], c["pg_advantages"], c["gamma"],
+                        c["lambda_"], c["rho_bar"], c["c_bar"], time_major=tm)
+    elif kind == "retrace":
+        R.rlscan_retrace(c["rewards"], c["q_values"], c["next_q_values_all"], c["next_target_probs"], c["log_rhos"],
+                         c["terminateds"], c["truncateds"], c["q_ret"], c["gamma"], c["lambda_"], c["c_bar"],
+                         time_major=tm)
+    elif kind == "lambda_returns":
+        R.rlscan_lambda_returns(c["rewards"], c["values"], c["terminateds"], c["truncateds"], c["bootstrap_values"],
+                                c["last_values"], c["returns"], c["gamma"], c["lambda_"], time_major=tm)
+    elif kind == "discounted_returns":
+        R.rlscan_discounted_returns(c["rewards"], c["terminateds"], c["truncateds"], c["bootstrap_values"],
+                                    c["last_values"], c["returns"], c["gamma"], time_major=tm)
+    elif kind == "eligibility_traces":
+        R.rlscan_eligibility_traces(c["x"], c["dones"], c["traces"], c["gamma"], c["lambda_"], time_major=tm,
+                                    done_starts_episode=c.get("done_starts_episode", False))
+    else:
+        R.rlscan_episodic_prefix_sum(c["x"], c["dones"], c["out"], time_major=tm,
+                                     done_starts_episode=c.get("done_starts_episode", False))
+    return outs
+
+
+def _check_batch(calls, refs, time_major=False):
+    singles = [_single(c) for c in calls]
+    R.rlscan_batch(calls)
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    for n, (call, ref, single) in enumerate(zip(calls, refs, singles)):
+        for k, want in single.items():
+            got = call[k]
+            assert torch.equal(got, want) or (got.dtype == torch.float32 and
+                                              torch.equal(torch.nan_to_num(got), torch.nan_to_num(want))), \
+                f"call {n} ({call['kind']}) {k}: fused result differs from the single call"
+            g = got.t() if time_major else got
+            if ref[k].dtype == np.int32:
+                assert_equal_int(g, ref[k], f"{call['kind']}:{k}")
+            else:
+                assert_close(g, ref[k], 1e-4, f"{call['kind']}:{k}")
+
+
+# shapes whose plan is the fused 1024-element tile: warp mode (T <= 256) and
+# block mode (T = 512, 1024), ragged E
+@pytest.mark.parametrize("E,T", [(4096, 128), (1, 1), (37, 32), (300, 256), (129, 512), (64, 1024)], ids=str)
+@pytest.mark.parametrize("trunc", [False, True], ids=["term", "trunc"])
+def test_batch_of_every_kind_matches_single_calls_and_oracle(E, T, trunc):
+    calls, refs = _calls_for(E, T, seed=E + T, trunc=trunc)
+    _check_batch(calls, refs)
+
+
+def test_batch_mixes_fused_and_separate_launches():
+    # fused: 4096 x 128; separate: rows split over tiles (look-back), a
+    # time-major call, T = 96 (no 1024-element plan), multi-action Retrace
+    fused, fref = _calls_for(4096, 128, seed=1)
+    lb, lref = _calls_for(3, 70000, seed=2)
+    tm, tref = _calls_for(100, 130, seed=3, time_major=True)
+    odd, oref = _calls_for(50, 96, seed=4)
+    calls = fused[:3] + [lb[5], lb[7]] + [tm[0], tm[8]] + [odd[1], odd[6]]
+    refs = fref[:3] + [lref[5], lref[7]] + [tref[0], tref[8]] + [oref[1], oref[6]]
+    singles = [_single(c) for c in calls]
+    d = W.off_policy_inputs(64, 128, A=18, seed=5)
+    t = {k: dev(v) for k, v in d.items()}
+    multi = dict(kind="retrace", rewards=t["rewards"], q_values=t["q_values"],
+                 next_q_values_all=t["next_q_values_all"], next_target_probs=t["next_target_probs"],
+                 log_rhos=t["log_rhos"], terminateds=t["terminateds"], truncateds=t["truncateds"],
+                 q_ret=_nan((64, 128)), gamma=G, lambda_=L, c_bar=1.0)
+    mref = oracle.retrace(d["rewards"], d["q_values"], d["next_q_values_all"], d["log_rhos"], d["terminateds"],
+                          d["truncateds"], np.float32(G), np.float32(L), np.float32(1.0), d["next_target_probs"])
+    R.rlscan_batch(calls + [multi])
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    for n, (call, ref, single) in enumerate(zip(calls, refs, singles)):
+        tmj = call.get("time_major", False)
+        for k, want in single.items():
+            assert torch.equal(torch.nan_to_num(call[k]), torch.nan_to_num(want)), f"call {n} {k}"
+            g = call[k].t() if tmj else call[k]
+            if ref[k].dtype == np.int32:
+                assert_equal_int(g, ref[k], f"call {n}:{k}")
+            else:
+                tol = 1e-4 if ref[k].shape[-1] <= 8192 else 1e-3
+                assert_close(g, ref[k], tol, f"call {n}:{k}", row_scale=True)
+    assert_close(multi["q_ret"], mref, 1e-4, "multi-action retrace")
+
+
+def test_batch_done_starts_episode_option():
+    E, T = 512, 128
+    f = W.trace_inputs(E, T, seed=8, p_done=0.05)
+    x, d = dev(f["x"]), dev(f["dones"])
+    calls = [dict(kind="eligibility_traces", x=x, dones=d, traces=_nan((E, T)), gamma=G, lambda_=L,
+                  done_starts_episode=True),
+             dict(kind="episodic_prefix_sum", x=x, dones=d, out=_nan((E, T)), done_starts_episode=True)]
+    R.rlscan_batch(calls)
+    torch.cuda.synchronize()
+    assert_close(calls[0]["traces"], oracle.eligibility_traces(f["x"], f["dones"], np.float32(G), np.float32(L),
+                                                               True), 1e-4, "traces")
+    assert_close(calls[1]["out"], oracle.episodic_prefix_sum(f["x"], f["dones"], True), 1e-4, "prefix")
+
+
+def test_batch_rejects_overlap_across_calls_and_enqueues_nothing():
+    E, T = 256, 128
+    calls, _ = _calls_for(E, T, seed=9)
+    a, b = calls[0], calls[6]
+    shared = _nan((E, T))
+    a["advantages"] = shared
+    b["traces"] = shared  # two calls write the same buffer
+    with pytest.raises(R.RlscanError) as ei:
+        R.rlscan_batch([a, b])
+    assert ei.value.status == R.RLSCAN_ERR_INVALID_ARG
+    assert "calls 0 and 1" in str(ei.value)
+    c = dict(calls[4])
+    c["returns"] = calls[0]["rewards"]  # an output over another call's input
+    with pytest.raises(R.RlscanError):
+        R.rlscan_batch([calls[1], c])
+    # a call that fails its own checks: nothing of the request runs
+    bad = dict(calls[2])
+    bad["c_bar"] = float("nan")
+    with pytest.raises(R.RlscanError) as ei:
+        R.rlscan_batch([calls[3], bad])
+    assert "call 1" in str(ei.value)
+    torch.cuda.synchronize()
+    assert torch.isnan(shared).all() and torch.isnan(calls[3]["q_ret"]).all()
+
+
+def test_batch_empty_and_single():
+    R.rlscan_batch([])
+    calls, refs = _calls_for(64, 512, seed=11)
+    _check_batch(calls[:1], refs[:1])
