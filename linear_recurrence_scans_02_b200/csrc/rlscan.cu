@@ -291,6 +291,7 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
         lb.hdr = static_cast<WsHeader *>(ws);
         lb.slots = reinterpret_cast<TileSlot *>(static_cast<char *>(ws) + sizeof(WsHeader));
         lb.withhold = g_withhold.load();
+        lb.row_tiles = (T % kCfgTile[plan.cfg] == 0) ? T / kCfgTile[plan.cfg] : 0;
     }
     if (batch_dry()) return ok();
     if constexpr (FusedKindOf<Est>::value >= 0) {
@@ -348,6 +349,7 @@ int run_multi(const char *name, const typename Est::Params &P, long long E, long
         lb.hdr = static_cast<WsHeader *>(ws);
         lb.slots = reinterpret_cast<TileSlot *>(static_cast<char *>(ws) + sizeof(WsHeader));
         lb.withhold = g_withhold.load();
+        lb.row_tiles = (T % kCfgTile[plan.cfg] == 0) ? T / kCfgTile[plan.cfg] : 0;
     }
     if (batch_dry()) return ok();
     const size_t smem = multi_smem_bytes(plan.cfg, actions);

@@ -228,7 +228,9 @@ struct Lookback {
     TileSlot *slots;
     unsigned spin_limit; // polls before a wait gives up
     long long withhold;  // scan-order tile that never publishes (test hook), -1 = none
+    long long row_tiles; // tiles per row when rows are whole multiples of a tile, else 0
 };
+
 
 // Geometry of one launch over the flattened [E*T] array.
 struct Geometry {
@@ -240,6 +242,17 @@ struct Geometry {
     int vec_ok;        // every plane pointer of the call is 16-byte aligned
     int scan_lanes;    // warp-local mode: lanes one row spans (a power of two <= 32)
 };
+
+// Scan-order tile of the t-th tile taken from the counter.  When every row
+// is a whole number of tiles, the counter deals the rows' tiles out in
+// turn (row r's c-th tile is ticket c E + r), so the tiles running at once
+// spread over all rows and each row's chain of carries stays short; a tile
+// still only waits on tiles of its own row with smaller tickets, which have
+// started.  Otherwise tiles are taken in scan order.
+__device__ __forceinline__ long long lookback_tile(const Lookback &lb, const Geometry &g, long long t) {
+    if (lb.row_tiles <= 0) return t;
+    return (t % g.rows) * lb.row_tiles + t / g.rows;
+}
 
 // Where a thread's V elements sit in their rows, as bit masks over k:
 // end bit k = element k is the last step of its row (t == T-1), start bit
@@ -326,8 +339,12 @@ __device__ __forceinline__ long long elem_row(const RowMasks &m, int k) {
 // word and the walk ends as if the carry were zero.
 constexpr int kLbPerLane = 1;
 
+// k_min: the lowest tile the walk may read; tiles before it are never
+// needed (the row's first tile always publishes an inclusive value) and
+// may not have started yet when the counter deals tiles out row by row.
 template <class AT, class BT>
-__device__ BT lookback_carry(const Lookback &lb, long long j, bool needs_carry, AT ta, BT tb, int lane) {
+__device__ BT lookback_carry(const Lookback &lb, long long j, long long k_min, bool needs_carry, AT ta, BT tb,
+                             int lane) {
     TileSlot *me = lb.slots + j;
     const bool publish = (j != lb.withhold) && lane == 0;
     if (!needs_carry) {
@@ -358,7 +375,7 @@ __device__ BT lookback_carry(const Lookback &lb, long long j, bool needs_carry, 
         // (relaxed load + fence = acquire) before the published values are read
         unsigned st[M];
 #pragma unroll
-        for (int m = 0; m < M; ++m) st[m] = (k0 - m >= 0) ? ld_relaxed_gpu(&lb.slots[k0 - m].status) : 2u;
+        for (int m = 0; m < M; ++m) st[m] = (k0 - m >= k_min) ? ld_relaxed_gpu(&lb.slots[k0 - m].status) : 2u;
         bool gave_up = false;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
@@ -382,7 +399,7 @@ __device__ BT lookback_carry(const Lookback &lb, long long j, bool needs_carry, 
         uint4 slot[M];
 #pragma unroll
         for (int m = 0; m < M; ++m)
-            slot[m] = (k0 - m >= 0) ? ld_relaxed_gpu_v4(&lb.slots[k0 - m]) : make_uint4(0u, 0u, 0u, 0u);
+            slot[m] = (k0 - m >= k_min) ? ld_relaxed_gpu_v4(&lb.slots[k0 - m]) : make_uint4(0u, 0u, 0u, 0u);
         // this lane's M tiles composed nearest-outermost, stopping at the
         // first inclusive value or cut (a == 0: the map ignores what came before)
         AT la = identity_a(ta);
@@ -394,7 +411,7 @@ __device__ BT lookback_carry(const Lookback &lb, long long j, bool needs_carry, 
             const long long k = k0 - m;
             AT ka;
             BT kb;
-            if (k < 0) { // nothing flows in from before the array (unreachable in a well-formed walk)
+            if (k < k_min) { // nothing flows in from before the row / array
                 ka = AT(0);
                 kb = identity_b(tb);
             } else if (st[m] == 2u) { // an inclusive value: the map x -> x_k
@@ -821,7 +838,7 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     // Once the wait returns, let the next grid launch (it waits for this one
     // to complete before touching memory).
     {
-        const long long jg = block;
+        const long long jg = kLookback ? lookback_tile(lb, g, block) : block;
         const long long mg = kBwd ? (g.ntiles - 1 - jg) : jg;
         Est::prefetch(P, g, mg * (long long)(NT * V), NT * V);
     }
@@ -832,11 +849,11 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     if constexpr (kLookback) {
         if (tid == 0) s_tile = (long long)atomicAdd(&lb.hdr->tile_counter, 1u);
         __syncthreads();
-        j = s_tile;
-        if (j >= g.ntiles) { // counter was not zero at launch: touch nothing, report
+        if (s_tile >= g.ntiles) { // counter was not zero at launch: touch nothing, report
             if (tid == 0) atomicOr(&g_device_error, kErrWorkspaceState);
             return;
         }
+        j = lookback_tile(lb, g, s_tile);
     } else {
         j = block;
     }
@@ -916,7 +933,8 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
                 } else {
                     needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
                 }
-                carry = lookback_carry<AT, BT>(lb, j, needs_carry, tile_a, tile_b, lane);
+                const long long k_min = lb.row_tiles > 0 ? (j / lb.row_tiles) * lb.row_tiles : 0;
+                carry = lookback_carry<AT, BT>(lb, j, k_min, needs_carry, tile_a, tile_b, lane);
             }
             if (lane < NW) s_wx[lane] = apply_pair(wea, web, carry);
         }
