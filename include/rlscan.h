@@ -340,7 +340,11 @@ RLSCAN_API int rlscan_episodic_prefix_sum_ex(const void *x, int dtype, const flo
  * whose rows fit whole in 1024-element tiles (row-major, 1024 a multiple of
  * T, every kind below, A == 1 for Retrace) as ONE fused kernel, each block
  * running one tile of one call, and each remaining call by its own launch.
- * Results are those of the individual calls, bit for bit.
+ * Results are those of the individual calls, bit for bit, except that a
+ * request fusing three or more kinds whose rows all fit 512 elements runs
+ * 4 elements per thread (smaller code per kind), which re-associates the
+ * fp32 scans: those results agree with the individual calls to fp32
+ * rounding (int32 stays exact).
  *
  * kind and argument slots (the pointer arguments of the entry point, in its
  * order; unused slots NULL):

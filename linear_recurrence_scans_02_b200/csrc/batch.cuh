@@ -3,8 +3,11 @@
 // A fused grid is the concatenation of the calls' tile grids: block b runs
 // tile b - tile_begin of the call whose range holds b, through the same tile
 // body (and so the same arithmetic, bit for bit) as that call's own launch.
-// Only calls whose plan is the 128-thread x 8-element tile without the
-// look-back are fused, so every block of the grid has the same shape.
+// Only calls whose rows fit whole in one tile are fused, so every block of
+// the grid has the same shape: 128 threads x 8 elements, or x 4 elements
+// when the request mixes several estimators (blocks of different
+// estimators then share each SM, and the smaller unrolled bodies fit the
+// instruction caches better).
 #pragma once
 
 #include "estimators.cuh"
@@ -65,8 +68,8 @@ struct FusedKindOf<PrefixI32Est> {
     static constexpr int value = kFkPrefixI32;
 };
 
-constexpr int kFusedNT = 128; // the 1024-element tile: 128 threads x 8 elements
-constexpr int kFusedV = 8;
+constexpr int kFusedNT = 128; // 128 threads x 8 (or 4) elements per tile
+constexpr int kFusedVMax = 8;
 constexpr int kFusedParamBytes = 128;
 constexpr int kFusedMax = 16;
 
@@ -83,21 +86,22 @@ struct FusedBatch {
     int n;
 };
 
-template <class Est, int kMode>
+template <class Est, int V, int kMode>
 __device__ __forceinline__ void fused_tile(const FusedItem &it, long long block, unsigned char *smem) {
     const auto &P = *reinterpret_cast<const typename Est::Params *>(it.params);
     const Lookback lb{nullptr, nullptr, 0u, -1}; // no look-back in a fused launch
-    tile_scan_body<Est, kFusedNT, kFusedV, kMode>(P, it.g, lb, block, smem);
+    tile_scan_body<Est, kFusedNT, V, kMode>(P, it.g, lb, block, smem);
 }
 
-template <class Est>
+template <class Est, int V>
 __device__ __forceinline__ void fused_tile_any_mode(const FusedItem &it, long long block, unsigned char *smem) {
     if (it.mode == kModeWarp)
-        fused_tile<Est, kModeWarp>(it, block, smem);
+        fused_tile<Est, V, kModeWarp>(it, block, smem);
     else
-        fused_tile<Est, kModeBlock>(it, block, smem);
+        fused_tile<Est, V, kModeBlock>(it, block, smem);
 }
 
+template <int V>
 __global__ void __launch_bounds__(kFusedNT) fused_tile_kernel(const __grid_constant__ FusedBatch b) {
     extern __shared__ __align__(128) unsigned char dyn_smem[];
     int idx = 0;
@@ -106,15 +110,15 @@ __global__ void __launch_bounds__(kFusedNT) fused_tile_kernel(const __grid_const
     const FusedItem &it = b.item[idx];
     const long long block = (long long)blockIdx.x - it.tile_begin;
     switch (it.kind) {
-    case kFkGae: fused_tile_any_mode<GaeEst>(it, block, dyn_smem); break;
-    case kFkGaeReturns: fused_tile_any_mode<GaeReturnsEst>(it, block, dyn_smem); break;
-    case kFkVtrace: fused_tile_any_mode<VtraceEst>(it, block, dyn_smem); break;
-    case kFkRetrace1: fused_tile_any_mode<RetraceEst<false>>(it, block, dyn_smem); break;
-    case kFkLambda: fused_tile_any_mode<LambdaReturnsEst>(it, block, dyn_smem); break;
-    case kFkReturns: fused_tile_any_mode<ReturnsEst>(it, block, dyn_smem); break;
-    case kFkTraces: fused_tile_any_mode<TracesEst>(it, block, dyn_smem); break;
-    case kFkPrefixF32: fused_tile_any_mode<PrefixF32Est>(it, block, dyn_smem); break;
-    case kFkPrefixI32: fused_tile_any_mode<PrefixI32Est>(it, block, dyn_smem); break;
+    case kFkGae: fused_tile_any_mode<GaeEst, V>(it, block, dyn_smem); break;
+    case kFkGaeReturns: fused_tile_any_mode<GaeReturnsEst, V>(it, block, dyn_smem); break;
+    case kFkVtrace: fused_tile_any_mode<VtraceEst, V>(it, block, dyn_smem); break;
+    case kFkRetrace1: fused_tile_any_mode<RetraceEst<false>, V>(it, block, dyn_smem); break;
+    case kFkLambda: fused_tile_any_mode<LambdaReturnsEst, V>(it, block, dyn_smem); break;
+    case kFkReturns: fused_tile_any_mode<ReturnsEst, V>(it, block, dyn_smem); break;
+    case kFkTraces: fused_tile_any_mode<TracesEst, V>(it, block, dyn_smem); break;
+    case kFkPrefixF32: fused_tile_any_mode<PrefixF32Est, V>(it, block, dyn_smem); break;
+    case kFkPrefixI32: fused_tile_any_mode<PrefixI32Est, V>(it, block, dyn_smem); break;
     default: break;
     }
 }

@@ -1,11 +1,14 @@
 """GPU tests of rlscan_batch: several independent calls in one request.
 
 A fused launch runs each call's tiles through the same tile body as the
-call's own launch, so every output must equal the individual call's output
-bit for bit; the individual calls are themselves checked against the oracle
-by the parity tests, and the fused outputs are also compared with the oracle
-here, at the parity tolerance (|gpu - oracle| <= 1e-4 (1 + |oracle|); the
-int32 prefix sum exactly).
+call's own launch.  With 8 elements per thread (requests of one or two
+estimators) its tiles are the call's own, so every output equals the
+individual call's bit for bit; requests mixing three or more estimators use
+4 elements per thread, which re-associates the fp32 scan, so there the
+outputs agree with the individual calls to fp32 rounding (1e-5 (1 + |x|)).
+The int32 prefix sum is exact either way.  The fused outputs are also
+compared with the oracle at the parity tolerance (|gpu - oracle| <=
+1e-4 (1 + |oracle|)).
 """
 import numpy as np
 import pytest
@@ -113,17 +116,33 @@ def _single(call):
     return outs
 
 
+def _same_as_single(got, want, exact, what):
+    if got.dtype != torch.float32 or exact:
+        assert torch.equal(torch.nan_to_num(got), torch.nan_to_num(want)), f"{what}: differs from the single call"
+    else:
+        assert_close(got, want.double().cpu().numpy(), 1e-5, f"{what} vs the single call")
+
+
+def _mixes_three_kinds(calls):
+    return len({c["kind"] for c in calls}) >= 3
+
+
+def _first_in(call):
+    return {"vtrace": "log_rhos", "eligibility_traces": "x", "episodic_prefix_sum": "x"}.get(call["kind"], "rewards")
+
+
 def _check_batch(calls, refs, time_major=False):
     singles = [_single(c) for c in calls]
     R.rlscan_batch(calls)
     torch.cuda.synchronize()
     R.rlscan_check()
+    # bit-exact unless the request takes the 4-element fused tile (three or
+    # more estimators and rows that fit 512 elements)
+    exact = not (_mixes_three_kinds(calls) and all(512 % c[_first_in(c)].shape[-1] == 0 for c in calls))
     for n, (call, ref, single) in enumerate(zip(calls, refs, singles)):
         for k, want in single.items():
             got = call[k]
-            assert torch.equal(got, want) or (got.dtype == torch.float32 and
-                                              torch.equal(torch.nan_to_num(got), torch.nan_to_num(want))), \
-                f"call {n} ({call['kind']}) {k}: fused result differs from the single call"
+            _same_as_single(got, want, exact, f"call {n} ({call['kind']}) {k}")
             g = got.t() if time_major else got
             if ref[k].dtype == np.int32:
                 assert_equal_int(g, ref[k], f"{call['kind']}:{k}")
@@ -164,7 +183,8 @@ def test_batch_mixes_fused_and_separate_launches():
     for n, (call, ref, single) in enumerate(zip(calls, refs, singles)):
         tmj = call.get("time_major", False)
         for k, want in single.items():
-            assert torch.equal(torch.nan_to_num(call[k]), torch.nan_to_num(want)), f"call {n} {k}"
+            # the fused calls (first three) take the 4-element tile: fp32 rounding may differ
+            _same_as_single(call[k], want, n >= 3, f"call {n} {k}")
             g = call[k].t() if tmj else call[k]
             if ref[k].dtype == np.int32:
                 assert_equal_int(g, ref[k], f"call {n}:{k}")
