@@ -281,10 +281,13 @@ RLSCAN_API int rlscan_gae_noalloc(const float *rewards, const float *values, con
  *     one row of E per step.  last_values stays [E].  Rows are still scanned
  *     independently; a time-major call needs no workspace (ws may be NULL)
  *     and reads and writes each element once with coalesced accesses along E.
- *     rlscan_retrace_ex takes it with A == 1 only (RLSCAN_ERR_UNSUPPORTED
- *     otherwise).
+ *     rlscan_retrace_ex takes it with A == 1 only, and E up to
+ *     238,609,294 (offsets between timesteps are 32-bit); beyond either,
+ *     RLSCAN_ERR_UNSUPPORTED.
  *   RLSCAN_OPT_DONE_STARTS_EPISODE (forward estimators only: eligibility
- *     traces and the episodic prefix sum): dones[e, t] != 0 marks step t as
+ *     traces and the episodic prefix sum; the rl-triton README's "Kernels"
+ *     table writes the trace's (1-d) factor with no time index, and this is
+ *     its other reading): dones[e, t] != 0 marks step t as
  *     the FIRST step of a new episode (the reset-flag convention: a "first" or
  *     "is_init" mask), instead of the default, where it marks t as the last
  *     step so that t+1 starts afresh.  With it, y_t = x_t where dones[t] != 0

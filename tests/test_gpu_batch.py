@@ -237,3 +237,43 @@ def test_batch_empty_and_single():
     R.rlscan_batch([])
     calls, refs = _calls_for(64, 512, seed=11)
     _check_batch(calls[:1], refs[:1])
+
+
+def test_batch_of_sixteen_calls_and_the_limit():
+    E, T = 256, 64
+    d = W.gae_inputs(E, T, seed=21, p_term=0.02)
+    t = {k: dev(v) for k, v in d.items()}
+    ref = oracle.gae(d["rewards"], d["values"], d["terminateds"], np.float32(G), np.float32(L))
+    calls = [dict(kind="gae", rewards=t["rewards"], values=t["values"], terminateds=t["terminateds"],
+                  advantages=_nan((E, T)), gamma=G, lambda_=L) for _ in range(16)]
+    R.rlscan_batch(calls)
+    torch.cuda.synchronize()
+    for c in calls:  # one estimator: 8 elements per thread, the single call's tiles
+        assert_close(c["advantages"], ref, 1e-4, "gae x16")
+    with pytest.raises(ValueError):
+        R.rlscan_batch(calls + calls[:1])
+
+
+def test_batch_in_a_cuda_graph_follows_new_inputs():
+    # a captured request replays with whatever its buffers hold at replay time
+    E, T = 1024, 128
+    calls, _ = _calls_for(E, T, seed=31)
+    srcs = [W.vtrace_inputs(E, T, seed=40 + k, p_term=0.01, last_values=True) for k in range(3)]
+    R.rlscan_batch(calls)  # warm-up outside capture
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        R.rlscan_batch(calls)
+    for src in srcs:
+        for k in ("rewards", "values", "terminateds", "last_values"):
+            calls[0][k].copy_(torch.from_numpy(src[k]))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = oracle.gae(src["rewards"], src["values"], src["terminateds"], np.float32(G), np.float32(L), None,
+                         None, src["last_values"])
+        assert_close(calls[0]["advantages"], ref, 1e-4, "gae in a replayed batch")
+        ref_dr = oracle.discounted_returns(src["rewards"], src["terminateds"], np.float32(G), None, None,
+                                          src["last_values"])
+        assert_close(calls[5]["returns"], ref_dr, 1e-4, "returns in a replayed batch")
+    R.rlscan_check()
