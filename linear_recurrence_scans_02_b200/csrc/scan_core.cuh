@@ -210,8 +210,9 @@ __device__ __forceinline__ void warp_exclusive_from_inclusive(AT ia, BT ib, int 
 
 struct WsHeader {
     unsigned tile_counter;
-    unsigned done_counter;
-    unsigned pad[30];
+    unsigned pad0[15];
+    unsigned done_counter; // its own 32-byte sector: the two counters are hit at different times
+    unsigned pad1[15];
 };
 static_assert(sizeof(WsHeader) == 128, "header is one 128-byte line");
 
@@ -458,10 +459,12 @@ __device__ __forceinline__ void lookback_release(const Lookback &lb, long long n
     __shared__ int s_last;
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        unsigned prev = atomicAdd(&lb.hdr->done_counter, 1u);
+        // release: this block's slot traffic (ordered before thread 0 by the
+        // barrier) precedes the increment; acquire: the last block sees every
+        // other block's before it clears the slots
+        unsigned prev;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(&lb.hdr->done_counter) : "memory");
         s_last = (prev == (unsigned)(ntiles - 1));
-        __threadfence();
     }
     __syncthreads();
     if (s_last) {
