@@ -384,13 +384,14 @@ struct TmPlan {
 };
 
 // Wider env groups (longer contiguous runs per load) while the grid keeps
-// about one block per SM; rows of several segments (T > 256) favour more,
-// smaller blocks.  Measured at E x T = 1024..65536 x 128, 4096 x 1024 and
-// 512 x 4096.  The segment covers the row, up to 16 warps.
+// enough blocks: 32-env groups from about four blocks per SM up, 16-env
+// groups from about one, else 8; rows of several segments (T > 256) favour
+// more, smaller blocks.  Measured at E x T = 1024..65536 x 128, 4096 x 1024
+// and 512 x 4096.  The segment covers the row, up to 16 warps.
 TmPlan tm_plan(long long E, long long T) {
     TmPlan p;
     const long long kMinBlocks = 120;
-    p.G = (E / 32 >= kMinBlocks && T <= 256) ? 32 : (E / 16 >= kMinBlocks ? 16 : 8);
+    p.G = (E / 32 >= 4 * 148 && T <= 256) ? 32 : (E / 16 >= kMinBlocks ? 16 : 8);
     const long long chunks = ceil_div(T, kTmV);
     const long long nw = ceil_div(chunks, 32 / p.G);
     p.nw = (int)(nw < 1 ? 1 : (nw > kTmMaxWarps ? kTmMaxWarps : nw));

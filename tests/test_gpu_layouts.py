@@ -25,8 +25,8 @@ pytestmark = pytest.mark.gpu
 # (E, T): one env and one step; E below, at and above an env group with
 # ragged tails; T below, at and across one segment (up to 16 warps x 32 / G
 # chunks x 8 steps) with ragged tails; the 4096 x 128 workload; and shapes
-# whose launch plan takes the 16-env groups (2000 x 300) and the 32-env
-# groups (4096 x 128, 5000 x 33, 19000 x 70)
+# whose launch plan takes the 16-env groups (4096 x 128, 5000 x 33,
+# 2000 x 300) and the 32-env groups (19000 x 70)
 SHAPES = [(1, 1), (1, 7), (5, 3), (31, 17), (32, 128), (33, 130), (100, 257), (64, 512), (7, 1000),
           (9, 4099), (4096, 128), (5000, 33), (2000, 300), (19000, 70)]
 
