@@ -37,6 +37,7 @@ import os
 import re
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -259,7 +260,10 @@ class ClockSampler:
         except Exception:
             pass
         self.proc = None
-        self.path = path or os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # the samples go to a scratch file (RLSCAN_CLOCKS_DIR, else the temp
+        # directory); their summary is part of the JSON line
+        out_dir = os.environ.get("RLSCAN_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = path or os.path.join(out_dir, f"rlscan_clocks_gpu{gpu_index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
