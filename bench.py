@@ -835,6 +835,17 @@ def run_profile_case(args):
     import torch
     from linear_recurrence_scans_02_b200 import rlscan as R
     torch.cuda.set_device(0)
+    if args.profile_shape:  # GAE at another shape, e.g. 16,262144 (long rows: the look-back path)
+        from linear_recurrence_scans_02_b200 import workloads as W
+        E, T = (int(v) for v in args.profile_shape.split(","))
+        d = W.device_inputs("gae", E, T, seed=0, device=torch.device("cuda", 0), p_done=1e-4)
+        out = torch.empty(E, T, device="cuda")
+        for _ in range(args.profile_launches):
+            R.rlscan_gae(d["rewards"], d["values"], d["terminateds"], None, None, None, out, 0.999, LAMBDA)
+        torch.cuda.synchronize()
+        R.rlscan_check()
+        print(f"profile case done: {args.profile_launches} GAE launches at {E} x {T}")
+        return 0
     bs = BufferSet(torch, torch.device("cuda", 0), PLANES)
     bs.fill_from_host(host_inputs(seed=0))
     calls = bs.calls(R)
@@ -865,6 +876,7 @@ def main(argv=None):
     ap.add_argument("--profile-launches", type=int, default=0,
                     help="run N eager launches of each estimator and exit (small case for ncu)")
     ap.add_argument("--profile-only", default="", help="comma-separated estimators for --profile-launches")
+    ap.add_argument("--profile-shape", default="", help="E,T: --profile-launches runs GAE at this shape instead")
     ap.add_argument("--sweep", action="store_true",
                     help="time four estimators over the E x T size grid and 16 x 262144, one JSON line per point")
     args = ap.parse_args(argv)
