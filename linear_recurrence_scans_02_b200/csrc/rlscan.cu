@@ -2,10 +2,12 @@
 // the extern "C" entry points declared in include/rlscan.h.
 //
 // Each entry point validates its arguments on the host (nothing touches the
-// GPU before the launch), picks a tile plan for the [E, T] shape, and
-// launches one tile_scan_kernel instantiation on the caller's stream with
-// programmatic dependent launch allowed, so the kernel's prologue can
-// overlap the tail of whatever ran before it on that stream.
+// GPU before the launch), picks a tile plan for the [E, T] shape (or the
+// env-group plan of the time-major layout), and launches one kernel
+// instantiation on the caller's stream with programmatic dependent launch
+// allowed, so the kernel's prologue can overlap the tail of whatever ran
+// before it on that stream.  rlscan_batch runs the same checks for several
+// calls and launches the fusable ones as one kernel.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
