@@ -290,3 +290,20 @@ def test_batch_call_layout_matches_the_header(tmp_path):
             Mirror.out.offset]
     assert got == want
     assert [ctypes.sizeof(_Call), _Call.inp.offset] == [want[0], want[4]]
+
+
+@pytest.mark.parametrize("E_,T_,tile,threads,lookback", [
+    (4096, 128, 1024, 128, False),     # the 4096 x 128 workload: 128 threads x 8, whole rows
+    (64, 512, 1024, 128, False),
+    (4096, 2048, 2048, 256, False),    # a row needs a bigger tile to stay whole
+    (256, 4096, 4096, 512, False),
+    (16, 262144, 2048, 256, True),     # long rows: the look-back over 2048-element tiles
+    (1024, 8192, 2048, 256, True),
+    (3, 70000, 512, 128, True),        # few tiles: 512-element tiles (4 per thread)
+    (4096, 129, 1024, 128, True),      # rows not dividing any tile
+])
+def test_plan_choices(lib, E_, T_, tile, threads, lookback):
+    # the launch plans the measurements in the design notes were taken with
+    t, th, lb, nt = plan(lib, E_, T_)
+    assert (t, th, lb) == (tile, threads, lookback)
+    assert nt == -(-E_ * T_ // t)
