@@ -302,6 +302,11 @@ RLSCAN_API int rlscan_gae_ex(const float *rewards, const float *values, const fl
                              const float *truncateds, const float *bootstrap_values, const float *last_values,
                              float *advantages, int64_t E, int64_t T, float gamma, float lambda_,
                              unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream);
+RLSCAN_API int rlscan_gae_typed_ex(const void *rewards, const void *values, const void *terminateds,
+                                   const void *truncateds, const void *bootstrap_values, const float *last_values,
+                                   float *advantages, float *returns, int64_t E, int64_t T, float gamma,
+                                   float lambda_, int value_dtype, int flag_dtype, unsigned options, void *ws,
+                                   size_t ws_bytes, cudaStream_t stream);
 RLSCAN_API int rlscan_gae_with_returns_ex(const float *rewards, const float *values, const float *terminateds,
                                           const float *truncateds, const float *bootstrap_values,
                                           const float *last_values, float *advantages, float *returns, int64_t E,

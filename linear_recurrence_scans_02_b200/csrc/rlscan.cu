@@ -540,10 +540,11 @@ int rlscan_gae_with_returns(const float *rewards, const float *values, const flo
     return rlscan_gae_with_returns_ex(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages, returns, E, T, gamma, lambda_, 0u, ws, ws_bytes, stream);
 }
 
-int rlscan_gae_typed(const void *rewards, const void *values, const void *terminateds, const void *truncateds,
-                     const void *bootstrap_values, const float *last_values, float *advantages, float *returns,
-                     int64_t E, int64_t T, float gamma, float lambda_, int value_dtype, int flag_dtype, void *ws,
-                     size_t ws_bytes, cudaStream_t stream) {
+int rlscan_gae_typed_ex(const void *rewards, const void *values, const void *terminateds, const void *truncateds,
+                        const void *bootstrap_values, const float *last_values, float *advantages, float *returns,
+                        int64_t E, int64_t T, float gamma, float lambda_, int value_dtype, int flag_dtype,
+                        unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, false));
     size_t vsz, fsz;
     switch (value_dtype) {
     case RLSCAN_F32: vsz = 4; break;
@@ -578,6 +579,8 @@ int rlscan_gae_typed(const void *rewards, const void *values, const void *termin
                                                static_cast<const FT *>(terminateds),                               \
                                                static_cast<const FT *>(truncateds), static_cast<const VT *>(bv),  \
                                                last_values, advantages, returns, gamma, lambda_};                  \
+        if (options & RLSCAN_OPT_TIME_MAJOR)                                                                      \
+            return run_time_major<GaeTypedEst<VT, FT>>("rlscan_gae_typed", P, E, T, stream);                     \
         return run<GaeTypedEst<VT, FT>>("rlscan_gae_typed", P, E, T, 1, ws, ws_bytes, stream, vec);              \
     } while (0)
     if (flag_dtype == RLSCAN_U8) {
@@ -589,6 +592,14 @@ int rlscan_gae_typed(const void *rewards, const void *values, const void *termin
     if (value_dtype == RLSCAN_F16) RLSCAN_GAE_TYPED(__half, float);
     RLSCAN_GAE_TYPED(float, float);
 #undef RLSCAN_GAE_TYPED
+}
+
+int rlscan_gae_typed(const void *rewards, const void *values, const void *terminateds, const void *truncateds,
+                     const void *bootstrap_values, const float *last_values, float *advantages, float *returns,
+                     int64_t E, int64_t T, float gamma, float lambda_, int value_dtype, int flag_dtype, void *ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_gae_typed_ex(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages,
+                               returns, E, T, gamma, lambda_, value_dtype, flag_dtype, 0u, ws, ws_bytes, stream);
 }
 
 int rlscan_vtrace_ex(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,

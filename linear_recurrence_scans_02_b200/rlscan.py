@@ -101,6 +101,7 @@ def _load_library():
         "rlscan_eligibility_traces": [P] * 3 + [I64, I64, F, F, P, SZ, S],
         "rlscan_episodic_prefix_sum": [P, INT, P, P, I64, I64, P, SZ, S],
         "rlscan_gae_ex": [P] * 7 + [I64, I64, F, F, U, P, SZ, S],
+        "rlscan_gae_typed_ex": [P] * 8 + [I64, I64, F, F, INT, INT, U, P, SZ, S],
         "rlscan_gae_with_returns_ex": [P] * 8 + [I64, I64, F, F, U, P, SZ, S],
         "rlscan_vtrace_ex": [P] * 9 + [I64, I64, F, F, F, F, U, P, SZ, S],
         "rlscan_retrace_ex": [P] * 8 + [I64, I64, I64, F, F, F, U, P, SZ, S],
@@ -273,13 +274,12 @@ def rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_
 
 
 def rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, advantages,
-                     returns, gamma, lambda_, ws=None):
+                     returns, gamma, lambda_, ws=None, *, time_major=False):
     """GAE (+ TD(lambda) returns when `returns` is given) from reduced-byte
     inputs: rewards / values / bootstrap_values float32, bfloat16 or float16
     (one dtype for the three), flags float32, uint8 or bool; fp32 outputs."""
-    E, T = _shape(rewards, "rewards")
+    E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
-    sh = (E, T)
     vdt = _VALUE_DTYPES.get(rewards.dtype)
     if vdt is None:
         raise TypeError(f"rewards dtype {rewards.dtype} not supported")
@@ -289,13 +289,13 @@ def rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values,
         raise TypeError(f"flag dtype {flags[0].dtype} not supported")
     vt = (rewards.dtype,)
     ft = (flags[0].dtype,) if flags else (torch.float32,)
-    wp, wn, s = _workspace(dev, E, T, ws)
-    _raise_on(_lib.rlscan_gae_typed(
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_gae_typed_ex(
         _ptr(rewards, "rewards", sh, vt, dev), _ptr(values, "values", sh, vt, dev),
         _ptr(terminateds, "terminateds", sh, ft, dev), _ptr(truncateds, "truncateds", sh, ft, dev),
         _ptr(bootstrap_values, "bootstrap_values", sh, vt, dev),
         _ptr(last_values, "last_values", (E,), device=dev), _ptr(advantages, "advantages", sh, device=dev),
-        _ptr(returns, "returns", sh, device=dev), E, T, float(gamma), float(lambda_), vdt, fdt, wp, wn, s))
+        _ptr(returns, "returns", sh, device=dev), E, T, float(gamma), float(lambda_), vdt, fdt, opts, wp, wn, s))
 
 
 def _reduced_bytes(*tensors):
@@ -476,13 +476,11 @@ def rlscan_batch(calls, ws=None):
 def compute_gae(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
                 bootstrap_values=None, last_values=None, time_major=False):
     """Advantages (fp32).  bf16/fp16 values or uint8/bool flags take the
-    reduced-byte entry point (row-major only)."""
+    reduced-byte entry point."""
     adv = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
     if _reduced_bytes(rewards, values, terminateds, truncateds, bootstrap_values):
-        if time_major:
-            raise ValueError("reduced-byte inputs take the row-major [num_envs, seq_len] layout only")
         rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, None, gamma,
-                         lambda_)
+                         lambda_, time_major=time_major)
     else:
         rlscan_gae(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, gamma, lambda_,
                    time_major=time_major)
@@ -492,15 +490,12 @@ def compute_gae(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, trunc
 def compute_gae_with_returns(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
                              bootstrap_values=None, last_values=None, time_major=False):
     """(advantages, returns) from one pass: returns = advantages + values.
-    bf16/fp16 values or uint8/bool flags take the reduced-byte entry point
-    (row-major only)."""
+    bf16/fp16 values or uint8/bool flags take the reduced-byte entry point."""
     adv = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
     ret = torch.empty(rewards.shape, dtype=torch.float32, device=rewards.device)
     if _reduced_bytes(rewards, values, terminateds, truncateds, bootstrap_values):
-        if time_major:
-            raise ValueError("reduced-byte inputs take the row-major [num_envs, seq_len] layout only")
         rlscan_gae_typed(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret, gamma,
-                         lambda_)
+                         lambda_, time_major=time_major)
     else:
         rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret,
                                 gamma, lambda_, time_major=time_major)

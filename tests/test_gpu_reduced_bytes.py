@@ -82,3 +82,26 @@ def test_compute_gae_dispatches_on_dtypes():
     want = oracle.gae(_wide(r), _wide(v), _wide(done), np.float32(0.99), np.float32(0.95))
     assert_close(adv, want, 1e-4, "compute_gae bf16/bool")
     assert_close(adv2, want, 1e-4, "compute_gae_with_returns bf16/bool")
+
+
+@pytest.mark.parametrize("vdt", VALUE_DTYPES, ids=str)
+@pytest.mark.parametrize("fdt", [torch.uint8, torch.float32], ids=str)
+@pytest.mark.parametrize("E,T", [(5, 3), (33, 130), (4096, 128), (9, 1000), (5000, 33)], ids=str)
+def test_reduced_byte_gae_time_major(vdt, fdt, E, T):
+    # the same call on [T, E] planes (envs contiguous): transposed inputs,
+    # outputs transposed back, against the oracle on the widened values
+    d = W.gae_inputs(E, T, seed=E * 3 + T, p_term=0.02, p_trunc=0.02, last_values=True)
+    tm = lambda a, dt: _narrow(np.ascontiguousarray(a.T), dt)
+    r, v, bv = tm(d["rewards"], vdt), tm(d["values"], vdt), tm(d["bootstrap_values"], vdt)
+    te, tr = tm(d["terminateds"], fdt), tm(d["truncateds"], fdt)
+    lv = torch.from_numpy(d["last_values"]).cuda()
+    adv = torch.full((T, E), float("nan"), device="cuda")
+    ret = torch.full((T, E), float("nan"), device="cuda")
+    R.rlscan_gae_typed(r, v, te, tr, bv, lv, adv, ret, 0.99, 0.95, time_major=True)
+    torch.cuda.synchronize()
+    w = lambda t: np.ascontiguousarray(_wide(t).T)
+    g, l = np.float32(0.99), np.float32(0.95)
+    args = (w(tr), w(bv), d["last_values"])
+    assert_close(adv.t(), oracle.gae(w(r), w(v), w(te), g, l, *args), tol_for(T), "time-major typed gae")
+    assert_close(ret.t(), oracle.lambda_returns(w(r), w(v), w(te), g, l, *args), tol_for(T),
+                 "time-major typed returns")
