@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define RLSCAN_VERSION 100 /* 1.0.0 */
+#define RLSCAN_VERSION 110 /* 1.1.0: the _ex entry points (layout and done-convention options) and rlscan_batch */
 
 /* Every entry point is exported from librlscan.so (built with hidden
  * visibility for everything else). */

@@ -69,7 +69,10 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version(lib):
-    assert lib.rlscan_version() == 100
+    # the library reports the version its header declares
+    text = open(HEADER).read()
+    declared = int(re.search(r"#define RLSCAN_VERSION (\d+)", text).group(1))
+    assert lib.rlscan_version() == declared == 110
 
 
 # fake, never-dereferenced device addresses, far apart

@@ -62,6 +62,9 @@ MUTANTS = {
     # int32 prefix sum under the done-starts-episode reading resets one step early (reads the next flag)
     "prefix_i32_starts_reads_next": ("done_starts_episode ? is_set(dones, i) : (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += prev;\n            /* reduce",
                                      "done_starts_episode ? (t + 1 < T && is_set(dones, i + 1)) : (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += prev;\n            /* reduce"),
+    # f32 prefix sum under the done-starts-episode reading never resets
+    "prefix_f32_starts_ignored": ("done_starts_episode ? is_set(dones, i) : (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += prev;\n            out[i] = cur;",
+                                  "done_starts_episode ? 0 : (t > 0 && is_set(dones, i - 1));\n            if (t > 0 && !reset)\n                cur += prev;\n            out[i] = cur;"),
     # int32 prefix sum saturates instead of wrapping
     "prefix_i32_saturates": ("int64_t wrapped = (low >= 0x80000000u) ? (int64_t)low - 4294967296LL : (int64_t)low;",
                              "int64_t wrapped = cur > 2147483647LL ? 2147483647LL : (cur < -2147483648LL ? -2147483648LL : cur); (void)low;"),
