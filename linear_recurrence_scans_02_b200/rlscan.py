@@ -158,12 +158,6 @@ def _ptr(t, name, shape=None, dtypes=(torch.float32,), device=None):
     return t.data_ptr() or None
 
 
-def _shape(t, name):
-    if not isinstance(t, torch.Tensor) or t.dim() != 2:
-        raise ValueError(f"{name} must be a [num_envs, seq_len] tensor")
-    return int(t.shape[0]), int(t.shape[1])
-
-
 def _stream_handle(device):
     return torch.cuda.current_stream(device).cuda_stream
 
