@@ -368,9 +368,13 @@ RLSCAN_API int rlscan_episodic_prefix_sum_ex(const void *x, int dtype, const flo
  *                                   out: returns
  *   RLSCAN_KIND_ELIGIBILITY_TRACES  in: x dones; out: traces
  *   RLSCAN_KIND_EPISODIC_PREFIX_SUM in: x dones; out: out  (dtype RLSCAN_F32 or RLSCAN_I32)
+ *   RLSCAN_KIND_GAE_TYPED           in: as GAE; out: advantages returns (returns nullable);
+ *                                   dtype = value_dtype, flag_dtype = flag_dtype of
+ *                                   rlscan_gae_typed
  * Scalars a kind does not take are ignored (lambda_ for discounted returns,
  * rho_bar and c_bar outside V-Trace and Retrace, A outside Retrace, dtype
- * outside the prefix sum).  options: as for the _ex entry points.
+ * outside the prefix sum and typed GAE, flag_dtype outside typed GAE).
+ * options: as for the _ex entry points.
  *
  * The calls run concurrently: no call's output may overlap any other
  * call's inputs or outputs (RLSCAN_ERR_INVALID_ARG).  ws / ws_bytes: one
@@ -388,7 +392,8 @@ typedef enum rlscan_kind {
     RLSCAN_KIND_LAMBDA_RETURNS = 5,
     RLSCAN_KIND_DISCOUNTED_RETURNS = 6,
     RLSCAN_KIND_ELIGIBILITY_TRACES = 7,
-    RLSCAN_KIND_EPISODIC_PREFIX_SUM = 8
+    RLSCAN_KIND_EPISODIC_PREFIX_SUM = 8,
+    RLSCAN_KIND_GAE_TYPED = 9
 } rlscan_kind;
 
 #define RLSCAN_CALL_MAX_IN 8
@@ -398,7 +403,8 @@ typedef enum rlscan_kind {
 
 typedef struct rlscan_call {
     int kind;       /* rlscan_kind */
-    int dtype;      /* RLSCAN_KIND_EPISODIC_PREFIX_SUM: RLSCAN_F32 or RLSCAN_I32 */
+    int dtype;      /* prefix sum: RLSCAN_F32 or RLSCAN_I32; typed GAE: the value dtype */
+    int flag_dtype; /* typed GAE: the flag dtype */
     unsigned options;
     int64_t E, T, A;
     float gamma, lambda_, rho_bar, c_bar;

@@ -908,13 +908,30 @@ int rlscan_plan(int64_t E, int64_t T, int64_t actions, int64_t *tile_elems, int 
 
 // Byte extent of argument slot `slot` of a call (its input when in_slot,
 // else its output); 0 for slots the kind does not have.
+static size_t dtype_bytes(int dtype) {
+    switch (dtype) {
+    case RLSCAN_BF16:
+    case RLSCAN_F16: return 2;
+    case RLSCAN_U8: return 1;
+    default: return 4;
+    }
+}
+
 static size_t call_slot_bytes(const rlscan_call &c, bool in_slot, int slot) {
-    const size_t plane = (size_t)(c.E * c.T) * 4u, row = (size_t)c.E * 4u;
+    const size_t n = (size_t)(c.E * c.T), plane = n * 4u, row = (size_t)c.E * 4u;
     if (!in_slot) {
-        const int nout = (c.kind == RLSCAN_KIND_GAE_WITH_RETURNS || c.kind == RLSCAN_KIND_VTRACE) ? 2 : 1;
+        const int nout = (c.kind == RLSCAN_KIND_GAE_WITH_RETURNS || c.kind == RLSCAN_KIND_VTRACE ||
+                          c.kind == RLSCAN_KIND_GAE_TYPED)
+                             ? 2
+                             : 1;
         return slot < nout ? plane : 0;
     }
     switch (c.kind) {
+    case RLSCAN_KIND_GAE_TYPED: {
+        const size_t v = n * dtype_bytes(c.dtype), f = n * dtype_bytes(c.flag_dtype);
+        const size_t by_slot[6] = {v, v, f, f, v, row};
+        return slot < 6 ? by_slot[slot] : 0;
+    }
     case RLSCAN_KIND_GAE:
     case RLSCAN_KIND_GAE_WITH_RETURNS:
     case RLSCAN_KIND_LAMBDA_RETURNS: return slot < 5 ? plane : (slot == 5 ? row : 0);
@@ -955,6 +972,9 @@ static int call_dispatch(const rlscan_call &c, void *ws, size_t ws_bytes, cudaSt
     case RLSCAN_KIND_EPISODIC_PREFIX_SUM:
         return rlscan_episodic_prefix_sum_ex(c.in[0], c.dtype, in[1], c.out[0], c.E, c.T, c.options, ws, ws_bytes,
                                              stream);
+    case RLSCAN_KIND_GAE_TYPED:
+        return rlscan_gae_typed_ex(c.in[0], c.in[1], c.in[2], c.in[3], c.in[4], in[5], out[0], out[1], c.E, c.T,
+                                   c.gamma, c.lambda_, c.dtype, c.flag_dtype, c.options, ws, ws_bytes, stream);
     default: return fail(RLSCAN_ERR_INVALID_ARG, "unknown kind %d", c.kind);
     }
 }

@@ -70,7 +70,8 @@ class RlscanError(RuntimeError):
 
 class _Call(ctypes.Structure):
     """struct rlscan_call of include/rlscan.h."""
-    _fields_ = [("kind", ctypes.c_int), ("dtype", ctypes.c_int), ("options", ctypes.c_uint),
+    _fields_ = [("kind", ctypes.c_int), ("dtype", ctypes.c_int), ("flag_dtype", ctypes.c_int),
+                ("options", ctypes.c_uint),
                 ("E", ctypes.c_int64), ("T", ctypes.c_int64), ("A", ctypes.c_int64),
                 ("gamma", ctypes.c_float), ("lambda_", ctypes.c_float), ("rho_bar", ctypes.c_float),
                 ("c_bar", ctypes.c_float), ("inp", ctypes.c_void_p * 8), ("out", ctypes.c_void_p * 2)]
@@ -401,6 +402,7 @@ _BATCH_KINDS = {
                            ("returns",)),
     "eligibility_traces": (7, ("x", "dones"), ("traces",)),
     "episodic_prefix_sum": (8, ("x", "dones"), ("out",)),
+    "gae_typed": (9, _BACKWARD_IN, ("advantages", "returns")),
 }
 _BATCH_SCALARS = {"gamma": 0.99, "lambda_": 0.95, "rho_bar": 1.0, "c_bar": 1.0}
 
@@ -409,7 +411,7 @@ def rlscan_batch(calls, ws=None):
     """Several independent estimator calls in one request (C: rlscan_batch).
 
     `calls` is a list of dicts, each with "kind" (a key of the rlscan_*
-    functions: "gae", "gae_with_returns", "vtrace", "retrace",
+    functions: "gae", "gae_with_returns", "gae_typed", "vtrace", "retrace",
     "lambda_returns", "discounted_returns", "eligibility_traces",
     "episodic_prefix_sum"), its tensors under the argument names of that
     function (outputs preallocated), its scalars (gamma, lambda_, rho_bar,
@@ -437,16 +439,27 @@ def rlscan_batch(calls, ws=None):
         for k, v in _BATCH_SCALARS.items():
             setattr(c, k, float(call.get(k, 1.0 if (kind == "vtrace" and k == "lambda_") else v)))
         dtypes = (torch.float32,)
+        slot_dtypes = {}
         if kind == "episodic_prefix_sum":
             dtypes = (torch.float32, torch.int32)
             c.dtype = RLSCAN_F32 if first.dtype == torch.float32 else RLSCAN_I32
+        if kind == "gae_typed":  # value and flag dtypes from the tensors, as rlscan_gae_typed
+            c.dtype = _VALUE_DTYPES.get(first.dtype, -1)
+            flags = [call[k] for k in ("terminateds", "truncateds") if call.get(k) is not None]
+            c.flag_dtype = _FLAG_DTYPES.get(flags[0].dtype, -1) if flags else RLSCAN_F32
+            if c.dtype < 0 or c.flag_dtype < 0:
+                raise TypeError("gae_typed: unsupported value or flag dtype")
+            for k in ("rewards", "values", "bootstrap_values"):
+                slot_dtypes[k] = (first.dtype,)
+            for k in ("terminateds", "truncateds"):
+                slot_dtypes[k] = (flags[0].dtype,) if flags else (torch.float32,)
         if kind == "retrace" and call["next_q_values_all"].dim() == 3:
             c.A = int(call["next_q_values_all"].shape[2])
         for i, name in enumerate(in_names):
             shape = (E,) if name == "last_values" else (sh + (c.A,) if name in ("next_q_values_all",
                                                                                "next_target_probs") and c.A > 1
                                                          else sh)
-            dt = dtypes if name == "x" else (torch.float32,)
+            dt = slot_dtypes.get(name, dtypes if name == "x" else (torch.float32,))
             c.inp[i] = _ptr(call.get(name), name, shape, dt, dev)
         for i, name in enumerate(out_names):
             dt = dtypes if name == "out" else (torch.float32,)

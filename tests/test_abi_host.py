@@ -235,7 +235,8 @@ def test_ex_time_major_limits(lib):
 
 
 class _Call(ctypes.Structure):
-    _fields_ = [("kind", ctypes.c_int), ("dtype", ctypes.c_int), ("options", ctypes.c_uint),
+    _fields_ = [("kind", ctypes.c_int), ("dtype", ctypes.c_int), ("flag_dtype", ctypes.c_int),
+                ("options", ctypes.c_uint),
                 ("E", ctypes.c_int64), ("T", ctypes.c_int64), ("A", ctypes.c_int64),
                 ("gamma", ctypes.c_float), ("lambda_", ctypes.c_float), ("rho_bar", ctypes.c_float),
                 ("c_bar", ctypes.c_float), ("inp", ctypes.c_void_p * 8), ("out", ctypes.c_void_p * 2)]

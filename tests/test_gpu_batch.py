@@ -277,3 +277,41 @@ def test_batch_in_a_cuda_graph_follows_new_inputs():
                                           src["last_values"])
         assert_close(calls[5]["returns"], ref_dr, 1e-4, "returns in a replayed batch")
     R.rlscan_check()
+
+
+def test_batch_with_reduced_byte_gae():
+    # bf16 values + uint8 flags (its own launch) and fp32 typed GAE (fused
+    # with the one-pass GAE + returns kernel) in one request with V-Trace
+    E, T = 512, 128
+    d = W.gae_inputs(E, T, seed=51, p_term=0.02, p_trunc=0.02, last_values=True)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(torch.bfloat16)
+    u8 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(torch.uint8)
+    wide = lambda t: t.to(torch.float32).cpu().numpy()
+    lv = dev(d["last_values"])
+    narrow = dict(kind="gae_typed", rewards=bf(d["rewards"]), values=bf(d["values"]),
+                  terminateds=u8(d["terminateds"]), truncateds=u8(d["truncateds"]),
+                  bootstrap_values=bf(d["bootstrap_values"]), last_values=lv, advantages=_nan((E, T)),
+                  returns=_nan((E, T)), gamma=G, lambda_=L)
+    full = dict(kind="gae_typed", rewards=dev(d["rewards"]), values=dev(d["values"]),
+                terminateds=dev(d["terminateds"]), truncateds=dev(d["truncateds"]),
+                bootstrap_values=dev(d["bootstrap_values"]), last_values=lv, advantages=_nan((E, T)),
+                returns=None, gamma=G, lambda_=L)
+    v = W.vtrace_inputs(E, T, seed=52, p_term=0.01)
+    vt = dict(kind="vtrace", log_rhos=dev(v["log_rhos"]), rewards=dev(v["rewards"]), values=dev(v["values"]),
+              terminateds=dev(v["terminateds"]), vs=_nan((E, T)), pg_advantages=_nan((E, T)), gamma=G)
+    R.rlscan_batch([narrow, full, vt])
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    g32, l32 = np.float32(G), np.float32(L)
+    nargs = (wide(narrow["truncateds"]), wide(narrow["bootstrap_values"]), d["last_values"])
+    assert_close(narrow["advantages"], oracle.gae(wide(narrow["rewards"]), wide(narrow["values"]),
+                                                  wide(narrow["terminateds"]), g32, l32, *nargs), 1e-4, "bf16/u8 adv")
+    assert_close(narrow["returns"], oracle.lambda_returns(wide(narrow["rewards"]), wide(narrow["values"]),
+                                                          wide(narrow["terminateds"]), g32, l32, *nargs),
+                 1e-4, "bf16/u8 returns")
+    fargs = (d["truncateds"], d["bootstrap_values"], d["last_values"])
+    assert_close(full["advantages"], oracle.gae(d["rewards"], d["values"], d["terminateds"], g32, l32, *fargs),
+                 1e-4, "fp32 typed adv")
+    rvs, _ = oracle.vtrace(v["log_rhos"], v["rewards"], v["values"], v["terminateds"], g32, np.float32(1.0),
+                           np.float32(1.0), np.float32(1.0))
+    assert_close(vt["vs"], rvs, 1e-4, "vtrace beside typed gae")
