@@ -49,11 +49,27 @@ if ROOT not in sys.path:
 E_ENVS, T_STEPS = 4096, 128
 GAMMA, LAMBDA = 0.99, 0.95
 P_DONE = 0.005
-L2_BYTES = 126 * 1024 * 1024
-ROTATE_BYTES = 4 * L2_BYTES
+DEFAULT_L2_BYTES = 126 * 1024 * 1024  # B200; the device's own figure is used when it can be read
+
+
+def rotate_bytes(device=None) -> int:
+    """Buffer bytes a timing loop rotates through: 4x the device's L2, so
+    every launch streams its inputs from HBM."""
+    l2 = DEFAULT_L2_BYTES
+    try:
+        import torch
+        if torch.cuda.is_available():
+            l2 = int(torch.cuda.get_device_properties(device or 0).L2_cache_size) or l2
+    except Exception:
+        pass
+    return 4 * l2
+
+
 FALLBACK_HBM_GBS = 6650.0
 REPEATS = 5            # timed repeats per estimator (median reported)
 ISOLATED_SAMPLES = 21  # single calls on an idle stream per estimator
+SUBMIT_SPIN_CYCLES = 2_000_000  # ~1 ms device spin ahead of a timed region (host enqueues meanwhile)
+TIMED_GRAPH_STEPS = 256         # steps per graph launch in the timed region
 WORKLOAD = "all seven estimators fp32, num_envs=4096, seq_len=128"
 
 # estimator -> (input planes, output planes, bytes per env-step moved)
@@ -76,6 +92,10 @@ EXTRA_CALLS = {
     "gae_with_returns_bf16_u8": (["rewards", "values", "terminateds"], ["advantages", "returns"]),
     # GAE on the time-major layout: every plane [seq_len, num_envs]
     "gae_time_major": (["rewards", "values", "terminateds"], ["advantages"]),
+    # GAE advantages, TD(lambda) returns and V-Trace vs / pg from one pass
+    # (replaces gae_with_returns + vtrace on the same inputs)
+    "gae_returns_vtrace": (["log_rhos", "rewards", "values", "terminateds"],
+                           ["advantages", "returns", "vs", "pg_advantages"]),
 }
 TIME_MAJOR = {"gae_time_major"}
 PLANES = {**ESTIMATORS, **EXTRA_CALLS}
@@ -108,7 +128,7 @@ def host_inputs(seed: int = 0) -> dict:
     gt = {k: np.ascontiguousarray(v.T) for k, v in W.gae_inputs(E, T, seed + 9, p_term=P_DONE).items()}
     return {"gae": g, "vtrace": v, "retrace": r, "lambda_returns": lr, "discounted_returns": dr,
             "eligibility_traces": et, "prefix_sum_f32": pf, "prefix_sum_i32": pi, "gae_with_returns": gr,
-            "gae_with_returns_bf16_u8": gr, "gae_time_major": gt}
+            "gae_with_returns_bf16_u8": gr, "gae_time_major": gt, "gae_returns_vtrace": v}
 
 
 # ---------------------------------------------------------------------------
@@ -196,6 +216,12 @@ class BufferSet:
             k = "gae_time_major"
             c[k] = lambda: R.rlscan_gae(t[k, "rewards"], t[k, "values"], t[k, "terminateds"], None, None, None,
                                         t[k, "advantages"], GAMMA, LAMBDA, time_major=True)
+        if "gae_returns_vtrace" in self.estimators:
+            k = "gae_returns_vtrace"
+            c[k] = lambda: R.rlscan_gae_vtrace(t[k, "log_rhos"], t[k, "rewards"], t[k, "values"],
+                                               t[k, "terminateds"], None, None, None, t[k, "advantages"],
+                                               t[k, "returns"], t[k, "vs"], t[k, "pg_advantages"], GAMMA, LAMBDA,
+                                               1.0, 1.0, 1.0)
         if "prefix_sum_i32" in self.estimators:
             c["prefix_sum_i32"] = lambda: R.rlscan_episodic_prefix_sum(
                 t["prefix_sum_i32", "x"], t["prefix_sum_i32", "dones"], t["prefix_sum_i32", "out"])
@@ -445,6 +471,139 @@ def capture(torch, fns, stream):
     return g
 
 
+def time_launches(torch, R, fns, side, stream, world=1, min_launches=200):
+    """Per-launch device time of `fns` (one launch each) replayed back to back
+    in one CUDA graph: median over REPEATS repeats of >= min_launches
+    launches, with the range.  Returns (us, [min, max], launches)."""
+    for f in fns:
+        f()
+    R.rlscan_check()
+    g = capture(torch, fns, side)
+    reps = max(3, -(-min_launches // len(fns)))
+    for _ in range(2):
+        g.replay()
+    samples = []
+    for _ in range(REPEATS):
+        barrier_sync(world)
+        torch.cuda._sleep(SUBMIT_SPIN_CYCLES)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        barrier_sync(world)
+        samples.append(1000.0 * max_over_ranks(a.elapsed_time(b), world) / (reps * len(fns)))
+    R.rlscan_check()
+    del g
+    return float(np.median(samples)), [min(samples), max(samples)], reps * len(fns)
+
+
+# ---------------------------------------------------------------------------
+# the other workloads of the path, each timed like per_estimator: back-to-back
+# launches over rotating device copies of one seeded batch (>= 4x L2 in all)
+# ---------------------------------------------------------------------------
+TRUNC_P = 0.005  # terminated and truncated, each (mutually exclusive per step)
+
+
+def config_cases():
+    """(key, E, T, host-input builder, {estimator: (call, streamed bytes per
+    env-step, outputs, input planes)}).  Streamed bytes count every dense plane read once and every
+    output written once; bootstrap values are read only at truncated steps
+    (about 1 % of steps here) and are not counted."""
+    from linear_recurrence_scans_02_b200 import workloads as W
+
+    def trunc_inputs():
+        d = W.vtrace_inputs(E_ENVS, T_STEPS, 20, p_term=TRUNC_P, p_trunc=TRUNC_P)
+        r = W.retrace_inputs(E_ENVS, T_STEPS, 21, p_term=TRUNC_P, p_trunc=TRUNC_P)
+        d.update({"q_values": r["q_values"], "next_q_values_all": r["next_q_values_all"]})
+        return d
+
+    def gae(R, t, o, g=GAMMA):
+        return lambda: R.rlscan_gae(t["rewards"], t["values"], t["terminateds"], t.get("truncateds"),
+                                    t.get("bootstrap_values"), None, o[0], g, LAMBDA)
+
+    trunc = {
+        "gae": (gae, 20, 1, ("rewards", "values", "terminateds", "truncateds", "bootstrap_values")),
+        "vtrace": (lambda R, t, o: lambda: R.rlscan_vtrace(
+            t["log_rhos"], t["rewards"], t["values"], t["terminateds"], t["truncateds"], t["bootstrap_values"],
+            None, o[0], o[1], GAMMA, 1.0, 1.0, 1.0), 28, 2,
+                   ("log_rhos", "rewards", "values", "terminateds", "truncateds", "bootstrap_values")),
+        "retrace": (lambda R, t, o: lambda: R.rlscan_retrace(
+            t["rewards"], t["q_values"], t["next_q_values_all"], None, t["log_rhos"], t["terminateds"],
+            t["truncateds"], o[0], GAMMA, LAMBDA, 1.0), 28, 1,
+                    ("rewards", "q_values", "next_q_values_all", "log_rhos", "terminateds", "truncateds")),
+        "lambda_returns": (lambda R, t, o: lambda: R.rlscan_lambda_returns(
+            t["rewards"], t["values"], t["terminateds"], t["truncateds"], t["bootstrap_values"], None, o[0],
+            GAMMA, LAMBDA), 20, 1, ("rewards", "values", "terminateds", "truncateds", "bootstrap_values")),
+        "discounted_returns": (lambda R, t, o: lambda: R.rlscan_discounted_returns(
+            t["rewards"], t["terminateds"], t["truncateds"], t["bootstrap_values"], None, o[0], GAMMA), 16, 1,
+                               ("rewards", "terminateds", "truncateds", "bootstrap_values")),
+    }
+    A = 18
+    off = {
+        "vtrace": (lambda R, t, o: lambda: R.rlscan_vtrace(
+            t["log_rhos"], t["rewards"], t["values"], t["terminateds"], None, None, None, o[0], o[1],
+            GAMMA, 1.0, 1.0, 1.0), 24, 2, ("log_rhos", "rewards", "values", "terminateds")),
+        "retrace": (lambda R, t, o: lambda: R.rlscan_retrace(
+            t["rewards"], t["q_values"], t["next_q_values_all"], t["next_target_probs"], t["log_rhos"],
+            t["terminateds"], t["truncateds"], o[0], GAMMA, LAMBDA, 1.0), 8 * A + 24, 1,
+                    ("rewards", "q_values", "next_q_values_all", "next_target_probs", "log_rhos", "terminateds",
+                     "truncateds")),
+    }
+    long_rows = {
+        "gae": (lambda R, t, o: lambda: R.rlscan_gae(t["rewards"], t["values"], t["terminateds"], None, None,
+                                                     None, o[0], 0.999, LAMBDA), 16, 1,
+                ("rewards", "values", "terminateds")),
+        "discounted_returns": (lambda R, t, o: lambda: R.rlscan_discounted_returns(
+            t["rewards"], t["terminateds"], None, None, None, o[0], 0.999), 12, 1, ("rewards", "terminateds")),
+        "eligibility_traces": (lambda R, t, o: lambda: R.rlscan_eligibility_traces(
+            t["x"], t["dones"], o[0], 0.999, LAMBDA), 12, 1, ("x", "dones")),
+        "prefix_sum_f32": (lambda R, t, o: lambda: R.rlscan_episodic_prefix_sum(t["x"], t["dones"], o[0]), 12, 1,
+                           ("x", "dones")),
+    }
+
+    def long_inputs():
+        d = W.gae_inputs(16, 262144, 30, p_term=1e-4)
+        d.update(W.trace_inputs(16, 262144, 31, p_done=1e-4))
+        return d
+
+    return [
+        ("gae_64x512", 64, 512, lambda: W.gae_inputs(64, 512, 10, p_term=0.01),
+         {"gae": (gae, 16, 1, ("rewards", "values", "terminateds"))}),
+        ("truncation_4096x128", E_ENVS, T_STEPS, trunc_inputs, trunc),
+        ("off_policy_1024x2048_18_actions", 1024, 2048, lambda: W.off_policy_inputs(1024, 2048, A=A, seed=40),
+         off),
+        ("long_rows_16x262144", 16, 262144, long_inputs, long_rows),
+    ]
+
+
+def run_configs(torch, R, device, side, stream, world, peak, max_sets=2048):
+    out = {}
+    rot = rotate_bytes(device)
+    for key, E, T, build, cases in config_cases():
+        host = build()
+        res = {"num_envs": E, "seq_len": T}
+        for est, (make, bpe, nout, keys) in cases.items():
+            nbytes = bpe * E * T
+            nset = min(max_sets, max(2, -(-rot // nbytes)))
+            # one device copy of the inputs per set (only the planes this call reads)
+            planes = {k: torch.from_numpy(np.ascontiguousarray(host[k])) for k in keys}
+            fns = []
+            for _ in range(nset):
+                t = {k: v.to(device) for k, v in planes.items()}
+                o = [torch.empty(E, T, device=device) for _ in range(nout)]
+                fns.append(make(R, t, o))
+            us, rng, launches = time_launches(torch, R, fns, side, stream, world)
+            gbs = nbytes / (us * 1e-6) / 1e9
+            res[est] = {"us_per_launch": us, "us_per_launch_range": rng, "launches": launches,
+                        "buffer_sets": nset, "bytes_per_launch": nbytes, "bytes_per_env_step": bpe,
+                        "env_steps_per_s": E * T / (us * 1e-6), "gb_per_s": gbs, "frac_of_hbm_peak": gbs / peak}
+            del fns
+            torch.cuda.empty_cache()
+        out[key] = res
+    return out
+
+
 def run_gpu(args):
     import torch
     from linear_recurrence_scans_02_b200 import rlscan as R
@@ -453,7 +612,8 @@ def run_gpu(args):
     device = torch.device("cuda", local)
     host = host_inputs(seed=rank_seed(rank))
     per_set_bytes = STEP_BYTES_PER_ENV_STEP * E_ENVS * T_STEPS
-    n_sets = max(2, -(-ROTATE_BYTES // per_set_bytes))
+    rot_bytes = rotate_bytes(device)
+    n_sets = max(2, -(-rot_bytes // per_set_bytes))
     sets = [BufferSet(torch, device, ESTIMATORS) for _ in range(n_sets)]
     for s in sets:
         s.fill_from_host(host)
@@ -508,6 +668,16 @@ def run_gpu(args):
     round_graph = capture(torch, [f for s in sets for f in step_fns(s, how)], side)
     ref_rounds = {h: capture(torch, [f for s in sets for f in step_fns(s, h)], side)
                   for h in ("batch", "parallel", "serial") if h != how}
+    # the timed steps: one graph of up to TIMED_GRAPH_STEPS consecutive steps
+    # (steps k, k+1, ... over the rotating sets), replayed as often as K needs,
+    # and one more graph for the remainder, so K steps cost at most
+    # K // TIMED_GRAPH_STEPS + 1 graph launches (each launch adds a gap of a
+    # few microseconds on the device)
+    chunk = args.steps if args.steps <= TIMED_GRAPH_STEPS else (TIMED_GRAPH_STEPS // n_sets) * n_sets
+    steps_graph = capture(torch, [f for k in range(chunk) for f in step_fns(sets[k % n_sets], how)], side)
+    rest = args.steps % chunk
+    rest_graph = (capture(torch, [f for k in range(rest) for f in step_fns(sets[k % n_sets], how)], side)
+                  if rest else None)
     torch.cuda.synchronize()
 
     def run_steps(k0, count):
@@ -522,14 +692,31 @@ def run_gpu(args):
                 k += 1
                 count -= 1
 
+    def run_timed_steps():
+        for _ in range(args.steps // chunk):
+            steps_graph.replay()
+        if rest_graph is not None:
+            rest_graph.replay()
+
     clocks = ClockSampler(local)
     with clocks:
         stream = torch.cuda.current_stream(device)
+        # every graph the timed region may replay is replayed once first (its
+        # first replay uploads it to the device), then the warm-up steps
+        round_graph.replay()
+        for sg in step_graphs:
+            sg.replay()
+        steps_graph.replay()
+        if rest_graph is not None:
+            rest_graph.replay()
         run_steps(0, args.warmup)
         barrier_sync(world)
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # the device idles on a short spin while the host enqueues the timed
+        # replays, so the region times the steps and not their submission
+        torch.cuda._sleep(SUBMIT_SPIN_CYCLES)
         ev0.record(stream)
-        run_steps(0, args.steps)
+        run_timed_steps()
         ev1.record(stream)
         barrier_sync(world)
         step_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
@@ -554,7 +741,7 @@ def run_gpu(args):
         per_est = {}
         for est in names + list(EXTRA_CALLS):
             nbytes = bytes_per_env_step(est) * E_ENVS * T_STEPS
-            n_rot = max(2, -(-ROTATE_BYTES // nbytes))
+            n_rot = max(2, -(-rot_bytes // nbytes))
             if est in ESTIMATORS:
                 est_sets = sets + [BufferSet(torch, device, [est]) for _ in range(max(0, n_rot - n_sets))]
             else:  # a call outside the step: buffers of its own only
@@ -601,6 +788,11 @@ def run_gpu(args):
             del g
             del est_sets, fns
         R.rlscan_check()
+
+        # the other workloads of the path (usage shape, truncations,
+        # off-policy with 18 actions, long rows)
+        peak, peak_kind = measured_hbm_peak()
+        configs = {} if args.no_configs else run_configs(torch, R, device, side, stream, world, peak)
 
         # e2e: every step copies its inputs host -> device from pinned memory,
         # runs the eight calls and copies its outputs device -> host, on three
@@ -668,6 +860,11 @@ def run_gpu(args):
     if "gae_with_returns" in extra:
         extra["gae_with_returns"]["separate_gae_plus_lambda_returns_us"] = (
             per_est["gae"]["us_per_launch"] + per_est["lambda_returns"]["us_per_launch"])
+    if "gae_returns_vtrace" in extra and "gae_with_returns" in extra:
+        rec = extra["gae_returns_vtrace"]
+        rec["separate_gae_with_returns_plus_vtrace_us"] = (
+            extra["gae_with_returns"]["us_per_launch"] + per_est["vtrace"]["us_per_launch"])
+        rec["separate_bytes_per_env_step"] = bytes_per_env_step("gae_with_returns") + bytes_per_env_step("vtrace")
     dominant = max(per_est, key=lambda e: per_est[e]["us_per_launch"])
     d = per_est[dominant]
     for est, rec in per_est.items():
@@ -703,7 +900,7 @@ def run_gpu(args):
                    "estimators": names, "gamma": GAMMA, "lambda": LAMBDA, "p_done": P_DONE,
                    "bytes_per_env_step": STEP_BYTES_PER_ENV_STEP,
                    "l2": f"inputs larger than L2: {n_sets} rotating buffer sets, "
-                         f"{n_sets * per_set_bytes / 2**20:.0f} MiB > 4x126 MB",
+                         f"{n_sets * per_set_bytes / 2**20:.0f} MiB >= 4x the L2 ({rot_bytes // 4 / 2**20:.0f} MiB)",
                    "timing": "CUDA events around CUDA-graph replays (a graph holds a round of steps)",
                    "step": {"batch": "the eight calls of a step as one rlscan_batch request (one fused launch)",
                             "parallel": "the eight calls of a step as parallel graph branches",
@@ -712,6 +909,7 @@ def run_gpu(args):
         "hbm_gb_per_s_step": STEP_BYTES_PER_ENV_STEP * E_ENVS * T_STEPS * args.steps / (step_ms * 1e-3) / 1e9,
         "per_estimator": per_est,
         "fused_calls": extra,
+        "configs": configs,
         "roofline": roofline,
         "e2e": {"value": job_value(world, e2e_steps, e2e_ms), "unit": "env-steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -783,7 +981,7 @@ def run_sweep(args):
         gamma, p_done = (0.999, 1e-4) if long_row else (GAMMA, P_DONE)
         for est in SWEEP_EST:
             nbytes = bytes_per_env_step(est) * E * T
-            nset = min(64, max(2, -(-ROTATE_BYTES // nbytes)))
+            nset = min(64, max(2, -(-rotate_bytes(device) // nbytes)))
             fns = []
             for k in range(nset):
                 fam = "gae" if est in ("gae", "discounted_returns") else "trace"
@@ -835,7 +1033,18 @@ def run_profile_case(args):
     import torch
     from linear_recurrence_scans_02_b200 import rlscan as R
     torch.cuda.set_device(0)
-    if args.profile_shape:  # GAE at another shape, e.g. 16,262144 (long rows: the look-back path)
+    if args.profile_config == "off_policy":  # multi-action Retrace, 256 x 2048, 18 actions (~90 MB)
+        from linear_recurrence_scans_02_b200 import workloads as W
+        d = {k: torch.from_numpy(v).cuda() for k, v in W.off_policy_inputs(256, 2048, A=18, seed=0).items()}
+        out = torch.empty(256, 2048, device="cuda")
+        for _ in range(args.profile_launches):
+            R.rlscan_retrace(d["rewards"], d["q_values"], d["next_q_values_all"], d["next_target_probs"],
+                             d["log_rhos"], d["terminateds"], d["truncateds"], out, GAMMA, LAMBDA, 1.0)
+        torch.cuda.synchronize()
+        R.rlscan_check()
+        print(f"profile case done: {args.profile_launches} multi-action Retrace launches at 256 x 2048 x 18")
+        return 0
+    if args.profile_shape:  # GAE at another shape, e.g. 16,262144 (long rows: the two-pass path)
         from linear_recurrence_scans_02_b200 import workloads as W
         E, T = (int(v) for v in args.profile_shape.split(","))
         d = W.device_inputs("gae", E, T, seed=0, device=torch.device("cuda", 0), p_done=1e-4)
@@ -872,11 +1081,15 @@ def main(argv=None):
     ap.add_argument("--parallel-steps", action="store_true",
                     help="time a step as its eight calls in parallel graph branches (not one batch request)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other workloads (64x512, truncations, off-policy, long rows)")
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--profile-launches", type=int, default=0,
                     help="run N eager launches of each estimator and exit (small case for ncu)")
     ap.add_argument("--profile-only", default="", help="comma-separated estimators for --profile-launches")
     ap.add_argument("--profile-shape", default="", help="E,T: --profile-launches runs GAE at this shape instead")
+    ap.add_argument("--profile-config", default="", choices=["", "off_policy"],
+                    help="off_policy: --profile-launches runs multi-action Retrace (256 x 2048, 18 actions)")
     ap.add_argument("--sweep", action="store_true",
                     help="time four estimators over the E x T size grid and 16 x 262144, one JSON line per point")
     args = ap.parse_args(argv)

@@ -61,7 +61,14 @@
 extern "C" {
 #endif
 
-#define RLSCAN_VERSION 110 /* 1.1.0: the _ex entry points (layout and done-convention options) and rlscan_batch */
+/* 1.2.0: rlscan_gae_vtrace (GAE, TD(lambda) returns and V-Trace in one pass)
+ * and its batch kind; rlscan_call holds four outputs and a vtrace_lambda
+ * field at its end, so its size changed: clients built against an earlier
+ * rlscan_call must be rebuilt (their rlscan_version() check fails).
+ * 1.1.1: rlscan_call gained flag_dtype after dtype, which moved every later
+ * field.  1.1.0: the _ex entry points (layout and done-convention options)
+ * and rlscan_batch. */
+#define RLSCAN_VERSION 120
 
 /* Every entry point is exported from librlscan.so (built with hidden
  * visibility for everything else). */
@@ -168,6 +175,28 @@ RLSCAN_API int rlscan_vtrace(const float *log_rhos, const float *rewards, const 
                   float rho_bar, float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * GAE advantages, TD(lambda) returns and V-Trace targets and advantages in
+ * one pass (README "Kernels": compute_gae, compute_lambda_returns and
+ * compute_vtrace over the same rewards, values and flags).  The two
+ * recurrences, GAE's (gamma lambda, delta_t) and V-Trace's (gamma c_t,
+ * rho_t delta_t) with the common delta_t = r_t + gamma boot_t - V_t, are
+ * scanned together as one pair, so the inputs are read once for all four
+ * outputs (32 bytes per env-step instead of 44 for rlscan_gae_with_returns
+ * plus rlscan_vtrace).  advantages_t as rlscan_gae; returns_t = A_t + V_t as
+ * rlscan_gae_with_returns (NULL: not written); vs_t and pg_advantages_t as
+ * rlscan_vtrace with its lambda_ = vtrace_lambda (1 = IMPALA).  Each output
+ * equals the separate entry point's on the same inputs up to fp32 rounding.
+ * Inputs as rlscan_vtrace; outputs [E,T] (four, none overlapping another or
+ * an input).  Errors as rlscan_vtrace.
+ */
+RLSCAN_API int rlscan_gae_vtrace(const float *log_rhos, const float *rewards, const float *values,
+                                 const float *terminateds, const float *truncateds, const float *bootstrap_values,
+                                 const float *last_values, float *advantages, float *returns, float *vs,
+                                 float *pg_advantages, int64_t E, int64_t T, float gamma, float lambda_,
+                                 float vtrace_lambda, float rho_bar, float c_bar, void *ws, size_t ws_bytes,
+                                 cudaStream_t stream);
+
+/*
  * Retrace(lambda) (README "Kernels": compute_retrace, "off-policy return
  * estimate with truncated IS ratios"; with-truncations paragraph:
  * terminated and truncated are both mandatory and there is no bootstrap
@@ -250,8 +279,11 @@ RLSCAN_API int rlscan_episodic_prefix_sum(const void *x, int dtype, const float 
  * held on every GPU that loads the library until the process exits.  The
  * first call on a device looks up that array's device address (with that
  * device current) and caches it; make that first call before any stream
- * capture.  Every call clears the part of the array it uses with
- * cudaMemsetAsync on `stream` and allocates nothing.
+ * capture.  The cached address belongs to the device's context as it was
+ * then: after cudaDeviceReset on that device it is stale, so a process that
+ * resets a device must not call this entry point on it again.  Every call
+ * clears the part of the array it uses with cudaMemsetAsync on `stream` and
+ * allocates nothing.
  * Limit: shapes whose tile plan needs more scratch than the array holds
  * (rows split over more than about 65,000 tiles) return RLSCAN_ERR_WORKSPACE
  * with the sizes in rlscan_last_error().
@@ -317,6 +349,12 @@ RLSCAN_API int rlscan_vtrace_ex(const float *log_rhos, const float *rewards, con
                                 const float *last_values, float *vs, float *pg_advantages, int64_t E, int64_t T,
                                 float gamma, float lambda_, float rho_bar, float c_bar, unsigned options,
                                 void *ws, size_t ws_bytes, cudaStream_t stream);
+RLSCAN_API int rlscan_gae_vtrace_ex(const float *log_rhos, const float *rewards, const float *values,
+                                    const float *terminateds, const float *truncateds,
+                                    const float *bootstrap_values, const float *last_values, float *advantages,
+                                    float *returns, float *vs, float *pg_advantages, int64_t E, int64_t T,
+                                    float gamma, float lambda_, float vtrace_lambda, float rho_bar, float c_bar,
+                                    unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream);
 RLSCAN_API int rlscan_retrace_ex(const float *rewards, const float *q_values, const float *next_q_values_all,
                                  const float *next_target_probs, const float *log_rhos, const float *terminateds,
                                  const float *truncateds, float *q_ret, int64_t E, int64_t T, int64_t A,
@@ -371,9 +409,12 @@ RLSCAN_API int rlscan_episodic_prefix_sum_ex(const void *x, int dtype, const flo
  *   RLSCAN_KIND_GAE_TYPED           in: as GAE; out: advantages returns (returns nullable);
  *                                   dtype = value_dtype, flag_dtype = flag_dtype of
  *                                   rlscan_gae_typed
+ *   RLSCAN_KIND_GAE_VTRACE          in: as VTRACE; out: advantages returns vs pg_advantages
+ *                                   (returns nullable); lambda_ = GAE's, vtrace_lambda = V-Trace's
  * Scalars a kind does not take are ignored (lambda_ for discounted returns,
- * rho_bar and c_bar outside V-Trace and Retrace, A outside Retrace, dtype
- * outside the prefix sum and typed GAE, flag_dtype outside typed GAE).
+ * vtrace_lambda outside GAE_VTRACE, rho_bar and c_bar outside V-Trace and
+ * Retrace, A outside Retrace, dtype outside the prefix sum and typed GAE,
+ * flag_dtype outside typed GAE).
  * options: as for the _ex entry points.
  *
  * The calls run concurrently: no call's output may overlap any other
@@ -393,11 +434,12 @@ typedef enum rlscan_kind {
     RLSCAN_KIND_DISCOUNTED_RETURNS = 6,
     RLSCAN_KIND_ELIGIBILITY_TRACES = 7,
     RLSCAN_KIND_EPISODIC_PREFIX_SUM = 8,
-    RLSCAN_KIND_GAE_TYPED = 9
+    RLSCAN_KIND_GAE_TYPED = 9,
+    RLSCAN_KIND_GAE_VTRACE = 10
 } rlscan_kind;
 
 #define RLSCAN_CALL_MAX_IN 8
-#define RLSCAN_CALL_MAX_OUT 2
+#define RLSCAN_CALL_MAX_OUT 4
 /* Largest number of calls in one rlscan_batch request. */
 #define RLSCAN_BATCH_MAX 16
 
@@ -410,6 +452,7 @@ typedef struct rlscan_call {
     float gamma, lambda_, rho_bar, c_bar;
     const void *in[RLSCAN_CALL_MAX_IN];
     void *out[RLSCAN_CALL_MAX_OUT];
+    float vtrace_lambda; /* RLSCAN_KIND_GAE_VTRACE: V-Trace's lambda (lambda_ is GAE's) */
 } rlscan_call;
 
 RLSCAN_API int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes, cudaStream_t stream);

@@ -216,14 +216,13 @@ struct LambdaReturnsEst {
                 const bool rowend = elem_row_end<kFast, V>(rm, k);
                 // G_t = r_t + gamma * boot_t + (scan) gamma lambda G_{t+1}, with
                 // boot_t = (1 - lambda) V_{t+1} inside the row, the last value at a
-                // row end (G_{t+1} = V_{t+1} = last value), the bootstrap value at a
-                // truncation and 0 at a termination
+                // row end ((1 - lambda) V_T + lambda G_T with V_T = G_T = the last
+                // value), the bootstrap value at a truncation and 0 at a termination
                 float boot = 0.0f;
                 if (f.trn) boot = pos.one(P.bootstrap_values, k);
                 if (f.cont) {
                     if (rowend) {
-                        const float lv = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
-                        boot = fmaf(one_minus_l, lv, P.lambda_ * lv);
+                        boot = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
                     } else {
                         boot = one_minus_l * ((k + 1 < V) ? S.v[k + 1] : S.v_next);
                     }
@@ -435,6 +434,114 @@ struct VtraceEst {
     }
     template <int V, class Pos>
     static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.vs, S.vs);
+        pos.store(P.pg_advantages, S.pg);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// GAE (with the TD(lambda) returns G_t = A_t + V_t) and V-Trace from one pass
+// over their common inputs: the two recurrences are scanned together as one
+// pair, x = (A, D) with D = vs - V.  Both share delta_t = r_t + gamma boot_t -
+// V_t; GAE's a_t = gamma lambda, b_t = delta_t; V-Trace's a_t = gamma c_t,
+// b_t = rho_t delta_t (rho, c from the V-Trace lambda, rho_bar, c_bar).  Each
+// component's arithmetic is that of GaeEstT and VtraceEst, in the same order.
+// ---------------------------------------------------------------------------
+struct GaeVtraceEst {
+    static constexpr bool kBackward = true;
+    using AT = float2;
+    using BT = float2;
+    struct Params {
+        const float *log_rhos, *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        float *advantages, *returns, *vs, *pg_advantages; // returns may be null
+        float gamma, lambda_, vtrace_lambda, rho_bar, c_bar;
+    };
+    template <int V>
+    struct State {
+        float lr[V], r[V], v[V], te[V], tr[V];
+        float rho[V];
+        float adv[V], ret[V], vs[V], pg[V];
+        float v_next;
+        unsigned chained; // bit k: the traces go on to t+1 inside the row
+    };
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds);
+    }
+    static constexpr int kInputPlanes = 5;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        const float *p[5] = {P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds};
+        return {i < 5 ? p[i] : nullptr, 4};
+    }
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
+                                                State<V> &S, unsigned char *) {
+        const float h_v_next = pos.fetch_next(P.values);
+        pos.load(P.log_rhos, S.lr);
+        pos.load(P.rewards, S.r);
+        pos.load(P.values, S.v);
+        pos.load(P.terminateds, S.te);
+        pos.load(P.truncateds, S.tr);
+        S.v_next = pos.next(S.v, h_v_next);
+    }
+    template <int V, bool kTrunc, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
+                                                  const RowMasks &rm, State<V> &S,
+                                                  float2 (&a)[V], float2 (&b)[V]) {
+        const float gl = P.gamma * P.lambda_;
+        S.chained = 0u;
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (elem_valid<kFast, V>(rm, k)) {
+                const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
+                const bool rowend = elem_row_end<kFast, V>(rm, k);
+                const float ratio = __expf(S.lr[k]);
+                const float rho = fminf(P.rho_bar, ratio);
+                const float c = P.vtrace_lambda * fminf(P.c_bar, ratio);
+                float boot;
+                if (f.cont) {
+                    boot = rowend ? row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows)
+                                  : ((k + 1 < V) ? S.v[k + 1] : S.v_next);
+                } else {
+                    boot = f.trn ? pos.one(P.bootstrap_values, k) : 0.0f;
+                }
+                const bool go = f.cont && !rowend;
+                const float delta = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
+                a[k] = make_float2(go ? gl : 0.0f, go ? P.gamma * c : 0.0f);
+                b[k] = make_float2(delta, rho * delta);
+                S.rho[k] = rho;
+                if (go) S.chained |= (1u << k);
+            } else {
+                a[k] = make_float2(1.0f, 1.0f);
+                b[k] = make_float2(0.0f, 0.0f);
+                S.rho[k] = 0.0f;
+            }
+        }
+    }
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
+                                                  const RowMasks &rm, State<V> &S, float2 (&a)[V],
+                                                  float2 (&b)[V]) {
+        if (P.truncateds != nullptr) {
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
+        } else {
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, pos, rm, S, a, b);
+        }
+    }
+    // as VtraceEst: pg_t = b_t + rho_t gamma D_{t+1} where the trace goes on
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &P, State<V> &S, int k, float2 x, float2 x_next,
+                                               float2 b_k) {
+        S.adv[k] = x.x;
+        S.ret[k] = x.x + S.v[k];
+        S.vs[k] = S.v[k] + x.y;
+        S.pg[k] = ((S.chained >> k) & 1u) ? fmaf(S.rho[k] * P.gamma, x_next.y, b_k.y) : b_k.y;
+    }
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.advantages, S.adv);
+        if (P.returns != nullptr) pos.store(P.returns, S.ret);
         pos.store(P.vs, S.vs);
         pos.store(P.pg_advantages, S.pg);
     }

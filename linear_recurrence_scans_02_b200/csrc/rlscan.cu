@@ -83,9 +83,30 @@ Plan with_mode(Plan p, long long T) {
     return p;
 }
 
-// Fill the GPU: with fewer tiles than this the plan prefers smaller tiles.
-constexpr long long kNumSMs = 148;
-constexpr long long kMinTiles = 2 * kNumSMs;
+// SM count of the current device (queried once per device; B200's 148 when
+// no device can be asked, e.g. when a plan is computed on a host without a
+// GPU).  Plans fill the GPU: with fewer tiles than two per SM a plan prefers
+// smaller tiles.
+constexpr long long kDefaultSMs = 148;
+constexpr int kMaxPlanDevices = 256;
+std::atomic<int> g_sm_count[kMaxPlanDevices];
+
+long long num_sms() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxPlanDevices) {
+        (void)cudaGetLastError();
+        return kDefaultSMs;
+    }
+    int v = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (v <= 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+            (void)cudaGetLastError();
+            return kDefaultSMs;
+        }
+        g_sm_count[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 
@@ -109,6 +130,8 @@ Plan make_plan_tiles(long long E, long long T, long long actions) {
     // Small CTAs (128 threads x 8 elements) overlap best, both with each
     // other inside a launch and with the neighbouring launches; larger tiles
     // only where a row needs them to stay inside one tile.
+    const long long sms = num_sms();
+    const long long min_tiles = 2 * sms;
     const Cfg whole_rows[3] = {C1024, C2048, C4096};
     for (Cfg c : whole_rows) {
         const long long S = kCfgTile[c];
@@ -116,7 +139,7 @@ Plan make_plan_tiles(long long E, long long T, long long actions) {
         const long long nt = ceil_div(n, S);
         const long long nt_split = ceil_div(n, kCfgTile[C1024]);
         // whole rows, unless that leaves SMs idle while split rows would not
-        if (nt >= kNumSMs || nt_split <= nt) {
+        if (nt >= sms || nt_split <= nt) {
             p.cfg = c;
             p.ntiles = nt;
             p.lookback = false;
@@ -127,9 +150,9 @@ Plan make_plan_tiles(long long E, long long T, long long actions) {
     // rows span tiles (long or odd-length rows, or too few rows to fill the
     // GPU): look-back over 2048-element tiles (fewer tiles per row, so a
     // shorter chain of carries), 1024 or 512 when that gives too few tiles
-    p.cfg = ceil_div(n, kCfgTile[C2048]) >= kMinTiles
+    p.cfg = ceil_div(n, kCfgTile[C2048]) >= min_tiles
                 ? C2048
-                : (ceil_div(n, kCfgTile[C1024]) >= kMinTiles ? C1024 : C512);
+                : (ceil_div(n, kCfgTile[C1024]) >= min_tiles ? C1024 : C512);
     p.ntiles = ceil_div(n, kCfgTile[p.cfg]);
     p.lookback = p.ntiles > 1 && (kCfgTile[p.cfg] % T != 0);
     return p;
@@ -229,6 +252,8 @@ struct BatchState {
     int pass;
     FusedBatch fb;
     long long tiles;
+    AnyParams any[kFusedMax]; // each fused fp32 call in the shared body's form
+    bool has_any[kFusedMax];  // false for calls that body does not take
 };
 thread_local BatchState *g_batch = nullptr;
 
@@ -239,14 +264,14 @@ bool batch_dry() { return g_batch != nullptr && g_batch->pass == kBatchDry; }
 // ---------------------------------------------------------------------------
 template <class Est, int NT, int V, int kMode>
 cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const Lookback &lb, size_t smem,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, long long grid = -1) {
     auto kern = tile_scan_kernel<Est, NT, V, kMode>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)g.ntiles);
+    cfg.gridDim = dim3((unsigned)(grid < 0 ? g.ntiles : grid));
     cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -260,14 +285,57 @@ cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const L
 
 template <class Est, Cfg C>
 cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, const Lookback &lb, int mode,
-                       size_t smem, cudaStream_t s) {
+                       size_t smem, cudaStream_t s, long long grid = -1) {
     constexpr int NT = kCfgThreads[C];
     constexpr int V = kCfgTile[C] / NT;
+    // rows that span tiles: the one-pass look-back for multi-action Retrace
+    // (re-reading its per-action rows would cost more than waiting), the two
+    // passes for every other call (split-row plans use 512- to 2048-element
+    // tiles, make_plan_tiles)
+    constexpr bool kMultiAction = std::is_same<Est, RetraceEst<true>>::value;
     switch (mode) {
-    case kModeLookback: return launch_one<Est, NT, V, kModeLookback>(P, g, lb, smem, s);
+    case kModeLookback:
+        if constexpr (kMultiAction) return launch_one<Est, NT, V, kModeLookback>(P, g, lb, smem, s);
+        return cudaErrorInvalidConfiguration;
     case kModeWarp: return launch_one<Est, NT, V, kModeWarp>(P, g, lb, smem, s);
+    case kModeReduce:
+    case kModeCarry:
+        if constexpr (!kMultiAction && (C == C512 || C == C1024 || C == C2048)) {
+            if (mode == kModeReduce) return launch_one<Est, NT, V, kModeReduce>(P, g, lb, smem, s, grid);
+            return launch_one<Est, NT, V, kModeCarry>(P, g, lb, smem, s, grid);
+        }
+        return cudaErrorInvalidConfiguration;
     default: return launch_one<Est, NT, V, kModeBlock>(P, g, lb, smem, s);
     }
+}
+
+// Input bytes per tile a two-pass wave may hold so that pass two re-reads
+// them from L2: a wave's pass one streams them from HBM, pass two finds them
+// in L2 (B200: 126 MB).
+constexpr long long kTwoPassWaveBytes = 64ll << 20;
+
+// Rows that span tiles, single-action calls: pass one (aggregates) and pass
+// two (scan with carries) over waves of consecutive scan-order tiles.
+template <class Est>
+int run_two_pass(const char *name, const typename Est::Params &P, const Geometry &g, Lookback lb, Cfg cfg,
+                 cudaStream_t stream) {
+    const long long tile_bytes = (long long)kCfgTile[cfg] * 4 * Est::kInputPlanes;
+    const long long wave = std::max<long long>(1, kTwoPassWaveBytes / tile_bytes);
+    for (long long t0 = 0; t0 < g.ntiles; t0 += wave) {
+        lb.tile_base = t0;
+        const long long cnt = std::min<long long>(wave, g.ntiles - t0);
+        for (int mode : {kModeReduce, kModeCarry}) {
+            cudaError_t e;
+            switch (cfg) {
+            case C512: e = launch_cfg<Est, C512>(P, g, lb, mode, 0, stream, cnt); break;
+            case C1024: e = launch_cfg<Est, C1024>(P, g, lb, mode, 0, stream, cnt); break;
+            case C2048: e = launch_cfg<Est, C2048>(P, g, lb, mode, 0, stream, cnt); break;
+            default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+            }
+            if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
+        }
+    }
+    return ok();
 }
 
 template <class Est>
@@ -303,14 +371,17 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
         constexpr long long kS = (long long)kFusedNT * kFusedVMax;
         if (g_batch != nullptr && actions == 1 && kS % T == 0 && g_batch->fb.n < kFusedMax) {
             static_assert(sizeof(typename Est::Params) <= kFusedParamBytes, "params fit a fused item");
-            FusedItem &it = g_batch->fb.item[g_batch->fb.n++];
+            const int slot = g_batch->fb.n++;
+            FusedItem &it = g_batch->fb.item[slot];
             std::memset(it.params, 0, sizeof it.params);
             std::memcpy(it.params, &P, sizeof P);
             it.g = g;
             it.kind = FusedKindOf<Est>::value;
+            g_batch->has_any[slot] = to_any(P, g_batch->any[slot]);
             return ok();
         }
     }
+    if (plan.lookback && actions == 1) return run_two_pass<Est>(name, P, g, lb, plan.cfg, stream);
     const size_t smem = actions > 1 ? multi_smem_bytes(plan.cfg, actions) : 0;
     cudaError_t e;
     switch (plan.cfg) {
@@ -355,6 +426,12 @@ int run_multi(const char *name, const typename Est::Params &P, long long E, long
     if (batch_dry()) return ok();
     const size_t smem = multi_smem_bytes(plan.cfg, actions);
     cudaError_t e;
+    if (plan.lookback) {
+        // the one-pass look-back needs zeroed progress flags; a two-pass call
+        // before this one may have left its aggregates in the workspace
+        e = cudaMemsetAsync(ws, 0, workspace_for(plan), stream);
+        if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: cudaMemsetAsync(workspace): %s", name, cudaGetErrorString(e));
+    }
     switch (plan.cfg) {
     case R512: e = launch_cfg<Est, R512>(P, g, lb, plan.mode, smem, stream); break;
     case R256: e = launch_cfg<Est, R256>(P, g, lb, plan.mode, smem, stream); break;
@@ -393,7 +470,7 @@ struct TmPlan {
 TmPlan tm_plan(long long E, long long T) {
     TmPlan p;
     const long long kMinBlocks = 120;
-    p.G = (E / 32 >= 4 * 148 && T <= 256) ? 32 : (E / 16 >= kMinBlocks ? 16 : 8);
+    p.G = (E / 32 >= 4 * num_sms() && T <= 256) ? 32 : (E / 16 >= kMinBlocks ? 16 : 8);
     const long long chunks = ceil_div(T, kTmV);
     const long long nw = ceil_div(chunks, 32 / p.G);
     p.nw = (int)(nw < 1 ? 1 : (nw > kTmMaxWarps ? kTmMaxWarps : nw));
@@ -637,6 +714,52 @@ int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *valu
                   float *pg_advantages, int64_t E, int64_t T, float gamma, float lambda_, float rho_bar,
                   float c_bar, void *ws, size_t ws_bytes, cudaStream_t stream) {
     return rlscan_vtrace_ex(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values, vs, pg_advantages, E, T, gamma, lambda_, rho_bar, c_bar, 0u, ws, ws_bytes, stream);
+}
+
+int rlscan_gae_vtrace_ex(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
+                         const float *truncateds, const float *bootstrap_values, const float *last_values,
+                         float *advantages, float *returns, float *vs, float *pg_advantages, int64_t E, int64_t T,
+                         float gamma, float lambda_, float vtrace_lambda, float rho_bar, float c_bar,
+                         unsigned options, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    RLSCAN_TRY(check_options(options, false));
+    RLSCAN_TRY(check_shape(E, T));
+    RLSCAN_TRY(check_scalar(gamma, "gamma"));
+    RLSCAN_TRY(check_scalar(lambda_, "lambda_"));
+    RLSCAN_TRY(check_scalar(vtrace_lambda, "vtrace_lambda"));
+    RLSCAN_TRY(check_scalar(rho_bar, "rho_bar"));
+    RLSCAN_TRY(check_scalar(c_bar, "c_bar"));
+    if (E == 0 || T == 0) return ok();
+    RLSCAN_TRY(require(log_rhos, "log_rhos"));
+    RLSCAN_TRY(require(rewards, "rewards"));
+    RLSCAN_TRY(require(values, "values"));
+    RLSCAN_TRY(require(advantages, "advantages"));
+    RLSCAN_TRY(require(vs, "vs"));
+    RLSCAN_TRY(require(pg_advantages, "pg_advantages"));
+    if (truncateds && !bootstrap_values) return fail(RLSCAN_ERR_INVALID_ARG, "truncateds given without bootstrap_values");
+    const size_t pb = plane_bytes(E, T);
+    const Span ins[] = {{log_rhos, pb, "log_rhos"}, {rewards, pb, "rewards"}, {values, pb, "values"},
+                        {terminateds, pb, "terminateds"}, {truncateds, pb, "truncateds"},
+                        {bootstrap_values, pb, "bootstrap_values"}, {last_values, (size_t)E * 4, "last_values"}};
+    const Span outs[] = {{advantages, pb, "advantages"}, {returns, pb, "returns"}, {vs, pb, "vs"},
+                         {pg_advantages, pb, "pg_advantages"}};
+    RLSCAN_TRY(check_aliasing(ins, 7, outs, 4));
+    GaeVtraceEst::Params P{log_rhos, rewards, values, terminateds, truncateds,
+                           truncateds ? bootstrap_values : nullptr, last_values, advantages, returns, vs,
+                           pg_advantages, gamma, lambda_, vtrace_lambda, rho_bar, c_bar};
+    if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<GaeVtraceEst>("rlscan_gae_vtrace", P, E, T, stream);
+    return run<GaeVtraceEst>("rlscan_gae_vtrace", P, E, T, 1, ws, ws_bytes, stream,
+                             aligned16({log_rhos, rewards, values, terminateds, truncateds, advantages, returns, vs,
+                                        pg_advantages}));
+}
+
+int rlscan_gae_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
+                      const float *truncateds, const float *bootstrap_values, const float *last_values,
+                      float *advantages, float *returns, float *vs, float *pg_advantages, int64_t E, int64_t T,
+                      float gamma, float lambda_, float vtrace_lambda, float rho_bar, float c_bar, void *ws,
+                      size_t ws_bytes, cudaStream_t stream) {
+    return rlscan_gae_vtrace_ex(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values,
+                                advantages, returns, vs, pg_advantages, E, T, gamma, lambda_, vtrace_lambda, rho_bar,
+                                c_bar, 0u, ws, ws_bytes, stream);
 }
 
 int rlscan_retrace_ex(const float *rewards, const float *q_values, const float *next_q_values_all,
@@ -906,24 +1029,32 @@ int rlscan_plan(int64_t E, int64_t T, int64_t actions, int64_t *tile_elems, int 
 // rlscan_batch
 // ---------------------------------------------------------------------------
 
-// Byte extent of argument slot `slot` of a call (its input when in_slot,
-// else its output); 0 for slots the kind does not have.
+// Element size of a plane dtype; 0 for a value that names no dtype.  Only
+// called on calls that the dry pass (step 1 of rlscan_batch) has accepted,
+// so every dtype reaching it is one its kind takes.
 static size_t dtype_bytes(int dtype) {
     switch (dtype) {
+    case RLSCAN_F32:
+    case RLSCAN_I32: return 4;
     case RLSCAN_BF16:
     case RLSCAN_F16: return 2;
     case RLSCAN_U8: return 1;
-    default: return 4;
+    default: return 0;
     }
 }
+
+// Byte extent of argument slot `slot` of a call (its input when in_slot,
+// else its output); 0 for slots the kind does not have.
 
 static size_t call_slot_bytes(const rlscan_call &c, bool in_slot, int slot) {
     const size_t n = (size_t)(c.E * c.T), plane = n * 4u, row = (size_t)c.E * 4u;
     if (!in_slot) {
-        const int nout = (c.kind == RLSCAN_KIND_GAE_WITH_RETURNS || c.kind == RLSCAN_KIND_VTRACE ||
-                          c.kind == RLSCAN_KIND_GAE_TYPED)
-                             ? 2
-                             : 1;
+        const int nout = c.kind == RLSCAN_KIND_GAE_VTRACE
+                             ? 4
+                             : ((c.kind == RLSCAN_KIND_GAE_WITH_RETURNS || c.kind == RLSCAN_KIND_VTRACE ||
+                                 c.kind == RLSCAN_KIND_GAE_TYPED)
+                                    ? 2
+                                    : 1);
         return slot < nout ? plane : 0;
     }
     switch (c.kind) {
@@ -935,7 +1066,8 @@ static size_t call_slot_bytes(const rlscan_call &c, bool in_slot, int slot) {
     case RLSCAN_KIND_GAE:
     case RLSCAN_KIND_GAE_WITH_RETURNS:
     case RLSCAN_KIND_LAMBDA_RETURNS: return slot < 5 ? plane : (slot == 5 ? row : 0);
-    case RLSCAN_KIND_VTRACE: return slot < 6 ? plane : (slot == 6 ? row : 0);
+    case RLSCAN_KIND_VTRACE:
+    case RLSCAN_KIND_GAE_VTRACE: return slot < 6 ? plane : (slot == 6 ? row : 0);
     case RLSCAN_KIND_RETRACE: return (slot == 2 || slot == 3) ? plane * (size_t)(c.A > 0 ? c.A : 1) : (slot < 7 ? plane : 0);
     case RLSCAN_KIND_DISCOUNTED_RETURNS: return slot < 4 ? plane : (slot == 4 ? row : 0);
     case RLSCAN_KIND_ELIGIBILITY_TRACES:
@@ -957,6 +1089,10 @@ static int call_dispatch(const rlscan_call &c, void *ws, size_t ws_bytes, cudaSt
     case RLSCAN_KIND_VTRACE:
         return rlscan_vtrace_ex(in[0], in[1], in[2], in[3], in[4], in[5], in[6], out[0], out[1], c.E, c.T, c.gamma,
                                 c.lambda_, c.rho_bar, c.c_bar, c.options, ws, ws_bytes, stream);
+    case RLSCAN_KIND_GAE_VTRACE:
+        return rlscan_gae_vtrace_ex(in[0], in[1], in[2], in[3], in[4], in[5], in[6], out[0], out[1], out[2], out[3],
+                                    c.E, c.T, c.gamma, c.lambda_, c.vtrace_lambda, c.rho_bar, c.c_bar, c.options, ws,
+                                    ws_bytes, stream);
     case RLSCAN_KIND_RETRACE:
         return rlscan_retrace_ex(in[0], in[1], in[2], in[3], in[4], in[5], in[6], out[0], c.E, c.T, c.A, c.gamma,
                                  c.lambda_, c.c_bar, c.options, ws, ws_bytes, stream);
@@ -979,18 +1115,52 @@ static int call_dispatch(const rlscan_call &c, void *ws, size_t ws_bytes, cudaSt
     }
 }
 
-// Elements per thread of a fused launch: 4 when it mixes three or more
-// estimators and every row fits a 512-element tile, else 8 (measured at
-// 4096 x 128: eight estimators 15.4 us at 4 against 17.7 us at 8; eight
-// GAE calls 10.5 us at 8 against 12.8 us at 4).  Then each item's tiling.
-static int fused_layout(FusedBatch &fb, long long *tiles) {
+// Which kernel and how many elements per thread a fused request takes.
+// Requests mixing three or more estimators run every fp32 call on the shared
+// body (one instruction stream for all of them, fused_any.cuh) when every
+// fp32 call's rows hold whole multiples of V elements; otherwise each call
+// runs its own estimator's body, 4 elements per thread when the request
+// mixes three or more estimators and every row fits a 512-element tile
+// (smaller code per estimator), else 8.
+struct FusedChoice {
+    bool shared_body;
+    int V;
+};
+static FusedChoice choose_fused(const BatchState &st) {
+    const FusedBatch &fb = st.fb;
     unsigned kinds = 0u;
     bool fit4 = true;
     for (int i = 0; i < fb.n; ++i) {
         kinds |= 1u << fb.item[i].kind;
         if ((long long)(kFusedNT * 4) % fb.item[i].g.seq_len != 0) fit4 = false;
     }
-    const int V = (__builtin_popcount(kinds) >= 3 && fit4) ? 4 : 8;
+    const bool mixed = __builtin_popcount(kinds) >= 3;
+    if (mixed) {
+        constexpr int kSharedV = 4;
+        bool shared_ok = true;
+        for (int i = 0; i < fb.n; ++i) {
+            const long long T = fb.item[i].g.seq_len;
+            if ((long long)(kFusedNT * kSharedV) % T != 0) shared_ok = false; // rows whole in a tile
+            if (st.has_any[i] && T < kSharedV) shared_ok = false;             // and whole in a thread
+        }
+        if (shared_ok) return {true, kSharedV};
+    }
+    return {false, (mixed && fit4) ? 4 : 8};
+}
+
+// Tiling of each item of a fused launch of V elements per thread; with the
+// shared body, fp32 items carry their AnyParams.
+static void fused_layout(BatchState &st, const FusedChoice &ch, long long *tiles) {
+    FusedBatch &fb = st.fb;
+    const int V = ch.V;
+    if (ch.shared_body) {
+        for (int i = 0; i < fb.n; ++i) {
+            if (!st.has_any[i]) continue;
+            static_assert(sizeof(AnyParams) <= kFusedParamBytes, "shared-body params fit a fused item");
+            std::memset(fb.item[i].params, 0, sizeof fb.item[i].params);
+            std::memcpy(fb.item[i].params, &st.any[i], sizeof(AnyParams));
+        }
+    }
     long long begin = 0;
     for (int i = 0; i < fb.n; ++i) {
         FusedItem &it = fb.item[i];
@@ -1002,7 +1172,6 @@ static int fused_layout(FusedBatch &fb, long long *tiles) {
         begin += it.g.ntiles;
     }
     *tiles = begin;
-    return V;
 }
 
 // Runs every call of the request in the given pass; the first failure is
@@ -1056,7 +1225,9 @@ int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes
     st.pass = kBatchRecord;
     RLSCAN_TRY(batch_pass(st, calls, ncalls, ws, ws_bytes, stream));
     if (st.fb.n == 0) return ok();
-    const int V = fused_layout(st.fb, &st.tiles);
+    const FusedChoice ch = choose_fused(st);
+    fused_layout(st, ch, &st.tiles);
+    const int V = ch.V;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)st.tiles);
     cfg.blockDim = dim3(kFusedNT);
@@ -1066,8 +1237,13 @@ int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    const cudaError_t e = V == 4 ? cudaLaunchKernelEx(&cfg, fused_tile_kernel<4>, st.fb)
-                                 : cudaLaunchKernelEx(&cfg, fused_tile_kernel<8>, st.fb);
+    cudaError_t e;
+    if (ch.shared_body)
+        e = V == 4 ? cudaLaunchKernelEx(&cfg, fused_any_kernel<4>, st.fb)
+                   : cudaLaunchKernelEx(&cfg, fused_any_kernel<8>, st.fb);
+    else
+        e = V == 4 ? cudaLaunchKernelEx(&cfg, fused_tile_kernel<4>, st.fb)
+                   : cudaLaunchKernelEx(&cfg, fused_tile_kernel<8>, st.fb);
     if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "rlscan_batch: fused launch failed: %s", cudaGetErrorString(e));
     return ok();
 }

@@ -164,6 +164,45 @@ __device__ __forceinline__ unsigned to_bits(int32_t v) { return static_cast<unsi
 __device__ __forceinline__ uint32_t from_bits(unsigned u, uint32_t) { return u; }
 __device__ __forceinline__ int32_t from_bits(unsigned u, int32_t) { return static_cast<int32_t>(u); }
 
+// A pair of independent fp32 recurrences scanned together with the
+// component-wise operator: two estimators that share one pass over their
+// common inputs (the pair is cut only where both components are).
+__device__ __forceinline__ float2 apply_pair(float2 a, float2 b, float2 x) {
+    return make_float2(apply_pair(a.x, b.x, x.x), apply_pair(a.y, b.y, x.y));
+}
+__device__ __forceinline__ void combine(float2 &a1, float2 &b1, float2 a2, float2 b2) {
+    b1 = apply_pair(a1, b1, b2);
+    a1 = make_float2(a1.x * a2.x, a1.y * a2.y);
+}
+__device__ __forceinline__ float2 identity_a(float2) { return make_float2(1.0f, 1.0f); }
+__device__ __forceinline__ float2 identity_b(float2) { return make_float2(0.0f, 0.0f); }
+
+// The multiplier of a map that ignores its input (a cut chain), and the test
+// for one.
+__device__ __forceinline__ float cut_a(float) { return 0.0f; }
+__device__ __forceinline__ uint32_t cut_a(uint32_t) { return 0u; }
+__device__ __forceinline__ float2 cut_a(float2) { return make_float2(0.0f, 0.0f); }
+__device__ __forceinline__ bool is_cut(float a) { return a == 0.0f; }
+__device__ __forceinline__ bool is_cut(uint32_t a) { return a == 0u; }
+__device__ __forceinline__ bool is_cut(float2 a) { return a.x == 0.0f && a.y == 0.0f; }
+
+// Warp shuffles of scan values (full warp).
+template <class T>
+__device__ __forceinline__ T shfl_down(T v, int d) { return __shfl_down_sync(kFullMask, v, d); }
+template <class T>
+__device__ __forceinline__ T shfl_up(T v, int d) { return __shfl_up_sync(kFullMask, v, d); }
+template <class T>
+__device__ __forceinline__ T shfl_idx(T v, int l) { return __shfl_sync(kFullMask, v, l); }
+__device__ __forceinline__ float2 shfl_down(float2 v, int d) {
+    return make_float2(__shfl_down_sync(kFullMask, v.x, d), __shfl_down_sync(kFullMask, v.y, d));
+}
+__device__ __forceinline__ float2 shfl_up(float2 v, int d) {
+    return make_float2(__shfl_up_sync(kFullMask, v.x, d), __shfl_up_sync(kFullMask, v.y, d));
+}
+__device__ __forceinline__ float2 shfl_idx(float2 v, int l) {
+    return make_float2(__shfl_sync(kFullMask, v.x, l), __shfl_sync(kFullMask, v.y, l));
+}
+
 // Inclusive warp scan in scan order: forward = increasing lane, backward =
 // decreasing lane.  `width` (a power of two) bounds the distance a value
 // must travel: when rows start every `width` lanes, later steps would only
@@ -174,12 +213,12 @@ __device__ __forceinline__ void warp_inclusive_scan(AT &a, BT &b, int lane, int 
     for (int d = 1; d < 32; d <<= 1) {
         if (d >= width) break;
         if (kBackward) {
-            AT ao = __shfl_down_sync(kFullMask, a, d);
-            BT bo = __shfl_down_sync(kFullMask, b, d);
+            AT ao = shfl_down(a, d);
+            BT bo = shfl_down(b, d);
             if (lane + d < 32) combine(a, b, ao, bo);
         } else {
-            AT ao = __shfl_up_sync(kFullMask, a, d);
-            BT bo = __shfl_up_sync(kFullMask, b, d);
+            AT ao = shfl_up(a, d);
+            BT bo = shfl_up(b, d);
             if (lane >= d) combine(a, b, ao, bo);
         }
     }
@@ -190,12 +229,12 @@ __device__ __forceinline__ void warp_inclusive_scan(AT &a, BT &b, int lane, int 
 template <bool kBackward, class AT, class BT>
 __device__ __forceinline__ void warp_exclusive_from_inclusive(AT ia, BT ib, int lane, AT &ea, BT &eb) {
     if (kBackward) {
-        ea = __shfl_down_sync(kFullMask, ia, 1);
-        eb = __shfl_down_sync(kFullMask, ib, 1);
+        ea = shfl_down(ia, 1);
+        eb = shfl_down(ib, 1);
         if (lane == 31) { ea = identity_a(ia); eb = identity_b(ib); }
     } else {
-        ea = __shfl_up_sync(kFullMask, ia, 1);
-        eb = __shfl_up_sync(kFullMask, ib, 1);
+        ea = shfl_up(ia, 1);
+        eb = shfl_up(ib, 1);
         if (lane == 0) { ea = identity_a(ia); eb = identity_b(ib); }
     }
 }
@@ -230,6 +269,7 @@ struct Lookback {
     unsigned spin_limit; // polls before a wait gives up
     long long withhold;  // scan-order tile that never publishes (test hook), -1 = none
     long long row_tiles; // tiles per row when rows are whole multiples of a tile, else 0
+    long long tile_base; // two-pass modes: scan-order index of the launch's first tile
 };
 
 
@@ -434,12 +474,12 @@ __device__ BT lookback_carry(const Lookback &lb, long long j, long long k_min, b
         // ordered composition over lanes 0..last: lane 0 (nearest) applied last
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            const AT oa = __shfl_down_sync(kFullMask, la, d);
-            const BT ob = __shfl_down_sync(kFullMask, lb_, d);
+            const AT oa = shfl_down(la, d);
+            const BT ob = shfl_down(lb_, d);
             if (lane + d < 32) combine(la, lb_, oa, ob);
         }
-        la = __shfl_sync(kFullMask, la, 0);
-        lb_ = __shfl_sync(kFullMask, lb_, 0);
+        la = shfl_idx(la, 0);
+        lb_ = shfl_idx(lb_, 0);
         combine(acc_a, acc_b, la, lb_);
         if (stops) { // the composed map starts from a cut: its b is the carry
             carry = acc_b;
@@ -450,6 +490,115 @@ __device__ BT lookback_carry(const Lookback &lb, long long j, long long k_min, b
         st_relaxed_gpu(&me->x, to_bits(apply_pair(ta, tb, carry)));
         st_release_gpu(&me->status, 2u);
     }
+    return carry;
+}
+
+// ---------------------------------------------------------------------------
+// Two-pass carries (rows that span tiles, single-action calls).  Pass one
+// (kModeReduce) writes every tile's aggregate (a, b), composed in scan
+// order, into its 16-byte slot as {a, b, 0, 0}; pass two (kModeCarry), a
+// later launch on the same stream, re-reads each tile (from L2 when the
+// launch's tiles fit it), scans it, and takes its carry from the complete
+// aggregates of the tiles before it in its row.  Pass two also publishes
+// each tile's inclusive value in the slot's second half, {1, x} as one
+// 64-bit store, as a shortcut for later tiles: a reader sees either 0 there
+// (not yet) or the whole pair, never half of it.  Nothing ever waits: the
+// aggregates are complete before pass two starts (it waits for pass one's
+// grid first), and the walk over them ends at the row's first tile at the
+// latest.  Every slot a launch reads is written by its own pass one, so the
+// workspace needs no initial content.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ld_slot_halves(const TileSlot *slot, unsigned long long &ab,
+                                               unsigned long long &fx) {
+    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(ab), "=l"(fx) : "l"(slot) : "memory");
+}
+// Scalar recurrences (fp32, int32): {a, b} then {flag, x}.
+template <class AT, class BT>
+__device__ __forceinline__ void publish_aggregate(TileSlot *slot, AT a, BT b) {
+    *reinterpret_cast<uint4 *>(slot) = make_uint4(to_bits(a), to_bits(b), 0u, 0u);
+}
+template <class BT>
+__device__ __forceinline__ void publish_inclusive(TileSlot *slot, BT x) {
+    const unsigned long long v = 1ull | ((unsigned long long)to_bits(x) << 32);
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(reinterpret_cast<char *>(slot) + 8), "l"(v)
+                 : "memory");
+}
+// The map slot k stands for: its inclusive value when published (a cut map),
+// else its aggregate.
+template <class AT, class BT>
+__device__ __forceinline__ void read_slot(const TileSlot *slot, AT &a, BT &b) {
+    unsigned long long ab, fx;
+    ld_slot_halves(slot, ab, fx);
+    if ((unsigned)fx != 0u) {
+        a = cut_a(a);
+        b = from_bits((unsigned)(fx >> 32), b);
+    } else {
+        a = from_bits((unsigned)ab, a);
+        b = from_bits((unsigned)(ab >> 32), b);
+    }
+}
+// Pairs of recurrences: the aggregate {a.x, a.y, b.x, b.y} fills the slot,
+// so pairs publish no inclusive values and walks compose aggregates only.
+__device__ __forceinline__ void publish_aggregate(TileSlot *slot, float2 a, float2 b) {
+    *reinterpret_cast<uint4 *>(slot) =
+        make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
+}
+__device__ __forceinline__ void publish_inclusive(TileSlot *, float2) {}
+__device__ __forceinline__ void read_slot(const TileSlot *slot, float2 &a, float2 &b) {
+    const uint4 v = ld_relaxed_gpu_v4(slot);
+    a = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+    b = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+
+// Carry into scan-order tile j from the aggregates of tiles k_min .. j-1,
+// called by all 32 lanes of one warp.  Lane i reads tile base - i of each
+// window of 32 (nearest first); a tile with a published inclusive value, or
+// whose aggregate cuts the chain (a == 0), ends the walk.  Lane 0 publishes
+// this tile's inclusive value.
+template <class AT, class BT>
+__device__ BT carry_from_aggregates(const Lookback &lb, long long j, long long k_min, bool needs_carry, AT ta,
+                                    BT tb, int lane) {
+    TileSlot *me = lb.slots + j;
+    if (!needs_carry) {
+        if (lane == 0) publish_inclusive(me, tb);
+        return identity_b(tb);
+    }
+    AT acc_a = identity_a(ta);
+    BT acc_b = identity_b(tb);
+    BT carry = identity_b(tb);
+    for (long long base = j - 1;; base -= 32) {
+        const long long k = base - lane;
+        AT la = ta;
+        BT lb_ = tb;
+        if (k < k_min) { // nothing flows in from before the row / array
+            la = cut_a(ta);
+            lb_ = identity_b(tb);
+        } else {
+            read_slot(lb.slots + k, la, lb_);
+        }
+        const bool stop = is_cut(la);
+        const unsigned stops = __ballot_sync(kFullMask, stop);
+        const int last = stops ? __ffs(stops) - 1 : 31;
+        if (lane > last) { // farther than the nearest stop: contributes nothing
+            la = identity_a(ta);
+            lb_ = identity_b(tb);
+        }
+        // ordered composition over lanes 0..last: lane 0 (nearest) applied last
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const AT oa = shfl_down(la, d);
+            const BT ob = shfl_down(lb_, d);
+            if (lane + d < 32) combine(la, lb_, oa, ob);
+        }
+        la = shfl_idx(la, 0);
+        lb_ = shfl_idx(lb_, 0);
+        combine(acc_a, acc_b, la, lb_);
+        if (stops) {
+            carry = acc_b;
+            break;
+        }
+    }
+    if (lane == 0) publish_inclusive(me, apply_pair(ta, tb, carry));
     return carry;
 }
 
@@ -684,7 +833,7 @@ struct RowMajorPos {
         return lane == 31 ? load_one_widen(p, i0 + V, n) : 0.0f;
     }
     __device__ __forceinline__ float next(const float (&own)[V], float fetched) const {
-        const float h = __shfl_down_sync(kFullMask, own[0], 1);
+        const float h = shfl_down(own[0], 1);
         return lane == 31 ? fetched : h;
     }
     template <class T>
@@ -692,7 +841,7 @@ struct RowMajorPos {
         return lane == 0 ? load_one_widen(p, i0 - 1, n) : 0.0f;
     }
     __device__ __forceinline__ float prev(const float (&own)[V], float fetched) const {
-        const float h = __shfl_up_sync(kFullMask, own[V - 1], 1);
+        const float h = shfl_up(own[V - 1], 1);
         return lane == 0 ? fetched : h;
     }
     template <class T>
@@ -807,10 +956,16 @@ __device__ __forceinline__ RowMasks time_major_masks(const TimeMajorPos<V> &pos)
 // Scan modes of one launch:
 //   kModeBlock     tiles hold whole rows; warps exchange carries in shared memory
 //   kModeLookback  rows span tiles; tiles exchange carries through the workspace
+//                  in one pass (decoupled look-back with bounded waits)
 //   kModeWarp      every warp's 32*V elements hold whole rows: no block scan at all
+//   kModeReduce    rows span tiles, pass one of two: write each tile's aggregate
+//   kModeCarry     rows span tiles, pass two: scan each tile with the carry
+//                  composed from the complete aggregates (no waiting)
 constexpr int kModeBlock = 0;
 constexpr int kModeLookback = 1;
 constexpr int kModeWarp = 2;
+constexpr int kModeReduce = 3;
+constexpr int kModeCarry = 4;
 
 // The body of one tile, for a launch whose block `block` owns that tile
 // (the tile kernel below, or one part of a fused launch).
@@ -822,6 +977,9 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     constexpr bool kBwd = Est::kBackward;
     constexpr bool kLookback = kMode == kModeLookback;
     constexpr bool kWarpLocal = kMode == kModeWarp;
+    constexpr bool kReduce = kMode == kModeReduce;
+    constexpr bool kCarry = kMode == kModeCarry;
+    constexpr bool kTwoPass = kReduce || kCarry;
     constexpr int NW = NT / 32;
     static_assert(NT % 32 == 0 && NW <= 32, "block must be whole warps, at most 32");
 
@@ -841,7 +999,7 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     // Once the wait returns, let the next grid launch (it waits for this one
     // to complete before touching memory).
     {
-        const long long jg = kLookback ? lookback_tile(lb, g, block) : block;
+        const long long jg = kLookback ? lookback_tile(lb, g, block) : (kTwoPass ? lb.tile_base + block : block);
         const long long mg = kBwd ? (g.ntiles - 1 - jg) : jg;
         Est::prefetch(P, g, mg * (long long)(NT * V), NT * V);
     }
@@ -857,6 +1015,8 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
             return;
         }
         j = lookback_tile(lb, g, s_tile);
+    } else if constexpr (kTwoPass) {
+        j = lb.tile_base + block;
     } else {
         j = block;
     }
@@ -926,9 +1086,9 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
             BT web;
             warp_exclusive_from_inclusive<kBwd>(wa, wb, lane, wea, web);
             BT carry = identity_b(tb);
-            if constexpr (kLookback) {
-                const AT tile_a = __shfl_sync(kFullMask, wa, kBwd ? 0 : NW - 1);
-                const BT tile_b = __shfl_sync(kFullMask, wb, kBwd ? 0 : NW - 1);
+            if constexpr (kLookback || kTwoPass) {
+                const AT tile_a = shfl_idx(wa, kBwd ? 0 : NW - 1);
+                const BT tile_b = shfl_idx(wb, kBwd ? 0 : NW - 1);
                 bool needs_carry;
                 if (kBwd) {
                     const long long end = tile0 + (long long)(NT * V);
@@ -937,10 +1097,17 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
                     needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
                 }
                 const long long k_min = lb.row_tiles > 0 ? (j / lb.row_tiles) * lb.row_tiles : 0;
-                carry = lookback_carry<AT, BT>(lb, j, k_min, needs_carry, tile_a, tile_b, lane);
+                if constexpr (kLookback) {
+                    carry = lookback_carry<AT, BT>(lb, j, k_min, needs_carry, tile_a, tile_b, lane);
+                } else if constexpr (kCarry) {
+                    carry = carry_from_aggregates<AT, BT>(lb, j, k_min, needs_carry, tile_a, tile_b, lane);
+                } else if (lane == 0) {
+                    publish_aggregate(lb.slots + j, tile_a, tile_b);
+                }
             }
             if (lane < NW) s_wx[lane] = apply_pair(wea, web, carry);
         }
+        if constexpr (kReduce) return; // pass one: the aggregate is all it writes
         __syncthreads();
         x = apply_pair(ea, eb, s_wx[warp]);
     }
@@ -1087,20 +1254,20 @@ __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const
 #pragma unroll
         for (int d = 1; d < CPW; d <<= 1) {
             if (kBwd) {
-                const AT oa = __shfl_down_sync(kFullMask, ia, d * G);
-                const BT ob = __shfl_down_sync(kFullMask, ib, d * G);
+                const AT oa = shfl_down(ia, d * G);
+                const BT ob = shfl_down(ib, d * G);
                 if (cs + d < CPW) combine(ia, ib, oa, ob);
             } else {
-                const AT oa = __shfl_up_sync(kFullMask, ia, d * G);
-                const BT ob = __shfl_up_sync(kFullMask, ib, d * G);
+                const AT oa = shfl_up(ia, d * G);
+                const BT ob = shfl_up(ib, d * G);
                 if (cs >= d) combine(ia, ib, oa, ob);
             }
         }
         AT ea = identity_a(own_a);
         BT eb = identity_b(ib);
         if constexpr (CPW > 1) {
-            const AT xa = kBwd ? __shfl_down_sync(kFullMask, ia, G) : __shfl_up_sync(kFullMask, ia, G);
-            const BT xb = kBwd ? __shfl_down_sync(kFullMask, ib, G) : __shfl_up_sync(kFullMask, ib, G);
+            const AT xa = kBwd ? shfl_down(ia, G) : shfl_up(ia, G);
+            const BT xb = kBwd ? shfl_down(ib, G) : shfl_up(ib, G);
             if (kBwd ? (cs + 1 < CPW) : (cs > 0)) {
                 ea = xa;
                 eb = xb;

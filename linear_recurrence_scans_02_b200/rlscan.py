@@ -36,10 +36,10 @@ from . import _build
 
 __all__ = [
     "RlscanError", "library_path",
-    "rlscan_gae", "rlscan_gae_with_returns", "rlscan_gae_typed", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
+    "rlscan_gae", "rlscan_gae_with_returns", "rlscan_gae_typed", "rlscan_gae_vtrace", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
     "rlscan_discounted_returns", "rlscan_eligibility_traces", "rlscan_episodic_prefix_sum",
     "rlscan_batch", "rlscan_workspace_bytes", "rlscan_check", "rlscan_plan", "rlscan_debug_set_lookback",
-    "compute_gae", "compute_gae_with_returns", "compute_vtrace", "compute_retrace", "compute_lambda_returns",
+    "compute_gae", "compute_gae_with_returns", "compute_gae_vtrace", "compute_vtrace", "compute_retrace", "compute_lambda_returns",
     "compute_discounted_returns", "compute_eligibility_traces", "compute_episodic_prefix_sum",
 ]
 
@@ -74,7 +74,8 @@ class _Call(ctypes.Structure):
                 ("options", ctypes.c_uint),
                 ("E", ctypes.c_int64), ("T", ctypes.c_int64), ("A", ctypes.c_int64),
                 ("gamma", ctypes.c_float), ("lambda_", ctypes.c_float), ("rho_bar", ctypes.c_float),
-                ("c_bar", ctypes.c_float), ("inp", ctypes.c_void_p * 8), ("out", ctypes.c_void_p * 2)]
+                ("c_bar", ctypes.c_float), ("inp", ctypes.c_void_p * 8), ("out", ctypes.c_void_p * 4),
+                ("vtrace_lambda", ctypes.c_float)]
 
 
 def library_path() -> str:
@@ -96,6 +97,7 @@ def _load_library():
         "rlscan_gae_with_returns": [P] * 8 + [I64, I64, F, F, P, SZ, S],
         "rlscan_gae_typed": [P] * 8 + [I64, I64, F, F, INT, INT, P, SZ, S],
         "rlscan_vtrace": [P] * 9 + [I64, I64, F, F, F, F, P, SZ, S],
+        "rlscan_gae_vtrace": [P] * 11 + [I64, I64, F, F, F, F, F, P, SZ, S],
         "rlscan_retrace": [P] * 8 + [I64, I64, I64, F, F, F, P, SZ, S],
         "rlscan_lambda_returns": [P] * 7 + [I64, I64, F, F, P, SZ, S],
         "rlscan_discounted_returns": [P] * 6 + [I64, I64, F, P, SZ, S],
@@ -105,6 +107,7 @@ def _load_library():
         "rlscan_gae_typed_ex": [P] * 8 + [I64, I64, F, F, INT, INT, U, P, SZ, S],
         "rlscan_gae_with_returns_ex": [P] * 8 + [I64, I64, F, F, U, P, SZ, S],
         "rlscan_vtrace_ex": [P] * 9 + [I64, I64, F, F, F, F, U, P, SZ, S],
+        "rlscan_gae_vtrace_ex": [P] * 11 + [I64, I64, F, F, F, F, F, U, P, SZ, S],
         "rlscan_retrace_ex": [P] * 8 + [I64, I64, I64, F, F, F, U, P, SZ, S],
         "rlscan_lambda_returns_ex": [P] * 7 + [I64, I64, F, F, U, P, SZ, S],
         "rlscan_discounted_returns_ex": [P] * 6 + [I64, I64, F, U, P, SZ, S],
@@ -164,9 +167,10 @@ def _stream_handle(device):
 
 
 class _WorkspaceCache:
-    """One zero-filled workspace per (device, stream), grown on demand.
+    """One workspace per (device, stream), grown on demand.
 
-    The library leaves a workspace zero-filled after every call, so a cached
+    The library needs no particular workspace content (a call writes every
+    workspace word it reads, or clears what it needs first), so a cached
     buffer is reused as is by later calls on the same stream (which the
     stream orders)."""
 
@@ -312,6 +316,25 @@ def rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_
         E, T, float(gamma), float(lambda_), float(rho_bar), float(c_bar), opts, wp, wn, s))
 
 
+def rlscan_gae_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values,
+                      advantages, returns, vs, pg_advantages, gamma, lambda_, vtrace_lambda=1.0, rho_bar=1.0,
+                      c_bar=1.0, ws=None, *, time_major=False):
+    """GAE advantages (and TD(lambda) returns when `returns` is given) and
+    V-Trace vs / pg_advantages from one pass over the common inputs."""
+    E, T, sh, opts = _layout(rewards, "rewards", time_major)
+    dev = rewards.device
+    wp, wn, s = _ws_for(dev, E, T, ws, opts)
+    _raise_on(_lib.rlscan_gae_vtrace_ex(
+        _ptr(log_rhos, "log_rhos", sh, device=dev), _ptr(rewards, "rewards", sh, device=dev),
+        _ptr(values, "values", sh, device=dev), _ptr(terminateds, "terminateds", sh, device=dev),
+        _ptr(truncateds, "truncateds", sh, device=dev),
+        _ptr(bootstrap_values, "bootstrap_values", sh, device=dev),
+        _ptr(last_values, "last_values", (E,), device=dev), _ptr(advantages, "advantages", sh, device=dev),
+        _ptr(returns, "returns", sh, device=dev), _ptr(vs, "vs", sh, device=dev),
+        _ptr(pg_advantages, "pg_advantages", sh, device=dev),
+        E, T, float(gamma), float(lambda_), float(vtrace_lambda), float(rho_bar), float(c_bar), opts, wp, wn, s))
+
+
 def rlscan_retrace(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds,
                    truncateds, q_ret, gamma, lambda_, c_bar=1.0, ws=None, *, time_major=False):
     E, T, sh, opts = _layout(rewards, "rewards", time_major)
@@ -403,19 +426,20 @@ _BATCH_KINDS = {
     "eligibility_traces": (7, ("x", "dones"), ("traces",)),
     "episodic_prefix_sum": (8, ("x", "dones"), ("out",)),
     "gae_typed": (9, _BACKWARD_IN, ("advantages", "returns")),
+    "gae_vtrace": (10, ("log_rhos",) + _BACKWARD_IN, ("advantages", "returns", "vs", "pg_advantages")),
 }
-_BATCH_SCALARS = {"gamma": 0.99, "lambda_": 0.95, "rho_bar": 1.0, "c_bar": 1.0}
+_BATCH_SCALARS = {"gamma": 0.99, "lambda_": 0.95, "rho_bar": 1.0, "c_bar": 1.0, "vtrace_lambda": 1.0}
 
 
 def rlscan_batch(calls, ws=None):
     """Several independent estimator calls in one request (C: rlscan_batch).
 
     `calls` is a list of dicts, each with "kind" (a key of the rlscan_*
-    functions: "gae", "gae_with_returns", "gae_typed", "vtrace", "retrace",
-    "lambda_returns", "discounted_returns", "eligibility_traces",
+    functions: "gae", "gae_with_returns", "gae_typed", "gae_vtrace", "vtrace",
+    "retrace", "lambda_returns", "discounted_returns", "eligibility_traces",
     "episodic_prefix_sum"), its tensors under the argument names of that
     function (outputs preallocated), its scalars (gamma, lambda_, rho_bar,
-    c_bar; V-Trace's lambda_ defaults to 1.0) and optionally time_major /
+    c_bar, vtrace_lambda; V-Trace's lambda_ defaults to 1.0) and optionally time_major /
     done_starts_episode.  Calls whose rows fit 1024-element tiles run as one
     fused launch; the results equal the individual calls bit for bit."""
     if len(calls) > 16:
@@ -507,6 +531,17 @@ def compute_gae_with_returns(rewards, values, terminateds, gamma=0.99, lambda_=0
         rlscan_gae_with_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, adv, ret,
                                 gamma, lambda_, time_major=time_major)
     return adv, ret
+
+
+def compute_gae_vtrace(log_rhos, rewards, values, terminateds, gamma=0.99, lambda_=0.95, vtrace_lambda=1.0,
+                       rho_bar=1.0, c_bar=1.0, *, truncateds=None, bootstrap_values=None, last_values=None,
+                       time_major=False):
+    """(advantages, returns, vs, pg_advantages) from one pass: GAE and its
+    TD(lambda) returns with lambda_, V-Trace with vtrace_lambda."""
+    outs = [torch.empty_like(rewards) for _ in range(4)]
+    rlscan_gae_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values, *outs,
+                      gamma, lambda_, vtrace_lambda, rho_bar, c_bar, time_major=time_major)
+    return tuple(outs)
 
 
 def compute_vtrace(log_rhos, rewards, values, terminateds, gamma=0.99, lambda_=1.0, rho_bar=1.0, c_bar=1.0, *,

@@ -72,7 +72,7 @@ def test_version(lib):
     # the library reports the version its header declares
     text = open(HEADER).read()
     declared = int(re.search(r"#define RLSCAN_VERSION (\d+)", text).group(1))
-    assert lib.rlscan_version() == declared == 110
+    assert lib.rlscan_version() == declared == 120
 
 
 # fake, never-dereferenced device addresses, far apart
@@ -239,7 +239,8 @@ class _Call(ctypes.Structure):
                 ("options", ctypes.c_uint),
                 ("E", ctypes.c_int64), ("T", ctypes.c_int64), ("A", ctypes.c_int64),
                 ("gamma", ctypes.c_float), ("lambda_", ctypes.c_float), ("rho_bar", ctypes.c_float),
-                ("c_bar", ctypes.c_float), ("inp", ctypes.c_void_p * 8), ("out", ctypes.c_void_p * 2)]
+                ("c_bar", ctypes.c_float), ("inp", ctypes.c_void_p * 8), ("out", ctypes.c_void_p * 4),
+                ("vtrace_lambda", ctypes.c_float)]
 
 
 def _gae_call(r, v, d, out):
@@ -280,9 +281,10 @@ def test_batch_call_layout_matches_the_header(tmp_path):
     import sys
     src = tmp_path / "lay.c"
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "rlscan.h"\n'
-                   'int main(void) { printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(rlscan_call), '
+                   'int main(void) { printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(rlscan_call), '
                    'offsetof(rlscan_call, E), offsetof(rlscan_call, gamma), offsetof(rlscan_call, c_bar), '
-                   'offsetof(rlscan_call, in), offsetof(rlscan_call, out)); return 0; }\n')
+                   'offsetof(rlscan_call, in), offsetof(rlscan_call, out), offsetof(rlscan_call, vtrace_lambda)); '
+                   'return 0; }\n')
     exe = tmp_path / "lay"
     cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, "-o", str(exe), str(src)],
@@ -291,7 +293,7 @@ def test_batch_call_layout_matches_the_header(tmp_path):
     sys.path.insert(0, ROOT)
     from linear_recurrence_scans_02_b200.rlscan import _Call as Mirror
     want = [ctypes.sizeof(Mirror), Mirror.E.offset, Mirror.gamma.offset, Mirror.c_bar.offset, Mirror.inp.offset,
-            Mirror.out.offset]
+            Mirror.out.offset, Mirror.vtrace_lambda.offset]
     assert got == want
     assert [ctypes.sizeof(_Call), _Call.inp.offset] == [want[0], want[4]]
 

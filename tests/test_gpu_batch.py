@@ -28,19 +28,20 @@ def _nan(shape, dtype=torch.float32):
     return torch.full(shape, float("nan") if dtype == torch.float32 else -123456, dtype=dtype, device="cuda")
 
 
-def _calls_for(E, T, seed, trunc=False, time_major=False):
+def _calls_for(E, T, seed, trunc=False, time_major=False, offset=0):
     """One call of every fusable kind on seeded [E, T] inputs; returns the
-    calls (outputs NaN-filled) and the oracle's outputs for each."""
+    calls (outputs NaN-filled) and the oracle's outputs for each.  offset > 0
+    places every input that many elements past a 16-byte boundary."""
     tmx = (lambda a: np.ascontiguousarray(a.T)) if time_major else (lambda a: a)
     sh = (T, E) if time_major else (E, T)
     b = W.vtrace_inputs(E, T, seed, p_term=0.01, p_trunc=0.01 if trunc else 0.0, last_values=True)
     r = W.retrace_inputs(E, T, seed + 1, p_term=0.01, p_trunc=0.01)
     f = W.trace_inputs(E, T, seed + 2, p_done=0.02)
     fi = W.prefix_inputs_i32(E, T, seed + 3, p_done=0.02)
-    t = {k: dev(tmx(v) if v.ndim == 2 else v) for k, v in b.items()}
-    tr = {k: dev(tmx(v)) for k, v in r.items()}
-    tf = {k: dev(tmx(v)) for k, v in f.items()}
-    tfi = {k: dev(tmx(v)) for k, v in fi.items()}
+    t = {k: dev(tmx(v) if v.ndim == 2 else v, offset) for k, v in b.items()}
+    tr = {k: dev(tmx(v), offset) for k, v in r.items()}
+    tf = {k: dev(tmx(v), offset) for k, v in f.items()}
+    tfi = {k: dev(tmx(v), offset) for k, v in fi.items()}
     back = {k: t.get(k) for k in ("rewards", "values", "terminateds", "truncateds", "bootstrap_values",
                                   "last_values")}
     extra = {"time_major": time_major}
@@ -151,8 +152,11 @@ def _check_batch(calls, refs, time_major=False):
 
 
 # shapes whose plan is the fused 1024-element tile: warp mode (T <= 256) and
-# block mode (T = 512, 1024), ragged E
-@pytest.mark.parametrize("E,T", [(4096, 128), (1, 1), (37, 32), (300, 256), (129, 512), (64, 1024)], ids=str)
+# block mode (T = 512, 1024), ragged E; requests of every kind mix more than
+# three estimators, so rows of 4 to 512 steps run on the shared fp32 body
+# (T = 4: one row per thread), T = 1 and 1024 on each estimator's own body
+@pytest.mark.parametrize("E,T", [(4096, 128), (1, 1), (1000, 4), (513, 8), (77, 16), (37, 32), (3, 64),
+                                 (300, 256), (129, 512), (64, 1024)], ids=str)
 @pytest.mark.parametrize("trunc", [False, True], ids=["term", "trunc"])
 def test_batch_of_every_kind_matches_single_calls_and_oracle(E, T, trunc):
     calls, refs = _calls_for(E, T, seed=E + T, trunc=trunc)
@@ -190,7 +194,7 @@ def test_batch_mixes_fused_and_separate_launches():
                 assert_equal_int(g, ref[k], f"call {n}:{k}")
             else:
                 tol = 1e-4 if ref[k].shape[-1] <= 8192 else 1e-3
-                assert_close(g, ref[k], tol, f"call {n}:{k}", row_scale=True)
+                assert_close(g, ref[k], tol, f"call {n}:{k}")
     assert_close(multi["q_ret"], mref, 1e-4, "multi-action retrace")
 
 
@@ -206,6 +210,40 @@ def test_batch_done_starts_episode_option():
     assert_close(calls[0]["traces"], oracle.eligibility_traces(f["x"], f["dones"], np.float32(G), np.float32(L),
                                                                True), 1e-4, "traces")
     assert_close(calls[1]["out"], oracle.episodic_prefix_sum(f["x"], f["dones"], True), 1e-4, "prefix")
+
+
+@pytest.mark.parametrize("offset", [1, 2, 3])
+def test_batch_of_every_kind_unaligned_inputs(offset):
+    # inputs off a 16-byte boundary take the scalar loads of the fused bodies
+    calls, refs = _calls_for(300, 64, seed=60 + offset, trunc=True, offset=offset)
+    _check_batch(calls, refs)
+
+
+def test_batch_mixed_kinds_done_starts_episode():
+    # the forward estimators' other done convention inside a request that
+    # mixes estimators (the shared body's mirrored forward path)
+    E, T = 700, 128
+    f = W.trace_inputs(E, T, seed=70, p_done=0.05)
+    fi = W.prefix_inputs_i32(E, T, seed=71, p_done=0.05)
+    b = W.gae_inputs(E, T, seed=72, p_term=0.02)
+    x, d, xi, di = dev(f["x"]), dev(f["dones"]), dev(fi["x"]), dev(fi["dones"])
+    calls = [dict(kind="gae", rewards=dev(b["rewards"]), values=dev(b["values"]),
+                  terminateds=dev(b["terminateds"]), advantages=_nan((E, T)), gamma=G, lambda_=L),
+             dict(kind="eligibility_traces", x=x, dones=d, traces=_nan((E, T)), gamma=G, lambda_=L,
+                  done_starts_episode=True),
+             dict(kind="episodic_prefix_sum", x=x, dones=d, out=_nan((E, T)), done_starts_episode=True),
+             dict(kind="episodic_prefix_sum", x=xi, dones=di, out=_nan((E, T), torch.int32),
+                  done_starts_episode=True)]
+    R.rlscan_batch(calls)
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    g32, l32 = np.float32(G), np.float32(L)
+    assert_close(calls[0]["advantages"], oracle.gae(b["rewards"], b["values"], b["terminateds"], g32, l32),
+                 1e-4, "gae")
+    assert_close(calls[1]["traces"], oracle.eligibility_traces(f["x"], f["dones"], g32, l32, True), 1e-4,
+                 "traces")
+    assert_close(calls[2]["out"], oracle.episodic_prefix_sum(f["x"], f["dones"], True), 1e-4, "prefix f32")
+    assert_equal_int(calls[3]["out"], oracle.episodic_prefix_sum(fi["x"], fi["dones"], True), "prefix i32")
 
 
 def test_batch_rejects_overlap_across_calls_and_enqueues_nothing():

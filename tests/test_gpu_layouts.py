@@ -154,8 +154,7 @@ def test_done_starts_episode_row_major(E, T):
     torch.cuda.synchronize()
     assert_close(tr, oracle.eligibility_traces(d["x"], d["dones"], np.float32(g), np.float32(lam), True),
                  tol_for(T), "traces")
-    assert_close(ps, oracle.episodic_prefix_sum(d["x"], d["dones"], True), tol_for(T), "prefix_f32",
-                 row_scale=True)
+    assert_close(ps, oracle.episodic_prefix_sum(d["x"], d["dones"], True), tol_for(T), "prefix_f32")
     assert_equal_int(pi, oracle.episodic_prefix_sum(di["x"], di["dones"], True), "prefix_i32")
 
 

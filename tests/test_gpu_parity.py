@@ -10,6 +10,8 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
+
 from gpu_common import (BACKWARD_KEYS, BACKWARD_RUN, check, dev, inputs_backward, run_gae, run_gae_with_returns,
                         run_prefix, run_retrace, run_traces, run_vtrace, strip)
 from linear_recurrence_scans_02_b200 import rlscan as R
@@ -141,21 +143,34 @@ def test_nonfinite_input_stays_in_its_episode():
     np.testing.assert_allclose(g[:, :100], ref["advantages"][:, :100], rtol=1e-4, atol=1e-4)
 
 
-def test_workspace_left_zero_and_reused():
+def test_workspace_needs_no_initial_content_and_is_reused():
+    """Split-row calls write every workspace slot they read: a workspace of
+    arbitrary bytes works, and one workspace serves a sequence of calls,
+    including a multi-action Retrace call (the one-pass look-back, which
+    clears the flags it needs) between two-pass calls."""
     E, T = 3, 70000  # rows split over tiles
     plan = R.rlscan_plan(E, T)
     assert plan["lookback"]
-    need = R.rlscan_workspace_bytes(E, T)
-    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    need = max(R.rlscan_workspace_bytes(E, T), R.rlscan_workspace_bytes(2, 2048))
+    ws = torch.full((need,), 0xA5, dtype=torch.uint8, device="cuda")
     d = strip(inputs_backward(E, T, seed=1, p_term=0.0005), BACKWARD_KEYS["gae"])
     t = {k: dev(v) for k, v in d.items()}
+    m = W.off_policy_inputs(2, 2048, A=18, seed=3)
+    tm = {k: dev(v) for k, v in m.items()}
+    assert R.rlscan_plan(2, 2048, 18)["lookback"]
     outs = []
     for _ in range(3):
         out = torch.empty(E, T, device="cuda")
         R.rlscan_gae(t["rewards"], t["values"], t["terminateds"], None, None, None, out, 0.99, 0.95, ws=ws)
-        torch.cuda.synchronize()
-        assert int(ws.count_nonzero()) == 0, "workspace not left zero-filled"
         outs.append(out)
+        q_ret = torch.full((2, 2048), float("nan"), device="cuda")
+        R.rlscan_retrace(tm["rewards"], tm["q_values"], tm["next_q_values_all"], tm["next_target_probs"],
+                         tm["log_rhos"], tm["terminateds"], tm["truncateds"], q_ret, W.GAMMA, W.LAMBDA, 1.0, ws=ws)
+        torch.cuda.synchronize()
+        ref_q = oracle.retrace(m["rewards"], m["q_values"], m["next_q_values_all"], m["log_rhos"],
+                               m["terminateds"], m["truncateds"], np.float32(W.GAMMA), np.float32(W.LAMBDA),
+                               np.float32(1.0), m["next_target_probs"])
+        check(({"q_ret": q_ret}, {"q_ret": ref_q}), 2048, "multi-action retrace sharing the workspace")
     R.rlscan_check()
     _, ref = run_gae(d)
     for out in outs:
@@ -173,25 +188,28 @@ def test_non_default_stream():
 
 
 def test_lookback_wait_times_out_cleanly():
-    """A tile that never publishes makes its successors' bounded waits run
-    out: the call must finish, report RLSCAN_ERR_TIMEOUT, leave the workspace
-    zero-filled, and the next normal call must be correct."""
-    E, T = 2, 4096 * 4
-    assert R.rlscan_plan(E, T)["lookback"]
-    d = strip(inputs_backward(E, T, seed=9, p_term=0.0), BACKWARD_KEYS["discounted_returns"])
+    """The one-pass look-back (multi-action Retrace with rows split over
+    tiles): a tile that never publishes makes its successors' bounded waits
+    run out.  The call must finish, report RLSCAN_ERR_TIMEOUT, and the next
+    normal calls must be correct."""
+    E, T, A = 2, 2048, 18
+    assert R.rlscan_plan(E, T, A)["lookback"]
+    d = W.off_policy_inputs(E, T, A=A, seed=9)
     t = {k: dev(v) for k, v in d.items()}
     out = torch.empty(E, T, device="cuda")
     try:
         R.rlscan_debug_set_lookback(spin_limit=2000, withhold_tile=0)
-        # tile 0 in scan order never publishes; rows split over tiles wait on it
-        R.rlscan_discounted_returns(t["rewards"], t["terminateds"], None, None, None, out, 0.99)
+        # tile 0 in scan order never publishes; the row's later tiles wait on it
+        R.rlscan_retrace(t["rewards"], t["q_values"], t["next_q_values_all"], t["next_target_probs"],
+                         t["log_rhos"], t["terminateds"], t["truncateds"], out, W.GAMMA, W.LAMBDA, 1.0)
         with pytest.raises(R.RlscanError) as ei:
             R.rlscan_check()
         assert ei.value.status == R.RLSCAN_ERR_TIMEOUT
     finally:
         R.rlscan_debug_set_lookback(0, -1)
     R.rlscan_check()  # error word was cleared
-    check(run_gae(strip(inputs_backward(E, T, seed=10), BACKWARD_KEYS["gae"])), T, "gae after a timeout")
+    check(run_retrace(d), T, "retrace after a timeout")
+    check(run_gae(strip(inputs_backward(E, 4096 * 4, seed=10), BACKWARD_KEYS["gae"])), 4096 * 4, "gae after a timeout")
     R.rlscan_check()
 
 

@@ -6,8 +6,9 @@ call cudaMalloc because it synchronises the device.  For them the library
 keeps a fixed scratch array on each device and rlscan_gae_noalloc uses it in
 place of the caller's workspace.  This test calls it through the C ABI twice
 in a row (the array keeps the previous call's contents, which each call must
-clear) and checks both outputs against rlscan_gae run with its own workspace,
-within the parity tolerance of the other GPU tests.  It imports nothing from
+clear) and checks both outputs against rlscan_gae run with its own workspace
+and against the CPU oracle's GAE, element by element, within the parity
+tolerance of the other GPU tests.  It imports nothing from
 the other test modules, so it passes alone in a fresh process as well as
 after the whole suite; its file name makes pytest collect it last.
 """
@@ -17,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from linear_recurrence_scans_02_b200 import rlscan as R
 from linear_recurrence_scans_02_b200 import workloads as W
 
@@ -61,8 +63,11 @@ def test_noalloc_matches_workspace_entry_point(E, T):
     torch.cuda.synchronize()
     R.rlscan_check()
     r = ref.double().cpu().numpy()
+    want = oracle.gae(d["rewards"], d["values"], d["terminateds"], np.float32(0.99), np.float32(0.95),
+                      d["truncateds"], d["bootstrap_values"], d["last_values"])
     for k, out in enumerate(outs):
         g = out.double().cpu().numpy()
-        bound = _tol(T) * (1.0 + np.abs(r))
-        bad = ~(np.abs(g - r) <= bound)
-        assert not bad.any(), f"call {k}: {int(bad.sum())} elements differ from rlscan_gae"
+        for name, other in (("rlscan_gae", r), ("the oracle", want)):
+            bound = _tol(T) * (1.0 + np.abs(other))
+            bad = ~(np.abs(g - other) <= bound)
+            assert not bad.any(), f"call {k}: {int(bad.sum())} elements differ from {name}"
