@@ -26,8 +26,9 @@
  *     is nonzero.  terminated at t: the episode ends at t, nothing is
  *     bootstrapped and the trace is cut.  truncated at t: the episode ends at
  *     t, its value is bootstrapped from bootstrap_values[e, t] and the trace is
- *     cut.  If both are set, terminated wins.  bootstrap_values is read only
- *     where a step is truncated.
+ *     cut.  If both are set, terminated wins.  bootstrap_values is read in
+ *     full whenever truncateds is given (one streamed plane, no dependent
+ *     loads); only its values at truncated steps matter.
  *   - last_values (nullable, [E]): the value after the last step of each row
  *     when that step carries no flag; NULL means 0.
  *   - Forward estimators (eligibility traces, prefix sum) reset after a done:
@@ -40,11 +41,13 @@
  *     returning RLSCAN_OK.  Calls are thread-safe.
  *   - Workspace: long rows (a row that spans several tiles) and rows that do
  *     not align with tiles need a device workspace of
- *     rlscan_workspace_bytes(E, T) bytes, 16-byte aligned, zero-filled before
- *     its first use (rlscan_workspace_init or cudaMemset) and left zero-filled
- *     by every call.  Shapes that need none accept ws = NULL.  A workspace
- *     holds one call's progress flags: calls that share one must be ordered
- *     on one stream (or otherwise serialised).
+ *     rlscan_workspace_bytes(E, T) bytes, 16-byte aligned, of any content
+ *     (such a call runs two launches: the first writes one 16-byte aggregate
+ *     per tile, the second scans each tile with the carry it composes from
+ *     them; no kernel ever waits for another block).  Shapes that need none
+ *     accept ws = NULL.  A workspace holds one call's aggregates between its
+ *     two launches: calls that share one must be ordered on one stream (or
+ *     otherwise serialised).
  *   - Errors: a nonzero return is an rlscan_status; nothing was enqueued
  *     unless it is RLSCAN_ERR_CUDA from the launch itself.
  *     rlscan_last_error() gives a message for the calling thread.
@@ -87,10 +90,8 @@ typedef enum rlscan_status {
     RLSCAN_ERR_WORKSPACE = 3,   /* the shape needs a workspace and ws is NULL, too small or
                                    not 16-byte aligned */
     RLSCAN_ERR_CUDA = 4,        /* a CUDA runtime call failed (message in rlscan_last_error) */
-    RLSCAN_ERR_TIMEOUT = 5      /* reported by rlscan_check: a kernel gave up a bounded wait
-                                   for a neighbouring tile, or found its workspace not
-                                   zero-filled; that call's output is invalid and the
-                                   workspace should be re-initialised */
+    RLSCAN_ERR_TIMEOUT = 5      /* reserved: returned by no call since 1.2.0, whose kernels
+                                   never wait on one another */
 } rlscan_status;
 
 typedef enum rlscan_dtype {
@@ -211,7 +212,10 @@ RLSCAN_API int rlscan_gae_vtrace(const float *log_rhos, const float *rewards, co
  * next_q_values_all[e,t,:] = Q(x_{t+1}, .) (the final observation's values at
  * a truncation; ignored at a termination); next_target_probs[e,t,:] =
  * pi(. | x_{t+1}); log_rhos[e,t] = log pi(a_t|x_t) - log mu(a_t|x_t);
- * q_values[e,t] = Q(x_t, a_t).  1 <= A <= RLSCAN_MAX_ACTIONS.
+ * q_values[e,t] = Q(x_t, a_t).  1 <= A <= RLSCAN_MAX_ACTIONS.  With A > 1
+ * the call first writes V' into q_ret (one streaming launch over the
+ * per-action arrays), then runs the recurrence on it as with A == 1,
+ * rewriting q_ret in place.
  */
 RLSCAN_API int rlscan_retrace(const float *rewards, const float *q_values, const float *next_q_values_all,
                    const float *next_target_probs, const float *log_rhos,
@@ -384,13 +388,16 @@ RLSCAN_API int rlscan_episodic_prefix_sum_ex(const void *x, int dtype, const flo
  * Each rlscan_call describes one call of an entry point above; rlscan_batch
  * validates every call as that entry point would, then launches every call
  * whose rows fit whole in 1024-element tiles (row-major, 1024 a multiple of
- * T, every kind below, A == 1 for Retrace) as ONE fused kernel, each block
- * running one tile of one call, and each remaining call by its own launch.
- * Results are those of the individual calls, bit for bit, except that a
- * request fusing three or more kinds whose rows all fit 512 elements runs
- * 4 elements per thread (smaller code per kind), which re-associates the
- * fp32 scans: those results agree with the individual calls to fp32
- * rounding (int32 stays exact).
+ * T, A == 1 for Retrace; every kind below except GAE_VTRACE and typed GAE
+ * with narrow inputs) as ONE fused kernel, each block running one tile of
+ * one call, and each remaining call by its own launch.  Results are those
+ * of the individual calls, bit for bit, except that a request whose fused
+ * calls span three or more of the families {GAE, GAE + returns, TD(lambda)
+ * returns, discounted returns}, {V-Trace}, {Retrace}, {eligibility traces,
+ * fp32 prefix sum}, {int32 prefix sum}, with rows that all fit 512
+ * elements, runs 4 elements per thread (smaller code per family), which
+ * re-associates the fp32 scans: those results agree with the individual
+ * calls to fp32 rounding (int32 stays exact).
  *
  * kind and argument slots (the pointer arguments of the entry point, in its
  * order; unused slots NULL):
@@ -459,19 +466,20 @@ RLSCAN_API int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size
 
 /*
  * Workspace size in bytes that any entry point above needs for an [E, T]
- * problem (any A); 0 if no call of that shape needs one.  Negative or
- * overflowing shapes return 0 and the compute call then rejects them.
+ * problem (any A): 16 bytes per tile when rows span tiles, 0 when no call of
+ * that shape needs one.  Negative or overflowing shapes return 0 and the
+ * compute call then rejects them.
  */
 RLSCAN_API size_t rlscan_workspace_bytes(int64_t E, int64_t T);
 
-/* Zero-fill a workspace on `stream` (cudaMemsetAsync). */
+/* Zero-fill a workspace on `stream` (cudaMemsetAsync).  Not required: calls
+ * accept a workspace of any content. */
 RLSCAN_API int rlscan_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
- * Synchronise `stream`, then read and clear this device's error word, which
- * kernels set when a bounded wait gave up.  Returns RLSCAN_OK,
- * RLSCAN_ERR_TIMEOUT, or RLSCAN_ERR_CUDA if the stream reports an error.
- * For debugging and tests; compute calls never synchronise.
+ * Synchronise `stream` and report any error of the work on it or of the
+ * last launch: RLSCAN_OK, or RLSCAN_ERR_CUDA with the CUDA message.  For
+ * debugging and tests; compute calls never synchronise.
  */
 RLSCAN_API int rlscan_check(cudaStream_t stream);
 
@@ -482,23 +490,13 @@ RLSCAN_API const char *rlscan_last_error(void);
 RLSCAN_API int rlscan_version(void);
 
 /*
- * Test hook for the bounded waits between tiles.  spin_limit: maximum
- * polls (each with a short sleep) before a tile gives up waiting for its
- * predecessor (0 restores the default, about a second).  withhold_tile: the
- * index, in scan order, of one tile that never publishes its result (-1,
- * the default, for none), so that a test can make the wait run out and
- * check that rlscan_check reports RLSCAN_ERR_TIMEOUT without hanging.  Not
- * for production use; applies to calls made after it on any thread.
- */
-RLSCAN_API int rlscan_debug_set_lookback(uint32_t spin_limit, int64_t withhold_tile);
-
-/*
  * Launch plan that a call of this shape takes (for tests and tools):
  * writes tile size in elements, threads per block, whether tiles exchange
  * carries through the workspace (1) or not (0), and the tile count.
  * actions: 1 for every estimator except rlscan_retrace with A > 1, whose
- * action count it is (that call stages per-action rows in shared memory and
- * uses smaller tiles).
+ * action count it is (1 .. RLSCAN_MAX_ACTIONS); every call scans on the same
+ * plans, multi-action Retrace after a first launch that writes its expected
+ * next-state values.
  */
 RLSCAN_API int rlscan_plan(int64_t E, int64_t T, int64_t actions, int64_t *tile_elems, int *threads,
                 int *lookback, int64_t *num_tiles);

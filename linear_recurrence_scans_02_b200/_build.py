@@ -1,8 +1,9 @@
 """Build ``librlscan.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
 
-The library is compiled from ``csrc/rlscan.cu`` (which includes the kernel
-headers) into ``linear_recurrence_scans_02_b200/librlscan.so``, with the CUDA
-runtime linked statically so the library loads next to any PyTorch build.
+The library is compiled from the translation units ``csrc/*.cu`` (in
+parallel; they include the kernel headers) and linked into
+``linear_recurrence_scans_02_b200/librlscan.so``, with the CUDA runtime linked
+statically so the library loads next to any PyTorch build.
 No GPU is needed to build.  Rebuilds only when a source is newer than the
 library (or when forced).
 """
@@ -39,25 +40,45 @@ def needs_build() -> bool:
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def compile_cmd(out: str, extra=()) -> list:
-    return [nvcc_path(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "--cudart", "static",
-            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared",
-            f"-I{INCLUDE}", "-DRLSCAN_BUILDING_LIBRARY", *extra,
-            "-o", out, os.path.join(CSRC, "rlscan.cu")]
+def units() -> list:
+    """The library's translation units (compiled in parallel)."""
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+
+def compile_cmd(src: str, obj: str, extra=()) -> list:
+    return [nvcc_path(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC",
+            "-Xcompiler", "-fvisibility=hidden", f"-I{INCLUDE}", "-DRLSCAN_BUILDING_LIBRARY", *extra,
+            "-c", "-o", obj, src]
+
+
+def link_cmd(objs: list, out: str) -> list:
+    return [nvcc_path(), *ARCH_FLAGS, "--cudart", "static", "-shared", "-o", out, *objs]
+
+
+def _run(cmd, verbose):
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
+    if verbose and (res.stdout or res.stderr):
+        print(res.stdout + res.stderr)
 
 
 def build_library(force: bool = False, verbose: bool = False, extra=()) -> str:
     if force or needs_build():
-        tmp = LIB + f".tmp{os.getpid()}"
-        cmd = compile_cmd(tmp, extra)
-        if verbose:
-            print(" ".join(cmd), flush=True)
-        res = subprocess.run(cmd, capture_output=True, text=True)
-        if res.returncode != 0:
-            raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
-        if verbose and (res.stdout or res.stderr):
-            print(res.stdout + res.stderr)
-        os.replace(tmp, LIB)
+        from concurrent.futures import ThreadPoolExecutor
+        tag = f".tmp{os.getpid()}"
+        objs = [os.path.join(PKG, os.path.basename(src)[:-3] + tag + ".o") for src in units()]
+        try:
+            with ThreadPoolExecutor(max_workers=max(1, min(len(objs), os.cpu_count() or 1))) as pool:
+                list(pool.map(lambda so: _run(compile_cmd(so[0], so[1], extra), verbose), zip(units(), objs)))
+            _run(link_cmd(objs, LIB + tag), verbose)
+            os.replace(LIB + tag, LIB)
+        finally:
+            for o in objs:
+                if os.path.exists(o):
+                    os.remove(o)
     return LIB
 
 

@@ -10,63 +10,159 @@
 // instruction caches better).
 #pragma once
 
-#include "fused_any.cuh"
+#include "estimators.cuh"
 
 namespace rlscan {
 
-enum FusedKind {
-    kFkGae = 0,
-    kFkGaeReturns,
-    kFkVtrace,
-    kFkRetrace1,
-    kFkLambda,
-    kFkReturns,
-    kFkTraces,
-    kFkPrefixF32,
-    kFkPrefixI32,
-    kNumFusedKinds
+// Tile bodies of a fused launch.  Calls whose estimators are one recurrence
+// with different constants share a body, so that fewer distinct bodies share
+// each SM's instruction caches: GAE, GAE + returns, TD(lambda) returns and
+// discounted returns run the backward family body; eligibility traces and
+// the fp32 prefix sum the forward body (the prefix sum is a trace with decay
+// 1).  Each call's arithmetic in its family body is its own estimator's, in
+// the same order, so results equal its own kernel's bit for bit on the same
+// tiles.
+enum FusedBody {
+    kBodyBackward = 0, // BackwardFamilyEst
+    kBodyVtrace,       // VtraceEst
+    kBodyRetrace1,     // RetraceEst
+    kBodyForward,      // TracesEst (ForwardF32Est)
+    kBodyPrefixI32,    // PrefixI32Est
+    kNumFusedBodies
 };
 
+// GAE (+ returns), TD(lambda) returns and discounted returns as one
+// backward recurrence x_t = a_t x_{t+1} + b_t with
+//   a_t = gamma lambda  while the episode goes on inside the row, else 0
+//   b_t = r_t + gamma boot_t - [V_t]
+//   boot_t = w_nv V_{t+1} inside the episode, the row's last value at a row
+//            end, the bootstrap value at a truncation, 0 at a termination
+// GAE: w_nv = 1, V subtracted (x = A; returns x + V); TD(lambda): w_nv =
+// 1 - lambda, nothing subtracted (x = G); discounted returns: lambda = 1,
+// no values (w_nv = 0), nothing subtracted (x = R).  Used by fused launches.
+struct BackwardFamilyEst {
+    static constexpr bool kBackward = true;
+    using AT = float;
+    using BT = float;
+    struct Params {
+        const float *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        float *out0; // x
+        float *out1; // x + V (the TD(lambda) returns beside GAE), may be null
+        float gamma, lambda_, w_nv;
+        int sub_v;
+    };
+    template <int V>
+    struct State {
+        float r[V], v[V], te[V], tr[V], bv[V], o0[V], o1[V];
+        float v_next;
+    };
+    static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
+        prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values);
+    }
+    static constexpr int kInputPlanes = 5;
+    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+        const float *p[5] = {P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values};
+        return {i < 5 ? p[i] : nullptr, 4};
+    }
+    template <int NT, int V, class Pos>
+    static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
+                                                State<V> &S, unsigned char *) {
+        const float h_v_next = pos.fetch_next(P.values);
+        pos.load(P.rewards, S.r);
+        pos.load(P.values, S.v);
+        pos.load(P.terminateds, S.te);
+        pos.load(P.truncateds, S.tr);
+        pos.load(P.bootstrap_values, S.bv);
+        S.v_next = pos.next(S.v, h_v_next);
+    }
+    template <int V, bool kTrunc, bool kFast, class Pos>
+    static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
+                                                  const RowMasks &rm, State<V> &S,
+                                                  float (&a)[V], float (&b)[V]) {
+        const float gl = P.gamma * P.lambda_;
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            if (elem_valid<kFast, V>(rm, k)) {
+                const StepFlags f = step_flags<kTrunc>(S.te[k], S.tr[k]);
+                const bool rowend = elem_row_end<kFast, V>(rm, k);
+                float boot;
+                if (f.cont) {
+                    boot = rowend ? row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows)
+                                  : P.w_nv * ((k + 1 < V) ? S.v[k + 1] : S.v_next);
+                } else {
+                    boot = f.trn ? S.bv[k] : 0.0f;
+                }
+                a[k] = (f.cont && !rowend) ? gl : 0.0f;
+                float bb = fmaf(P.gamma, boot, S.r[k]);
+                if (P.sub_v) bb = bb - S.v[k];
+                b[k] = bb;
+            } else {
+                a[k] = 1.0f;
+                b[k] = 0.0f;
+            }
+        }
+    }
+    template <int V, class Pos>
+    static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
+                                                  const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
+        if (P.truncateds != nullptr) {
+            if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
+        } else {
+            if (rm.fast) coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+            else coeffs_impl<V, false, false>(P, g, pos, rm, S, a, b);
+        }
+    }
+    template <int V>
+    static __device__ __forceinline__ void out(const Params &, State<V> &S, int k, float x, float, float) {
+        S.o0[k] = x;
+        S.o1[k] = x + S.v[k];
+    }
+    template <int V, class Pos>
+    static __device__ __forceinline__ void store(const Params &P, const Geometry &, const Pos &pos, State<V> &S) {
+        pos.store(P.out0, S.o0);
+        if (P.out1 != nullptr) pos.store(P.out1, S.o1);
+    }
+};
+
+// Body of each fusable estimator and its parameters in that body's form.
 template <class Est>
-struct FusedKindOf {
+struct FusedBodyOf {
     static constexpr int value = -1;
 };
-template <>
-struct FusedKindOf<GaeEst> {
-    static constexpr int value = kFkGae;
-};
-template <>
-struct FusedKindOf<GaeReturnsEst> {
-    static constexpr int value = kFkGaeReturns;
-};
-template <>
-struct FusedKindOf<VtraceEst> {
-    static constexpr int value = kFkVtrace;
-};
-template <>
-struct FusedKindOf<RetraceEst<false>> {
-    static constexpr int value = kFkRetrace1;
-};
-template <>
-struct FusedKindOf<LambdaReturnsEst> {
-    static constexpr int value = kFkLambda;
-};
-template <>
-struct FusedKindOf<ReturnsEst> {
-    static constexpr int value = kFkReturns;
-};
-template <>
-struct FusedKindOf<TracesEst> {
-    static constexpr int value = kFkTraces;
-};
-template <>
-struct FusedKindOf<PrefixF32Est> {
-    static constexpr int value = kFkPrefixF32;
-};
-template <>
-struct FusedKindOf<PrefixI32Est> {
-    static constexpr int value = kFkPrefixI32;
-};
+template <> struct FusedBodyOf<GaeEst> { static constexpr int value = kBodyBackward; };
+template <> struct FusedBodyOf<GaeReturnsEst> { static constexpr int value = kBodyBackward; };
+template <> struct FusedBodyOf<LambdaReturnsEst> { static constexpr int value = kBodyBackward; };
+template <> struct FusedBodyOf<ReturnsEst> { static constexpr int value = kBodyBackward; };
+template <> struct FusedBodyOf<VtraceEst> { static constexpr int value = kBodyVtrace; };
+template <> struct FusedBodyOf<RetraceEst> { static constexpr int value = kBodyRetrace1; };
+template <> struct FusedBodyOf<TracesEst> { static constexpr int value = kBodyForward; };
+template <> struct FusedBodyOf<PrefixF32Est> { static constexpr int value = kBodyForward; };
+template <> struct FusedBodyOf<PrefixI32Est> { static constexpr int value = kBodyPrefixI32; };
+
+inline BackwardFamilyEst::Params family_params(const GaeEst::Params &p) {
+    return {p.rewards, p.values, p.terminateds, p.truncateds, p.bootstrap_values, p.last_values,
+            p.advantages, nullptr, p.gamma, p.lambda_, 1.0f, 1};
+}
+inline BackwardFamilyEst::Params family_params(const GaeReturnsEst::Params &p) {
+    return {p.rewards, p.values, p.terminateds, p.truncateds, p.bootstrap_values, p.last_values,
+            p.advantages, p.returns, p.gamma, p.lambda_, 1.0f, 1};
+}
+inline BackwardFamilyEst::Params family_params(const LambdaReturnsEst::Params &p) {
+    return {p.rewards, p.values, p.terminateds, p.truncateds, p.bootstrap_values, p.last_values,
+            p.returns, nullptr, p.gamma, p.lambda_, 1.0f - p.lambda_, 0};
+}
+inline BackwardFamilyEst::Params family_params(const ReturnsEst::Params &p) {
+    return {p.rewards, nullptr, p.terminateds, p.truncateds, p.bootstrap_values, p.last_values,
+            p.returns, nullptr, p.gamma, 1.0f, 0.0f, 0};
+}
+inline TracesEst::Params family_params(const PrefixF32Est::Params &p) {
+    return {p.x, p.dones, p.out, p.decay, p.reset_on_flag};
+}
+template <class P>
+inline const P &family_params(const P &p) { // estimators that are their own body
+    return p;
+}
 
 constexpr int kFusedNT = 128; // 128 threads x 8 (or 4) elements per tile
 constexpr int kFusedVMax = 8;
@@ -74,10 +170,10 @@ constexpr int kFusedParamBytes = 128;
 constexpr int kFusedMax = 16;
 
 struct FusedItem {
-    alignas(16) unsigned char params[kFusedParamBytes]; // the call's Est::Params
+    alignas(16) unsigned char params[kFusedParamBytes]; // the call's parameters in its body's form
     Geometry g;
     long long tile_begin; // first block of this call in the fused grid
-    int kind;             // FusedKind
+    int kind;             // FusedBody: the tile body that runs the call
     int mode;             // kModeWarp or kModeBlock
 };
 
@@ -89,7 +185,7 @@ struct FusedBatch {
 template <class Est, int V, int kMode>
 __device__ __forceinline__ void fused_tile(const FusedItem &it, long long block, unsigned char *smem) {
     const auto &P = *reinterpret_cast<const typename Est::Params *>(it.params);
-    const Lookback lb{nullptr, nullptr, 0u, -1}; // no look-back in a fused launch
+    const Lookback lb{}; // whole rows per tile: no carries between tiles
     tile_scan_body<Est, kFusedNT, V, kMode>(P, it.g, lb, block, smem);
 }
 
@@ -101,79 +197,6 @@ __device__ __forceinline__ void fused_tile_any_mode(const FusedItem &it, long lo
         fused_tile<Est, V, kModeBlock>(it, block, smem);
 }
 
-// ---------------------------------------------------------------------------
-// The same calls on the shared fp32 body (fused_any.cuh): each fp32 call's
-// parameters in AnyParams form.  Returns false for calls that body does not
-// take (the int32 prefix sum).
-// ---------------------------------------------------------------------------
-inline AnyParams any_base() {
-    AnyParams a{};
-    a.lam = 1.0f;
-    a.rho_bar = 1.0f;
-    a.c_bar = 1.0f;
-    return a;
-}
-inline bool to_any(const GaeEst::Params &p, AnyParams &a) {
-    a = any_base();
-    a.r = p.rewards; a.v = p.values; a.f = p.terminateds; a.tr = p.truncateds;
-    a.bv = p.bootstrap_values; a.lv = p.last_values; a.out0 = p.advantages;
-    a.gamma = p.gamma; a.lam = p.lambda_; a.w_nv = 1.0f; a.halo = kAnyHaloV;
-    a.flags = kAnySubV;
-    return true;
-}
-inline bool to_any(const GaeReturnsEst::Params &p, AnyParams &a) {
-    a = any_base();
-    a.r = p.rewards; a.v = p.values; a.f = p.terminateds; a.tr = p.truncateds;
-    a.bv = p.bootstrap_values; a.lv = p.last_values; a.out0 = p.advantages; a.out1 = p.returns;
-    a.gamma = p.gamma; a.lam = p.lambda_; a.w_nv = 1.0f; a.halo = kAnyHaloV;
-    a.flags = kAnySubV | (p.returns != nullptr ? kAnyOut1PlusV : 0u);
-    return true;
-}
-inline bool to_any(const VtraceEst::Params &p, AnyParams &a) {
-    a = any_base();
-    a.r = p.rewards; a.v = p.values; a.f = p.terminateds; a.tr = p.truncateds; a.lr = p.log_rhos;
-    a.bv = p.bootstrap_values; a.lv = p.last_values; a.out0 = p.vs; a.out1 = p.pg_advantages;
-    a.gamma = p.gamma; a.lam = p.lambda_; a.rho_bar = p.rho_bar; a.c_bar = p.c_bar; a.w_nv = 1.0f;
-    a.halo = kAnyHaloV;
-    a.flags = kAnyRatioOwn | kAnySubV | kAnyOut0PlusV | kAnyOut1Pg;
-    return true;
-}
-inline bool to_any(const RetraceEst<false>::Params &p, AnyParams &a) {
-    a = any_base();
-    a.r = p.rewards; a.v = p.q_values; a.f = p.terminateds; a.tr = p.truncateds; a.lr = p.log_rhos;
-    a.nq = p.next_q_values_all; a.out0 = p.q_ret;
-    a.gamma = p.gamma; a.lam = p.lambda_; a.c_bar = p.c_bar; a.halo = kAnyHaloLogRho;
-    a.flags = kAnyRatioNext | kAnySubV | kAnyRetraceBoot | kAnyOut0PlusV;
-    return true;
-}
-inline bool to_any(const LambdaReturnsEst::Params &p, AnyParams &a) {
-    a = any_base();
-    a.r = p.rewards; a.v = p.values; a.f = p.terminateds; a.tr = p.truncateds;
-    a.bv = p.bootstrap_values; a.lv = p.last_values; a.out0 = p.returns;
-    a.gamma = p.gamma; a.lam = p.lambda_; a.w_nv = 1.0f - p.lambda_; a.halo = kAnyHaloV;
-    a.flags = 0u;
-    return true;
-}
-inline bool to_any(const ReturnsEst::Params &p, AnyParams &a) {
-    a = any_base();
-    a.r = p.rewards; a.f = p.terminateds; a.tr = p.truncateds;
-    a.bv = p.bootstrap_values; a.lv = p.last_values; a.out0 = p.returns;
-    a.gamma = p.gamma; a.w_nv = 0.0f; a.halo = kAnyHaloNone;
-    a.flags = 0u;
-    return true;
-}
-template <int kKind>
-inline bool to_any(const typename ForwardF32Est<kKind>::Params &p, AnyParams &a) {
-    a = any_base();
-    a.r = p.x; a.f = p.dones; a.out0 = p.out;
-    a.gamma = p.decay; a.halo = kAnyHaloDone;
-    a.flags = kAnyFwd | (p.reset_on_flag ? kAnyResetOnFlag : 0u);
-    return true;
-}
-inline bool to_any(const TracesEst::Params &p, AnyParams &a) { return to_any<0>(p, a); }
-inline bool to_any(const PrefixF32Est::Params &p, AnyParams &a) { return to_any<1>(p, a); }
-inline bool to_any(const PrefixI32Est::Params &, AnyParams &) { return false; }
-
 template <int V>
 __global__ void __launch_bounds__(kFusedNT) fused_tile_kernel(const __grid_constant__ FusedBatch b) {
     extern __shared__ __align__(128) unsigned char dyn_smem[];
@@ -183,33 +206,13 @@ __global__ void __launch_bounds__(kFusedNT) fused_tile_kernel(const __grid_const
     const FusedItem &it = b.item[idx];
     const long long block = (long long)blockIdx.x - it.tile_begin;
     switch (it.kind) {
-    case kFkGae: fused_tile_any_mode<GaeEst, V>(it, block, dyn_smem); break;
-    case kFkGaeReturns: fused_tile_any_mode<GaeReturnsEst, V>(it, block, dyn_smem); break;
-    case kFkVtrace: fused_tile_any_mode<VtraceEst, V>(it, block, dyn_smem); break;
-    case kFkRetrace1: fused_tile_any_mode<RetraceEst<false>, V>(it, block, dyn_smem); break;
-    case kFkLambda: fused_tile_any_mode<LambdaReturnsEst, V>(it, block, dyn_smem); break;
-    case kFkReturns: fused_tile_any_mode<ReturnsEst, V>(it, block, dyn_smem); break;
-    case kFkTraces: fused_tile_any_mode<TracesEst, V>(it, block, dyn_smem); break;
-    case kFkPrefixF32: fused_tile_any_mode<PrefixF32Est, V>(it, block, dyn_smem); break;
-    case kFkPrefixI32: fused_tile_any_mode<PrefixI32Est, V>(it, block, dyn_smem); break;
+    case kBodyBackward: fused_tile_any_mode<BackwardFamilyEst, V>(it, block, dyn_smem); break;
+    case kBodyVtrace: fused_tile_any_mode<VtraceEst, V>(it, block, dyn_smem); break;
+    case kBodyRetrace1: fused_tile_any_mode<RetraceEst, V>(it, block, dyn_smem); break;
+    case kBodyForward: fused_tile_any_mode<TracesEst, V>(it, block, dyn_smem); break;
+    case kBodyPrefixI32: fused_tile_any_mode<PrefixI32Est, V>(it, block, dyn_smem); break;
     default: break;
     }
-}
-
-// Fused launch on the shared body: every fp32 call runs any_tile_body, the
-// int32 prefix sum its own tile body.  Items carry AnyParams for fp32 calls.
-template <int V>
-__global__ void __launch_bounds__(kFusedNT) fused_any_kernel(const __grid_constant__ FusedBatch b) {
-    extern __shared__ __align__(128) unsigned char dyn_smem[];
-    int idx = 0;
-    for (int i = 1; i < b.n; ++i)
-        if ((long long)blockIdx.x >= b.item[i].tile_begin) idx = i;
-    const FusedItem &it = b.item[idx];
-    const long long block = (long long)blockIdx.x - it.tile_begin;
-    if (it.kind == kFkPrefixI32)
-        fused_tile_any_mode<PrefixI32Est, V>(it, block, dyn_smem);
-    else
-        any_tile_body<V>(*reinterpret_cast<const AnyParams *>(it.params), it.g, block, it.mode);
 }
 
 } // namespace rlscan

@@ -78,7 +78,7 @@ struct GaeEstT {
     };
     template <int V>
     struct State {
-        float r[V], v[V], out[V], ret[V];
+        float r[V], v[V], bv[V], out[V], ret[V];
         FlagReg<FlagT> te[V], tr[V];
         float v_next;
     };
@@ -90,17 +90,19 @@ struct GaeEstT {
         case 1: prefetch_l2(P.values, tile0, cnt, sizeof(ValT)); break;
         case 2: prefetch_l2(P.terminateds, tile0, cnt, sizeof(FlagT)); break;
         case 3: prefetch_l2(P.truncateds, tile0, cnt, sizeof(FlagT)); break;
+        case 4: prefetch_l2(P.bootstrap_values, tile0, cnt, sizeof(ValT)); break;
         default: break;
         }
     }
     // Input planes read element by element (the time-major kernel's prefetch).
-    static constexpr int kInputPlanes = 4;
+    static constexpr int kInputPlanes = 5;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         switch (i) {
         case 0: return {P.rewards, (int)sizeof(ValT)};
         case 1: return {P.values, (int)sizeof(ValT)};
         case 2: return {P.terminateds, (int)sizeof(FlagT)};
         case 3: return {P.truncateds, (int)sizeof(FlagT)};
+        case 4: return {P.bootstrap_values, (int)sizeof(ValT)};
         default: return {nullptr, 0};
         }
     }
@@ -112,6 +114,7 @@ struct GaeEstT {
         pos.load_widen(P.values, S.v);
         pos.load_flag(P.terminateds, S.te);
         pos.load_flag(P.truncateds, S.tr);
+        pos.load_widen(P.bootstrap_values, S.bv); // null (no truncations): zeros, no load
         S.v_next = pos.next(S.v, h_v_next);
     }
     template <int V, bool kTrunc, bool kFast, class Pos>
@@ -126,7 +129,7 @@ struct GaeEstT {
                 const bool rowend = elem_row_end<kFast, V>(rm, k);
                 float nv = (k + 1 < V) ? S.v[k + 1] : S.v_next;
                 if (rowend) nv = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
-                const float boot = f.cont ? nv : (f.trn ? pos.one(P.bootstrap_values, k) : 0.0f);
+                const float boot = f.cont ? nv : (f.trn ? S.bv[k] : 0.0f);
                 a[k] = (f.cont && !rowend) ? gl : 0.0f;
                 b[k] = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
             } else {
@@ -182,16 +185,16 @@ struct LambdaReturnsEst {
     };
     template <int V>
     struct State {
-        float r[V], v[V], te[V], tr[V], out[V];
+        float r[V], v[V], te[V], tr[V], bv[V], out[V];
         float v_next;
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
-        prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds);
+        prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values);
     }
-    static constexpr int kInputPlanes = 4;
+    static constexpr int kInputPlanes = 5;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[4] = {P.rewards, P.values, P.terminateds, P.truncateds};
-        return {i < 4 ? p[i] : nullptr, 4};
+        const float *p[5] = {P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values};
+        return {i < 5 ? p[i] : nullptr, 4};
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
@@ -201,6 +204,7 @@ struct LambdaReturnsEst {
         pos.load(P.values, S.v);
         pos.load(P.terminateds, S.te);
         pos.load(P.truncateds, S.tr);
+        pos.load(P.bootstrap_values, S.bv);
         S.v_next = pos.next(S.v, h_v_next);
     }
     template <int V, bool kTrunc, bool kFast, class Pos>
@@ -219,7 +223,7 @@ struct LambdaReturnsEst {
                 // row end ((1 - lambda) V_T + lambda G_T with V_T = G_T = the last
                 // value), the bootstrap value at a truncation and 0 at a termination
                 float boot = 0.0f;
-                if (f.trn) boot = pos.one(P.bootstrap_values, k);
+                if (f.trn) boot = S.bv[k];
                 if (f.cont) {
                     if (rowend) {
                         boot = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
@@ -273,15 +277,15 @@ struct ReturnsEst {
     };
     template <int V>
     struct State {
-        float r[V], te[V], tr[V], out[V];
+        float r[V], te[V], tr[V], bv[V], out[V];
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
-        prefetch_planes(g, tile0, S, P.rewards, P.terminateds, P.truncateds);
+        prefetch_planes(g, tile0, S, P.rewards, P.terminateds, P.truncateds, P.bootstrap_values);
     }
-    static constexpr int kInputPlanes = 3;
+    static constexpr int kInputPlanes = 4;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[3] = {P.rewards, P.terminateds, P.truncateds};
-        return {i < 3 ? p[i] : nullptr, 4};
+        const float *p[4] = {P.rewards, P.terminateds, P.truncateds, P.bootstrap_values};
+        return {i < 4 ? p[i] : nullptr, 4};
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
@@ -289,6 +293,7 @@ struct ReturnsEst {
         pos.load(P.rewards, S.r);
         pos.load(P.terminateds, S.te);
         pos.load(P.truncateds, S.tr);
+        pos.load(P.bootstrap_values, S.bv);
     }
     template <int V, bool kTrunc, bool kFast, class Pos>
     static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
@@ -303,7 +308,7 @@ struct ReturnsEst {
                 // last value at a row end, the bootstrap value at a
                 // truncation, nothing otherwise (the scan carries R_{t+1})
                 float boot = 0.0f;
-                if (f.trn) boot = pos.one(P.bootstrap_values, k);
+                if (f.trn) boot = S.bv[k];
                 if (f.cont && rowend) boot = row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows);
                 a[k] = (f.cont && !rowend) ? P.gamma : 0.0f;
                 b[k] = fmaf(P.gamma, boot, S.r[k]);
@@ -352,19 +357,20 @@ struct VtraceEst {
     };
     template <int V>
     struct State {
-        float lr[V], r[V], v[V], te[V], tr[V];
+        float lr[V], r[V], v[V], te[V], tr[V], bv[V];
         float rho[V];
         float vs[V], pg[V];
         float v_next;
         unsigned chained; // bit k: the trace goes on to t+1 inside the row
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
-        prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds);
+        prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds,
+                        P.bootstrap_values);
     }
-    static constexpr int kInputPlanes = 5;
+    static constexpr int kInputPlanes = 6;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[5] = {P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds};
-        return {i < 5 ? p[i] : nullptr, 4};
+        const float *p[6] = {P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values};
+        return {i < 6 ? p[i] : nullptr, 4};
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
@@ -375,6 +381,7 @@ struct VtraceEst {
         pos.load(P.values, S.v);
         pos.load(P.terminateds, S.te);
         pos.load(P.truncateds, S.tr);
+        pos.load(P.bootstrap_values, S.bv);
         S.v_next = pos.next(S.v, h_v_next);
     }
     template <int V, bool kTrunc, bool kFast, class Pos>
@@ -395,7 +402,7 @@ struct VtraceEst {
                     boot = rowend ? row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows)
                                   : ((k + 1 < V) ? S.v[k + 1] : S.v_next);
                 } else {
-                    boot = f.trn ? pos.one(P.bootstrap_values, k) : 0.0f;
+                    boot = f.trn ? S.bv[k] : 0.0f;
                 }
                 a[k] = (f.cont && !rowend) ? P.gamma * c : 0.0f;
                 b[k] = rho * (fmaf(P.gamma, boot, S.r[k]) - S.v[k]);
@@ -458,19 +465,20 @@ struct GaeVtraceEst {
     };
     template <int V>
     struct State {
-        float lr[V], r[V], v[V], te[V], tr[V];
+        float lr[V], r[V], v[V], te[V], tr[V], bv[V];
         float rho[V];
         float adv[V], ret[V], vs[V], pg[V];
         float v_next;
         unsigned chained; // bit k: the traces go on to t+1 inside the row
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
-        prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds);
+        prefetch_planes(g, tile0, S, P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds,
+                        P.bootstrap_values);
     }
-    static constexpr int kInputPlanes = 5;
+    static constexpr int kInputPlanes = 6;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[5] = {P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds};
-        return {i < 5 ? p[i] : nullptr, 4};
+        const float *p[6] = {P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values};
+        return {i < 6 ? p[i] : nullptr, 4};
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
@@ -481,6 +489,7 @@ struct GaeVtraceEst {
         pos.load(P.values, S.v);
         pos.load(P.terminateds, S.te);
         pos.load(P.truncateds, S.tr);
+        pos.load(P.bootstrap_values, S.bv);
         S.v_next = pos.next(S.v, h_v_next);
     }
     template <int V, bool kTrunc, bool kFast, class Pos>
@@ -502,7 +511,7 @@ struct GaeVtraceEst {
                     boot = rowend ? row_last_value(P.last_values, elem_row<kFast>(rm, k), g.rows)
                                   : ((k + 1 < V) ? S.v[k + 1] : S.v_next);
                 } else {
-                    boot = f.trn ? pos.one(P.bootstrap_values, k) : 0.0f;
+                    boot = f.trn ? S.bv[k] : 0.0f;
                 }
                 const bool go = f.cont && !rowend;
                 const float delta = fmaf(P.gamma, boot, S.r[k]) - S.v[k];
@@ -548,22 +557,18 @@ struct GaeVtraceEst {
 };
 
 // ---------------------------------------------------------------------------
-// Retrace(lambda): x = Q_ret - q,  a_t = gamma c_{t+1}, b_t = delta_t.
-// kMulti: V'_t = sum_a pi'[t,a] Q'[t,a] from the per-action rows, staged in
-// shared memory by 1-D bulk copies; otherwise V'_t = next_q_values_all[t].
+// Retrace(lambda): x = Q_ret - q,  a_t = gamma c_{t+1}, b_t = delta_t, with
+// the expected next-state value V'_t = next_q_values_all[t] (one action, or
+// the plane expected_value_kernel writes for several).
 // ---------------------------------------------------------------------------
-template <bool kMulti>
 struct RetraceEst {
     static constexpr bool kBackward = true;
     using AT = float;
     using BT = float;
     struct Params {
-        const float *rewards, *q_values, *next_q_values_all, *next_target_probs, *log_rhos, *terminateds,
-            *truncateds;
+        const float *rewards, *q_values, *next_q_values_all, *log_rhos, *terminateds, *truncateds;
         float *q_ret;
-        long long actions;
         float gamma, lambda_, c_bar;
-        unsigned copy_spin_limit;
     };
     template <int V>
     struct State {
@@ -573,87 +578,16 @@ struct RetraceEst {
 
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.rewards, P.q_values, P.log_rhos, P.terminateds, P.truncateds,
-                        kMulti ? nullptr : P.next_q_values_all);
-        if constexpr (kMulti) {
-            const long long left = g.n - tile0;
-            const long long cnt = left < S ? left : S;
-            if (threadIdx.x == 6) prefetch_l2(P.next_q_values_all, tile0 * P.actions, cnt * P.actions, 4);
-            if (threadIdx.x == 7) prefetch_l2(P.next_target_probs, tile0 * P.actions, cnt * P.actions, 4);
-        }
+                        P.next_q_values_all);
     }
-    // single-action form only (the time-major kernel takes A == 1)
     static constexpr int kInputPlanes = 6;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[6] = {P.rewards, P.q_values, P.log_rhos, P.terminateds, P.truncateds,
-                             kMulti ? nullptr : P.next_q_values_all};
+        const float *p[6] = {P.rewards, P.q_values, P.log_rhos, P.terminateds, P.truncateds, P.next_q_values_all};
         return {i < 6 ? p[i] : nullptr, 4};
     }
-
-    // Expected next-state value of each of this thread's elements.
-    template <int NT, int V>
-    static __device__ __forceinline__ void stage_expected_values(const Params &P, const Geometry &g, long long i0,
-                                                                 State<V> &S, unsigned char *smem) {
-        constexpr int TILE = NT * V;
-        const int tid = threadIdx.x;
-        const long long tile0 = i0 - (long long)tid * V;
-        const long long left = g.n - tile0;
-        const int nvalid = left < TILE ? (int)left : TILE;
-        const int A = (int)P.actions;
-        uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
-        float *sq = reinterpret_cast<float *>(smem + 128);
-        float *sp = sq + (size_t)TILE * A;
-        float *vp = sp + (size_t)TILE * A;
-        const float *gq = P.next_q_values_all + tile0 * A;
-        const float *gp = P.next_target_probs + tile0 * A;
-        const uint32_t bytes = (uint32_t)nvalid * (uint32_t)A * 4u;
-        const bool bulk = (bytes % 16u == 0u) && ((reinterpret_cast<uintptr_t>(gq) & 15u) == 0) &&
-                          ((reinterpret_cast<uintptr_t>(gp) & 15u) == 0);
-        if (bulk) {
-            if (tid == 0) {
-                // the previous grid wrote these rows with ordinary stores; order
-                // them before the bulk copies, which read through the async proxy
-                asm volatile("fence.proxy.async;" ::: "memory");
-                mbar_init(bar, 1);
-                mbar_arrive_expect_tx(bar, 2u * bytes);
-                bulk_copy_g2s(sq, gq, bytes, bar);
-                bulk_copy_g2s(sp, gp, bytes, bar);
-            }
-            __syncthreads(); // barrier initialised before anyone polls it
-            bool ok = mbar_try_wait(bar, 0);
-            for (unsigned polls = 0; !ok && polls < P.copy_spin_limit; ++polls) ok = mbar_try_wait(bar, 0);
-            if (!ok) atomicOr(&g_device_error, kErrCopyTimeout);
-        } else {
-            const int total = nvalid * A;
-            for (int idx = tid; idx < total; idx += NT) {
-                sq[idx] = __ldcg(gq + idx);
-                sp[idx] = __ldcg(gp + idx);
-            }
-            __syncthreads();
-        }
-        // one element per thread per pass, neighbouring lanes on neighbouring
-        // elements (row stride A words: at most 2-way bank conflicts for even A)
-#pragma unroll
-        for (int k = 0; k < V; ++k) {
-            const int e = tid + NT * k;
-            if (e < nvalid) {
-                const float *qe = sq + (size_t)e * A;
-                const float *pe = sp + (size_t)e * A;
-                float s = 0.0f;
-                for (int act = 0; act < A; ++act) s = fmaf(pe[act], qe[act], s);
-                vp[e] = s;
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int k = 0; k < V; ++k) {
-            const int e = tid * V + k;
-            S.vnext[k] = e < nvalid ? vp[e] : 0.0f;
-        }
-    }
-
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
-                                                State<V> &S, unsigned char *smem) {
+                                                State<V> &S, unsigned char *) {
         const float h_lr_next = pos.fetch_next(P.log_rhos);
         pos.load(P.rewards, S.r);
         pos.load(P.q_values, S.q);
@@ -661,13 +595,7 @@ struct RetraceEst {
         pos.load(P.terminateds, S.te);
         pos.load(P.truncateds, S.tr);
         S.lr_next = pos.next(S.lr, h_lr_next);
-        if constexpr (kMulti) {
-            // per-action rows are staged for row-major tiles only (time-major
-            // calls with more than one action are rejected on the host)
-            stage_expected_values<NT, V>(P, g, pos.index(0), S, smem);
-        } else {
-            pos.load(P.next_q_values_all, S.vnext);
-        }
+        pos.load(P.next_q_values_all, S.vnext);
     }
     template <int V, bool kFast, class Pos>
     static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,

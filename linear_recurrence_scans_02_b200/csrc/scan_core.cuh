@@ -3,8 +3,8 @@
 // The rl-triton paper (arXiv:2608.17641, abstract) solves every estimator as
 // one first-order linear recurrence x_t = a_t x_{t-+1} + b_t with the
 // associative operator (a1, b1) o (a2, b2) = (a1 a2, a1 b2 + b1), where
-// (a2, b2) is the map applied first.  This file holds that operator and one
-// single-pass scan over the flattened [E*T] array:
+// (a2, b2) is the map applied first.  This file holds that operator and the
+// scan over the flattened [E*T] array:
 //
 //   * the array is cut into tiles of S = NT*V consecutive elements, one CTA
 //     per tile; each thread owns V consecutive elements (128-bit loads);
@@ -12,12 +12,11 @@
 //     builder sets a = 0 on the first element of a row in scan order (the
 //     row's last value is folded into b there), the same cut a done makes;
 //   * in-thread sequential compose -> warp shuffle scan -> shared-memory scan
-//     of warp aggregates -> (optional) decoupled look-back over the
-//     aggregates of earlier tiles -> per-thread carry -> sequential epilogue;
-//   * look-back is only compiled in when a tile boundary can fall inside a
-//     row; tiles take their scan-order index from an atomic counter so a
-//     tile only ever waits for tiles that are already running, and every
-//     wait is bounded.
+//     of warp aggregates -> per-thread carry -> sequential epilogue;
+//   * when rows span tiles, two launches: the first writes every tile's
+//     aggregate, the second scans each tile with the carry composed from the
+//     complete aggregates of the tiles before it (no block ever waits for
+//     another).
 //
 // Scan order is memory order for forward recurrences and reversed memory
 // order for backward ones.  "Earlier" below always means earlier in scan
@@ -34,14 +33,6 @@ namespace rlscan {
 
 constexpr unsigned kFullMask = 0xffffffffu;
 
-// Device-wide error word: bit 0 = a look-back wait gave up, bit 1 = a bulk
-// copy wait gave up, bit 2 = a workspace was not zero-filled at launch.
-// Read and cleared by rlscan_check().
-__device__ unsigned int g_device_error = 0;
-constexpr unsigned kErrLookbackTimeout = 1u;
-constexpr unsigned kErrCopyTimeout = 2u;
-constexpr unsigned kErrWorkspaceState = 4u; // workspace was not zero-filled at launch
-
 // ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
@@ -54,16 +45,6 @@ __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 // Four relaxed 32-bit loads in one instruction (no ordering among them).
 __device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const void *p) {
     uint4 v;
@@ -72,48 +53,6 @@ __device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const void *p) {
                  : "l"(p)
                  : "memory");
     return v;
-}
-// With a preceding relaxed load, the acquire pattern of the PTX memory model.
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-__device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_relaxed_gpu(unsigned *p, unsigned v) {
-    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// mbarrier + 1-D bulk copy (TMA engine, no tensor map, no multicast).
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase)
-        : "memory");
-    return ok != 0;
-}
-// Copy `bytes` (multiple of 16; both addresses 16-byte aligned) from global
-// to this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
 }
 
 // Hint: bring [p + first, p + first + count) elements of a plane into L2.  The
@@ -240,38 +179,21 @@ __device__ __forceinline__ void warp_exclusive_from_inclusive(AT ia, BT ib, int 
 }
 
 // ---------------------------------------------------------------------------
-// Workspace for the look-back: a header with the tile counter, and one
-// 16-byte slot per tile.  status: 0 = nothing yet, 1 = the tile's aggregate
-// (a, b) is published, 2 = its inclusive value x (the carry into the next
-// tile) is published.  The last CTA to finish zeroes every slot and both
-// counters, so the workspace is left zero-filled, as it was found.
+// Workspace of a split-row call: one 16-byte slot per tile.  Pass one writes
+// the tile's aggregate {a, b} in the first half; pass two may publish the
+// tile's inclusive value {1, x} in the second half (see the two-pass carries
+// below).
 // ---------------------------------------------------------------------------
-
-struct WsHeader {
-    unsigned tile_counter;
-    unsigned pad0[15];
-    unsigned done_counter; // its own 32-byte sector: the two counters are hit at different times
-    unsigned pad1[15];
-};
-static_assert(sizeof(WsHeader) == 128, "header is one 128-byte line");
-
 struct TileSlot {
-    unsigned status;
-    unsigned a;
-    unsigned b;
-    unsigned x;
+    unsigned w[4];
 };
 static_assert(sizeof(TileSlot) == 16, "slot is 16 bytes");
 
 struct Lookback {
-    WsHeader *hdr;       // nullptr when the launch needs no look-back
-    TileSlot *slots;
-    unsigned spin_limit; // polls before a wait gives up
-    long long withhold;  // scan-order tile that never publishes (test hook), -1 = none
+    TileSlot *slots;     // the call's workspace (split-row calls), else nullptr
     long long row_tiles; // tiles per row when rows are whole multiples of a tile, else 0
-    long long tile_base; // two-pass modes: scan-order index of the launch's first tile
+    long long tile_base; // scan-order index of the launch's first tile
 };
-
 
 // Geometry of one launch over the flattened [E*T] array.
 struct Geometry {
@@ -283,17 +205,6 @@ struct Geometry {
     int vec_ok;        // every plane pointer of the call is 16-byte aligned
     int scan_lanes;    // warp-local mode: lanes one row spans (a power of two <= 32)
 };
-
-// Scan-order tile of the t-th tile taken from the counter.  When every row
-// is a whole number of tiles, the counter deals the rows' tiles out in
-// turn (row r's c-th tile is ticket c E + r), so the tiles running at once
-// spread over all rows and each row's chain of carries stays short; a tile
-// still only waits on tiles of its own row with smaller tickets, which have
-// started.  Otherwise tiles are taken in scan order.
-__device__ __forceinline__ long long lookback_tile(const Lookback &lb, const Geometry &g, long long t) {
-    if (lb.row_tiles <= 0) return t;
-    return (t % g.rows) * lb.row_tiles + t / g.rows;
-}
 
 // Where a thread's V elements sit in their rows, as bit masks over k:
 // end bit k = element k is the last step of its row (t == T-1), start bit
@@ -364,133 +275,6 @@ __device__ __forceinline__ bool elem_row_start(const RowMasks &m, int k) {
 template <bool kFast>
 __device__ __forceinline__ long long elem_row(const RowMasks &m, int k) {
     return kFast ? m.row0 : row_of(m, k);
-}
-
-// Warp-wide decoupled look-back, called by all 32 lanes of one warp.
-// Lane 0 publishes this tile's aggregate (or its inclusive value when it
-// needs no carry, or when its own chain is cut).  The warp then inspects
-// 32 x kLbPerLane earlier tiles at once, lane i reading tiles
-// base - i kLbPerLane - m, m = 0 .. kLbPerLane - 1 (nearest first): when one
-// of them holds an inclusive value, the carry is that value passed through
-// the aggregates of the nearer tiles; otherwise all hold aggregates, whose
-// composition is folded in before the next window.  A tile whose own chain
-// is cut always publishes an inclusive value, so the walk ends at the row's
-// first tile at the latest.  Lane 0 then publishes this tile's inclusive
-// value.  Every wait is bounded; a wait that gives up sets the device error
-// word and the walk ends as if the carry were zero.
-constexpr int kLbPerLane = 1;
-
-// k_min: the lowest tile the walk may read; tiles before it are never
-// needed (the row's first tile always publishes an inclusive value) and
-// may not have started yet when the counter deals tiles out row by row.
-template <class AT, class BT>
-__device__ BT lookback_carry(const Lookback &lb, long long j, long long k_min, bool needs_carry, AT ta, BT tb,
-                             int lane) {
-    TileSlot *me = lb.slots + j;
-    const bool publish = (j != lb.withhold) && lane == 0;
-    if (!needs_carry) {
-        if (publish) {
-            st_relaxed_gpu(&me->x, to_bits(tb));
-            st_release_gpu(&me->status, 2u);
-        }
-        return identity_b(tb);
-    }
-    const bool cut = (ta == AT(0)); // the tile's own chain is cut: its output needs no carry
-    if (publish) {
-        if (cut) {
-            st_relaxed_gpu(&me->x, to_bits(tb));
-            st_release_gpu(&me->status, 2u);
-        } else {
-            st_relaxed_gpu(&me->a, to_bits(ta));
-            st_relaxed_gpu(&me->b, to_bits(tb));
-            st_release_gpu(&me->status, 1u);
-        }
-    }
-    constexpr int M = kLbPerLane;
-    AT acc_a = identity_a(ta); // composition of the aggregates walked so far
-    BT acc_b = identity_b(tb);
-    BT carry = identity_b(tb);
-    for (long long base = j - 1;; base -= 32 * M) {
-        const long long k0 = base - (long long)lane * M;
-        // statuses by relaxed loads, all in flight together; then one fence
-        // (relaxed load + fence = acquire) before the published values are read
-        unsigned st[M];
-#pragma unroll
-        for (int m = 0; m < M; ++m) st[m] = (k0 - m >= k_min) ? ld_relaxed_gpu(&lb.slots[k0 - m].status) : 2u;
-        bool gave_up = false;
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            unsigned ns = 32, polls = 0;
-            while (st[m] == 0u) {
-                if (++polls > lb.spin_limit) {
-                    gave_up = true;
-                    break;
-                }
-                __nanosleep(ns);
-                if (ns < 256u) ns <<= 1;
-                st[m] = ld_relaxed_gpu(&lb.slots[k0 - m].status);
-            }
-        }
-        if (__any_sync(kFullMask, gave_up)) {
-            if (lane == 0) atomicOr(&g_device_error, kErrLookbackTimeout);
-            carry = acc_b;
-            break;
-        }
-        fence_acq_rel_gpu();
-        uint4 slot[M];
-#pragma unroll
-        for (int m = 0; m < M; ++m)
-            slot[m] = (k0 - m >= k_min) ? ld_relaxed_gpu_v4(&lb.slots[k0 - m]) : make_uint4(0u, 0u, 0u, 0u);
-        // this lane's M tiles composed nearest-outermost, stopping at the
-        // first inclusive value or cut (a == 0: the map ignores what came before)
-        AT la = identity_a(ta);
-        BT lb_ = identity_b(tb);
-        bool stop = false;
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            if (stop) break;
-            const long long k = k0 - m;
-            AT ka;
-            BT kb;
-            if (k < k_min) { // nothing flows in from before the row / array
-                ka = AT(0);
-                kb = identity_b(tb);
-            } else if (st[m] == 2u) { // an inclusive value: the map x -> x_k
-                ka = AT(0);
-                kb = from_bits(slot[m].w, tb);
-            } else { // an aggregate (a, b), published before status 1
-                ka = from_bits(slot[m].y, ta);
-                kb = from_bits(slot[m].z, tb);
-            }
-            combine(la, lb_, ka, kb);
-            stop = (ka == AT(0));
-        }
-        const unsigned stops = __ballot_sync(kFullMask, stop);
-        const int last = stops ? __ffs(stops) - 1 : 31;
-        if (lane > last) { // farther than the nearest stop: contributes nothing
-            la = identity_a(ta);
-            lb_ = identity_b(tb);
-        }
-        // ordered composition over lanes 0..last: lane 0 (nearest) applied last
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const AT oa = shfl_down(la, d);
-            const BT ob = shfl_down(lb_, d);
-            if (lane + d < 32) combine(la, lb_, oa, ob);
-        }
-        la = shfl_idx(la, 0);
-        lb_ = shfl_idx(lb_, 0);
-        combine(acc_a, acc_b, la, lb_);
-        if (stops) { // the composed map starts from a cut: its b is the carry
-            carry = acc_b;
-            break;
-        }
-    }
-    if (publish && !cut) {
-        st_relaxed_gpu(&me->x, to_bits(apply_pair(ta, tb, carry)));
-        st_release_gpu(&me->status, 2u);
-    }
-    return carry;
 }
 
 // ---------------------------------------------------------------------------
@@ -600,31 +384,6 @@ __device__ BT carry_from_aggregates(const Lookback &lb, long long j, long long k
     }
     if (lane == 0) publish_inclusive(me, apply_pair(ta, tb, carry));
     return carry;
-}
-
-// Last CTA out resets the workspace.
-template <int NT>
-__device__ __forceinline__ void lookback_release(const Lookback &lb, long long ntiles) {
-    __shared__ int s_last;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        // release: this block's slot traffic (ordered before thread 0 by the
-        // barrier) precedes the increment; acquire: the last block sees every
-        // other block's before it clears the slots
-        unsigned prev;
-        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(&lb.hdr->done_counter) : "memory");
-        s_last = (prev == (unsigned)(ntiles - 1));
-    }
-    __syncthreads();
-    if (s_last) {
-        for (long long i = threadIdx.x; i < ntiles; i += NT)
-            *reinterpret_cast<uint4 *>(lb.slots + i) = make_uint4(0u, 0u, 0u, 0u);
-        if (threadIdx.x == 0) {
-            lb.hdr->tile_counter = 0u;
-            lb.hdr->done_counter = 0u;
-        }
-        __threadfence();
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -955,14 +714,11 @@ __device__ __forceinline__ RowMasks time_major_masks(const TimeMajorPos<V> &pos)
 
 // Scan modes of one launch:
 //   kModeBlock     tiles hold whole rows; warps exchange carries in shared memory
-//   kModeLookback  rows span tiles; tiles exchange carries through the workspace
-//                  in one pass (decoupled look-back with bounded waits)
 //   kModeWarp      every warp's 32*V elements hold whole rows: no block scan at all
 //   kModeReduce    rows span tiles, pass one of two: write each tile's aggregate
 //   kModeCarry     rows span tiles, pass two: scan each tile with the carry
 //                  composed from the complete aggregates (no waiting)
 constexpr int kModeBlock = 0;
-constexpr int kModeLookback = 1;
 constexpr int kModeWarp = 2;
 constexpr int kModeReduce = 3;
 constexpr int kModeCarry = 4;
@@ -975,7 +731,6 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     using AT = typename Est::AT;
     using BT = typename Est::BT;
     constexpr bool kBwd = Est::kBackward;
-    constexpr bool kLookback = kMode == kModeLookback;
     constexpr bool kWarpLocal = kMode == kModeWarp;
     constexpr bool kReduce = kMode == kModeReduce;
     constexpr bool kCarry = kMode == kModeCarry;
@@ -986,40 +741,24 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     __shared__ AT s_wa[NW];
     __shared__ BT s_wb[NW];
     __shared__ BT s_wx[NW];
-    __shared__ long long s_tile;
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
 
+    // tile index in scan order
+    const long long j = kTwoPass ? lb.tile_base + block : block;
     // Start this tile's DRAM reads before waiting for the previous grid on
-    // the stream: the L2 prefetch overlaps them with that grid's tail.  With
-    // the look-back the tile index is only known after the wait; the block
-    // index is the likely one (a wrong guess only costs a wasted prefetch).
-    // Once the wait returns, let the next grid launch (it waits for this one
-    // to complete before touching memory).
+    // the stream: the L2 prefetch overlaps them with that grid's tail.  Once
+    // the wait returns, let the next grid launch (it waits for this one to
+    // complete before touching memory).
     {
-        const long long jg = kLookback ? lookback_tile(lb, g, block) : (kTwoPass ? lb.tile_base + block : block);
-        const long long mg = kBwd ? (g.ntiles - 1 - jg) : jg;
+        const long long mg = kBwd ? (g.ntiles - 1 - j) : j;
         Est::prefetch(P, g, mg * (long long)(NT * V), NT * V);
     }
     griddep_wait();
     griddep_launch_dependents();
 
-    long long j; // tile index in scan order
-    if constexpr (kLookback) {
-        if (tid == 0) s_tile = (long long)atomicAdd(&lb.hdr->tile_counter, 1u);
-        __syncthreads();
-        if (s_tile >= g.ntiles) { // counter was not zero at launch: touch nothing, report
-            if (tid == 0) atomicOr(&g_device_error, kErrWorkspaceState);
-            return;
-        }
-        j = lookback_tile(lb, g, s_tile);
-    } else if constexpr (kTwoPass) {
-        j = lb.tile_base + block;
-    } else {
-        j = block;
-    }
     const long long m = kBwd ? (g.ntiles - 1 - j) : j; // tile index in memory
     const long long tile0 = m * (long long)(NT * V);
     const long long i0 = tile0 + (long long)tid * V;
@@ -1086,7 +825,7 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
             BT web;
             warp_exclusive_from_inclusive<kBwd>(wa, wb, lane, wea, web);
             BT carry = identity_b(tb);
-            if constexpr (kLookback || kTwoPass) {
+            if constexpr (kTwoPass) {
                 const AT tile_a = shfl_idx(wa, kBwd ? 0 : NW - 1);
                 const BT tile_b = shfl_idx(wb, kBwd ? 0 : NW - 1);
                 bool needs_carry;
@@ -1097,9 +836,7 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
                     needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
                 }
                 const long long k_min = lb.row_tiles > 0 ? (j / lb.row_tiles) * lb.row_tiles : 0;
-                if constexpr (kLookback) {
-                    carry = lookback_carry<AT, BT>(lb, j, k_min, needs_carry, tile_a, tile_b, lane);
-                } else if constexpr (kCarry) {
+                if constexpr (kCarry) {
                     carry = carry_from_aggregates<AT, BT>(lb, j, k_min, needs_carry, tile_a, tile_b, lane);
                 } else if (lane == 0) {
                     publish_aggregate(lb.slots + j, tile_a, tile_b);
@@ -1130,7 +867,6 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     }
     Est::template store<V>(P, g, pos, S);
 
-    if constexpr (kLookback) lookback_release<NT>(lb, g.ntiles);
 }
 
 template <class Est, int NT, int V, int kMode>

@@ -38,7 +38,7 @@ __all__ = [
     "RlscanError", "library_path",
     "rlscan_gae", "rlscan_gae_with_returns", "rlscan_gae_typed", "rlscan_gae_vtrace", "rlscan_vtrace", "rlscan_retrace", "rlscan_lambda_returns",
     "rlscan_discounted_returns", "rlscan_eligibility_traces", "rlscan_episodic_prefix_sum",
-    "rlscan_batch", "rlscan_workspace_bytes", "rlscan_check", "rlscan_plan", "rlscan_debug_set_lookback",
+    "rlscan_batch", "rlscan_workspace_bytes", "rlscan_check", "rlscan_plan",
     "compute_gae", "compute_gae_with_returns", "compute_gae_vtrace", "compute_vtrace", "compute_retrace", "compute_lambda_returns",
     "compute_discounted_returns", "compute_eligibility_traces", "compute_episodic_prefix_sum",
 ]
@@ -117,7 +117,6 @@ def _load_library():
         "rlscan_workspace_init": [P, SZ, S],
         "rlscan_check": [S],
         "rlscan_version": [],
-        "rlscan_debug_set_lookback": [ctypes.c_uint32, I64],
         "rlscan_plan": [I64, I64, I64, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int),
                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int64)],
     }
@@ -208,7 +207,7 @@ def rlscan_workspace_bytes(num_envs: int, seq_len: int) -> int:
 
 
 def rlscan_check(stream=None) -> None:
-    """Synchronise the stream and raise if a kernel reported a timed-out wait."""
+    """Synchronise the stream and raise if the work on it failed."""
     s = torch.cuda.current_stream().cuda_stream if stream is None else stream
     _raise_on(_lib.rlscan_check(s))
 
@@ -218,10 +217,6 @@ def rlscan_plan(num_envs: int, seq_len: int, actions: int = 1) -> dict:
     _raise_on(_lib.rlscan_plan(num_envs, seq_len, actions, ctypes.byref(te), ctypes.byref(th),
                                ctypes.byref(lb), ctypes.byref(nt)))
     return {"tile_elems": te.value, "threads": th.value, "lookback": bool(lb.value), "num_tiles": nt.value}
-
-
-def rlscan_debug_set_lookback(spin_limit: int = 0, withhold_tile: int = -1) -> None:
-    _raise_on(_lib.rlscan_debug_set_lookback(int(spin_limit), int(withhold_tile)))
 
 
 # ---------------------------------------------------------------------------

@@ -155,14 +155,14 @@ def test_plan_split_rows_need_workspace(lib, E_, T_):
     tile, threads, lookback, ntiles = plan(lib, E_, T_)
     assert lookback
     need = lib.rlscan_workspace_bytes(E_, T_)
-    assert need >= 128 + 16 * ntiles
+    assert need >= 16 * ntiles
 
 
 def test_missing_workspace_rejected(lib):
     # 16 x 262144 splits rows over tiles: a workspace is required
     assert lib.rlscan_gae(A, B, C, None, None, None, O1, 16, 262144, 0.99, 0.95, None, 0, None) == WORKSPACE
     _, _, lookback, ntiles = plan(lib, 16, 262144)
-    need = 128 + 16 * ntiles  # what this call's plan needs
+    need = 16 * ntiles  # what this call's plan needs: one 16-byte slot per tile
     assert lookback and lib.rlscan_workspace_bytes(16, 262144) >= need
     assert lib.rlscan_gae(A, B, C, None, None, None, O1, 16, 262144, 0.99, 0.95, D, need - 16, None) == WORKSPACE
     assert lib.rlscan_gae(A, B, C, None, None, None, O1, 16, 262144, 0.99, 0.95, D + 4, need, None) == WORKSPACE
@@ -171,7 +171,7 @@ def test_missing_workspace_rejected(lib):
 def test_workspace_bytes_bounds(lib):
     assert lib.rlscan_workspace_bytes(0, 10) == 0
     assert lib.rlscan_workspace_bytes(-1, 10) == 0
-    # multi-action Retrace with 512-element tiles splits 4096-step rows
+    # whole rows: no call of this shape needs a workspace
     assert lib.rlscan_workspace_bytes(4096, 128) == 0
     assert lib.rlscan_workspace_bytes(16, 262144) > 0
 
