@@ -34,7 +34,6 @@ import concurrent.futures as cf
 import hashlib
 import json
 import os
-import re
 import subprocess
 import sys
 import tempfile
@@ -355,16 +354,21 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(est: str):
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
-    if not os.path.exists(path):
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+
+
+def recorded_traffic(name: str):
+    """DRAM bytes (read + write) per launch of `name` from the ncu launch
+    list summarised in profiles/dram_traffic.json, or None when that record
+    was taken from other kernel sources than these."""
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+    except (OSError, ValueError):
         return None
-    sha = kernel_source_sha()
-    for line in open(path):
-        m = re.match(r"\|\s*(\w+)\s*\|\s*([0-9]+)\s*\|\s*([0-9a-f]+)\s*\|", line)
-        if m and m.group(1) == est and m.group(3) == sha:
-            return int(m.group(2))
-    return None
+    if rec.get("kernel_sha") != kernel_source_sha():
+        return None
+    e = rec.get("launches", {}).get(name)
+    return None if e is None else int(e["dram_read_bytes"] + e["dram_write_bytes"])
 
 
 def measured_hbm_peak():
@@ -507,7 +511,7 @@ TRUNC_P = 0.005  # terminated and truncated, each (mutually exclusive per step)
 
 def config_cases():
     """(key, E, T, host-input builder, {estimator: (call, streamed bytes per
-    env-step, outputs, input planes)}).  Streamed bytes count every dense plane read once and every
+    env-step, outputs, input planes[, element types of the planes])}).  Streamed bytes count every dense plane read once and every
     output written once; bootstrap values are read only at truncated steps
     (about 1 % of steps here) and are not counted."""
     from linear_recurrence_scans_02_b200 import workloads as W
@@ -567,6 +571,42 @@ def config_cases():
         d.update(W.trace_inputs(16, 262144, 31, p_done=1e-4))
         return d
 
+    # reduced-byte inputs (bf16 values, uint8 flags) beside the same calls on
+    # fp32 inputs, at the 4096 x 128 workload and at 65536 x 128
+    BF, U8 = "bfloat16", "uint8"
+    narrow_dt = {"rewards": BF, "values": BF, "log_rhos": BF, "x": BF, "terminateds": U8, "dones": U8}
+
+    def narrow_cases(E):
+        def gae_ret(R, t, o):
+            return lambda: R.rlscan_gae_typed(t["rewards"], t["values"], t["terminateds"], None, None, None, o[0],
+                                              o[1], GAMMA, LAMBDA)
+
+        def vtrace(R, t, o):
+            return lambda: R.rlscan_vtrace(t["log_rhos"], t["rewards"], t["values"], t["terminateds"], None, None,
+                                           None, o[0], o[1], GAMMA, 1.0, 1.0, 1.0)
+
+        def returns(R, t, o):
+            return lambda: R.rlscan_discounted_returns(t["rewards"], t["terminateds"], None, None, None, o[0], GAMMA)
+
+        def traces(R, t, o):
+            return lambda: R.rlscan_eligibility_traces(t["x"], t["dones"], o[0], GAMMA, LAMBDA)
+
+        gk, vk, rk, tk = (("rewards", "values", "terminateds"), ("log_rhos", "rewards", "values", "terminateds"),
+                          ("rewards", "terminateds"), ("x", "dones"))
+        return {"gae_with_returns_fp32": (gae_ret, 20, 2, gk), "gae_with_returns_bf16_u8": (gae_ret, 13, 2, gk, narrow_dt),
+                "vtrace_fp32": (vtrace, 24, 2, vk), "vtrace_bf16_u8": (vtrace, 15, 2, vk, narrow_dt),
+                "discounted_returns_fp32": (returns, 12, 1, rk),
+                "discounted_returns_bf16_u8": (returns, 7, 1, rk, narrow_dt),
+                "eligibility_traces_fp32": (traces, 12, 1, tk),
+                "eligibility_traces_bf16_u8": (traces, 7, 1, tk, narrow_dt)}
+
+    def narrow_inputs(E):
+        def build():
+            d = W.vtrace_inputs(E, T_STEPS, 50, p_term=P_DONE)
+            d.update(W.trace_inputs(E, T_STEPS, 51, p_done=P_DONE))
+            return d
+        return build
+
     return [
         ("gae_64x512", 64, 512, lambda: W.gae_inputs(64, 512, 10, p_term=0.01),
          {"gae": (gae, 16, 1, ("rewards", "values", "terminateds"))}),
@@ -574,6 +614,8 @@ def config_cases():
         ("off_policy_1024x2048_18_actions", 1024, 2048, lambda: W.off_policy_inputs(1024, 2048, A=A, seed=40),
          off),
         ("long_rows_16x262144", 16, 262144, long_inputs, long_rows),
+        ("reduced_bytes_4096x128", E_ENVS, T_STEPS, narrow_inputs(E_ENVS), narrow_cases(E_ENVS)),
+        ("reduced_bytes_65536x128", 65536, T_STEPS, narrow_inputs(65536), narrow_cases(65536)),
     ]
 
 
@@ -583,11 +625,15 @@ def run_configs(torch, R, device, side, stream, world, peak, max_sets=2048):
     for key, E, T, build, cases in config_cases():
         host = build()
         res = {"num_envs": E, "seq_len": T}
-        for est, (make, bpe, nout, keys) in cases.items():
+        for est, case in cases.items():
+            make, bpe, nout, keys = case[:4]
+            dts = case[4] if len(case) > 4 else {}
             nbytes = bpe * E * T
             nset = min(max_sets, max(2, -(-rot // nbytes)))
-            # one device copy of the inputs per set (only the planes this call reads)
+            # one device copy of the inputs per set (only the planes this call
+            # reads, each in the element type the case names, else fp32)
             planes = {k: torch.from_numpy(np.ascontiguousarray(host[k])) for k in keys}
+            planes = {k: v.to(getattr(torch, dts[k])) if k in dts else v for k, v in planes.items()}
             fns = []
             for _ in range(nset):
                 t = {k: v.to(device) for k, v in planes.items()}

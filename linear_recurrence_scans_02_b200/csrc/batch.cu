@@ -2,7 +2,7 @@
 // fusable calls run as one launch of the fused kernels (batch.cuh), whose
 // blocks run one tile of one call each; the others through their own entry
 // points, which this file calls.
-#include "host.cuh"
+#include "typed.cuh"
 
 using namespace rlscan;
 
@@ -40,21 +40,32 @@ static size_t call_slot_bytes(const rlscan_call &c, bool in_slot, int slot) {
                                     : 1);
         return slot < nout ? plane : 0;
     }
+    // value planes of the call's dtype, flag planes of its flag_dtype
+    const size_t v = n * dtype_bytes(c.dtype), f = n * dtype_bytes(c.flag_dtype);
     switch (c.kind) {
-    case RLSCAN_KIND_GAE_TYPED: {
-        const size_t v = n * dtype_bytes(c.dtype), f = n * dtype_bytes(c.flag_dtype);
+    case RLSCAN_KIND_GAE:
+    case RLSCAN_KIND_GAE_WITH_RETURNS:
+    case RLSCAN_KIND_GAE_TYPED:
+    case RLSCAN_KIND_LAMBDA_RETURNS: {
         const size_t by_slot[6] = {v, v, f, f, v, row};
         return slot < 6 ? by_slot[slot] : 0;
     }
-    case RLSCAN_KIND_GAE:
-    case RLSCAN_KIND_GAE_WITH_RETURNS:
-    case RLSCAN_KIND_LAMBDA_RETURNS: return slot < 5 ? plane : (slot == 5 ? row : 0);
     case RLSCAN_KIND_VTRACE:
-    case RLSCAN_KIND_GAE_VTRACE: return slot < 6 ? plane : (slot == 6 ? row : 0);
-    case RLSCAN_KIND_RETRACE: return (slot == 2 || slot == 3) ? plane * (size_t)(c.A > 0 ? c.A : 1) : (slot < 7 ? plane : 0);
-    case RLSCAN_KIND_DISCOUNTED_RETURNS: return slot < 4 ? plane : (slot == 4 ? row : 0);
+    case RLSCAN_KIND_GAE_VTRACE: {
+        const size_t by_slot[7] = {v, v, v, f, f, v, row};
+        return slot < 7 ? by_slot[slot] : 0;
+    }
+    case RLSCAN_KIND_RETRACE: {
+        const size_t A = (size_t)(c.A > 0 ? c.A : 1);
+        const size_t by_slot[7] = {v, v, v * A, v * A, v, f, f};
+        return slot < 7 ? by_slot[slot] : 0;
+    }
+    case RLSCAN_KIND_DISCOUNTED_RETURNS: {
+        const size_t by_slot[5] = {v, f, f, v, row};
+        return slot < 5 ? by_slot[slot] : 0;
+    }
     case RLSCAN_KIND_ELIGIBILITY_TRACES:
-    case RLSCAN_KIND_EPISODIC_PREFIX_SUM: return slot < 2 ? plane : 0;
+    case RLSCAN_KIND_EPISODIC_PREFIX_SUM: return slot == 0 ? v : (slot == 1 ? f : 0);
     default: return 0;
     }
 }
@@ -62,6 +73,25 @@ static size_t call_slot_bytes(const rlscan_call &c, bool in_slot, int slot) {
 static int call_dispatch(const rlscan_call &c, void *ws, size_t ws_bytes, cudaStream_t stream) {
     const float *const *in = reinterpret_cast<const float *const *>(c.in);
     float *const *out = reinterpret_cast<float *const *>(c.out);
+    if (call_is_typed(c)) { // reduced-byte inputs
+        switch (c.kind) {
+        case RLSCAN_KIND_GAE:
+        case RLSCAN_KIND_GAE_WITH_RETURNS:
+            return rlscan_gae_typed_ex(c.in[0], c.in[1], c.in[2], c.in[3], c.in[4], in[5], out[0],
+                                       c.kind == RLSCAN_KIND_GAE_WITH_RETURNS ? out[1] : nullptr, c.E, c.T, c.gamma,
+                                       c.lambda_, c.dtype, c.flag_dtype, c.options, ws, ws_bytes, stream);
+        case RLSCAN_KIND_VTRACE: return typed_vtrace(c, ws, ws_bytes, stream);
+        case RLSCAN_KIND_RETRACE: return typed_retrace(c, ws, ws_bytes, stream);
+        case RLSCAN_KIND_LAMBDA_RETURNS: return typed_lambda_returns(c, ws, ws_bytes, stream);
+        case RLSCAN_KIND_DISCOUNTED_RETURNS: return typed_discounted_returns(c, ws, ws_bytes, stream);
+        case RLSCAN_KIND_ELIGIBILITY_TRACES: return typed_eligibility_traces(c, ws, ws_bytes, stream);
+        case RLSCAN_KIND_EPISODIC_PREFIX_SUM: return typed_episodic_prefix_sum(c, ws, ws_bytes, stream);
+        case RLSCAN_KIND_GAE_TYPED: break; // its own entry point reads dtype and flag_dtype
+        case RLSCAN_KIND_GAE_VTRACE:
+            return fail(RLSCAN_ERR_UNSUPPORTED, "GAE_VTRACE takes fp32 inputs only (dtype and flag_dtype F32)");
+        default: return fail(RLSCAN_ERR_INVALID_ARG, "unknown kind %d", c.kind);
+        }
+    }
     switch (c.kind) {
     case RLSCAN_KIND_GAE:
         return rlscan_gae_ex(in[0], in[1], in[2], in[3], in[4], in[5], out[0], c.E, c.T, c.gamma, c.lambda_,

@@ -26,7 +26,7 @@ enum FusedBody {
     kBodyBackward = 0, // BackwardFamilyEst
     kBodyVtrace,       // VtraceEst
     kBodyRetrace1,     // RetraceEst
-    kBodyForward,      // TracesEst (ForwardF32Est)
+    kBodyForward,      // TracesEst (the fp32 prefix sum is the same estimator)
     kBodyPrefixI32,    // PrefixI32Est
     kNumFusedBodies
 };
@@ -137,7 +137,6 @@ template <> struct FusedBodyOf<ReturnsEst> { static constexpr int value = kBodyB
 template <> struct FusedBodyOf<VtraceEst> { static constexpr int value = kBodyVtrace; };
 template <> struct FusedBodyOf<RetraceEst> { static constexpr int value = kBodyRetrace1; };
 template <> struct FusedBodyOf<TracesEst> { static constexpr int value = kBodyForward; };
-template <> struct FusedBodyOf<PrefixF32Est> { static constexpr int value = kBodyForward; };
 template <> struct FusedBodyOf<PrefixI32Est> { static constexpr int value = kBodyPrefixI32; };
 
 inline BackwardFamilyEst::Params family_params(const GaeEst::Params &p) {
@@ -155,9 +154,6 @@ inline BackwardFamilyEst::Params family_params(const LambdaReturnsEst::Params &p
 inline BackwardFamilyEst::Params family_params(const ReturnsEst::Params &p) {
     return {p.rewards, nullptr, p.terminateds, p.truncateds, p.bootstrap_values, p.last_values,
             p.returns, nullptr, p.gamma, 1.0f, 0.0f, 0};
-}
-inline TracesEst::Params family_params(const PrefixF32Est::Params &p) {
-    return {p.x, p.dones, p.out, p.decay, p.reset_on_flag};
 }
 template <class P>
 inline const P &family_params(const P &p) { // estimators that are their own body

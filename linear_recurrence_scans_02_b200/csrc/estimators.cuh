@@ -33,24 +33,21 @@ __device__ __forceinline__ StepFlags step_flags(F te, F tr) {
     return f;
 }
 
-// L2 prefetch of one tile of up to six input planes, one plane per thread
-// (threads 0..5), before the kernel waits for the previous grid.
-__device__ __forceinline__ void prefetch_planes(const Geometry &g, long long tile0, int S, const void *p0,
-                                                const void *p1 = nullptr, const void *p2 = nullptr,
-                                                const void *p3 = nullptr, const void *p4 = nullptr,
-                                                const void *p5 = nullptr) {
+// L2 prefetch of one tile of the given input planes (each of its own
+// element type), one plane per thread (threads 0, 1, ...), before the kernel
+// waits for the previous grid.
+template <class... Ts>
+__device__ __forceinline__ void prefetch_planes(const Geometry &g, long long tile0, int S, const Ts *... planes) {
     const long long left = g.n - tile0;
     const long long cnt = left < S ? left : S;
-    switch (threadIdx.x) {
-    case 0: prefetch_l2(p0, tile0, cnt, 4); break;
-    case 1: prefetch_l2(p1, tile0, cnt, 4); break;
-    case 2: prefetch_l2(p2, tile0, cnt, 4); break;
-    case 3: prefetch_l2(p3, tile0, cnt, 4); break;
-    case 4: prefetch_l2(p4, tile0, cnt, 4); break;
-    case 5: prefetch_l2(p5, tile0, cnt, 4); break;
-    default: break;
-    }
+    int i = 0;
+    ((threadIdx.x == i++ ? prefetch_l2(planes, tile0, cnt, (int)sizeof(Ts)) : (void)0), ...);
 }
+
+// A flag register is set iff nonzero (fp32 flags stay floats, byte flags
+// integers).
+__device__ __forceinline__ bool flag_set(float f) { return f != 0.0f; }
+__device__ __forceinline__ bool flag_set(uint32_t f) { return f != 0u; }
 
 __device__ __forceinline__ float row_last_value(const float *__restrict__ lv, long long row, long long rows) {
     return load_one(lv, row, rows);
@@ -174,18 +171,23 @@ using GaeTypedEst = GaeEstT<true, ValT, FlagT>;
 // ---------------------------------------------------------------------------
 // TD(lambda): x = G,  a_t = gamma lambda, b_t = r_t + gamma (1 - lambda) V_{t+1}
 // ---------------------------------------------------------------------------
-struct LambdaReturnsEst {
+template <class ValT = float, class FlagT = float>
+struct LambdaReturnsEstT {
     static constexpr bool kBackward = true;
     using AT = float;
     using BT = float;
     struct Params {
-        const float *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        const ValT *rewards, *values;
+        const FlagT *terminateds, *truncateds;
+        const ValT *bootstrap_values;
+        const float *last_values;
         float *returns;
         float gamma, lambda_;
     };
     template <int V>
     struct State {
-        float r[V], v[V], te[V], tr[V], bv[V], out[V];
+        float r[V], v[V], bv[V], out[V];
+        FlagReg<FlagT> te[V], tr[V];
         float v_next;
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
@@ -193,18 +195,24 @@ struct LambdaReturnsEst {
     }
     static constexpr int kInputPlanes = 5;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[5] = {P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values};
-        return {i < 5 ? p[i] : nullptr, 4};
+        switch (i) {
+        case 0: return {P.rewards, (int)sizeof(ValT)};
+        case 1: return {P.values, (int)sizeof(ValT)};
+        case 2: return {P.terminateds, (int)sizeof(FlagT)};
+        case 3: return {P.truncateds, (int)sizeof(FlagT)};
+        case 4: return {P.bootstrap_values, (int)sizeof(ValT)};
+        default: return {nullptr, 0};
+        }
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
         const float h_v_next = pos.fetch_next(P.values);
-        pos.load(P.rewards, S.r);
-        pos.load(P.values, S.v);
-        pos.load(P.terminateds, S.te);
-        pos.load(P.truncateds, S.tr);
-        pos.load(P.bootstrap_values, S.bv);
+        pos.load_widen(P.rewards, S.r);
+        pos.load_widen(P.values, S.v);
+        pos.load_flag(P.terminateds, S.te);
+        pos.load_flag(P.truncateds, S.tr);
+        pos.load_widen(P.bootstrap_values, S.bv);
         S.v_next = pos.next(S.v, h_v_next);
     }
     template <int V, bool kTrunc, bool kFast, class Pos>
@@ -262,38 +270,49 @@ struct LambdaReturnsEst {
         pos.store(P.returns, S.out);
     }
 };
+using LambdaReturnsEst = LambdaReturnsEstT<>;
 
 // ---------------------------------------------------------------------------
 // Discounted returns: x = R,  a_t = gamma, b_t = r_t
 // ---------------------------------------------------------------------------
-struct ReturnsEst {
+template <class ValT = float, class FlagT = float>
+struct ReturnsEstT {
     static constexpr bool kBackward = true;
     using AT = float;
     using BT = float;
     struct Params {
-        const float *rewards, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        const ValT *rewards;
+        const FlagT *terminateds, *truncateds;
+        const ValT *bootstrap_values;
+        const float *last_values;
         float *returns;
         float gamma;
     };
     template <int V>
     struct State {
-        float r[V], te[V], tr[V], bv[V], out[V];
+        float r[V], bv[V], out[V];
+        FlagReg<FlagT> te[V], tr[V];
     };
     static __device__ __forceinline__ void prefetch(const Params &P, const Geometry &g, long long tile0, int S) {
         prefetch_planes(g, tile0, S, P.rewards, P.terminateds, P.truncateds, P.bootstrap_values);
     }
     static constexpr int kInputPlanes = 4;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[4] = {P.rewards, P.terminateds, P.truncateds, P.bootstrap_values};
-        return {i < 4 ? p[i] : nullptr, 4};
+        switch (i) {
+        case 0: return {P.rewards, (int)sizeof(ValT)};
+        case 1: return {P.terminateds, (int)sizeof(FlagT)};
+        case 2: return {P.truncateds, (int)sizeof(FlagT)};
+        case 3: return {P.bootstrap_values, (int)sizeof(ValT)};
+        default: return {nullptr, 0};
+        }
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
-        pos.load(P.rewards, S.r);
-        pos.load(P.terminateds, S.te);
-        pos.load(P.truncateds, S.tr);
-        pos.load(P.bootstrap_values, S.bv);
+        pos.load_widen(P.rewards, S.r);
+        pos.load_flag(P.terminateds, S.te);
+        pos.load_flag(P.truncateds, S.tr);
+        pos.load_widen(P.bootstrap_values, S.bv);
     }
     template <int V, bool kTrunc, bool kFast, class Pos>
     static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
@@ -341,23 +360,29 @@ struct ReturnsEst {
         pos.store(P.returns, S.out);
     }
 };
+using ReturnsEst = ReturnsEstT<>;
 
 // ---------------------------------------------------------------------------
 // V-Trace: x = D = vs - V,  a_t = gamma c_t, b_t = rho_t delta_t;
 // epilogue vs_t = V_t + D_t and pg_t = rho_t (r_t + gamma vs_{t+1} - V_t).
 // ---------------------------------------------------------------------------
-struct VtraceEst {
+template <class ValT = float, class FlagT = float>
+struct VtraceEstT {
     static constexpr bool kBackward = true;
     using AT = float;
     using BT = float;
     struct Params {
-        const float *log_rhos, *rewards, *values, *terminateds, *truncateds, *bootstrap_values, *last_values;
+        const ValT *log_rhos, *rewards, *values;
+        const FlagT *terminateds, *truncateds;
+        const ValT *bootstrap_values;
+        const float *last_values;
         float *vs, *pg_advantages;
         float gamma, lambda_, rho_bar, c_bar;
     };
     template <int V>
     struct State {
-        float lr[V], r[V], v[V], te[V], tr[V], bv[V];
+        float lr[V], r[V], v[V], bv[V];
+        FlagReg<FlagT> te[V], tr[V];
         float rho[V];
         float vs[V], pg[V];
         float v_next;
@@ -369,19 +394,26 @@ struct VtraceEst {
     }
     static constexpr int kInputPlanes = 6;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[6] = {P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values};
-        return {i < 6 ? p[i] : nullptr, 4};
+        switch (i) {
+        case 0: return {P.log_rhos, (int)sizeof(ValT)};
+        case 1: return {P.rewards, (int)sizeof(ValT)};
+        case 2: return {P.values, (int)sizeof(ValT)};
+        case 3: return {P.terminateds, (int)sizeof(FlagT)};
+        case 4: return {P.truncateds, (int)sizeof(FlagT)};
+        case 5: return {P.bootstrap_values, (int)sizeof(ValT)};
+        default: return {nullptr, 0};
+        }
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
         const float h_v_next = pos.fetch_next(P.values);
-        pos.load(P.log_rhos, S.lr);
-        pos.load(P.rewards, S.r);
-        pos.load(P.values, S.v);
-        pos.load(P.terminateds, S.te);
-        pos.load(P.truncateds, S.tr);
-        pos.load(P.bootstrap_values, S.bv);
+        pos.load_widen(P.log_rhos, S.lr);
+        pos.load_widen(P.rewards, S.r);
+        pos.load_widen(P.values, S.v);
+        pos.load_flag(P.terminateds, S.te);
+        pos.load_flag(P.truncateds, S.tr);
+        pos.load_widen(P.bootstrap_values, S.bv);
         S.v_next = pos.next(S.v, h_v_next);
     }
     template <int V, bool kTrunc, bool kFast, class Pos>
@@ -445,6 +477,7 @@ struct VtraceEst {
         pos.store(P.pg_advantages, S.pg);
     }
 };
+using VtraceEst = VtraceEstT<>;
 
 // ---------------------------------------------------------------------------
 // GAE (with the TD(lambda) returns G_t = A_t + V_t) and V-Trace from one pass
@@ -561,18 +594,25 @@ struct GaeVtraceEst {
 // the expected next-state value V'_t = next_q_values_all[t] (one action, or
 // the plane expected_value_kernel writes for several).
 // ---------------------------------------------------------------------------
-struct RetraceEst {
+// NqT: the element type of the V' plane (ValT for a single action; fp32 for
+// the plane expected_value_kernel writes for several).
+template <class ValT = float, class FlagT = float, class NqT = ValT>
+struct RetraceEstT {
     static constexpr bool kBackward = true;
     using AT = float;
     using BT = float;
     struct Params {
-        const float *rewards, *q_values, *next_q_values_all, *log_rhos, *terminateds, *truncateds;
+        const ValT *rewards, *q_values;
+        const NqT *next_q_values_all;
+        const ValT *log_rhos;
+        const FlagT *terminateds, *truncateds;
         float *q_ret;
         float gamma, lambda_, c_bar;
     };
     template <int V>
     struct State {
-        float r[V], q[V], vnext[V], lr[V], te[V], tr[V], out[V];
+        float r[V], q[V], vnext[V], lr[V], out[V];
+        FlagReg<FlagT> te[V], tr[V];
         float lr_next;
     };
 
@@ -582,20 +622,27 @@ struct RetraceEst {
     }
     static constexpr int kInputPlanes = 6;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const float *p[6] = {P.rewards, P.q_values, P.log_rhos, P.terminateds, P.truncateds, P.next_q_values_all};
-        return {i < 6 ? p[i] : nullptr, 4};
+        switch (i) {
+        case 0: return {P.rewards, (int)sizeof(ValT)};
+        case 1: return {P.q_values, (int)sizeof(ValT)};
+        case 2: return {P.log_rhos, (int)sizeof(ValT)};
+        case 3: return {P.terminateds, (int)sizeof(FlagT)};
+        case 4: return {P.truncateds, (int)sizeof(FlagT)};
+        case 5: return {P.next_q_values_all, (int)sizeof(NqT)};
+        default: return {nullptr, 0};
+        }
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
         const float h_lr_next = pos.fetch_next(P.log_rhos);
-        pos.load(P.rewards, S.r);
-        pos.load(P.q_values, S.q);
-        pos.load(P.log_rhos, S.lr);
-        pos.load(P.terminateds, S.te);
-        pos.load(P.truncateds, S.tr);
+        pos.load_widen(P.rewards, S.r);
+        pos.load_widen(P.q_values, S.q);
+        pos.load_widen(P.log_rhos, S.lr);
+        pos.load_flag(P.terminateds, S.te);
+        pos.load_flag(P.truncateds, S.tr);
         S.lr_next = pos.next(S.lr, h_lr_next);
-        pos.load(P.next_q_values_all, S.vnext);
+        pos.load_widen(P.next_q_values_all, S.vnext);
     }
     template <int V, bool kFast, class Pos>
     static __device__ __forceinline__ void coeffs_impl(const Params &P, const Geometry &g, const Pos &pos,
@@ -636,19 +683,21 @@ struct RetraceEst {
         pos.store(P.q_ret, S.out);
     }
 };
+using RetraceEst = RetraceEstT<>;
 
 // ---------------------------------------------------------------------------
 // Forward estimators.  Eligibility traces: x = e, a_t = gamma lambda,
-// b_t = x_t.  fp32 prefix sum: the same with a_t = 1 (kind tag only names
-// the kernel).
+// b_t = x_t.  fp32 prefix sum: the same with a_t = 1.  Flags are widened to
+// 0 / 1 floats (the halo flag comes from the neighbouring lane).
 // ---------------------------------------------------------------------------
-template <int kKind> // 0 = eligibility traces, 1 = fp32 episodic prefix sum
-struct ForwardF32Est {
+template <class ValT = float, class FlagT = float>
+struct ForwardEstT {
     static constexpr bool kBackward = false;
     using AT = float;
     using BT = float;
     struct Params {
-        const float *x, *dones;
+        const ValT *x;
+        const FlagT *dones;
         float *out;
         float decay;       // gamma lambda, or 1
         int reset_on_flag; // 0: dones[t-1] != 0 resets at t; 1: dones[t] != 0 resets at t
@@ -663,15 +712,18 @@ struct ForwardF32Est {
     }
     static constexpr int kInputPlanes = 2;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const void *p[2] = {P.x, P.dones};
-        return {i < 2 ? p[i] : nullptr, 4};
+        switch (i) {
+        case 0: return {P.x, (int)sizeof(ValT)};
+        case 1: return {P.dones, (int)sizeof(FlagT)};
+        default: return {nullptr, 0};
+        }
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
         const float h_d_prev = pos.fetch_prev(P.dones);
-        pos.load(P.x, S.x);
-        pos.load(P.dones, S.d);
+        pos.load_widen(P.x, S.x);
+        pos.load_widen(P.dones, S.d);
         S.d_prev = pos.prev(S.d, h_d_prev);
     }
     template <int V, bool kFast, class Pos>
@@ -706,19 +758,20 @@ struct ForwardF32Est {
         pos.store(P.out, S.out);
     }
 };
-using TracesEst = ForwardF32Est<0>;
-using PrefixF32Est = ForwardF32Est<1>;
+using TracesEst = ForwardEstT<>;
+using PrefixF32Est = TracesEst; // a trace with decay 1
 
 // int32 episodic prefix sum: a in {0, 1}, exact wrapping sums.
-struct PrefixI32Est {
+template <class FlagT = float>
+struct PrefixI32EstT {
     static constexpr bool kBackward = false;
     using AT = uint32_t;
     using BT = int32_t;
     struct Params {
         const int32_t *x;
-        const float *dones;
+        const FlagT *dones;
         int32_t *out;
-        int reset_on_flag; // as ForwardF32Est
+        int reset_on_flag; // as ForwardEstT
     };
     template <int V>
     struct State {
@@ -731,15 +784,18 @@ struct PrefixI32Est {
     }
     static constexpr int kInputPlanes = 2;
     static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
-        const void *p[2] = {P.x, P.dones};
-        return {i < 2 ? p[i] : nullptr, 4};
+        switch (i) {
+        case 0: return {P.x, 4};
+        case 1: return {P.dones, (int)sizeof(FlagT)};
+        default: return {nullptr, 0};
+        }
     }
     template <int NT, int V, class Pos>
     static __device__ __forceinline__ void load(const Params &P, const Geometry &g, const Pos &pos,
                                                 State<V> &S, unsigned char *) {
         const float h_d_prev = pos.fetch_prev(P.dones);
         pos.load(P.x, S.x);
-        pos.load(P.dones, S.d);
+        pos.load_widen(P.dones, S.d);
         S.d_prev = pos.prev(S.d, h_d_prev);
     }
     template <int V, bool kFast, class Pos>
@@ -774,5 +830,6 @@ struct PrefixI32Est {
         pos.store(P.out, S.out);
     }
 };
+using PrefixI32Est = PrefixI32EstT<>;
 
 } // namespace rlscan

@@ -10,63 +10,8 @@
 // allowed, so a kernel's prologue can overlap the tail of whatever ran
 // before it on that stream.  No kernel waits on another block: rows that
 // span tiles take two launches (aggregates, then the scan with carries).
-#include "host.cuh"
+#include "expect.cuh"
 
-namespace rlscan {
-
-// Expected next-state values of multi-action Retrace: out[i] = sum over a of
-// pi[i, a] q[i, a] (a = 0 .. A-1 in order) for the n elements of the
-// flattened [E, T] array, with q = next_q_values_all and pi =
-// next_target_probs, both [E, T, A].  A block stages its tile's rows of
-// both planes (contiguous) in shared memory with 16-byte loads (scalar loads
-// when `vec` is 0: a base not 16-byte aligned, or a tail not a whole number
-// of 16-byte words), then each thread sums one element's products and the
-// block writes its values coalesced.  Dynamic shared memory: 2 NT A floats.
-constexpr int kExpectNT = 256;
-
-__global__ void __launch_bounds__(kExpectNT) expected_value_kernel(const float *__restrict__ q,
-                                                                   const float *__restrict__ pi,
-                                                                   float *__restrict__ out, long long n, int A,
-                                                                   int vec) {
-    extern __shared__ __align__(16) float smem_f[];
-    float *sq = smem_f;
-    float *sp = smem_f + (size_t)kExpectNT * A;
-    const long long e0 = (long long)blockIdx.x * kExpectNT;
-    const int cnt = (int)((n - e0) < kExpectNT ? (n - e0) : kExpectNT);
-    const int total = cnt * A;
-    const float *gq = q + e0 * A;
-    const float *gp = pi + e0 * A;
-    if (threadIdx.x == 0) prefetch_l2(gq, 0, total, 4);
-    if (threadIdx.x == 1) prefetch_l2(gp, 0, total, 4);
-    griddep_wait();
-    griddep_launch_dependents();
-    if (vec && (total & 3) == 0) {
-        const float4 *q4 = reinterpret_cast<const float4 *>(gq);
-        const float4 *p4 = reinterpret_cast<const float4 *>(gp);
-#pragma unroll 4
-        for (int i = threadIdx.x; i < total / 4; i += kExpectNT) {
-            const float4 vq = __ldcg(q4 + i);
-            const float4 vp = __ldcg(p4 + i);
-            reinterpret_cast<float4 *>(sq)[i] = vq;
-            reinterpret_cast<float4 *>(sp)[i] = vp;
-        }
-    } else {
-        for (int i = threadIdx.x; i < total; i += kExpectNT) {
-            sq[i] = __ldcg(gq + i);
-            sp[i] = __ldcg(gp + i);
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < cnt) {
-        const float *qe = sq + (size_t)threadIdx.x * A;
-        const float *pe = sp + (size_t)threadIdx.x * A;
-        float s = 0.0f;
-        for (int act = 0; act < A; ++act) s = fmaf(pe[act], qe[act], s);
-        out[e0 + threadIdx.x] = s;
-    }
-}
-
-} // namespace rlscan
 
 using namespace rlscan;
 
@@ -123,25 +68,7 @@ int rlscan_retrace_ex(const float *rewards, const float *q_values, const float *
         const Plan plan = make_plan(E, T);
         if (plan.lookback && (ws == nullptr || ws_bytes < workspace_for(plan) || ((uintptr_t)ws & 15u) != 0))
             return run<RetraceEst>("rlscan_retrace", P, E, T, ws, ws_bytes, stream, vec);
-        const size_t smem = (size_t)2 * kExpectNT * (size_t)A * sizeof(float);
-        cudaError_t e = cudaSuccess;
-        if (smem > 48 * 1024)
-            e = cudaFuncSetAttribute(expected_value_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3((unsigned)ceil_div(E * T, kExpectNT));
-            cfg.blockDim = dim3(kExpectNT);
-            cfg.dynamicSmemBytes = smem;
-            cfg.stream = stream;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[0].val.programmaticStreamSerializationAllowed = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = pdl_enabled() ? 1 : 0;
-            e = cudaLaunchKernelEx(&cfg, expected_value_kernel, next_q_values_all, next_target_probs, q_ret,
-                                   (long long)(E * T), (int)A,
-                                   aligned16({next_q_values_all, next_target_probs}) ? 1 : 0);
-        }
+        const cudaError_t e = launch_expected_values(next_q_values_all, next_target_probs, q_ret, E * T, A, stream);
         if (e != cudaSuccess)
             return fail(RLSCAN_ERR_CUDA, "rlscan_retrace: expected-value launch failed: %s", cudaGetErrorString(e));
     }

@@ -296,8 +296,19 @@ def _reduced_bytes(*tensors):
     return any(t is not None and t.dtype != torch.float32 for t in tensors)
 
 
+def _one_call(ws, **call):
+    """A call with reduced-byte inputs: one rlscan_batch request holding it
+    (rlscan_call's dtype and flag_dtype carry the element types)."""
+    rlscan_batch([call], ws)
+
+
 def rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values,
                   vs, pg_advantages, gamma, lambda_=1.0, rho_bar=1.0, c_bar=1.0, ws=None, *, time_major=False):
+    if _reduced_bytes(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values):
+        return _one_call(ws, kind="vtrace", log_rhos=log_rhos, rewards=rewards, values=values,
+                         terminateds=terminateds, truncateds=truncateds, bootstrap_values=bootstrap_values,
+                         last_values=last_values, vs=vs, pg_advantages=pg_advantages, gamma=gamma, lambda_=lambda_,
+                         rho_bar=rho_bar, c_bar=c_bar, time_major=time_major)
     E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
     wp, wn, s = _ws_for(dev, E, T, ws, opts)
@@ -332,6 +343,11 @@ def rlscan_gae_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootst
 
 def rlscan_retrace(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds,
                    truncateds, q_ret, gamma, lambda_, c_bar=1.0, ws=None, *, time_major=False):
+    if _reduced_bytes(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds, truncateds):
+        return _one_call(ws, kind="retrace", rewards=rewards, q_values=q_values,
+                         next_q_values_all=next_q_values_all, next_target_probs=next_target_probs,
+                         log_rhos=log_rhos, terminateds=terminateds, truncateds=truncateds, q_ret=q_ret,
+                         gamma=gamma, lambda_=lambda_, c_bar=c_bar, time_major=time_major)
     E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
     if next_q_values_all.dim() == 2:
@@ -351,6 +367,10 @@ def rlscan_retrace(rewards, q_values, next_q_values_all, next_target_probs, log_
 
 def rlscan_lambda_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, returns,
                           gamma, lambda_, ws=None, *, time_major=False):
+    if _reduced_bytes(rewards, values, terminateds, truncateds, bootstrap_values):
+        return _one_call(ws, kind="lambda_returns", rewards=rewards, values=values, terminateds=terminateds,
+                         truncateds=truncateds, bootstrap_values=bootstrap_values, last_values=last_values,
+                         returns=returns, gamma=gamma, lambda_=lambda_, time_major=time_major)
     E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
     wp, wn, s = _ws_for(dev, E, T, ws, opts)
@@ -364,6 +384,10 @@ def rlscan_lambda_returns(rewards, values, terminateds, truncateds, bootstrap_va
 
 def rlscan_discounted_returns(rewards, terminateds, truncateds, bootstrap_values, last_values, returns,
                               gamma, ws=None, *, time_major=False):
+    if _reduced_bytes(rewards, terminateds, truncateds, bootstrap_values):
+        return _one_call(ws, kind="discounted_returns", rewards=rewards, terminateds=terminateds,
+                         truncateds=truncateds, bootstrap_values=bootstrap_values, last_values=last_values,
+                         returns=returns, gamma=gamma, time_major=time_major)
     E, T, sh, opts = _layout(rewards, "rewards", time_major)
     dev = rewards.device
     wp, wn, s = _ws_for(dev, E, T, ws, opts)
@@ -377,6 +401,9 @@ def rlscan_discounted_returns(rewards, terminateds, truncateds, bootstrap_values
 
 def rlscan_eligibility_traces(x, dones, traces, gamma, lambda_, ws=None, *, time_major=False,
                               done_starts_episode=False):
+    if _reduced_bytes(x, dones):
+        return _one_call(ws, kind="eligibility_traces", x=x, dones=dones, traces=traces, gamma=gamma,
+                         lambda_=lambda_, time_major=time_major, done_starts_episode=done_starts_episode)
     E, T, sh, opts = _layout(x, "x", time_major)
     if done_starts_episode:
         opts |= RLSCAN_OPT_DONE_STARTS_EPISODE
@@ -388,6 +415,9 @@ def rlscan_eligibility_traces(x, dones, traces, gamma, lambda_, ws=None, *, time
 
 
 def rlscan_episodic_prefix_sum(x, dones, out, ws=None, *, time_major=False, done_starts_episode=False):
+    if x.dtype in (torch.bfloat16, torch.float16) or _reduced_bytes(dones):
+        return _one_call(ws, kind="episodic_prefix_sum", x=x, dones=dones, out=out, time_major=time_major,
+                         done_starts_episode=done_starts_episode)
     E, T, sh, opts = _layout(x, "x", time_major)
     if done_starts_episode:
         opts |= RLSCAN_OPT_DONE_STARTS_EPISODE
@@ -424,6 +454,9 @@ _BATCH_KINDS = {
     "gae_vtrace": (10, ("log_rhos",) + _BACKWARD_IN, ("advantages", "returns", "vs", "pg_advantages")),
 }
 _BATCH_SCALARS = {"gamma": 0.99, "lambda_": 0.95, "rho_bar": 1.0, "c_bar": 1.0, "vtrace_lambda": 1.0}
+_FLAG_SLOTS = {"terminateds", "truncateds", "dones"}
+_PREFIX_DTYPES = {torch.float32: RLSCAN_F32, torch.int32: RLSCAN_I32, torch.bfloat16: RLSCAN_BF16,
+                  torch.float16: RLSCAN_F16}
 
 
 def rlscan_batch(calls, ws=None):
@@ -457,32 +490,34 @@ def rlscan_batch(calls, ws=None):
         c.kind, c.options, c.E, c.T, c.A = code, opts, E, T, 1
         for k, v in _BATCH_SCALARS.items():
             setattr(c, k, float(call.get(k, 1.0 if (kind == "vtrace" and k == "lambda_") else v)))
-        dtypes = (torch.float32,)
-        slot_dtypes = {}
+        # element types from the tensors: the value planes share one dtype
+        # (float32, bfloat16, float16; int32 x for the prefix sum), the flag
+        # planes one (float32, uint8, bool); outputs are float32 (int32 for
+        # an int32 prefix sum)
+        vals = [call[k] for k in in_names if k not in _FLAG_SLOTS and k != "last_values"
+                and call.get(k) is not None]
+        flags = [call[k] for k in in_names if k in _FLAG_SLOTS and call.get(k) is not None]
+        vt = vals[0].dtype if vals else torch.float32
+        ft = flags[0].dtype if flags else torch.float32
         if kind == "episodic_prefix_sum":
-            dtypes = (torch.float32, torch.int32)
-            c.dtype = RLSCAN_F32 if first.dtype == torch.float32 else RLSCAN_I32
-        if kind == "gae_typed":  # value and flag dtypes from the tensors, as rlscan_gae_typed
-            c.dtype = _VALUE_DTYPES.get(first.dtype, -1)
-            flags = [call[k] for k in ("terminateds", "truncateds") if call.get(k) is not None]
-            c.flag_dtype = _FLAG_DTYPES.get(flags[0].dtype, -1) if flags else RLSCAN_F32
-            if c.dtype < 0 or c.flag_dtype < 0:
-                raise TypeError("gae_typed: unsupported value or flag dtype")
-            for k in ("rewards", "values", "bootstrap_values"):
-                slot_dtypes[k] = (first.dtype,)
-            for k in ("terminateds", "truncateds"):
-                slot_dtypes[k] = (flags[0].dtype,) if flags else (torch.float32,)
+            c.dtype = _PREFIX_DTYPES.get(vt, -1)
+        else:
+            c.dtype = _VALUE_DTYPES.get(vt, -1)
+        c.flag_dtype = _FLAG_DTYPES.get(ft, -1)
+        if c.dtype < 0 or c.flag_dtype < 0:
+            raise TypeError(f"{kind}: unsupported value dtype {vt} or flag dtype {ft}")
+        slot_dtypes = {k: ((ft,) if k in _FLAG_SLOTS else ((torch.float32,) if k == "last_values" else (vt,)))
+                       for k in in_names}
+        out_dtype = (torch.int32,) if vt == torch.int32 else (torch.float32,)
         if kind == "retrace" and call["next_q_values_all"].dim() == 3:
             c.A = int(call["next_q_values_all"].shape[2])
         for i, name in enumerate(in_names):
             shape = (E,) if name == "last_values" else (sh + (c.A,) if name in ("next_q_values_all",
                                                                                "next_target_probs") and c.A > 1
                                                          else sh)
-            dt = slot_dtypes.get(name, dtypes if name == "x" else (torch.float32,))
-            c.inp[i] = _ptr(call.get(name), name, shape, dt, dev)
+            c.inp[i] = _ptr(call.get(name), name, shape, slot_dtypes[name], dev)
         for i, name in enumerate(out_names):
-            dt = dtypes if name == "out" else (torch.float32,)
-            c.out[i] = _ptr(call.get(name), name, sh, dt, dev)
+            c.out[i] = _ptr(call.get(name), name, sh, out_dtype, dev)
         if not tm:
             ws_need = max(ws_need, int(_lib.rlscan_workspace_bytes(E, T)))
     if not calls:
@@ -498,6 +533,10 @@ def rlscan_batch(calls, ws=None):
 # ---------------------------------------------------------------------------
 # compute_* : allocate outputs, call the above (README "Kernels" names)
 # ---------------------------------------------------------------------------
+
+def _f32_like(t):
+    return torch.empty(t.shape, dtype=torch.float32, device=t.device)
+
 
 def compute_gae(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
                 bootstrap_values=None, last_values=None, time_major=False):
@@ -541,8 +580,8 @@ def compute_gae_vtrace(log_rhos, rewards, values, terminateds, gamma=0.99, lambd
 
 def compute_vtrace(log_rhos, rewards, values, terminateds, gamma=0.99, lambda_=1.0, rho_bar=1.0, c_bar=1.0, *,
                    truncateds=None, bootstrap_values=None, last_values=None, time_major=False):
-    vs = torch.empty_like(rewards)
-    pg = torch.empty_like(rewards)
+    vs = _f32_like(rewards)
+    pg = _f32_like(rewards)
     rlscan_vtrace(log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, last_values, vs, pg,
                   gamma, lambda_, rho_bar, c_bar, time_major=time_major)
     return vs, pg
@@ -550,7 +589,7 @@ def compute_vtrace(log_rhos, rewards, values, terminateds, gamma=0.99, lambda_=1
 
 def compute_retrace(rewards, q_values, next_q_values_all, log_rhos, terminateds, truncateds, gamma=0.99,
                     lambda_=0.95, c_bar=1.0, *, next_target_probs=None, time_major=False):
-    q_ret = torch.empty_like(rewards)
+    q_ret = _f32_like(rewards)
     rlscan_retrace(rewards, q_values, next_q_values_all, next_target_probs, log_rhos, terminateds, truncateds,
                    q_ret, gamma, lambda_, c_bar, time_major=time_major)
     return q_ret
@@ -558,7 +597,7 @@ def compute_retrace(rewards, q_values, next_q_values_all, log_rhos, terminateds,
 
 def compute_lambda_returns(rewards, values, terminateds, gamma=0.99, lambda_=0.95, *, truncateds=None,
                            bootstrap_values=None, last_values=None, time_major=False):
-    ret = torch.empty_like(rewards)
+    ret = _f32_like(rewards)
     rlscan_lambda_returns(rewards, values, terminateds, truncateds, bootstrap_values, last_values, ret, gamma,
                           lambda_, time_major=time_major)
     return ret
@@ -566,7 +605,7 @@ def compute_lambda_returns(rewards, values, terminateds, gamma=0.99, lambda_=0.9
 
 def compute_discounted_returns(rewards, terminateds=None, gamma=0.99, *, truncateds=None, bootstrap_values=None,
                                last_values=None, time_major=False):
-    ret = torch.empty_like(rewards)
+    ret = _f32_like(rewards)
     rlscan_discounted_returns(rewards, terminateds, truncateds, bootstrap_values, last_values, ret, gamma,
                               time_major=time_major)
     return ret
@@ -574,13 +613,13 @@ def compute_discounted_returns(rewards, terminateds=None, gamma=0.99, *, truncat
 
 def compute_eligibility_traces(x, dones=None, gamma=0.99, lambda_=0.95, *, time_major=False,
                                done_starts_episode=False):
-    out = torch.empty_like(x)
+    out = _f32_like(x)
     rlscan_eligibility_traces(x, dones, out, gamma, lambda_, time_major=time_major,
                               done_starts_episode=done_starts_episode)
     return out
 
 
 def compute_episodic_prefix_sum(x, dones=None, *, time_major=False, done_starts_episode=False):
-    out = torch.empty_like(x)
+    out = torch.empty_like(x) if x.dtype == torch.int32 else _f32_like(x)
     rlscan_episodic_prefix_sum(x, dones, out, time_major=time_major, done_starts_episode=done_starts_episode)
     return out

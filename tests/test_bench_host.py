@@ -29,14 +29,17 @@ def test_clock_summary(tmp_path):
     assert bench.summarize_clocks(None)["reasons"] == ["unsampled"]
 
 
-def test_traffic_table_only_for_matching_kernel_source(tmp_path, monkeypatch):
+def test_traffic_record_only_for_matching_kernel_source(tmp_path, monkeypatch):
+    import json
     sha = bench.kernel_source_sha()
-    prof = tmp_path / "profiles"
-    prof.mkdir()
-    (prof / "dram_traffic.md").write_text(f"| estimator | bytes | sha |\n|---|---|---|\n| gae | 123 | {sha} |\n"
-                                          f"| vtrace | 456 | 0000000000000000 |\n")
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: sha)
+    path = tmp_path / "dram_traffic.json"
+    path.write_text(json.dumps({"kernel_sha": sha, "launches": {
+        "gae": {"dram_read_bytes": 100, "dram_write_bytes": 23}}}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
     assert bench.recorded_traffic("gae") == 123
-    assert bench.recorded_traffic("vtrace") is None  # captured from another kernel source
     assert bench.recorded_traffic("retrace") is None
+    path.write_text(json.dumps({"kernel_sha": "0000000000000000", "launches": {
+        "gae": {"dram_read_bytes": 100, "dram_write_bytes": 23}}}))
+    assert bench.recorded_traffic("gae") is None  # captured from another kernel source
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.recorded_traffic("gae") is None

@@ -21,7 +21,7 @@ from gpu_common import assert_close, assert_equal_int, check, dev, run_gae, run_
 from linear_recurrence_scans_02_b200 import rlscan as R
 from linear_recurrence_scans_02_b200 import workloads as W
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 G, L = 0.99, 0.95
 
 
