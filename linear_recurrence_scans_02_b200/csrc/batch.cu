@@ -131,9 +131,11 @@ static int call_dispatch(const rlscan_call &c, void *ws, size_t ws_bytes, cudaSt
 // Elements per thread of a fused launch: 4 when it mixes three or more tile
 // bodies and every row fits a 512-element tile, else 8 (measured at 4096 x
 // 128: the eight estimators of one step 16.1 us at 4 against 17.6 us at 8;
-// eight GAE calls 11.0 us either way).  Then the items are ordered by body
-// (blocks of one body then share each SM's instruction caches), and each
-// item is tiled.
+// eight GAE calls 11.0 us either way).  The items arrive ordered by body
+// (blocks of one body then share each SM's instruction caches); each is
+// tiled.
+constexpr int kMaxBodiesPerLaunch = kNumFusedBodies; // every fused call in one launch
+
 static int fused_layout(FusedBatch &fb, long long *tiles) {
     unsigned bodies = 0u;
     bool fit4 = true;
@@ -142,7 +144,6 @@ static int fused_layout(FusedBatch &fb, long long *tiles) {
         if ((long long)(kFusedNT * 4) % fb.item[i].g.seq_len != 0) fit4 = false;
     }
     const int V = (__builtin_popcount(bodies) >= 3 && fit4) ? 4 : 8;
-    std::stable_sort(fb.item, fb.item + fb.n, [](const FusedItem &x, const FusedItem &y) { return x.kind < y.kind; });
     long long begin = 0;
     for (int i = 0; i < fb.n; ++i) {
         FusedItem &it = fb.item[i];
@@ -208,19 +209,38 @@ int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes
     st.pass = kBatchRecord;
     RLSCAN_TRY(batch_pass(st, calls, ncalls, ws, ws_bytes, stream));
     if (st.fb.n == 0) return ok();
-    const int V = fused_layout(st.fb, &st.tiles);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)st.tiles);
-    cfg.blockDim = dim3(kFusedNT);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    const cudaError_t e = V == 4 ? cudaLaunchKernelEx(&cfg, fused_tile_kernel<4>, st.fb)
-                                 : cudaLaunchKernelEx(&cfg, fused_tile_kernel<8>, st.fb);
-    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "rlscan_batch: fused launch failed: %s", cudaGetErrorString(e));
+    // the recorded calls ordered by body, then cut into launches of at most
+    // kMaxBodiesPerLaunch bodies each (consecutive launches overlap through
+    // programmatic dependent launch)
+    std::stable_sort(st.fb.item, st.fb.item + st.fb.n,
+                     [](const FusedItem &x, const FusedItem &y) { return x.kind < y.kind; });
+    for (int first = 0; first < st.fb.n;) {
+        int last = first, bodies = 1;
+        while (last + 1 < st.fb.n &&
+               (st.fb.item[last + 1].kind == st.fb.item[last].kind || bodies < kMaxBodiesPerLaunch)) {
+            if (st.fb.item[last + 1].kind != st.fb.item[last].kind) ++bodies;
+            ++last;
+        }
+        FusedBatch part{};
+        part.n = last - first + 1;
+        std::copy(st.fb.item + first, st.fb.item + last + 1, part.item);
+        long long tiles = 0;
+        const int V = fused_layout(part, &tiles);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)tiles);
+        cfg.blockDim = dim3(kFusedNT);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl_enabled() ? 1 : 0;
+        const cudaError_t e = V == 4 ? cudaLaunchKernelEx(&cfg, fused_tile_kernel<4>, part)
+                                     : cudaLaunchKernelEx(&cfg, fused_tile_kernel<8>, part);
+        if (e != cudaSuccess)
+            return fail(RLSCAN_ERR_CUDA, "rlscan_batch: fused launch failed: %s", cudaGetErrorString(e));
+        first = last + 1;
+    }
     return ok();
 }
 

@@ -335,13 +335,20 @@ __device__ __forceinline__ void read_slot(const TileSlot *slot, float2 &a, float
 }
 
 // Carry into scan-order tile j from the aggregates of tiles k_min .. j-1,
-// called by all 32 lanes of one warp.  Lane i reads tile base - i of each
-// window of 32 (nearest first); a tile with a published inclusive value, or
-// whose aggregate cuts the chain (a == 0), ends the walk.  Lane 0 publishes
-// this tile's inclusive value.
+// called by all 32 lanes of one warp.  Each window covers 32 x kSlotsPerLane
+// tiles, nearest first: lane i reads tiles base - i M - m, m = 0 .. M-1,
+// all M loads in flight at once, and composes them nearest-outermost up to
+// the first that ends the walk (a published inclusive value, or an
+// aggregate that cuts the chain, a == 0); the lanes' maps are then composed
+// in order.  A row of up to 32 M tiles thus costs one round trip even when
+// none of its tiles has published an inclusive value yet.  Lane 0
+// publishes this tile's inclusive value.
+constexpr int kSlotsPerLane = 4;
+
 template <class AT, class BT>
 __device__ BT carry_from_aggregates(const Lookback &lb, long long j, long long k_min, bool needs_carry, AT ta,
                                     BT tb, int lane) {
+    constexpr int M = kSlotsPerLane;
     TileSlot *me = lb.slots + j;
     if (!needs_carry) {
         if (lane == 0) publish_inclusive(me, tb);
@@ -350,17 +357,31 @@ __device__ BT carry_from_aggregates(const Lookback &lb, long long j, long long k
     AT acc_a = identity_a(ta);
     BT acc_b = identity_b(tb);
     BT carry = identity_b(tb);
-    for (long long base = j - 1;; base -= 32) {
-        const long long k = base - lane;
-        AT la = ta;
-        BT lb_ = tb;
-        if (k < k_min) { // nothing flows in from before the row / array
-            la = cut_a(ta);
-            lb_ = identity_b(tb);
-        } else {
-            read_slot(lb.slots + k, la, lb_);
+    for (long long base = j - 1;; base -= 32 * M) {
+        const long long k0 = base - (long long)lane * M;
+        AT sa[M];
+        BT sb[M];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            sa[m] = ta;
+            sb[m] = tb;
+            if (k0 - m < k_min) { // nothing flows in from before the row / array
+                sa[m] = cut_a(ta);
+                sb[m] = identity_b(tb);
+            } else {
+                read_slot(lb.slots + (k0 - m), sa[m], sb[m]);
+            }
         }
-        const bool stop = is_cut(la);
+        AT la = identity_a(ta);
+        BT lb_ = identity_b(tb);
+        bool stop = false;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            if (!stop) {
+                combine(la, lb_, sa[m], sb[m]);
+                stop = is_cut(sa[m]);
+            }
+        }
         const unsigned stops = __ballot_sync(kFullMask, stop);
         const int last = stops ? __ffs(stops) - 1 : 31;
         if (lane > last) { // farther than the nearest stop: contributes nothing
