@@ -58,9 +58,25 @@ inline bool pdl_enabled() {
 // Eight elements per thread keeps a grid's share of each SM small, so the
 // next launch on the stream can be resident (and prefetching) while this one
 // runs; the 512-element tile (four per thread) is for small split-row plans.
-enum Cfg { C512 = 0, C1024, C2048, C4096, kNumCfg };
-constexpr int kCfgTile[kNumCfg] = {512, 1024, 2048, 4096};
-constexpr int kCfgThreads[kNumCfg] = {128, 128, 256, 512};
+// N512 .. N4096 are the same tiles at 16 elements per thread (half the
+// threads), for calls whose value planes are 2 bytes wide: each thread then
+// keeps as many bytes in flight as an fp32 thread of the twin tile.
+enum Cfg { C512 = 0, C1024, C2048, C4096, N512, N1024, N2048, N4096, kNumCfg };
+constexpr int kCfgTile[kNumCfg] = {512, 1024, 2048, 4096, 512, 1024, 2048, 4096};
+constexpr int kCfgThreads[kNumCfg] = {128, 128, 256, 512, 32, 64, 128, 256};
+
+// Whether an estimator reads 2-byte value planes (takes the N configs).
+template <class Est>
+struct NarrowOf {
+    static constexpr bool value = false;
+};
+template <bool R, class V, class F> struct NarrowOf<GaeEstT<R, V, F>> { static constexpr bool value = sizeof(V) == 2; };
+template <class V, class F> struct NarrowOf<VtraceEstT<V, F>> { static constexpr bool value = sizeof(V) == 2; };
+template <class V, class F> struct NarrowOf<LambdaReturnsEstT<V, F>> { static constexpr bool value = sizeof(V) == 2; };
+template <class V, class F> struct NarrowOf<ReturnsEstT<V, F>> { static constexpr bool value = sizeof(V) == 2; };
+template <class V, class F, class N> struct NarrowOf<RetraceEstT<V, F, N>> { static constexpr bool value = sizeof(V) == 2; };
+template <class V, class F> struct NarrowOf<ForwardEstT<V, F>> { static constexpr bool value = sizeof(V) == 2; };
+constexpr Cfg narrow_twin(Cfg c) { return c <= C4096 ? (Cfg)(c + N512) : c; }
 
 struct Plan {
     Cfg cfg;
@@ -150,6 +166,15 @@ inline Plan make_plan_tiles(long long E, long long T) {
 }
 
 inline Plan make_plan(long long E, long long T) { return with_mode(make_plan_tiles(E, T), T); }
+
+// The plan an estimator runs: narrow-value estimators take the twin of the
+// plan's tile at 16 elements per thread (same tiles, same workspace).
+template <class Est>
+inline Plan make_plan_for(long long E, long long T) {
+    Plan p = make_plan_tiles(E, T);
+    if constexpr (NarrowOf<Est>::value) p.cfg = narrow_twin(p.cfg);
+    return with_mode(p, T);
+}
 
 // Warp-local mode: a row spans T / V lanes (T a power of two dividing 32 V);
 // the shuffle scan needs to reach that far only.
@@ -277,7 +302,7 @@ cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, const L
     case kModeReduce:
     case kModeCarry:
         // split-row plans use 512- to 2048-element tiles (make_plan_tiles)
-        if constexpr (C == C512 || C == C1024 || C == C2048) {
+        if constexpr (C == C512 || C == C1024 || C == C2048 || C == N512 || C == N1024 || C == N2048) {
             if (mode == kModeReduce) return launch_one<Est, NT, V, kModeReduce>(P, g, lb, smem, s, grid);
             return launch_one<Est, NT, V, kModeCarry>(P, g, lb, smem, s, grid);
         }
@@ -303,11 +328,20 @@ int run_two_pass(const char *name, const typename Est::Params &P, const Geometry
         const long long cnt = std::min<long long>(wave, g.ntiles - t0);
         for (int mode : {kModeReduce, kModeCarry}) {
             cudaError_t e;
-            switch (cfg) {
-            case C512: e = launch_cfg<Est, C512>(P, g, lb, mode, 0, stream, cnt); break;
-            case C1024: e = launch_cfg<Est, C1024>(P, g, lb, mode, 0, stream, cnt); break;
-            case C2048: e = launch_cfg<Est, C2048>(P, g, lb, mode, 0, stream, cnt); break;
-            default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+            if constexpr (NarrowOf<Est>::value) {
+                switch (cfg) {
+                case N512: e = launch_cfg<Est, N512>(P, g, lb, mode, 0, stream, cnt); break;
+                case N1024: e = launch_cfg<Est, N1024>(P, g, lb, mode, 0, stream, cnt); break;
+                case N2048: e = launch_cfg<Est, N2048>(P, g, lb, mode, 0, stream, cnt); break;
+                default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+                }
+            } else {
+                switch (cfg) {
+                case C512: e = launch_cfg<Est, C512>(P, g, lb, mode, 0, stream, cnt); break;
+                case C1024: e = launch_cfg<Est, C1024>(P, g, lb, mode, 0, stream, cnt); break;
+                case C2048: e = launch_cfg<Est, C2048>(P, g, lb, mode, 0, stream, cnt); break;
+                default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+                }
             }
             if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
         }
@@ -318,7 +352,7 @@ int run_two_pass(const char *name, const typename Est::Params &P, const Geometry
 template <class Est>
 int run(const char *name, const typename Est::Params &P, long long E, long long T, void *ws, size_t ws_bytes,
         cudaStream_t stream, bool vec_ok) {
-    const Plan plan = make_plan(E, T);
+    const Plan plan = make_plan_for<Est>(E, T);
     Geometry g;
     g.n = E * T;
     g.seq_len = T;
@@ -355,12 +389,22 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
     }
     if (plan.lookback) return run_two_pass<Est>(name, P, g, lb, plan.cfg, stream);
     cudaError_t e;
-    switch (plan.cfg) {
-    case C512: e = launch_cfg<Est, C512>(P, g, lb, plan.mode, 0, stream); break;
-    case C1024: e = launch_cfg<Est, C1024>(P, g, lb, plan.mode, 0, stream); break;
-    case C2048: e = launch_cfg<Est, C2048>(P, g, lb, plan.mode, 0, stream); break;
-    case C4096: e = launch_cfg<Est, C4096>(P, g, lb, plan.mode, 0, stream); break;
-    default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+    if constexpr (NarrowOf<Est>::value) {
+        switch (plan.cfg) {
+        case N512: e = launch_cfg<Est, N512>(P, g, lb, plan.mode, 0, stream); break;
+        case N1024: e = launch_cfg<Est, N1024>(P, g, lb, plan.mode, 0, stream); break;
+        case N2048: e = launch_cfg<Est, N2048>(P, g, lb, plan.mode, 0, stream); break;
+        case N4096: e = launch_cfg<Est, N4096>(P, g, lb, plan.mode, 0, stream); break;
+        default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+        }
+    } else {
+        switch (plan.cfg) {
+        case C512: e = launch_cfg<Est, C512>(P, g, lb, plan.mode, 0, stream); break;
+        case C1024: e = launch_cfg<Est, C1024>(P, g, lb, plan.mode, 0, stream); break;
+        case C2048: e = launch_cfg<Est, C2048>(P, g, lb, plan.mode, 0, stream); break;
+        case C4096: e = launch_cfg<Est, C4096>(P, g, lb, plan.mode, 0, stream); break;
+        default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
+        }
     }
     if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
     return ok();

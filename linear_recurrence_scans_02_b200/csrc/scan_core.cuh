@@ -498,14 +498,19 @@ __device__ __forceinline__ void load_plane_widen(const T *__restrict__ p, long l
         constexpr int kBytes = V * (int)sizeof(T);
         if (vec) {
             uint32_t w[kBytes / 4 > 0 ? kBytes / 4 : 1];
-            if constexpr (kBytes == 16) {
+            if constexpr (kBytes == 32) {
+                const uint4 v0 = __ldcg(reinterpret_cast<const uint4 *>(q + i0));
+                const uint4 v1 = __ldcg(reinterpret_cast<const uint4 *>(q + i0) + 1);
+                w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+                w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+            } else if constexpr (kBytes == 16) {
                 const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(q + i0));
                 w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
             } else if constexpr (kBytes == 8) {
                 const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(q + i0));
                 w[0] = v.x; w[1] = v.y;
             } else {
-                static_assert(kBytes == 4, "V * sizeof(T) must be 4, 8 or 16 bytes");
+                static_assert(kBytes == 4, "V * sizeof(T) must be 4, 8, 16 or 32 bytes");
                 w[0] = __ldcg(reinterpret_cast<const unsigned int *>(q + i0));
             }
 #pragma unroll
@@ -548,11 +553,14 @@ __device__ __forceinline__ void load_flags(const T *__restrict__ p, long long i0
         }
         if (vec) {
             uint32_t w[V / 4];
-            if constexpr (V == 8) {
+            if constexpr (V == 16) {
+                const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(p + i0));
+                w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+            } else if constexpr (V == 8) {
                 const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(p + i0));
                 w[0] = v.x; w[1] = v.y;
             } else {
-                static_assert(V == 4, "V must be 4 or 8");
+                static_assert(V == 4, "V must be 4, 8 or 16");
                 w[0] = __ldcg(reinterpret_cast<const unsigned int *>(p + i0));
             }
 #pragma unroll

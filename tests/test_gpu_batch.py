@@ -353,3 +353,38 @@ def test_batch_with_reduced_byte_gae():
     rvs, _ = oracle.vtrace(v["log_rhos"], v["rewards"], v["values"], v["terminateds"], g32, np.float32(1.0),
                            np.float32(1.0), np.float32(1.0))
     assert_close(vt["vs"], rvs, 1e-4, "vtrace beside typed gae")
+
+
+def test_batch_time_major_reduced_byte_calls():
+    # reduced-byte calls on the time-major layout inside one request: typed
+    # GAE (bf16 / uint8) and V-Trace (fp16 / bool), beside an fp32 call
+    E, T = 300, 96
+    d = W.vtrace_inputs(E, T, seed=61, p_term=0.02, p_trunc=0.02, last_values=True)
+    tm = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a.T)).cuda().to(dt)
+    wide_t = lambda t: t.to(torch.float32).t().contiguous().cpu().numpy()
+    nan_tm = lambda: torch.full((T, E), float("nan"), device="cuda")
+    lv = dev(d["last_values"])
+    g = dict(kind="gae_typed", rewards=tm(d["rewards"], torch.bfloat16), values=tm(d["values"], torch.bfloat16),
+             terminateds=tm(d["terminateds"], torch.uint8), truncateds=tm(d["truncateds"], torch.uint8),
+             bootstrap_values=tm(d["bootstrap_values"], torch.bfloat16), last_values=lv, advantages=nan_tm(),
+             returns=nan_tm(), gamma=G, lambda_=L, time_major=True)
+    v = dict(kind="vtrace", log_rhos=tm(d["log_rhos"], torch.float16), rewards=tm(d["rewards"], torch.float16),
+             values=tm(d["values"], torch.float16), terminateds=tm(d["terminateds"], torch.bool),
+             vs=nan_tm(), pg_advantages=nan_tm(), gamma=G, time_major=True)
+    r = dict(kind="discounted_returns", rewards=dev(d["rewards"]), terminateds=dev(d["terminateds"]),
+             returns=_nan((E, T)), gamma=G)
+    R.rlscan_batch([g, v, r])
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    g32, l32 = np.float32(G), np.float32(L)
+    ga = (wide_t(g["truncateds"]), wide_t(g["bootstrap_values"]), d["last_values"])
+    assert_close(g["advantages"].t(), oracle.gae(wide_t(g["rewards"]), wide_t(g["values"]),
+                                                 wide_t(g["terminateds"]), g32, l32, *ga), 1e-4, "tm bf16/u8 gae")
+    assert_close(g["returns"].t(), oracle.lambda_returns(wide_t(g["rewards"]), wide_t(g["values"]),
+                                                         wide_t(g["terminateds"]), g32, l32, *ga), 1e-4,
+                 "tm bf16/u8 returns")
+    rvs, rpg = oracle.vtrace(wide_t(v["log_rhos"]), wide_t(v["rewards"]), wide_t(v["values"]),
+                             wide_t(v["terminateds"]), g32)
+    assert_close(v["vs"].t(), rvs, 1e-4, "tm fp16/bool vtrace vs")
+    assert_close(v["pg_advantages"].t(), rpg, 1e-4, "tm fp16/bool vtrace pg")
+    assert_close(r["returns"], oracle.discounted_returns(d["rewards"], d["terminateds"], g32), 1e-4, "fp32 returns")
