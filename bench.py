@@ -511,9 +511,10 @@ TRUNC_P = 0.005  # terminated and truncated, each (mutually exclusive per step)
 
 def config_cases():
     """(key, E, T, host-input builder, {estimator: (call, streamed bytes per
-    env-step, outputs, input planes[, element types of the planes])}).  Streamed bytes count every dense plane read once and every
-    output written once; bootstrap values are read only at truncated steps
-    (about 1 % of steps here) and are not counted."""
+    env-step, outputs, input planes[, element types of the planes])}).
+    Streamed bytes count every plane read once (the bootstrap plane too: it
+    is streamed whenever truncations are given) and every output written
+    once."""
     from linear_recurrence_scans_02_b200 import workloads as W
 
     def trunc_inputs():
@@ -527,10 +528,10 @@ def config_cases():
                                     t.get("bootstrap_values"), None, o[0], g, LAMBDA)
 
     trunc = {
-        "gae": (gae, 20, 1, ("rewards", "values", "terminateds", "truncateds", "bootstrap_values")),
+        "gae": (gae, 24, 1, ("rewards", "values", "terminateds", "truncateds", "bootstrap_values")),
         "vtrace": (lambda R, t, o: lambda: R.rlscan_vtrace(
             t["log_rhos"], t["rewards"], t["values"], t["terminateds"], t["truncateds"], t["bootstrap_values"],
-            None, o[0], o[1], GAMMA, 1.0, 1.0, 1.0), 28, 2,
+            None, o[0], o[1], GAMMA, 1.0, 1.0, 1.0), 32, 2,
                    ("log_rhos", "rewards", "values", "terminateds", "truncateds", "bootstrap_values")),
         "retrace": (lambda R, t, o: lambda: R.rlscan_retrace(
             t["rewards"], t["q_values"], t["next_q_values_all"], None, t["log_rhos"], t["terminateds"],
@@ -538,9 +539,9 @@ def config_cases():
                     ("rewards", "q_values", "next_q_values_all", "log_rhos", "terminateds", "truncateds")),
         "lambda_returns": (lambda R, t, o: lambda: R.rlscan_lambda_returns(
             t["rewards"], t["values"], t["terminateds"], t["truncateds"], t["bootstrap_values"], None, o[0],
-            GAMMA, LAMBDA), 20, 1, ("rewards", "values", "terminateds", "truncateds", "bootstrap_values")),
+            GAMMA, LAMBDA), 24, 1, ("rewards", "values", "terminateds", "truncateds", "bootstrap_values")),
         "discounted_returns": (lambda R, t, o: lambda: R.rlscan_discounted_returns(
-            t["rewards"], t["terminateds"], t["truncateds"], t["bootstrap_values"], None, o[0], GAMMA), 16, 1,
+            t["rewards"], t["terminateds"], t["truncateds"], t["bootstrap_values"], None, o[0], GAMMA), 20, 1,
                                ("rewards", "terminateds", "truncateds", "bootstrap_values")),
     }
     A = 18
@@ -600,6 +601,16 @@ def config_cases():
                 "eligibility_traces_fp32": (traces, 12, 1, tk),
                 "eligibility_traces_bf16_u8": (traces, 7, 1, tk, narrow_dt)}
 
+    # GAE on the time-major layout beside row-major, few envs with long rows
+    # (the time-major rows are split over blocks); host inputs are [E, T],
+    # the time-major call gets their transposes
+    def gae_tm(R, t, o):
+        return lambda: R.rlscan_gae(t["rewards_tm"], t["values_tm"], t["terminateds_tm"], None, None, None,
+                                    o[0].view(o[0].shape[1], o[0].shape[0]), GAMMA, LAMBDA, time_major=True)
+
+    tm_cases = {"gae_row_major": (gae, 16, 1, ("rewards", "values", "terminateds")),
+                "gae_time_major": (gae_tm, 16, 1, ("rewards_tm", "values_tm", "terminateds_tm"))}
+
     def narrow_inputs(E):
         def build():
             d = W.vtrace_inputs(E, T_STEPS, 50, p_term=P_DONE)
@@ -614,6 +625,7 @@ def config_cases():
         ("off_policy_1024x2048_18_actions", 1024, 2048, lambda: W.off_policy_inputs(1024, 2048, A=A, seed=40),
          off),
         ("long_rows_16x262144", 16, 262144, long_inputs, long_rows),
+        ("time_major_512x4096", 512, 4096, lambda: W.gae_inputs(512, 4096, 60, p_term=P_DONE), tm_cases),
         ("reduced_bytes_4096x128", E_ENVS, T_STEPS, narrow_inputs(E_ENVS), narrow_cases(E_ENVS)),
         ("reduced_bytes_65536x128", 65536, T_STEPS, narrow_inputs(65536), narrow_cases(65536)),
     ]
@@ -624,6 +636,8 @@ def run_configs(torch, R, device, side, stream, world, peak, max_sets=2048):
     rot = rotate_bytes(device)
     for key, E, T, build, cases in config_cases():
         host = build()
+        for k in [k for k in host if isinstance(host[k], np.ndarray) and host[k].ndim == 2]:
+            host[k + "_tm"] = np.ascontiguousarray(host[k].T)
         res = {"num_envs": E, "seq_len": T}
         for est, case in cases.items():
             make, bpe, nout, keys = case[:4]
@@ -1093,13 +1107,19 @@ def run_profile_case(args):
     if args.profile_shape:  # GAE at another shape, e.g. 16,262144 (long rows: the two-pass path)
         from linear_recurrence_scans_02_b200 import workloads as W
         E, T = (int(v) for v in args.profile_shape.split(","))
-        d = W.device_inputs("gae", E, T, seed=0, device=torch.device("cuda", 0), p_done=1e-4)
-        out = torch.empty(E, T, device="cuda")
+        tm = args.profile_time_major
+        # the planes are iid per element, so [T, E] inputs for the time-major
+        # layout are drawn the same way as [E, T] ones
+        shape = (T, E) if tm else (E, T)
+        d = W.device_inputs("gae", *shape, seed=0, device=torch.device("cuda", 0), p_done=1e-4)
+        out = torch.empty(*shape, device="cuda")
         for _ in range(args.profile_launches):
-            R.rlscan_gae(d["rewards"], d["values"], d["terminateds"], None, None, None, out, 0.999, LAMBDA)
+            R.rlscan_gae(d["rewards"], d["values"], d["terminateds"], None, None, None, out, 0.999, LAMBDA,
+                         time_major=tm)
         torch.cuda.synchronize()
         R.rlscan_check()
-        print(f"profile case done: {args.profile_launches} GAE launches at {E} x {T}")
+        print(f"profile case done: {args.profile_launches} GAE launches at {E} x {T}"
+              + (" (time-major)" if tm else ""))
         return 0
     bs = BufferSet(torch, torch.device("cuda", 0), PLANES)
     bs.fill_from_host(host_inputs(seed=0))
@@ -1134,6 +1154,8 @@ def main(argv=None):
                     help="run N eager launches of each estimator and exit (small case for ncu)")
     ap.add_argument("--profile-only", default="", help="comma-separated estimators for --profile-launches")
     ap.add_argument("--profile-shape", default="", help="E,T: --profile-launches runs GAE at this shape instead")
+    ap.add_argument("--profile-time-major", action="store_true",
+                    help="with --profile-shape: GAE on the time-major layout [T, E]")
     ap.add_argument("--profile-config", default="", choices=["", "off_policy"],
                     help="off_policy: --profile-launches runs multi-action Retrace (256 x 2048, 18 actions)")
     ap.add_argument("--sweep", action="store_true",

@@ -315,8 +315,11 @@ RLSCAN_API int rlscan_gae_noalloc(const float *rewards, const float *values, con
  *     instead [T, E], E (num_envs) fastest: element (e, t) is at index
  *     t*E + e, the rollout-buffer layout of vectorised environments that write
  *     one row of E per step.  last_values stays [E].  Rows are still scanned
- *     independently; a time-major call needs no workspace (ws may be NULL)
- *     and reads and writes each element once with coalesced accesses along E.
+ *     independently, reading and writing each element once with coalesced
+ *     accesses along E.  With few envs and long rows, each row is split over
+ *     several blocks (two launches: each split's map per env, then the
+ *     splits with their carries) when ws holds rlscan_workspace_bytes(E, T)
+ *     bytes (any content); with ws = NULL every row runs in one block.
  *     rlscan_retrace_ex takes it with A == 1 only, and E up to
  *     238,609,294 (offsets between timesteps are 32-bit); beyond either,
  *     RLSCAN_ERR_UNSUPPORTED.

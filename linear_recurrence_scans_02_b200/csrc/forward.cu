@@ -21,7 +21,7 @@ int rlscan_eligibility_traces_ex(const float *x, const float *dones, float *trac
     RLSCAN_TRY(check_aliasing(ins, 2, outs, 1));
     TracesEst::Params P{x, dones, traces, gamma * lambda_, (options & RLSCAN_OPT_DONE_STARTS_EPISODE) ? 1 : 0};
     if (options & RLSCAN_OPT_TIME_MAJOR)
-        return run_time_major<TracesEst>("rlscan_eligibility_traces", P, E, T, stream);
+        return run_time_major<TracesEst>("rlscan_eligibility_traces", P, E, T, stream, ws, ws_bytes);
     return run<TracesEst>("rlscan_eligibility_traces", P, E, T, ws, ws_bytes, stream,
                           aligned16({x, dones, traces}));
 }
@@ -46,13 +46,13 @@ int rlscan_episodic_prefix_sum_ex(const void *x, int dtype, const float *dones, 
     if (dtype == RLSCAN_F32) {
         PrefixF32Est::Params P{static_cast<const float *>(x), dones, static_cast<float *>(out), 1.0f, (options & RLSCAN_OPT_DONE_STARTS_EPISODE) ? 1 : 0};
         if (options & RLSCAN_OPT_TIME_MAJOR)
-            return run_time_major<PrefixF32Est>("rlscan_episodic_prefix_sum", P, E, T, stream);
+            return run_time_major<PrefixF32Est>("rlscan_episodic_prefix_sum", P, E, T, stream, ws, ws_bytes);
         return run<PrefixF32Est>("rlscan_episodic_prefix_sum", P, E, T, ws, ws_bytes, stream,
                                  aligned16({x, dones, out}));
     }
     PrefixI32Est::Params P{static_cast<const int32_t *>(x), dones, static_cast<int32_t *>(out), (options & RLSCAN_OPT_DONE_STARTS_EPISODE) ? 1 : 0};
     if (options & RLSCAN_OPT_TIME_MAJOR)
-        return run_time_major<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, stream);
+        return run_time_major<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, stream, ws, ws_bytes);
     return run<PrefixI32Est>("rlscan_episodic_prefix_sum", P, E, T, ws, ws_bytes, stream,
                              aligned16({x, dones, out}));
 }

@@ -63,7 +63,7 @@ int rlscan_gae_ex(const float *rewards, const float *values, const float *termin
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
     GaeEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                      last_values, advantages, nullptr, gamma, lambda_};
-    if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<GaeEst>("rlscan_gae", P, E, T, stream);
+    if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<GaeEst>("rlscan_gae", P, E, T, stream, ws, ws_bytes);
     return run<GaeEst>("rlscan_gae", P, E, T, ws, ws_bytes, stream,
                        aligned16({rewards, values, terminateds, truncateds, advantages}));
 }
@@ -97,7 +97,7 @@ int rlscan_gae_with_returns_ex(const float *rewards, const float *values, const 
     GaeReturnsEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                             last_values, advantages, returns, gamma, lambda_};
     if (options & RLSCAN_OPT_TIME_MAJOR)
-        return run_time_major<GaeReturnsEst>("rlscan_gae_with_returns", P, E, T, stream);
+        return run_time_major<GaeReturnsEst>("rlscan_gae_with_returns", P, E, T, stream, ws, ws_bytes);
     return run<GaeReturnsEst>("rlscan_gae_with_returns", P, E, T, ws, ws_bytes, stream,
                               aligned16({rewards, values, terminateds, truncateds, advantages, returns}));
 }
@@ -149,7 +149,7 @@ int rlscan_gae_typed_ex(const void *rewards, const void *values, const void *ter
                                                static_cast<const FT *>(truncateds), static_cast<const VT *>(bv),  \
                                                last_values, advantages, returns, gamma, lambda_};                  \
         if (options & RLSCAN_OPT_TIME_MAJOR)                                                                      \
-            return run_time_major<GaeTypedEst<VT, FT>>("rlscan_gae_typed", P, E, T, stream);                     \
+            return run_time_major<GaeTypedEst<VT, FT>>("rlscan_gae_typed", P, E, T, stream, ws, ws_bytes);                     \
         return run<GaeTypedEst<VT, FT>>("rlscan_gae_typed", P, E, T, ws, ws_bytes, stream, vec);              \
     } while (0)
     if (flag_dtype == RLSCAN_U8) {

@@ -428,6 +428,9 @@ constexpr int kTmV = 8;
 
 struct TmPlan {
     int G, nw;
+    long long nseg; // segments per row
+    int nsplit;     // blocks per row (1: whole rows)
+    int sps;        // segments per split
 };
 
 // Wider env groups (longer contiguous runs per load) while the grid keeps
@@ -442,11 +445,30 @@ inline TmPlan tm_plan(long long E, long long T) {
     const long long chunks = ceil_div(T, kTmV);
     const long long nw = ceil_div(chunks, 32 / p.G);
     p.nw = (int)(nw < 1 ? 1 : (nw > kTmMaxWarps ? kTmMaxWarps : nw));
+    p.nseg = ceil_div(T, (long long)p.nw * (32 / p.G) * kTmV);
+    // rows split over blocks when the env groups alone leave the GPU short of
+    // two blocks per SM and rows hold several segments
+    const long long blocks = ceil_div(E, p.G), want = 2 * num_sms();
+    p.nsplit = 1;
+    p.sps = (int)p.nseg;
+    if (blocks < want && p.nseg > 1) {
+        const long long ns = std::min<long long>(p.nseg, ceil_div(want, blocks));
+        p.sps = (int)ceil_div(p.nseg, ns);
+        p.nsplit = (int)ceil_div(p.nseg, p.sps);
+    }
     return p;
 }
 
+// Workspace of a time-major call: one 16-byte slot per env and split when
+// its rows are split over blocks, else none.
+inline size_t tm_workspace_for(long long E, long long T) {
+    const TmPlan p = tm_plan(E, T);
+    return p.nsplit > 1 ? sizeof(TileSlot) * (size_t)E * (size_t)p.nsplit : 0;
+}
+
 template <class Est>
-int run_time_major(const char *name, const typename Est::Params &P, long long E, long long T, cudaStream_t stream) {
+int run_time_major(const char *name, const typename Est::Params &P, long long E, long long T, cudaStream_t stream,
+                   void *ws = nullptr, size_t ws_bytes = 0) {
     if (E > (long long)INT_MAX / (kTmV + 1))
         return fail(RLSCAN_ERR_UNSUPPORTED, "%s: the time-major layout takes E <= %d", name, INT_MAX / (kTmV + 1));
     if (batch_dry()) return ok();
@@ -455,12 +477,18 @@ int run_time_major(const char *name, const typename Est::Params &P, long long E,
     g.n = E * T;
     g.seq_len = T;
     g.rows = E;
-    g.ntiles = ceil_div(T, (long long)tp.nw * (32 / tp.G) * kTmV); // segments per row
+    g.ntiles = tp.nseg; // segments per row
     g.t_shift = pow2_shift(T);
     g.vec_ok = 0;
     g.scan_lanes = 32;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)ceil_div(E, tp.G));
+    // split rows need a workspace (of any content); without one (or too
+    // small) the rows run whole
+    TmSplit sp{nullptr, 1, (int)tp.nseg};
+    const size_t need = tp.nsplit > 1 ? sizeof(TileSlot) * (size_t)E * (size_t)tp.nsplit : 0;
+    if (need > 0 && ws != nullptr && ws_bytes >= need && ((uintptr_t)ws & 15u) == 0)
+        sp = TmSplit{static_cast<TileSlot *>(ws), tp.nsplit, tp.sps};
+    cfg.gridDim = dim3((unsigned)ceil_div(E, tp.G), (unsigned)sp.nsplit);
     cfg.blockDim = dim3(tp.nw * 32);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -468,13 +496,23 @@ int run_time_major(const char *name, const typename Est::Params &P, long long E,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    cudaError_t e;
-    switch (tp.G) {
-    case 32: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 32, kTmV>, P, g); break;
-    case 16: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 16, kTmV>, P, g); break;
-    default: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 8, kTmV>, P, g); break;
+    cudaError_t e = cudaSuccess;
+    const int passes[2] = {sp.nsplit > 1 ? kTmMaps : kTmWhole, kTmCarry};
+    for (int i = 0; i < (sp.nsplit > 1 ? 2 : 1); ++i) {
+        const int pass = passes[i];
+        switch (tp.G * 4 + pass) {
+        case 32 * 4 + kTmWhole: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 32, kTmV, kTmWhole>, P, g, sp); break;
+        case 32 * 4 + kTmMaps: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 32, kTmV, kTmMaps>, P, g, sp); break;
+        case 32 * 4 + kTmCarry: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 32, kTmV, kTmCarry>, P, g, sp); break;
+        case 16 * 4 + kTmWhole: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 16, kTmV, kTmWhole>, P, g, sp); break;
+        case 16 * 4 + kTmMaps: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 16, kTmV, kTmMaps>, P, g, sp); break;
+        case 16 * 4 + kTmCarry: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 16, kTmV, kTmCarry>, P, g, sp); break;
+        case 8 * 4 + kTmWhole: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 8, kTmV, kTmWhole>, P, g, sp); break;
+        case 8 * 4 + kTmMaps: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 8, kTmV, kTmMaps>, P, g, sp); break;
+        default: e = cudaLaunchKernelEx(&cfg, time_major_scan_kernel<Est, 8, kTmV, kTmCarry>, P, g, sp); break;
+        }
+        if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
     }
-    if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
     return ok();
 }
 

@@ -27,7 +27,7 @@ int rlscan_lambda_returns_ex(const float *rewards, const float *values, const fl
     LambdaReturnsEst::Params P{rewards, values, terminateds, truncateds, truncateds ? bootstrap_values : nullptr,
                                last_values, returns, gamma, lambda_};
     if (options & RLSCAN_OPT_TIME_MAJOR)
-        return run_time_major<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, stream);
+        return run_time_major<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, stream, ws, ws_bytes);
     return run<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, ws, ws_bytes, stream,
                                  aligned16({rewards, values, terminateds, truncateds, returns}));
 }
@@ -57,7 +57,7 @@ int rlscan_discounted_returns_ex(const float *rewards, const float *terminateds,
     ReturnsEst::Params P{rewards, terminateds, truncateds, truncateds ? bootstrap_values : nullptr, last_values,
                          returns, gamma};
     if (options & RLSCAN_OPT_TIME_MAJOR)
-        return run_time_major<ReturnsEst>("rlscan_discounted_returns", P, E, T, stream);
+        return run_time_major<ReturnsEst>("rlscan_discounted_returns", P, E, T, stream, ws, ws_bytes);
     return run<ReturnsEst>("rlscan_discounted_returns", P, E, T, ws, ws_bytes, stream,
                            aligned16({rewards, terminateds, truncateds, returns}));
 }

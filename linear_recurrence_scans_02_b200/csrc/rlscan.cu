@@ -49,7 +49,7 @@ int rlscan_retrace_ex(const float *rewards, const float *q_values, const float *
     if (A == 1) {
         RetraceEst::Params P{rewards, q_values, next_q_values_all, log_rhos, terminateds, truncateds, q_ret, gamma,
                              lambda_, c_bar};
-        if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<RetraceEst>("rlscan_retrace", P, E, T, stream);
+        if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<RetraceEst>("rlscan_retrace", P, E, T, stream, ws, ws_bytes);
         return run<RetraceEst>("rlscan_retrace", P, E, T, ws, ws_bytes, stream,
                                aligned16({rewards, q_values, next_q_values_all, log_rhos, terminateds, truncateds,
                                           q_ret}));
@@ -84,7 +84,7 @@ int rlscan_retrace(const float *rewards, const float *q_values, const float *nex
 
 size_t rlscan_workspace_bytes(int64_t E, int64_t T) {
     if (E <= 0 || T <= 0 || E > kMaxElems / T) return 0;
-    return workspace_for(make_plan(E, T));
+    return std::max(workspace_for(make_plan(E, T)), tm_workspace_for(E, T));
 }
 
 int rlscan_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream) {

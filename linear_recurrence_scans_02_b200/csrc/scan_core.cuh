@@ -924,13 +924,29 @@ struct PlaneRef {
 
 constexpr int kTmMaxWarps = 16;
 
+// Rows of the time-major kernel split over several blocks (few envs with
+// long rows): blockIdx.y is the split, each split a run of `sps` consecutive
+// segments in scan order.  Pass kTmMaps writes, per env, the map of its
+// split (the composition of its elements' (a, b) in scan order) into
+// slots[e * nsplit + split]; pass kTmCarry starts each split from the value
+// the maps of the splits before it carry in, and writes the outputs.
+// kTmWhole runs every row in one block (nsplit = 1, no workspace).
+struct TmSplit {
+    TileSlot *slots;
+    int nsplit;
+    int sps;
+};
+constexpr int kTmWhole = 0;
+constexpr int kTmMaps = 1;
+constexpr int kTmCarry = 2;
+
 __device__ __forceinline__ void prefetch_line_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-template <class Est, int G, int V>
+template <class Est, int G, int V, int kPass>
 __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const typename Est::Params P,
-                                                                           const Geometry g) {
+                                                                           const Geometry g, const TmSplit sp) {
     using AT = typename Est::AT;
     using BT = typename Est::BT;
     constexpr bool kBwd = Est::kBackward;
@@ -940,6 +956,8 @@ __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const
     __shared__ BT s_b[kTmMaxWarps][G];
     __shared__ BT s_x[kTmMaxWarps][G];
     __shared__ BT s_carry[G];
+    __shared__ AT s_ma[G]; // kTmMaps: each env's map of the segments so far
+    __shared__ BT s_mb[G];
 
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
@@ -952,11 +970,14 @@ __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const
     const bool env_ok = e < E;
     const int S = nw * CPW * V;       // timesteps per segment (<= 16 * 32 * V)
     const long long nseg = g.ntiles;  // ceil(T / S), from the host
+    const int split = blockIdx.y;
+    const long long s_begin = (long long)split * sp.sps;            // this block's segments,
+    const long long s_end = min(nseg, s_begin + (long long)sp.sps); // in scan order
 
     // L2 prefetch of the first segment's input rows, before waiting for the
     // previous grid (L2 is coherent, so a prefetched line is never stale)
     {
-        const long long t_first = kBwd ? (nseg - 1) * S : 0;
+        const long long t_first = (kBwd ? nseg - 1 - s_begin : s_begin) * S;
         const int rows = (int)((T - t_first) < S ? (T - t_first) : S);
         const int envs = (int)((E - e0) < G ? (E - e0) : G);
 #pragma unroll
@@ -974,9 +995,26 @@ __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const
     griddep_wait();
     griddep_launch_dependents();
 
-    if (threadIdx.x < G) s_carry[threadIdx.x] = identity_b(BT());
+    if (threadIdx.x < G) {
+        const int ee = threadIdx.x;
+        BT x = identity_b(BT());
+        if constexpr (kPass == kTmCarry) { // the value the earlier splits carry in
+            if (e0 + ee < E) {
+                const TileSlot *row = sp.slots + (e0 + ee) * sp.nsplit;
+                for (int k = 0; k < split; ++k) {
+                    AT ka = AT();
+                    BT kb = BT();
+                    read_slot(row + k, ka, kb);
+                    x = apply_pair(ka, kb, x);
+                }
+            }
+        }
+        s_carry[ee] = x;
+        s_ma[ee] = identity_a(AT());
+        s_mb[ee] = identity_b(BT());
+    }
 
-    for (long long si = 0; si < nseg; ++si) {
+    for (long long si = s_begin; si < s_end; ++si) {
         const long long seg = kBwd ? nseg - 1 - si : si;
         const long long t0 = seg * S + (w * CPW + cs) * V;
         const TimeMajorPos<V> pos = TimeMajorPos<V>::make(e, t0, E, T, env_ok);
@@ -1043,7 +1081,21 @@ __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const
             s_b[w][es] = ib;
         }
         __syncthreads();
-        if (threadIdx.x < G) { // chain this env's warps in scan order
+        if (kPass == kTmMaps && threadIdx.x < G) { // compose this env's warp maps in scan order
+            const int ee = threadIdx.x;
+            AT ma = s_ma[ee];
+            BT mb = s_mb[ee];
+            for (int j = 0; j < nw; ++j) {
+                const int ww = kBwd ? nw - 1 - j : j;
+                AT na = s_a[ww][ee];
+                BT nb = s_b[ww][ee];
+                combine(na, nb, ma, mb); // the later warp applied after the map so far
+                ma = na;
+                mb = nb;
+            }
+            s_ma[ee] = ma;
+            s_mb[ee] = mb;
+        } else if (threadIdx.x < G) { // chain this env's warps in scan order
             const int ee = threadIdx.x;
             BT x = s_carry[ee];
             // four warps at a time: their shared loads issue together, ahead
@@ -1070,6 +1122,7 @@ __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const
             s_carry[ee] = x;
         }
         __syncthreads();
+        if constexpr (kPass == kTmMaps) continue; // maps only: no outputs
         // shared arrays: the next segment writes s_a / s_b before its first
         // barrier, after every read of them here (before this barrier), and
         // s_x / s_carry only after that barrier, when every thread has read
@@ -1091,6 +1144,11 @@ __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const
             }
         }
         Est::template store<V>(P, g, pos, St);
+    }
+    if constexpr (kPass == kTmMaps) {
+        if (threadIdx.x < G && e0 + threadIdx.x < E)
+            publish_aggregate(sp.slots + (e0 + threadIdx.x) * sp.nsplit + split, s_ma[threadIdx.x],
+                              s_mb[threadIdx.x]);
     }
 }
 

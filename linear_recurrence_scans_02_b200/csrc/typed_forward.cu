@@ -23,7 +23,7 @@ int check_forward(const rlscan_call &c, const char *name, const char *out_name) 
 template <class Est>
 int run_forward(const char *name, const typename Est::Params &P, const rlscan_call &c, void *ws, size_t ws_bytes,
                 cudaStream_t stream) {
-    if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream);
+    if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream, ws, ws_bytes);
     return run<Est>(name, P, c.E, c.T, ws, ws_bytes, stream, aligned16({c.in[0], c.in[1], c.out[0]}));
 }
 } // namespace

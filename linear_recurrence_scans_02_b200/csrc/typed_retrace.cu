@@ -46,7 +46,7 @@ int typed_retrace(const rlscan_call &c, void *ws, size_t ws_bytes, cudaStream_t 
                                    static_cast<const VT *>(in[2]), static_cast<const VT *>(in[4]),
                                    static_cast<const FT *>(in[5]), static_cast<const FT *>(in[6]), q_ret, c.gamma,
                                    c.lambda_, c.c_bar};
-            if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream);
+            if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream, ws, ws_bytes);
             return run<Est>(name, P, c.E, c.T, ws, ws_bytes, stream,
                             aligned16({in[0], in[1], in[2], in[4], in[5], in[6], q_ret}));
         }

@@ -34,7 +34,7 @@ int typed_lambda_returns(const rlscan_call &c, void *ws, size_t ws_bytes, cudaSt
                                in[3] ? static_cast<const VT *>(in[4]) : nullptr,
                                static_cast<const float *>(in[5]), static_cast<float *>(c.out[0]), c.gamma,
                                c.lambda_};
-        if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream);
+        if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream, ws, ws_bytes);
         return run<Est>(name, P, c.E, c.T, ws, ws_bytes, stream, vec);
     });
 }
@@ -64,7 +64,7 @@ int typed_discounted_returns(const rlscan_call &c, void *ws, size_t ws_bytes, cu
         typename Est::Params P{static_cast<const VT *>(in[0]), static_cast<const FT *>(in[1]),
                                static_cast<const FT *>(in[2]), in[2] ? static_cast<const VT *>(in[3]) : nullptr,
                                static_cast<const float *>(in[4]), static_cast<float *>(c.out[0]), c.gamma};
-        if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream);
+        if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream, ws, ws_bytes);
         return run<Est>(name, P, c.E, c.T, ws, ws_bytes, stream, vec);
     });
 }

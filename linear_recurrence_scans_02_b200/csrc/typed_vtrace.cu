@@ -39,7 +39,7 @@ int typed_vtrace(const rlscan_call &c, void *ws, size_t ws_bytes, cudaStream_t s
                                in[4] ? static_cast<const VT *>(in[5]) : nullptr,
                                static_cast<const float *>(in[6]), static_cast<float *>(c.out[0]),
                                static_cast<float *>(c.out[1]), c.gamma, c.lambda_, c.rho_bar, c.c_bar};
-        if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream);
+        if (c.options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<Est>(name, P, c.E, c.T, stream, ws, ws_bytes);
         return run<Est>(name, P, c.E, c.T, ws, ws_bytes, stream, vec);
     });
 }

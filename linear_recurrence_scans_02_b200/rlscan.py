@@ -236,8 +236,8 @@ def _layout(t, name, time_major):
 
 
 def _ws_for(dev, E, T, ws, opts):
-    if opts & RLSCAN_OPT_TIME_MAJOR:  # rows never span blocks: no workspace
-        return None, 0, _stream_handle(dev)
+    # row-major calls whose rows span tiles, and time-major calls whose rows
+    # are split over blocks, use it; the size covers both layouts
     return _workspace(dev, E, T, ws)
 
 
@@ -518,8 +518,7 @@ def rlscan_batch(calls, ws=None):
             c.inp[i] = _ptr(call.get(name), name, shape, slot_dtypes[name], dev)
         for i, name in enumerate(out_names):
             c.out[i] = _ptr(call.get(name), name, sh, out_dtype, dev)
-        if not tm:
-            ws_need = max(ws_need, int(_lib.rlscan_workspace_bytes(E, T)))
+        ws_need = max(ws_need, int(_lib.rlscan_workspace_bytes(E, T)))
     if not calls:
         return
     stream = _stream_handle(dev)
