@@ -60,7 +60,7 @@ struct BackwardFamilyEst {
         prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values);
     }
     static constexpr int kInputPlanes = 5;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         const float *p[5] = {P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values};
         return {i < 5 ? p[i] : nullptr, 4};
     }

@@ -93,7 +93,7 @@ struct GaeEstT {
     }
     // Input planes read element by element (the time-major kernel's prefetch).
     static constexpr int kInputPlanes = 5;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         switch (i) {
         case 0: return {P.rewards, (int)sizeof(ValT)};
         case 1: return {P.values, (int)sizeof(ValT)};
@@ -194,7 +194,7 @@ struct LambdaReturnsEstT {
         prefetch_planes(g, tile0, S, P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values);
     }
     static constexpr int kInputPlanes = 5;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         switch (i) {
         case 0: return {P.rewards, (int)sizeof(ValT)};
         case 1: return {P.values, (int)sizeof(ValT)};
@@ -297,7 +297,7 @@ struct ReturnsEstT {
         prefetch_planes(g, tile0, S, P.rewards, P.terminateds, P.truncateds, P.bootstrap_values);
     }
     static constexpr int kInputPlanes = 4;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         switch (i) {
         case 0: return {P.rewards, (int)sizeof(ValT)};
         case 1: return {P.terminateds, (int)sizeof(FlagT)};
@@ -393,7 +393,7 @@ struct VtraceEstT {
                         P.bootstrap_values);
     }
     static constexpr int kInputPlanes = 6;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         switch (i) {
         case 0: return {P.log_rhos, (int)sizeof(ValT)};
         case 1: return {P.rewards, (int)sizeof(ValT)};
@@ -509,7 +509,7 @@ struct GaeVtraceEst {
                         P.bootstrap_values);
     }
     static constexpr int kInputPlanes = 6;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         const float *p[6] = {P.log_rhos, P.rewards, P.values, P.terminateds, P.truncateds, P.bootstrap_values};
         return {i < 6 ? p[i] : nullptr, 4};
     }
@@ -621,7 +621,7 @@ struct RetraceEstT {
                         P.next_q_values_all);
     }
     static constexpr int kInputPlanes = 6;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         switch (i) {
         case 0: return {P.rewards, (int)sizeof(ValT)};
         case 1: return {P.q_values, (int)sizeof(ValT)};
@@ -711,7 +711,7 @@ struct ForwardEstT {
         prefetch_planes(g, tile0, S, P.x, P.dones);
     }
     static constexpr int kInputPlanes = 2;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         switch (i) {
         case 0: return {P.x, (int)sizeof(ValT)};
         case 1: return {P.dones, (int)sizeof(FlagT)};
@@ -783,7 +783,7 @@ struct PrefixI32EstT {
         prefetch_planes(g, tile0, S, P.x, P.dones);
     }
     static constexpr int kInputPlanes = 2;
-    static __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
+    static __host__ __device__ __forceinline__ PlaneRef input_plane(const Params &P, int i) {
         switch (i) {
         case 0: return {P.x, 4};
         case 1: return {P.dones, (int)sizeof(FlagT)};

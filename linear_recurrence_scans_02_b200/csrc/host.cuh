@@ -311,18 +311,30 @@ cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, const L
     }
 }
 
-// Input bytes per tile a two-pass wave may hold so that pass two re-reads
-// them from L2: a wave's pass one streams them from HBM, pass two finds them
-// in L2 (B200: 126 MB).
+// Input bytes a two-pass wave may hold so that pass two re-reads them from
+// L2: a wave's pass one streams them from HBM, pass two finds them in L2
+// (B200: 126 MB).
 constexpr long long kTwoPassWaveBytes = 64ll << 20;
 
+// Bytes per element of the input planes a call streams (its given planes).
+template <class Est>
+inline long long streamed_input_bytes(const typename Est::Params &P) {
+    long long b = 0;
+    for (int i = 0; i < Est::kInputPlanes; ++i) {
+        const PlaneRef r = Est::input_plane(P, i);
+        if (r.p != nullptr) b += r.bytes;
+    }
+    return b;
+}
+
 // Rows that span tiles: pass one (aggregates) and pass two (scan with
-// carries) over waves of consecutive scan-order tiles.
+// carries) over waves of consecutive scan-order tiles, as few waves as keep
+// each wave's inputs within kTwoPassWaveBytes, of equal size.
 template <class Est>
 int run_two_pass(const char *name, const typename Est::Params &P, const Geometry &g, Lookback lb, Cfg cfg,
                  cudaStream_t stream) {
-    const long long tile_bytes = (long long)kCfgTile[cfg] * 4 * Est::kInputPlanes;
-    const long long wave = std::max<long long>(1, kTwoPassWaveBytes / tile_bytes);
+    const long long in_bytes = std::max<long long>(1, streamed_input_bytes<Est>(P)) * g.n;
+    const long long wave = ceil_div(g.ntiles, ceil_div(in_bytes, kTwoPassWaveBytes));
     for (long long t0 = 0; t0 < g.ntiles; t0 += wave) {
         lb.tile_base = t0;
         const long long cnt = std::min<long long>(wave, g.ntiles - t0);
