@@ -209,15 +209,15 @@ class BufferSet:
                 t["gae_with_returns", "returns"], GAMMA, LAMBDA)
         if "gae_with_returns_bf16_u8" in self.estimators:
             k = "gae_with_returns_bf16_u8"
-            c[k] = lambda: R.rlscan_gae_typed(t[k, "rewards"], t[k, "values"], t[k, "terminateds"], None, None, None,
+            c[k] = lambda k=k: R.rlscan_gae_typed(t[k, "rewards"], t[k, "values"], t[k, "terminateds"], None, None, None,
                                               t[k, "advantages"], t[k, "returns"], GAMMA, LAMBDA)
         if "gae_time_major" in self.estimators:
             k = "gae_time_major"
-            c[k] = lambda: R.rlscan_gae(t[k, "rewards"], t[k, "values"], t[k, "terminateds"], None, None, None,
+            c[k] = lambda k=k: R.rlscan_gae(t[k, "rewards"], t[k, "values"], t[k, "terminateds"], None, None, None,
                                         t[k, "advantages"], GAMMA, LAMBDA, time_major=True)
         if "gae_returns_vtrace" in self.estimators:
             k = "gae_returns_vtrace"
-            c[k] = lambda: R.rlscan_gae_vtrace(t[k, "log_rhos"], t[k, "rewards"], t[k, "values"],
+            c[k] = lambda k=k: R.rlscan_gae_vtrace(t[k, "log_rhos"], t[k, "rewards"], t[k, "values"],
                                                t[k, "terminateds"], None, None, None, t[k, "advantages"],
                                                t[k, "returns"], t[k, "vs"], t[k, "pg_advantages"], GAMMA, LAMBDA,
                                                1.0, 1.0, 1.0)

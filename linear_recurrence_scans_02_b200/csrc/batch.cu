@@ -128,22 +128,15 @@ static int call_dispatch(const rlscan_call &c, void *ws, size_t ws_bytes, cudaSt
     }
 }
 
-// Elements per thread of a fused launch: 4 when it mixes three or more tile
-// bodies and every row fits a 512-element tile, else 8 (measured at 4096 x
-// 128: the eight estimators of one step 16.1 us at 4 against 17.6 us at 8;
-// eight GAE calls 11.0 us either way).  The items arrive ordered by body
-// (blocks of one body then share each SM's instruction caches); each is
+// Fused calls are tiled at 128 threads x 8 elements (measured at 4096 x
+// 128: the eight estimators of one step in 15.2 us, against 15.6 us with 4
+// elements per thread whenever three or more bodies meet).  The items arrive
+// ordered by body (blocks of one body then mostly share each SM); each is
 // tiled.
 constexpr int kMaxBodiesPerLaunch = kNumFusedBodies; // every fused call in one launch
 
-static int fused_layout(FusedBatch &fb, long long *tiles) {
-    unsigned bodies = 0u;
-    bool fit4 = true;
-    for (int i = 0; i < fb.n; ++i) {
-        bodies |= 1u << fb.item[i].kind;
-        if ((long long)(kFusedNT * 4) % fb.item[i].g.seq_len != 0) fit4 = false;
-    }
-    const int V = (__builtin_popcount(bodies) >= 3 && fit4) ? 4 : 8;
+static void fused_layout(FusedBatch &fb, long long *tiles) {
+    constexpr int V = kFusedV;
     long long begin = 0;
     for (int i = 0; i < fb.n; ++i) {
         FusedItem &it = fb.item[i];
@@ -155,7 +148,6 @@ static int fused_layout(FusedBatch &fb, long long *tiles) {
         begin += it.g.ntiles;
     }
     *tiles = begin;
-    return V;
 }
 
 // Runs every call of the request in the given pass; the first failure is
@@ -225,7 +217,7 @@ int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes
         part.n = last - first + 1;
         std::copy(st.fb.item + first, st.fb.item + last + 1, part.item);
         long long tiles = 0;
-        const int V = fused_layout(part, &tiles);
+        fused_layout(part, &tiles);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)tiles);
         cfg.blockDim = dim3(kFusedNT);
@@ -235,8 +227,7 @@ int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = pdl_enabled() ? 1 : 0;
-        const cudaError_t e = V == 4 ? cudaLaunchKernelEx(&cfg, fused_tile_kernel<4>, part)
-                                     : cudaLaunchKernelEx(&cfg, fused_tile_kernel<8>, part);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_tile_kernel<kFusedV>, part);
         if (e != cudaSuccess)
             return fail(RLSCAN_ERR_CUDA, "rlscan_batch: fused launch failed: %s", cudaGetErrorString(e));
         first = last + 1;

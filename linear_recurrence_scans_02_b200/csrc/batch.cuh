@@ -4,10 +4,7 @@
 // tile b - tile_begin of the call whose range holds b, through the same tile
 // body (and so the same arithmetic, bit for bit) as that call's own launch.
 // Only calls whose rows fit whole in one tile are fused, so every block of
-// the grid has the same shape: 128 threads x 8 elements, or x 4 elements
-// when the request mixes several estimators (blocks of different
-// estimators then share each SM, and the smaller unrolled bodies fit the
-// instruction caches better).
+// the grid has the same shape: 128 threads x 8 elements.
 #pragma once
 
 #include "estimators.cuh"
@@ -160,8 +157,8 @@ inline const P &family_params(const P &p) { // estimators that are their own bod
     return p;
 }
 
-constexpr int kFusedNT = 128; // 128 threads x 8 (or 4) elements per tile
-constexpr int kFusedVMax = 8;
+constexpr int kFusedNT = 128; // 128 threads x 8 elements per tile
+constexpr int kFusedV = 8;
 constexpr int kFusedParamBytes = 128;
 constexpr int kFusedMax = 16;
 

@@ -387,7 +387,7 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
     if constexpr (FusedBodyOf<Est>::value >= 0) {
         // fused when whole rows fit the largest fused tile; the fused launch
         // tiles the call itself (fused_layout, once the request is known)
-        constexpr long long kS = (long long)kFusedNT * kFusedVMax;
+        constexpr long long kS = (long long)kFusedNT * kFusedV;
         if (g_batch != nullptr && kS % T == 0 && g_batch->fb.n < kFusedMax) {
             const auto body_params = family_params(P);
             static_assert(sizeof(body_params) <= kFusedParamBytes, "params fit a fused item");

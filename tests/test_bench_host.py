@@ -43,3 +43,28 @@ def test_traffic_record_only_for_matching_kernel_source(tmp_path, monkeypatch):
     assert bench.recorded_traffic("gae") is None  # captured from another kernel source
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
     assert bench.recorded_traffic("gae") is None
+
+
+def test_each_timed_call_reads_its_own_planes():
+    # every closure of BufferSet.calls passes its own estimator's buffers
+    # (in their element types and layouts), never another call's
+    import torch
+    bs = bench.BufferSet(torch, torch.device("cpu"), bench.PLANES)
+    owner = {bs.t[key].data_ptr(): key for key in bs.t}
+    seen = []
+
+    class Recorder:
+        def __getattr__(self, name):
+            def call(*args, **kwargs):
+                seen.extend(a for a in args if isinstance(a, torch.Tensor))
+            return call
+
+    for est, fn in bs.calls(Recorder()).items():
+        seen.clear()
+        fn()
+        assert seen, est
+        for tensor in seen:
+            assert owner[tensor.data_ptr()][0] == est, (est, owner[tensor.data_ptr()])
+            assert tensor.shape == bs.t[owner[tensor.data_ptr()]].shape
+    assert bs.t["gae_with_returns_bf16_u8", "rewards"].dtype == torch.bfloat16
+    assert tuple(bs.t["gae_time_major", "rewards"].shape) == (bench.T_STEPS, bench.E_ENVS)
