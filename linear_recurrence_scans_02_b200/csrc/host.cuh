@@ -282,6 +282,18 @@ cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const L
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(grid < 0 ? g.ntiles : grid));
     cfg.blockDim = dim3(NT);
+    // resident blocks per SM of this kernel, queried once
+    static int resident = 0;
+    if (resident == 0) {
+        int r = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, NT, smem) != cudaSuccess || r < 1) {
+            (void)cudaGetLastError();
+            r = 1 << 16; // unknown: every block prefetches
+        }
+        resident = r;
+    }
+    Geometry gl = g;
+    gl.pf_blocks = (long long)num_sms() * resident;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -289,7 +301,7 @@ cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const L
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, P, g, lb);
+    return cudaLaunchKernelEx(&cfg, kern, P, gl, lb);
 }
 
 template <class Est, Cfg C>

@@ -204,6 +204,11 @@ struct Geometry {
     int t_shift;       // log2(T) when T is a power of two, else -1
     int vec_ok;        // every plane pointer of the call is 16-byte aligned
     int scan_lanes;    // warp-local mode: lanes one row spans (a power of two <= 32)
+    // Blocks with blockIdx.x below this prefetch their tile into L2 before
+    // waiting for the previous grid: the first wave of resident blocks, which
+    // overlaps that grid's tail.  Later blocks start once it has finished and
+    // load directly (their prefetch would only add L2 requests).
+    long long pf_blocks = 1ll << 62;
 };
 
 // Where a thread's V elements sit in their rows, as bit masks over k:
@@ -783,7 +788,7 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     // complete before touching memory).
     {
         const long long mg = kBwd ? (g.ntiles - 1 - j) : j;
-        Est::prefetch(P, g, mg * (long long)(NT * V), NT * V);
+        if ((long long)blockIdx.x < g.pf_blocks) Est::prefetch(P, g, mg * (long long)(NT * V), NT * V);
     }
     griddep_wait();
     griddep_launch_dependents();
