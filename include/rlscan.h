@@ -42,9 +42,11 @@
  *   - Workspace: long rows (a row that spans several tiles) and rows that do
  *     not align with tiles need a device workspace of
  *     rlscan_workspace_bytes(E, T) bytes, 16-byte aligned, of any content
- *     (such a call runs two launches: the first writes one 16-byte aggregate
- *     per tile, the second scans each tile with the carry it composes from
- *     them; no kernel ever waits for another block).  Shapes that need none
+ *     (such a call runs two launches over chunks of consecutive elements, one
+ *     chunk per warp: the first writes each chunk's 16-byte aggregate, the
+ *     second scans each chunk with the carry it composes from the
+ *     aggregates of the chunks before it; no kernel ever waits for another
+ *     block or warp).  Shapes that need none
  *     accept ws = NULL.  A workspace holds one call's aggregates between its
  *     two launches: calls that share one must be ordered on one stream (or
  *     otherwise serialised).
@@ -288,9 +290,10 @@ RLSCAN_API int rlscan_episodic_prefix_sum(const void *x, int dtype, const float 
  * resets a device must not call this entry point on it again.  Every call
  * clears the part of the array it uses with cudaMemsetAsync on `stream` and
  * allocates nothing.
- * Limit: shapes whose tile plan needs more scratch than the array holds
- * (rows split over more than about 65,000 tiles) return RLSCAN_ERR_WORKSPACE
- * with the sizes in rlscan_last_error().
+ * Limit: shapes whose plan needs more scratch than the array holds (rows
+ * that span tiles, over more than about 33 million elements in all: one
+ * 16-byte slot per 512 elements) return RLSCAN_ERR_WORKSPACE with the sizes
+ * in rlscan_last_error().
  * All calls on one device share that device's array, which keeps the last
  * call's contents: two calls whose kernels may run at the same time on one
  * device (for example on two streams with no ordering between them) race on
@@ -469,7 +472,7 @@ RLSCAN_API int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size
 
 /*
  * Workspace size in bytes that any entry point above needs for an [E, T]
- * problem (any A): 16 bytes per tile when rows span tiles, 0 when no call of
+ * problem (any A): 16 bytes per 512 elements when rows span tiles, 0 when no call of
  * that shape needs one.  Negative or overflowing shapes return 0 and the
  * compute call then rejects them.
  */
@@ -495,7 +498,10 @@ RLSCAN_API int rlscan_version(void);
 /*
  * Launch plan that a call of this shape takes (for tests and tools):
  * writes tile size in elements, threads per block, whether tiles exchange
- * carries through the workspace (1) or not (0), and the tile count.
+ * carries through the workspace (1) or not (0), and the tile count.  For
+ * rows that span tiles (1) the call runs the chunked two passes: it writes
+ * the workspace's granularity (512 elements a slot), the passes' block size
+ * and the workspace's slot count, an upper bound on the chunks.
  * actions: 1 for every estimator except rlscan_retrace with A > 1, whose
  * action count it is (1 .. RLSCAN_MAX_ACTIONS); every call scans on the same
  * plans, multi-action Retrace after a first launch that writes its expected

@@ -189,7 +189,7 @@ int rlscan_gae_noalloc(const float *rewards, const float *values, const float *t
                         {last_values, (size_t)E * 4, "last_values"}};
     const Span outs[] = {{advantages, pb, "advantages"}};
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 1));
-    const size_t need = workspace_for(make_plan(E, T));
+    const size_t need = workspace_for(make_plan(E, T), E * T);
     if (need > RLSCAN_NOALLOC_SCRATCH_BYTES)
         return fail(RLSCAN_ERR_WORKSPACE,
                     "rlscan_gae_noalloc: shape E=%lld T=%lld needs %zu bytes of scratch; the fixed scratch holds %u",
@@ -197,8 +197,8 @@ int rlscan_gae_noalloc(const float *rewards, const float *values, const float *t
     void *ws = nullptr;
     if (need > 0) {
         RLSCAN_TRY(noalloc_scratch(&ws));
-        // the array keeps the previous call's contents: the tile counters and
-        // flags this call uses must start at zero
+        // the array keeps the previous call's contents: cleared, so that
+        // each call starts from the same state as with a fresh workspace
         cudaError_t e = cudaMemsetAsync(ws, 0, need, stream);
         if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
     }

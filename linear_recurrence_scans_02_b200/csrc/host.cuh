@@ -192,9 +192,11 @@ inline bool aligned16(std::initializer_list<const void *> ptrs) {
     return true;
 }
 
-// One 16-byte slot per tile (its aggregate, then its inclusive value) when
-// rows span tiles; nothing otherwise.
-inline size_t workspace_for(const Plan &p) { return p.lookback ? sizeof(TileSlot) * (size_t)p.ntiles : 0; }
+// Rows that span tiles: one 16-byte slot per chunk of the chunked two
+// passes, at most one per 512 elements; nothing otherwise.
+inline size_t workspace_for(const Plan &p, long long n) {
+    return p.lookback ? sizeof(TileSlot) * (size_t)ceil_div(n, 2LL * 32 * kChunkV) : 0;
+}
 
 // ---------------------------------------------------------------------------
 // Argument checks
@@ -339,36 +341,55 @@ inline long long streamed_input_bytes(const typename Est::Params &P) {
     return b;
 }
 
-// Rows that span tiles: pass one (aggregates) and pass two (scan with
-// carries) over waves of consecutive scan-order tiles, as few waves as keep
-// each wave's inputs within kTwoPassWaveBytes, of equal size.
-template <class Est>
-int run_two_pass(const char *name, const typename Est::Params &P, const Geometry &g, Lookback lb, Cfg cfg,
-                 cudaStream_t stream) {
-    const long long in_bytes = std::max<long long>(1, streamed_input_bytes<Est>(P)) * g.n;
-    const long long wave = ceil_div(g.ntiles, ceil_div(in_bytes, kTwoPassWaveBytes));
-    for (long long t0 = 0; t0 < g.ntiles; t0 += wave) {
-        lb.tile_base = t0;
-        const long long cnt = std::min<long long>(wave, g.ntiles - t0);
-        for (int mode : {kModeReduce, kModeCarry}) {
-            cudaError_t e;
-            if constexpr (NarrowOf<Est>::value) {
-                switch (cfg) {
-                case N512: e = launch_cfg<Est, N512>(P, g, lb, mode, 0, stream, cnt); break;
-                case N1024: e = launch_cfg<Est, N1024>(P, g, lb, mode, 0, stream, cnt); break;
-                case N2048: e = launch_cfg<Est, N2048>(P, g, lb, mode, 0, stream, cnt); break;
-                default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
-                }
-            } else {
-                switch (cfg) {
-                case C512: e = launch_cfg<Est, C512>(P, g, lb, mode, 0, stream, cnt); break;
-                case C1024: e = launch_cfg<Est, C1024>(P, g, lb, mode, 0, stream, cnt); break;
-                case C2048: e = launch_cfg<Est, C2048>(P, g, lb, mode, 0, stream, cnt); break;
-                default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
-                }
-            }
-            if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
+// Resident blocks per SM of a kernel, queried once per kernel.
+template <class K>
+inline int resident_blocks(K kern, int threads, int &cache) {
+    if (cache == 0) {
+        int r = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, threads, 0) != cudaSuccess || r < 1) {
+            (void)cudaGetLastError();
+            r = 1;
         }
+        cache = r;
+    }
+    return cache;
+}
+
+// Rows that span tiles: the chunked two passes (chunk_scan_kernel).  One
+// chunk per warp the GPU holds at once (at least two steps a chunk, so the
+// chunks fit the workspace of workspace_for), over as few waves as keep each
+// wave's inputs within kTwoPassWaveBytes.
+template <class Est>
+int run_chunked(const char *name, const typename Est::Params &P, const Geometry &g, TileSlot *slots,
+                cudaStream_t stream) {
+    constexpr long long SW = 32LL * kChunkV;
+    constexpr int WPB = kChunkNT / 32;
+    static int res_cache = 0;
+    const long long resident = resident_blocks(chunk_scan_kernel<Est, kChunkScan>, kChunkNT, res_cache);
+    const long long warps = (long long)num_sms() * resident * WPB;
+    const long long nsteps = ceil_div(g.n, SW);
+    const long long in_bytes = std::max<long long>(1, streamed_input_bytes<Est>(P)) * g.n;
+    const long long nwaves = ceil_div(in_bytes, kTwoPassWaveBytes);
+    const long long wave_steps = ceil_div(nsteps, nwaves);
+    const long long chunk_steps = std::max<long long>(2, ceil_div(wave_steps, warps));
+    const long long nchunks = ceil_div(nsteps, chunk_steps);
+    const long long wave_chunks = ceil_div(wave_steps, chunk_steps);
+    ChunkSplit cs{slots, nsteps, chunk_steps, 0, 0, (long long)num_sms() * resident};
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kChunkNT);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    for (long long c0 = 0; c0 < nchunks; c0 += wave_chunks) {
+        cs.chunk_begin = c0;
+        cs.chunk_end = std::min(nchunks, c0 + wave_chunks);
+        cfg.gridDim = dim3((unsigned)ceil_div(cs.chunk_end - cs.chunk_begin, (long long)WPB));
+        cudaError_t e = cudaLaunchKernelEx(&cfg, chunk_scan_kernel<Est, kChunkAggregates>, P, g, cs);
+        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, chunk_scan_kernel<Est, kChunkScan>, P, g, cs);
+        if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
     }
     return ok();
 }
@@ -387,7 +408,7 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
     g.scan_lanes = scan_lanes_for(plan, T);
     Lookback lb{};
     if (plan.lookback) {
-        const size_t need = workspace_for(plan);
+        const size_t need = workspace_for(plan, E * T);
         if (ws == nullptr || ws_bytes < need)
             return fail(RLSCAN_ERR_WORKSPACE, "%s: shape E=%lld T=%lld needs a %zu-byte workspace (got %s, %zu bytes)",
                         name, E, T, need, ws ? "a buffer" : "NULL", ws_bytes);
@@ -411,7 +432,7 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
             return ok();
         }
     }
-    if (plan.lookback) return run_two_pass<Est>(name, P, g, lb, plan.cfg, stream);
+    if (plan.lookback) return run_chunked<Est>(name, P, g, lb.slots, stream);
     cudaError_t e;
     if constexpr (NarrowOf<Est>::value) {
         switch (plan.cfg) {

@@ -66,7 +66,7 @@ int rlscan_retrace_ex(const float *rewards, const float *q_values, const float *
         // checks of the scan's own (workspace) come first: nothing is enqueued
         // if the call is rejected
         const Plan plan = make_plan(E, T);
-        if (plan.lookback && (ws == nullptr || ws_bytes < workspace_for(plan) || ((uintptr_t)ws & 15u) != 0))
+        if (plan.lookback && (ws == nullptr || ws_bytes < workspace_for(plan, E * T) || ((uintptr_t)ws & 15u) != 0))
             return run<RetraceEst>("rlscan_retrace", P, E, T, ws, ws_bytes, stream, vec);
         const cudaError_t e = launch_expected_values(next_q_values_all, next_target_probs, q_ret, E * T, A, stream);
         if (e != cudaSuccess)
@@ -84,7 +84,7 @@ int rlscan_retrace(const float *rewards, const float *q_values, const float *nex
 
 size_t rlscan_workspace_bytes(int64_t E, int64_t T) {
     if (E <= 0 || T <= 0 || E > kMaxElems / T) return 0;
-    return std::max(workspace_for(make_plan(E, T)), tm_workspace_for(E, T));
+    return std::max(workspace_for(make_plan(E, T), E * T), tm_workspace_for(E, T));
 }
 
 int rlscan_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream) {
@@ -113,10 +113,14 @@ int rlscan_plan(int64_t E, int64_t T, int64_t actions, int64_t *tile_elems, int 
     if (actions < 1 || actions > RLSCAN_MAX_ACTIONS) return fail(RLSCAN_ERR_INVALID_ARG, "bad action count");
     RLSCAN_TRY(check_shape(E, T, actions));
     const Plan p = make_plan(E, T); // every call scans on the single-action plan
-    if (tile_elems) *tile_elems = kCfgTile[p.cfg];
-    if (threads) *threads = kCfgThreads[p.cfg];
+    // rows that span tiles run the chunked two passes: report the workspace's
+    // granularity (one slot per 512 elements) and its slot count, an upper
+    // bound on the chunks (their number depends on the device)
+    const long long slot_elems = 2LL * 32 * kChunkV;
+    if (tile_elems) *tile_elems = p.lookback ? slot_elems : kCfgTile[p.cfg];
+    if (threads) *threads = p.lookback ? kChunkNT : kCfgThreads[p.cfg];
     if (lookback) *lookback = p.lookback ? 1 : 0;
-    if (num_tiles) *num_tiles = p.ntiles;
+    if (num_tiles) *num_tiles = p.lookback ? ceil_div(E * T, slot_elems) : p.ntiles;
     return ok();
 }
 

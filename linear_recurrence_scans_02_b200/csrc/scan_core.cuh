@@ -911,6 +911,211 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
 }
 
 // ---------------------------------------------------------------------------
+// Rows that span tiles: chunked two passes.  The flattened array is cut into
+// warp steps of 32 V consecutive elements (lane l owns V of them), and the
+// steps, in scan order, into equal chunks of consecutive steps, one chunk per
+// warp.  A warp walks its chunk step by step and carries its running value
+// from one step to the next itself, so no block barrier and no other warp is
+// involved inside a chunk:
+//   pass one (kChunkAggregates): compose the maps of the chunk's steps into
+//     the chunk's aggregate and write it to the chunk's 16-byte slot;
+//   pass two (kChunkScan), the next launch on the stream: compose the
+//     aggregates of the earlier chunks up to the first that cuts the chain
+//     (an episode or row start, a == 0, or the array's start) into the
+//     chunk's carry, then scan the steps again with that carry, writing the
+//     outputs.
+// Every slot pass two reads was written by pass one, which has completed
+// before pass two reads it, so nothing waits and the workspace needs no
+// initial content.  A launch covers the chunks [chunk_begin, chunk_end), so a
+// long array runs in waves whose inputs pass two finds in L2.
+// ---------------------------------------------------------------------------
+constexpr int kChunkNT = 128; // 4 independent warps per block
+constexpr int kChunkV = 8;    // elements per lane and step
+constexpr int kChunkAggregates = 0;
+constexpr int kChunkScan = 1;
+
+struct ChunkSplit {
+    TileSlot *slots;       // one per chunk, in scan order
+    long long nsteps;      // warp steps over the array: ceil(n / (32 V))
+    long long chunk_steps; // steps per chunk (the last chunk may hold fewer)
+    long long chunk_begin; // this launch's chunks
+    long long chunk_end;
+    long long pf_blocks;   // blocks that prefetch their chunks into L2 before the grid wait
+};
+
+// The aggregate a chunk slot holds (pass one writes all 16 bytes).
+template <class AT, class BT>
+__device__ __forceinline__ void read_aggregate(const TileSlot *slot, AT &a, BT &b) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(slot);
+    a = from_bits(v.x, a);
+    b = from_bits(v.y, b);
+}
+__device__ __forceinline__ void read_aggregate(const TileSlot *slot, float2 &a, float2 &b) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(slot);
+    a = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+    b = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+
+// Carry into chunk c: the composition of the aggregates of chunks c-1, c-2,
+// ... up to the first that cuts the chain, applied to the identity value.
+// Called by all 32 lanes of one warp; each round trip reads 32 x M slots
+// (lane i: chunks base - i M - m, m = 0 .. M-1, nearest first).
+template <class AT, class BT>
+__device__ BT chunk_carry(const TileSlot *slots, long long c, int lane, AT proto_a, BT proto_b) {
+    constexpr int M = kSlotsPerLane;
+    AT acc_a = identity_a(proto_a);
+    BT acc_b = identity_b(proto_b);
+    for (long long base = c - 1;; base -= 32 * M) {
+        const long long k0 = base - (long long)lane * M;
+        AT sa[M];
+        BT sb[M];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            sa[m] = cut_a(proto_a); // before the array's start: nothing flows in
+            sb[m] = identity_b(proto_b);
+            if (k0 - m >= 0) read_aggregate(slots + (k0 - m), sa[m], sb[m]);
+        }
+        AT la = identity_a(proto_a);
+        BT lb = identity_b(proto_b);
+        bool stop = false;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            if (!stop) {
+                combine(la, lb, sa[m], sb[m]);
+                stop = is_cut(sa[m]);
+            }
+        }
+        const unsigned stops = __ballot_sync(kFullMask, stop);
+        const int last = stops ? __ffs(stops) - 1 : 31;
+        if (lane > last) { // farther than the nearest stop: contributes nothing
+            la = identity_a(proto_a);
+            lb = identity_b(proto_b);
+        }
+        // ordered composition over lanes 0..last: lane 0 (nearest) applied last
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const AT oa = shfl_down(la, d);
+            const BT ob = shfl_down(lb, d);
+            if (lane + d < 32) combine(la, lb, oa, ob);
+        }
+        la = shfl_idx(la, 0);
+        lb = shfl_idx(lb, 0);
+        combine(acc_a, acc_b, la, lb);
+        if (stops) return acc_b;
+    }
+}
+
+template <class Est, int kPass>
+__global__ void __launch_bounds__(kChunkNT) chunk_scan_kernel(const typename Est::Params P, const Geometry g,
+                                                              const ChunkSplit cs) {
+    using AT = typename Est::AT;
+    using BT = typename Est::BT;
+    constexpr int V = kChunkV;
+    constexpr bool kBwd = Est::kBackward;
+    constexpr long long SW = 32LL * V; // elements per warp step
+    constexpr int WPB = kChunkNT / 32;
+    const int lane = threadIdx.x & 31;
+    const long long c = cs.chunk_begin + (long long)blockIdx.x * WPB + (threadIdx.x >> 5);
+
+    // L2 prefetch of the block's chunks (consecutive in memory) before
+    // waiting for the previous grid, by the first wave of blocks
+    if ((long long)blockIdx.x < cs.pf_blocks) {
+        const long long cb = cs.chunk_begin + (long long)blockIdx.x * WPB;
+        const long long ce = min(cs.chunk_end, cb + WPB);
+        const long long sb = cb * cs.chunk_steps, se = min(cs.nsteps, ce * cs.chunk_steps);
+        if (se > sb) {
+            const long long m0 = kBwd ? cs.nsteps - se : sb; // first memory step of the range
+            Est::prefetch(P, g, m0 * SW, (int)min((se - sb) * SW, 1LL << 18)); // at most 1 MB a plane
+        }
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    if (c >= cs.chunk_end) return; // the whole warp
+
+    const long long s0 = c * cs.chunk_steps;
+    const long long s1 = min(cs.nsteps, s0 + cs.chunk_steps);
+    AT agg_a = identity_a(AT{});
+    BT agg_b = identity_b(BT{});
+    BT carry = identity_b(BT{});
+    if constexpr (kPass == kChunkScan) carry = chunk_carry<AT, BT>(cs.slots, c, lane, AT{}, BT{});
+
+    for (long long s = s0; s < s1; ++s) {
+        const long long m = kBwd ? (cs.nsteps - 1 - s) : s; // step in memory order
+        const long long i0 = m * SW + (long long)lane * V;
+        const RowMajorPos<V> pos{i0, g.n, g.vec_ok != 0 && i0 + V <= g.n, lane};
+        typename Est::template State<V> S;
+        Est::template load<32, V>(P, g, pos, S, nullptr);
+        AT a[V];
+        BT b[V];
+        const RowMasks rm = row_masks<V>(i0, g);
+        Est::template coeffs<V>(P, g, pos, rm, S, a, b);
+
+        // lane map, composed in scan order
+        AT ta;
+        BT tb;
+        if (kBwd) {
+            ta = a[V - 1];
+            tb = b[V - 1];
+#pragma unroll
+            for (int k = V - 2; k >= 0; --k) {
+                AT na = a[k];
+                BT nb = b[k];
+                combine(na, nb, ta, tb);
+                ta = na;
+                tb = nb;
+            }
+        } else {
+            ta = a[0];
+            tb = b[0];
+#pragma unroll
+            for (int k = 1; k < V; ++k) {
+                AT na = a[k];
+                BT nb = b[k];
+                combine(na, nb, ta, tb);
+                ta = na;
+                tb = nb;
+            }
+        }
+        AT ia = ta;
+        BT ib = tb;
+        warp_inclusive_scan<kBwd>(ia, ib, lane);
+        // the step's map: the inclusive value of its last lane in scan order
+        AT sa = shfl_idx(ia, kBwd ? 0 : 31);
+        BT sb = shfl_idx(ib, kBwd ? 0 : 31);
+        if constexpr (kPass == kChunkAggregates) {
+            combine(sa, sb, agg_a, agg_b); // this step after the earlier ones
+            agg_a = sa;
+            agg_b = sb;
+        } else {
+            AT ea;
+            BT eb;
+            warp_exclusive_from_inclusive<kBwd>(ia, ib, lane, ea, eb);
+            BT x = apply_pair(ea, eb, carry);
+            if (kBwd) {
+#pragma unroll
+                for (int k = V - 1; k >= 0; --k) {
+                    const BT prev = x;
+                    x = apply_pair(a[k], b[k], x);
+                    Est::template out<V>(P, S, k, x, prev, b[k]);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < V; ++k) {
+                    const BT prev = x;
+                    x = apply_pair(a[k], b[k], x);
+                    Est::template out<V>(P, S, k, x, prev, b[k]);
+                }
+            }
+            Est::template store<V>(P, g, pos, S);
+            carry = apply_pair(sa, sb, carry);
+        }
+    }
+    if constexpr (kPass == kChunkAggregates) {
+        if (lane == 0) publish_aggregate(cs.slots + c, agg_a, agg_b);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // The time-major kernel, for [T, E] arrays (E contiguous).  A block owns G
 // consecutive envs and walks their rows in segments, in scan order.  Within
 // a warp, lane l serves env l % G and chunk l / G: the warp covers 32 / G

@@ -58,7 +58,7 @@ int typed_retrace(const rlscan_call &c, void *ws, size_t ws_bytes, cudaStream_t 
         const bool vec = aligned16({in[0], in[1], in[4], in[5], in[6], q_ret});
         if (!batch_dry()) {
             const Plan plan = make_plan(c.E, c.T);
-            if (plan.lookback && (ws == nullptr || ws_bytes < workspace_for(plan) || ((uintptr_t)ws & 15u) != 0))
+            if (plan.lookback && (ws == nullptr || ws_bytes < workspace_for(plan, c.E * c.T) || ((uintptr_t)ws & 15u) != 0))
                 return run<Est>(name, P, c.E, c.T, ws, ws_bytes, stream, vec); // reports the workspace error
             const cudaError_t e = launch_expected_values(static_cast<const VT *>(in[2]),
                                                          static_cast<const VT *>(in[3]), q_ret, c.E * c.T, A, stream);

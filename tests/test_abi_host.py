@@ -303,10 +303,12 @@ def test_batch_call_layout_matches_the_header(tmp_path):
     (64, 512, 1024, 128, False),
     (4096, 2048, 2048, 256, False),    # a row needs a bigger tile to stay whole
     (256, 4096, 4096, 512, False),
-    (16, 262144, 2048, 256, True),     # long rows: the look-back over 2048-element tiles
-    (1024, 8192, 2048, 256, True),
-    (3, 70000, 512, 128, True),        # few tiles: 512-element tiles (4 per thread)
-    (4096, 129, 1024, 128, True),      # rows not dividing any tile
+    # rows that span tiles: the chunked two passes (128-thread blocks of
+    # independent warps), reported as one workspace slot per 512 elements
+    (16, 262144, 512, 128, True),      # long rows
+    (1024, 8192, 512, 128, True),
+    (3, 70000, 512, 128, True),
+    (4096, 129, 512, 128, True),       # rows not dividing any tile
 ])
 def test_plan_choices(lib, E_, T_, tile, threads, lookback):
     # the launch plans the measurements in the design notes were taken with
