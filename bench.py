@@ -1104,7 +1104,7 @@ def run_profile_case(args):
         R.rlscan_check()
         print(f"profile case done: {args.profile_launches} multi-action Retrace launches at 256 x 2048 x 18")
         return 0
-    if args.profile_shape:  # GAE at another shape, e.g. 16,262144 (long rows: the two-pass path)
+    if args.profile_shape:  # GAE at another shape, e.g. 16,262144 (long rows: the chunked two passes)
         from linear_recurrence_scans_02_b200 import workloads as W
         E, T = (int(v) for v in args.profile_shape.split(","))
         tm = args.profile_time_major

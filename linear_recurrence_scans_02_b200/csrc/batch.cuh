@@ -183,8 +183,7 @@ struct FusedBatch {
 template <class Est, int V, int kMode>
 __device__ __forceinline__ void fused_tile(const FusedItem &it, long long block, unsigned char *smem) {
     const auto &P = *reinterpret_cast<const typename Est::Params *>(it.params);
-    const Lookback lb{}; // whole rows per tile: no carries between tiles
-    tile_scan_body<Est, kFusedNT, V, kMode>(P, it.g, lb, block, smem);
+    tile_scan_body<Est, kFusedNT, V, kMode>(P, it.g, block, smem);
 }
 
 template <class Est, int V>

@@ -5,7 +5,7 @@
 
 #include "host.cuh"
 
-// Fixed scratch of rlscan_gae_noalloc: the look-back workspace for callers
+// Fixed scratch of rlscan_gae_noalloc: the split-row workspace for callers
 // that cannot allocate one.  In host code this name is only a handle for
 // cudaGetSymbolAddress, never an address to pass to a kernel.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RLSCAN_NOALLOC_SCRATCH_BYTES];

@@ -2,8 +2,8 @@
 // status and message helpers, argument checks, tile plans, batch-request
 // state, and the launch helpers that instantiate the kernels (each
 // translation unit instantiates the kernels of the estimators it serves).
-// State shared by all units (the thread's last error message, the look-back
-// test hooks, the SM counts, the batch request being served) is held in
+// State shared by all units (the thread's last error message, the SM
+// counts, the batch request being served) is held in
 // inline variables, one instance per process.
 #pragma once
 
@@ -51,39 +51,27 @@ inline bool pdl_enabled() {
 
 // ---------------------------------------------------------------------------
 // Tile plans.  A tile is S = NT * V consecutive elements of the flattened
-// [E*T] array.  Tiles need carries from earlier tiles (the two passes) only
+// [E*T] array.  Rows need carries across tiles (the chunked two passes) only
 // when a tile boundary can fall inside a row (S not a multiple of T, more
 // than one tile).
 // ---------------------------------------------------------------------------
 // Eight elements per thread keeps a grid's share of each SM small, so the
 // next launch on the stream can be resident (and prefetching) while this one
-// runs; the 512-element tile (four per thread) is for small split-row plans.
-// N512 .. N4096 are the same tiles at 16 elements per thread (half the
-// threads), for calls whose value planes are 2 bytes wide: each thread then
-// keeps as many bytes in flight as an fp32 thread of the twin tile.
-enum Cfg { C512 = 0, C1024, C2048, C4096, N512, N1024, N2048, N4096, kNumCfg };
-constexpr int kCfgTile[kNumCfg] = {512, 1024, 2048, 4096, 512, 1024, 2048, 4096};
-constexpr int kCfgThreads[kNumCfg] = {128, 128, 256, 512, 32, 64, 128, 256};
-
-// Whether an estimator reads 2-byte value planes (takes the N configs).
-template <class Est>
-struct NarrowOf {
-    static constexpr bool value = false;
-};
-template <bool R, class V, class F> struct NarrowOf<GaeEstT<R, V, F>> { static constexpr bool value = sizeof(V) == 2; };
-template <class V, class F> struct NarrowOf<VtraceEstT<V, F>> { static constexpr bool value = sizeof(V) == 2; };
-template <class V, class F> struct NarrowOf<LambdaReturnsEstT<V, F>> { static constexpr bool value = sizeof(V) == 2; };
-template <class V, class F> struct NarrowOf<ReturnsEstT<V, F>> { static constexpr bool value = sizeof(V) == 2; };
-template <class V, class F, class N> struct NarrowOf<RetraceEstT<V, F, N>> { static constexpr bool value = sizeof(V) == 2; };
-template <class V, class F> struct NarrowOf<ForwardEstT<V, F>> { static constexpr bool value = sizeof(V) == 2; };
-constexpr Cfg narrow_twin(Cfg c) { return c <= C4096 ? (Cfg)(c + N512) : c; }
+// runs; the 512-element tile (four per thread) is for small plans.  Calls on
+// 2-byte value planes take the same tiles (measured at 4096 x 128 and 65536
+// x 128: 8 elements per thread in 128-thread blocks beat 16 elements per
+// thread in half as many threads, 23.7 against 28.9 us for bf16 / uint8 GAE
+// + returns at 65536 x 128).
+enum Cfg { C512 = 0, C1024, C2048, C4096, kNumCfg };
+constexpr int kCfgTile[kNumCfg] = {512, 1024, 2048, 4096};
+constexpr int kCfgThreads[kNumCfg] = {128, 128, 256, 512};
 
 struct Plan {
     Cfg cfg;
     bool lookback;
     long long ntiles;
     int mode; // kModeBlock / kModeWarp (whole rows per tile); rows that span
-              // tiles take the two passes (kModeReduce, kModeCarry)
+              // tiles (lookback) take the chunked two passes instead
 };
 
 // Scan mode of a whole-row plan: warp-local when every warp's 32*V elements
@@ -154,9 +142,8 @@ inline Plan make_plan_tiles(long long E, long long T) {
         break;
     }
     // rows span tiles (long or odd-length rows, or too few rows to fill the
-    // GPU): two passes over 2048-element tiles (fewer tiles per row, so
-    // shorter walks over the aggregates), 1024 or 512 when that gives too few
-    // tiles
+    // GPU): the chunked two passes (run_chunked), unless the whole array fits
+    // one tile
     p.cfg = ceil_div(n, kCfgTile[C2048]) >= min_tiles
                 ? C2048
                 : (ceil_div(n, kCfgTile[C1024]) >= min_tiles ? C1024 : C512);
@@ -166,15 +153,6 @@ inline Plan make_plan_tiles(long long E, long long T) {
 }
 
 inline Plan make_plan(long long E, long long T) { return with_mode(make_plan_tiles(E, T), T); }
-
-// The plan an estimator runs: narrow-value estimators take the twin of the
-// plan's tile at 16 elements per thread (same tiles, same workspace).
-template <class Est>
-inline Plan make_plan_for(long long E, long long T) {
-    Plan p = make_plan_tiles(E, T);
-    if constexpr (NarrowOf<Est>::value) p.cfg = narrow_twin(p.cfg);
-    return with_mode(p, T);
-}
 
 // Warp-local mode: a row spans T / V lanes (T a power of two dividing 32 V);
 // the shuffle scan needs to reach that far only.
@@ -274,15 +252,14 @@ inline bool batch_dry() { return g_batch != nullptr && g_batch->pass == kBatchDr
 // Launch
 // ---------------------------------------------------------------------------
 template <class Est, int NT, int V, int kMode>
-cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const Lookback &lb, size_t smem,
-                       cudaStream_t stream, long long grid = -1) {
+cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, size_t smem, cudaStream_t stream) {
     auto kern = tile_scan_kernel<Est, NT, V, kMode>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(grid < 0 ? g.ntiles : grid));
+    cfg.gridDim = dim3((unsigned)g.ntiles);
     cfg.blockDim = dim3(NT);
     // resident blocks per SM of this kernel, queried once
     static int resident = 0;
@@ -303,26 +280,15 @@ cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, const L
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, P, gl, lb);
+    return cudaLaunchKernelEx(&cfg, kern, P, gl);
 }
 
 template <class Est, Cfg C>
-cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, const Lookback &lb, int mode,
-                       size_t smem, cudaStream_t s, long long grid = -1) {
+cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, int mode, size_t smem, cudaStream_t s) {
     constexpr int NT = kCfgThreads[C];
     constexpr int V = kCfgTile[C] / NT;
-    switch (mode) {
-    case kModeWarp: return launch_one<Est, NT, V, kModeWarp>(P, g, lb, smem, s);
-    case kModeReduce:
-    case kModeCarry:
-        // split-row plans use 512- to 2048-element tiles (make_plan_tiles)
-        if constexpr (C == C512 || C == C1024 || C == C2048 || C == N512 || C == N1024 || C == N2048) {
-            if (mode == kModeReduce) return launch_one<Est, NT, V, kModeReduce>(P, g, lb, smem, s, grid);
-            return launch_one<Est, NT, V, kModeCarry>(P, g, lb, smem, s, grid);
-        }
-        return cudaErrorInvalidConfiguration;
-    default: return launch_one<Est, NT, V, kModeBlock>(P, g, lb, smem, s);
-    }
+    if (mode == kModeWarp) return launch_one<Est, NT, V, kModeWarp>(P, g, smem, s);
+    return launch_one<Est, NT, V, kModeBlock>(P, g, smem, s);
 }
 
 // Input bytes a two-pass wave may hold so that pass two re-reads them from
@@ -364,8 +330,10 @@ int run_chunked(const char *name, const typename Est::Params &P, const Geometry 
                 cudaStream_t stream) {
     constexpr long long SW = 32LL * kChunkV;
     constexpr int WPB = kChunkNT / 32;
-    static int res_cache = 0;
-    const long long resident = resident_blocks(chunk_scan_kernel<Est, kChunkScan>, kChunkNT, res_cache);
+    // both passes run on the same grid, which the GPU holds at once
+    static int res_a = 0, res_b = 0;
+    const long long resident = std::min(resident_blocks(chunk_scan_kernel<Est, kChunkAggregates>, kChunkNT, res_a),
+                                        resident_blocks(chunk_scan_kernel<Est, kChunkScan>, kChunkNT, res_b));
     const long long warps = (long long)num_sms() * resident * WPB;
     const long long nsteps = ceil_div(g.n, SW);
     const long long in_bytes = std::max<long long>(1, streamed_input_bytes<Est>(P)) * g.n;
@@ -397,7 +365,7 @@ int run_chunked(const char *name, const typename Est::Params &P, const Geometry 
 template <class Est>
 int run(const char *name, const typename Est::Params &P, long long E, long long T, void *ws, size_t ws_bytes,
         cudaStream_t stream, bool vec_ok) {
-    const Plan plan = make_plan_for<Est>(E, T);
+    const Plan plan = make_plan(E, T);
     Geometry g;
     g.n = E * T;
     g.seq_len = T;
@@ -406,15 +374,14 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
     g.t_shift = pow2_shift(T);
     g.vec_ok = vec_ok ? 1 : 0;
     g.scan_lanes = scan_lanes_for(plan, T);
-    Lookback lb{};
+    TileSlot *slots = nullptr;
     if (plan.lookback) {
         const size_t need = workspace_for(plan, E * T);
         if (ws == nullptr || ws_bytes < need)
             return fail(RLSCAN_ERR_WORKSPACE, "%s: shape E=%lld T=%lld needs a %zu-byte workspace (got %s, %zu bytes)",
                         name, E, T, need, ws ? "a buffer" : "NULL", ws_bytes);
         if (((uintptr_t)ws & 15u) != 0) return fail(RLSCAN_ERR_WORKSPACE, "%s: workspace must be 16-byte aligned", name);
-        lb.slots = static_cast<TileSlot *>(ws);
-        lb.row_tiles = (T % kCfgTile[plan.cfg] == 0) ? T / kCfgTile[plan.cfg] : 0;
+        slots = static_cast<TileSlot *>(ws);
     }
     if (batch_dry()) return ok();
     if constexpr (FusedBodyOf<Est>::value >= 0) {
@@ -432,24 +399,14 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
             return ok();
         }
     }
-    if (plan.lookback) return run_chunked<Est>(name, P, g, lb.slots, stream);
+    if (plan.lookback) return run_chunked<Est>(name, P, g, slots, stream);
     cudaError_t e;
-    if constexpr (NarrowOf<Est>::value) {
-        switch (plan.cfg) {
-        case N512: e = launch_cfg<Est, N512>(P, g, lb, plan.mode, 0, stream); break;
-        case N1024: e = launch_cfg<Est, N1024>(P, g, lb, plan.mode, 0, stream); break;
-        case N2048: e = launch_cfg<Est, N2048>(P, g, lb, plan.mode, 0, stream); break;
-        case N4096: e = launch_cfg<Est, N4096>(P, g, lb, plan.mode, 0, stream); break;
-        default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
-        }
-    } else {
-        switch (plan.cfg) {
-        case C512: e = launch_cfg<Est, C512>(P, g, lb, plan.mode, 0, stream); break;
-        case C1024: e = launch_cfg<Est, C1024>(P, g, lb, plan.mode, 0, stream); break;
-        case C2048: e = launch_cfg<Est, C2048>(P, g, lb, plan.mode, 0, stream); break;
-        case C4096: e = launch_cfg<Est, C4096>(P, g, lb, plan.mode, 0, stream); break;
-        default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
-        }
+    switch (plan.cfg) {
+    case C512: e = launch_cfg<Est, C512>(P, g, plan.mode, 0, stream); break;
+    case C1024: e = launch_cfg<Est, C1024>(P, g, plan.mode, 0, stream); break;
+    case C2048: e = launch_cfg<Est, C2048>(P, g, plan.mode, 0, stream); break;
+    case C4096: e = launch_cfg<Est, C4096>(P, g, plan.mode, 0, stream); break;
+    default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
     }
     if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
     return ok();

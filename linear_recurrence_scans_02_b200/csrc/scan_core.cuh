@@ -13,9 +13,10 @@
 //     row's last value is folded into b there), the same cut a done makes;
 //   * in-thread sequential compose -> warp shuffle scan -> shared-memory scan
 //     of warp aggregates -> per-thread carry -> sequential epilogue;
-//   * when rows span tiles, two launches: the first writes every tile's
-//     aggregate, the second scans each tile with the carry composed from the
-//     complete aggregates of the tiles before it (no block ever waits for
+//   * when rows span tiles, two launches over chunks of consecutive warp
+//     steps, one chunk per warp: the first writes every chunk's aggregate,
+//     the second scans each chunk with the carry composed from the complete
+//     aggregates of the chunks before it (no block or warp ever waits for
 //     another).
 //
 // Scan order is memory order for forward recurrences and reversed memory
@@ -43,16 +44,6 @@ constexpr unsigned kFullMask = 0xffffffffu;
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// Four relaxed 32-bit loads in one instruction (no ordering among them).
-__device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const void *p) {
-    uint4 v;
-    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p)
-                 : "memory");
-    return v;
 }
 
 // Hint: bring [p + first, p + first + count) elements of a plane into L2.  The
@@ -179,21 +170,15 @@ __device__ __forceinline__ void warp_exclusive_from_inclusive(AT ia, BT ib, int 
 }
 
 // ---------------------------------------------------------------------------
-// Workspace of a split-row call: one 16-byte slot per tile.  Pass one writes
-// the tile's aggregate {a, b} in the first half; pass two may publish the
-// tile's inclusive value {1, x} in the second half (see the two-pass carries
-// below).
+// Workspace slot of a split-row call (one per chunk of the chunked two
+// passes; one per env and split of a time-major call whose rows are split
+// over blocks): a map's aggregate, {a, b, 0, 0} or, for a pair of
+// recurrences, {a.x, a.y, b.x, b.y}.
 // ---------------------------------------------------------------------------
 struct TileSlot {
     unsigned w[4];
 };
 static_assert(sizeof(TileSlot) == 16, "slot is 16 bytes");
-
-struct Lookback {
-    TileSlot *slots;     // the call's workspace (split-row calls), else nullptr
-    long long row_tiles; // tiles per row when rows are whole multiples of a tile, else 0
-    long long tile_base; // scan-order index of the launch's first tile
-};
 
 // Geometry of one launch over the flattened [E*T] array.
 struct Geometry {
@@ -282,135 +267,30 @@ __device__ __forceinline__ long long elem_row(const RowMasks &m, int k) {
     return kFast ? m.row0 : row_of(m, k);
 }
 
-// ---------------------------------------------------------------------------
-// Two-pass carries (rows that span tiles, single-action calls).  Pass one
-// (kModeReduce) writes every tile's aggregate (a, b), composed in scan
-// order, into its 16-byte slot as {a, b, 0, 0}; pass two (kModeCarry), a
-// later launch on the same stream, re-reads each tile (from L2 when the
-// launch's tiles fit it), scans it, and takes its carry from the complete
-// aggregates of the tiles before it in its row.  Pass two also publishes
-// each tile's inclusive value in the slot's second half, {1, x} as one
-// 64-bit store, as a shortcut for later tiles: a reader sees either 0 there
-// (not yet) or the whole pair, never half of it.  Nothing ever waits: the
-// aggregates are complete before pass two starts (it waits for pass one's
-// grid first), and the walk over them ends at the row's first tile at the
-// latest.  Every slot a launch reads is written by its own pass one, so the
-// workspace needs no initial content.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void ld_slot_halves(const TileSlot *slot, unsigned long long &ab,
-                                               unsigned long long &fx) {
-    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(ab), "=l"(fx) : "l"(slot) : "memory");
-}
-// Scalar recurrences (fp32, int32): {a, b} then {flag, x}.
+// Aggregate of a map into a workspace slot (all 16 bytes written).
 template <class AT, class BT>
 __device__ __forceinline__ void publish_aggregate(TileSlot *slot, AT a, BT b) {
     *reinterpret_cast<uint4 *>(slot) = make_uint4(to_bits(a), to_bits(b), 0u, 0u);
 }
-template <class BT>
-__device__ __forceinline__ void publish_inclusive(TileSlot *slot, BT x) {
-    const unsigned long long v = 1ull | ((unsigned long long)to_bits(x) << 32);
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(reinterpret_cast<char *>(slot) + 8), "l"(v)
-                 : "memory");
-}
-// The map slot k stands for: its inclusive value when published (a cut map),
-// else its aggregate.
-template <class AT, class BT>
-__device__ __forceinline__ void read_slot(const TileSlot *slot, AT &a, BT &b) {
-    unsigned long long ab, fx;
-    ld_slot_halves(slot, ab, fx);
-    if ((unsigned)fx != 0u) {
-        a = cut_a(a);
-        b = from_bits((unsigned)(fx >> 32), b);
-    } else {
-        a = from_bits((unsigned)ab, a);
-        b = from_bits((unsigned)(ab >> 32), b);
-    }
-}
-// Pairs of recurrences: the aggregate {a.x, a.y, b.x, b.y} fills the slot,
-// so pairs publish no inclusive values and walks compose aggregates only.
 __device__ __forceinline__ void publish_aggregate(TileSlot *slot, float2 a, float2 b) {
     *reinterpret_cast<uint4 *>(slot) =
         make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
 }
-__device__ __forceinline__ void publish_inclusive(TileSlot *, float2) {}
-__device__ __forceinline__ void read_slot(const TileSlot *slot, float2 &a, float2 &b) {
-    const uint4 v = ld_relaxed_gpu_v4(slot);
+// The aggregate a slot holds.
+template <class AT, class BT>
+__device__ __forceinline__ void read_aggregate(const TileSlot *slot, AT &a, BT &b) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(slot);
+    a = from_bits(v.x, a);
+    b = from_bits(v.y, b);
+}
+__device__ __forceinline__ void read_aggregate(const TileSlot *slot, float2 &a, float2 &b) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(slot);
     a = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
     b = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
 }
 
-// Carry into scan-order tile j from the aggregates of tiles k_min .. j-1,
-// called by all 32 lanes of one warp.  Each window covers 32 x kSlotsPerLane
-// tiles, nearest first: lane i reads tiles base - i M - m, m = 0 .. M-1,
-// all M loads in flight at once, and composes them nearest-outermost up to
-// the first that ends the walk (a published inclusive value, or an
-// aggregate that cuts the chain, a == 0); the lanes' maps are then composed
-// in order.  A row of up to 32 M tiles thus costs one round trip even when
-// none of its tiles has published an inclusive value yet.  Lane 0
-// publishes this tile's inclusive value.
+// Slots a lane reads per round trip when composing earlier aggregates.
 constexpr int kSlotsPerLane = 4;
-
-template <class AT, class BT>
-__device__ BT carry_from_aggregates(const Lookback &lb, long long j, long long k_min, bool needs_carry, AT ta,
-                                    BT tb, int lane) {
-    constexpr int M = kSlotsPerLane;
-    TileSlot *me = lb.slots + j;
-    if (!needs_carry) {
-        if (lane == 0) publish_inclusive(me, tb);
-        return identity_b(tb);
-    }
-    AT acc_a = identity_a(ta);
-    BT acc_b = identity_b(tb);
-    BT carry = identity_b(tb);
-    for (long long base = j - 1;; base -= 32 * M) {
-        const long long k0 = base - (long long)lane * M;
-        AT sa[M];
-        BT sb[M];
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            sa[m] = ta;
-            sb[m] = tb;
-            if (k0 - m < k_min) { // nothing flows in from before the row / array
-                sa[m] = cut_a(ta);
-                sb[m] = identity_b(tb);
-            } else {
-                read_slot(lb.slots + (k0 - m), sa[m], sb[m]);
-            }
-        }
-        AT la = identity_a(ta);
-        BT lb_ = identity_b(tb);
-        bool stop = false;
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            if (!stop) {
-                combine(la, lb_, sa[m], sb[m]);
-                stop = is_cut(sa[m]);
-            }
-        }
-        const unsigned stops = __ballot_sync(kFullMask, stop);
-        const int last = stops ? __ffs(stops) - 1 : 31;
-        if (lane > last) { // farther than the nearest stop: contributes nothing
-            la = identity_a(ta);
-            lb_ = identity_b(tb);
-        }
-        // ordered composition over lanes 0..last: lane 0 (nearest) applied last
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const AT oa = shfl_down(la, d);
-            const BT ob = shfl_down(lb_, d);
-            if (lane + d < 32) combine(la, lb_, oa, ob);
-        }
-        la = shfl_idx(la, 0);
-        lb_ = shfl_idx(lb_, 0);
-        combine(acc_a, acc_b, la, lb_);
-        if (stops) {
-            carry = acc_b;
-            break;
-        }
-    }
-    if (lane == 0) publish_inclusive(me, apply_pair(ta, tb, carry));
-    return carry;
-}
 
 // ---------------------------------------------------------------------------
 // Vector loads / stores of V consecutive elements (V a multiple of 4).  The
@@ -746,29 +626,22 @@ __device__ __forceinline__ RowMasks time_major_masks(const TimeMajorPos<V> &pos)
 // TimeMajorPos).
 // ---------------------------------------------------------------------------
 
-// Scan modes of one launch:
-//   kModeBlock     tiles hold whole rows; warps exchange carries in shared memory
+// Scan modes of a tile launch (tiles always hold whole rows; rows that span
+// tiles run the chunked two passes below):
+//   kModeBlock     warps exchange carries in shared memory
 //   kModeWarp      every warp's 32*V elements hold whole rows: no block scan at all
-//   kModeReduce    rows span tiles, pass one of two: write each tile's aggregate
-//   kModeCarry     rows span tiles, pass two: scan each tile with the carry
-//                  composed from the complete aggregates (no waiting)
 constexpr int kModeBlock = 0;
 constexpr int kModeWarp = 2;
-constexpr int kModeReduce = 3;
-constexpr int kModeCarry = 4;
 
 // The body of one tile, for a launch whose block `block` owns that tile
 // (the tile kernel below, or one part of a fused launch).
 template <class Est, int NT, int V, int kMode>
-__device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, const Geometry &g, const Lookback &lb,
+__device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, const Geometry &g,
                                                const long long block, unsigned char *dyn_smem) {
     using AT = typename Est::AT;
     using BT = typename Est::BT;
     constexpr bool kBwd = Est::kBackward;
     constexpr bool kWarpLocal = kMode == kModeWarp;
-    constexpr bool kReduce = kMode == kModeReduce;
-    constexpr bool kCarry = kMode == kModeCarry;
-    constexpr bool kTwoPass = kReduce || kCarry;
     constexpr int NW = NT / 32;
     static_assert(NT % 32 == 0 && NW <= 32, "block must be whole warps, at most 32");
 
@@ -781,7 +654,7 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     const int warp = tid >> 5;
 
     // tile index in scan order
-    const long long j = kTwoPass ? lb.tile_base + block : block;
+    const long long j = block;
     // Start this tile's DRAM reads before waiting for the previous grid on
     // the stream: the L2 prefetch overlaps them with that grid's tail.  Once
     // the wait returns, let the next grid launch (it waits for this one to
@@ -844,8 +717,7 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
         // the warp's first element in scan order starts a row: nothing flows in
         x = apply_pair(ea, eb, identity_b(tb));
     } else {
-        // value flowing into this warp: block scan of warp aggregates, plus
-        // the carry from earlier tiles when rows span tiles
+        // value flowing into this warp: block scan of warp aggregates
         if (lane == (kBwd ? 0 : 31)) {
             s_wa[warp] = ia;
             s_wb[warp] = ib;
@@ -858,27 +730,9 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
             AT wea;
             BT web;
             warp_exclusive_from_inclusive<kBwd>(wa, wb, lane, wea, web);
-            BT carry = identity_b(tb);
-            if constexpr (kTwoPass) {
-                const AT tile_a = shfl_idx(wa, kBwd ? 0 : NW - 1);
-                const BT tile_b = shfl_idx(wb, kBwd ? 0 : NW - 1);
-                bool needs_carry;
-                if (kBwd) {
-                    const long long end = tile0 + (long long)(NT * V);
-                    needs_carry = end < g.n && (end % g.seq_len) != 0;
-                } else {
-                    needs_carry = tile0 > 0 && (tile0 % g.seq_len) != 0;
-                }
-                const long long k_min = lb.row_tiles > 0 ? (j / lb.row_tiles) * lb.row_tiles : 0;
-                if constexpr (kCarry) {
-                    carry = carry_from_aggregates<AT, BT>(lb, j, k_min, needs_carry, tile_a, tile_b, lane);
-                } else if (lane == 0) {
-                    publish_aggregate(lb.slots + j, tile_a, tile_b);
-                }
-            }
-            if (lane < NW) s_wx[lane] = apply_pair(wea, web, carry);
+            // the tile's first warp in scan order starts a row: nothing flows in
+            if (lane < NW) s_wx[lane] = apply_pair(wea, web, identity_b(tb));
         }
-        if constexpr (kReduce) return; // pass one: the aggregate is all it writes
         __syncthreads();
         x = apply_pair(ea, eb, s_wx[warp]);
     }
@@ -904,10 +758,9 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
 }
 
 template <class Est, int NT, int V, int kMode>
-__global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Params P, const Geometry g,
-                                                       const Lookback lb) {
+__global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Params P, const Geometry g) {
     extern __shared__ __align__(128) unsigned char dyn_smem[];
-    tile_scan_body<Est, NT, V, kMode>(P, g, lb, (long long)blockIdx.x, dyn_smem);
+    tile_scan_body<Est, NT, V, kMode>(P, g, (long long)blockIdx.x, dyn_smem);
 }
 
 // ---------------------------------------------------------------------------
@@ -942,19 +795,6 @@ struct ChunkSplit {
     long long chunk_end;
     long long pf_blocks;   // blocks that prefetch their chunks into L2 before the grid wait
 };
-
-// The aggregate a chunk slot holds (pass one writes all 16 bytes).
-template <class AT, class BT>
-__device__ __forceinline__ void read_aggregate(const TileSlot *slot, AT &a, BT &b) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(slot);
-    a = from_bits(v.x, a);
-    b = from_bits(v.y, b);
-}
-__device__ __forceinline__ void read_aggregate(const TileSlot *slot, float2 &a, float2 &b) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(slot);
-    a = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
-    b = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
-}
 
 // Carry into chunk c: the composition of the aggregates of chunks c-1, c-2,
 // ... up to the first that cuts the chain, applied to the identity value.
@@ -1125,7 +965,7 @@ __global__ void __launch_bounds__(kChunkNT) chunk_scan_kernel(const typename Est
 // are scanned across a warp's chunks with shuffles (stride G lanes), the
 // warps of a segment are chained per env through shared memory, and the
 // value a segment leaves is the carry into the next one.  Rows never span
-// blocks, so no workspace and no look-back are needed.
+// blocks unless the host splits them (below), with a workspace then.
 // ---------------------------------------------------------------------------
 struct PlaneRef {
     const void *p;
@@ -1214,7 +1054,7 @@ __global__ void __launch_bounds__(kTmMaxWarps * 32) time_major_scan_kernel(const
                 for (int k = 0; k < split; ++k) {
                     AT ka = AT();
                     BT kb = BT();
-                    read_slot(row + k, ka, kb);
+                    read_aggregate(row + k, ka, kb);
                     x = apply_pair(ka, kb, x);
                 }
             }

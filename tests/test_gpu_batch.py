@@ -164,7 +164,7 @@ def test_batch_of_every_kind_matches_single_calls_and_oracle(E, T, trunc):
 
 
 def test_batch_mixes_fused_and_separate_launches():
-    # fused: 4096 x 128; separate: rows split over tiles (look-back), a
+    # fused: 4096 x 128; separate: rows split over tiles (chunked two passes), a
     # time-major call, T = 96 (no 1024-element plan), multi-action Retrace
     fused, fref = _calls_for(4096, 128, seed=1)
     lb, lref = _calls_for(3, 70000, seed=2)

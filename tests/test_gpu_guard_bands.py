@@ -5,7 +5,7 @@ each side) hold a sentinel bit pattern; after the call the margins must be
 bit for bit unchanged, and so must every input.  The shapes cover the paths
 where an out-of-range store would come from: ragged tails and pointers off
 a 16-byte boundary (scalar loads and stores), rows split over tiles (both
-passes of the two-pass carry, and the one-pass look-back of multi-action
+chunked passes, also after the expected-value pass of multi-action
 Retrace), the time-major layout, and fused batch requests.  Outputs are also
 compared with the oracle, so a test cannot pass by writing nothing.
 """

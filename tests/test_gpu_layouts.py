@@ -139,7 +139,7 @@ def test_time_major_forward(E, T, starts):
 
 
 # row-major shapes across the tile plans: whole rows per warp, per block, and
-# rows split over tiles (look-back), with ragged tails
+# rows split over tiles (chunked two passes), with ragged tails
 ROW_SHAPES = [(1, 1), (3, 5), (64, 512), (4096, 128), (4096, 129), (2, 5000), (3, 70000)]
 
 

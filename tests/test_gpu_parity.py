@@ -2,7 +2,7 @@
 seeded inputs, element by element (tests/gpu_common.py gives the tolerance).
 
 Shapes span every tile plan the library picks: whole rows per tile (512 to
-4096-element tiles), rows split over tiles with the decoupled look-back,
+4096-element tiles), rows split over tiles (the chunked two passes),
 ragged tails (E*T not a multiple of the tile or of 4), single-step rows and
 rows shorter than a vector.
 """

@@ -41,7 +41,7 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-# (E, T): rows split over tiles (the fixed scratch carries the look-back),
+# (E, T): rows split over tiles (the fixed scratch holds the chunk aggregates),
 # rows that straddle tiles, and whole rows per tile (no scratch needed)
 @pytest.mark.parametrize("E,T", [(3, 70000), (16, 262144), (4096, 129), (4096, 128)], ids=str)
 def test_noalloc_matches_workspace_entry_point(E, T):
