@@ -251,6 +251,19 @@ inline bool batch_dry() { return g_batch != nullptr && g_batch->pass == kBatchDr
 // ---------------------------------------------------------------------------
 // Launch
 // ---------------------------------------------------------------------------
+// Bytes per element of the input planes a call streams (its given planes).
+template <class Est>
+inline long long streamed_input_bytes(const typename Est::Params &P) {
+    long long b = 0;
+    for (int i = 0; i < Est::kInputPlanes; ++i) {
+        const PlaneRef r = Est::input_plane(P, i);
+        if (r.p != nullptr) b += r.bytes;
+    }
+    return b;
+}
+
+constexpr long long kPrefetchAllBelowBytes = 8; // input bytes per element
+
 template <class Est, int NT, int V, int kMode>
 cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, size_t smem, cudaStream_t stream) {
     auto kern = tile_scan_kernel<Est, NT, V, kMode>;
@@ -271,8 +284,13 @@ cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, size_t 
         }
         resident = r;
     }
+    // Calls that stream few bytes per element (reduced-byte planes) keep few
+    // bytes in flight per thread: every block prefetches its tile there, so
+    // the L2 fetches run ahead of the loads (measured: bf16 / uint8 GAE +
+    // returns at 65536 x 128 in 23.7 us this way, 28.0 us with the first
+    // wave alone).  Elsewhere the first wave of blocks alone prefetches.
     Geometry gl = g;
-    gl.pf_blocks = (long long)num_sms() * resident;
+    gl.pf_blocks = streamed_input_bytes<Est>(P) < kPrefetchAllBelowBytes ? (1ll << 62) : (long long)num_sms() * resident;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -295,17 +313,6 @@ cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, int mod
 // L2: a wave's pass one streams them from HBM, pass two finds them in L2
 // (B200: 126 MB).
 constexpr long long kTwoPassWaveBytes = 64ll << 20;
-
-// Bytes per element of the input planes a call streams (its given planes).
-template <class Est>
-inline long long streamed_input_bytes(const typename Est::Params &P) {
-    long long b = 0;
-    for (int i = 0; i < Est::kInputPlanes; ++i) {
-        const PlaneRef r = Est::input_plane(P, i);
-        if (r.p != nullptr) b += r.bytes;
-    }
-    return b;
-}
 
 // Resident blocks per SM of a kernel, queried once per kernel.
 template <class K>
