@@ -340,7 +340,7 @@ def summarize_clocks(path) -> dict:
 
 
 # ---------------------------------------------------------------------------
-# ncu DRAM traffic (profiles/dram_traffic.md): valid only for the exact
+# ncu DRAM traffic (profiles/dram_traffic.json): valid only for the exact
 # kernel source it was captured from
 # ---------------------------------------------------------------------------
 
