@@ -65,7 +65,7 @@ int rlscan_gae_ex(const float *rewards, const float *values, const float *termin
                      last_values, advantages, nullptr, gamma, lambda_};
     if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<GaeEst>("rlscan_gae", P, E, T, stream, ws, ws_bytes);
     return run<GaeEst>("rlscan_gae", P, E, T, ws, ws_bytes, stream,
-                       aligned16({rewards, values, terminateds, truncateds, advantages}));
+                       aligned16({rewards, values, terminateds, truncateds, bootstrap_values, advantages}));
 }
 
 int rlscan_gae(const float *rewards, const float *values, const float *terminateds, const float *truncateds,
@@ -99,7 +99,7 @@ int rlscan_gae_with_returns_ex(const float *rewards, const float *values, const 
     if (options & RLSCAN_OPT_TIME_MAJOR)
         return run_time_major<GaeReturnsEst>("rlscan_gae_with_returns", P, E, T, stream, ws, ws_bytes);
     return run<GaeReturnsEst>("rlscan_gae_with_returns", P, E, T, ws, ws_bytes, stream,
-                              aligned16({rewards, values, terminateds, truncateds, advantages, returns}));
+                              aligned16({rewards, values, terminateds, truncateds, bootstrap_values, advantages, returns}));
 }
 
 int rlscan_gae_with_returns(const float *rewards, const float *values, const float *terminateds,
@@ -140,7 +140,7 @@ int rlscan_gae_typed_ex(const void *rewards, const void *values, const void *ter
                         {bootstrap_values, n * vsz, "bootstrap_values"}, {last_values, (size_t)E * 4, "last_values"}};
     const Span outs[] = {{advantages, n * 4, "advantages"}, {returns, n * 4, "returns"}};
     RLSCAN_TRY(check_aliasing(ins, 6, outs, 2));
-    const bool vec = aligned16({rewards, values, terminateds, truncateds, advantages, returns});
+    const bool vec = aligned16({rewards, values, terminateds, truncateds, bootstrap_values, advantages, returns});
     const void *bv = truncateds ? bootstrap_values : nullptr;
 #define RLSCAN_GAE_TYPED(VT, FT)                                                                                  \
     do {                                                                                                          \

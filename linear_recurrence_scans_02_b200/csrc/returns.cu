@@ -29,7 +29,7 @@ int rlscan_lambda_returns_ex(const float *rewards, const float *values, const fl
     if (options & RLSCAN_OPT_TIME_MAJOR)
         return run_time_major<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, stream, ws, ws_bytes);
     return run<LambdaReturnsEst>("rlscan_lambda_returns", P, E, T, ws, ws_bytes, stream,
-                                 aligned16({rewards, values, terminateds, truncateds, returns}));
+                                 aligned16({rewards, values, terminateds, truncateds, bootstrap_values, returns}));
 }
 
 int rlscan_lambda_returns(const float *rewards, const float *values, const float *terminateds,
@@ -59,7 +59,7 @@ int rlscan_discounted_returns_ex(const float *rewards, const float *terminateds,
     if (options & RLSCAN_OPT_TIME_MAJOR)
         return run_time_major<ReturnsEst>("rlscan_discounted_returns", P, E, T, stream, ws, ws_bytes);
     return run<ReturnsEst>("rlscan_discounted_returns", P, E, T, ws, ws_bytes, stream,
-                           aligned16({rewards, terminateds, truncateds, returns}));
+                           aligned16({rewards, terminateds, truncateds, bootstrap_values, returns}));
 }
 
 int rlscan_discounted_returns(const float *rewards, const float *terminateds, const float *truncateds,

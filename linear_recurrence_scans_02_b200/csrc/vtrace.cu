@@ -33,7 +33,7 @@ int rlscan_vtrace_ex(const float *log_rhos, const float *rewards, const float *v
                         last_values, vs, pg_advantages, gamma, lambda_, rho_bar, c_bar};
     if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<VtraceEst>("rlscan_vtrace", P, E, T, stream, ws, ws_bytes);
     return run<VtraceEst>("rlscan_vtrace", P, E, T, ws, ws_bytes, stream,
-                          aligned16({log_rhos, rewards, values, terminateds, truncateds, vs, pg_advantages}));
+                          aligned16({log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, vs, pg_advantages}));
 }
 
 int rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,
@@ -75,8 +75,8 @@ int rlscan_gae_vtrace_ex(const float *log_rhos, const float *rewards, const floa
                            pg_advantages, gamma, lambda_, vtrace_lambda, rho_bar, c_bar};
     if (options & RLSCAN_OPT_TIME_MAJOR) return run_time_major<GaeVtraceEst>("rlscan_gae_vtrace", P, E, T, stream, ws, ws_bytes);
     return run<GaeVtraceEst>("rlscan_gae_vtrace", P, E, T, ws, ws_bytes, stream,
-                             aligned16({log_rhos, rewards, values, terminateds, truncateds, advantages, returns, vs,
-                                        pg_advantages}));
+                             aligned16({log_rhos, rewards, values, terminateds, truncateds, bootstrap_values, advantages,
+                                        returns, vs, pg_advantages}));
 }
 
 int rlscan_gae_vtrace(const float *log_rhos, const float *rewards, const float *values, const float *terminateds,

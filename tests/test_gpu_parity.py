@@ -12,7 +12,8 @@ import torch
 
 import oracle
 
-from gpu_common import (BACKWARD_KEYS, BACKWARD_RUN, check, dev, inputs_backward, run_gae, run_gae_with_returns,
+from gpu_common import (BACKWARD_KEYS, BACKWARD_RUN, assert_close, check, dev, inputs_backward, run_gae,
+                        run_gae_with_returns, tol_for,
                         run_prefix, run_retrace, run_traces, run_vtrace, strip)
 from linear_recurrence_scans_02_b200 import rlscan as R
 from linear_recurrence_scans_02_b200 import workloads as W
@@ -225,3 +226,89 @@ def test_gae_with_returns(E, T, variant):
 def test_gae_with_returns_unaligned(offset):
     d = inputs_backward(5, 129, seed=offset, p_term=0.02, p_trunc=0.02, last_values=True)
     check(run_gae_with_returns(strip(d, BACKWARD_KEYS["gae"]), offset=offset), 129, f"gae+returns offset={offset}")
+
+
+@pytest.mark.parametrize("E,T", [(64, 128), (5, 3000)], ids=str)
+def test_only_the_bootstrap_plane_unaligned(E, T):
+    # every plane 16-byte aligned except bootstrap_values (one element off):
+    # the bootstrap plane is streamed like the others, so it must count in
+    # the call's alignment test (single calls, the one-pass forms, a batch
+    # request, reduced-byte inputs)
+    d = W.vtrace_inputs(E, T, seed=7, p_term=0.02, p_trunc=0.02, last_values=True)
+    g32, l32 = np.float32(W.GAMMA), np.float32(W.LAMBDA)
+    t = {k: dev(v) for k, v in d.items()}
+    bv = dev(d["bootstrap_values"], offset=1)
+    assert bv.data_ptr() % 16 != 0 and t["rewards"].data_ptr() % 16 == 0
+    targs = (d["truncateds"], d["bootstrap_values"], d["last_values"])
+    r_adv = oracle.gae(d["rewards"], d["values"], d["terminateds"], g32, l32, *targs)
+    r_ret = oracle.lambda_returns(d["rewards"], d["values"], d["terminateds"], g32, l32, *targs)
+    r_dr = oracle.discounted_returns(d["rewards"], d["terminateds"], g32, *targs)
+    r_vs, r_pg = oracle.vtrace(d["log_rhos"], d["rewards"], d["values"], d["terminateds"], g32, np.float32(1.0),
+                               np.float32(1.0), np.float32(1.0), *targs)
+    tol = tol_for(T)
+    out = lambda: torch.full((E, T), float("nan"), device="cuda")
+    adv, ret, dr, vs, pg = out(), out(), out(), out(), out()
+    R.rlscan_gae(t["rewards"], t["values"], t["terminateds"], t["truncateds"], bv, t["last_values"], adv,
+                 W.GAMMA, W.LAMBDA)
+    R.rlscan_lambda_returns(t["rewards"], t["values"], t["terminateds"], t["truncateds"], bv, t["last_values"],
+                            ret, W.GAMMA, W.LAMBDA)
+    R.rlscan_discounted_returns(t["rewards"], t["terminateds"], t["truncateds"], bv, t["last_values"], dr, W.GAMMA)
+    R.rlscan_vtrace(t["log_rhos"], t["rewards"], t["values"], t["terminateds"], t["truncateds"], bv,
+                    t["last_values"], vs, pg, W.GAMMA, 1.0, 1.0, 1.0)
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    assert_close(adv, r_adv, tol, "gae")
+    assert_close(ret, r_ret, tol, "lambda returns")
+    assert_close(dr, r_dr, tol, "discounted returns")
+    assert_close(vs, r_vs, tol, "vtrace vs")
+    assert_close(pg, r_pg, tol, "vtrace pg")
+    # the one-pass forms
+    adv, ret, vs, pg = out(), out(), out(), out()
+    R.rlscan_gae_with_returns(t["rewards"], t["values"], t["terminateds"], t["truncateds"], bv, t["last_values"],
+                              adv, ret, W.GAMMA, W.LAMBDA)
+    torch.cuda.synchronize()
+    assert_close(adv, r_adv, tol, "gae + returns: advantages")
+    assert_close(ret, r_ret, tol, "gae + returns: returns")
+    adv, ret = out(), out()
+    R.rlscan_gae_vtrace(t["log_rhos"], t["rewards"], t["values"], t["terminateds"], t["truncateds"], bv,
+                        t["last_values"], adv, ret, vs, pg, W.GAMMA, W.LAMBDA, 1.0, 1.0, 1.0)
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    assert_close(adv, r_adv, tol, "gae + vtrace: advantages")
+    assert_close(vs, r_vs, tol, "gae + vtrace: vs")
+    # a batch request (fused when rows fit a tile)
+    adv, dr = out(), out()
+    R.rlscan_batch([dict(kind="gae", rewards=t["rewards"], values=t["values"], terminateds=t["terminateds"],
+                         truncateds=t["truncateds"], bootstrap_values=bv, last_values=t["last_values"],
+                         advantages=adv, gamma=W.GAMMA, lambda_=W.LAMBDA),
+                    dict(kind="discounted_returns", rewards=t["rewards"], terminateds=t["terminateds"],
+                         truncateds=t["truncateds"], bootstrap_values=bv, last_values=t["last_values"], returns=dr,
+                         gamma=W.GAMMA)])
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    assert_close(adv, r_adv, tol, "batch gae")
+    assert_close(dr, r_dr, tol, "batch returns")
+    # reduced-byte inputs with a bf16 bootstrap plane one element off
+    bf = lambda a, off=0: dev(a, off).to(torch.bfloat16) if off == 0 else _bf16_offset(a, off)
+    wide = lambda x: x.float().cpu().numpy()
+    rb, vb, bvb = bf(d["rewards"]), bf(d["values"]), bf(d["bootstrap_values"], 1)
+    assert bvb.data_ptr() % 16 != 0
+    adv, ret = out(), out()
+    R.rlscan_gae_typed(rb, vb, t["terminateds"], t["truncateds"], bvb, t["last_values"], adv, ret,
+                       W.GAMMA, W.LAMBDA)
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    nargs = (d["truncateds"], wide(bvb), d["last_values"])
+    assert_close(adv, oracle.gae(wide(rb), wide(vb), d["terminateds"], g32, l32, *nargs), tol, "bf16 gae")
+    assert_close(ret, oracle.lambda_returns(wide(rb), wide(vb), d["terminateds"], g32, l32, *nargs), tol,
+                 "bf16 returns")
+
+
+def _bf16_offset(a, offset):
+    """A bf16 CUDA copy of `a` whose data pointer is `offset` elements past
+    a 16-byte boundary."""
+    t = torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16)
+    flat = torch.empty(t.numel() + offset, dtype=torch.bfloat16, device="cuda")
+    view = flat[offset:].view(t.shape)
+    view.copy_(t.cuda())
+    return view
