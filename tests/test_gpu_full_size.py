@@ -116,3 +116,51 @@ def test_shape_grid(E, T):
                  f"traces {E}x{T} sampled rows")
     assert_close(ps[rows], oracle.episodic_prefix_sum(hx["x"], hx["dones"]), tol_for(T), f"prefix {E}x{T} sampled rows")
     R.rlscan_check()
+
+
+def test_bench_step_4096x128_as_timed():
+    """The step bench.py times, in its launch configuration: the eight calls
+    on bench.host_inputs as ONE rlscan_batch request (one fused launch),
+    every output compared with the oracle on the same host inputs."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    host = bench.host_inputs(seed=0)
+    bs = bench.BufferSet(torch, torch.device("cuda"), bench.ESTIMATORS)
+    bs.fill_from_host(host)
+    for key in bs.out_names:  # outputs start as NaN (int32: a sentinel) so unwritten ones show
+        t = bs.t[key]
+        t.fill_(-123456 if t.dtype == torch.int32 else float("nan"))
+    bs.batch_call(R)()
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    T = bench.T_STEPS
+    g32, l32, one = np.float32(bench.GAMMA), np.float32(bench.LAMBDA), np.float32(1.0)
+    h = host["gae"]
+    assert_close(bs.t["gae", "advantages"], oracle.gae(h["rewards"], h["values"], h["terminateds"], g32, l32),
+                 tol_for(T), "step gae")
+    h = host["vtrace"]
+    vs, pg = oracle.vtrace(h["log_rhos"], h["rewards"], h["values"], h["terminateds"], g32, one, one, one)
+    assert_close(bs.t["vtrace", "vs"], vs, tol_for(T), "step vtrace vs")
+    assert_close(bs.t["vtrace", "pg_advantages"], pg, tol_for(T), "step vtrace pg")
+    h = host["retrace"]
+    ref = oracle.retrace(h["rewards"], h["q_values"], h["next_q_values_all"], h["log_rhos"], h["terminateds"],
+                         h["truncateds"], g32, l32, one)
+    assert_close(bs.t["retrace", "q_ret"], ref, tol_for(T), "step retrace")
+    h = host["lambda_returns"]
+    assert_close(bs.t["lambda_returns", "returns"],
+                 oracle.lambda_returns(h["rewards"], h["values"], h["terminateds"], g32, l32), tol_for(T),
+                 "step lambda returns")
+    h = host["discounted_returns"]
+    assert_close(bs.t["discounted_returns", "returns"],
+                 oracle.discounted_returns(h["rewards"], h["terminateds"], g32), tol_for(T), "step returns")
+    h = host["eligibility_traces"]
+    assert_close(bs.t["eligibility_traces", "traces"], oracle.eligibility_traces(h["x"], h["dones"], g32, l32),
+                 tol_for(T), "step traces")
+    h = host["prefix_sum_f32"]
+    assert_close(bs.t["prefix_sum_f32", "out"], oracle.episodic_prefix_sum(h["x"], h["dones"]), tol_for(T),
+                 "step prefix f32")
+    h = host["prefix_sum_i32"]
+    assert_equal_int(bs.t["prefix_sum_i32", "out"], oracle.episodic_prefix_sum(h["x"], h["dones"]),
+                     "step prefix i32")
