@@ -129,7 +129,8 @@ def test_forward_estimators_reduced_bytes(vdt, fdt, E, T):
     assert_equal_int(pi, oracle.episodic_prefix_sum(fi["x"], wdi), f"prefix i32 {fdt} {E}x{T}")
 
 
-@pytest.mark.parametrize("E,T", [(7, 9), (100, 130)], ids=str)
+# (7, 1000) and (33, 4100): few envs with long rows, split over blocks
+@pytest.mark.parametrize("E,T", [(7, 9), (100, 130), (7, 1000), (33, 4100)], ids=str)
 def test_reduced_bytes_time_major_and_done_starts(E, T):
     vdt, fdt = torch.bfloat16, torch.uint8
     t, w = _backward_inputs(E, T, 11, vdt, fdt, tm=True)
