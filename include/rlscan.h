@@ -69,7 +69,10 @@ extern "C" {
 /* 1.2.0: rlscan_gae_vtrace (GAE, TD(lambda) returns and V-Trace in one pass)
  * and its batch kind; rlscan_call holds four outputs and a vtrace_lambda
  * field at its end, so its size changed: clients built against an earlier
- * rlscan_call must be rebuilt (their rlscan_version() check fails).
+ * rlscan_call must be rebuilt (their rlscan_version() check fails).  Rows
+ * that span tiles run the chunked two passes and need 16 bytes of workspace
+ * per 512 elements (time-major calls on few envs may need one too): size
+ * workspaces with rlscan_workspace_bytes, never from a fixed formula.
  * 1.1.1: rlscan_call gained flag_dtype after dtype, which moved every later
  * field.  1.1.0: the _ex entry points (layout and done-convention options)
  * and rlscan_batch. */
