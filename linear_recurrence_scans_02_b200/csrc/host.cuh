@@ -262,6 +262,21 @@ inline long long streamed_input_bytes(const typename Est::Params &P) {
     return b;
 }
 
+// Resident blocks per SM of a kernel, queried once per kernel (`unknown`
+// when the query fails).
+template <class K>
+inline int resident_blocks(K kern, int threads, size_t smem, std::atomic<int> &cache, int unknown) {
+    int r = cache.load(std::memory_order_relaxed);
+    if (r == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, threads, smem) != cudaSuccess || r < 1) {
+            (void)cudaGetLastError();
+            r = unknown;
+        }
+        cache.store(r, std::memory_order_relaxed);
+    }
+    return r;
+}
+
 constexpr long long kPrefetchAllBelowBytes = 8; // input bytes per element
 
 template <class Est, int NT, int V, int kMode>
@@ -274,16 +289,8 @@ cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, size_t 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)g.ntiles);
     cfg.blockDim = dim3(NT);
-    // resident blocks per SM of this kernel, queried once
-    static int resident = 0;
-    if (resident == 0) {
-        int r = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, NT, smem) != cudaSuccess || r < 1) {
-            (void)cudaGetLastError();
-            r = 1 << 16; // unknown: every block prefetches
-        }
-        resident = r;
-    }
+    static std::atomic<int> resident_cache{0};
+    const int resident = resident_blocks(kern, NT, smem, resident_cache, 1 << 16); // unknown: all prefetch
     // Calls that stream few bytes per element (reduced-byte planes) keep few
     // bytes in flight per thread: every block prefetches its tile there, so
     // the L2 fetches run ahead of the loads (measured: bf16 / uint8 GAE +
@@ -314,20 +321,6 @@ cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, int mod
 // (B200: 126 MB).
 constexpr long long kTwoPassWaveBytes = 64ll << 20;
 
-// Resident blocks per SM of a kernel, queried once per kernel.
-template <class K>
-inline int resident_blocks(K kern, int threads, int &cache) {
-    if (cache == 0) {
-        int r = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, threads, 0) != cudaSuccess || r < 1) {
-            (void)cudaGetLastError();
-            r = 1;
-        }
-        cache = r;
-    }
-    return cache;
-}
-
 // Rows that span tiles: the chunked two passes (chunk_scan_kernel).  One
 // chunk per warp the GPU holds at once (at least two steps a chunk, so the
 // chunks fit the workspace of workspace_for), over as few waves as keep each
@@ -338,9 +331,9 @@ int run_chunked(const char *name, const typename Est::Params &P, const Geometry 
     constexpr long long SW = 32LL * kChunkV;
     constexpr int WPB = kChunkNT / 32;
     // both passes run on the same grid, which the GPU holds at once
-    static int res_a = 0, res_b = 0;
-    const long long resident = std::min(resident_blocks(chunk_scan_kernel<Est, kChunkAggregates>, kChunkNT, res_a),
-                                        resident_blocks(chunk_scan_kernel<Est, kChunkScan>, kChunkNT, res_b));
+    static std::atomic<int> res_a{0}, res_b{0};
+    const long long resident = std::min(resident_blocks(chunk_scan_kernel<Est, kChunkAggregates>, kChunkNT, 0, res_a, 1),
+                                        resident_blocks(chunk_scan_kernel<Est, kChunkScan>, kChunkNT, 0, res_b, 1));
     const long long warps = (long long)num_sms() * resident * WPB;
     const long long nsteps = ceil_div(g.n, SW);
     const long long in_bytes = std::max<long long>(1, streamed_input_bytes<Est>(P)) * g.n;
