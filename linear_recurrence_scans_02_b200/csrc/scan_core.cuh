@@ -7,7 +7,7 @@
 // scan over the flattened [E*T] array:
 //
 //   * the array is cut into tiles of S = NT*V consecutive elements, one CTA
-//     per tile; each thread owns V consecutive elements (128-bit loads);
+//     per tile; each thread owns V consecutive elements (256-bit loads);
 //   * rows never leak into each other because each estimator's coefficient
 //     builder sets a = 0 on the first element of a row in scan order (the
 //     row's last value is folded into b there), the same cut a done makes;
@@ -293,10 +293,13 @@ __device__ __forceinline__ void read_aggregate(const TileSlot *slot, float2 &a, 
 constexpr int kSlotsPerLane = 4;
 
 // ---------------------------------------------------------------------------
-// Vector loads / stores of V consecutive elements (V a multiple of 4).  The
-// 128-bit path needs a 16-byte-aligned base and a full vector; otherwise each
-// element is loaded on its own.  Elements at or past n read as zero / are not
-// written.  A null plane reads as zeros.
+// Vector loads / stores of V consecutive elements (V a multiple of 4).  When
+// the thread's elements all exist and every plane is 16-byte aligned (`vec`),
+// a plane whose run starts on a 32-byte boundary moves in 256-bit accesses
+// (one full 32-byte sector per lane and access: a warp's stores never leave
+// half-written sectors for L2 to merge), any other in 128-bit ones; otherwise
+// each element is loaded on its own.  Elements at or past n read as zero / are
+// not written.  A null plane reads as zeros.
 //
 // Loads are coherent and cached in L2 only (ld.global.cg), never through the
 // read-only path: with programmatic dependent launch this kernel starts while
@@ -304,6 +307,20 @@ constexpr int kSlotsPerLane = 4;
 // read-only for the whole life of this kernel.  Every element is read once,
 // so L1 would not help anyway.
 // ---------------------------------------------------------------------------
+
+// 256-bit accesses (sm_100 and later): eight 32-bit words at a 32-byte-aligned
+// address.  Both are volatile so that they stay after the grid-dependency
+// wait like every other memory access.
+__device__ __forceinline__ void ld_cg_v8(const void *p, unsigned (&w)[8]) {
+    asm volatile("ld.global.cg.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p));
+}
+__device__ __forceinline__ void st_cs_v8(void *p, const unsigned (&w)[8]) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
 
 // `vec`: the caller's per-thread flag "all planes 16-byte aligned and this
 // thread's V elements all exist" (one test per thread, not per plane).
@@ -316,6 +333,18 @@ __device__ __forceinline__ void load_plane(const T *__restrict__ p, long long i0
 #pragma unroll
         for (int k = 0; k < V; ++k) o[k] = T(0);
         return;
+    }
+    if constexpr (V % 8 == 0) {
+        if (vec && (reinterpret_cast<uintptr_t>(p + i0) & 31u) == 0) {
+#pragma unroll
+            for (int k = 0; k < V; k += 8) {
+                unsigned w[8];
+                ld_cg_v8(p + i0 + k, w);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[k + j] = from_bits(w[j], T());
+            }
+            return;
+        }
     }
     if (vec) {
 #pragma unroll
@@ -337,6 +366,18 @@ __device__ __forceinline__ void load_plane(const T *__restrict__ p, long long i0
 template <int V, class T>
 __device__ __forceinline__ void store_plane(T *__restrict__ p, long long i0, long long n, bool vec,
                                             const T (&o)[V]) {
+    if constexpr (V % 8 == 0) {
+        if (vec && (reinterpret_cast<uintptr_t>(p + i0) & 31u) == 0) {
+#pragma unroll
+            for (int k = 0; k < V; k += 8) {
+                unsigned w[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[j] = to_bits(o[k + j]);
+                st_cs_v8(p + i0 + k, w);
+            }
+            return;
+        }
+    }
     if (vec) {
 #pragma unroll
         for (int k = 0; k < V; k += 4) {
@@ -478,7 +519,7 @@ __device__ __forceinline__ float load_one_widen(const T *__restrict__ p, long lo
 // (or before) them, for element k of a sparse plane, and to store its V
 // outputs.  Two layouts:
 //   RowMajorPos   [E, T] with T contiguous: a thread owns V consecutive
-//                 elements of the flattened array (128-bit vector loads; the
+//                 elements of the flattened array (256-bit vector loads; the
 //                 halo comes from the neighbouring lane by a shuffle);
 //   TimeMajorPos  [T, E] with E contiguous: a thread owns V consecutive
 //                 timesteps of one env; lanes are consecutive envs, so each

@@ -22,7 +22,9 @@ def tol_for(T):
 
 def dev(a, offset=0):
     """numpy -> CUDA tensor; offset > 0 gives a contiguous view whose data
-    pointer is `offset` elements past a 16-byte boundary (unaligned path)."""
+    pointer is `offset` elements past the allocation's start (a 512-byte
+    boundary): 1-3 fp32 elements take the unaligned path, 4 (16 bytes) the
+    128-bit one instead of the 256-bit one."""
     if a is None:
         return None
     t = torch.from_numpy(np.ascontiguousarray(a))

@@ -12,7 +12,8 @@ import torch
 
 import oracle
 
-from gpu_common import (BACKWARD_KEYS, BACKWARD_RUN, assert_close, check, dev, inputs_backward, run_gae,
+from gpu_common import (BACKWARD_KEYS, BACKWARD_RUN, assert_close, check, dev, empty_like_dev, inputs_backward,
+                        run_gae,
                         run_gae_with_returns, tol_for,
                         run_prefix, run_retrace, run_traces, run_vtrace, strip)
 from linear_recurrence_scans_02_b200 import rlscan as R
@@ -104,7 +105,9 @@ def test_parameter_extremes(gamma, lam):
     check(run_traces(x, gamma=gamma, lam=lam), T, f"traces g={gamma} l={lam}")
 
 
-@pytest.mark.parametrize("offset", [1, 2, 3])
+# offsets 1-3: scalar loads and stores; 4 (16 bytes): 128-bit accesses, since
+# the runs then never start on a 32-byte boundary
+@pytest.mark.parametrize("offset", [1, 2, 3, 4])
 @pytest.mark.parametrize("E,T", [(64, 128), (5, 129), (4, 3000)], ids=lambda v: str(v))
 def test_unaligned_pointers(offset, E, T):
     d = inputs_backward(E, T, seed=offset, p_term=0.02, p_trunc=0.02, last_values=True)
@@ -226,6 +229,55 @@ def test_gae_with_returns(E, T, variant):
 def test_gae_with_returns_unaligned(offset):
     d = inputs_backward(5, 129, seed=offset, p_term=0.02, p_trunc=0.02, last_values=True)
     check(run_gae_with_returns(strip(d, BACKWARD_KEYS["gae"]), offset=offset), 129, f"gae+returns offset={offset}")
+
+
+@pytest.mark.parametrize("E,T", [(64, 128), (7, 1000), (3, 70000)], ids=lambda v: str(v))
+def test_planes_on_16_and_32_byte_boundaries(E, T):
+    # each plane picks its own access width: planes starting on a 32-byte
+    # boundary move in 256-bit accesses, the others (16 bytes past one) in
+    # 128-bit ones, in the same call (tiles, chunked long rows, the fused
+    # batch launch, the one-pass forms)
+    d = W.vtrace_inputs(E, T, seed=8, p_term=0.02, p_trunc=0.02, last_values=True)
+    g32, l32 = np.float32(W.GAMMA), np.float32(W.LAMBDA)
+    t = {k: dev(v, 4 if k in ("values", "truncateds", "log_rhos") else 0) for k, v in d.items()}
+    assert t["values"].data_ptr() % 32 == 16 and t["rewards"].data_ptr() % 32 == 0
+    targs = (d["truncateds"], d["bootstrap_values"], d["last_values"])
+    r_adv = oracle.gae(d["rewards"], d["values"], d["terminateds"], g32, l32, *targs)
+    r_ret = oracle.lambda_returns(d["rewards"], d["values"], d["terminateds"], g32, l32, *targs)
+    r_vs, r_pg = oracle.vtrace(d["log_rhos"], d["rewards"], d["values"], d["terminateds"], g32, np.float32(1.0),
+                               np.float32(1.0), np.float32(1.0), *targs)
+    tol = tol_for(T)
+    out16 = lambda: empty_like_dev(d["rewards"], 4)
+    out32 = lambda: empty_like_dev(d["rewards"])
+    args = (t["rewards"], t["values"], t["terminateds"], t["truncateds"], t["bootstrap_values"], t["last_values"])
+    adv = out16()
+    R.rlscan_gae(*args, adv, W.GAMMA, W.LAMBDA)
+    ret, vs, pg = out32(), out16(), out32()
+    R.rlscan_lambda_returns(*args, ret, W.GAMMA, W.LAMBDA)
+    R.rlscan_vtrace(t["log_rhos"], *args, vs, pg, W.GAMMA, 1.0, 1.0, 1.0)
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    assert_close(adv, r_adv, tol, "gae")
+    assert_close(ret, r_ret, tol, "lambda returns")
+    assert_close(vs, r_vs, tol, "vtrace vs")
+    assert_close(pg, r_pg, tol, "vtrace pg")
+    adv, ret = out32(), out16()
+    R.rlscan_gae_with_returns(*args, adv, ret, W.GAMMA, W.LAMBDA)
+    torch.cuda.synchronize()
+    assert_close(adv, r_adv, tol, "gae + returns: advantages")
+    assert_close(ret, r_ret, tol, "gae + returns: returns")
+    adv, vs = out16(), out32()
+    R.rlscan_batch([dict(kind="gae", rewards=t["rewards"], values=t["values"], terminateds=t["terminateds"],
+                         truncateds=t["truncateds"], bootstrap_values=t["bootstrap_values"],
+                         last_values=t["last_values"], advantages=adv, gamma=W.GAMMA, lambda_=W.LAMBDA),
+                    dict(kind="vtrace", log_rhos=t["log_rhos"], rewards=t["rewards"], values=t["values"],
+                         terminateds=t["terminateds"], truncateds=t["truncateds"],
+                         bootstrap_values=t["bootstrap_values"], last_values=t["last_values"], vs=vs,
+                         pg_advantages=out16(), gamma=W.GAMMA)])
+    torch.cuda.synchronize()
+    R.rlscan_check()
+    assert_close(adv, r_adv, tol, "batch gae")
+    assert_close(vs, r_vs, tol, "batch vtrace vs")
 
 
 @pytest.mark.parametrize("E,T", [(64, 128), (5, 3000)], ids=str)
