@@ -7,6 +7,8 @@
 // the grid has the same shape: 128 threads x 8 elements.
 #pragma once
 
+#include <utility>
+
 #include "estimators.cuh"
 
 namespace rlscan {
@@ -99,10 +101,12 @@ struct BackwardFamilyEst {
             }
         }
     }
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr) {
+        if constexpr (kCase == kCasePlain) {
+            coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
@@ -173,28 +177,49 @@ struct FusedItem {
     long long tile_begin; // first block of this call in the fused grid
     int kind;             // FusedBody: the tile body that runs the call
     int mode;             // kModeWarp or kModeBlock
+    int truncation_code;  // the call needs its body's truncation variants (not kCasePlain)
 };
+
+// Host side: whether a call, in its body's form, passes truncations to a
+// builder whose kCasePlain variant compiles them out.  Retrace's builder
+// tests its truncation flags in every variant, and bodies without a
+// truncation plane never pass any.
+template <class P, class = void>
+struct HasTruncations : std::false_type {};
+template <class P>
+struct HasTruncations<P, std::void_t<decltype(std::declval<P>().truncateds)>> : std::true_type {};
+template <class Est, class P>
+inline bool needs_truncation_code(const P &p) {
+    if constexpr (std::is_same<Est, RetraceEst>::value || !HasTruncations<P>::value) return false;
+    else return p.truncateds != nullptr;
+}
 
 struct FusedBatch {
     FusedItem item[kFusedMax];
     int n;
 };
 
-template <class Est, int V, int kMode>
+template <class Est, int V, int kMode, int kCase>
 __device__ __forceinline__ void fused_tile(const FusedItem &it, long long block, unsigned char *smem) {
     const auto &P = *reinterpret_cast<const typename Est::Params *>(it.params);
-    tile_scan_body<Est, kFusedNT, V, kMode>(P, it.g, block, smem);
+    tile_scan_body<Est, kFusedNT, V, kMode, kCase>(P, it.g, block, smem);
 }
 
-template <class Est, int V>
+// kCasePlain launches hold warp-local calls only (see fused_plain); the
+// others pick the scan mode per call.
+template <class Est, int V, int kCase>
 __device__ __forceinline__ void fused_tile_any_mode(const FusedItem &it, long long block, unsigned char *smem) {
-    if (it.mode == kModeWarp)
-        fused_tile<Est, V, kModeWarp>(it, block, smem);
-    else
-        fused_tile<Est, V, kModeBlock>(it, block, smem);
+    if constexpr (kCase == kCasePlain) {
+        fused_tile<Est, V, kModeWarp, kCasePlain>(it, block, smem);
+    } else {
+        if (it.mode == kModeWarp)
+            fused_tile<Est, V, kModeWarp, kCase>(it, block, smem);
+        else
+            fused_tile<Est, V, kModeBlock, kCase>(it, block, smem);
+    }
 }
 
-template <int V>
+template <int V, int kCase>
 __global__ void __launch_bounds__(kFusedNT, kFusedMinBlocks) fused_tile_kernel(const __grid_constant__ FusedBatch b) {
     extern __shared__ __align__(128) unsigned char dyn_smem[];
     int idx = 0;
@@ -203,11 +228,11 @@ __global__ void __launch_bounds__(kFusedNT, kFusedMinBlocks) fused_tile_kernel(c
     const FusedItem &it = b.item[idx];
     const long long block = (long long)blockIdx.x - it.tile_begin;
     switch (it.kind) {
-    case kBodyBackward: fused_tile_any_mode<BackwardFamilyEst, V>(it, block, dyn_smem); break;
-    case kBodyVtrace: fused_tile_any_mode<VtraceEst, V>(it, block, dyn_smem); break;
-    case kBodyRetrace1: fused_tile_any_mode<RetraceEst, V>(it, block, dyn_smem); break;
-    case kBodyForward: fused_tile_any_mode<TracesEst, V>(it, block, dyn_smem); break;
-    case kBodyPrefixI32: fused_tile_any_mode<PrefixI32Est, V>(it, block, dyn_smem); break;
+    case kBodyBackward: fused_tile_any_mode<BackwardFamilyEst, V, kCase>(it, block, dyn_smem); break;
+    case kBodyVtrace: fused_tile_any_mode<VtraceEst, V, kCase>(it, block, dyn_smem); break;
+    case kBodyRetrace1: fused_tile_any_mode<RetraceEst, V, kCase>(it, block, dyn_smem); break;
+    case kBodyForward: fused_tile_any_mode<TracesEst, V, kCase>(it, block, dyn_smem); break;
+    case kBodyPrefixI32: fused_tile_any_mode<PrefixI32Est, V, kCase>(it, block, dyn_smem); break;
     default: break;
     }
 }

@@ -138,10 +138,12 @@ struct GaeEstT {
     // uniform branches per thread: without truncations the truncation logic
     // is compiled out of the per-element loop, and on the fast path (all V
     // elements present, V divides T) so are the per-element row tests
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr) {
+        if constexpr (kCase == kCasePlain) {
+            coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
@@ -250,10 +252,12 @@ struct LambdaReturnsEstT {
     // uniform branches per thread: without truncations the truncation logic
     // is compiled out of the per-element loop, and on the fast path (all V
     // elements present, V divides T) so are the per-element row tests
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr) {
+        if constexpr (kCase == kCasePlain) {
+            coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
@@ -340,10 +344,12 @@ struct ReturnsEstT {
     // uniform branches per thread: without truncations the truncation logic
     // is compiled out of the per-element loop, and on the fast path (all V
     // elements present, V divides T) so are the per-element row tests
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr) {
+        if constexpr (kCase == kCasePlain) {
+            coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
@@ -454,10 +460,12 @@ struct VtraceEstT {
     // uniform branches per thread: without truncations the truncation logic
     // is compiled out of the per-element loop, and on the fast path (all V
     // elements present, V divides T) so are the per-element row tests
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
-        if (P.truncateds != nullptr) {
+        if constexpr (kCase == kCasePlain) {
+            coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
@@ -559,11 +567,13 @@ struct GaeVtraceEst {
             }
         }
     }
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float2 (&a)[V],
                                                   float2 (&b)[V]) {
-        if (P.truncateds != nullptr) {
+        if constexpr (kCase == kCasePlain) {
+            coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
         } else {
@@ -667,11 +677,12 @@ struct RetraceEstT {
             }
         }
     }
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V],
                                                   float (&b)[V]) {
-        if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        if constexpr (kCase == kCasePlain) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        else if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }
     template <int V>
@@ -742,11 +753,12 @@ struct ForwardEstT {
             }
         }
     }
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V],
                                                   float (&b)[V]) {
-        if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        if constexpr (kCase == kCasePlain) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        else if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }
     template <int V>
@@ -814,11 +826,12 @@ struct PrefixI32EstT {
             }
         }
     }
-    template <int V, class Pos>
+    template <int V, int kCase = kCaseAny, class Pos>
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, uint32_t (&a)[V],
                                                   int32_t (&b)[V]) {
-        if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        if constexpr (kCase == kCasePlain) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        else if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }
     template <int V>

@@ -396,6 +396,7 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
             std::memcpy(it.params, &body_params, sizeof body_params);
             it.g = g;
             it.kind = FusedBodyOf<Est>::value;
+            it.truncation_code = needs_truncation_code<Est>(body_params) ? 1 : 0;
             return ok();
         }
     }

@@ -208,6 +208,16 @@ struct RowMasks {
     long long row0;
     bool fast; // all V elements exist and V divides T: only element V-1 can end a row, only 0 start one
 };
+
+// What a launch knows at compile time about its calls, for the coefficient
+// builders (`coeffs<V, kCase>`):
+//   kCaseAny    truncations and the fast path are decided per call and
+//               thread at run time (every variant is compiled in);
+//   kCasePlain  no call passes truncations and every thread takes the fast
+//               path (V divides T and the array is a whole number of tiles):
+//               one variant per builder, a smaller kernel.
+constexpr int kCaseAny = 0;
+constexpr int kCasePlain = 1;
 template <int V>
 __device__ __forceinline__ RowMasks row_masks(long long i0, const Geometry &g) {
     RowMasks m;
@@ -658,7 +668,7 @@ __device__ __forceinline__ RowMasks time_major_masks(const TimeMajorPos<V> &pos)
 // The tile kernel.  Est supplies (see estimators.cuh):
 //   kBackward, AT, BT, Params, State<V>,
 //   load<NT, V>(P, g, pos, S, dyn_smem)         -- every thread, incl. past n
-//   coeffs<V>(P, g, pos, rm, S, a, b)           -- (a, b) per element, identity past n
+//   coeffs<V, kCase>(P, g, pos, rm, S, a, b)    -- (a, b) per element, identity past n
 //   out<V>(P, S, k, x, x_prev, b_k)             -- record output k (x_prev = value
 //                                                  of the element before it in scan order,
 //                                                  b_k = its scan coefficient b)
@@ -676,7 +686,7 @@ constexpr int kModeWarp = 2;
 
 // The body of one tile, for a launch whose block `block` owns that tile
 // (the tile kernel below, or one part of a fused launch).
-template <class Est, int NT, int V, int kMode>
+template <class Est, int NT, int V, int kMode, int kCase = kCaseAny>
 __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, const Geometry &g,
                                                const long long block, unsigned char *dyn_smem) {
     using AT = typename Est::AT;
@@ -718,7 +728,7 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     AT a[V];
     BT b[V];
     const RowMasks rm = row_masks<V>(i0, g);
-    Est::template coeffs<V>(P, g, pos, rm, S, a, b);
+    Est::template coeffs<V, kCase>(P, g, pos, rm, S, a, b);
 
     // thread aggregate, composed in scan order
     AT ta;

@@ -163,6 +163,21 @@ def test_batch_of_every_kind_matches_single_calls_and_oracle(E, T, trunc):
     _check_batch(calls, refs)
 
 
+@pytest.mark.parametrize("shapes,trunc", [(((64, 128), (8, 128)), False), (((64, 128), (9, 128)), False),
+                                          (((64, 128), (8, 128)), True), (((16, 256), (4, 256)), False)],
+                         ids=["plain", "partial-tile", "truncations", "plain-256"])
+def test_batch_plain_and_general_fused_kernels(shapes, trunc):
+    # every kind on one shape plus GAE on a second: "plain" requests (warp-local
+    # rows of a multiple of 8 steps, whole 1024-element tiles, truncations on
+    # Retrace only) take the fused kernel built without the other builder
+    # variants; a call off a whole tile or truncations elsewhere take the
+    # general one.  Both must match the single calls and the oracle.
+    (E0, T0), (E1, T1) = shapes
+    calls, refs = _calls_for(E0, T0, seed=70, trunc=trunc)
+    c1, r1 = _calls_for(E1, T1, seed=71, trunc=trunc)
+    _check_batch(calls + c1[:1], refs + r1[:1])
+
+
 def test_batch_mixes_fused_and_separate_launches():
     # fused: 4096 x 128; separate: rows split over tiles (chunked two passes), a
     # time-major call, T = 96 (no 1024-element plan), multi-action Retrace
