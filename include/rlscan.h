@@ -71,7 +71,7 @@ extern "C" {
  * field at its end, so its size changed: clients built against an earlier
  * rlscan_call must be rebuilt (their rlscan_version() check fails).  Rows
  * that span tiles run the chunked two passes and need 16 bytes of workspace
- * per 512 elements (time-major calls on few envs may need one too): size
+ * per 1024 elements (time-major calls on few envs may need one too): size
  * workspaces with rlscan_workspace_bytes, never from a fixed formula.
  * 1.1.1: rlscan_call gained flag_dtype after dtype, which moved every later
  * field.  1.1.0: the _ex entry points (layout and done-convention options)
@@ -294,8 +294,8 @@ RLSCAN_API int rlscan_episodic_prefix_sum(const void *x, int dtype, const float 
  * clears the part of the array it uses with cudaMemsetAsync on `stream` and
  * allocates nothing.
  * Limit: shapes whose plan needs more scratch than the array holds (rows
- * that span tiles, over more than about 33 million elements in all: one
- * 16-byte slot per 512 elements) return RLSCAN_ERR_WORKSPACE with the sizes
+ * that span tiles, over more than about 67 million elements in all: one
+ * 16-byte slot per 1024 elements) return RLSCAN_ERR_WORKSPACE with the sizes
  * in rlscan_last_error().
  * All calls on one device share that device's array, which keeps the last
  * call's contents: two calls whose kernels may run at the same time on one
@@ -475,7 +475,7 @@ RLSCAN_API int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size
 
 /*
  * Workspace size in bytes that any entry point above needs for an [E, T]
- * problem (any A): 16 bytes per 512 elements when rows span tiles, 0 when no call of
+ * problem (any A): 16 bytes per 1024 elements when rows span tiles, 0 when no call of
  * that shape needs one.  Negative or overflowing shapes return 0 and the
  * compute call then rejects them.
  */
@@ -503,7 +503,7 @@ RLSCAN_API int rlscan_version(void);
  * writes tile size in elements, threads per block, whether tiles exchange
  * carries through the workspace (1) or not (0), and the tile count.  For
  * rows that span tiles (1) the call runs the chunked two passes: it writes
- * the workspace's granularity (512 elements a slot), the passes' block size
+ * the workspace's granularity (1024 elements a slot), the passes' block size
  * and the workspace's slot count, an upper bound on the chunks.
  * actions: 1 for every estimator except rlscan_retrace with A > 1, whose
  * action count it is (1 .. RLSCAN_MAX_ACTIONS); every call scans on the same

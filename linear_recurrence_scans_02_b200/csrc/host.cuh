@@ -171,7 +171,8 @@ inline bool aligned16(std::initializer_list<const void *> ptrs) {
 }
 
 // Rows that span tiles: one 16-byte slot per chunk of the chunked two
-// passes, at most one per 512 elements; nothing otherwise.
+// passes, at most one per 1024 elements (a chunk holds at least two warp
+// steps of 512); nothing otherwise.
 inline size_t workspace_for(const Plan &p, long long n) {
     return p.lookback ? sizeof(TileSlot) * (size_t)ceil_div(n, 2LL * 32 * kChunkV) : 0;
 }

@@ -114,7 +114,7 @@ int rlscan_plan(int64_t E, int64_t T, int64_t actions, int64_t *tile_elems, int 
     RLSCAN_TRY(check_shape(E, T, actions));
     const Plan p = make_plan(E, T); // every call scans on the single-action plan
     // rows that span tiles run the chunked two passes: report the workspace's
-    // granularity (one slot per 512 elements) and its slot count, an upper
+    // granularity (one slot per 1024 elements) and its slot count, an upper
     // bound on the chunks (their number depends on the device)
     const long long slot_elems = 2LL * 32 * kChunkV;
     if (tile_elems) *tile_elems = p.lookback ? slot_elems : kCfgTile[p.cfg];

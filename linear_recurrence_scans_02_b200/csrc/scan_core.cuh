@@ -834,7 +834,8 @@ __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Param
 // long array runs in waves whose inputs pass two finds in L2.
 // ---------------------------------------------------------------------------
 constexpr int kChunkNT = 128; // 4 independent warps per block
-constexpr int kChunkV = 8;    // elements per lane and step
+constexpr int kChunkV = 16;   // elements per lane and step: two 256-bit loads per plane
+                              // (GAE at 16 x 262144: 22.0 us, against 25.7 us with 8)
 constexpr int kChunkAggregates = 0;
 constexpr int kChunkScan = 1;
 

@@ -183,7 +183,7 @@ def test_binding_imports_without_gpu():
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
-    # 1 x (2^27 + 1) steps split over ~65,600 tiles needs more than 1 MiB of scratch
+    # 1 x (2^27 + 1) steps split over tiles needs about 2 MiB of scratch (one slot per 1024)
     T_big = (1 << 27) + 1
     far = [(k + 1) << 32 for k in range(4)]  # 512 MiB planes, 4 GiB apart: no overlap
     assert lib.rlscan_gae_noalloc(far[0], far[1], far[2], None, None, None, far[3], 1, T_big, 0.99, 0.95,
@@ -304,11 +304,11 @@ def test_batch_call_layout_matches_the_header(tmp_path):
     (4096, 2048, 2048, 256, False),    # a row needs a bigger tile to stay whole
     (256, 4096, 4096, 512, False),
     # rows that span tiles: the chunked two passes (128-thread blocks of
-    # independent warps), reported as one workspace slot per 512 elements
-    (16, 262144, 512, 128, True),      # long rows
-    (1024, 8192, 512, 128, True),
-    (3, 70000, 512, 128, True),
-    (4096, 129, 512, 128, True),       # rows not dividing any tile
+    # independent warps), reported as one workspace slot per 1024 elements
+    (16, 262144, 1024, 128, True),     # long rows
+    (1024, 8192, 1024, 128, True),
+    (3, 70000, 1024, 128, True),
+    (4096, 129, 1024, 128, True),       # rows not dividing any tile
 ])
 def test_plan_choices(lib, E_, T_, tile, threads, lookback):
     # the launch plans the measurements in the design notes were taken with

@@ -25,7 +25,7 @@ def test_c_program_links_and_calls_the_library(tmp_path, rlscan_lib_path):
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines()
     assert out[0] == "version 120"
     assert out[1].startswith("plan 4096 128 rc=0 tile=1024 threads=128 lookback=0 ntiles=512 ws=0")
-    assert out[2].startswith("plan 16 262144 rc=0 tile=512 threads=128 lookback=1 ntiles=8192")
-    assert out[3].startswith("plan 3 70000 rc=0 tile=512 threads=128 lookback=1")
+    assert out[2].startswith("plan 16 262144 rc=0 tile=1024 threads=128 lookback=1 ntiles=4096")
+    assert out[3].startswith("plan 3 70000 rc=0 tile=1024 threads=128 lookback=1")
     assert out[4].startswith("null rc=1 msg=") and "rewards" in out[4]
     assert out[5] == "batch rc=0"
