@@ -148,7 +148,6 @@ static void fused_layout(FusedBatch &fb, long long *tiles) {
         it.mode = ((32LL * V) % T == 0) ? kModeWarp : kModeBlock;
         it.g.scan_lanes = it.mode == kModeWarp ? (int)std::min<long long>(32, T >= V ? T / V : 1) : 32;
         it.tile_begin = begin;
-        it.g.pf_blocks = (long long)num_sms() * kFusedMinBlocks;
         begin += it.g.ntiles;
     }
     *tiles = begin;
@@ -248,9 +247,14 @@ int rlscan_batch(const rlscan_call *calls, int ncalls, void *ws, size_t ws_bytes
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = pdl_enabled() ? 1 : 0;
-        const cudaError_t e = fused_plain(part)
-                                  ? cudaLaunchKernelEx(&cfg, fused_tile_kernel<kFusedV, kCasePlain>, part)
-                                  : cudaLaunchKernelEx(&cfg, fused_tile_kernel<kFusedV, kCaseAny>, part);
+        const bool plain = fused_plain(part);
+        // the first wave of blocks (the instance's resident blocks on every
+        // SM) prefetches its tiles into L2
+        const long long pf = num_sms() * (long long)(plain ? fused_min_blocks<kCasePlain>()
+                                                           : fused_min_blocks<kCaseAny>());
+        for (int i = 0; i < part.n; ++i) part.item[i].g.pf_blocks = pf;
+        const cudaError_t e = plain ? cudaLaunchKernelEx(&cfg, fused_tile_kernel<kFusedV, kCasePlain>, part)
+                                    : cudaLaunchKernelEx(&cfg, fused_tile_kernel<kFusedV, kCaseAny>, part);
         if (e != cudaSuccess)
             return fail(RLSCAN_ERR_CUDA, "rlscan_batch: fused launch failed: %s", cudaGetErrorString(e));
         first = last + 1;

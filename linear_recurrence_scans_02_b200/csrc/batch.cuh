@@ -163,11 +163,19 @@ inline const P &family_params(const P &p) { // estimators that are their own bod
 
 constexpr int kFusedNT = 128; // 128 threads x 8 elements per tile
 constexpr int kFusedV = 8;
-// Blocks per SM the fused kernel is compiled to fit (64 registers a thread;
-// measured at 4096 x 128: the step's eight calls 13.9 us at 8 blocks per SM
-// against 14.5 us at the 72 registers the bodies take unbounded, 7 blocks
-// per SM, despite a few spilled registers).
+// Blocks per SM the fused kernel is compiled to fit.  General instance: 8
+// (64 registers a thread; measured at 4096 x 128: the step's eight calls
+// 13.9 us at 8 blocks per SM against 14.5 us at the 72 registers the bodies
+// take unbounded, 7 blocks per SM, despite a few spilled registers).  Plain
+// instance: 9 (56 registers, 28 bytes of spills; the step 12.15 against
+// 12.95 us at 8 and 12.15 at 10, where eight Retrace calls slow from 17.0
+// to 19.7 us).
 constexpr int kFusedMinBlocks = 8;
+constexpr int kFusedMinBlocksPlain = 9;
+template <int kCase>
+constexpr int fused_min_blocks() {
+    return kCase == kCasePlain ? kFusedMinBlocksPlain : kFusedMinBlocks;
+}
 constexpr int kFusedParamBytes = 128;
 constexpr int kFusedMax = 16;
 
@@ -220,7 +228,8 @@ __device__ __forceinline__ void fused_tile_any_mode(const FusedItem &it, long lo
 }
 
 template <int V, int kCase>
-__global__ void __launch_bounds__(kFusedNT, kFusedMinBlocks) fused_tile_kernel(const __grid_constant__ FusedBatch b) {
+__global__ void __launch_bounds__(kFusedNT, fused_min_blocks<kCase>())
+    fused_tile_kernel(const __grid_constant__ FusedBatch b) {
     extern __shared__ __align__(128) unsigned char dyn_smem[];
     int idx = 0;
     for (int i = 1; i < b.n; ++i)
