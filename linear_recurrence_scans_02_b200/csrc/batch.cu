@@ -158,7 +158,8 @@ static void fused_layout(FusedBatch &fb, long long *tiles) {
 // truncations (except to Retrace, whose builder always tests them), runs the
 // kCasePlain kernel: one builder variant per body, so the five bodies take
 // less of each SM's instruction caches (the 4096 x 128 step of eight calls:
-// 12.9 against 13.4 us; eight Retrace calls alone 16.9 against 16.4 us).
+// 12.9 against 13.4 us; eight Retrace calls alone, on inputs that stay in
+// L2, 16.9 against 16.4 us).
 static bool fused_plain(const FusedBatch &fb) {
     constexpr long long S = (long long)kFusedNT * kFusedV;
     for (int i = 0; i < fb.n; ++i) {
