@@ -154,17 +154,19 @@ static void fused_layout(FusedBatch &fb, long long *tiles) {
 }
 
 // A launch whose calls all have whole rows in every warp (warp-local scans),
-// rows a multiple of V steps long and a whole number of tiles, and pass no
-// truncations (except to Retrace, whose builder always tests them), runs the
-// kCasePlain kernel: one builder variant per body, so the five bodies take
-// less of each SM's instruction caches (the 4096 x 128 step of eight calls:
+// rows a multiple of V steps long, a whole number of tiles and 16-byte
+// aligned planes, and pass no truncations (except to Retrace, whose builder
+// always tests them), runs the kCasePlain kernel: one builder variant per
+// body and no scalar loads, so the five bodies take less of each SM's
+// instruction caches (the 4096 x 128 step of eight calls:
 // 12.9 against 13.4 us; eight Retrace calls alone, on inputs that stay in
 // L2, 16.9 against 16.4 us).
 static bool fused_plain(const FusedBatch &fb) {
     constexpr long long S = (long long)kFusedNT * kFusedV;
     for (int i = 0; i < fb.n; ++i) {
         const FusedItem &it = fb.item[i];
-        if (it.truncation_code || it.mode != kModeWarp || it.g.seq_len % kFusedV != 0 || it.g.n % S != 0)
+        if (it.truncation_code || it.mode != kModeWarp || it.g.seq_len % kFusedV != 0 || it.g.n % S != 0 ||
+            it.g.vec_ok == 0)
             return false;
     }
     return true;

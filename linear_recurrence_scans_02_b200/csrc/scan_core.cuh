@@ -213,9 +213,10 @@ struct RowMasks {
 // builders (`coeffs<V, kCase>`):
 //   kCaseAny    truncations and the fast path are decided per call and
 //               thread at run time (every variant is compiled in);
-//   kCasePlain  no call passes truncations and every thread takes the fast
-//               path (V divides T and the array is a whole number of tiles):
-//               one variant per builder, a smaller kernel.
+//   kCasePlain  no call passes truncations, every thread takes the fast
+//               path (V divides T and the array is a whole number of tiles)
+//               and every plane is 16-byte aligned: one variant per builder
+//               and vector accesses only, a smaller kernel.
 constexpr int kCaseAny = 0;
 constexpr int kCasePlain = 1;
 template <int V>
@@ -721,7 +722,10 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     const long long tile0 = m * (long long)(NT * V);
     const long long i0 = tile0 + (long long)tid * V;
 
-    const RowMajorPos<V> pos{i0, g.n, g.vec_ok != 0 && i0 + V <= g.n, lane};
+    // kCasePlain launches guarantee vector accesses (every plane 16-byte
+    // aligned, every thread's V elements present): no scalar path compiled in
+    const bool vec = kCase == kCasePlain || (g.vec_ok != 0 && i0 + V <= g.n);
+    const RowMajorPos<V> pos{i0, g.n, vec, lane};
     typename Est::template State<V> S;
     Est::template load<NT, V>(P, g, pos, S, dyn_smem);
 

@@ -163,18 +163,22 @@ def test_batch_of_every_kind_matches_single_calls_and_oracle(E, T, trunc):
     _check_batch(calls, refs)
 
 
-@pytest.mark.parametrize("shapes,trunc", [(((64, 128), (8, 128)), False), (((64, 128), (9, 128)), False),
-                                          (((64, 128), (8, 128)), True), (((16, 256), (4, 256)), False)],
-                         ids=["plain", "partial-tile", "truncations", "plain-256"])
-def test_batch_plain_and_general_fused_kernels(shapes, trunc):
+@pytest.mark.parametrize("shapes,trunc,offset", [(((64, 128), (8, 128)), False, 0),
+                                                 (((64, 128), (9, 128)), False, 0),
+                                                 (((64, 128), (8, 128)), True, 0),
+                                                 (((16, 256), (4, 256)), False, 0),
+                                                 (((64, 128), (8, 128)), False, 1)],
+                         ids=["plain", "partial-tile", "truncations", "plain-256", "unaligned"])
+def test_batch_plain_and_general_fused_kernels(shapes, trunc, offset):
     # every kind on one shape plus GAE on a second: "plain" requests (warp-local
-    # rows of a multiple of 8 steps, whole 1024-element tiles, truncations on
-    # Retrace only) take the fused kernel built without the other builder
-    # variants; a call off a whole tile or truncations elsewhere take the
+    # rows of a multiple of 8 steps, whole 1024-element tiles, 16-byte aligned
+    # planes, truncations on Retrace only) take the fused kernel built without
+    # the other builder variants and the scalar loads; a call off a whole
+    # tile, truncations elsewhere or a plane off a 16-byte boundary take the
     # general one.  Both must match the single calls and the oracle.
     (E0, T0), (E1, T1) = shapes
     calls, refs = _calls_for(E0, T0, seed=70, trunc=trunc)
-    c1, r1 = _calls_for(E1, T1, seed=71, trunc=trunc)
+    c1, r1 = _calls_for(E1, T1, seed=71, trunc=trunc, offset=offset)
     _check_batch(calls + c1[:1], refs + r1[:1])
 
 
