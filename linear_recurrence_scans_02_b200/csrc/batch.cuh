@@ -167,7 +167,7 @@ constexpr int kFusedV = 8;
 // (64 registers a thread; measured at 4096 x 128: the step's eight calls
 // 13.9 us at 8 blocks per SM against 14.5 us at the 72 registers the bodies
 // take unbounded, 7 blocks per SM, despite a few spilled registers).  Plain
-// instance: 9 (56 registers, 28 bytes of spills; the step 12.15 against
+// instance: 9 (56 registers; the step 12.15 against
 // 12.95 us at 8 and 12.15 at 10, where eight Retrace calls on inputs that
 // stay in L2 slow from 17.0 to 19.7 us).
 constexpr int kFusedMinBlocks = 8;
