@@ -188,17 +188,21 @@ struct FusedItem {
     int truncation_code;  // the call needs its body's truncation variants (not kCasePlain)
 };
 
-// Host side: whether a call, in its body's form, passes truncations to a
-// builder whose kCasePlain variant compiles them out.  Retrace's builder
-// tests its truncation flags in every variant, and bodies without a
-// truncation plane never pass any.
+// Host side: whether a call, in its builder's parameter form P, passes
+// truncations to a builder whose kCasePlain variant compiles them out.
+// Retrace's builder tests its truncation flags in every variant, and
+// builders without a truncation plane never take any.
 template <class P, class = void>
 struct HasTruncations : std::false_type {};
 template <class P>
 struct HasTruncations<P, std::void_t<decltype(std::declval<P>().truncateds)>> : std::true_type {};
+template <class Est>
+struct PlainTestsTruncations : std::false_type {};
+template <class V, class F, class N>
+struct PlainTestsTruncations<RetraceEstT<V, F, N>> : std::true_type {};
 template <class Est, class P>
 inline bool needs_truncation_code(const P &p) {
-    if constexpr (std::is_same<Est, RetraceEst>::value || !HasTruncations<P>::value) return false;
+    if constexpr (PlainTestsTruncations<Est>::value || !HasTruncations<P>::value) return false;
     else return p.truncateds != nullptr;
 }
 

@@ -812,10 +812,10 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
 
 }
 
-template <class Est, int NT, int V, int kMode>
+template <class Est, int NT, int V, int kMode, int kCase>
 __global__ void __launch_bounds__(NT) tile_scan_kernel(const typename Est::Params P, const Geometry g) {
     extern __shared__ __align__(128) unsigned char dyn_smem[];
-    tile_scan_body<Est, NT, V, kMode>(P, g, (long long)blockIdx.x, dyn_smem);
+    tile_scan_body<Est, NT, V, kMode, kCase>(P, g, (long long)blockIdx.x, dyn_smem);
 }
 
 // ---------------------------------------------------------------------------
