@@ -901,7 +901,7 @@ __device__ BT chunk_carry(const TileSlot *slots, long long c, int lane, AT proto
     }
 }
 
-template <class Est, int kPass>
+template <class Est, int kPass, int kCase>
 __global__ void __launch_bounds__(kChunkNT) chunk_scan_kernel(const typename Est::Params P, const Geometry g,
                                                               const ChunkSplit cs) {
     using AT = typename Est::AT;
@@ -938,13 +938,15 @@ __global__ void __launch_bounds__(kChunkNT) chunk_scan_kernel(const typename Est
     for (long long s = s0; s < s1; ++s) {
         const long long m = kBwd ? (cs.nsteps - 1 - s) : s; // step in memory order
         const long long i0 = m * SW + (long long)lane * V;
-        const RowMajorPos<V> pos{i0, g.n, g.vec_ok != 0 && i0 + V <= g.n, lane};
+        // kCasePlain: every plane 16-byte aligned and every step whole
+        const bool vec = kCase == kCasePlain || (g.vec_ok != 0 && i0 + V <= g.n);
+        const RowMajorPos<V> pos{i0, g.n, vec, lane};
         typename Est::template State<V> S;
         Est::template load<32, V>(P, g, pos, S, nullptr);
         AT a[V];
         BT b[V];
         const RowMasks rm = row_masks<V>(i0, g);
-        Est::template coeffs<V>(P, g, pos, rm, S, a, b);
+        Est::template coeffs<V, kCase>(P, g, pos, rm, S, a, b);
 
         // lane map, composed in scan order
         AT ta;
