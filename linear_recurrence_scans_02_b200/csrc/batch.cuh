@@ -106,6 +106,8 @@ struct BackwardFamilyEst {
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if constexpr (kCase == kCasePlain) {
             coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if constexpr (kCase == kCasePlainTrunc) {
+            coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
         } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);

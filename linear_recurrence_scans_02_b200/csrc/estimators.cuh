@@ -143,6 +143,8 @@ struct GaeEstT {
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if constexpr (kCase == kCasePlain) {
             coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if constexpr (kCase == kCasePlainTrunc) {
+            coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
         } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
@@ -257,6 +259,8 @@ struct LambdaReturnsEstT {
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if constexpr (kCase == kCasePlain) {
             coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if constexpr (kCase == kCasePlainTrunc) {
+            coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
         } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
@@ -349,6 +353,8 @@ struct ReturnsEstT {
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if constexpr (kCase == kCasePlain) {
             coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if constexpr (kCase == kCasePlainTrunc) {
+            coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
         } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
@@ -465,6 +471,8 @@ struct VtraceEstT {
                                                   const RowMasks &rm, State<V> &S, float (&a)[V], float (&b)[V]) {
         if constexpr (kCase == kCasePlain) {
             coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if constexpr (kCase == kCasePlainTrunc) {
+            coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
         } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
@@ -573,6 +581,8 @@ struct GaeVtraceEst {
                                                   float2 (&b)[V]) {
         if constexpr (kCase == kCasePlain) {
             coeffs_impl<V, false, true>(P, g, pos, rm, S, a, b);
+        } else if constexpr (kCase == kCasePlainTrunc) {
+            coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
         } else if (P.truncateds != nullptr) {
             if (rm.fast) coeffs_impl<V, true, true>(P, g, pos, rm, S, a, b);
             else coeffs_impl<V, true, false>(P, g, pos, rm, S, a, b);
@@ -681,7 +691,7 @@ struct RetraceEstT {
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V],
                                                   float (&b)[V]) {
-        if constexpr (kCase == kCasePlain) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        if constexpr (kCase != kCaseAny) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }
@@ -757,7 +767,7 @@ struct ForwardEstT {
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, float (&a)[V],
                                                   float (&b)[V]) {
-        if constexpr (kCase == kCasePlain) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        if constexpr (kCase != kCaseAny) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }
@@ -830,7 +840,7 @@ struct PrefixI32EstT {
     static __device__ __forceinline__ void coeffs(const Params &P, const Geometry &g, const Pos &pos,
                                                   const RowMasks &rm, State<V> &S, uint32_t (&a)[V],
                                                   int32_t (&b)[V]) {
-        if constexpr (kCase == kCasePlain) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
+        if constexpr (kCase != kCaseAny) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else if (rm.fast) coeffs_impl<V, true>(P, g, pos, rm, S, a, b);
         else coeffs_impl<V, false>(P, g, pos, rm, S, a, b);
     }

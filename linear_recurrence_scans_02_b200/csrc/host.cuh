@@ -310,11 +310,17 @@ cudaError_t launch_one(const typename Est::Params &P, const Geometry &g, size_t 
 }
 
 template <class Est, Cfg C>
-cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, int mode, bool plain, size_t smem,
+cudaError_t launch_cfg(const typename Est::Params &P, const Geometry &g, int mode, int kcase, size_t smem,
                        cudaStream_t s) {
     constexpr int NT = kCfgThreads[C];
     constexpr int V = kCfgTile[C] / NT;
-    if (plain) {
+    if constexpr (HasTruncations<typename Est::Params>::value && !PlainTestsTruncations<Est>::value) {
+        if (kcase == kCasePlainTrunc) {
+            if (mode == kModeWarp) return launch_one<Est, NT, V, kModeWarp, kCasePlainTrunc>(P, g, smem, s);
+            return launch_one<Est, NT, V, kModeBlock, kCasePlainTrunc>(P, g, smem, s);
+        }
+    }
+    if (kcase == kCasePlain) {
         if (mode == kModeWarp) return launch_one<Est, NT, V, kModeWarp, kCasePlain>(P, g, smem, s);
         return launch_one<Est, NT, V, kModeBlock, kCasePlain>(P, g, smem, s);
     }
@@ -416,18 +422,20 @@ int run(const char *name, const typename Est::Params &P, long long E, long long 
                      : run_chunked<Est, kCaseAny>(name, P, g, slots, stream);
     }
     // the plain kernel (one builder variant, vector accesses only) when every
-    // thread has all its elements (V divides T, whole tiles), every plane is
-    // 16-byte aligned and no truncation logic is needed (measured at 4096 x
-    // 128: GAE 2.34 against 2.41 us, V-Trace 3.03 against 3.19, bf16 / uint8
-    // GAE + returns 2.52 against 2.99)
+    // thread has all its elements (V divides T, whole tiles) and every plane
+    // is 16-byte aligned (measured at 4096 x 128: GAE 2.34 against 2.41 us,
+    // V-Trace 3.03 against 3.19, bf16 / uint8 GAE + returns 2.52 against
+    // 2.99); with truncation logic when the call passes truncations (GAE
+    // with truncations 2.88 against 3.01 us)
     const long long S = kCfgTile[plan.cfg], Vp = S / kCfgThreads[plan.cfg];
-    const bool plain = vec_ok && T % Vp == 0 && g.n % S == 0 && !needs_truncation_code<Est>(P);
+    const bool whole = vec_ok && T % Vp == 0 && g.n % S == 0;
+    const int kcase = !whole ? kCaseAny : (needs_truncation_code<Est>(P) ? kCasePlainTrunc : kCasePlain);
     cudaError_t e;
     switch (plan.cfg) {
-    case C512: e = launch_cfg<Est, C512>(P, g, plan.mode, plain, 0, stream); break;
-    case C1024: e = launch_cfg<Est, C1024>(P, g, plan.mode, plain, 0, stream); break;
-    case C2048: e = launch_cfg<Est, C2048>(P, g, plan.mode, plain, 0, stream); break;
-    case C4096: e = launch_cfg<Est, C4096>(P, g, plan.mode, plain, 0, stream); break;
+    case C512: e = launch_cfg<Est, C512>(P, g, plan.mode, kcase, 0, stream); break;
+    case C1024: e = launch_cfg<Est, C1024>(P, g, plan.mode, kcase, 0, stream); break;
+    case C2048: e = launch_cfg<Est, C2048>(P, g, plan.mode, kcase, 0, stream); break;
+    case C4096: e = launch_cfg<Est, C4096>(P, g, plan.mode, kcase, 0, stream); break;
     default: return fail(RLSCAN_ERR_UNSUPPORTED, "%s: internal plan error", name);
     }
     if (e != cudaSuccess) return fail(RLSCAN_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));

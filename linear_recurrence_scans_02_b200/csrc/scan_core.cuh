@@ -216,9 +216,12 @@ struct RowMasks {
 //   kCasePlain  no call passes truncations, every thread takes the fast
 //               path (V divides T and the array is a whole number of tiles)
 //               and every plane is 16-byte aligned: one variant per builder
-//               and vector accesses only, a smaller kernel.
+//               and vector accesses only, a smaller kernel;
+//   kCasePlainTrunc  the same with truncations: the fast builder with its
+//               truncation logic, vector accesses only (tile kernels).
 constexpr int kCaseAny = 0;
 constexpr int kCasePlain = 1;
+constexpr int kCasePlainTrunc = 2;
 template <int V>
 __device__ __forceinline__ RowMasks row_masks(long long i0, const Geometry &g) {
     RowMasks m;
@@ -722,9 +725,9 @@ __device__ __forceinline__ void tile_scan_body(const typename Est::Params &P, co
     const long long tile0 = m * (long long)(NT * V);
     const long long i0 = tile0 + (long long)tid * V;
 
-    // kCasePlain launches guarantee vector accesses (every plane 16-byte
-    // aligned, every thread's V elements present): no scalar path compiled in
-    const bool vec = kCase == kCasePlain || (g.vec_ok != 0 && i0 + V <= g.n);
+    // the plain cases guarantee vector accesses (every plane 16-byte aligned,
+    // every thread's V elements present): no scalar path compiled in
+    const bool vec = kCase != kCaseAny || (g.vec_ok != 0 && i0 + V <= g.n);
     const RowMajorPos<V> pos{i0, g.n, vec, lane};
     typename Est::template State<V> S;
     Est::template load<NT, V>(P, g, pos, S, dyn_smem);
